@@ -1,0 +1,451 @@
+"""Benchmark: paged decode attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--kernel auto|simt|mma] [--partition P]
+
+A step is one pass of the decode hot path over one batch: the new token of
+every sequence is appended to the paged cache (kv_cache_append, at the slot of
+its last position) and paged decode attention runs over every sequence's full
+context (partition kernel + log-sum-exp reduce).  Default workload: the
+Llama-2-13B-shaped layer (64 sequences, 40 heads MHA, head_dim 128, fp16 KV,
+block 16, context lengths uniform in [128, 2048], shuffled pool 1.2x).
+
+Metric: algorithmic bytes of the step (K and V of every context token, q and
+out, table entries, lengths, the appended tokens' reads and writes) per second.
+Inputs are larger than L2 (about 1.4 GB of K/V per step), so no flush runs
+between steps.  Time is measured with CUDA events on the launching stream,
+bracketed by a barrier and a synchronize, max over ranks.  One JSON line is
+printed by rank 0.  For N > 1 every rank runs its own replica of the workload
+(sequences are independent: weak scaling, no data-path collective).
+
+--impl reference times the CPU oracle (float64, all host cores) on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import CONFIGS, ELEM_BYTES, algorithmic_bytes, make_decode_inputs  # noqa: E402
+
+METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak) and tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------------------
+# helpers
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            return json.load(open(p))
+        except Exception:
+            return None
+    return None
+
+
+def step_bytes(cfg, lens) -> int:
+    """Decode algorithmic bytes + the append: read k, v of each new token,
+    write them, read the slot."""
+    e = ELEM_BYTES[cfg.dtype]
+    append = len(lens) * (2 * 2 * cfg.num_kv_heads * cfg.head_dim * e + 8)
+    return algorithmic_bytes(cfg, lens) + append
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.idx = device_index
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for n, bit in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def kernel_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_346_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.startswith("decode") or f in ("device_common.cuh",):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per decode launch from a committed ncu summary, if it was
+    taken on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", f"decode_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    rec = {}
+    for line in open(p):
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            rec[k.strip()] = v.strip().strip("`")
+    if rec.get("kernel_sources_sha256_16") != kernel_source_digest():
+        return None
+    if rec.get("kernel_variant") not in (None, kernel):
+        return None
+    try:
+        return int(rec["dram_bytes_per_decode_call"])
+    except (KeyError, ValueError):
+        return None
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline field)
+
+def oracle_rate(inp, budget_s: float, seed: int = 0):
+    """Time the float64 oracle on whole sequences (all heads) until about
+    budget_s of wall time; returns (bytes/s, seconds, sample description,
+    threads)."""
+    import oracle
+    cfg = inp.cfg
+    threads = oracle.max_threads()
+    order = np.random.default_rng(seed).permutation(cfg.num_seqs)
+    done, nbytes, t_total = [], 0, 0.0
+    for b in order:
+        rows = np.array([[b, h] for h in range(cfg.num_q_heads)], dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.paged_decode_inputs(inp, rows=rows, threads=threads)
+        t_total += time.perf_counter() - t0
+        done.append(int(b))
+        nbytes += algorithmic_bytes(cfg, inp.context_lens[[b]])
+        if t_total >= budget_s:
+            break
+    desc = (f"{len(done)} of {cfg.num_seqs} sequences (all {cfg.num_q_heads} heads, "
+            f"{int(inp.context_lens[done].sum())} context tokens) of {cfg.name}")
+    return nbytes / t_total, t_total, desc, threads
+
+
+def run_reference(args, cfg):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = make_decode_inputs(cfg, seed=args.seed)
+    import oracle
+    threads = oracle.max_threads()
+    # calibrate on one sequence, then size each step's sample so the whole
+    # run stays within about --ref-budget seconds
+    rate, _, _, _ = oracle_rate(inp, 0.0, seed=args.seed)
+    steps_total = args.steps + args.warmup
+    budget = args.ref_budget / max(steps_total, 1)
+    seq_bytes = algorithmic_bytes(cfg, inp.context_lens) / cfg.num_seqs
+    nseq = int(max(1, min(cfg.num_seqs, math.floor(rate * budget / seq_bytes))))
+    g = np.random.default_rng(args.seed)
+    samples = []
+    times = []
+    nbytes = []
+    for i in range(steps_total):
+        seqs = g.choice(cfg.num_seqs, size=nseq, replace=False)
+        rows = np.array([[b, h] for b in seqs for h in range(cfg.num_q_heads)], dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.paged_decode_inputs(inp, rows=rows, threads=threads)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+            nbytes.append(algorithmic_bytes(cfg, inp.context_lens[seqs]))
+    value = sum(nbytes) / sum(times) / 1e9
+    sample = (f"{nseq} of {cfg.num_seqs} sequences per step (all {cfg.num_q_heads} heads), "
+              f"float64 C oracle, {threads} threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sum(times) / len(times), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "global_batch": cfg.num_seqs,
+                   "seq_len": float(np.mean(inp.context_lens)), "parallelism": "none (host CPU)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_346_b200 as pkv
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[cfg.dtype]
+    kern = {"auto": pkv.PKV_KERNEL_AUTO, "simt": pkv.PKV_KERNEL_SIMT,
+            "mma": pkv.PKV_KERNEL_MMA}[args.kernel]
+
+    # ---- inputs (seeded; each rank its own replica)
+    inp = make_decode_inputs(cfg, seed=args.seed + rank)
+
+    def dev(a):
+        if cfg.dtype == "bf16" and a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+    q, kc, vc = dev(inp.q), dev(inp.k_cache), dev(inp.v_cache)
+    bt, cl = dev(inp.block_tables), dev(inp.context_lens)
+    B, H, D, bs = cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
+    lens = inp.context_lens.astype(np.int64)
+    last = lens - 1
+    slots_np = (inp.block_tables[np.arange(B), last // bs].astype(np.int64) * bs + last % bs)
+    slots = dev(slots_np)
+    # the new token of each sequence: the K/V already at its last position
+    # (so every step rewrites identical bits and the workload stays fixed)
+    knew = kc.view(-1, H, bs, D)[torch.from_numpy(slots_np // bs).cuda(), :,
+                                 torch.from_numpy(slots_np % bs).cuda(), :].contiguous()
+    vnew = vc.view(-1, H, bs, D)[torch.from_numpy(slots_np // bs).cuda(), :,
+                                 torch.from_numpy(slots_np % bs).cuda(), :].contiguous()
+    out = torch.empty_like(q)
+    mcl = inp.max_context_len
+    P = args.partition
+    ws_bytes = pkv.pkv_decode_workspace_size(B, cfg.num_q_heads, H, D, mcl, P)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+    Pused = P or pkv.pkv_decode_default_partition(B, H, mcl)
+    launches_per_step = 1 + 1 + (1 if math.ceil(mcl / Pused) > 1 else 0)
+    stream = torch.cuda.current_stream()
+
+    def decode():
+        pkv.pkv_paged_attention_decode(out, q, kc, vc, bt, cl, cfg.scale, bs, mcl,
+                                       partition_size=P, workspace=ws, kernel=kern,
+                                       stream=stream)
+
+    def step():
+        pkv.pkv_kv_cache_append(kc, vc, knew, vnew, slots, stream=stream)
+        decode()
+
+    nbytes = step_bytes(cfg, lens)
+    dec_bytes = algorithmic_bytes(cfg, lens)
+
+    # ---- device-resident timing
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            pkv.pkv_kv_cache_append(kc, vc, knew, vnew, slots, stream=stream)
+            ev_dec[i][0].record(stream)
+            decode()
+            ev_dec[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = t_start.elapsed_time(t_end)
+    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_dec)
+    flags = pkv.pkv_device_status(clear=True)
+    if flags:
+        raise SystemExit(f"device status flags {flags:#x} during the benchmark")
+
+    # ---- end to end through the public API: step inputs from pinned host
+    # memory each step, the output read back each step
+    h_q = torch.from_numpy(inp.q.view(np.int16) if cfg.dtype == "bf16" else inp.q)
+    h_q = (h_q.view(torch.bfloat16) if cfg.dtype == "bf16" else h_q).pin_memory()
+    h_knew, h_vnew = knew.cpu().pin_memory(), vnew.cpu().pin_memory()
+    h_slots = torch.from_numpy(slots_np).pin_memory()
+    h_bt = torch.from_numpy(inp.block_tables).pin_memory()
+    h_cl = torch.from_numpy(inp.context_lens).pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    d_knew, d_vnew = torch.empty_like(knew), torch.empty_like(vnew)
+    d_q, d_slots, d_bt, d_cl = (torch.empty_like(q), torch.empty_like(slots),
+                                torch.empty_like(bt), torch.empty_like(cl))
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_knew, h_vnew, h_slots, h_bt, h_cl))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        d_q.copy_(h_q, non_blocking=True)
+        d_knew.copy_(h_knew, non_blocking=True)
+        d_vnew.copy_(h_vnew, non_blocking=True)
+        d_slots.copy_(h_slots, non_blocking=True)
+        d_bt.copy_(h_bt, non_blocking=True)
+        d_cl.copy_(h_cl, non_blocking=True)
+        pkv.pkv_kv_cache_append(kc, vc, d_knew, d_vnew, d_slots, stream=stream)
+        pkv.pkv_paged_attention_decode(out, d_q, kc, vc, d_bt, d_cl, cfg.scale, bs, mcl,
+                                       partition_size=P, workspace=ws, kernel=kern,
+                                       stream=stream)
+        h_out.copy_(out, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 200))
+    for _ in range(max(args.warmup, 3)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    assert torch.equal(h_out, out.cpu())
+
+    # ---- max over ranks
+    vals = torch.tensor([ms, dec_ms, e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms, dec_ms, e2e_ms = vals.tolist()
+
+    if rank == 0:
+        per_step_ms = ms / args.steps
+        value = world * nbytes / (per_step_ms * 1e-3) / 1e9
+        peaks = measured_peaks()
+        if peaks and "hbm_gbs" in peaks:
+            peak, peak_src = float(peaks["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+        else:
+            peak, peak_src = FALLBACK_HBM_GBS, "fallback"
+        achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": cfg.name, "global_batch": B * world,
+                       "seq_len": round(float(lens.mean()), 1),
+                       "num_q_heads": cfg.num_q_heads, "num_kv_heads": H, "head_dim": D,
+                       "block_size": bs, "partition_size": Pused, "kernel": args.kernel,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (%.2f GB of K/V per step)" % (
+                           dec_bytes / 1e9)},
+            "tokens_per_s": round(world * B / (per_step_ms * 1e-3), 1),
+            "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+            "e2e": {"value": round(world * nbytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": launches_per_step * args.steps,
+            "roofline": {"bound": "hbm", "kernel": "paged decode (partition kernel + LSE reduce)",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_source": peak_src,
+                         "decode_ms": round(dec_ms, 5), "bytes_per_launch": int(dec_bytes),
+                         "traffic": recorded_traffic(cfg.name, args.kernel)},
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            rate, secs, desc, threads = oracle_rate(inp, args.cpu_budget, seed=args.seed)
+            line["cpu_baseline"] = {"value": round(rate / 1e9, 4), "unit": "GB/s",
+                                    "cores": threads, "kind": "oracle",
+                                    "sample": desc + f", {secs:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama2_13b_layer", choices=sorted(CONFIGS))
+    ap.add_argument("--kernel", choices=["auto", "simt", "mma"], default="auto")
+    ap.add_argument("--partition", type=int, default=None,
+                    help="tokens per partition (default: the workload's, else automatic)")
+    ap.add_argument("--seed", type=int, default=2)
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of oracle work for the cpu_baseline field")
+    ap.add_argument("--ref-budget", type=float, default=90.0,
+                    help="seconds of oracle work for --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    cfg = CONFIGS[args.workload]
+    if args.partition is None:
+        args.partition = cfg.partition_size
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,250 @@
+/*
+ * pagedkv -- PagedAttention decode for NVIDIA B200 (sm_100a), C ABI.
+ *
+ * What the library does, in the pages' terms:
+ *   A sequence's key/value cache is stored in fixed-size blocks of
+ *   `block_size` tokens (16 by default in vLLM) that sit anywhere in a
+ *   physical pool; a per-sequence block table maps logical block i to a
+ *   physical block, like an OS page table ("What is PagedAttention ..."
+ *   §How it works; lastdictionary "PagedAttention"; "pagedattention vllm"
+ *   §PagedAttention Design).  The attention kernel reads keys and values
+ *   through that table and computes the same result as attention over a
+ *   contiguous cache ("pagedattention vllm" §Attention Computation).
+ *   Blocks are handed out on demand from a free list, shared between
+ *   sequences with a common prefix under reference counts, and copied before
+ *   a sequence writes into a shared one ("pagedattention vllm"
+ *   §Copy-on-Write Sharing, §Memory Management).
+ *
+ * Layouts (all row-major, contiguous):
+ *   q, out          [num_seqs, num_q_heads, head_dim]           dtype
+ *   k_cache,v_cache [num_blocks, num_kv_heads, block_size, head_dim] dtype
+ *   block_tables    int32 [num_seqs, max_blocks_per_seq]; entry i of row b is
+ *                   the physical block holding tokens [i*bs, (i+1)*bs) of
+ *                   sequence b; entries past ceil(len/bs) are never read.
+ *                   4-byte entries, as the pages size the table
+ *                   ("pagedattention vllm" §Implementation Details).
+ *   context_lens    int32 [num_seqs]
+ *   k, v (append)   [num_tokens, num_kv_heads, head_dim]        dtype
+ *   slot_mapping    int64 [num_tokens]; slot = block * block_size + offset,
+ *                   negative = padding token, nothing written
+ *   block_pairs     int32 [num_pairs][2] = (src, dst)
+ * Query head h reads KV head h / (num_q_heads / num_kv_heads).
+ *
+ * Conventions:
+ *   - Device calls take device pointers, enqueue work on `stream` and return
+ *     without synchronising.  The caller owns all memory; device calls never
+ *     allocate.  Pointers must not alias (K and V are separate buffers).
+ *   - Every call returns a pkv_status.  Arguments are checked on the host
+ *     before anything is launched (PKV_EINVAL / PKV_EUNSUPPORTED); a failed
+ *     launch gives PKV_ECUDA.
+ *   - Data the host cannot see (table entries, lengths, slots, pairs) is
+ *     checked on the device: an access that would leave its buffer is not
+ *     made, and a bit is set in the device status word
+ *     (pkv_device_status).  Results of such a call are unspecified.
+ *   - The allocator (pkv_alloc_*) is host-only and not thread-safe: one
+ *     caller at a time per allocator.
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA stream type (identical to cudaStream_t); NULL = legacy default. */
+typedef struct CUstream_st* pkv_stream_t;
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_EINVAL = -1,       /* bad argument (host-side check) */
+    PKV_ENOMEM = -2,       /* allocator: no free block */
+    PKV_ENOSEQ = -3,       /* allocator: unknown sequence id */
+    PKV_EEXIST = -4,       /* allocator: sequence id already present */
+    PKV_EBOUNDS = -5,      /* an index out of range */
+    PKV_ECUDA = -6,        /* a CUDA runtime call or launch failed */
+    PKV_EUNSUPPORTED = -7  /* valid but not built (e.g. head_dim 96) */
+} pkv_status;
+
+typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+
+/* Decode kernel choice.  AUTO takes the tensor-core kernel for 16-bit caches
+ * with a query group of 4 or more heads per KV head, else the CUDA-core one. */
+typedef enum { PKV_KERNEL_AUTO = 0, PKV_KERNEL_SIMT = 1, PKV_KERNEL_MMA = 2 } pkv_kernel;
+
+/* Device status bits (pkv_device_status) */
+#define PKV_DEV_BAD_BLOCK 1u    /* a table entry or copy pair outside [0, num_blocks) */
+#define PKV_DEV_BAD_LEN 2u      /* a context length < 0 or past the caller's bounds */
+#define PKV_DEV_BAD_SLOT 4u     /* a slot at or past num_blocks * block_size */
+#define PKV_DEV_TIMEOUT 8u      /* a bounded wait inside a kernel gave up */
+
+/* Name of a status code. */
+PKV_API const char* pkv_status_string(int status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+PKV_API int pkv_version(void);
+
+/* 1 if this build of the library contains decode kernel `kernel`, else 0. */
+PKV_API int pkv_decode_has_kernel(pkv_kernel kernel);
+
+/*
+ * Partition size the decode uses when `partition_size` is 0, for this shape.
+ */
+PKV_API int pkv_decode_default_partition(int num_seqs, int num_kv_heads, int max_context_len);
+
+/*
+ * Bytes of device workspace pkv_paged_attention_decode needs: float32 partial
+ * results (m, l and the normalised output of each partition) for sequences
+ * longer than one partition.  0 when max_context_len fits one partition.
+ * partition_size 0 = pkv_decode_default_partition(num_seqs, num_kv_heads,
+ * max_context_len).  Returns 0 for invalid sizes.
+ */
+PKV_API size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                 int head_dim, int max_context_len, int partition_size);
+
+/*
+ * Paged decode attention: for every sequence b and query head h,
+ *   out[b,h,:] = softmax_t(scale * q[b,h,:] . k_t) weighted sum of v_t,
+ * over the tokens t < context_lens[b], k_t and v_t read from the physical
+ * block block_tables[b][t / block_size] at offset t % block_size
+ * ("pagedattention vllm" §Attention Computation: gather physical blocks,
+ * compute as if contiguous).  A sequence with length 0 gets a zero row.
+ *
+ * The context of each sequence is cut into partitions of `partition_size`
+ * tokens; one CTA takes one (sequence, KV head, partition) with all the query
+ * heads of that KV head's group; sequences longer than one partition are
+ * merged by a log-sum-exp reduce over the workspace.  Accumulation is float32;
+ * `out` is written in `dtype` (round to nearest even).
+ *
+ * Arguments:
+ *   out, q, k_cache, v_cache, block_tables, context_lens: device pointers,
+ *       layouts above; k_cache and v_cache 16-byte aligned.
+ *   num_q_heads % num_kv_heads == 0; head_dim in {64, 128, 256};
+ *   block_size in {16, 32, 64}; dtype f32, f16 or bf16.
+ *   max_context_len: host-side upper bound of context_lens, and
+ *       <= max_blocks_per_seq * block_size.
+ *   partition_size: 0 for the default, else a multiple of 64 in [64, 8192].
+ *   workspace: device memory of at least pkv_decode_workspace_size(...)
+ *       bytes, 16-byte aligned; may be NULL when that size is 0.
+ *   kernel: PKV_KERNEL_AUTO, or force one kernel (for measurements);
+ *       PKV_KERNEL_MMA needs f16/bf16 and a group of at most 16 heads.
+ * Returns PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED or PKV_ECUDA.
+ */
+PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* block_tables,
+                               const int32_t* context_lens, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim,
+                               int block_size, int max_blocks_per_seq, int num_blocks,
+                               int max_context_len, float scale, pkv_dtype dtype,
+                               int partition_size, void* workspace,
+                               size_t workspace_bytes, pkv_kernel kernel,
+                               pkv_stream_t stream);
+
+/*
+ * KV append: the key and value of each new token go into the slot the block
+ * manager gave it ("What is PagedAttention ..." §How it works: blocks are
+ * filled as the answer grows):
+ *   k_cache[s / bs, h, s % bs, :] = k[t, h, :], same for v, s = slot_mapping[t];
+ * s < 0 writes nothing.  Two tokens with the same non-negative slot in one
+ * call leave that slot undefined.  A slot >= num_blocks * block_size is
+ * skipped and flagged (PKV_DEV_BAD_SLOT).  Bit copy; any head_dim with
+ * head_dim * element size a multiple of 16 bytes.
+ */
+PKV_API int pkv_kv_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
+                        const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                        int head_dim, int block_size, int num_blocks, pkv_dtype dtype,
+                        pkv_stream_t stream);
+
+/*
+ * Copy-on-write block copies ("pagedattention vllm" §Copy-on-Write Sharing:
+ * a shared block is copied before a sequence modifies it): for each pair,
+ * k_cache[dst] = k_cache[src] and v_cache[dst] = v_cache[src], the whole block
+ * (all heads, all slots).  block_pairs: device int32 [num_pairs][2].
+ * A dst must not appear twice nor also be a src in the same call.  Pairs with
+ * an id outside [0, num_blocks) are skipped and flagged (PKV_DEV_BAD_BLOCK).
+ */
+PKV_API int pkv_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_pairs,
+                    int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, pkv_dtype dtype, pkv_stream_t stream);
+
+/*
+ * Reads (and with clear != 0, resets) the device status word of the current
+ * device: an OR of PKV_DEV_* bits set by earlier calls.  Synchronises the
+ * device.
+ */
+PKV_API int pkv_device_status(unsigned int* flags, int clear);
+
+/* ------------------------------------------------------------------------
+ * Host block allocator ("pagedattention vllm" §Memory Management: a free list,
+ * allocate on demand, free when the sequence completes; §Copy-on-Write
+ * Sharing: reference counts, free at zero, copy before writing a shared
+ * block).  Rules:
+ *   - the free list is a stack; a new allocator pops 0, 1, 2, ...;
+ *   - add_seq(n) takes ceil(n / block_size) blocks in logical order, or none;
+ *   - append_slot: a full (or absent) last block -> take a new block; a
+ *     shared last block (count > 1) -> take a block dst, report (last, dst)
+ *     for pkv_copy_blocks, drop one reference to last and use dst; the sole
+ *     holder writes in place.  Returns the token's slot;
+ *   - fork(parent, child): child gets the parent's table and length, every
+ *     block one more reference;
+ *   - free_seq: drop one reference per table entry in logical order, push
+ *     each block that reaches zero;
+ *   - a failed call changes nothing.
+ * ------------------------------------------------------------------------ */
+typedef struct pkv_alloc pkv_alloc;
+
+typedef struct {
+    int32_t num_blocks;
+    int32_t block_size;
+    int32_t free_blocks;
+    int32_t used_blocks;     /* blocks with a reference count > 0 */
+    int32_t shared_blocks;   /* blocks with a reference count > 1 */
+    int32_t num_seqs;
+    int64_t refcount_sum;    /* = total block-table entries over sequences */
+    int64_t logical_tokens;  /* sum of sequence lengths */
+} pkv_alloc_stats_t;
+
+/* num_blocks > 0, block_size > 0.  *out = new allocator (free with destroy). */
+PKV_API int pkv_alloc_create(int num_blocks, int block_size, pkv_alloc** out);
+PKV_API void pkv_alloc_destroy(pkv_alloc* a);
+/* New sequence holding num_tokens >= 0 tokens. */
+PKV_API int pkv_alloc_add_seq(pkv_alloc* a, int64_t seq_id, int num_tokens);
+PKV_API int pkv_alloc_fork(pkv_alloc* a, int64_t parent, int64_t child);
+/* One more token for seq_id: *slot gets its slot; *cow_src / *cow_dst get the
+ * block copy to run first, or -1 / -1. */
+PKV_API int pkv_alloc_append_slot(pkv_alloc* a, int64_t seq_id, int64_t* slot,
+                          int32_t* cow_src, int32_t* cow_dst);
+/* append_slot for n sequences in order.  slots[i] gets sequence i's slot;
+ * cow_pairs ([n][2] capacity) gets the copies in order, *num_cow their
+ * count.  Stops at the first failure: *num_done sequences were appended. */
+PKV_API int pkv_alloc_append_slots(pkv_alloc* a, const int64_t* seq_ids, int n, int64_t* slots,
+                           int32_t* cow_pairs, int* num_cow, int* num_done);
+PKV_API int pkv_alloc_free_seq(pkv_alloc* a, int64_t seq_id);
+PKV_API int pkv_alloc_seq_len(const pkv_alloc* a, int64_t seq_id, int* len);
+/* Copies seq_id's table to out (capacity entries); *n_out = its length.
+ * PKV_EBOUNDS (and nothing copied) when capacity is too small. */
+PKV_API int pkv_alloc_block_table(const pkv_alloc* a, int64_t seq_id, int32_t* out,
+                          int capacity, int* n_out);
+/* Batch tables for a decode call: row i of tables ([n][max_blocks]) gets the
+ * table of seq_ids[i], padded with `fill`; context_lens[i] its length. */
+PKV_API int pkv_alloc_build_block_tables(const pkv_alloc* a, const int64_t* seq_ids, int n,
+                                 int32_t* tables, int max_blocks, int32_t fill,
+                                 int32_t* context_lens);
+PKV_API int pkv_alloc_refcount(const pkv_alloc* a, int32_t block, int* out);
+PKV_API int pkv_alloc_stats(const pkv_alloc* a, pkv_alloc_stats_t* out);
+/* Free blocks in the order they will be handed out. */
+PKV_API int pkv_alloc_free_list(const pkv_alloc* a, int32_t* out, int capacity, int* n_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H_ */

@@ -1,0 +1,262 @@
+"""pagedkv: PagedAttention decode for NVIDIA B200 (sm_100a).
+
+Python face of the C library (include/pagedkv.h).  The functions carry the C
+names and take torch tensors; they pass pointers, sizes and the current CUDA
+stream through and raise PagedKVError on a non-zero status.  All computation
+happens in libpagedkv.so.
+
+    pkv_paged_attention_decode   paged decode attention (+ log-sum-exp reduce)
+    pkv_kv_cache_append          new tokens' K/V -> their slots
+    pkv_copy_blocks              copy-on-write block copies
+    BlockAllocator               host block manager (free list, refcounts, CoW)
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _binding as _b
+from ._binding import (PKV_BF16, PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD_SLOT,
+                       PKV_DEV_TIMEOUT, PKV_F16, PKV_F32, PKV_KERNEL_AUTO, PKV_KERNEL_MMA,
+                       PKV_KERNEL_SIMT, PagedKVError, check, lib)
+
+__all__ = [
+    "pkv_paged_attention_decode", "pkv_decode_workspace_size", "pkv_decode_has_kernel", "pkv_decode_default_partition",
+    "pkv_kv_cache_append", "pkv_copy_blocks", "pkv_device_status", "BlockAllocator",
+    "PagedKVError", "lib", "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_KERNEL_AUTO",
+    "PKV_KERNEL_SIMT", "PKV_KERNEL_MMA", "PKV_DEV_BAD_BLOCK", "PKV_DEV_BAD_LEN",
+    "PKV_DEV_BAD_SLOT", "PKV_DEV_TIMEOUT", "torch_dtype_code",
+]
+
+_DTYPE = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16}
+
+
+def torch_dtype_code(dt: torch.dtype) -> int:
+    try:
+        return _DTYPE[dt]
+    except KeyError:
+        raise PagedKVError(_b.PKV_EINVAL, f"dtype {dt}") from None
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not t.is_cuda:
+        raise PagedKVError(_b.PKV_EINVAL, f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise PagedKVError(_b.PKV_EINVAL, f"{name} must be contiguous")
+    return t
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def pkv_decode_has_kernel(kernel: int) -> bool:
+    return bool(lib.pkv_decode_has_kernel(int(kernel)))
+
+
+def pkv_decode_default_partition(num_seqs: int, num_kv_heads: int, max_context_len: int) -> int:
+    return int(lib.pkv_decode_default_partition(num_seqs, num_kv_heads, max_context_len))
+
+
+def pkv_decode_workspace_size(num_seqs: int, num_q_heads: int, num_kv_heads: int,
+                              head_dim: int, max_context_len: int,
+                              partition_size: int = 0) -> int:
+    return int(lib.pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                             max_context_len, partition_size))
+
+
+def pkv_paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                               v_cache: torch.Tensor, block_tables: torch.Tensor,
+                               context_lens: torch.Tensor, scale: float, block_size: int,
+                               max_context_len: int, *, partition_size: int = 0,
+                               workspace: torch.Tensor | None = None,
+                               kernel: int = PKV_KERNEL_AUTO, stream=None) -> torch.Tensor:
+    """out [B, Hq, D] <- paged decode attention (see pkv_paged_attention_decode
+    in pagedkv.h).  k_cache/v_cache [N, Hkv, block_size, D]; block_tables
+    int32 [B, max_blocks]; context_lens int32 [B]; max_context_len is a host
+    bound of context_lens.  workspace: a CUDA tensor of at least
+    pkv_decode_workspace_size(...) bytes when sequences span partitions."""
+    for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+                 (block_tables, "block_tables"), (context_lens, "context_lens")):
+        _dev(t, n)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise PagedKVError(_b.PKV_EINVAL, "block_tables / context_lens must be int32")
+    if not (q.dtype == out.dtype == k_cache.dtype == v_cache.dtype):
+        raise PagedKVError(_b.PKV_EINVAL, "q, out, k_cache, v_cache must share a dtype")
+    B, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    if (D2 != D or bs != block_size or tuple(out.shape) != (B, Hq, D) or
+            tuple(v_cache.shape) != tuple(k_cache.shape) or block_tables.shape[0] != B or
+            context_lens.shape[0] != B):
+        raise PagedKVError(_b.PKV_EINVAL, "shape mismatch")
+    ws_bytes = 0
+    if workspace is not None:
+        _dev(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    check(lib.pkv_paged_attention_decode(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], N,
+        int(max_context_len), float(scale), torch_dtype_code(q.dtype), int(partition_size),
+        _ptr(workspace), ws_bytes, int(kernel), _stream(stream)), "pkv_paged_attention_decode")
+    return out
+
+
+def pkv_kv_cache_append(k_cache: torch.Tensor, v_cache: torch.Tensor, k: torch.Tensor,
+                        v: torch.Tensor, slot_mapping: torch.Tensor, *, stream=None) -> None:
+    """k/v [T, Hkv, D] -> cache slots slot_mapping (int64 [T], < 0 = skip)."""
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache"), (k, "k"), (v, "v"),
+                 (slot_mapping, "slot_mapping")):
+        _dev(t, n)
+    if slot_mapping.dtype != torch.int64:
+        raise PagedKVError(_b.PKV_EINVAL, "slot_mapping must be int64")
+    if not (k.dtype == v.dtype == k_cache.dtype == v_cache.dtype):
+        raise PagedKVError(_b.PKV_EINVAL, "dtype mismatch")
+    N, Hkv, bs, D = k_cache.shape
+    T = k.shape[0]
+    if (tuple(k.shape) != (T, Hkv, D) or tuple(v.shape) != (T, Hkv, D) or
+            slot_mapping.shape[0] != T or tuple(v_cache.shape) != tuple(k_cache.shape)):
+        raise PagedKVError(_b.PKV_EINVAL, "shape mismatch")
+    check(lib.pkv_kv_cache_append(_ptr(k_cache), _ptr(v_cache), _ptr(k), _ptr(v),
+                                  _ptr(slot_mapping), T, Hkv, D, bs, N,
+                                  torch_dtype_code(k.dtype), _stream(stream)),
+          "pkv_kv_cache_append")
+
+
+def pkv_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_pairs: torch.Tensor,
+                    *, stream=None) -> None:
+    """block_pairs int32 [n, 2] of (src, dst): whole-block copies of K and V."""
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache"), (block_pairs, "block_pairs")):
+        _dev(t, n)
+    if block_pairs.dtype != torch.int32 or (block_pairs.numel() and block_pairs.shape[-1] != 2):
+        raise PagedKVError(_b.PKV_EINVAL, "block_pairs must be int32 [n, 2]")
+    N, Hkv, bs, D = k_cache.shape
+    check(lib.pkv_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_pairs),
+                              block_pairs.numel() // 2, Hkv, D, bs, N,
+                              torch_dtype_code(k_cache.dtype), _stream(stream)),
+          "pkv_copy_blocks")
+
+
+def pkv_device_status(clear: bool = False) -> int:
+    """OR of PKV_DEV_* bits set on the current device (synchronises)."""
+    flags = ctypes.c_uint(0)
+    check(lib.pkv_device_status(ctypes.byref(flags), int(bool(clear))), "pkv_device_status")
+    return int(flags.value)
+
+
+class BlockAllocator:
+    """Host block manager (pkv_alloc_*): free list, reference counts, fork and
+    copy-on-write.  Not thread-safe."""
+
+    def __init__(self, num_blocks: int, block_size: int):
+        h = ctypes.c_void_p()
+        check(lib.pkv_alloc_create(num_blocks, block_size, ctypes.byref(h)), "pkv_alloc_create")
+        self._h = h
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib.pkv_alloc_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    # operations: return the status code (callers compare against the model)
+    def add_seq(self, seq_id: int, num_tokens: int) -> int:
+        return lib.pkv_alloc_add_seq(self._h, seq_id, num_tokens)
+
+    def fork(self, parent: int, child: int) -> int:
+        return lib.pkv_alloc_fork(self._h, parent, child)
+
+    def append_slot(self, seq_id: int):
+        """-> (status, slot, cow_src, cow_dst)"""
+        slot = ctypes.c_int64(-1)
+        src = ctypes.c_int32(-1)
+        dst = ctypes.c_int32(-1)
+        st = lib.pkv_alloc_append_slot(self._h, seq_id, ctypes.byref(slot), ctypes.byref(src),
+                                       ctypes.byref(dst))
+        if st != 0:
+            return st, -1, -1, -1
+        return st, slot.value, src.value, dst.value
+
+    def append_slots(self, seq_ids):
+        """-> (status, slots int64 [n], cow_pairs int32 [n_cow, 2], num_done)"""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.size
+        slots = np.full(n, -1, dtype=np.int64)
+        pairs = np.full((max(n, 1), 2), -1, dtype=np.int32)
+        ncow = ctypes.c_int(0)
+        done = ctypes.c_int(0)
+        st = lib.pkv_alloc_append_slots(self._h, ids.ctypes.data, n, slots.ctypes.data,
+                                        pairs.ctypes.data, ctypes.byref(ncow),
+                                        ctypes.byref(done))
+        return st, slots, pairs[:ncow.value].copy(), done.value
+
+    def free_seq(self, seq_id: int) -> int:
+        return lib.pkv_alloc_free_seq(self._h, seq_id)
+
+    def apply(self, op):
+        kind = op[0]
+        if kind == "add":
+            return self.add_seq(op[1], op[2])
+        if kind == "fork":
+            return self.fork(op[1], op[2])
+        if kind == "append":
+            return self.append_slot(op[1])
+        if kind == "free":
+            return self.free_seq(op[1])
+        raise ValueError(kind)
+
+    # queries
+    def seq_len(self, seq_id: int) -> int:
+        n = ctypes.c_int(0)
+        check(lib.pkv_alloc_seq_len(self._h, seq_id, ctypes.byref(n)), "pkv_alloc_seq_len")
+        return n.value
+
+    def block_table(self, seq_id: int) -> list[int]:
+        n = ctypes.c_int(0)
+        st = lib.pkv_alloc_block_table(self._h, seq_id, None, 0, ctypes.byref(n))
+        if st not in (0, _b.PKV_EBOUNDS):
+            check(st, "pkv_alloc_block_table")
+        buf = (ctypes.c_int32 * max(n.value, 1))()
+        check(lib.pkv_alloc_block_table(self._h, seq_id, buf, n.value, ctypes.byref(n)),
+              "pkv_alloc_block_table")
+        return list(buf[:n.value])
+
+    def build_block_tables(self, seq_ids, max_blocks: int, fill: int = -1):
+        """-> (tables int32 [n, max_blocks], context_lens int32 [n]) numpy arrays"""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        tables = np.empty((ids.size, max_blocks), dtype=np.int32)
+        lens = np.empty(ids.size, dtype=np.int32)
+        check(lib.pkv_alloc_build_block_tables(self._h, ids.ctypes.data, ids.size,
+                                               tables.ctypes.data, max_blocks, fill,
+                                               lens.ctypes.data),
+              "pkv_alloc_build_block_tables")
+        return tables, lens
+
+    def refcount(self, block: int) -> int:
+        n = ctypes.c_int(0)
+        check(lib.pkv_alloc_refcount(self._h, block, ctypes.byref(n)), "pkv_alloc_refcount")
+        return n.value
+
+    def stats(self) -> dict:
+        s = _b.AllocStats()
+        check(lib.pkv_alloc_stats(self._h, ctypes.byref(s)), "pkv_alloc_stats")
+        return s.as_dict()
+
+    def free_list(self) -> list[int]:
+        n = ctypes.c_int(0)
+        buf = (ctypes.c_int32 * max(self.num_blocks, 1))()
+        check(lib.pkv_alloc_free_list(self._h, buf, self.num_blocks, ctypes.byref(n)),
+              "pkv_alloc_free_list")
+        return list(buf[:n.value])

@@ -1,0 +1,231 @@
+// Host-side KV block manager: free list, reference counts, fork and
+// copy-on-write ("pagedattention vllm" §Memory Management and §Copy-on-Write
+// Sharing; "What is PagedAttention ..." §How it works).  The rules each
+// operation follows are stated next to the declarations in pagedkv.h.
+//
+// Data structures: a vector used as a stack of free block ids, a reference
+// count per block, and a hash map from sequence id to (block table, length).
+// Every operation either completes or leaves all three untouched.
+#include <cstdint>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "pagedkv.h"
+
+struct pkv_alloc {
+    int32_t num_blocks;
+    int32_t block_size;
+    std::vector<int32_t> free_stack;  // back() is handed out next
+    std::vector<int32_t> ref;
+    struct Seq {
+        std::vector<int32_t> table;
+        int64_t len;
+    };
+    std::unordered_map<int64_t, Seq> seqs;
+    int64_t refcount_sum = 0;
+    int64_t logical_tokens = 0;
+    int32_t used_blocks = 0;
+    int32_t shared_blocks = 0;
+
+    int32_t take() {
+        int32_t b = free_stack.back();
+        free_stack.pop_back();
+        ref[b] = 1;
+        ++used_blocks;
+        ++refcount_sum;
+        return b;
+    }
+    void add_ref(int32_t b) {
+        if (ref[b] == 1) ++shared_blocks;
+        ++ref[b];
+        ++refcount_sum;
+    }
+    void drop_ref(int32_t b) {
+        --ref[b];
+        --refcount_sum;
+        if (ref[b] == 1) --shared_blocks;
+        if (ref[b] == 0) {
+            --used_blocks;
+            free_stack.push_back(b);
+        }
+    }
+};
+
+extern "C" {
+
+int pkv_alloc_create(int num_blocks, int block_size, pkv_alloc** out) {
+    if (!out || num_blocks <= 0 || block_size <= 0) return PKV_EINVAL;
+    pkv_alloc* a = new (std::nothrow) pkv_alloc();
+    if (!a) return PKV_ENOMEM;
+    a->num_blocks = num_blocks;
+    a->block_size = block_size;
+    try {
+        a->free_stack.resize(num_blocks);
+        for (int32_t i = 0; i < num_blocks; ++i) a->free_stack[i] = num_blocks - 1 - i;
+        a->ref.assign(num_blocks, 0);
+    } catch (...) {
+        delete a;
+        return PKV_ENOMEM;
+    }
+    *out = a;
+    return PKV_OK;
+}
+
+void pkv_alloc_destroy(pkv_alloc* a) { delete a; }
+
+int pkv_alloc_add_seq(pkv_alloc* a, int64_t seq_id, int num_tokens) {
+    if (!a || num_tokens < 0) return PKV_EINVAL;
+    if (a->seqs.count(seq_id)) return PKV_EEXIST;
+    const int64_t need = ((int64_t)num_tokens + a->block_size - 1) / a->block_size;
+    if (need > (int64_t)a->free_stack.size()) return PKV_ENOMEM;
+    pkv_alloc::Seq s;
+    s.len = num_tokens;
+    s.table.reserve(need);
+    for (int64_t i = 0; i < need; ++i) s.table.push_back(a->take());
+    a->logical_tokens += num_tokens;
+    a->seqs.emplace(seq_id, std::move(s));
+    return PKV_OK;
+}
+
+int pkv_alloc_fork(pkv_alloc* a, int64_t parent, int64_t child) {
+    if (!a) return PKV_EINVAL;
+    auto it = a->seqs.find(parent);
+    if (it == a->seqs.end()) return PKV_ENOSEQ;
+    if (a->seqs.count(child)) return PKV_EEXIST;
+    pkv_alloc::Seq s = it->second;  // copy of table and length
+    for (int32_t b : s.table) a->add_ref(b);
+    a->logical_tokens += s.len;
+    a->seqs.emplace(child, std::move(s));
+    return PKV_OK;
+}
+
+int pkv_alloc_append_slot(pkv_alloc* a, int64_t seq_id, int64_t* slot, int32_t* cow_src,
+                          int32_t* cow_dst) {
+    if (!a || !slot || !cow_src || !cow_dst) return PKV_EINVAL;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PKV_ENOSEQ;
+    pkv_alloc::Seq& s = it->second;
+    const int64_t off = s.len % a->block_size;
+    int32_t src = -1, dst = -1;
+    if (off == 0) {
+        if (a->free_stack.empty()) return PKV_ENOMEM;
+        s.table.push_back(a->take());
+    } else if (a->ref[s.table.back()] > 1) {
+        if (a->free_stack.empty()) return PKV_ENOMEM;
+        dst = a->take();
+        src = s.table.back();
+        a->drop_ref(src);  // stays > 0: another sequence still holds it
+        s.table.back() = dst;
+    }
+    *slot = (int64_t)s.table.back() * a->block_size + off;
+    *cow_src = src;
+    *cow_dst = dst;
+    s.len += 1;
+    a->logical_tokens += 1;
+    return PKV_OK;
+}
+
+int pkv_alloc_append_slots(pkv_alloc* a, const int64_t* seq_ids, int n, int64_t* slots,
+                           int32_t* cow_pairs, int* num_cow, int* num_done) {
+    if (!a || n < 0 || (n > 0 && (!seq_ids || !slots || !cow_pairs)) || !num_cow ||
+        !num_done)
+        return PKV_EINVAL;
+    *num_cow = 0;
+    *num_done = 0;
+    for (int i = 0; i < n; ++i) {
+        int32_t src, dst;
+        int rc = pkv_alloc_append_slot(a, seq_ids[i], &slots[i], &src, &dst);
+        if (rc != PKV_OK) return rc;
+        if (src >= 0) {
+            cow_pairs[2 * *num_cow] = src;
+            cow_pairs[2 * *num_cow + 1] = dst;
+            ++*num_cow;
+        }
+        ++*num_done;
+    }
+    return PKV_OK;
+}
+
+int pkv_alloc_free_seq(pkv_alloc* a, int64_t seq_id) {
+    if (!a) return PKV_EINVAL;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PKV_ENOSEQ;
+    for (int32_t b : it->second.table) a->drop_ref(b);
+    a->logical_tokens -= it->second.len;
+    a->seqs.erase(it);
+    return PKV_OK;
+}
+
+int pkv_alloc_seq_len(const pkv_alloc* a, int64_t seq_id, int* len) {
+    if (!a || !len) return PKV_EINVAL;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PKV_ENOSEQ;
+    *len = (int)it->second.len;
+    return PKV_OK;
+}
+
+int pkv_alloc_block_table(const pkv_alloc* a, int64_t seq_id, int32_t* out, int capacity,
+                          int* n_out) {
+    if (!a || !n_out || capacity < 0 || (capacity > 0 && !out)) return PKV_EINVAL;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PKV_ENOSEQ;
+    const auto& t = it->second.table;
+    *n_out = (int)t.size();
+    if ((int64_t)t.size() > capacity) return PKV_EBOUNDS;
+    for (size_t i = 0; i < t.size(); ++i) out[i] = t[i];
+    return PKV_OK;
+}
+
+int pkv_alloc_build_block_tables(const pkv_alloc* a, const int64_t* seq_ids, int n,
+                                 int32_t* tables, int max_blocks, int32_t fill,
+                                 int32_t* context_lens) {
+    if (!a || n < 0 || max_blocks < 0 ||
+        (n > 0 && (!seq_ids || !context_lens || (max_blocks > 0 && !tables))))
+        return PKV_EINVAL;
+    for (int i = 0; i < n; ++i) {  // check everything before writing anything
+        auto it = a->seqs.find(seq_ids[i]);
+        if (it == a->seqs.end()) return PKV_ENOSEQ;
+        if ((int64_t)it->second.table.size() > max_blocks) return PKV_EBOUNDS;
+    }
+    for (int i = 0; i < n; ++i) {
+        const auto& s = a->seqs.find(seq_ids[i])->second;
+        int32_t* row = tables + (int64_t)i * max_blocks;
+        size_t j = 0;
+        for (; j < s.table.size(); ++j) row[j] = s.table[j];
+        for (; j < (size_t)max_blocks; ++j) row[j] = fill;
+        context_lens[i] = (int32_t)s.len;
+    }
+    return PKV_OK;
+}
+
+int pkv_alloc_refcount(const pkv_alloc* a, int32_t block, int* out) {
+    if (!a || !out) return PKV_EINVAL;
+    if (block < 0 || block >= a->num_blocks) return PKV_EBOUNDS;
+    *out = a->ref[block];
+    return PKV_OK;
+}
+
+int pkv_alloc_stats(const pkv_alloc* a, pkv_alloc_stats_t* out) {
+    if (!a || !out) return PKV_EINVAL;
+    out->num_blocks = a->num_blocks;
+    out->block_size = a->block_size;
+    out->free_blocks = (int32_t)a->free_stack.size();
+    out->used_blocks = a->used_blocks;
+    out->shared_blocks = a->shared_blocks;
+    out->num_seqs = (int32_t)a->seqs.size();
+    out->refcount_sum = a->refcount_sum;
+    out->logical_tokens = a->logical_tokens;
+    return PKV_OK;
+}
+
+int pkv_alloc_free_list(const pkv_alloc* a, int32_t* out, int capacity, int* n_out) {
+    if (!a || !n_out || capacity < 0 || (capacity > 0 && !out)) return PKV_EINVAL;
+    const auto& fs = a->free_stack;
+    *n_out = (int)fs.size();
+    if ((int64_t)fs.size() > capacity) return PKV_EBOUNDS;
+    for (size_t i = 0; i < fs.size(); ++i) out[i] = fs[fs.size() - 1 - i];
+    return PKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,115 @@
+// KV append (slot-mapping scatter) and copy-on-write block copies.
+//
+// Both are pure bit moves bound by HBM bandwidth: 16-byte vector loads and
+// stores, several in flight per thread, no shared memory.
+#include "cache_ops.cuh"
+
+namespace pkv {
+
+// One thread per 16-byte vector of the new tokens' [T, Hkv, D] rows.
+// Token t's vector r (r < H * D * e / 16) lands in its slot's row: block
+// s / bs, KV head r / head_vecs, offset s % bs ("What is PagedAttention ..."
+// §How it works: blocks fill as the sequence grows).
+__global__ void __launch_bounds__(256) kv_append_kernel(uint4* __restrict__ kc,
+                                                         uint4* __restrict__ vc,
+                                                         const uint4* __restrict__ k,
+                                                         const uint4* __restrict__ v,
+                                                         const int64_t* __restrict__ slots,
+                                                         int64_t total_vecs, int row_vecs,
+                                                         int head_vecs, int num_kv_heads,
+                                                         int block_size, int64_t num_slots,
+                                                         unsigned int* status) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total_vecs; i += stride) {
+        const int64_t t = i / row_vecs;
+        const int r = (int)(i - t * row_vecs);
+        const int64_t s = slots[t];
+        if (s < 0) continue;  // padding token
+        if (s >= num_slots) {
+            if (r == 0) flag(status, PKV_DEV_BAD_SLOT);
+            continue;
+        }
+        const int h = r / head_vecs;
+        const int c = r - h * head_vecs;
+        const int64_t blk = s / block_size;
+        const int off = (int)(s - blk * block_size);
+        const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_vecs + c;
+        const uint4 kx = k[i];
+        const uint4 vx = v[i];
+        kc[dst] = kx;
+        vc[dst] = vx;
+    }
+}
+
+// Grid (chunks, pairs, 2): blockIdx.z picks K or V.  Each thread moves UNROLL
+// vectors per pass with all loads issued before the stores.
+template <int UNROLL>
+__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ kc,
+                                                           uint4* __restrict__ vc,
+                                                           const int32_t* __restrict__ pairs,
+                                                           int num_pairs, int64_t block_vecs,
+                                                           int num_blocks,
+                                                           unsigned int* status) {
+    uint4* base = blockIdx.z ? vc : kc;
+    for (int pr = blockIdx.y; pr < num_pairs; pr += gridDim.y) {
+        const int32_t src = pairs[2 * pr];
+        const int32_t dst = pairs[2 * pr + 1];
+        if ((unsigned)src >= (unsigned)num_blocks || (unsigned)dst >= (unsigned)num_blocks) {
+            if (blockIdx.x == 0 && blockIdx.z == 0 && threadIdx.x == 0)
+                flag(status, PKV_DEV_BAD_BLOCK);
+            continue;
+        }
+        const uint4* s = base + (int64_t)src * block_vecs;
+        uint4* d = base + (int64_t)dst * block_vecs;
+        const int64_t step = (int64_t)gridDim.x * blockDim.x * UNROLL;
+        for (int64_t i0 = ((int64_t)blockIdx.x * blockDim.x) * UNROLL + threadIdx.x;
+             i0 < block_vecs; i0 += step) {
+            uint4 x[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int64_t i = i0 + (int64_t)u * blockDim.x;
+                if (i < block_vecs) x[u] = s[i];
+            }
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int64_t i = i0 + (int64_t)u * blockDim.x;
+                if (i < block_vecs) d[i] = x[u];
+            }
+        }
+    }
+}
+
+cudaError_t launch_kv_append(void* k_cache, void* v_cache, const void* k, const void* v,
+                             const int64_t* slots, int num_tokens, int num_kv_heads,
+                             int row_bytes_per_head, int block_size, int num_blocks,
+                             unsigned int* status, cudaStream_t stream) {
+    const int head_vecs = row_bytes_per_head / 16;
+    const int row_vecs = head_vecs * num_kv_heads;
+    const int64_t total = (int64_t)num_tokens * row_vecs;
+    if (total == 0) return cudaSuccess;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    kv_append_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slots, total, row_vecs,
+        head_vecs, num_kv_heads, block_size, (int64_t)num_blocks * block_size, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs,
+                               int num_pairs, int64_t block_bytes, int num_blocks,
+                               unsigned int* status, cudaStream_t stream) {
+    if (num_pairs == 0) return cudaSuccess;
+    constexpr int UNROLL = 4;
+    const int64_t block_vecs = block_bytes / 16;
+    int64_t chunks = (block_vecs + 256 * UNROLL - 1) / (256 * UNROLL);
+    if (chunks > 1024) chunks = 1024;
+    const int ys = num_pairs < 65535 ? num_pairs : 65535;
+    dim3 grid((unsigned)chunks, (unsigned)ys, 2);
+    copy_blocks_kernel<UNROLL><<<grid, 256, 0, stream>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, num_pairs,
+        block_vecs, num_blocks, status);
+    return cudaGetLastError();
+}
+
+}  // namespace pkv

@@ -1,0 +1,19 @@
+// Launchers of the KV append and block copy kernels.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace pkv {
+
+// row_bytes_per_head = head_dim * element size (a multiple of 16).
+cudaError_t launch_kv_append(void* k_cache, void* v_cache, const void* k, const void* v,
+                             const int64_t* slots, int num_tokens, int num_kv_heads,
+                             int row_bytes_per_head, int block_size, int num_blocks,
+                             unsigned int* status, cudaStream_t stream);
+
+// block_bytes = num_kv_heads * block_size * head_dim * element size.
+cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs,
+                               int num_pairs, int64_t block_bytes, int num_blocks,
+                               unsigned int* status, cudaStream_t stream);
+
+}  // namespace pkv

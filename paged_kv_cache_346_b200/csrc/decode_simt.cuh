@@ -1,0 +1,348 @@
+// Paged decode attention on the CUDA cores.
+//
+// One CTA takes one (partition of a sequence's context, KV head, slice of HG
+// query heads of that KV head's group).  The steps follow "pagedattention vllm"
+// §Attention Computation: translate each logical block to its physical block
+// through the table, load the physical block, compute attention over the
+// gathered tokens as if they were contiguous.
+//
+//   1. The table entries of the partition are read once, coalesced, into
+//      shared memory (4-byte entries, "pagedattention vllm" §Implementation
+//      Details).
+//   2. One thread issues 1-D bulk copies (TMA, cp.async.bulk) of whole
+//      (block, KV head) pages -- BS x D contiguous elements each for K and for
+//      V -- into a ring of STAGES shared-memory stages of TILE = 16 * NW tokens,
+//      completing on an mbarrier per stage; the copy of stage i + STAGES is
+//      issued as soon as every warp has finished with stage i.
+//   3. Warp w takes tokens [16w, 16w + 16) of each stage.  QK: 8 lanes per
+//      token, each with D/8 dims of q (float32, pre-scaled by scale*log2 e) in
+//      registers; 3 xor-shuffles finish each dot product.  Tokens past the
+//      sequence end get a logit of -inf and their values are never read, so
+//      whatever sits in the unused slots of the last block cannot leak in.
+//   4. Per-warp online softmax in base 2: running max m, sum l, accumulator
+//      rescaled by 2^(m_old - m_new).
+//   5. PV: LPV lanes per token read one 16-byte chunk of v each; the weights
+//      go through a 16-entry per-warp shared array.
+//   6. The NW per-warp (m, l, acc) are merged in shared memory; a one-partition
+//      sequence writes out directly, a longer one writes (m, l, acc / l) to the
+//      workspace for the log-sum-exp reduce.
+#pragma once
+
+#include "decode_common.cuh"
+
+namespace pkv {
+
+template <int ROW_BYTES, int NW>
+struct SimtStages {
+    static constexpr int kTile = 16 * NW;
+    static constexpr int kStageBytes = 2 * kTile * ROW_BYTES;  // K + V
+    static constexpr int kBudget = 98304;                       // two CTAs per SM
+    static constexpr int kStages =
+        kBudget / kStageBytes >= 4 ? 4 : (kBudget / kStageBytes >= 3 ? 3 : 2);
+};
+
+__host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+template <typename T, int D, int BS, int HG, int NW>
+struct SimtCfg {
+    static constexpr int ROW = D * (int)sizeof(T);
+    static constexpr int CPR = ROW / 16;
+    static constexpr int EPC = Elem<T>::kPerVec;
+    static constexpr int TILE = 16 * NW;
+    static constexpr int BPT = TILE / BS;
+    static constexpr int BLK_BYTES = BS * ROW;
+    static constexpr int STAGE_BYTES = TILE * ROW;  // one of K / V
+    static constexpr int STAGES = SimtStages<ROW, NW>::kStages;
+    static constexpr int CPL = CPR / 8;
+    static constexpr int LPV = CPR < 32 ? CPR : 32;
+    static constexpr int TPV = 32 / LPV;
+    static constexpr int CPV = CPR / LPV;
+    static_assert(TILE % BS == 0, "a stage holds whole blocks");
+    static_assert(CPR % 8 == 0, "rows of at least 128 bytes");
+
+    static int smem_bytes(int partition_size) {
+        return 128 + round_up(partition_size / BS * 4, 128) + STAGES * 2 * STAGE_BYTES;
+    }
+};
+
+template <typename T, int D, int BS, int HG, int NW>
+__global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeArgs a) {
+    using C = SimtCfg<T, D, BS, HG, NW>;
+    using E = Elem<T>;
+    constexpr int ROW = C::ROW, EPC = C::EPC, TILE = C::TILE, BPT = C::BPT;
+    constexpr int BLK_BYTES = C::BLK_BYTES, STAGE_BYTES = C::STAGE_BYTES;
+    constexpr int STAGES = C::STAGES, CPL = C::CPL, LPV = C::LPV, TPV = C::TPV;
+    constexpr int CPV = C::CPV;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ float s_p[NW][HG][16];
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.z;
+    const int kvh = blockIdx.y / a.head_chunks;
+    const int hc = blockIdx.y - kvh * a.head_chunks;
+    const int part = blockIdx.x;
+    const int h0 = kvh * a.group + hc * HG;
+    const int nh = min(HG, a.group - hc * HG);
+    const bool reporter = (tid == 0 && part == 0 && blockIdx.y == 0);
+
+    const int L = seq_len(a, b, reporter);
+    const int np = num_partitions(a, L, reporter);
+    T* out = reinterpret_cast<T*>(a.out);
+    if (L == 0) {  // empty sequence: a zero row
+        if (part == 0)
+            for (int i = tid; i < nh * D; i += NW * 32)
+                out[((int64_t)b * a.num_q_heads + h0 + i / D) * D + i % D] = E::from_f32(0.f);
+        return;
+    }
+    if (part >= np) return;
+
+    const int P = a.partition_size;
+    const int t0 = part * P;
+    const int ntok = min(L, t0 + P) - t0;
+    const int ntiles = (ntok + TILE - 1) / TILE;
+    const int nblk = (ntok + BS - 1) / BS;
+
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    int32_t* s_tab = reinterpret_cast<int32_t*>(smem + 128);
+    unsigned char* s_kv = smem + 128 + round_up(P / BS * 4, 128);
+
+    // 1. table slice -> shared memory
+    {
+        const int32_t* trow = a.block_tables + (int64_t)b * a.max_blocks_per_seq + t0 / BS;
+        for (int i = tid; i < nblk; i += NW * 32) {
+            int32_t p = trow[i];
+            if ((unsigned)p >= (unsigned)a.num_blocks) {
+                flag(a.status, PKV_DEV_BAD_BLOCK);
+                p = 0;  // stay inside the pool; the result is flagged as invalid
+            }
+            s_tab[i] = p;
+        }
+    }
+    if (tid == 0) {
+        s_abort = 0;
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    const unsigned char* kbase = reinterpret_cast<const unsigned char*>(a.k_cache);
+    const unsigned char* vbase = reinterpret_cast<const unsigned char*>(a.v_cache);
+    const uint64_t pol = policy_evict_first();
+    auto issue = [&](int tile, int stage) {
+        const int jb = tile * BPT;
+        const int je = min(nblk, jb + BPT);
+        mbar_arrive_expect_tx(&full[stage], (uint32_t)((je - jb) * BLK_BYTES * 2));
+        unsigned char* kd = s_kv + stage * 2 * STAGE_BYTES;
+        unsigned char* vd = kd + STAGE_BYTES;
+        for (int j = jb; j < je; ++j) {
+            const int64_t off = ((int64_t)s_tab[j] * a.num_kv_heads + kvh) * BLK_BYTES;
+            bulk_load(kd + (j - jb) * BLK_BYTES, kbase + off, BLK_BYTES, &full[stage], pol);
+            bulk_load(vd + (j - jb) * BLK_BYTES, vbase + off, BLK_BYTES, &full[stage], pol);
+        }
+    };
+    if (tid == 0) {
+        const int pre = min(STAGES, ntiles);
+        for (int s = 0; s < pre; ++s) issue(s, s);
+    }
+
+    // 3. query slice in registers, scaled to base-2 logits
+    const int grp = lane >> 3, sub = lane & 7;
+    float qf[HG][CPL][EPC];
+    {
+        const T* qb = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D;
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                if (hh < nh) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(qb + hh * D + (sub + 8 * i) * EPC);
+                    E::to_f32(v, qf[hh][i]);
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) qf[hh][i][e] *= a.scale_log2;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) qf[hh][i][e] = 0.f;
+                }
+            }
+    }
+
+    float m[HG], l[HG], acc[HG][CPV][EPC];
+#pragma unroll
+    for (int hh = 0; hh < HG; ++hh) {
+        m[hh] = -INFINITY;
+        l[hh] = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPV; ++c)
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) acc[hh][c][e] = 0.f;
+    }
+    const int lv = lane % LPV, tv = lane / LPV;
+
+    for (int it = 0; it < ntiles; ++it) {
+        const int stage = it % STAGES;
+        const bool ok = mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status);
+        if (!ok) {
+            s_abort = 1;
+        } else {
+            const int wvalid = ntok - (it * TILE + warp * 16);  // tokens this warp owns
+            if (wvalid > 0) {
+                const unsigned char* Kw = s_kv + stage * 2 * STAGE_BYTES + warp * 16 * ROW;
+                const unsigned char* Vw = Kw + STAGE_BYTES;
+                float s[HG][4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int tok = r * 4 + grp;
+                    float d[HG];
+#pragma unroll
+                    for (int hh = 0; hh < HG; ++hh) d[hh] = 0.f;
+#pragma unroll
+                    for (int i = 0; i < CPL; ++i) {
+                        const uint4 kv =
+                            *reinterpret_cast<const uint4*>(Kw + tok * ROW + (sub + 8 * i) * 16);
+                        float kf[EPC];
+                        E::to_f32(kv, kf);
+#pragma unroll
+                        for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+                            for (int e = 0; e < EPC; ++e) d[hh] = fmaf(qf[hh][i][e], kf[e], d[hh]);
+                    }
+#pragma unroll
+                    for (int hh = 0; hh < HG; ++hh) {
+                        d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 1);
+                        d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 2);
+                        d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 4);
+                        s[hh][r] = tok < wvalid ? d[hh] : -INFINITY;
+                    }
+                }
+#pragma unroll
+                for (int hh = 0; hh < HG; ++hh) {
+                    float mx = fmaxf(fmaxf(s[hh][0], s[hh][1]), fmaxf(s[hh][2], s[hh][3]));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    const float mnew = fmaxf(m[hh], mx);  // finite: wvalid > 0
+                    const float alpha = exp2f(m[hh] - mnew);
+                    float ps = 0.f;
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        s[hh][r] = exp2f(s[hh][r] - mnew);
+                        ps += s[hh][r];
+                    }
+                    ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+                    ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+                    l[hh] = l[hh] * alpha + ps;
+                    m[hh] = mnew;
+#pragma unroll
+                    for (int c = 0; c < CPV; ++c)
+#pragma unroll
+                        for (int e = 0; e < EPC; ++e) acc[hh][c][e] *= alpha;
+                    if (sub == 0) {
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) s_p[warp][hh][r * 4 + grp] = s[hh][r];
+                    }
+                }
+                __syncwarp();
+#pragma unroll 4
+                for (int t = tv; t < 16; t += TPV) {
+                    if (t < wvalid) {
+#pragma unroll
+                        for (int c = 0; c < CPV; ++c) {
+                            const uint4 vv =
+                                *reinterpret_cast<const uint4*>(Vw + t * ROW + (lv + c * LPV) * 16);
+                            float vf[EPC];
+                            E::to_f32(vv, vf);
+#pragma unroll
+                            for (int hh = 0; hh < HG; ++hh) {
+                                const float p = s_p[warp][hh][t];
+#pragma unroll
+                                for (int e = 0; e < EPC; ++e)
+                                    acc[hh][c][e] = fmaf(p, vf[e], acc[hh][c][e]);
+                            }
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        __syncthreads();  // every warp is done with this stage
+        if (s_abort) break;
+        if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage);
+    }
+    if (s_abort) return;
+    pdl_launch_dependents();
+
+    // 6. merge the warps
+#pragma unroll
+    for (int msk = LPV; msk < 32; msk <<= 1)
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+            for (int c = 0; c < CPV; ++c)
+#pragma unroll
+                for (int e = 0; e < EPC; ++e)
+                    acc[hh][c][e] += __shfl_xor_sync(0xffffffffu, acc[hh][c][e], msk);
+    float* red = reinterpret_cast<float*>(s_kv);  // [NW][HG][D]
+    float* red_m = red + NW * HG * D;              // [NW][HG]
+    float* red_l = red_m + NW * HG;
+    if (tv == 0) {
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+            for (int c = 0; c < CPV; ++c)
+#pragma unroll
+                for (int e = 0; e < EPC; ++e)
+                    red[(warp * HG + hh) * D + (lv + c * LPV) * EPC + e] = acc[hh][c][e];
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh) {
+            red_m[warp * HG + hh] = m[hh];
+            red_l[warp * HG + hh] = l[hh];
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < nh * D; i += NW * 32) {
+        const int hh = i / D, d = i - hh * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * HG + hh]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float f = exp2f(red_m[w * HG + hh] - M);  // 0 for a warp with no tokens
+            num = fmaf(f, red[(w * HG + hh) * D + d], num);
+            den = fmaf(f, red_l[w * HG + hh], den);
+        }
+        const int64_t row = (int64_t)b * a.num_q_heads + h0 + hh;
+        if (np == 1) {
+            out[row * D + d] = E::from_f32(num / den);
+        } else {
+            const int64_t pr = row * a.max_partitions + part;
+            a.ws_o[pr * D + d] = num / den;
+            if (d == 0) {
+                a.ws_ml[pr * 2] = M;
+                a.ws_ml[pr * 2 + 1] = den;
+            }
+        }
+    }
+}
+
+template <typename T, int D, int BS, int HG>
+cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
+    constexpr int NW = 4;
+    using C = SimtCfg<T, D, BS, HG, NW>;
+    static SmemAttr attr;
+    const int smem = C::smem_bytes(a.partition_size);
+    auto kern = decode_simt_kernel<T, D, BS, HG, NW>;
+    cudaError_t e = attr.ensure(kern, C::smem_bytes(8192));
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
+    kern<<<grid, NW * 32, smem, stream>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || a.max_partitions <= 1) return e;
+    return launch_lse_reduce<T, D>(a, stream);
+}
+
+}  // namespace pkv

@@ -1,0 +1,102 @@
+"""The C-ABI library loads, exports every function include/*.h declares, and
+rejects bad arguments on the host before touching a device."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_346_b200 import _binding as b
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names |= set(re.findall(r"^PKV_API\s+[\w\s\*]+?\b(pkv_\w+)\s*\(", text, flags=re.M))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 20
+    for n in sorted(names):
+        assert hasattr(b.lib, n), n
+    # and the binding declares a signature for each
+    assert names == set(b.SIGNATURES), names ^ set(b.SIGNATURES)
+
+
+def test_status_strings_and_version():
+    assert b.lib.pkv_status_string(0) == b"ok"
+    assert b.lib.pkv_status_string(-2) == b"no free block"
+    assert b.lib.pkv_version() >= 10000
+
+
+def _decode(**over):
+    a = dict(out=None, q=None, k=None, v=None, bt=None, cl=None, B=4, Hq=8, Hkv=2, D=128,
+             bs=16, mb=8, N=64, maxlen=100, scale=0.1, dt=b.PKV_F16, P=0, ws=None, wsb=0,
+             kern=0, stream=None)
+    a.update(over)
+    return b.lib.pkv_paged_attention_decode(
+        a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["B"], a["Hq"], a["Hkv"], a["D"],
+        a["bs"], a["mb"], a["N"], a["maxlen"], a["scale"], a["dt"], a["P"], a["ws"], a["wsb"],
+        a["kern"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(Hq=6, Hkv=4), b.PKV_EINVAL),                 # heads do not divide
+    (dict(B=-1), b.PKV_EINVAL),
+    (dict(maxlen=8 * 16 + 1), b.PKV_EINVAL),            # longer than the table allows
+    (dict(P=100), b.PKV_EINVAL),                        # not a multiple of 64
+    (dict(P=16384), b.PKV_EINVAL),
+    (dict(scale=float("nan")), b.PKV_EINVAL),
+    (dict(dt=7), b.PKV_EINVAL),
+    (dict(kern=9), b.PKV_EINVAL),
+    (dict(D=96), b.PKV_EUNSUPPORTED),
+    (dict(bs=8, maxlen=50), b.PKV_EUNSUPPORTED),
+    (dict(dt=b.PKV_F32, D=256), b.PKV_EUNSUPPORTED),
+    (dict(), b.PKV_EINVAL),                             # null pointers
+])
+def test_decode_host_checks(over, code):
+    assert _decode(**over) == code
+
+
+def test_decode_empty_batch_is_a_no_op():
+    assert _decode(B=0) == b.PKV_OK
+
+
+def test_decode_needs_workspace_for_long_contexts():
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the check fails first
+    assert _decode(out=fake, q=fake, k=fake, v=fake, bt=fake, cl=fake, maxlen=1000,
+                   P=512) == b.PKV_EINVAL
+
+
+def test_workspace_size_formula():
+    f = b.lib.pkv_decode_workspace_size
+    assert f(8, 32, 8, 128, 512, 512) == 0                    # one partition
+    assert f(8, 32, 8, 128, 513, 512) == 8 * 32 * 2 * 130 * 4
+    assert f(8, 32, 8, 128, 131072, 512) == 8 * 32 * 256 * 130 * 4
+    p = b.lib.pkv_decode_default_partition(8, 8, 131072)
+    assert f(8, 32, 8, 128, 131072, 0) == f(8, 32, 8, 128, 131072, p)
+
+
+def test_default_partition_rule():
+    d = b.lib.pkv_decode_default_partition
+    assert d(64, 40, 2048) == 512
+    assert d(1, 1, 4096) == 64          # tiny batches split finer
+    p = d(4, 4, 512)
+    assert 64 <= p <= 512 and p % 64 == 0
+
+
+def test_append_and_copy_host_checks():
+    f = b.lib.pkv_kv_cache_append
+    assert f(None, None, None, None, None, 0, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_OK
+    assert f(None, None, None, None, None, 3, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL
+    assert f(None, None, None, None, None, 3, 4, 7, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL
+    g = b.lib.pkv_copy_blocks
+    assert g(None, None, None, 0, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_OK
+    assert g(None, None, None, 2, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL
+    assert g(None, None, None, -1, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL
