@@ -149,6 +149,42 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
                                pkv_stream_t stream);
 
 /*
+ * Size of the workspace compiled into the library for
+ * pkv_paged_attention_decode_static_ws: 64 MiB per GPU.
+ */
+#define PKV_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
+
+/*
+ * pkv_paged_attention_decode for callers that cannot allocate device memory.
+ * The pages have no counterpart of this call: it exists for callers such as a
+ * plugin inside a host application that owns all device memory and forbids
+ * cudaMalloc, or a serving loop that must not take cudaMalloc's implicit
+ * device synchronisation.  Same arguments, checks, kernels and results as
+ * pkv_paged_attention_decode, minus the workspace: the partition scratch comes
+ * from a fixed array of PKV_STATIC_WORKSPACE_BYTES inside the library, which
+ * every GPU that loads the library's device code holds until the process
+ * exits.  The call itself allocates nothing.
+ *
+ *   - Returns PKV_EBOUNDS, before launching anything, when the shape needs
+ *     more scratch than that (pkv_decode_workspace_size(...) >
+ *     PKV_STATIC_WORKSPACE_BYTES), e.g. far longer contexts or bigger
+ *     batches; use pkv_paged_attention_decode with a caller workspace then.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ *     first call before any stream capture begins.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents.  Nothing in it needs to start at zero, but calls that can
+ *     overlap on the GPU (different streams, no ordering between them) race
+ *     on it: order them, or use the caller-workspace entry point.
+ */
+PKV_API int pkv_paged_attention_decode_static_ws(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_q_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+    int max_context_len, float scale, pkv_dtype dtype, int partition_size, pkv_kernel kernel,
+    pkv_stream_t stream);
+
+/*
  * KV append: the key and value of each new token go into the slot the block
  * manager gave it ("What is PagedAttention ..." §How it works: blocks are
  * filled as the answer grows):

@@ -22,7 +22,8 @@ from ._binding import (PKV_BF16, PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD
                        PKV_KERNEL_SIMT, PagedKVError, check, lib)
 
 __all__ = [
-    "pkv_paged_attention_decode", "pkv_decode_workspace_size", "pkv_decode_has_kernel", "pkv_decode_default_partition",
+    "pkv_paged_attention_decode", "pkv_decode_workspace_size", "pkv_decode_has_kernel",
+    "pkv_paged_attention_decode_static_ws", "pkv_decode_default_partition",
     "pkv_kv_cache_append", "pkv_copy_blocks", "pkv_device_status", "BlockAllocator",
     "PagedKVError", "lib", "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_KERNEL_AUTO",
     "PKV_KERNEL_SIMT", "PKV_KERNEL_MMA", "PKV_DEV_BAD_BLOCK", "PKV_DEV_BAD_LEN",
@@ -105,6 +106,33 @@ def pkv_paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torc
         _ptr(context_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], N,
         int(max_context_len), float(scale), torch_dtype_code(q.dtype), int(partition_size),
         _ptr(workspace), ws_bytes, int(kernel), _stream(stream)), "pkv_paged_attention_decode")
+    return out
+
+
+def pkv_paged_attention_decode_static_ws(out: torch.Tensor, q: torch.Tensor,
+                                         k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                         block_tables: torch.Tensor, context_lens: torch.Tensor,
+                                         scale: float, block_size: int, max_context_len: int, *,
+                                         partition_size: int = 0,
+                                         kernel: int = PKV_KERNEL_AUTO,
+                                         stream=None) -> torch.Tensor:
+    """pkv_paged_attention_decode without a caller workspace, for callers that
+    cannot allocate device memory: the partition scratch is a fixed
+    PKV_STATIC_WORKSPACE_BYTES array inside the library (shared by all calls
+    on a device; calls that overlap on the GPU race on it).  Shapes needing
+    more scratch than that raise PagedKVError (PKV_EBOUNDS)."""
+    for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+                 (block_tables, "block_tables"), (context_lens, "context_lens")):
+        _dev(t, n)
+    B, Hq, D = q.shape
+    N, Hkv, bs, _ = k_cache.shape
+    check(lib.pkv_paged_attention_decode_static_ws(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], N,
+        int(max_context_len), float(scale), torch_dtype_code(q.dtype), int(partition_size),
+        int(kernel), _stream(stream)),
+        f"pkv_paged_attention_decode_static_ws (scratch limit "
+        f"{_b.PKV_STATIC_WORKSPACE_BYTES} bytes)")
     return out
 
 
