@@ -129,20 +129,32 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
 
 
-def kernel_source_digest() -> str:
+KERNEL_SOURCES = {
+    "simt": ("decode_common.cuh", "decode_simt.cuh", "device_common.cuh"),
+    "mma": ("decode_common.cuh", "decode_mma.cuh", "device_common.cuh"),
+}
+
+
+def kernel_source_digest(variant: str) -> str:
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_346_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.startswith("decode") or f in ("device_common.cuh",):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in KERNEL_SOURCES[variant]:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str, kernel: str):
-    """DRAM bytes per decode launch from a committed ncu summary, if it was
+def resolve_variant(cfg, kernel: str) -> str:
+    """The decode kernel the library's automatic choice takes for cfg."""
+    if kernel != "auto":
+        return kernel
+    return "mma" if cfg.dtype != "f32" and 4 <= cfg.group <= 16 else "simt"
+
+
+def recorded_traffic(workload: str, variant: str):
+    """DRAM bytes per decode call from a committed ncu summary, if it was
     taken on the current kernel sources (else None)."""
-    p = os.path.join(ROOT, "profiles", f"decode_{workload}.md")
+    p = os.path.join(ROOT, "profiles", f"decode_{variant}_{workload}.md")
     if not os.path.exists(p):
         return None
     rec = {}
@@ -150,9 +162,7 @@ def recorded_traffic(workload: str, kernel: str):
         if line.startswith("- ") and ":" in line:
             k, v = line[2:].split(":", 1)
             rec[k.strip()] = v.strip().strip("`")
-    if rec.get("kernel_sources_sha256_16") != kernel_source_digest():
-        return None
-    if rec.get("kernel_variant") not in (None, kernel):
+    if rec.get("kernel_sources_sha256_16") != kernel_source_digest(variant):
         return None
     try:
         return int(rec["dram_bytes_per_decode_call"])
@@ -410,7 +420,8 @@ def run_ours(args, cfg):
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": peak_src,
                          "decode_ms": round(dec_ms, 5), "bytes_per_launch": int(dec_bytes),
-                         "traffic": recorded_traffic(cfg.name, args.kernel)},
+                         "variant": resolve_variant(cfg, args.kernel),
+                         "traffic": recorded_traffic(cfg.name, resolve_variant(cfg, args.kernel))},
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -8,6 +8,8 @@
 
 namespace pkv {
 
+__host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
 struct DecodeArgs {
     void* out;                    // [B, Hq, D] T
     const void* q;                // [B, Hq, D] T

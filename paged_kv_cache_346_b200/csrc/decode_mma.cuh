@@ -1,11 +1,417 @@
-// Tensor-core paged decode (query groups of 4..16 heads, f16 / bf16 caches).
+// Paged decode attention on the tensor cores, for query groups of 4 to 16
+// heads per KV head with fp16 / bf16 caches.
+//
+// With G query heads sharing one KV head ("Paged Attention" glossary,
+// systemdesign.academy: grouped-query attention lets several heads share one
+// set of keys and values), each K/V page feeds G dot products per token: for
+// G >= 4 the two products of a CTA's tile are small dense contractions,
+//   S^T[h, t] = sum_d Q[h, d] K[t, d]           (M = heads, N = tokens, K = dims)
+//   O^T[d, h] = sum_t V[t, d] P[h, t]           (M = dims, N = heads, K = tokens)
+// done with mma.sync m16n8k16 (fp16/bf16 inputs, fp32 accumulation).  The QK
+// accumulator layout of S^T is exactly the B-operand layout P^T needs for PV,
+// so P never leaves registers.
+//
+// Pages are staged with 2-D tiled TMA (cp.async.bulk.tensor) over the cache
+// viewed as [N * Hkv * BS rows, D columns], boxes of 64 columns x BS rows,
+// 128-byte swizzle: row r of a box keeps its 16-byte chunk c at position
+// c ^ (r % 8), so the ldmatrix reads of 8 rows at one column hit 8 different
+// bank groups.  Everything else (table hoist, mbarrier ring, per-warp online
+// softmax, warp merge, split-K workspace) mirrors the CUDA-core kernel.
 #pragma once
+
+#include <cuda.h>
 
 #include "decode_common.cuh"
 
 namespace pkv {
 
-constexpr bool kMmaBuilt = false;
+constexpr bool kMmaBuilt = true;
+
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+template <typename T>
+struct Mma;
+
+template <>
+struct Mma<__half> {
+    __device__ __forceinline__ static void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+            "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    // round a pair to the mma input type; lo goes to the low half
+    __device__ __forceinline__ static uint32_t pack(float lo, float hi, float& rlo, float& rhi) {
+        __half2 h = __floats2half2_rn(lo, hi);
+        float2 f = __half22float2(h);
+        rlo = f.x;
+        rhi = f.y;
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+};
+
+template <>
+struct Mma<__nv_bfloat16> {
+    __device__ __forceinline__ static void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+            "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    __device__ __forceinline__ static uint32_t pack(float lo, float hi, float& rlo, float& rhi) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        float2 f = __bfloat1622float2(h);
+        rlo = f.x;
+        rhi = f.y;
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+};
+
+// STAGES_ = 0: the most stages (2 or 3) whose ring lets three CTAs share an SM.
+template <int D, int BS, int NW, int STAGES_ = 0>
+struct MmaCfg {
+    static constexpr int TILE = 16 * NW;         // tokens per stage
+    static constexpr int NX = D / 64;            // 64-column boxes per row
+    static constexpr int BOX_BYTES = BS * 128;   // one box: BS rows x 128 bytes
+    static constexpr int BLK_BYTES = BS * D * 2; // one (block, head) page
+    static constexpr int BPT = TILE / BS;
+    static constexpr int STAGE_BYTES = TILE * D * 2;  // one of K / V
+    static constexpr int STAGES = STAGES_ ? STAGES_ : ((2 * STAGE_BYTES) * 3 <= 73728 ? 3 : 2);
+    static_assert(TILE % BS == 0 && BS % 8 == 0, "whole blocks per stage, swizzle rows");
+
+    static int smem_bytes(int partition_size) {
+        return 1024 + round_up(partition_size / BS * 4, 128) + 1024 + STAGES * 2 * STAGE_BYTES;
+    }
+};
+
+// NH = 8 or 16 query heads per CTA (the M rows of the QK product / the N
+// columns of the PV product); heads past the group are zero rows.
+template <typename T, int D, int BS, int NH, int NW, int STAGES_>
+__global__ void __launch_bounds__(NW * 32)
+    decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv) {
+    using C = MmaCfg<D, BS, NW, STAGES_>;
+    using M = Mma<T>;
+    constexpr int TILE = C::TILE, NX = C::NX, BOX_BYTES = C::BOX_BYTES;
+    constexpr int BLK_BYTES = C::BLK_BYTES, BPT = C::BPT, STAGE_BYTES = C::STAGE_BYTES;
+    constexpr int STAGES = C::STAGES;
+    constexpr int KSTEPS = D / 16;   // k-steps of the QK product, m-tiles of PV
+    constexpr int RB = NH / 8;       // 8-head row blocks
+
+    extern __shared__ __align__(1024) unsigned char smem_mma[];
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int b = blockIdx.z;
+    const int kvh = blockIdx.y / a.head_chunks;
+    const int hc = blockIdx.y - kvh * a.head_chunks;
+    const int part = blockIdx.x;
+    const int h0 = kvh * a.group + hc * NH;
+    const int nh = min(NH, a.group - hc * NH);
+    const bool reporter = (tid == 0 && part == 0 && blockIdx.y == 0);
+
+    const int L = seq_len(a, b, reporter);
+    const int np = num_partitions(a, L, reporter);
+    T* out = reinterpret_cast<T*>(a.out);
+    if (L == 0) {
+        if (part == 0)
+            for (int i = tid; i < nh * D; i += NW * 32)
+                out[((int64_t)b * a.num_q_heads + h0 + i / D) * D + i % D] = Elem<T>::from_f32(0.f);
+        return;
+    }
+    if (part >= np) return;
+
+    const int P = a.partition_size;
+    const int t0 = part * P;
+    const int ntok = min(L, t0 + P) - t0;
+    const int ntiles = (ntok + TILE - 1) / TILE;
+    const int nblk = (ntok + BS - 1) / BS;
+
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem_mma);
+    int32_t* s_tab = reinterpret_cast<int32_t*>(smem_mma + 1024);
+    unsigned char* s_kv;
+    {
+        const uint32_t base = smem_u32(smem_mma + 1024 + round_up(P / BS * 4, 128));
+        const uint32_t aligned = (base + 1023u) & ~1023u;  // 128-byte swizzle: 1 KB atoms
+        s_kv = smem_mma + 1024 + round_up(P / BS * 4, 128) + (aligned - base);
+    }
+
+    {
+        const int32_t* trow = a.block_tables + (int64_t)b * a.max_blocks_per_seq + t0 / BS;
+        for (int i = tid; i < nblk; i += NW * 32) {
+            int32_t p = trow[i];
+            if ((unsigned)p >= (unsigned)a.num_blocks) {
+                flag(a.status, PKV_DEV_BAD_BLOCK);
+                p = 0;
+            }
+            s_tab[i] = p;
+        }
+    }
+    if (tid == 0) {
+        s_abort = 0;
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    const uint64_t pol = policy_evict_first();
+    auto issue = [&](int tile, int stage) {
+        const int jb = tile * BPT;
+        const int je = min(nblk, jb + BPT);
+        mbar_arrive_expect_tx(&full[stage], (uint32_t)((je - jb) * BLK_BYTES * 2));
+        unsigned char* kd = s_kv + stage * 2 * STAGE_BYTES;
+        unsigned char* vd = kd + STAGE_BYTES;
+        for (int j = jb; j < je; ++j) {
+            const int y = (s_tab[j] * a.num_kv_heads + kvh) * BS;
+#pragma unroll
+            for (int x = 0; x < NX; ++x) {
+                const int off = ((j - jb) * NX + x) * BOX_BYTES;
+                tma_load_2d(kd + off, &tmk, x * 64, y, &full[stage], pol);
+                tma_load_2d(vd + off, &tmv, x * 64, y, &full[stage], pol);
+            }
+        }
+    };
+    if (tid == 0) {
+        const int pre = min(STAGES, ntiles);
+        for (int s = 0; s < pre; ++s) issue(s, s);
+    }
+
+    // Q as the A operand: rows = heads (g, g + 8), columns = dims.
+    uint32_t qa[KSTEPS][4];
+    {
+        const T* qb = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {  // r = 0: head g, r = 1: head g + 8
+                const int hh = g + 8 * r;
+                uint32_t lo = 0, hi = 0;
+                if (hh < nh) {
+                    lo = *reinterpret_cast<const uint32_t*>(qb + hh * D + ks * 16 + 2 * t4);
+                    hi = *reinterpret_cast<const uint32_t*>(qb + hh * D + ks * 16 + 8 + 2 * t4);
+                }
+                qa[ks][r] = lo;       // a0 (r = 0) / a1 (r = 1)
+                qa[ks][2 + r] = hi;   // a2 / a3
+            }
+        }
+    }
+
+    float m[RB], l[RB];
+    float o[KSTEPS][RB][4];
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) {
+        m[rb] = -INFINITY;
+        l[rb] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[mt][rb][i] = 0.f;
+    }
+
+    // ldmatrix row addresses: lane -> (token within the warp's 16, chunk parity)
+    const int lrow = (lane >> 4) * 8 + (lane & 7);
+    const int lchunk = (lane >> 3) & 1;
+
+    for (int it = 0; it < ntiles; ++it) {
+        const int stage = it % STAGES;
+        const bool ok = mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status);
+        if (!ok) {
+            s_abort = 1;
+        } else {
+            const int wvalid = ntok - (it * TILE + warp * 16);
+            if (wvalid > 0) {
+                const int tt0 = warp * 16;           // first token of the warp in the stage
+                const int jw = tt0 / BS;             // its block within the stage
+                const int rr = tt0 % BS + lrow;      // this lane's row within that block
+                const uint32_t kbase = smem_u32(s_kv + stage * 2 * STAGE_BYTES) +
+                                       (uint32_t)(jw * NX * BOX_BYTES + rr * 128);
+                const uint32_t vbase = kbase + STAGE_BYTES;
+                const int swz = rr & 7;
+
+                // S^T = Q K^T: two n-tiles of 8 tokens
+                float s[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    const int chunk = ks * 2 + lchunk;           // 16-byte chunk of the row
+                    const int x = chunk >> 3, c = chunk & 7;
+                    uint32_t kb[4];
+                    ldsm_x4(kbase + x * BOX_BYTES + ((c ^ swz) << 4), kb);
+                    M::run(s[0], qa[ks], kb[0], kb[1]);
+                    M::run(s[1], qa[ks], kb[2], kb[3]);
+                }
+                // logits in base 2, masked past the sequence end
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int tok = nt * 8 + 2 * t4 + (i & 1);
+                        s[nt][i] = tok < wvalid ? s[nt][i] * a.scale_log2 : -INFINITY;
+                    }
+                uint32_t pb[RB][2];
+                float alpha_c[RB][2];
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) {
+                    const int i0 = 2 * rb;  // s[nt][i0], s[nt][i0 + 1]: head g + 8 rb
+                    float mx = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    const float mnew = fmaxf(m[rb], mx);
+                    const float alpha = exp2f(m[rb] - mnew);
+                    float p[2][2], pr[2][2];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        p[nt][0] = exp2f(s[nt][i0] - mnew);
+                        p[nt][1] = exp2f(s[nt][i0 + 1] - mnew);
+                        pb[rb][nt] = M::pack(p[nt][0], p[nt][1], pr[nt][0], pr[nt][1]);
+                    }
+                    float ps = (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+                    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+                    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+                    l[rb] = l[rb] * alpha + ps;
+                    m[rb] = mnew;
+                    // O^T columns of this thread are heads 2 t4, 2 t4 + 1 (+ 8 rb)
+                    alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
+                    alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
+                }
+                // O^T += V^T P^T
+                const bool partial = wvalid < 16;
+#pragma unroll
+                for (int mt = 0; mt < KSTEPS; ++mt) {
+                    const int chunk = mt * 2 + lchunk;
+                    const int x = chunk >> 3, c = chunk & 7;
+                    uint32_t va[4];
+                    ldsm_x4_trans(vbase + x * BOX_BYTES + ((c ^ swz) << 4), va);
+                    if (partial) {
+                        // zero values of tokens past the end (0 * NaN would poison)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int tk = (i >> 1) * 8 + 2 * t4;
+                            const uint32_t keep = (tk < wvalid ? 0x0000ffffu : 0u) |
+                                                  (tk + 1 < wvalid ? 0xffff0000u : 0u);
+                            va[i] &= keep;
+                        }
+                    }
+#pragma unroll
+                    for (int rb = 0; rb < RB; ++rb) {
+                        o[mt][rb][0] *= alpha_c[rb][0];
+                        o[mt][rb][1] *= alpha_c[rb][1];
+                        o[mt][rb][2] *= alpha_c[rb][0];
+                        o[mt][rb][3] *= alpha_c[rb][1];
+                        M::run(o[mt][rb], va, pb[rb][0], pb[rb][1]);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (s_abort) break;
+        if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage);
+    }
+    if (s_abort) return;
+    pdl_launch_dependents();
+
+    // merge the warps: red[w][head][dim], red_m / red_l [w][head]
+    float* red = reinterpret_cast<float*>(s_kv);
+    float* red_m = red + NW * NH * D;
+    float* red_l = red_m + NW * NH;
+#pragma unroll
+    for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+        for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int head = 8 * rb + 2 * t4 + (i & 1);
+                const int dim = mt * 16 + g + 8 * (i >> 1);
+                red[(warp * NH + head) * D + dim] = o[mt][rb][i];
+            }
+    if (t4 == 0) {
+#pragma unroll
+        for (int rb = 0; rb < RB; ++rb) {
+            red_m[warp * NH + g + 8 * rb] = m[rb];
+            red_l[warp * NH + g + 8 * rb] = l[rb];
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < nh * D; i += NW * 32) {
+        const int hh = i / D, d = i - hh * D;
+        float Mx = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) Mx = fmaxf(Mx, red_m[w * NH + hh]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float f = exp2f(red_m[w * NH + hh] - Mx);
+            num = fmaf(f, red[(w * NH + hh) * D + d], num);
+            den = fmaf(f, red_l[w * NH + hh], den);
+        }
+        const int64_t row = (int64_t)b * a.num_q_heads + h0 + hh;
+        if (np == 1) {
+            out[row * D + d] = Elem<T>::from_f32(num / den);
+        } else {
+            const int64_t pr = row * a.max_partitions + part;
+            a.ws_o[pr * D + d] = num / den;
+            if (d == 0) {
+                a.ws_ml[pr * 2] = Mx;
+                a.ws_ml[pr * 2 + 1] = den;
+            }
+        }
+    }
+}
+
+// Host side: tensor maps over the K and V pools, launch, optional reduce.
+cudaError_t make_cache_tensor_map(CUtensorMap* map, const void* base, int dtype_bytes,
+                                  bool bf16, int head_dim, int64_t rows, int box_rows);
+
+template <typename T, int D, int BS, int NH, int NW = 4, int STAGES = 0>
+cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
+    using C = MmaCfg<D, BS, NW, STAGES>;
+    static SmemAttr attr;
+    auto kern = decode_mma_kernel<T, D, BS, NH, NW, STAGES>;
+    cudaError_t e = attr.ensure(kern, C::smem_bytes(8192));
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
+    CUtensorMap tk, tv;
+    const bool bf = std::is_same<T, __nv_bfloat16>::value;
+    e = make_cache_tensor_map(&tk, a.k_cache, 2, bf, D, rows, BS);
+    if (e != cudaSuccess) return e;
+    e = make_cache_tensor_map(&tv, a.v_cache, 2, bf, D, rows, BS);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
+    kern<<<grid, NW * 32, C::smem_bytes(a.partition_size), stream>>>(a, tk, tv);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || a.max_partitions <= 1) return e;
+    return launch_lse_reduce<T, D>(a, stream);
+}
 
 cudaError_t decode_mma_f16(const DecodeArgs& a, int head_dim, int block_size, int hg,
                            cudaStream_t stream);

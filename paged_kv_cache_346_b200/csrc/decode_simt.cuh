@@ -32,18 +32,24 @@
 
 namespace pkv {
 
+// Stage count: the most stages (2..4) whose ring still lets three CTAs share
+// an SM (<= 72 KB).  Measured on B200 for the 40-head fp16 layer: three
+// CTAs of 2 x 32 KB stages stream at 6.4 TB/s where two CTAs of 3 stages
+// reach 5.2 TB/s -- more independent CTAs per SM hide the DRAM latency and
+// the per-CTA start-up better than deeper rings.
 template <int ROW_BYTES, int NW>
 struct SimtStages {
     static constexpr int kTile = 16 * NW;
     static constexpr int kStageBytes = 2 * kTile * ROW_BYTES;  // K + V
-    static constexpr int kBudget = 98304;                       // two CTAs per SM
+    static constexpr int kBudget = 73728;
     static constexpr int kStages =
         kBudget / kStageBytes >= 4 ? 4 : (kBudget / kStageBytes >= 3 ? 3 : 2);
 };
 
-__host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
-
-template <typename T, int D, int BS, int HG, int NW>
+// STAGES_ = 0 picks the stage count by SimtStages; WS = true adds a
+// producer warp that re-arms each stage as soon as the consumer warps have
+// released it (per-stage "empty" mbarriers) instead of a CTA-wide barrier.
+template <typename T, int D, int BS, int HG, int NW, int STAGES_ = 0, bool WS = false>
 struct SimtCfg {
     static constexpr int ROW = D * (int)sizeof(T);
     static constexpr int CPR = ROW / 16;
@@ -52,11 +58,12 @@ struct SimtCfg {
     static constexpr int BPT = TILE / BS;
     static constexpr int BLK_BYTES = BS * ROW;
     static constexpr int STAGE_BYTES = TILE * ROW;  // one of K / V
-    static constexpr int STAGES = SimtStages<ROW, NW>::kStages;
+    static constexpr int STAGES = STAGES_ ? STAGES_ : SimtStages<ROW, NW>::kStages;
     static constexpr int CPL = CPR / 8;
     static constexpr int LPV = CPR < 32 ? CPR : 32;
     static constexpr int TPV = 32 / LPV;
     static constexpr int CPV = CPR / LPV;
+    static constexpr int THREADS = (NW + (WS ? 1 : 0)) * 32;
     static_assert(TILE % BS == 0, "a stage holds whole blocks");
     static_assert(CPR % 8 == 0, "rows of at least 128 bytes");
 
@@ -65,18 +72,199 @@ struct SimtCfg {
     }
 };
 
-template <typename T, int D, int BS, int HG, int NW>
-__global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeArgs a) {
-    using C = SimtCfg<T, D, BS, HG, NW>;
+// One consumer warp's share of a partition: its q slice, online-softmax state
+// and accumulator, and the per-stage work on its 16 tokens.
+template <typename T, int D, int HG, typename C>
+struct SimtWarp {
     using E = Elem<T>;
-    constexpr int ROW = C::ROW, EPC = C::EPC, TILE = C::TILE, BPT = C::BPT;
-    constexpr int BLK_BYTES = C::BLK_BYTES, STAGE_BYTES = C::STAGE_BYTES;
-    constexpr int STAGES = C::STAGES, CPL = C::CPL, LPV = C::LPV, TPV = C::TPV;
-    constexpr int CPV = C::CPV;
+    static constexpr int ROW = C::ROW, EPC = C::EPC, CPL = C::CPL, LPV = C::LPV;
+    static constexpr int TPV = C::TPV, CPV = C::CPV;
 
-    extern __shared__ __align__(128) unsigned char smem[];
+    float qf[HG][CPL][EPC];
+    float m[HG], l[HG], acc[HG][CPV][EPC];
+    int lane, grp, sub, lv, tv;
+
+    __device__ __forceinline__ void init(const T* qb, int nh, float scale_log2, int lane_) {
+        lane = lane_;
+        grp = lane >> 3;
+        sub = lane & 7;
+        lv = lane % LPV;
+        tv = lane / LPV;
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh) {
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                if (hh < nh) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(qb + hh * D + (sub + 8 * i) * EPC);
+                    E::to_f32(v, qf[hh][i]);
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) qf[hh][i][e] *= scale_log2;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) qf[hh][i][e] = 0.f;
+                }
+            }
+            m[hh] = -INFINITY;
+            l[hh] = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPV; ++c)
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc[hh][c][e] = 0.f;
+        }
+    }
+
+    // 16 tokens at Kw / Vw (rows of ROW bytes), the first `wvalid` of them
+    // inside the sequence.  s_p: this warp's [HG][16] weight scratch.
+    __device__ __forceinline__ void tile(const unsigned char* Kw, const unsigned char* Vw,
+                                         int wvalid, float (*s_p)[16]) {
+        float s[HG][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int tok = r * 4 + grp;
+            float d[HG];
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh) d[hh] = 0.f;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const uint4 kv = *reinterpret_cast<const uint4*>(Kw + tok * ROW + (sub + 8 * i) * 16);
+                float kf[EPC];
+                E::to_f32(kv, kf);
+#pragma unroll
+                for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) d[hh] = fmaf(qf[hh][i][e], kf[e], d[hh]);
+            }
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh) {
+                d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 1);
+                d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 2);
+                d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 4);
+                s[hh][r] = tok < wvalid ? d[hh] : -INFINITY;
+            }
+        }
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh) {
+            float mx = fmaxf(fmaxf(s[hh][0], s[hh][1]), fmaxf(s[hh][2], s[hh][3]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float mnew = fmaxf(m[hh], mx);  // finite: wvalid > 0
+            const float alpha = exp2f(m[hh] - mnew);
+            float ps = 0.f;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                s[hh][r] = exp2f(s[hh][r] - mnew);
+                ps += s[hh][r];
+            }
+            ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+            l[hh] = l[hh] * alpha + ps;
+            m[hh] = mnew;
+#pragma unroll
+            for (int c = 0; c < CPV; ++c)
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc[hh][c][e] *= alpha;
+            if (sub == 0) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r) s_p[hh][r * 4 + grp] = s[hh][r];
+            }
+        }
+        __syncwarp();
+#pragma unroll 4
+        for (int t = tv; t < 16; t += TPV) {
+            if (t < wvalid) {  // values past the end are never read (they may be NaN)
+#pragma unroll
+                for (int c = 0; c < CPV; ++c) {
+                    const uint4 vv = *reinterpret_cast<const uint4*>(Vw + t * ROW + (lv + c * LPV) * 16);
+                    float vf[EPC];
+                    E::to_f32(vv, vf);
+#pragma unroll
+                    for (int hh = 0; hh < HG; ++hh) {
+                        const float p = s_p[hh][t];
+#pragma unroll
+                        for (int e = 0; e < EPC; ++e) acc[hh][c][e] = fmaf(p, vf[e], acc[hh][c][e]);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    }
+
+    // Fold the token lanes together and park (m, l, acc) in red* for the merge.
+    __device__ __forceinline__ void park(int warp, float* red, float* red_m, float* red_l) {
+#pragma unroll
+        for (int msk = LPV; msk < 32; msk <<= 1)
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+                for (int c = 0; c < CPV; ++c)
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e)
+                        acc[hh][c][e] += __shfl_xor_sync(0xffffffffu, acc[hh][c][e], msk);
+        if (tv == 0) {
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+                for (int c = 0; c < CPV; ++c)
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e)
+                        red[(warp * HG + hh) * D + (lv + c * LPV) * EPC + e] = acc[hh][c][e];
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh) {
+                red_m[warp * HG + hh] = m[hh];
+                red_l[warp * HG + hh] = l[hh];
+            }
+        }
+    }
+};
+
+// Merge NW parked warp states (red*) of nh heads and write the output row (one
+// partition) or the partition's (m, l, o) to the workspace.
+template <typename T, int D, int NH, int NW>
+__device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, const float* red,
+                                                      const float* red_m, const float* red_l,
+                                                      int b, int h0, int nh, int part, int np,
+                                                      int tid, int nthreads) {
+    T* out = reinterpret_cast<T*>(a.out);
+    for (int i = tid; i < nh * D; i += nthreads) {
+        const int hh = i / D, d = i - hh * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * NH + hh]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float f = exp2f(red_m[w * NH + hh] - M);  // 0 for a warp with no tokens
+            num = fmaf(f, red[(w * NH + hh) * D + d], num);
+            den = fmaf(f, red_l[w * NH + hh], den);
+        }
+        const int64_t row = (int64_t)b * a.num_q_heads + h0 + hh;
+        if (np == 1) {
+            out[row * D + d] = Elem<T>::from_f32(num / den);
+        } else {
+            const int64_t pr = row * a.max_partitions + part;
+            a.ws_o[pr * D + d] = num / den;
+            if (d == 0) {
+                a.ws_ml[pr * 2] = M;
+                a.ws_ml[pr * 2 + 1] = den;
+            }
+        }
+    }
+}
+
+template <typename T, int D, int BS, int HG, int NW, int STAGES_, bool WS>
+__global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREADS)
+    decode_simt_kernel(const DecodeArgs a) {
+    using C = SimtCfg<T, D, BS, HG, NW, STAGES_, WS>;
+    using E = Elem<T>;
+    constexpr int ROW = C::ROW, TILE = C::TILE, BPT = C::BPT;
+    constexpr int BLK_BYTES = C::BLK_BYTES, STAGE_BYTES = C::STAGE_BYTES;
+    constexpr int STAGES = C::STAGES, THREADS = C::THREADS;
+
+    extern __shared__ __align__(128) unsigned char smem_simt[];
     __shared__ float s_p[NW][HG][16];
-    __shared__ int s_abort;
+    __shared__ volatile int s_abort;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z;
@@ -89,11 +277,12 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeArgs a
 
     const int L = seq_len(a, b, reporter);
     const int np = num_partitions(a, L, reporter);
-    T* out = reinterpret_cast<T*>(a.out);
     if (L == 0) {  // empty sequence: a zero row
-        if (part == 0)
-            for (int i = tid; i < nh * D; i += NW * 32)
+        if (part == 0) {
+            T* out = reinterpret_cast<T*>(a.out);
+            for (int i = tid; i < nh * D; i += THREADS)
                 out[((int64_t)b * a.num_q_heads + h0 + i / D) * D + i % D] = E::from_f32(0.f);
+        }
         return;
     }
     if (part >= np) return;
@@ -104,14 +293,15 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeArgs a
     const int ntiles = (ntok + TILE - 1) / TILE;
     const int nblk = (ntok + BS - 1) / BS;
 
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-    int32_t* s_tab = reinterpret_cast<int32_t*>(smem + 128);
-    unsigned char* s_kv = smem + 128 + round_up(P / BS * 4, 128);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem_simt);
+    uint64_t* empty = full + STAGES;  // WS only
+    int32_t* s_tab = reinterpret_cast<int32_t*>(smem_simt + 128);
+    unsigned char* s_kv = smem_simt + 128 + round_up(P / BS * 4, 128);
 
     // 1. table slice -> shared memory
     {
         const int32_t* trow = a.block_tables + (int64_t)b * a.max_blocks_per_seq + t0 / BS;
-        for (int i = tid; i < nblk; i += NW * 32) {
+        for (int i = tid; i < nblk; i += THREADS) {
             int32_t p = trow[i];
             if ((unsigned)p >= (unsigned)a.num_blocks) {
                 flag(a.status, PKV_DEV_BAD_BLOCK);
@@ -123,15 +313,17 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeArgs a
     if (tid == 0) {
         s_abort = 0;
 #pragma unroll
-        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            if (WS) mbar_init(&empty[s], NW);
+        }
         fence_barrier_init();
     }
     __syncthreads();
 
     const unsigned char* kbase = reinterpret_cast<const unsigned char*>(a.k_cache);
     const unsigned char* vbase = reinterpret_cast<const unsigned char*>(a.v_cache);
-    const uint64_t pol = policy_evict_first();
-    auto issue = [&](int tile, int stage) {
+    auto issue = [&](int tile, int stage, uint64_t pol) {
         const int jb = tile * BPT;
         const int je = min(nblk, jb + BPT);
         mbar_arrive_expect_tx(&full[stage], (uint32_t)((je - jb) * BLK_BYTES * 2));
@@ -143,203 +335,87 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeArgs a
             bulk_load(vd + (j - jb) * BLK_BYTES, vbase + off, BLK_BYTES, &full[stage], pol);
         }
     };
-    if (tid == 0) {
-        const int pre = min(STAGES, ntiles);
-        for (int s = 0; s < pre; ++s) issue(s, s);
-    }
 
-    // 3. query slice in registers, scaled to base-2 logits
-    const int grp = lane >> 3, sub = lane & 7;
-    float qf[HG][CPL][EPC];
-    {
-        const T* qb = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D;
-#pragma unroll
-        for (int hh = 0; hh < HG; ++hh)
-#pragma unroll
-            for (int i = 0; i < CPL; ++i) {
-                if (hh < nh) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(qb + hh * D + (sub + 8 * i) * EPC);
-                    E::to_f32(v, qf[hh][i]);
-#pragma unroll
-                    for (int e = 0; e < EPC; ++e) qf[hh][i][e] *= a.scale_log2;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < EPC; ++e) qf[hh][i][e] = 0.f;
+    float* red = reinterpret_cast<float*>(s_kv);  // [NW][HG][D], after the last stage
+    float* red_m = red + NW * HG * D;              // [NW][HG]
+    float* red_l = red_m + NW * HG;
+
+    if (WS && warp == NW) {
+        // 2. producer warp: keep every stage loaded as soon as it is released
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            for (int it = 0; it < ntiles; ++it) {
+                const int stage = it % STAGES;
+                if (it >= STAGES &&
+                    !mbar_wait(&empty[stage], (uint32_t)(((it / STAGES) - 1) & 1), a.status)) {
+                    s_abort = 1;
+                    break;
                 }
+                if (s_abort) break;
+                issue(it, stage, pol);
             }
+        }
+        __syncthreads();  // matches the consumers' barrier before the merge
+        if (s_abort) return;
+        pdl_launch_dependents();
+        __syncthreads();
+        merge_warps_and_store<T, D, HG, NW>(a, red, red_m, red_l, b, h0, nh, part, np, tid,
+                                            THREADS);
+        return;
     }
 
-    float m[HG], l[HG], acc[HG][CPV][EPC];
-#pragma unroll
-    for (int hh = 0; hh < HG; ++hh) {
-        m[hh] = -INFINITY;
-        l[hh] = 0.f;
-#pragma unroll
-        for (int c = 0; c < CPV; ++c)
-#pragma unroll
-            for (int e = 0; e < EPC; ++e) acc[hh][c][e] = 0.f;
+    if (!WS && tid == 0) {
+        const uint64_t pol = policy_evict_first();
+        const int pre = min(STAGES, ntiles);
+        for (int s = 0; s < pre; ++s) issue(s, s, pol);
     }
-    const int lv = lane % LPV, tv = lane / LPV;
 
+    // 3.-5. consumer warps
+    SimtWarp<T, D, HG, C> W;
+    W.init(reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D, nh,
+           a.scale_log2, lane);
+    const uint64_t pol = WS ? 0 : policy_evict_first();
     for (int it = 0; it < ntiles; ++it) {
         const int stage = it % STAGES;
-        const bool ok = mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status);
-        if (!ok) {
-            s_abort = 1;
-        } else {
+        if (!mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status)) s_abort = 1;
+        if (WS && s_abort) break;
+        if (!s_abort) {
             const int wvalid = ntok - (it * TILE + warp * 16);  // tokens this warp owns
             if (wvalid > 0) {
                 const unsigned char* Kw = s_kv + stage * 2 * STAGE_BYTES + warp * 16 * ROW;
-                const unsigned char* Vw = Kw + STAGE_BYTES;
-                float s[HG][4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int tok = r * 4 + grp;
-                    float d[HG];
-#pragma unroll
-                    for (int hh = 0; hh < HG; ++hh) d[hh] = 0.f;
-#pragma unroll
-                    for (int i = 0; i < CPL; ++i) {
-                        const uint4 kv =
-                            *reinterpret_cast<const uint4*>(Kw + tok * ROW + (sub + 8 * i) * 16);
-                        float kf[EPC];
-                        E::to_f32(kv, kf);
-#pragma unroll
-                        for (int hh = 0; hh < HG; ++hh)
-#pragma unroll
-                            for (int e = 0; e < EPC; ++e) d[hh] = fmaf(qf[hh][i][e], kf[e], d[hh]);
-                    }
-#pragma unroll
-                    for (int hh = 0; hh < HG; ++hh) {
-                        d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 1);
-                        d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 2);
-                        d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 4);
-                        s[hh][r] = tok < wvalid ? d[hh] : -INFINITY;
-                    }
-                }
-#pragma unroll
-                for (int hh = 0; hh < HG; ++hh) {
-                    float mx = fmaxf(fmaxf(s[hh][0], s[hh][1]), fmaxf(s[hh][2], s[hh][3]));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                    const float mnew = fmaxf(m[hh], mx);  // finite: wvalid > 0
-                    const float alpha = exp2f(m[hh] - mnew);
-                    float ps = 0.f;
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        s[hh][r] = exp2f(s[hh][r] - mnew);
-                        ps += s[hh][r];
-                    }
-                    ps += __shfl_xor_sync(0xffffffffu, ps, 8);
-                    ps += __shfl_xor_sync(0xffffffffu, ps, 16);
-                    l[hh] = l[hh] * alpha + ps;
-                    m[hh] = mnew;
-#pragma unroll
-                    for (int c = 0; c < CPV; ++c)
-#pragma unroll
-                        for (int e = 0; e < EPC; ++e) acc[hh][c][e] *= alpha;
-                    if (sub == 0) {
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) s_p[warp][hh][r * 4 + grp] = s[hh][r];
-                    }
-                }
-                __syncwarp();
-#pragma unroll 4
-                for (int t = tv; t < 16; t += TPV) {
-                    if (t < wvalid) {
-#pragma unroll
-                        for (int c = 0; c < CPV; ++c) {
-                            const uint4 vv =
-                                *reinterpret_cast<const uint4*>(Vw + t * ROW + (lv + c * LPV) * 16);
-                            float vf[EPC];
-                            E::to_f32(vv, vf);
-#pragma unroll
-                            for (int hh = 0; hh < HG; ++hh) {
-                                const float p = s_p[warp][hh][t];
-#pragma unroll
-                                for (int e = 0; e < EPC; ++e)
-                                    acc[hh][c][e] = fmaf(p, vf[e], acc[hh][c][e]);
-                            }
-                        }
-                    }
-                }
-                __syncwarp();
+                W.tile(Kw, Kw + STAGE_BYTES, wvalid, s_p[warp]);
             }
         }
-        __syncthreads();  // every warp is done with this stage
-        if (s_abort) break;
-        if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage);
+        if (WS) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+        } else {
+            __syncthreads();  // every warp is done with this stage
+            if (s_abort) break;
+            if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage, pol);
+        }
     }
+    if (WS) __syncthreads();  // producer and consumers: every stage consumed
     if (s_abort) return;
-    pdl_launch_dependents();
+    if (!WS) pdl_launch_dependents();
 
     // 6. merge the warps
-#pragma unroll
-    for (int msk = LPV; msk < 32; msk <<= 1)
-#pragma unroll
-        for (int hh = 0; hh < HG; ++hh)
-#pragma unroll
-            for (int c = 0; c < CPV; ++c)
-#pragma unroll
-                for (int e = 0; e < EPC; ++e)
-                    acc[hh][c][e] += __shfl_xor_sync(0xffffffffu, acc[hh][c][e], msk);
-    float* red = reinterpret_cast<float*>(s_kv);  // [NW][HG][D]
-    float* red_m = red + NW * HG * D;              // [NW][HG]
-    float* red_l = red_m + NW * HG;
-    if (tv == 0) {
-#pragma unroll
-        for (int hh = 0; hh < HG; ++hh)
-#pragma unroll
-            for (int c = 0; c < CPV; ++c)
-#pragma unroll
-                for (int e = 0; e < EPC; ++e)
-                    red[(warp * HG + hh) * D + (lv + c * LPV) * EPC + e] = acc[hh][c][e];
-    }
-    if (lane == 0) {
-#pragma unroll
-        for (int hh = 0; hh < HG; ++hh) {
-            red_m[warp * HG + hh] = m[hh];
-            red_l[warp * HG + hh] = l[hh];
-        }
-    }
+    W.park(warp, red, red_m, red_l);
     __syncthreads();
-    for (int i = tid; i < nh * D; i += NW * 32) {
-        const int hh = i / D, d = i - hh * D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * HG + hh]);
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-            const float f = exp2f(red_m[w * HG + hh] - M);  // 0 for a warp with no tokens
-            num = fmaf(f, red[(w * HG + hh) * D + d], num);
-            den = fmaf(f, red_l[w * HG + hh], den);
-        }
-        const int64_t row = (int64_t)b * a.num_q_heads + h0 + hh;
-        if (np == 1) {
-            out[row * D + d] = E::from_f32(num / den);
-        } else {
-            const int64_t pr = row * a.max_partitions + part;
-            a.ws_o[pr * D + d] = num / den;
-            if (d == 0) {
-                a.ws_ml[pr * 2] = M;
-                a.ws_ml[pr * 2 + 1] = den;
-            }
-        }
-    }
+    merge_warps_and_store<T, D, HG, NW>(a, red, red_m, red_l, b, h0, nh, part, np, tid,
+                                        WS ? THREADS : NW * 32);
 }
 
-template <typename T, int D, int BS, int HG>
+template <typename T, int D, int BS, int HG, int NW = 4, int STAGES = 0, bool WS = false>
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
-    constexpr int NW = 4;
-    using C = SimtCfg<T, D, BS, HG, NW>;
+    using C = SimtCfg<T, D, BS, HG, NW, STAGES, WS>;
     static SmemAttr attr;
-    const int smem = C::smem_bytes(a.partition_size);
-    auto kern = decode_simt_kernel<T, D, BS, HG, NW>;
+    const int smem_simt = C::smem_bytes(a.partition_size);
+    auto kern = decode_simt_kernel<T, D, BS, HG, NW, STAGES, WS>;
     cudaError_t e = attr.ensure(kern, C::smem_bytes(8192));
     if (e != cudaSuccess) return e;
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
-    kern<<<grid, NW * 32, smem, stream>>>(a);
+    kern<<<grid, C::THREADS, smem_simt, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess || a.max_partitions <= 1) return e;
     return launch_lse_reduce<T, D>(a, stream);

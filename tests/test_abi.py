@@ -85,7 +85,8 @@ def test_workspace_size_formula():
 
 def test_default_partition_rule():
     d = b.lib.pkv_decode_default_partition
-    assert d(64, 40, 2048) == 512
+    assert d(64, 40, 2048) == 1024
+    assert d(8, 8, 131072) == 1024
     assert d(1, 1, 4096) == 64          # tiny batches split finer
     p = d(4, 4, 512)
     assert 64 <= p <= 512 and p % 64 == 0
