@@ -53,6 +53,17 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(values, world: int, device: str = "cuda"):
+    """Element-wise max of per-rank values over the process group (timings
+    are reported as the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -151,7 +162,7 @@ def resolve_variant(cfg, kernel: str) -> str:
     return "mma" if cfg.dtype != "f32" and 4 <= cfg.group <= 16 else "simt"
 
 
-def recorded_traffic(workload: str, variant: str):
+def recorded_traffic(workload: str, variant: str, partition: int | None = None):
     """DRAM bytes per decode call from a committed ncu summary, if it was
     taken on the current kernel sources (else None)."""
     p = os.path.join(ROOT, "profiles", f"decode_{variant}_{workload}.md")
@@ -163,6 +174,8 @@ def recorded_traffic(workload: str, variant: str):
             k, v = line[2:].split(":", 1)
             rec[k.strip()] = v.strip().strip("`")
     if rec.get("kernel_sources_sha256_16") != kernel_source_digest(variant):
+        return None
+    if partition is not None and rec.get("partition_size") not in (None, str(partition)):
         return None
     try:
         return int(rec["dram_bytes_per_decode_call"])
@@ -384,10 +397,7 @@ def run_ours(args, cfg):
     assert torch.equal(h_out, out.cpu())
 
     # ---- max over ranks
-    vals = torch.tensor([ms, dec_ms, e2e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms, dec_ms, e2e_ms = vals.tolist()
+    ms, dec_ms, e2e_ms = max_over_ranks([ms, dec_ms, e2e_ms], world)
 
     if rank == 0:
         per_step_ms = ms / args.steps
@@ -421,7 +431,8 @@ def run_ours(args, cfg):
                          "frac": round(achieved / peak, 4), "peak_source": peak_src,
                          "decode_ms": round(dec_ms, 5), "bytes_per_launch": int(dec_bytes),
                          "variant": resolve_variant(cfg, args.kernel),
-                         "traffic": recorded_traffic(cfg.name, resolve_variant(cfg, args.kernel))},
+                         "traffic": recorded_traffic(cfg.name, resolve_variant(cfg, args.kernel),
+                                                     Pused)},
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -436,13 +447,160 @@ def run_ours(args, cfg):
     return 0
 
 
+def run_cow(args):
+    """Parallel sampling with copy-on-write prefix sharing: 32 prompts x 8
+    samples share 1024 + r tokens (r in [1, 15], so the last shared block is
+    partly filled).  Two timed phases, each replaying the same device work:
+    (i) the fork step -- every sample appends its first token, the allocator
+    hands out 7 block copies per prompt, and the step runs copy_blocks,
+    kv_cache_append and the decode; (ii) a steady step once every sample has
+    a private tail of U[1, 512] tokens -- append + decode, no copies."""
+    import torch
+
+    import paged_kv_cache_346_b200 as pkv
+    from workloads import COW_SAMPLING, draw_cow_recipe
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    c = COW_SAMPLING
+    rec = draw_cow_recipe(seed=args.seed)
+    P, S = rec.num_prompts, rec.samples
+    B, H, D, bs = P * S, c["num_kv_heads"], c["head_dim"], c["block_size"]
+    e = 2
+    N = sum(-(-int(L) // bs) for L in rec.shared_lens) + B * (3 + -(-c["tail_hi"] // bs))
+    alloc = pkv.BlockAllocator(N, bs)
+    for p in range(P):
+        assert alloc.add_seq(1_000_000 + p, int(rec.shared_lens[p])) == 0
+        for s_ in range(S):
+            assert alloc.fork(1_000_000 + p, p * S + s_) == 0
+        assert alloc.free_seq(1_000_000 + p) == 0
+    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    kc = torch.randn((N, H, bs, D), generator=g, device="cuda", dtype=torch.float32).half()
+    vc = torch.randn((N, H, bs, D), generator=g, device="cuda", dtype=torch.float32).half()
+    seqs = np.arange(B)
+    scale = 1.0 / math.sqrt(D)
+    stream = torch.cuda.current_stream()
+
+    def phase(pairs_np, slots_np, tables_np, lens_np):
+        q = torch.randn((B, H, D), generator=g, device="cuda", dtype=torch.float32).half()
+        knew = torch.randn((B, H, D), generator=g, device="cuda", dtype=torch.float32).half()
+        vnew = torch.randn((B, H, D), generator=g, device="cuda", dtype=torch.float32).half()
+        pairs = torch.from_numpy(pairs_np).cuda()
+        slots = torch.from_numpy(slots_np).cuda()
+        tables = torch.from_numpy(tables_np).cuda()
+        lens = torch.from_numpy(lens_np).cuda()
+        out = torch.empty_like(q)
+        L = int(lens_np.max())
+        ws = torch.empty(max(16, pkv.pkv_decode_workspace_size(B, H, H, D, L)),
+                         dtype=torch.uint8, device="cuda")
+        npairs = len(pairs_np)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(3)]
+
+        def step(timed=False):
+            if timed:
+                ev[0][0].record(stream)
+            if npairs:
+                pkv.pkv_copy_blocks(kc, vc, pairs, stream=stream)
+            if timed:
+                ev[0][1].record(stream)
+                ev[1][0].record(stream)
+            pkv.pkv_kv_cache_append(kc, vc, knew, vnew, slots, stream=stream)
+            if timed:
+                ev[1][1].record(stream)
+                ev[2][0].record(stream)
+            pkv.pkv_paged_attention_decode(out, q, kc, vc, tables, lens, scale, bs, L,
+                                           workspace=ws, stream=stream)
+            if timed:
+                ev[2][1].record(stream)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        parts = np.zeros(3)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(timed=True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / args.steps
+        # per-kernel times of the last step (events were re-recorded each step)
+        parts = [a.elapsed_time(b) for a, b in ev]
+        # bytes: logical = every sequence's K/V as read; unique = distinct
+        # physical (block, slot) entries the decode reads
+        kv_tok = 2 * H * D * e
+        logical = int(lens_np.astype(np.int64).sum()) * kv_tok
+        filled = {}
+        for i in range(B):
+            Li = int(lens_np[i])
+            for j in range(-(-Li // bs)):
+                blk = int(tables_np[i, j])
+                filled[blk] = max(filled.get(blk, 0), min(bs, Li - j * bs))
+        unique = sum(filled.values()) * kv_tok
+        qo = 2 * B * H * D * e
+        tab = int(sum(-(-int(x) // bs) for x in lens_np)) * 4 + 4 * B
+        copy = npairs * 4 * H * bs * D * e
+        append = B * (4 * H * D * e + 8)
+        return {
+            "ms_per_step": round(ms, 5),
+            "copy_pairs": npairs,
+            "kernel_ms_last_step": {"copy_blocks": round(parts[0], 5),
+                                    "kv_append": round(parts[1], 5),
+                                    "decode": round(parts[2], 5)},
+            "logical_bytes": logical + qo + tab + copy + append,
+            "unique_bytes": unique + qo + tab + copy + append,
+            "effective_GBps": round((logical + qo + tab + copy + append) / (ms * 1e-3) / 1e9, 1),
+            "unique_GBps": round((unique + qo + tab + copy + append) / (ms * 1e-3) / 1e9, 1),
+            "decode_unique_GBps": round((unique + qo + tab) / (parts[2] * 1e-3) / 1e9, 1),
+            "mean_context": round(float(lens_np.mean()), 1),
+        }
+
+    # (i) fork step
+    st, slots, pairs, done = alloc.append_slots(seqs)
+    assert st == 0 and done == B
+    tables, lens = alloc.build_block_tables(seqs, N)
+    maxb = int(max(-(-int(x) // bs) for x in lens))
+    fork = phase(pairs, slots, np.ascontiguousarray(tables[:, :maxb]), lens)
+    # (ii) grow private tails on the host, then one steady step
+    for i in range(B):
+        for _ in range(int(rec.tail_lens[i]) - 1):
+            r = alloc.append_slot(int(seqs[i]))
+            assert r[0] == 0 and r[2] < 0
+    st, slots, pairs, done = alloc.append_slots(seqs)
+    assert st == 0 and len(pairs) == 0
+    tables, lens = alloc.build_block_tables(seqs, N)
+    maxb = int(max(-(-int(x) // bs) for x in lens))
+    steady = phase(pairs, slots, np.ascontiguousarray(tables[:, :maxb]), lens)
+    stats = alloc.stats()
+    flags = pkv.pkv_device_status(clear=True)
+    if flags:
+        raise SystemExit(f"device status flags {flags:#x}")
+    if rank == 0:
+        peaks = measured_peaks() or {}
+        line = {
+            "metric": METRIC + " (copy-on-write sampling)", "value": steady["effective_GBps"],
+            "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic",
+            "config": {"workload": "cow_sampling", "prompts": P, "samples": S,
+                       "shared_tokens_mean": float(rec.shared_lens.mean()),
+                       "heads": H, "head_dim": D, "block_size": bs},
+            "fork_step": fork, "steady_step": steady,
+            "allocator": stats, "hbm_peak_GBps": peaks.get("hbm_gbs"),
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama2_13b_layer", choices=sorted(CONFIGS))
+    ap.add_argument("--workload", default="llama2_13b_layer",
+                    choices=sorted(CONFIGS) + ["cow_sampling"])
     ap.add_argument("--kernel", choices=["auto", "simt", "mma"], default="auto")
     ap.add_argument("--partition", type=int, default=None,
                     help="tokens per partition (default: the workload's, else automatic)")
@@ -454,6 +612,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    if args.workload == "cow_sampling":
+        return run_cow(args)
     cfg = CONFIGS[args.workload]
     if args.partition is None:
         args.partition = cfg.partition_size
