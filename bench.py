@@ -309,6 +309,9 @@ def run_ours(args, cfg):
                                  torch.from_numpy(slots_np % bs).cuda(), :].contiguous()
     out = torch.empty_like(q)
     mcl = inp.max_context_len
+    # schedule the longest sequences first (host-side order from host lengths)
+    order_np = pkv.pkv_decode_schedule_order(inp.context_lens) if args.order else None
+    order = dev(order_np) if order_np is not None else None
     P = args.partition
     ws_bytes = pkv.pkv_decode_workspace_size(B, cfg.num_q_heads, H, D, mcl, P)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
@@ -318,8 +321,8 @@ def run_ours(args, cfg):
 
     def decode():
         pkv.pkv_paged_attention_decode(out, q, kc, vc, bt, cl, cfg.scale, bs, mcl,
-                                       partition_size=P, workspace=ws, kernel=kern,
-                                       stream=stream)
+                                       partition_size=P, workspace=ws, seq_order=order,
+                                       kernel=kern, stream=stream)
 
     def step():
         pkv.pkv_kv_cache_append(kc, vc, knew, vnew, slots, stream=stream)
@@ -361,11 +364,14 @@ def run_ours(args, cfg):
     h_slots = torch.from_numpy(slots_np).pin_memory()
     h_bt = torch.from_numpy(inp.block_tables).pin_memory()
     h_cl = torch.from_numpy(inp.context_lens).pin_memory()
+    h_order = torch.from_numpy(order_np).pin_memory() if order_np is not None else None
+    d_order = torch.empty_like(order) if order is not None else None
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     d_knew, d_vnew = torch.empty_like(knew), torch.empty_like(vnew)
     d_q, d_slots, d_bt, d_cl = (torch.empty_like(q), torch.empty_like(slots),
                                 torch.empty_like(bt), torch.empty_like(cl))
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_knew, h_vnew, h_slots, h_bt, h_cl))
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_knew, h_vnew, h_slots, h_bt, h_cl)
+              + ((h_order,) if h_order is not None else ()))
     d2h = h_out.numel() * h_out.element_size()
 
     def e2e_step():
@@ -375,10 +381,12 @@ def run_ours(args, cfg):
         d_slots.copy_(h_slots, non_blocking=True)
         d_bt.copy_(h_bt, non_blocking=True)
         d_cl.copy_(h_cl, non_blocking=True)
+        if h_order is not None:
+            d_order.copy_(h_order, non_blocking=True)
         pkv.pkv_kv_cache_append(kc, vc, d_knew, d_vnew, d_slots, stream=stream)
         pkv.pkv_paged_attention_decode(out, d_q, kc, vc, d_bt, d_cl, cfg.scale, bs, mcl,
-                                       partition_size=P, workspace=ws, kernel=kern,
-                                       stream=stream)
+                                       partition_size=P, workspace=ws, seq_order=d_order,
+                                       kernel=kern, stream=stream)
         h_out.copy_(out, non_blocking=True)
 
     e2e_steps = max(3, min(args.steps, 200))
@@ -417,6 +425,7 @@ def run_ours(args, cfg):
                        "seq_len": round(float(lens.mean()), 1),
                        "num_q_heads": cfg.num_q_heads, "num_kv_heads": H, "head_dim": D,
                        "block_size": bs, "partition_size": Pused, "kernel": args.kernel,
+                       "schedule": "longest-first" if args.order else "batch order",
                        "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (%.2f GB of K/V per step)" % (
                            dec_bytes / 1e9)},
@@ -605,6 +614,8 @@ def main():
     ap.add_argument("--partition", type=int, default=None,
                     help="tokens per partition (default: the workload's, else automatic)")
     ap.add_argument("--seed", type=int, default=2)
+    ap.add_argument("--no-order", dest="order", action="store_false",
+                    help="schedule sequences in batch order instead of longest first")
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of oracle work for the cpu_baseline field")
     ap.add_argument("--ref-budget", type=float, default=90.0,

@@ -85,6 +85,7 @@ typedef enum { PKV_KERNEL_AUTO = 0, PKV_KERNEL_SIMT = 1, PKV_KERNEL_MMA = 2 } pk
 #define PKV_DEV_BAD_LEN 2u      /* a context length < 0 or past the caller's bounds */
 #define PKV_DEV_BAD_SLOT 4u     /* a slot at or past num_blocks * block_size */
 #define PKV_DEV_TIMEOUT 8u      /* a bounded wait inside a kernel gave up */
+#define PKV_DEV_BAD_ORDER 16u   /* a seq_order entry outside [0, num_seqs) */
 
 /* Name of a status code. */
 PKV_API const char* pkv_status_string(int status);
@@ -96,7 +97,10 @@ PKV_API int pkv_version(void);
 PKV_API int pkv_decode_has_kernel(pkv_kernel kernel);
 
 /*
- * Partition size the decode uses when `partition_size` is 0, for this shape.
+ * Partition size the decode uses when `partition_size` is 0, for this shape:
+ * 2048 tokens, halved while the grid would hold fewer than ~6 CTAs per SM.
+ * Tuned with a longest-first seq_order; without one, 1024 can be faster when
+ * lengths are very uneven.
  */
 PKV_API int pkv_decode_default_partition(int num_seqs, int num_kv_heads, int max_context_len);
 
@@ -129,6 +133,13 @@ PKV_API size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_
  *       layouts above; k_cache and v_cache 16-byte aligned.
  *   num_q_heads % num_kv_heads == 0; head_dim in {64, 128, 256};
  *   block_size in {16, 32, 64}; dtype f32, f16 or bf16.
+ *   seq_order: NULL, or a device int32 permutation of [0, num_seqs): the
+ *       order in which sequences are scheduled onto the GPU.  It changes no
+ *       result (every row is computed the same way), only the timing: with
+ *       the longest sequences first (pkv_decode_schedule_order) the grid
+ *       ends without a tail of long partitions.  An entry outside
+ *       [0, num_seqs) is skipped and flagged (PKV_DEV_BAD_ORDER); a repeated
+ *       entry leaves some row unwritten.
  *   max_context_len: host-side upper bound of context_lens, and
  *       <= max_blocks_per_seq * block_size.
  *   partition_size: 0 for the default, else a multiple of 64 in [64, 8192].
@@ -140,7 +151,8 @@ PKV_API size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_
  */
 PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
                                const void* v_cache, const int32_t* block_tables,
-                               const int32_t* context_lens, int num_seqs,
+                               const int32_t* context_lens, const int32_t* seq_order,
+                               int num_seqs,
                                int num_q_heads, int num_kv_heads, int head_dim,
                                int block_size, int max_blocks_per_seq, int num_blocks,
                                int max_context_len, float scale, pkv_dtype dtype,
@@ -179,10 +191,18 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
  */
 PKV_API int pkv_paged_attention_decode_static_ws(
     void* out, const void* q, const void* k_cache, const void* v_cache,
-    const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_q_heads,
-    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
-    int max_context_len, float scale, pkv_dtype dtype, int partition_size, pkv_kernel kernel,
-    pkv_stream_t stream);
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* seq_order,
+    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int num_blocks, int max_context_len, float scale, pkv_dtype dtype,
+    int partition_size, pkv_kernel kernel, pkv_stream_t stream);
+
+/*
+ * Host helper: order_out[0..n) = the sequence indices sorted by decreasing
+ * context length (ties by index), for the seq_order argument of the decode.
+ * context_lens is a host array.  Returns PKV_OK or PKV_EINVAL.
+ */
+PKV_API int pkv_decode_schedule_order(const int32_t* context_lens, int num_seqs,
+                                      int32_t* order_out);
 
 /*
  * KV append: the key and value of each new token go into the slot the block

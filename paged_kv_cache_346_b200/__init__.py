@@ -17,8 +17,8 @@ import ctypes
 import torch
 
 from . import _binding as _b
-from ._binding import (PKV_BF16, PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD_SLOT,
-                       PKV_DEV_TIMEOUT, PKV_F16, PKV_F32, PKV_KERNEL_AUTO, PKV_KERNEL_MMA,
+from ._binding import (PKV_BF16, PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD_ORDER,
+                       PKV_DEV_BAD_SLOT, PKV_DEV_TIMEOUT, PKV_F16, PKV_F32, PKV_KERNEL_AUTO, PKV_KERNEL_MMA,
                        PKV_KERNEL_SIMT, PagedKVError, check, lib)
 
 __all__ = [
@@ -27,7 +27,8 @@ __all__ = [
     "pkv_kv_cache_append", "pkv_copy_blocks", "pkv_device_status", "BlockAllocator",
     "PagedKVError", "lib", "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_KERNEL_AUTO",
     "PKV_KERNEL_SIMT", "PKV_KERNEL_MMA", "PKV_DEV_BAD_BLOCK", "PKV_DEV_BAD_LEN",
-    "PKV_DEV_BAD_SLOT", "PKV_DEV_TIMEOUT", "torch_dtype_code",
+    "PKV_DEV_BAD_SLOT", "PKV_DEV_TIMEOUT", "PKV_DEV_BAD_ORDER", "torch_dtype_code",
+    "pkv_decode_schedule_order",
 ]
 
 _DTYPE = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16}
@@ -78,15 +79,21 @@ def pkv_paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torc
                                context_lens: torch.Tensor, scale: float, block_size: int,
                                max_context_len: int, *, partition_size: int = 0,
                                workspace: torch.Tensor | None = None,
+                               seq_order: torch.Tensor | None = None,
                                kernel: int = PKV_KERNEL_AUTO, stream=None) -> torch.Tensor:
     """out [B, Hq, D] <- paged decode attention (see pkv_paged_attention_decode
     in pagedkv.h).  k_cache/v_cache [N, Hkv, block_size, D]; block_tables
     int32 [B, max_blocks]; context_lens int32 [B]; max_context_len is a host
     bound of context_lens.  workspace: a CUDA tensor of at least
-    pkv_decode_workspace_size(...) bytes when sequences span partitions."""
+    pkv_decode_workspace_size(...) bytes when sequences span partitions.
+    seq_order: optional int32 [B] schedule order (pkv_decode_schedule_order)."""
     for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
                  (block_tables, "block_tables"), (context_lens, "context_lens")):
         _dev(t, n)
+    if seq_order is not None:
+        _dev(seq_order, "seq_order")
+        if seq_order.dtype != torch.int32 or seq_order.numel() != q.shape[0]:
+            raise PagedKVError(_b.PKV_EINVAL, "seq_order must be int32 [num_seqs]")
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise PagedKVError(_b.PKV_EINVAL, "block_tables / context_lens must be int32")
     if not (q.dtype == out.dtype == k_cache.dtype == v_cache.dtype):
@@ -103,7 +110,7 @@ def pkv_paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torc
         ws_bytes = workspace.numel() * workspace.element_size()
     check(lib.pkv_paged_attention_decode(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
-        _ptr(context_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], N,
+        _ptr(context_lens), _ptr(seq_order), B, Hq, Hkv, D, bs, block_tables.shape[1], N,
         int(max_context_len), float(scale), torch_dtype_code(q.dtype), int(partition_size),
         _ptr(workspace), ws_bytes, int(kernel), _stream(stream)), "pkv_paged_attention_decode")
     return out
@@ -114,6 +121,7 @@ def pkv_paged_attention_decode_static_ws(out: torch.Tensor, q: torch.Tensor,
                                          block_tables: torch.Tensor, context_lens: torch.Tensor,
                                          scale: float, block_size: int, max_context_len: int, *,
                                          partition_size: int = 0,
+                                         seq_order: torch.Tensor | None = None,
                                          kernel: int = PKV_KERNEL_AUTO,
                                          stream=None) -> torch.Tensor:
     """pkv_paged_attention_decode without a caller workspace, for callers that
@@ -128,12 +136,23 @@ def pkv_paged_attention_decode_static_ws(out: torch.Tensor, q: torch.Tensor,
     N, Hkv, bs, _ = k_cache.shape
     check(lib.pkv_paged_attention_decode_static_ws(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
-        _ptr(context_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], N,
+        _ptr(context_lens), _ptr(seq_order), B, Hq, Hkv, D, bs, block_tables.shape[1], N,
         int(max_context_len), float(scale), torch_dtype_code(q.dtype), int(partition_size),
         int(kernel), _stream(stream)),
         f"pkv_paged_attention_decode_static_ws (scratch limit "
         f"{_b.PKV_STATIC_WORKSPACE_BYTES} bytes)")
     return out
+
+
+def pkv_decode_schedule_order(context_lens):
+    """Host int32 array [B]: sequence indices by decreasing length (ties by
+    index), for the decode's seq_order argument."""
+    import numpy as np
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    order = np.empty(lens.size, dtype=np.int32)
+    check(lib.pkv_decode_schedule_order(lens.ctypes.data, lens.size, order.ctypes.data),
+          "pkv_decode_schedule_order")
+    return order
 
 
 def pkv_kv_cache_append(k_cache: torch.Tensor, v_cache: torch.Tensor, k: torch.Tensor,

@@ -17,7 +17,8 @@ PKV_OK, PKV_EINVAL, PKV_ENOMEM, PKV_ENOSEQ, PKV_EEXIST, PKV_EBOUNDS, PKV_ECUDA, 
     PKV_EUNSUPPORTED = 0, -1, -2, -3, -4, -5, -6, -7
 PKV_F32, PKV_F16, PKV_BF16 = 0, 1, 2
 PKV_KERNEL_AUTO, PKV_KERNEL_SIMT, PKV_KERNEL_MMA = 0, 1, 2
-PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD_SLOT, PKV_DEV_TIMEOUT = 1, 2, 4, 8
+PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD_SLOT, PKV_DEV_TIMEOUT, PKV_DEV_BAD_ORDER = \
+    1, 2, 4, 8, 16
 PKV_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024
 
 if not os.path.exists(LIB_PATH):
@@ -35,12 +36,13 @@ SIGNATURES = {
     "pkv_decode_has_kernel": (_i32, [_i32]),
     "pkv_decode_default_partition": (_i32, [_i32, _i32, _i32]),
     "pkv_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
-    "pkv_paged_attention_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
-                                          _i32, _i32, _i32, _i32, _f32, _i32, _i32, _vp, _sz,
-                                          _i32, _vp]),
-    "pkv_paged_attention_decode_static_ws": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
-                                                    _i32, _i32, _i32, _i32, _i32, _i32, _f32,
-                                                    _i32, _i32, _i32, _vp]),
+    "pkv_paged_attention_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+                                          _i32, _i32, _i32, _i32, _i32, _f32, _i32, _i32, _vp,
+                                          _sz, _i32, _vp]),
+    "pkv_paged_attention_decode_static_ws": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
+                                                    _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                                    _f32, _i32, _i32, _i32, _vp]),
+    "pkv_decode_schedule_order": (_i32, [_vp, _i32, _vp]),
     "pkv_kv_cache_append": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                    _vp]),
     "pkv_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp]),

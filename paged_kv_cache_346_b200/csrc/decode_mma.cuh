@@ -15,8 +15,10 @@
 // viewed as [N * Hkv * BS rows, D columns], boxes of 64 columns x BS rows,
 // 128-byte swizzle: row r of a box keeps its 16-byte chunk c at position
 // c ^ (r % 8), so the ldmatrix reads of 8 rows at one column hit 8 different
-// bank groups.  Everything else (table hoist, mbarrier ring, per-warp online
-// softmax, warp merge, split-K workspace) mirrors the CUDA-core kernel.
+// bank groups.  Each warp copies its fragments of a stage into registers and
+// the stage is refilled before the math runs.  Everything else (table hoist,
+// mbarrier ring, per-warp online softmax, warp merge, split-K workspace)
+// mirrors the CUDA-core kernel.
 #pragma once
 
 #include <cuda.h>
@@ -110,7 +112,7 @@ struct MmaCfg {
 // NH = 8 or 16 query heads per CTA (the M rows of the QK product / the N
 // columns of the PV product); heads past the group are zero rows.
 template <typename T, int D, int BS, int NH, int NW, int STAGES_>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
     using C = MmaCfg<D, BS, NW, STAGES_>;
@@ -120,20 +122,25 @@ __global__ void __launch_bounds__(NW * 32)
     constexpr int STAGES = C::STAGES;
     constexpr int KSTEPS = D / 16;   // k-steps of the QK product, m-tiles of PV
     constexpr int RB = NH / 8;       // 8-head row blocks
+    // Hold the warp's K/V fragments in registers and release the stage before
+    // the math, when that keeps three CTAs per SM within the register file.
+    constexpr bool EARLY = D <= 128 && NH == 8;
 
     extern __shared__ __align__(1024) unsigned char smem_mma[];
     __shared__ int s_abort;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
-    const int b = blockIdx.z;
     const int kvh = blockIdx.y / a.head_chunks;
     const int hc = blockIdx.y - kvh * a.head_chunks;
     const int part = blockIdx.x;
     const int h0 = kvh * a.group + hc * NH;
     const int nh = min(NH, a.group - hc * NH);
     const bool reporter = (tid == 0 && part == 0 && blockIdx.y == 0);
+    const int b = scheduled_seq(a, blockIdx.z, reporter);
+    if (b < 0) return;
 
+    const TablePrefetch pf = table_prefetch(a, b, part, a.partition_size / BS, tid);
     const int L = seq_len(a, b, reporter);
     const int np = num_partitions(a, L, reporter);
     T* out = reinterpret_cast<T*>(a.out);
@@ -160,17 +167,7 @@ __global__ void __launch_bounds__(NW * 32)
         s_kv = smem_mma + 1024 + round_up(P / BS * 4, 128) + (aligned - base);
     }
 
-    {
-        const int32_t* trow = a.block_tables + (int64_t)b * a.max_blocks_per_seq + t0 / BS;
-        for (int i = tid; i < nblk; i += NW * 32) {
-            int32_t p = trow[i];
-            if ((unsigned)p >= (unsigned)a.num_blocks) {
-                flag(a.status, PKV_DEV_BAD_BLOCK);
-                p = 0;
-            }
-            s_tab[i] = p;
-        }
-    }
+    table_hoist(a, b, t0 / BS, nblk, pf, s_tab, tid, NW * 32);
     if (tid == 0) {
         s_abort = 0;
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
@@ -242,107 +239,128 @@ __global__ void __launch_bounds__(NW * 32)
     for (int it = 0; it < ntiles; ++it) {
         const int stage = it % STAGES;
         const bool ok = mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status);
-        if (!ok) {
-            s_abort = 1;
-        } else {
-            const int wvalid = ntok - (it * TILE + warp * 16);
-            if (wvalid > 0) {
-                const int tt0 = warp * 16;           // first token of the warp in the stage
-                const int jw = tt0 / BS;             // its block within the stage
-                const int rr = tt0 % BS + lrow;      // this lane's row within that block
-                const uint32_t kbase = smem_u32(s_kv + stage * 2 * STAGE_BYTES) +
-                                       (uint32_t)(jw * NX * BOX_BYTES + rr * 128);
-                const uint32_t vbase = kbase + STAGE_BYTES;
-                const int swz = rr & 7;
-
-                // S^T = Q K^T: two n-tiles of 8 tokens
-                float s[2][4];
+        if (!ok) s_abort = 1;
+        const int wvalid = ntok - (it * TILE + warp * 16);
+        const bool work = ok && wvalid > 0;
+        const int tt0 = warp * 16;           // first token of the warp in the stage
+        const int jw = tt0 / BS;             // its block within the stage
+        const int rr = tt0 % BS + lrow;      // this lane's row within that block
+        const uint32_t kbase = smem_u32(s_kv + stage * 2 * STAGE_BYTES) +
+                               (uint32_t)(jw * NX * BOX_BYTES + rr * 128);
+        const uint32_t vbase = kbase + STAGE_BYTES;
+        const int swz = rr & 7;
+        auto kaddr = [&](int ks) {
+            const int chunk = ks * 2 + lchunk;  // 16-byte chunk of the row
+            return kbase + (chunk >> 3) * BOX_BYTES + (((chunk & 7) ^ swz) << 4);
+        };
+        // EARLY: copy the warp's K and V fragments into registers, so the
+        // stage goes back to the producer before the math runs
+        uint32_t kf[EARLY ? KSTEPS : 1][4], vf[EARLY ? KSTEPS : 1][4];
+        if (EARLY && work) {
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
-#pragma unroll
-                for (int ks = 0; ks < KSTEPS; ++ks) {
-                    const int chunk = ks * 2 + lchunk;           // 16-byte chunk of the row
-                    const int x = chunk >> 3, c = chunk & 7;
-                    uint32_t kb[4];
-                    ldsm_x4(kbase + x * BOX_BYTES + ((c ^ swz) << 4), kb);
-                    M::run(s[0], qa[ks], kb[0], kb[1]);
-                    M::run(s[1], qa[ks], kb[2], kb[3]);
-                }
-                // logits in base 2, masked past the sequence end
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int tok = nt * 8 + 2 * t4 + (i & 1);
-                        s[nt][i] = tok < wvalid ? s[nt][i] * a.scale_log2 : -INFINITY;
-                    }
-                uint32_t pb[RB][2];
-                float alpha_c[RB][2];
-#pragma unroll
-                for (int rb = 0; rb < RB; ++rb) {
-                    const int i0 = 2 * rb;  // s[nt][i0], s[nt][i0 + 1]: head g + 8 rb
-                    float mx = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                    const float mnew = fmaxf(m[rb], mx);
-                    const float alpha = exp2f(m[rb] - mnew);
-                    float p[2][2], pr[2][2];
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        p[nt][0] = exp2f(s[nt][i0] - mnew);
-                        p[nt][1] = exp2f(s[nt][i0 + 1] - mnew);
-                        pb[rb][nt] = M::pack(p[nt][0], p[nt][1], pr[nt][0], pr[nt][1]);
-                    }
-                    float ps = (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-                    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-                    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-                    l[rb] = l[rb] * alpha + ps;
-                    m[rb] = mnew;
-                    // O^T columns of this thread are heads 2 t4, 2 t4 + 1 (+ 8 rb)
-                    alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
-                    alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
-                }
-                // O^T += V^T P^T
-                const bool partial = wvalid < 16;
-#pragma unroll
-                for (int mt = 0; mt < KSTEPS; ++mt) {
-                    const int chunk = mt * 2 + lchunk;
-                    const int x = chunk >> 3, c = chunk & 7;
-                    uint32_t va[4];
-                    ldsm_x4_trans(vbase + x * BOX_BYTES + ((c ^ swz) << 4), va);
-                    if (partial) {
-                        // zero values of tokens past the end (0 * NaN would poison)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int tk = (i >> 1) * 8 + 2 * t4;
-                            const uint32_t keep = (tk < wvalid ? 0x0000ffffu : 0u) |
-                                                  (tk + 1 < wvalid ? 0xffff0000u : 0u);
-                            va[i] &= keep;
-                        }
-                    }
-#pragma unroll
-                    for (int rb = 0; rb < RB; ++rb) {
-                        o[mt][rb][0] *= alpha_c[rb][0];
-                        o[mt][rb][1] *= alpha_c[rb][1];
-                        o[mt][rb][2] *= alpha_c[rb][0];
-                        o[mt][rb][3] *= alpha_c[rb][1];
-                        M::run(o[mt][rb], va, pb[rb][0], pb[rb][1]);
-                    }
-                }
+            for (int ks = 0; ks < (EARLY ? KSTEPS : 1); ++ks) {
+                ldsm_x4(kaddr(ks), kf[ks]);
+                ldsm_x4_trans(kaddr(ks) + STAGE_BYTES, vf[ks]);
             }
         }
-        __syncthreads();
+        auto math = [&]() {
+            // S^T = Q K^T: two n-tiles of 8 tokens
+            float s[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < KSTEPS; ++ks) {
+                uint32_t kb[4];
+                if constexpr (EARLY) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) kb[i] = kf[ks < (EARLY ? KSTEPS : 1) ? ks : 0][i];
+                } else {
+                    ldsm_x4(kaddr(ks), kb);
+                }
+                M::run(s[0], qa[ks], kb[0], kb[1]);
+                M::run(s[1], qa[ks], kb[2], kb[3]);
+            }
+            // logits in base 2, masked past the sequence end
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int tok = nt * 8 + 2 * t4 + (i & 1);
+                    s[nt][i] = tok < wvalid ? s[nt][i] * a.scale_log2 : -INFINITY;
+                }
+            uint32_t pb[RB][2];
+            float alpha_c[RB][2];
+#pragma unroll
+            for (int rb = 0; rb < RB; ++rb) {
+                const int i0 = 2 * rb;  // s[nt][i0], s[nt][i0 + 1]: head g + 8 rb
+                float mx = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float mnew = fmaxf(m[rb], mx);
+                const float alpha = exp2f(m[rb] - mnew);
+                float p[2][2], pr[2][2];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    p[nt][0] = exp2f(s[nt][i0] - mnew);
+                    p[nt][1] = exp2f(s[nt][i0 + 1] - mnew);
+                    pb[rb][nt] = M::pack(p[nt][0], p[nt][1], pr[nt][0], pr[nt][1]);
+                }
+                float ps = (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+                l[rb] = l[rb] * alpha + ps;
+                m[rb] = mnew;
+                // O^T columns of this thread are heads 2 t4, 2 t4 + 1 (+ 8 rb)
+                alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
+                alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
+            }
+            // O^T += V^T P^T
+            const bool partial = wvalid < 16;
+#pragma unroll
+            for (int mt = 0; mt < KSTEPS; ++mt) {
+                uint32_t va[4];
+                if constexpr (EARLY) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) va[i] = vf[mt < (EARLY ? KSTEPS : 1) ? mt : 0][i];
+                } else {
+                    ldsm_x4_trans(kaddr(mt) + STAGE_BYTES, va);
+                }
+                if (partial) {
+                    // zero values of tokens past the end (0 * NaN would poison)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int tk = (i >> 1) * 8 + 2 * t4;
+                        const uint32_t keep = (tk < wvalid ? 0x0000ffffu : 0u) |
+                                              (tk + 1 < wvalid ? 0xffff0000u : 0u);
+                        va[i] &= keep;
+                    }
+                }
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) {
+                    o[mt][rb][0] *= alpha_c[rb][0];
+                    o[mt][rb][1] *= alpha_c[rb][1];
+                    o[mt][rb][2] *= alpha_c[rb][0];
+                    o[mt][rb][3] *= alpha_c[rb][1];
+                    M::run(o[mt][rb], va, pb[rb][0], pb[rb][1]);
+                }
+            }
+        };
+        if (!EARLY && work) math();
+        __syncthreads();  // the stage is free again
         if (s_abort) break;
         if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage);
+        if (EARLY && work) math();
     }
     if (s_abort) return;
     pdl_launch_dependents();
 
-    // merge the warps: red[w][head][dim], red_m / red_l [w][head]
+    // merge the warps (padded rows: lanes of one store hit distinct banks)
+    using A = MergeArea<D, NH, NW>;
+    static_assert(A::BYTES <= STAGES * 2 * STAGE_BYTES, "merge area");
     float* red = reinterpret_cast<float*>(s_kv);
-    float* red_m = red + NW * NH * D;
+    float* red_m = red + NW * NH * A::RP;
     float* red_l = red_m + NW * NH;
 #pragma unroll
     for (int mt = 0; mt < KSTEPS; ++mt)
@@ -352,7 +370,7 @@ __global__ void __launch_bounds__(NW * 32)
             for (int i = 0; i < 4; ++i) {
                 const int head = 8 * rb + 2 * t4 + (i & 1);
                 const int dim = mt * 16 + g + 8 * (i >> 1);
-                red[(warp * NH + head) * D + dim] = o[mt][rb][i];
+                red[(warp * NH + head) * A::RP + dim] = o[mt][rb][i];
             }
     if (t4 == 0) {
 #pragma unroll
@@ -362,30 +380,7 @@ __global__ void __launch_bounds__(NW * 32)
         }
     }
     __syncthreads();
-    for (int i = tid; i < nh * D; i += NW * 32) {
-        const int hh = i / D, d = i - hh * D;
-        float Mx = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) Mx = fmaxf(Mx, red_m[w * NH + hh]);
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-            const float f = exp2f(red_m[w * NH + hh] - Mx);
-            num = fmaf(f, red[(w * NH + hh) * D + d], num);
-            den = fmaf(f, red_l[w * NH + hh], den);
-        }
-        const int64_t row = (int64_t)b * a.num_q_heads + h0 + hh;
-        if (np == 1) {
-            out[row * D + d] = Elem<T>::from_f32(num / den);
-        } else {
-            const int64_t pr = row * a.max_partitions + part;
-            a.ws_o[pr * D + d] = num / den;
-            if (d == 0) {
-                a.ws_ml[pr * 2] = Mx;
-                a.ws_ml[pr * 2 + 1] = den;
-            }
-        }
-    }
+    merge_warps_and_store<T, D, NH, NW>(a, red, b, h0, nh, part, np, tid, NW * 32);
 }
 
 // Host side: tensor maps over the K and V pools, launch, optional reduce.

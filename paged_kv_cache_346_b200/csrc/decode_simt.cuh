@@ -12,8 +12,9 @@
 //   2. One thread issues 1-D bulk copies (TMA, cp.async.bulk) of whole
 //      (block, KV head) pages -- BS x D contiguous elements each for K and for
 //      V -- into a ring of STAGES shared-memory stages of TILE = 16 * NW tokens,
-//      completing on an mbarrier per stage; the copy of stage i + STAGES is
-//      issued as soon as every warp has finished with stage i.
+//      completing on an mbarrier per stage.  Each warp first copies its part
+//      of a stage into registers; the stage is refilled (copy of stage
+//      i + STAGES) as soon as every warp has done so, before the math runs.
 //   3. Warp w takes tokens [16w, 16w + 16) of each stage.  QK: 8 lanes per
 //      token, each with D/8 dims of q (float32, pre-scaled by scale*log2 e) in
 //      registers; 3 xor-shuffles finish each dot product.  Tokens past the
@@ -79,10 +80,29 @@ struct SimtWarp {
     using E = Elem<T>;
     static constexpr int ROW = C::ROW, EPC = C::EPC, CPL = C::CPL, LPV = C::LPV;
     static constexpr int TPV = C::TPV, CPV = C::CPV;
+    static constexpr int NTV = 16 / TPV;  // tokens per lane in P.V
+    // Copy the warp's share of a stage into registers and release the stage
+    // before the math (EARLY), when that fits the register budget of three
+    // CTAs per SM; otherwise read from the stage and release it afterwards.
+    static constexpr bool EARLY = ROW <= 256 && (HG == 1 || ROW <= 128);
+    static constexpr int KR = EARLY ? CPL : 1, NV = EARLY ? NTV : 1, VC = EARLY ? CPV : 1;
 
     float qf[HG][CPL][EPC];
     float m[HG], l[HG], acc[HG][CPV][EPC];
+    uint4 kr[4][KR];      // this lane's K chunks of the warp's 16 tokens (EARLY)
+    uint4 vr[NV][VC];     // and its V chunks
+    const unsigned char* Kp;  // the stage rows otherwise
+    const unsigned char* Vp;
     int lane, grp, sub, lv, tv;
+
+    __device__ __forceinline__ uint4 kchunk(int r, int i) const {
+        if constexpr (EARLY) return kr[r][i];
+        else return *reinterpret_cast<const uint4*>(Kp + (r * 4 + grp) * ROW + (sub + 8 * i) * 16);
+    }
+    __device__ __forceinline__ uint4 vchunk(int j, int c) const {
+        if constexpr (EARLY) return vr[j][c];
+        else return *reinterpret_cast<const uint4*>(Vp + (tv + j * TPV) * ROW + (lv + c * LPV) * 16);
+    }
 
     __device__ __forceinline__ void init(const T* qb, int nh, float scale_log2, int lane_) {
         lane = lane_;
@@ -113,10 +133,28 @@ struct SimtWarp {
         }
     }
 
-    // 16 tokens at Kw / Vw (rows of ROW bytes), the first `wvalid` of them
-    // inside the sequence.  s_p: this warp's [HG][16] weight scratch.
-    __device__ __forceinline__ void tile(const unsigned char* Kw, const unsigned char* Vw,
-                                         int wvalid, float (*s_p)[16]) {
+    // Copy this lane's share of the warp's 16 tokens (rows of ROW bytes at Kw /
+    // Vw) into registers, so the stage can be refilled before the math runs.
+    __device__ __forceinline__ void fetch(const unsigned char* Kw, const unsigned char* Vw) {
+        Kp = Kw;
+        Vp = Vw;
+        if constexpr (EARLY) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int i = 0; i < CPL; ++i)
+                    kr[r][i] = *reinterpret_cast<const uint4*>(Kw + (r * 4 + grp) * ROW + (sub + 8 * i) * 16);
+#pragma unroll
+            for (int j = 0; j < NTV; ++j)
+#pragma unroll
+                for (int c = 0; c < CPV; ++c)
+                    vr[j][c] = *reinterpret_cast<const uint4*>(Vw + (tv + j * TPV) * ROW + (lv + c * LPV) * 16);
+        }
+    }
+
+    // The fetched 16 tokens, the first `wvalid` of them inside the sequence.
+    // s_p: this warp's [HG][16] weight scratch.
+    __device__ __forceinline__ void compute(int wvalid, float (*s_p)[16]) {
         float s[HG][4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -126,9 +164,8 @@ struct SimtWarp {
             for (int hh = 0; hh < HG; ++hh) d[hh] = 0.f;
 #pragma unroll
             for (int i = 0; i < CPL; ++i) {
-                const uint4 kv = *reinterpret_cast<const uint4*>(Kw + tok * ROW + (sub + 8 * i) * 16);
                 float kf[EPC];
-                E::to_f32(kv, kf);
+                E::to_f32(kchunk(r, i), kf);
 #pragma unroll
                 for (int hh = 0; hh < HG; ++hh)
 #pragma unroll
@@ -169,14 +206,14 @@ struct SimtWarp {
             }
         }
         __syncwarp();
-#pragma unroll 4
-        for (int t = tv; t < 16; t += TPV) {
-            if (t < wvalid) {  // values past the end are never read (they may be NaN)
+#pragma unroll
+        for (int j = 0; j < NTV; ++j) {
+            const int t = tv + j * TPV;
+            if (t < wvalid) {  // values past the end are never used (they may be NaN)
 #pragma unroll
                 for (int c = 0; c < CPV; ++c) {
-                    const uint4 vv = *reinterpret_cast<const uint4*>(Vw + t * ROW + (lv + c * LPV) * 16);
                     float vf[EPC];
-                    E::to_f32(vv, vf);
+                    E::to_f32(vchunk(j, c), vf);
 #pragma unroll
                     for (int hh = 0; hh < HG; ++hh) {
                         const float p = s_p[hh][t];
@@ -189,8 +226,12 @@ struct SimtWarp {
         __syncwarp();
     }
 
-    // Fold the token lanes together and park (m, l, acc) in red* for the merge.
-    __device__ __forceinline__ void park(int warp, float* red, float* red_m, float* red_l) {
+    // Fold the token lanes together and park (m, l, acc) in the merge area.
+    template <int NW>
+    __device__ __forceinline__ void park(int warp, float* red) {
+        using A = MergeArea<D, HG, NW>;
+        float* red_m = red + NW * HG * A::RP;
+        float* red_l = red_m + NW * HG;
 #pragma unroll
         for (int msk = LPV; msk < 32; msk <<= 1)
 #pragma unroll
@@ -206,8 +247,11 @@ struct SimtWarp {
 #pragma unroll
                 for (int c = 0; c < CPV; ++c)
 #pragma unroll
-                    for (int e = 0; e < EPC; ++e)
-                        red[(warp * HG + hh) * D + (lv + c * LPV) * EPC + e] = acc[hh][c][e];
+                    for (int e = 0; e < EPC; e += 4)
+                        *reinterpret_cast<float4*>(red + (warp * HG + hh) * A::RP +
+                                                   (lv + c * LPV) * EPC + e) =
+                            make_float4(acc[hh][c][e], acc[hh][c][e + 1], acc[hh][c][e + 2],
+                                        acc[hh][c][e + 3]);
         }
         if (lane == 0) {
 #pragma unroll
@@ -219,42 +263,9 @@ struct SimtWarp {
     }
 };
 
-// Merge NW parked warp states (red*) of nh heads and write the output row (one
-// partition) or the partition's (m, l, o) to the workspace.
-template <typename T, int D, int NH, int NW>
-__device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, const float* red,
-                                                      const float* red_m, const float* red_l,
-                                                      int b, int h0, int nh, int part, int np,
-                                                      int tid, int nthreads) {
-    T* out = reinterpret_cast<T*>(a.out);
-    for (int i = tid; i < nh * D; i += nthreads) {
-        const int hh = i / D, d = i - hh * D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * NH + hh]);
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-            const float f = exp2f(red_m[w * NH + hh] - M);  // 0 for a warp with no tokens
-            num = fmaf(f, red[(w * NH + hh) * D + d], num);
-            den = fmaf(f, red_l[w * NH + hh], den);
-        }
-        const int64_t row = (int64_t)b * a.num_q_heads + h0 + hh;
-        if (np == 1) {
-            out[row * D + d] = Elem<T>::from_f32(num / den);
-        } else {
-            const int64_t pr = row * a.max_partitions + part;
-            a.ws_o[pr * D + d] = num / den;
-            if (d == 0) {
-                a.ws_ml[pr * 2] = M;
-                a.ws_ml[pr * 2 + 1] = den;
-            }
-        }
-    }
-}
-
 template <typename T, int D, int BS, int HG, int NW, int STAGES_, bool WS>
-__global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREADS)
+__global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREADS,
+                                  SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::ROW <= 256 ? 3 : 1)
     decode_simt_kernel(const DecodeArgs a) {
     using C = SimtCfg<T, D, BS, HG, NW, STAGES_, WS>;
     using E = Elem<T>;
@@ -267,14 +278,16 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREAD
     __shared__ volatile int s_abort;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = blockIdx.z;
     const int kvh = blockIdx.y / a.head_chunks;
     const int hc = blockIdx.y - kvh * a.head_chunks;
     const int part = blockIdx.x;
     const int h0 = kvh * a.group + hc * HG;
     const int nh = min(HG, a.group - hc * HG);
     const bool reporter = (tid == 0 && part == 0 && blockIdx.y == 0);
+    const int b = scheduled_seq(a, blockIdx.z, reporter);
+    if (b < 0) return;
 
+    const TablePrefetch pf = table_prefetch(a, b, part, a.partition_size / BS, tid);
     const int L = seq_len(a, b, reporter);
     const int np = num_partitions(a, L, reporter);
     if (L == 0) {  // empty sequence: a zero row
@@ -299,17 +312,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREAD
     unsigned char* s_kv = smem_simt + 128 + round_up(P / BS * 4, 128);
 
     // 1. table slice -> shared memory
-    {
-        const int32_t* trow = a.block_tables + (int64_t)b * a.max_blocks_per_seq + t0 / BS;
-        for (int i = tid; i < nblk; i += THREADS) {
-            int32_t p = trow[i];
-            if ((unsigned)p >= (unsigned)a.num_blocks) {
-                flag(a.status, PKV_DEV_BAD_BLOCK);
-                p = 0;  // stay inside the pool; the result is flagged as invalid
-            }
-            s_tab[i] = p;
-        }
-    }
+    table_hoist(a, b, t0 / BS, nblk, pf, s_tab, tid, THREADS);
     if (tid == 0) {
         s_abort = 0;
 #pragma unroll
@@ -336,9 +339,8 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREAD
         }
     };
 
-    float* red = reinterpret_cast<float*>(s_kv);  // [NW][HG][D], after the last stage
-    float* red_m = red + NW * HG * D;              // [NW][HG]
-    float* red_l = red_m + NW * HG;
+    float* red = reinterpret_cast<float*>(s_kv);  // merge area, after the last stage
+    static_assert(MergeArea<D, HG, NW>::BYTES <= STAGES * 2 * STAGE_BYTES, "merge area");
 
     if (WS && warp == NW) {
         // 2. producer warp: keep every stage loaded as soon as it is released
@@ -359,8 +361,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREAD
         if (s_abort) return;
         pdl_launch_dependents();
         __syncthreads();
-        merge_warps_and_store<T, D, HG, NW>(a, red, red_m, red_l, b, h0, nh, part, np, tid,
-                                            THREADS);
+        merge_warps_and_store<T, D, HG, NW>(a, red, b, h0, nh, part, np, tid, THREADS);
         return;
     }
 
@@ -379,31 +380,31 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREAD
         const int stage = it % STAGES;
         if (!mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status)) s_abort = 1;
         if (WS && s_abort) break;
-        if (!s_abort) {
-            const int wvalid = ntok - (it * TILE + warp * 16);  // tokens this warp owns
-            if (wvalid > 0) {
-                const unsigned char* Kw = s_kv + stage * 2 * STAGE_BYTES + warp * 16 * ROW;
-                W.tile(Kw, Kw + STAGE_BYTES, wvalid, s_p[warp]);
-            }
+        const int wvalid = ntok - (it * TILE + warp * 16);  // tokens this warp owns
+        if (!s_abort && wvalid > 0) {
+            const unsigned char* Kw = s_kv + stage * 2 * STAGE_BYTES + warp * 16 * ROW;
+            W.fetch(Kw, Kw + STAGE_BYTES);
         }
+        if (!W.EARLY && !s_abort && wvalid > 0) W.compute(wvalid, s_p[warp]);
+        // the stage's data is in registers (or used): hand the stage back
         if (WS) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
         } else {
-            __syncthreads();  // every warp is done with this stage
+            __syncthreads();
             if (s_abort) break;
             if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage, pol);
         }
+        if (W.EARLY && wvalid > 0) W.compute(wvalid, s_p[warp]);
     }
     if (WS) __syncthreads();  // producer and consumers: every stage consumed
     if (s_abort) return;
     if (!WS) pdl_launch_dependents();
 
     // 6. merge the warps
-    W.park(warp, red, red_m, red_l);
+    W.template park<NW>(warp, red);
     __syncthreads();
-    merge_warps_and_store<T, D, HG, NW>(a, red, red_m, red_l, b, h0, nh, part, np, tid,
-                                        WS ? THREADS : NW * 32);
+    merge_warps_and_store<T, D, HG, NW>(a, red, b, h0, nh, part, np, tid, WS ? THREADS : NW * 32);
 }
 
 template <typename T, int D, int BS, int HG, int NW = 4, int STAGES = 0, bool WS = false>

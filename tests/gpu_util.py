@@ -30,7 +30,7 @@ class DeviceInputs:
         self.out = torch.empty_like(self.q)
 
     def decode(self, partition_size=0, kernel=pkv.PKV_KERNEL_AUTO, max_context_len=None,
-               fill_out=None):
+               fill_out=None, seq_order=None):
         c = self.inp.cfg
         mcl = self.inp.max_context_len if max_context_len is None else max_context_len
         ws_bytes = pkv.pkv_decode_workspace_size(c.num_seqs, c.num_q_heads, c.num_kv_heads,
@@ -41,7 +41,7 @@ class DeviceInputs:
         pkv.pkv_paged_attention_decode(self.out, self.q, self.k, self.v, self.bt, self.cl,
                                        c.scale, c.block_size, mcl,
                                        partition_size=partition_size, workspace=ws,
-                                       kernel=kernel)
+                                       seq_order=seq_order, kernel=kernel)
         torch.cuda.synchronize()
         return self.out
 

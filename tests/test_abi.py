@@ -36,12 +36,12 @@ def test_status_strings_and_version():
 
 
 def _decode(**over):
-    a = dict(out=None, q=None, k=None, v=None, bt=None, cl=None, B=4, Hq=8, Hkv=2, D=128,
+    a = dict(out=None, q=None, k=None, v=None, bt=None, cl=None, order=None, B=4, Hq=8, Hkv=2, D=128,
              bs=16, mb=8, N=64, maxlen=100, scale=0.1, dt=b.PKV_F16, P=0, ws=None, wsb=0,
              kern=0, stream=None)
     a.update(over)
     return b.lib.pkv_paged_attention_decode(
-        a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["B"], a["Hq"], a["Hkv"], a["D"],
+        a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["order"], a["B"], a["Hq"], a["Hkv"], a["D"],
         a["bs"], a["mb"], a["N"], a["maxlen"], a["scale"], a["dt"], a["P"], a["ws"], a["wsb"],
         a["kern"], a["stream"])
 
@@ -85,8 +85,8 @@ def test_workspace_size_formula():
 
 def test_default_partition_rule():
     d = b.lib.pkv_decode_default_partition
-    assert d(64, 40, 2048) == 1024
-    assert d(8, 8, 131072) == 1024
+    assert d(64, 40, 2048) == 2048
+    assert d(8, 8, 131072) == 2048
     assert d(1, 1, 4096) == 64          # tiny batches split finer
     p = d(4, 4, 512)
     assert 64 <= p <= 512 and p % 64 == 0
@@ -101,3 +101,11 @@ def test_append_and_copy_host_checks():
     assert g(None, None, None, 0, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_OK
     assert g(None, None, None, 2, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL
     assert g(None, None, None, -1, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL
+
+
+def test_schedule_order_longest_first():
+    import numpy as np
+    import paged_kv_cache_346_b200 as pkv
+    lens = np.array([5, 100, 7, 100, 0, 64], dtype=np.int32)
+    assert pkv.pkv_decode_schedule_order(lens).tolist() == [1, 3, 5, 2, 0, 4]
+    assert pkv.pkv_decode_schedule_order(np.zeros(0, np.int32)).tolist() == []

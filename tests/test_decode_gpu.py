@@ -221,3 +221,26 @@ def test_full_size_sampled_rows(name, full_inputs):
         # the N(0,1) value range, never beyond the largest |v| in the pool
         vmax = float(torch.max(torch.abs(dev.v.float())))
         assert np.all(np.abs(full) <= vmax * 1.01 + 1e-3)
+
+
+@pytest.mark.parametrize("dtype,G", [("f16", 1), ("bf16", 8), ("f32", 2)])
+def test_schedule_order_changes_no_bit(dtype, G):
+    """Scheduling the longest sequences first only changes timing: outputs
+    are bit-identical to the natural order."""
+    cfg = _cfg(dtype, 2 * G, 2, 128 if dtype != "f32" else 64, 16, RAGGED)
+    inp = make_decode_inputs(cfg, seed=40 + G)
+    dev = DeviceInputs(inp)
+    order = torch.from_numpy(pkv.pkv_decode_schedule_order(inp.context_lens)).cuda()
+    for kern in _kernels_for(dtype, G):
+        for P in (0, 64):
+            a = dev.decode(partition_size=P, kernel=kern).clone()
+            b = dev.decode(partition_size=P, kernel=kern, seq_order=order, fill_out=3.0).clone()
+            assert torch.equal(a, b), (kern, P)
+
+
+def test_bad_schedule_order_entry_is_flagged():
+    cfg = _cfg("f16", 4, 4, 128, 16, (40, 40))
+    dev = DeviceInputs(make_decode_inputs(cfg, seed=16))
+    pkv.pkv_device_status(clear=True)
+    dev.decode(seq_order=torch.tensor([1, 7], dtype=torch.int32, device="cuda"))
+    assert pkv.pkv_device_status(clear=True) & pkv.PKV_DEV_BAD_ORDER
