@@ -24,6 +24,7 @@ sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import math
 import os
@@ -74,12 +75,12 @@ def measured_peaks():
     return None
 
 
-def step_bytes(cfg, lens) -> int:
+def step_bytes(cfg, lens, window: int = 0) -> int:
     """Decode algorithmic bytes + the append: read k, v of each new token,
     write them, read the slot."""
     e = ELEM_BYTES[cfg.dtype]
     append = len(lens) * (2 * 2 * cfg.num_kv_heads * cfg.head_dim * e + 8)
-    return algorithmic_bytes(cfg, lens) + append
+    return algorithmic_bytes(cfg, lens, window) + append
 
 
 class ClockSampler:
@@ -313,23 +314,25 @@ def run_ours(args, cfg):
     order_np = pkv.pkv_decode_schedule_order(inp.context_lens) if args.order else None
     order = dev(order_np) if order_np is not None else None
     P = args.partition
-    ws_bytes = pkv.pkv_decode_workspace_size(B, cfg.num_q_heads, H, D, mcl, P)
+    W = args.window
+    span = min(mcl, W + bs - 1) if W > 0 else mcl
+    ws_bytes = pkv.pkv_decode_workspace_size(B, cfg.num_q_heads, H, D, span, P)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
-    Pused = P or pkv.pkv_decode_default_partition(B, H, mcl)
-    launches_per_step = 1 + 1 + (1 if math.ceil(mcl / Pused) > 1 else 0)
+    Pused = P or pkv.pkv_decode_default_partition(B, H, span)
+    launches_per_step = 1 + 1 + (1 if math.ceil(span / Pused) > 1 else 0)
     stream = torch.cuda.current_stream()
 
     def decode():
         pkv.pkv_paged_attention_decode(out, q, kc, vc, bt, cl, cfg.scale, bs, mcl,
                                        partition_size=P, workspace=ws, seq_order=order,
-                                       kernel=kern, stream=stream)
+                                       sliding_window=W, kernel=kern, stream=stream)
 
     def step():
         pkv.pkv_kv_cache_append(kc, vc, knew, vnew, slots, stream=stream)
         decode()
 
-    nbytes = step_bytes(cfg, lens)
-    dec_bytes = algorithmic_bytes(cfg, lens)
+    nbytes = step_bytes(cfg, lens, W)
+    dec_bytes = algorithmic_bytes(cfg, lens, W)
 
     # ---- device-resident timing
     for _ in range(args.warmup):
@@ -356,53 +359,86 @@ def run_ours(args, cfg):
     if flags:
         raise SystemExit(f"device status flags {flags:#x} during the benchmark")
 
-    # ---- end to end through the public API: step inputs from pinned host
-    # memory each step, the output read back each step
-    h_q = torch.from_numpy(inp.q.view(np.int16) if cfg.dtype == "bf16" else inp.q)
-    h_q = (h_q.view(torch.bfloat16) if cfg.dtype == "bf16" else h_q).pin_memory()
-    h_knew, h_vnew = knew.cpu().pin_memory(), vnew.cpu().pin_memory()
-    h_slots = torch.from_numpy(slots_np).pin_memory()
-    h_bt = torch.from_numpy(inp.block_tables).pin_memory()
-    h_cl = torch.from_numpy(inp.context_lens).pin_memory()
-    h_order = torch.from_numpy(order_np).pin_memory() if order_np is not None else None
-    d_order = torch.empty_like(order) if order is not None else None
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    d_knew, d_vnew = torch.empty_like(knew), torch.empty_like(vnew)
-    d_q, d_slots, d_bt, d_cl = (torch.empty_like(q), torch.empty_like(slots),
-                                torch.empty_like(bt), torch.empty_like(cl))
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_knew, h_vnew, h_slots, h_bt, h_cl)
-              + ((h_order,) if h_order is not None else ()))
-    d2h = h_out.numel() * h_out.element_size()
+    # ---- end to end through the public API: every step copies its inputs
+    # (q, the new tokens' K/V, slots, tables, lengths, schedule order) from
+    # pinned host memory and reads its output back.  The inputs of a step are
+    # packed in one pinned buffer (one upload), and the C ABI is called with
+    # argument lists prepared once, so the host keeps ahead of the GPU.  Two
+    # input and two output buffers and two copy streams let step i+1's upload
+    # and step i-1's readback run under step i's kernels; events order every
+    # reuse.
+    fields = [("q", q), ("knew", knew), ("vnew", vnew), ("slots", slots), ("bt", bt), ("cl", cl)]
+    if order is not None:
+        fields.append(("order", order))
+    offs, total = {}, 0
+    for name, t in fields:
+        offs[name] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    h_in = torch.empty(total, dtype=torch.uint8).pin_memory()
+    for name, t in fields:
+        nb_ = t.numel() * t.element_size()
+        h_in[offs[name]:offs[name] + nb_].copy_(t.reshape(-1).view(torch.uint8).cpu())
+    d_in = [torch.empty(total, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    d_out = [torch.empty_like(out) for _ in range(2)]
+    h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for _, t in fields)
+    d2h = h_out[0].numel() * h_out[0].element_size()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_done + ev_out:
+        e.record(stream)
+    c_stream = ctypes.c_void_p(stream.cuda_stream)
+    dt_code = pkv.torch_dtype_code(q.dtype)
+    N_blocks = kc.shape[0]
+    calls = []
+    for j in range(2):
+        ptr = {name: ctypes.c_void_p(d_in[j].data_ptr() + offs[name]) for name, _ in fields}
+        append_args = (ctypes.c_void_p(kc.data_ptr()), ctypes.c_void_p(vc.data_ptr()),
+                       ptr["knew"], ptr["vnew"], ptr["slots"], B, H, D, bs, N_blocks, dt_code,
+                       c_stream)
+        decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"],
+                       ctypes.c_void_p(kc.data_ptr()), ctypes.c_void_p(vc.data_ptr()), ptr["bt"],
+                       ptr["cl"], ptr.get("order"), B, cfg.num_q_heads, H, D, bs,
+                       bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
+                       ctypes.c_void_p(ws.data_ptr()), ws.numel(), kern, c_stream)
+        calls.append((append_args, decode_args))
 
-    def e2e_step():
-        d_q.copy_(h_q, non_blocking=True)
-        d_knew.copy_(h_knew, non_blocking=True)
-        d_vnew.copy_(h_vnew, non_blocking=True)
-        d_slots.copy_(h_slots, non_blocking=True)
-        d_bt.copy_(h_bt, non_blocking=True)
-        d_cl.copy_(h_cl, non_blocking=True)
-        if h_order is not None:
-            d_order.copy_(h_order, non_blocking=True)
-        pkv.pkv_kv_cache_append(kc, vc, d_knew, d_vnew, d_slots, stream=stream)
-        pkv.pkv_paged_attention_decode(out, d_q, kc, vc, d_bt, d_cl, cfg.scale, bs, mcl,
-                                       partition_size=P, workspace=ws, seq_order=d_order,
-                                       kernel=kern, stream=stream)
-        h_out.copy_(out, non_blocking=True)
+    def e2e_step(i):
+        j = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_done[j])          # the kernels of step i-2 are done with d_in[j]
+            d_in[j].copy_(h_in, non_blocking=True)
+            ev_in[j].record(s_in)
+        stream.wait_event(ev_in[j])
+        stream.wait_event(ev_out[j])             # d_out[j] of step i-2 has been read back
+        a_args, d_args = calls[j]
+        if pkv.lib.pkv_kv_cache_append(*a_args) or pkv.lib.pkv_paged_attention_decode(*d_args):
+            raise SystemExit("C-ABI call failed in the e2e loop")
+        ev_done[j].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[j])
+            h_out[j].copy_(d_out[j], non_blocking=True)
+            ev_out[j].record(s_out)
 
-    e2e_steps = max(3, min(args.steps, 200))
-    for _ in range(max(args.warmup, 3)):
-        e2e_step()
+    e2e_steps = max(4, min(args.steps, 400))
+    for i in range(max(args.warmup, 3)):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    s_in.wait_stream(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    stream.wait_event(ev_out[(e2e_steps - 1) % 2])
+    stream.wait_event(ev_out[(e2e_steps - 2) % 2])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    assert torch.equal(h_out, out.cpu())
+    assert torch.equal(h_out[0], out.cpu()) and torch.equal(h_out[1], out.cpu())
 
     # ---- max over ranks
     ms, dec_ms, e2e_ms = max_over_ranks([ms, dec_ms, e2e_ms], world)
@@ -426,6 +462,7 @@ def run_ours(args, cfg):
                        "num_q_heads": cfg.num_q_heads, "num_kv_heads": H, "head_dim": D,
                        "block_size": bs, "partition_size": Pused, "kernel": args.kernel,
                        "schedule": "longest-first" if args.order else "batch order",
+                       "sliding_window": W,
                        "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (%.2f GB of K/V per step)" % (
                            dec_bytes / 1e9)},
@@ -602,6 +639,74 @@ def run_cow(args):
     return 0
 
 
+def run_swap(args):
+    """Swapping: whole pages of the Llama-2-13B-shaped layer (40 heads x 16
+    tokens x 128 dims fp16 = 160 KB per page, K and V) moved between the
+    device pool and a page-locked host pool by pkv_swap_blocks, in a seeded
+    random scatter, both directions; next to it the host link's rate for one
+    contiguous copy of the same bytes (torch copy_, the copy engines)."""
+    import torch
+
+    import paged_kv_cache_346_b200 as pkv
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    H, bs, D = 40, 16, 128
+    n = 2048                                       # pages per direction (K and V each)
+    N_dev, N_host = 3 * n, 2 * n
+    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    dk = torch.randn((N_dev, H, bs, D), generator=g, device="cuda").half()
+    dv = torch.randn((N_dev, H, bs, D), generator=g, device="cuda").half()
+    hk = torch.empty((N_host, H, bs, D), dtype=torch.float16).pin_memory()
+    hv = torch.empty((N_host, H, bs, D), dtype=torch.float16).pin_memory()
+    rng_ = np.random.default_rng(args.seed)
+    out_pairs = np.stack([rng_.choice(N_dev, n, replace=False),
+                          rng_.choice(N_host, n, replace=False)], 1).astype(np.int32)
+    in_pairs = np.stack([out_pairs[:, 1], rng_.choice(N_dev, n, replace=False)], 1).astype(np.int32)
+    p_out, p_in = torch.from_numpy(out_pairs).cuda(), torch.from_numpy(in_pairs).cuda()
+    stream = torch.cuda.current_stream()
+    page = H * bs * D * 2
+    nbytes = 2 * n * page                          # K and V pages moved per call
+
+    def timed(fn, reps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    reps = max(3, min(args.steps, 20))
+    t_out = timed(lambda: pkv.pkv_swap_blocks(hk, hv, dk, dv, p_out, stream=stream), reps)
+    t_in = timed(lambda: pkv.pkv_swap_blocks(dk, dv, hk, hv, p_in, stream=stream), reps)
+    flat_h = hk.view(-1)[: n * page // 2]
+    flat_d = dk.view(-1)[: n * page // 2]
+    t_d2h = timed(lambda: flat_h.copy_(flat_d, non_blocking=True), reps)
+    t_h2d = timed(lambda: flat_d.copy_(flat_h, non_blocking=True), reps)
+    flags = pkv.pkv_device_status(clear=True)
+    if rank == 0:
+        line = {
+            "metric": "swap GB/s (pages between the device pool and page-locked host memory)",
+            "value": round(nbytes / (t_in * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "n_gpus": 1, "steps": reps, "warmup": args.warmup, "higher_is_better": True,
+            "data": "synthetic", "dtype": "f16",
+            "config": {"workload": "swap", "pages": n, "page_bytes": page,
+                       "bytes_per_call": nbytes},
+            "swap_in_GBps": round(nbytes / (t_in * 1e-3) / 1e9, 2),
+            "swap_out_GBps": round(nbytes / (t_out * 1e-3) / 1e9, 2),
+            "swap_in_ms": round(t_in, 4), "swap_out_ms": round(t_out, 4),
+            "contiguous_h2d_GBps": round((n * page) / (t_h2d * 1e-3) / 1e9, 2),
+            "contiguous_d2h_GBps": round((n * page) / (t_d2h * 1e-3) / 1e9, 2),
+            "device_status": flags,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -609,11 +714,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama2_13b_layer",
-                    choices=sorted(CONFIGS) + ["cow_sampling"])
+                    choices=sorted(CONFIGS) + ["cow_sampling", "swap"])
     ap.add_argument("--kernel", choices=["auto", "simt", "mma"], default="auto")
     ap.add_argument("--partition", type=int, default=None,
                     help="tokens per partition (default: the workload's, else automatic)")
     ap.add_argument("--seed", type=int, default=2)
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding window in tokens (0: attend to the whole context)")
     ap.add_argument("--no-order", dest="order", action="store_false",
                     help="schedule sequences in batch order instead of longest first")
     ap.add_argument("--cpu-budget", type=float, default=12.0,
@@ -625,6 +732,8 @@ def main():
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     if args.workload == "cow_sampling":
         return run_cow(args)
+    if args.workload == "swap":
+        return run_swap(args)
     cfg = CONFIGS[args.workload]
     if args.partition is None:
         args.partition = cfg.partition_size

@@ -117,7 +117,8 @@ PKV_API size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_
 /*
  * Paged decode attention: for every sequence b and query head h,
  *   out[b,h,:] = softmax_t(scale * q[b,h,:] . k_t) weighted sum of v_t,
- * over the tokens t < context_lens[b], k_t and v_t read from the physical
+ * over the tokens t < context_lens[b] (the last sliding_window of them when
+ * sliding_window > 0), k_t and v_t read from the physical
  * block block_tables[b][t / block_size] at offset t % block_size
  * ("pagedattention vllm" §Attention Computation: gather physical blocks,
  * compute as if contiguous).  A sequence with length 0 gets a zero row.
@@ -142,6 +143,13 @@ PKV_API size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_
  *       entry leaves some row unwritten.
  *   max_context_len: host-side upper bound of context_lens, and
  *       <= max_blocks_per_seq * block_size.
+ *   sliding_window: 0 to attend to the whole context, else W > 0: sequence
+ *       b attends only to its last W tokens, [max(0, L_b - W), L_b)
+ *       ("pagedattention vllm" §Advanced Features: sliding-window models
+ *       cache only recent blocks).  Table entries of blocks that lie wholly
+ *       before the window are never read (they may be -1 once released,
+ *       pkv_alloc_slide_window).  The workspace is then sized with
+ *       max_context_len = min(max_context_len, W + block_size - 1).
  *   partition_size: 0 for the default, else a multiple of 64 in [64, 8192].
  *   workspace: device memory of at least pkv_decode_workspace_size(...)
  *       bytes, 16-byte aligned; may be NULL when that size is 0.
@@ -155,8 +163,8 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
                                int num_seqs,
                                int num_q_heads, int num_kv_heads, int head_dim,
                                int block_size, int max_blocks_per_seq, int num_blocks,
-                               int max_context_len, float scale, pkv_dtype dtype,
-                               int partition_size, void* workspace,
+                               int max_context_len, float scale, int sliding_window,
+                               pkv_dtype dtype, int partition_size, void* workspace,
                                size_t workspace_bytes, pkv_kernel kernel,
                                pkv_stream_t stream);
 
@@ -193,8 +201,9 @@ PKV_API int pkv_paged_attention_decode_static_ws(
     void* out, const void* q, const void* k_cache, const void* v_cache,
     const int32_t* block_tables, const int32_t* context_lens, const int32_t* seq_order,
     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-    int max_blocks_per_seq, int num_blocks, int max_context_len, float scale, pkv_dtype dtype,
-    int partition_size, pkv_kernel kernel, pkv_stream_t stream);
+    int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+    int sliding_window, pkv_dtype dtype, int partition_size, pkv_kernel kernel,
+    pkv_stream_t stream);
 
 /*
  * Host helper: order_out[0..n) = the sequence indices sorted by decreasing
@@ -232,6 +241,23 @@ PKV_API int pkv_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_p
                     int num_blocks, pkv_dtype dtype, pkv_stream_t stream);
 
 /*
+ * Swap pages between two pools, one of which may be page-locked host memory
+ * (cudaHostAlloc / cudaHostRegister, e.g. torch's pin_memory): for each pair,
+ * dst_k[dst] = src_k[src] and dst_v[dst] = src_v[src], whole blocks of
+ * num_kv_heads x block_size x head_dim elements ("pagedattention vllm"
+ * §Memory Management: swapping).  One kernel moves all pairs, reading or
+ * writing the host pool directly over the host link.  Pools are checked on
+ * the host: pageable host memory is refused (PKV_EINVAL), since the GPU
+ * cannot reach it.  block_pairs: int32 [num_pairs][2] (src, dst) in device or
+ * page-locked host memory; pairs outside their pools are skipped and flagged
+ * (PKV_DEV_BAD_BLOCK).
+ */
+PKV_API int pkv_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                            const int32_t* block_pairs, int num_pairs, int src_num_blocks,
+                            int dst_num_blocks, int num_kv_heads, int head_dim, int block_size,
+                            pkv_dtype dtype, pkv_stream_t stream);
+
+/*
  * Reads (and with clear != 0, resets) the device status word of the current
  * device: an OR of PKV_DEV_* bits set by earlier calls.  Synchronises the
  * device.
@@ -264,12 +290,19 @@ typedef struct {
     int32_t used_blocks;     /* blocks with a reference count > 0 */
     int32_t shared_blocks;   /* blocks with a reference count > 1 */
     int32_t num_seqs;
-    int64_t refcount_sum;    /* = total block-table entries over sequences */
-    int64_t logical_tokens;  /* sum of sequence lengths */
+    int64_t refcount_sum;    /* = block-table entries of the resident sequences */
+    int64_t logical_tokens;  /* sum of sequence lengths (resident and swapped) */
+    int32_t num_host_blocks;
+    int32_t free_host_blocks;
+    int32_t swapped_seqs;
+    int32_t reserved;
 } pkv_alloc_stats_t;
 
 /* num_blocks > 0, block_size > 0.  *out = new allocator (free with destroy). */
 PKV_API int pkv_alloc_create(int num_blocks, int block_size, pkv_alloc** out);
+/* The same with a host pool of num_host_blocks >= 0 blocks for swapping. */
+PKV_API int pkv_alloc_create_swap(int num_blocks, int num_host_blocks, int block_size,
+                                  pkv_alloc** out);
 PKV_API void pkv_alloc_destroy(pkv_alloc* a);
 /* New sequence holding num_tokens >= 0 tokens. */
 PKV_API int pkv_alloc_add_seq(pkv_alloc* a, int64_t seq_id, int num_tokens);
@@ -298,6 +331,39 @@ PKV_API int pkv_alloc_refcount(const pkv_alloc* a, int32_t block, int* out);
 PKV_API int pkv_alloc_stats(const pkv_alloc* a, pkv_alloc_stats_t* out);
 /* Free blocks in the order they will be handed out. */
 PKV_API int pkv_alloc_free_list(const pkv_alloc* a, int32_t* out, int capacity, int* n_out);
+
+/*
+ * Swapping ("pagedattention vllm" §Memory Management: blocks can be swapped
+ * to CPU memory, trading latency for capacity).  swap_out moves a resident
+ * sequence to the host pool: for each table entry in logical order it takes a
+ * host block (LIFO free stack, a new pool pops 0, 1, 2, ...), reports the pair
+ * (device block, host block) and drops one reference to the device block
+ * (a block other sequences still share stays on the device); the table then
+ * holds host block ids.  swap_in does the reverse: one new device block per
+ * entry, pairs (host block, device block), host blocks pushed back in logical
+ * order.  Run pkv_swap_blocks on the pairs, in stream order, before the
+ * device blocks are reused.  A swapped sequence cannot be appended to,
+ * forked or put in a decode batch (PKV_EINVAL) until swapped in.
+ * pairs: host int32 [capacity][2]; *num_pairs = table length (PKV_EBOUNDS
+ * and nothing done when it exceeds capacity); PKV_ENOMEM when the target
+ * pool lacks free blocks.
+ */
+PKV_API int pkv_alloc_swap_out(pkv_alloc* a, int64_t seq_id, int32_t* pairs, int capacity,
+                               int* num_pairs);
+PKV_API int pkv_alloc_swap_in(pkv_alloc* a, int64_t seq_id, int32_t* pairs, int capacity,
+                              int* num_pairs);
+PKV_API int pkv_alloc_is_swapped(const pkv_alloc* a, int64_t seq_id, int* swapped);
+
+/*
+ * Sliding window ("pagedattention vllm" §Advanced Features: with sliding-window
+ * attention only recent blocks are kept): every block of resident sequence
+ * seq_id that lies wholly before its last `window` tokens ((j+1) * block_size
+ * <= len - window) drops one reference (freed at zero) and its table entry
+ * becomes -1; the length is unchanged.  *released = entries released by this
+ * call.  Entries that are -1 are skipped by fork, free, swap and the decode
+ * with the same or a smaller window.  window <= 0 -> PKV_EINVAL.
+ */
+PKV_API int pkv_alloc_slide_window(pkv_alloc* a, int64_t seq_id, int window, int* released);
 
 #ifdef __cplusplus
 }

@@ -62,7 +62,7 @@ def lib():
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                ctypes.c_int64, ctypes.c_double, ctypes.c_int, ctypes.c_void_p,
+                ctypes.c_int64, ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                 ctypes.c_int64, ctypes.c_int]
             L.pkvo_max_threads.restype = ctypes.c_int
             _lib = L
@@ -84,8 +84,9 @@ def decode_bits(arr: np.ndarray, dtype: str) -> np.ndarray:
 
 def paged_decode(q, k_cache, v_cache, block_tables, context_lens, *, scale: float,
                  dtype: str, num_kv_heads: int | None = None, rows=None,
-                 threads: int = 0) -> np.ndarray:
-    """float64 paged decode attention.
+                 threads: int = 0, window: int = 0) -> np.ndarray:
+    """float64 paged decode attention (window > 0: over each sequence's last
+    `window` tokens only).
 
     q [B, Hq, D]; k_cache, v_cache [N, Hkv, bs, D] in the storage dtype
     (bf16 as uint16 bits); block_tables int32 [B, max_blocks];
@@ -111,14 +112,15 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, *, scale: floa
     rc = lib().pkvo_paged_decode(out.ctypes.data, q.ctypes.data, k_cache.ctypes.data,
                                  v_cache.ctypes.data, bt.ctypes.data, cl.ctypes.data,
                                  B, Hq, Hkv, D, bs, bt.shape[1], N, float(scale),
-                                 DTYPE_CODE[dtype], rp, nr, int(threads))
+                                 int(window), DTYPE_CODE[dtype], rp, nr, int(threads))
     if rc != 0:
         raise ValueError(f"oracle rejected the inputs (code {rc})")
     return out
 
 
-def paged_decode_inputs(inp: DecodeInputs, rows=None, threads: int = 0) -> np.ndarray:
+def paged_decode_inputs(inp: DecodeInputs, rows=None, threads: int = 0,
+                        window: int = 0) -> np.ndarray:
     c = inp.cfg
     return paged_decode(inp.q, inp.k_cache, inp.v_cache, inp.block_tables,
                         inp.context_lens, scale=c.scale, dtype=c.dtype, rows=rows,
-                        threads=threads)
+                        threads=threads, window=window)

@@ -38,8 +38,9 @@ def attention_row(qrow, ks, vs, scale):
     return [sum(w * v[d] for w, v in zip(weights, vs)) / z for d in range(D)]
 
 
-def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale):
-    """q [B][Hq][D], caches [N][Hkv][bs][D] (float64 values) -> [B][Hq][D]."""
+def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, window=0):
+    """q [B][Hq][D], caches [N][Hkv][bs][D] (float64 values) -> [B][Hq][D];
+    window > 0: only each sequence's last `window` tokens."""
     B = len(q)
     Hq = len(q[0])
     Hkv = len(k_cache[0])
@@ -51,6 +52,8 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale):
         rows = []
         for h in range(Hq):
             ks, vs = contiguous_kv(k_cache, v_cache, block_tables[b], L, h // G, bs)
+            if window > 0:
+                ks, vs = ks[-window:], vs[-window:]
             rows.append(attention_row([float(x) for x in q[b][h]], ks, vs, scale))
         out.append(rows)
     return out

@@ -18,11 +18,13 @@
  *
  * So, for sequence b and query head h (G = Hq / Hkv query heads share KV head
  * g = h / G), with L = context_lens[b]:
- *     k_t = K[table[b][t / bs], g, t % bs, :]   (same for v_t), t < L
+ *     k_t = K[table[b][t / bs], g, t % bs, :]   (same for v_t), lo <= t < L
  *     s_t = scale * sum_d q[b,h,d] k_t[d]
  *     out[b,h,:] = sum_t exp(s_t - max s) v_t / sum_t exp(s_t - max s)
  * in float64, plain loops, no blocking and no online rescaling.  L = 0 gives a
- * zero row.  The inputs are decoded bit by bit from their storage type
+ * zero row.  lo = 0, or with a sliding window of W tokens lo = max(0, L - W):
+ * only the last W tokens are attended to ("pagedattention vllm" §Advanced
+ * Features: sliding-window models keep only recent blocks).  The inputs are decoded bit by bit from their storage type
  * (float32, IEEE binary16, bfloat16) by this file's own decoders.
  *
  * OpenMP spreads the independent (b, h) rows over host threads; each row's
@@ -108,10 +110,11 @@ static int decode_row(double* out_row, const void* q, const void* k_cache,
                       const int32_t* context_lens, int b, int h, int num_q_heads,
                       int num_kv_heads, int head_dim, int block_size,
                       int max_blocks_per_seq, int64_t num_blocks, double scale,
-                      int dtype, double* s /* scratch, >= L + head_dim */) {
+                      int window, int dtype, double* s /* scratch, >= L + head_dim */) {
     const int G = num_q_heads / num_kv_heads;
     const int g = h / G;
     const int L = context_lens[b];
+    const int lo = (window > 0 && L > window) ? L - window : 0;
     const int D = head_dim;
     for (int d = 0; d < D; ++d) out_row[d] = 0.0;
     if (L <= 0) return 0;
@@ -122,7 +125,7 @@ static int decode_row(double* out_row, const void* q, const void* k_cache,
     for (int d = 0; d < D; ++d) qrow[d] = load_elem(q, q_off + d, dtype);
 
     /* logits, gathered through the block table */
-    for (int t = 0; t < L; ++t) {
+    for (int t = lo; t < L; ++t) {
         int32_t phys = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
         if (phys < 0 || phys >= num_blocks) return -1;
         int64_t k_off = (((int64_t)phys * num_kv_heads + g) * block_size + t % block_size) * D;
@@ -131,11 +134,11 @@ static int decode_row(double* out_row, const void* q, const void* k_cache,
             acc += qrow[d] * load_elem(k_cache, k_off + d, dtype);
         s[t] = scale * acc;
     }
-    double m = s[0];
-    for (int t = 1; t < L; ++t)
+    double m = s[lo];
+    for (int t = lo + 1; t < L; ++t)
         if (s[t] > m) m = s[t];
     double denom = 0.0;
-    for (int t = 0; t < L; ++t) {
+    for (int t = lo; t < L; ++t) {
         double w = exp(s[t] - m);
         denom += w;
         int32_t phys = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
@@ -156,7 +159,7 @@ int pkvo_paged_decode(double* out, const void* q, const void* k_cache,
                       const int32_t* context_lens, int num_seqs, int num_q_heads,
                       int num_kv_heads, int head_dim, int block_size,
                       int max_blocks_per_seq, int64_t num_blocks, double scale,
-                      int dtype, const int32_t* rows, int64_t num_rows,
+                      int window, int dtype, const int32_t* rows, int64_t num_rows,
                       int num_threads) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         block_size <= 0 || num_q_heads % num_kv_heads != 0)
@@ -189,7 +192,8 @@ int pkvo_paged_decode(double* out, const void* q, const void* k_cache,
             }
             if (decode_row(out + i * head_dim, q, k_cache, v_cache, block_tables,
                            context_lens, b, h, num_q_heads, num_kv_heads, head_dim,
-                           block_size, max_blocks_per_seq, num_blocks, scale, dtype, s))
+                           block_size, max_blocks_per_seq, num_blocks, scale, window, dtype,
+                           s))
                 err |= 1;
         }
         free(s);

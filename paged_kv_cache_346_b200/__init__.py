@@ -23,7 +23,7 @@ from ._binding import (PKV_BF16, PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD
 
 __all__ = [
     "pkv_paged_attention_decode", "pkv_decode_workspace_size", "pkv_decode_has_kernel",
-    "pkv_paged_attention_decode_static_ws", "pkv_decode_default_partition",
+    "pkv_paged_attention_decode_static_ws", "pkv_swap_blocks", "pkv_decode_default_partition",
     "pkv_kv_cache_append", "pkv_copy_blocks", "pkv_device_status", "BlockAllocator",
     "PagedKVError", "lib", "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_KERNEL_AUTO",
     "PKV_KERNEL_SIMT", "PKV_KERNEL_MMA", "PKV_DEV_BAD_BLOCK", "PKV_DEV_BAD_LEN",
@@ -80,13 +80,15 @@ def pkv_paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torc
                                max_context_len: int, *, partition_size: int = 0,
                                workspace: torch.Tensor | None = None,
                                seq_order: torch.Tensor | None = None,
+                               sliding_window: int = 0,
                                kernel: int = PKV_KERNEL_AUTO, stream=None) -> torch.Tensor:
     """out [B, Hq, D] <- paged decode attention (see pkv_paged_attention_decode
     in pagedkv.h).  k_cache/v_cache [N, Hkv, block_size, D]; block_tables
     int32 [B, max_blocks]; context_lens int32 [B]; max_context_len is a host
     bound of context_lens.  workspace: a CUDA tensor of at least
     pkv_decode_workspace_size(...) bytes when sequences span partitions.
-    seq_order: optional int32 [B] schedule order (pkv_decode_schedule_order)."""
+    seq_order: optional int32 [B] schedule order (pkv_decode_schedule_order).
+    sliding_window: 0, or attend only to each sequence's last W tokens."""
     for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
                  (block_tables, "block_tables"), (context_lens, "context_lens")):
         _dev(t, n)
@@ -111,8 +113,9 @@ def pkv_paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torc
     check(lib.pkv_paged_attention_decode(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         _ptr(context_lens), _ptr(seq_order), B, Hq, Hkv, D, bs, block_tables.shape[1], N,
-        int(max_context_len), float(scale), torch_dtype_code(q.dtype), int(partition_size),
-        _ptr(workspace), ws_bytes, int(kernel), _stream(stream)), "pkv_paged_attention_decode")
+        int(max_context_len), float(scale), int(sliding_window), torch_dtype_code(q.dtype),
+        int(partition_size), _ptr(workspace), ws_bytes, int(kernel), _stream(stream)),
+        "pkv_paged_attention_decode")
     return out
 
 
@@ -122,6 +125,7 @@ def pkv_paged_attention_decode_static_ws(out: torch.Tensor, q: torch.Tensor,
                                          scale: float, block_size: int, max_context_len: int, *,
                                          partition_size: int = 0,
                                          seq_order: torch.Tensor | None = None,
+                                         sliding_window: int = 0,
                                          kernel: int = PKV_KERNEL_AUTO,
                                          stream=None) -> torch.Tensor:
     """pkv_paged_attention_decode without a caller workspace, for callers that
@@ -137,8 +141,8 @@ def pkv_paged_attention_decode_static_ws(out: torch.Tensor, q: torch.Tensor,
     check(lib.pkv_paged_attention_decode_static_ws(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         _ptr(context_lens), _ptr(seq_order), B, Hq, Hkv, D, bs, block_tables.shape[1], N,
-        int(max_context_len), float(scale), torch_dtype_code(q.dtype), int(partition_size),
-        int(kernel), _stream(stream)),
+        int(max_context_len), float(scale), int(sliding_window), torch_dtype_code(q.dtype),
+        int(partition_size), int(kernel), _stream(stream)),
         f"pkv_paged_attention_decode_static_ws (scratch limit "
         f"{_b.PKV_STATIC_WORKSPACE_BYTES} bytes)")
     return out
@@ -190,6 +194,30 @@ def pkv_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_pairs: t
           "pkv_copy_blocks")
 
 
+def pkv_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor,
+                    src_v: torch.Tensor, block_pairs: torch.Tensor, *, stream=None) -> None:
+    """Whole-block copies (src block of the src pools -> dst block of the dst
+    pools); either side may be a page-locked host tensor (pin_memory)."""
+    for t, n in ((dst_k, "dst_k"), (dst_v, "dst_v"), (src_k, "src_k"), (src_v, "src_v"),
+                 (block_pairs, "block_pairs")):
+        if not t.is_contiguous():
+            raise PagedKVError(_b.PKV_EINVAL, f"{n} must be contiguous")
+        if not t.is_cuda and not t.is_pinned():
+            raise PagedKVError(_b.PKV_EINVAL, f"{n} must be on the GPU or page-locked")
+    if block_pairs.dtype != torch.int32 or (block_pairs.numel() and block_pairs.shape[-1] != 2):
+        raise PagedKVError(_b.PKV_EINVAL, "block_pairs must be int32 [n, 2]")
+    if not (dst_k.dtype == dst_v.dtype == src_k.dtype == src_v.dtype):
+        raise PagedKVError(_b.PKV_EINVAL, "dtype mismatch")
+    Ns, Hkv, bs, D = src_k.shape
+    Nd = dst_k.shape[0]
+    if tuple(dst_k.shape[1:]) != (Hkv, bs, D):
+        raise PagedKVError(_b.PKV_EINVAL, "shape mismatch")
+    check(lib.pkv_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v),
+                              _ptr(block_pairs), block_pairs.numel() // 2, Ns, Nd, Hkv, D, bs,
+                              torch_dtype_code(src_k.dtype), _stream(stream)),
+          "pkv_swap_blocks")
+
+
 def pkv_device_status(clear: bool = False) -> int:
     """OR of PKV_DEV_* bits set on the current device (synchronises)."""
     flags = ctypes.c_uint(0)
@@ -201,16 +229,19 @@ class BlockAllocator:
     """Host block manager (pkv_alloc_*): free list, reference counts, fork and
     copy-on-write.  Not thread-safe."""
 
-    def __init__(self, num_blocks: int, block_size: int):
+    def __init__(self, num_blocks: int, block_size: int, num_host_blocks: int = 0):
         h = ctypes.c_void_p()
-        check(lib.pkv_alloc_create(num_blocks, block_size, ctypes.byref(h)), "pkv_alloc_create")
+        check(lib.pkv_alloc_create_swap(num_blocks, num_host_blocks, block_size,
+                                        ctypes.byref(h)), "pkv_alloc_create_swap")
         self._h = h
+        self._destroy = lib.pkv_alloc_destroy   # kept: module globals may be gone at exit
         self.num_blocks = num_blocks
+        self.num_host_blocks = num_host_blocks
         self.block_size = block_size
 
     def close(self):
         if getattr(self, "_h", None) is not None and self._h.value:
-            lib.pkv_alloc_destroy(self._h)
+            self._destroy(self._h)
             self._h = None
 
     def __del__(self):
@@ -251,8 +282,45 @@ class BlockAllocator:
     def free_seq(self, seq_id: int) -> int:
         return lib.pkv_alloc_free_seq(self._h, seq_id)
 
+    def _swap(self, fn, seq_id: int):
+        # size the pair buffer from the table length (a query that changes nothing)
+        n = ctypes.c_int(0)
+        st = lib.pkv_alloc_block_table(self._h, seq_id, None, 0, ctypes.byref(n))
+        if st not in (0, _b.PKV_EBOUNDS):
+            return st, []
+        buf = (ctypes.c_int32 * max(2 * n.value, 2))()
+        st = fn(self._h, seq_id, buf, n.value, ctypes.byref(n))
+        if st != 0:
+            return st, []
+        return st, [(buf[2 * i], buf[2 * i + 1]) for i in range(n.value)]
+
+    def swap_out(self, seq_id: int):
+        """-> (status, [(device block, host block), ...])"""
+        return self._swap(lib.pkv_alloc_swap_out, seq_id)
+
+    def swap_in(self, seq_id: int):
+        """-> (status, [(host block, device block), ...])"""
+        return self._swap(lib.pkv_alloc_swap_in, seq_id)
+
+    def slide_window(self, seq_id: int, window: int):
+        """-> (status, entries released)"""
+        n = ctypes.c_int(0)
+        st = lib.pkv_alloc_slide_window(self._h, seq_id, window, ctypes.byref(n))
+        return st, (n.value if st == 0 else 0)
+
+    def is_swapped(self, seq_id: int) -> bool:
+        v = ctypes.c_int(0)
+        check(lib.pkv_alloc_is_swapped(self._h, seq_id, ctypes.byref(v)), "pkv_alloc_is_swapped")
+        return bool(v.value)
+
     def apply(self, op):
         kind = op[0]
+        if kind == "swap_out":
+            return self.swap_out(op[1])
+        if kind == "swap_in":
+            return self.swap_in(op[1])
+        if kind == "slide":
+            return self.slide_window(op[1], op[2])
         if kind == "add":
             return self.add_seq(op[1], op[2])
         if kind == "fork":

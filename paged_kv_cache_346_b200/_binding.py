@@ -37,17 +37,24 @@ SIGNATURES = {
     "pkv_decode_default_partition": (_i32, [_i32, _i32, _i32]),
     "pkv_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "pkv_paged_attention_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
-                                          _i32, _i32, _i32, _i32, _i32, _f32, _i32, _i32, _vp,
-                                          _sz, _i32, _vp]),
+                                          _i32, _i32, _i32, _i32, _i32, _f32, _i32, _i32, _i32,
+                                          _vp, _sz, _i32, _vp]),
     "pkv_paged_attention_decode_static_ws": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                                     _i32, _i32, _i32, _i32, _i32, _i32, _i32,
-                                                    _f32, _i32, _i32, _i32, _vp]),
+                                                    _f32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_decode_schedule_order": (_i32, [_vp, _i32, _vp]),
     "pkv_kv_cache_append": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                    _vp]),
     "pkv_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
+    "pkv_swap_blocks": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+                               _i32, _vp]),
     "pkv_device_status": (_i32, [_c.POINTER(_c.c_uint), _i32]),
     "pkv_alloc_create": (_i32, [_i32, _i32, _c.POINTER(_vp)]),
+    "pkv_alloc_create_swap": (_i32, [_i32, _i32, _i32, _c.POINTER(_vp)]),
+    "pkv_alloc_swap_out": (_i32, [_vp, _i64, _vp, _i32, _c.POINTER(_i32)]),
+    "pkv_alloc_swap_in": (_i32, [_vp, _i64, _vp, _i32, _c.POINTER(_i32)]),
+    "pkv_alloc_is_swapped": (_i32, [_vp, _i64, _c.POINTER(_i32)]),
+    "pkv_alloc_slide_window": (_i32, [_vp, _i64, _i32, _c.POINTER(_i32)]),
     "pkv_alloc_destroy": (None, [_vp]),
     "pkv_alloc_add_seq": (_i32, [_vp, _i64, _i32]),
     "pkv_alloc_fork": (_i32, [_vp, _i64, _i64]),
@@ -87,7 +94,9 @@ class AllocStats(_c.Structure):
     _fields_ = [("num_blocks", _c.c_int32), ("block_size", _c.c_int32),
                 ("free_blocks", _c.c_int32), ("used_blocks", _c.c_int32),
                 ("shared_blocks", _c.c_int32), ("num_seqs", _c.c_int32),
-                ("refcount_sum", _c.c_int64), ("logical_tokens", _c.c_int64)]
+                ("refcount_sum", _c.c_int64), ("logical_tokens", _c.c_int64),
+                ("num_host_blocks", _c.c_int32), ("free_host_blocks", _c.c_int32),
+                ("swapped_seqs", _c.c_int32), ("reserved", _c.c_int32)]
 
     def as_dict(self) -> dict:
         return {f: getattr(self, f) for f, _ in self._fields_}

@@ -1,6 +1,7 @@
 // The C ABI of pagedkv (declared in include/pagedkv.h): host-side argument
 // checks, kernel selection and launches.  No call here allocates device
 // memory or synchronises, except pkv_device_status.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -48,6 +49,34 @@ int elem_size(pkv_dtype dt) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+
+// The address a kernel on the current device can use for p: device memory of
+// this device, managed memory, or page-locked host memory (through its mapped
+// view).  Pageable host memory and other devices' memory are refused.
+bool device_view(const void* p, void** out) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the error this query leaves behind
+        return false;
+    }
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    switch (at.type) {
+        case cudaMemoryTypeDevice:
+            if (at.device != dev) return false;
+            *out = at.devicePointer ? at.devicePointer : const_cast<void*>(p);
+            return true;
+        case cudaMemoryTypeManaged:
+            *out = at.devicePointer ? at.devicePointer : const_cast<void*>(p);
+            return true;
+        case cudaMemoryTypeHost:
+            if (!at.devicePointer) return false;
+            *out = at.devicePointer;
+            return true;
+        default:
+            return false;
+    }
+}
 
 constexpr int kNumSMs = 148;
 
@@ -110,15 +139,15 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
                                const int32_t* block_tables, const int32_t* context_lens,
                                const int32_t* seq_order, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                int block_size, int max_blocks_per_seq, int num_blocks,
-                               int max_context_len, float scale, pkv_dtype dtype,
-                               int partition_size, void* workspace, size_t workspace_bytes,
-                               pkv_kernel kernel, pkv_stream_t stream) {
+                               int max_context_len, float scale, int sliding_window,
+                               pkv_dtype dtype, int partition_size, void* workspace,
+                               size_t workspace_bytes, pkv_kernel kernel, pkv_stream_t stream) {
     // ---- host-side checks (nothing has been launched if these fail)
     const int es = elem_size(dtype);
     if (es == 0 || num_seqs < 0 || num_seqs > 65535 || num_q_heads <= 0 || num_kv_heads <= 0 ||
         num_q_heads % num_kv_heads != 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
         max_context_len < 0 || (int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size ||
-        !std::isfinite(scale) || partition_size < 0 ||
+        !std::isfinite(scale) || sliding_window < 0 || partition_size < 0 ||
         (partition_size != 0 && (partition_size % 64 != 0 || partition_size > 8192)))
         return PKV_EINVAL;
     if (kernel != PKV_KERNEL_AUTO && kernel != PKV_KERNEL_SIMT && kernel != PKV_KERNEL_MMA)
@@ -132,13 +161,18 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
         return PKV_EINVAL;
 
     const int G = num_q_heads / num_kv_heads;
+    // longest span a sequence attends to: with a window, at most the window
+    // plus the part of its first block ahead of it
+    const int span = sliding_window > 0
+                         ? (int)std::min<int64_t>(max_context_len,
+                                                  (int64_t)sliding_window + block_size - 1)
+                         : max_context_len;
     const int P = partition_size ? partition_size
-                                 : pkv_decode_default_partition(num_seqs, num_kv_heads,
-                                                                max_context_len);
-    const int np = max_context_len > 0 ? ceil_div(max_context_len, P) : 1;
+                                 : pkv_decode_default_partition(num_seqs, num_kv_heads, span);
+    const int np = span > 0 ? ceil_div(span, P) : 1;
     if (np > 1) {
         const size_t need = pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads,
-                                                      head_dim, max_context_len, P);
+                                                      head_dim, span, P);
         if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PKV_EINVAL;
     }
 
@@ -179,6 +213,8 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
     a.max_tokens = max_blocks_per_seq * block_size;
     a.partition_size = P;
     a.max_partitions = np;
+    a.block_size = block_size;
+    a.window = sliding_window;
     a.scale_log2 = scale * 1.4426950408889634f;
     if (status_word(&a.status) != cudaSuccess) return PKV_ECUDA;
 
@@ -234,6 +270,31 @@ int pkv_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_pairs, in
     if (status_word(&st) != cudaSuccess) return PKV_ECUDA;
     cudaError_t e = launch_copy_blocks(k_cache, v_cache, block_pairs, num_pairs, block_bytes,
                                        num_blocks, st, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+int pkv_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                    const int32_t* block_pairs, int num_pairs, int src_num_blocks,
+                    int dst_num_blocks, int num_kv_heads, int head_dim, int block_size,
+                    pkv_dtype dtype, pkv_stream_t stream) {
+    const int es = elem_size(dtype);
+    if (es == 0 || num_pairs < 0 || src_num_blocks <= 0 || dst_num_blocks <= 0 ||
+        num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
+        return PKV_EINVAL;
+    const int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * es;
+    if (block_bytes % 16 != 0) return PKV_EINVAL;
+    if (num_pairs == 0) return PKV_OK;
+    if (!dst_k || !dst_v || !src_k || !src_v || !block_pairs) return PKV_EINVAL;
+    void *dk, *dv, *sk, *sv, *pp;
+    if (!device_view(dst_k, &dk) || !device_view(dst_v, &dv) || !device_view(src_k, &sk) ||
+        !device_view(src_v, &sv) || !device_view(block_pairs, &pp))
+        return PKV_EINVAL;
+    if (!aligned16(dk) || !aligned16(dv) || !aligned16(sk) || !aligned16(sv)) return PKV_EINVAL;
+    unsigned int* st;
+    if (status_word(&st) != cudaSuccess) return PKV_ECUDA;
+    cudaError_t e = launch_swap_blocks(dk, dv, sk, sv, static_cast<const int32_t*>(pp), num_pairs,
+                                       block_bytes, src_num_blocks, dst_num_blocks, st,
+                                       reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
 

@@ -4,8 +4,11 @@
 // operation follows are stated next to the declarations in pagedkv.h.
 //
 // Data structures: a vector used as a stack of free block ids, a reference
-// count per block, and a hash map from sequence id to (block table, length).
-// Every operation either completes or leaves all three untouched.
+// count per block, and a hash map from sequence id to (block table, length,
+// swapped?).  An optional host pool (its own free stack) receives the blocks
+// of swapped-out sequences ("pagedattention vllm" §Memory Management:
+// swapping blocks to CPU memory).  Every operation either completes or
+// leaves all of it untouched.
 #include <cstdint>
 #include <new>
 #include <unordered_map>
@@ -16,12 +19,16 @@
 struct pkv_alloc {
     int32_t num_blocks;
     int32_t block_size;
-    std::vector<int32_t> free_stack;  // back() is handed out next
+    int32_t num_host_blocks = 0;
+    std::vector<int32_t> free_stack;       // back() is handed out next
+    std::vector<int32_t> host_free_stack;  // host pool, same discipline
     std::vector<int32_t> ref;
     struct Seq {
-        std::vector<int32_t> table;
+        std::vector<int32_t> table;  // device block ids, or host ids when swapped
         int64_t len;
+        bool swapped = false;
     };
+    int32_t swapped_seqs = 0;
     std::unordered_map<int64_t, Seq> seqs;
     int64_t refcount_sum = 0;
     int64_t logical_tokens = 0;
@@ -54,15 +61,20 @@ struct pkv_alloc {
 
 extern "C" {
 
-int pkv_alloc_create(int num_blocks, int block_size, pkv_alloc** out) {
-    if (!out || num_blocks <= 0 || block_size <= 0) return PKV_EINVAL;
+int pkv_alloc_create_swap(int num_blocks, int num_host_blocks, int block_size,
+                          pkv_alloc** out) {
+    if (!out || num_blocks <= 0 || num_host_blocks < 0 || block_size <= 0) return PKV_EINVAL;
     pkv_alloc* a = new (std::nothrow) pkv_alloc();
     if (!a) return PKV_ENOMEM;
     a->num_blocks = num_blocks;
+    a->num_host_blocks = num_host_blocks;
     a->block_size = block_size;
     try {
         a->free_stack.resize(num_blocks);
         for (int32_t i = 0; i < num_blocks; ++i) a->free_stack[i] = num_blocks - 1 - i;
+        a->host_free_stack.resize(num_host_blocks);
+        for (int32_t i = 0; i < num_host_blocks; ++i)
+            a->host_free_stack[i] = num_host_blocks - 1 - i;
         a->ref.assign(num_blocks, 0);
     } catch (...) {
         delete a;
@@ -70,6 +82,10 @@ int pkv_alloc_create(int num_blocks, int block_size, pkv_alloc** out) {
     }
     *out = a;
     return PKV_OK;
+}
+
+int pkv_alloc_create(int num_blocks, int block_size, pkv_alloc** out) {
+    return pkv_alloc_create_swap(num_blocks, 0, block_size, out);
 }
 
 void pkv_alloc_destroy(pkv_alloc* a) { delete a; }
@@ -93,8 +109,10 @@ int pkv_alloc_fork(pkv_alloc* a, int64_t parent, int64_t child) {
     auto it = a->seqs.find(parent);
     if (it == a->seqs.end()) return PKV_ENOSEQ;
     if (a->seqs.count(child)) return PKV_EEXIST;
+    if (it->second.swapped) return PKV_EINVAL;
     pkv_alloc::Seq s = it->second;  // copy of table and length
-    for (int32_t b : s.table) a->add_ref(b);
+    for (int32_t b : s.table)
+        if (b >= 0) a->add_ref(b);
     a->logical_tokens += s.len;
     a->seqs.emplace(child, std::move(s));
     return PKV_OK;
@@ -106,6 +124,7 @@ int pkv_alloc_append_slot(pkv_alloc* a, int64_t seq_id, int64_t* slot, int32_t* 
     auto it = a->seqs.find(seq_id);
     if (it == a->seqs.end()) return PKV_ENOSEQ;
     pkv_alloc::Seq& s = it->second;
+    if (s.swapped) return PKV_EINVAL;
     const int64_t off = s.len % a->block_size;
     int32_t src = -1, dst = -1;
     if (off == 0) {
@@ -151,7 +170,14 @@ int pkv_alloc_free_seq(pkv_alloc* a, int64_t seq_id) {
     if (!a) return PKV_EINVAL;
     auto it = a->seqs.find(seq_id);
     if (it == a->seqs.end()) return PKV_ENOSEQ;
-    for (int32_t b : it->second.table) a->drop_ref(b);
+    if (it->second.swapped) {
+        for (int32_t h : it->second.table)
+            if (h >= 0) a->host_free_stack.push_back(h);
+        --a->swapped_seqs;
+    } else {
+        for (int32_t b : it->second.table)
+            if (b >= 0) a->drop_ref(b);
+    }
     a->logical_tokens -= it->second.len;
     a->seqs.erase(it);
     return PKV_OK;
@@ -186,6 +212,7 @@ int pkv_alloc_build_block_tables(const pkv_alloc* a, const int64_t* seq_ids, int
     for (int i = 0; i < n; ++i) {  // check everything before writing anything
         auto it = a->seqs.find(seq_ids[i]);
         if (it == a->seqs.end()) return PKV_ENOSEQ;
+        if (it->second.swapped) return PKV_EINVAL;
         if ((int64_t)it->second.table.size() > max_blocks) return PKV_EBOUNDS;
     }
     for (int i = 0; i < n; ++i) {
@@ -206,8 +233,92 @@ int pkv_alloc_refcount(const pkv_alloc* a, int32_t block, int* out) {
     return PKV_OK;
 }
 
+int pkv_alloc_swap_out(pkv_alloc* a, int64_t seq_id, int32_t* pairs, int capacity,
+                       int* num_pairs) {
+    if (!a || !num_pairs || capacity < 0 || (capacity > 0 && !pairs)) return PKV_EINVAL;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PKV_ENOSEQ;
+    pkv_alloc::Seq& s = it->second;
+    if (s.swapped) return PKV_EINVAL;
+    int n = 0;
+    for (int32_t b : s.table) n += b >= 0;  // entries released by a sliding window stay -1
+    *num_pairs = n;
+    if (n > capacity) return PKV_EBOUNDS;
+    if (n > (int)a->host_free_stack.size()) return PKV_ENOMEM;
+    int k = 0;
+    for (int32_t& b : s.table) {
+        if (b < 0) continue;
+        const int32_t h = a->host_free_stack.back();
+        a->host_free_stack.pop_back();
+        pairs[2 * k] = b;
+        pairs[2 * k + 1] = h;
+        ++k;
+        a->drop_ref(b);  // other holders keep a shared block on the device
+        b = h;
+    }
+    s.swapped = true;
+    ++a->swapped_seqs;
+    return PKV_OK;
+}
+
+int pkv_alloc_swap_in(pkv_alloc* a, int64_t seq_id, int32_t* pairs, int capacity,
+                      int* num_pairs) {
+    if (!a || !num_pairs || capacity < 0 || (capacity > 0 && !pairs)) return PKV_EINVAL;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PKV_ENOSEQ;
+    pkv_alloc::Seq& s = it->second;
+    if (!s.swapped) return PKV_EINVAL;
+    int n = 0;
+    for (int32_t h : s.table) n += h >= 0;
+    *num_pairs = n;
+    if (n > capacity) return PKV_EBOUNDS;
+    if (n > (int)a->free_stack.size()) return PKV_ENOMEM;
+    int k = 0;
+    for (int32_t& h : s.table) {
+        if (h < 0) continue;
+        const int32_t d = a->take();
+        pairs[2 * k] = h;
+        pairs[2 * k + 1] = d;
+        ++k;
+        a->host_free_stack.push_back(h);
+        h = d;
+    }
+    s.swapped = false;
+    --a->swapped_seqs;
+    return PKV_OK;
+}
+
+int pkv_alloc_slide_window(pkv_alloc* a, int64_t seq_id, int window, int* released) {
+    if (!a || !released || window <= 0) return PKV_EINVAL;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PKV_ENOSEQ;
+    pkv_alloc::Seq& s = it->second;
+    if (s.swapped) return PKV_EINVAL;
+    *released = 0;
+    // block j holds tokens [j*bs, (j+1)*bs): gone once (j+1)*bs <= len - window
+    const int64_t keep_from = s.len - window;
+    for (size_t j = 0; j < s.table.size() && (int64_t)(j + 1) * a->block_size <= keep_from; ++j) {
+        if (s.table[j] < 0) continue;
+        a->drop_ref(s.table[j]);
+        s.table[j] = -1;
+        ++*released;
+    }
+    return PKV_OK;
+}
+
+int pkv_alloc_is_swapped(const pkv_alloc* a, int64_t seq_id, int* swapped) {
+    if (!a || !swapped) return PKV_EINVAL;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PKV_ENOSEQ;
+    *swapped = it->second.swapped ? 1 : 0;
+    return PKV_OK;
+}
+
 int pkv_alloc_stats(const pkv_alloc* a, pkv_alloc_stats_t* out) {
     if (!a || !out) return PKV_EINVAL;
+    out->num_host_blocks = a->num_host_blocks;
+    out->free_host_blocks = (int32_t)a->host_free_stack.size();
+    out->swapped_seqs = a->swapped_seqs;
     out->num_blocks = a->num_blocks;
     out->block_size = a->block_size;
     out->free_blocks = (int32_t)a->free_stack.size();

@@ -1,7 +1,7 @@
-// KV append (slot-mapping scatter) and copy-on-write block copies.
+// KV append (slot-mapping scatter), copy-on-write block copies and swapping.
 //
-// Both are pure bit moves bound by HBM bandwidth: 16-byte vector loads and
-// stores, several in flight per thread, no shared memory.
+// All are pure bit moves bound by HBM (or host-link) bandwidth: 16-byte vector
+// loads and stores, several in flight per thread, no shared memory.
 #include "cache_ops.cuh"
 
 namespace pkv {
@@ -41,26 +41,31 @@ __global__ void __launch_bounds__(256) kv_append_kernel(uint4* __restrict__ kc,
     }
 }
 
-// Grid (chunks, pairs, 2): blockIdx.z picks K or V.  Each thread moves UNROLL
-// vectors per pass with all loads issued before the stores.
+// Whole-page moves, shared by the copy-on-write copies (within one pool) and
+// swapping (between a device pool and a page-locked host pool).  Grid
+// (chunks, pairs, 2): blockIdx.z picks K or V; each thread keeps UNROLL
+// 16-byte loads in flight before its stores.  The source and destination
+// pools may be the same buffer (different blocks), so no pointer is declared
+// restrict.
 template <int UNROLL>
-__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ kc,
-                                                           uint4* __restrict__ vc,
-                                                           const int32_t* __restrict__ pairs,
-                                                           int num_pairs, int64_t block_vecs,
-                                                           int num_blocks,
-                                                           unsigned int* status) {
-    uint4* base = blockIdx.z ? vc : kc;
+__global__ void __launch_bounds__(256) move_pages_kernel(uint4* dk, uint4* dv, const uint4* sk,
+                                                          const uint4* sv,
+                                                          const int32_t* __restrict__ pairs,
+                                                          int num_pairs, int64_t block_vecs,
+                                                          int src_blocks, int dst_blocks,
+                                                          unsigned int* status) {
+    uint4* dbase = blockIdx.z ? dv : dk;
+    const uint4* sbase = blockIdx.z ? sv : sk;
     for (int pr = blockIdx.y; pr < num_pairs; pr += gridDim.y) {
         const int32_t src = pairs[2 * pr];
         const int32_t dst = pairs[2 * pr + 1];
-        if ((unsigned)src >= (unsigned)num_blocks || (unsigned)dst >= (unsigned)num_blocks) {
+        if ((unsigned)src >= (unsigned)src_blocks || (unsigned)dst >= (unsigned)dst_blocks) {
             if (blockIdx.x == 0 && blockIdx.z == 0 && threadIdx.x == 0)
                 flag(status, PKV_DEV_BAD_BLOCK);
             continue;
         }
-        const uint4* s = base + (int64_t)src * block_vecs;
-        uint4* d = base + (int64_t)dst * block_vecs;
+        const uint4* s = sbase + (int64_t)src * block_vecs;
+        uint4* d = dbase + (int64_t)dst * block_vecs;
         const int64_t step = (int64_t)gridDim.x * blockDim.x * UNROLL;
         for (int64_t i0 = ((int64_t)blockIdx.x * blockDim.x) * UNROLL + threadIdx.x;
              i0 < block_vecs; i0 += step) {
@@ -77,6 +82,33 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ kc
             }
         }
     }
+}
+
+template <int UNROLL>
+static cudaError_t launch_move_pages(void* dk, void* dv, const void* sk, const void* sv,
+                                     const int32_t* pairs, int num_pairs, int64_t block_bytes,
+                                     int src_blocks, int dst_blocks, unsigned int* status,
+                                     cudaStream_t stream) {
+    if (num_pairs == 0) return cudaSuccess;
+    const int64_t block_vecs = block_bytes / 16;
+    int64_t chunks = (block_vecs + 256 * UNROLL - 1) / (256 * UNROLL);
+    if (chunks > 1024) chunks = 1024;
+    const int ys = num_pairs < 65535 ? num_pairs : 65535;
+    dim3 grid((unsigned)chunks, (unsigned)ys, 2);
+    move_pages_kernel<UNROLL><<<grid, 256, 0, stream>>>(
+        static_cast<uint4*>(dk), static_cast<uint4*>(dv), static_cast<const uint4*>(sk),
+        static_cast<const uint4*>(sv), pairs, num_pairs, block_vecs, src_blocks, dst_blocks,
+        status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                               const int32_t* pairs, int num_pairs, int64_t block_bytes,
+                               int src_blocks, int dst_blocks, unsigned int* status,
+                               cudaStream_t stream) {
+    // more loads in flight: one side sits behind the host link
+    return launch_move_pages<8>(dst_k, dst_v, src_k, src_v, pairs, num_pairs, block_bytes,
+                                src_blocks, dst_blocks, status, stream);
 }
 
 cudaError_t launch_kv_append(void* k_cache, void* v_cache, const void* k, const void* v,
@@ -99,17 +131,8 @@ cudaError_t launch_kv_append(void* k_cache, void* v_cache, const void* k, const 
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs,
                                int num_pairs, int64_t block_bytes, int num_blocks,
                                unsigned int* status, cudaStream_t stream) {
-    if (num_pairs == 0) return cudaSuccess;
-    constexpr int UNROLL = 4;
-    const int64_t block_vecs = block_bytes / 16;
-    int64_t chunks = (block_vecs + 256 * UNROLL - 1) / (256 * UNROLL);
-    if (chunks > 1024) chunks = 1024;
-    const int ys = num_pairs < 65535 ? num_pairs : 65535;
-    dim3 grid((unsigned)chunks, (unsigned)ys, 2);
-    copy_blocks_kernel<UNROLL><<<grid, 256, 0, stream>>>(
-        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, num_pairs,
-        block_vecs, num_blocks, status);
-    return cudaGetLastError();
+    return launch_move_pages<4>(k_cache, v_cache, k_cache, v_cache, pairs, num_pairs,
+                                block_bytes, num_blocks, num_blocks, status, stream);
 }
 
 }  // namespace pkv

@@ -16,4 +16,10 @@ cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int32_t* pair
                                int num_pairs, int64_t block_bytes, int num_blocks,
                                unsigned int* status, cudaStream_t stream);
 
+// Pages between two pools (device or page-locked host, as device views).
+cudaError_t launch_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                               const int32_t* pairs, int num_pairs, int64_t block_bytes,
+                               int src_blocks, int dst_blocks, unsigned int* status,
+                               cudaStream_t stream);
+
 }  // namespace pkv

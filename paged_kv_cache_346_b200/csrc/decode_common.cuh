@@ -30,7 +30,9 @@ struct DecodeArgs {
     int num_blocks;
     int max_tokens;               // max_blocks_per_seq * BS
     int partition_size;           // tokens per partition
-    int max_partitions;           // grid.x = ceil(max_context_len / partition_size)
+    int max_partitions;           // grid.x = ceil(longest attended span / partition_size)
+    int block_size;
+    int window;                   // sliding window in tokens, 0 = attend to the whole context
     float scale_log2;             // scale * log2(e): logits are kept in base 2
 };
 
@@ -57,13 +59,30 @@ __device__ __forceinline__ int seq_len(const DecodeArgs& a, int b, bool report) 
     return L;
 }
 
-__device__ __forceinline__ int num_partitions(const DecodeArgs& a, int L, bool report) {
-    int n = (L + a.partition_size - 1) / a.partition_size;
+// The tokens a sequence attends to and how they are cut into partitions.
+// Without a window: [0, L).  With a window of W tokens: [lo, L), lo =
+// max(0, L - W) ("pagedattention vllm" §Advanced Features: sliding-window
+// models keep only the recent blocks); the partitions then start at the
+// block holding lo (base), and the first lo - base tokens are masked.
+struct Span {
+    int L;     // sequence length
+    int lo;    // first attended token
+    int base;  // first token of partition 0 (block aligned)
+    int np;    // partitions
+};
+
+__device__ __forceinline__ Span seq_span(const DecodeArgs& a, int b, bool report) {
+    Span sp;
+    sp.L = seq_len(a, b, report);
+    sp.lo = (a.window > 0 && sp.L > a.window) ? sp.L - a.window : 0;
+    sp.base = sp.lo - sp.lo % a.block_size;
+    int n = (sp.L - sp.base + a.partition_size - 1) / a.partition_size;
     if (n > a.max_partitions) {
         if (report) flag(a.status, PKV_DEV_BAD_LEN);
         n = a.max_partitions;
     }
-    return n;
+    sp.np = n;
+    return sp;
 }
 
 // The table slice of a partition goes to shared memory.  For partition 0 (the
@@ -79,7 +98,10 @@ struct TablePrefetch {
 
 __device__ __forceinline__ TablePrefetch table_prefetch(const DecodeArgs& a, int b, int part,
                                                         int blocks_per_part, int tid) {
-    TablePrefetch pf{0, part == 0 && tid < blocks_per_part && tid < a.max_blocks_per_seq};
+    // (with a sliding window partition 0 starts at a block known only after
+    // the length is read: no early read then)
+    TablePrefetch pf{0, part == 0 && a.window == 0 && tid < blocks_per_part &&
+                            tid < a.max_blocks_per_seq};
     if (pf.ok) pf.v = a.block_tables[(int64_t)b * a.max_blocks_per_seq + tid];
     return pf;
 }
@@ -203,8 +225,7 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
     pdl_wait_primary();
     const int h = blockIdx.x;
     const int b = blockIdx.y;
-    const int L = seq_len(a, b, false);
-    const int np = num_partitions(a, L, false);
+    const int np = seq_span(a, b, false).np;
     if (np <= 1) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row = (int64_t)b * a.num_q_heads + h;

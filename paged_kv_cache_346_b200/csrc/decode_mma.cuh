@@ -141,8 +141,8 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     if (b < 0) return;
 
     const TablePrefetch pf = table_prefetch(a, b, part, a.partition_size / BS, tid);
-    const int L = seq_len(a, b, reporter);
-    const int np = num_partitions(a, L, reporter);
+    const Span sp = seq_span(a, b, reporter);
+    const int L = sp.L, np = sp.np;
     T* out = reinterpret_cast<T*>(a.out);
     if (L == 0) {
         if (part == 0)
@@ -153,8 +153,9 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     if (part >= np) return;
 
     const int P = a.partition_size;
-    const int t0 = part * P;
+    const int t0 = sp.base + part * P;
     const int ntok = min(L, t0 + P) - t0;
+    const int mask_lo = part == 0 ? sp.lo - sp.base : 0;  // tokens ahead of the window
     const int ntiles = (ntok + TILE - 1) / TILE;
     const int nblk = (ntok + BS - 1) / BS;
 
@@ -241,7 +242,8 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         const bool ok = mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status);
         if (!ok) s_abort = 1;
         const int wvalid = ntok - (it * TILE + warp * 16);
-        const bool work = ok && wvalid > 0;
+        const int wlo = mask_lo - (it * TILE + warp * 16);
+        const bool work = ok && wvalid > 0 && wlo < 16 && wlo < wvalid;
         const int tt0 = warp * 16;           // first token of the warp in the stage
         const int jw = tt0 / BS;             // its block within the stage
         const int rr = tt0 % BS + lrow;      // this lane's row within that block
@@ -288,7 +290,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int tok = nt * 8 + 2 * t4 + (i & 1);
-                    s[nt][i] = tok < wvalid ? s[nt][i] * a.scale_log2 : -INFINITY;
+                    s[nt][i] = (tok >= wlo && tok < wvalid) ? s[nt][i] * a.scale_log2 : -INFINITY;
                 }
             uint32_t pb[RB][2];
             float alpha_c[RB][2];
@@ -317,7 +319,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                 alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
             }
             // O^T += V^T P^T
-            const bool partial = wvalid < 16;
+            const bool partial = wvalid < 16 || wlo > 0;
 #pragma unroll
             for (int mt = 0; mt < KSTEPS; ++mt) {
                 uint32_t va[4];
@@ -328,12 +330,13 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                     ldsm_x4_trans(kaddr(mt) + STAGE_BYTES, va);
                 }
                 if (partial) {
-                    // zero values of tokens past the end (0 * NaN would poison)
+                    // zero values of masked tokens (0 * NaN would poison)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int tk = (i >> 1) * 8 + 2 * t4;
-                        const uint32_t keep = (tk < wvalid ? 0x0000ffffu : 0u) |
-                                              (tk + 1 < wvalid ? 0xffff0000u : 0u);
+                        const uint32_t keep =
+                            (tk >= wlo && tk < wvalid ? 0x0000ffffu : 0u) |
+                            (tk + 1 >= wlo && tk + 1 < wvalid ? 0xffff0000u : 0u);
                         va[i] &= keep;
                     }
                 }

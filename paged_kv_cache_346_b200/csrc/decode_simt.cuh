@@ -152,9 +152,10 @@ struct SimtWarp {
         }
     }
 
-    // The fetched 16 tokens, the first `wvalid` of them inside the sequence.
+    // The fetched 16 tokens; tokens [wlo, wvalid) of them are attended to
+    // (before wlo: ahead of a sliding window; from wvalid: past the end).
     // s_p: this warp's [HG][16] weight scratch.
-    __device__ __forceinline__ void compute(int wvalid, float (*s_p)[16]) {
+    __device__ __forceinline__ void compute(int wlo, int wvalid, float (*s_p)[16]) {
         float s[HG][4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -176,7 +177,7 @@ struct SimtWarp {
                 d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 1);
                 d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 2);
                 d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 4);
-                s[hh][r] = tok < wvalid ? d[hh] : -INFINITY;
+                s[hh][r] = (tok >= wlo && tok < wvalid) ? d[hh] : -INFINITY;
             }
         }
 #pragma unroll
@@ -184,7 +185,7 @@ struct SimtWarp {
             float mx = fmaxf(fmaxf(s[hh][0], s[hh][1]), fmaxf(s[hh][2], s[hh][3]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            const float mnew = fmaxf(m[hh], mx);  // finite: wvalid > 0
+            const float mnew = fmaxf(m[hh], mx);  // finite: one token is attended to
             const float alpha = exp2f(m[hh] - mnew);
             float ps = 0.f;
 #pragma unroll
@@ -209,7 +210,7 @@ struct SimtWarp {
 #pragma unroll
         for (int j = 0; j < NTV; ++j) {
             const int t = tv + j * TPV;
-            if (t < wvalid) {  // values past the end are never used (they may be NaN)
+            if (t >= wlo && t < wvalid) {  // masked values are never used (they may be NaN)
 #pragma unroll
                 for (int c = 0; c < CPV; ++c) {
                     float vf[EPC];
@@ -288,8 +289,8 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREAD
     if (b < 0) return;
 
     const TablePrefetch pf = table_prefetch(a, b, part, a.partition_size / BS, tid);
-    const int L = seq_len(a, b, reporter);
-    const int np = num_partitions(a, L, reporter);
+    const Span sp = seq_span(a, b, reporter);
+    const int L = sp.L, np = sp.np;
     if (L == 0) {  // empty sequence: a zero row
         if (part == 0) {
             T* out = reinterpret_cast<T*>(a.out);
@@ -301,8 +302,9 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREAD
     if (part >= np) return;
 
     const int P = a.partition_size;
-    const int t0 = part * P;
+    const int t0 = sp.base + part * P;
     const int ntok = min(L, t0 + P) - t0;
+    const int mask_lo = part == 0 ? sp.lo - sp.base : 0;  // tokens ahead of the window
     const int ntiles = (ntok + TILE - 1) / TILE;
     const int nblk = (ntok + BS - 1) / BS;
 
@@ -381,11 +383,13 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREAD
         if (!mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status)) s_abort = 1;
         if (WS && s_abort) break;
         const int wvalid = ntok - (it * TILE + warp * 16);  // tokens this warp owns
-        if (!s_abort && wvalid > 0) {
+        const int wlo = mask_lo - (it * TILE + warp * 16);
+        const bool work = wvalid > 0 && wlo < 16 && wlo < wvalid;
+        if (!s_abort && work) {
             const unsigned char* Kw = s_kv + stage * 2 * STAGE_BYTES + warp * 16 * ROW;
             W.fetch(Kw, Kw + STAGE_BYTES);
         }
-        if (!W.EARLY && !s_abort && wvalid > 0) W.compute(wvalid, s_p[warp]);
+        if (!W.EARLY && !s_abort && work) W.compute(wlo, wvalid, s_p[warp]);
         // the stage's data is in registers (or used): hand the stage back
         if (WS) {
             __syncwarp();
@@ -395,7 +399,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREAD
             if (s_abort) break;
             if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage, pol);
         }
-        if (W.EARLY && wvalid > 0) W.compute(wvalid, s_p[warp]);
+        if (W.EARLY && work) W.compute(wlo, wvalid, s_p[warp]);
     }
     if (WS) __syncthreads();  // producer and consumers: every stage consumed
     if (s_abort) return;

@@ -48,10 +48,15 @@ extern "C" int pkv_paged_attention_decode_static_ws(
     void* out, const void* q, const void* k_cache, const void* v_cache,
     const int32_t* block_tables, const int32_t* context_lens, const int32_t* seq_order,
     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-    int max_blocks_per_seq, int num_blocks, int max_context_len, float scale, pkv_dtype dtype,
-    int partition_size, pkv_kernel kernel, pkv_stream_t stream) {
+    int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+    int sliding_window, pkv_dtype dtype, int partition_size, pkv_kernel kernel,
+    pkv_stream_t stream) {
+    const int64_t span = sliding_window > 0 && (int64_t)sliding_window + block_size - 1 <
+                                                   (int64_t)max_context_len
+                             ? (int64_t)sliding_window + block_size - 1
+                             : (int64_t)max_context_len;
     const size_t need = pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
-                                                  max_context_len, partition_size);
+                                                  (int)span, partition_size);
     if (need > (size_t)PKV_STATIC_WORKSPACE_BYTES) return PKV_EBOUNDS;
     void* ws = nullptr;
     if (need > 0) {
@@ -64,6 +69,6 @@ extern "C" int pkv_paged_attention_decode_static_ws(
     return pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
                                       seq_order, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                       max_blocks_per_seq, num_blocks, max_context_len, scale,
-                                      dtype, partition_size, ws,
+                                      sliding_window, dtype, partition_size, ws,
                                       ws ? (size_t)PKV_STATIC_WORKSPACE_BYTES : 0, kernel, stream);
 }

@@ -30,18 +30,20 @@ class DeviceInputs:
         self.out = torch.empty_like(self.q)
 
     def decode(self, partition_size=0, kernel=pkv.PKV_KERNEL_AUTO, max_context_len=None,
-               fill_out=None, seq_order=None):
+               fill_out=None, seq_order=None, sliding_window=0):
         c = self.inp.cfg
         mcl = self.inp.max_context_len if max_context_len is None else max_context_len
+        span = min(mcl, sliding_window + c.block_size - 1) if sliding_window > 0 else mcl
         ws_bytes = pkv.pkv_decode_workspace_size(c.num_seqs, c.num_q_heads, c.num_kv_heads,
-                                                 c.head_dim, mcl, partition_size)
+                                                 c.head_dim, span, partition_size)
         ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
         if fill_out is not None:
             self.out.fill_(fill_out)
         pkv.pkv_paged_attention_decode(self.out, self.q, self.k, self.v, self.bt, self.cl,
                                        c.scale, c.block_size, mcl,
                                        partition_size=partition_size, workspace=ws,
-                                       seq_order=seq_order, kernel=kernel)
+                                       seq_order=seq_order, sliding_window=sliding_window,
+                                       kernel=kernel)
         torch.cuda.synchronize()
         return self.out
 

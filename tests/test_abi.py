@@ -37,12 +37,12 @@ def test_status_strings_and_version():
 
 def _decode(**over):
     a = dict(out=None, q=None, k=None, v=None, bt=None, cl=None, order=None, B=4, Hq=8, Hkv=2, D=128,
-             bs=16, mb=8, N=64, maxlen=100, scale=0.1, dt=b.PKV_F16, P=0, ws=None, wsb=0,
+             bs=16, mb=8, N=64, maxlen=100, scale=0.1, win=0, dt=b.PKV_F16, P=0, ws=None, wsb=0,
              kern=0, stream=None)
     a.update(over)
     return b.lib.pkv_paged_attention_decode(
         a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["order"], a["B"], a["Hq"], a["Hkv"], a["D"],
-        a["bs"], a["mb"], a["N"], a["maxlen"], a["scale"], a["dt"], a["P"], a["ws"], a["wsb"],
+        a["bs"], a["mb"], a["N"], a["maxlen"], a["scale"], a["win"], a["dt"], a["P"], a["ws"], a["wsb"],
         a["kern"], a["stream"])
 
 
@@ -53,6 +53,7 @@ def _decode(**over):
     (dict(P=100), b.PKV_EINVAL),                        # not a multiple of 64
     (dict(P=16384), b.PKV_EINVAL),
     (dict(scale=float("nan")), b.PKV_EINVAL),
+    (dict(win=-1), b.PKV_EINVAL),
     (dict(dt=7), b.PKV_EINVAL),
     (dict(kern=9), b.PKV_EINVAL),
     (dict(D=96), b.PKV_EUNSUPPORTED),

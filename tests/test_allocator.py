@@ -95,3 +95,37 @@ def test_cow_sampling_setup_matches_model():
     # per prompt: samples - 1 copies of the shared partial block
     assert st["used_blocks"] == sum(int(np.ceil(L / bs)) for L in rec.shared_lens) + \
         rec.num_prompts * (rec.samples - 1)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_scripts_with_swapping_bit_exact(seed):
+    nat = BlockAllocator(40, 4, num_host_blocks=30)
+    mod = bm.BlockManagerModel(40, 4, num_host_blocks=30)
+    for i, op in enumerate(random_alloc_ops(seed, 400, max_len=50, swap=True)):
+        r_nat, r_mod = nat.apply(op), mod.apply(op)
+        assert r_nat == r_mod, (i, op, r_nat, r_mod)
+        if i % 20 == 0:
+            same_state(nat, mod)
+            for sid in mod.tables:
+                assert nat.is_swapped(sid) == (sid in mod.swapped)
+    same_state(nat, mod)
+
+
+def test_swapped_sequence_cannot_join_a_decode_batch():
+    nat = BlockAllocator(8, 4, num_host_blocks=8)
+    nat.add_seq(0, 5)
+    assert nat.swap_out(0)[0] == 0
+    with pytest.raises(Exception):
+        nat.build_block_tables([0], max_blocks=4)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_scripts_with_windows_bit_exact(seed):
+    nat = BlockAllocator(40, 4, num_host_blocks=30)
+    mod = bm.BlockManagerModel(40, 4, num_host_blocks=30)
+    for i, op in enumerate(random_alloc_ops(seed, 400, max_len=50, swap=True, slide=True)):
+        r_nat, r_mod = nat.apply(op), mod.apply(op)
+        assert r_nat == r_mod, (i, op, r_nat, r_mod)
+        if i % 20 == 0:
+            same_state(nat, mod)
+    same_state(nat, mod)

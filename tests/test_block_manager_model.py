@@ -21,8 +21,9 @@ def check_invariants(m: bm.BlockManagerModel):
     held = []
     for sid, table in m.tables.items():
         # a sequence holds the blocks it filled plus part of the last one
+        # (entries released by a sliding window are -1)
         assert len(table) == (m.lens[sid] + bs - 1) // bs
-        held.extend(table)
+        held.extend(b for b in table if b >= 0)
     assert sum(m.ref) == len(held)                        # one reference per table entry
     for blk in range(m.num_blocks):
         assert m.ref[blk] == held.count(blk)
@@ -160,3 +161,67 @@ def test_copy_on_write_on_data_matches_private_history():
             logits = 0.5 * ks[:, h] @ q[i, h].astype(np.float64)
             w = np.exp(logits - logits.max())
             np.testing.assert_allclose(out[i, h], (w @ vs[:, h]) / w.sum(), rtol=0, atol=1e-12)
+
+
+def check_swap_invariants(m: bm.BlockManagerModel):
+    bs = m.block_size
+    resident, host = [], []
+    for sid, table in m.tables.items():
+        assert len(table) == (m.lens[sid] + bs - 1) // bs
+        (host if sid in m.swapped else resident).extend(b for b in table if b >= 0)
+    assert sum(m.ref) == len(resident)
+    assert len(set(host)) == len(host)                       # host blocks are never shared
+    assert set(host).isdisjoint(m.host_free)
+    assert len(host) + len(m.host_free) == m.num_host_blocks
+    assert set(m.free).isdisjoint(resident)
+    assert len(m.free) + len(set(resident)) == m.num_blocks
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_scripts_with_swapping_keep_invariants(seed):
+    m = bm.BlockManagerModel(num_blocks=40, block_size=4, num_host_blocks=30)
+    for op in random_alloc_ops(seed, 400, max_len=50, swap=True):
+        m.apply(op)
+        check_swap_invariants(m)
+
+
+def test_swap_rules():
+    m = bm.BlockManagerModel(8, 4, num_host_blocks=4)
+    m.add_seq(0, 6)                                   # blocks [0, 1]
+    m.fork(0, 1)                                      # shared
+    st, pairs = m.swap_out(1)
+    assert st == bm.OK and pairs == [(0, 0), (1, 1)]
+    assert m.refcount(0) == 1 and m.refcount(1) == 1  # still held by seq 0
+    assert m.block_table(1) == [0, 1]                 # now host ids
+    assert m.append_slot(1)[0] == bm.EINVAL and m.fork(1, 2) == bm.EINVAL
+    assert m.swap_out(1)[0] == bm.EINVAL
+    st, pairs = m.swap_in(1)
+    assert st == bm.OK and pairs == [(0, 2), (1, 3)]  # fresh device blocks
+    assert m.host_free_list() == [1, 0, 2, 3]
+    m.add_seq(5, 16)                                  # 4 blocks: device now full but two
+    assert m.swap_out(5)[0] == bm.OK
+    assert m.swap_out(0)[0] == bm.ENOMEM              # host pool exhausted: nothing changes
+    assert 0 not in m.swapped and m.block_table(0) == [0, 1]
+    assert m.free_seq(5) == bm.OK and m.stats()["free_host_blocks"] == 4
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_scripts_with_windows_and_swapping_keep_invariants(seed):
+    m = bm.BlockManagerModel(num_blocks=40, block_size=4, num_host_blocks=30)
+    for op in random_alloc_ops(seed, 400, max_len=50, swap=True, slide=True):
+        m.apply(op)
+        check_swap_invariants(m)
+
+
+def test_slide_window_rules():
+    m = bm.BlockManagerModel(16, 4)
+    m.add_seq(0, 18)                                  # blocks 0..4, last one half full
+    m.fork(0, 1)
+    assert m.slide_window(0, 7) == (bm.OK, 2)         # tokens 0..10 gone: blocks 0, 1
+    assert m.block_table(0) == [-1, -1, 2, 3, 4]
+    assert m.refcount(0) == 1 and m.refcount(1) == 1  # still held by the fork
+    assert m.slide_window(0, 7) == (bm.OK, 0)         # idempotent
+    assert m.slide_window(0, 1) == (bm.OK, 2)         # keep only the last token's block
+    assert m.slide_window(0, 0)[0] == bm.EINVAL
+    m.free_seq(1)
+    assert m.free_list()[:4] == [3, 2, 1, 0]          # freed once their last holder left

@@ -244,3 +244,44 @@ def test_bad_schedule_order_entry_is_flagged():
     pkv.pkv_device_status(clear=True)
     dev.decode(seq_order=torch.tensor([1, 7], dtype=torch.int32, device="cuda"))
     assert pkv.pkv_device_status(clear=True) & pkv.PKV_DEV_BAD_ORDER
+
+
+
+# ---------------------------------------------------------------------------
+# sliding window
+
+@pytest.mark.parametrize("dtype,G", [("f16", 1), ("bf16", 8), ("f32", 1), ("bf16", 4)])
+@pytest.mark.parametrize("W", [1, 15, 16, 17, 100, 600, 5000])
+def test_sliding_window(dtype, G, W):
+    D = 128 if dtype != "f32" else 64
+    cfg = _cfg(dtype, 2 * G, 2, D, 16, RAGGED)
+    inp = make_decode_inputs(cfg, seed=50 + G)
+    ref = oracle.paged_decode_inputs(inp, window=W)
+    dev = DeviceInputs(inp)
+    for kern in _kernels_for(dtype, G):
+        for P in (0, 64):
+            got = to_f64(dev.decode(partition_size=P, kernel=kern, sliding_window=W,
+                                    fill_out=7.0))
+            assert_close(got, ref, dtype, f"{dtype} G={G} W={W} P={P} kernel={kern}")
+
+
+@pytest.mark.parametrize("dtype,G", [("f16", 1), ("bf16", 8)])
+def test_sliding_window_released_blocks_are_never_read(dtype, G):
+    """Blocks wholly before the window may be released (entry -1) and reused:
+    poisoning them and clearing their table entries changes no bit."""
+    W = 100
+    cfg = _cfg(dtype, 2 * G, 2, 128, 16, RAGGED)
+    inp = make_decode_inputs(cfg, seed=60)
+    a = DeviceInputs(inp).decode(sliding_window=W).clone()
+    from workloads import poison_value
+    pv = poison_value(dtype, "nan")
+    for bb, L in enumerate(inp.context_lens):
+        for j in range(max(0, (int(L) - W)) // 16):
+            phys = inp.block_tables[bb, j]
+            inp.k_cache[phys] = pv
+            inp.v_cache[phys] = pv
+            inp.block_tables[bb, j] = -1
+    pkv.pkv_device_status(clear=True)
+    b = DeviceInputs(inp).decode(sliding_window=W).clone()
+    assert pkv.pkv_device_status(clear=True) == 0
+    assert torch.equal(a, b)

@@ -330,3 +330,67 @@ def test_bad_table_entry_rejected():
     inp.block_tables[0, 1] = 999
     with pytest.raises(ValueError):
         oracle.paged_decode_inputs(inp)
+
+
+# ---------------------------------------------------------------------------
+# sliding window
+
+def test_window_at_least_the_length_is_full_attention():
+    inp = _tiny(seed=20, lens=(1, 7, 16, 33))
+    full = oracle.paged_decode_inputs(inp)
+    assert np.array_equal(oracle.paged_decode_inputs(inp, window=33), full)
+    assert np.array_equal(oracle.paged_decode_inputs(inp, window=1000), full)
+
+
+def test_window_of_one_returns_the_last_value():
+    inp = _tiny(seed=21, lens=(1, 7, 16, 33))
+    out = oracle.paged_decode_inputs(inp, window=1)
+    for b, L in enumerate(inp.context_lens):
+        t = int(L) - 1
+        phys = inp.block_tables[b, t // 16]
+        for h in range(4):
+            assert np.array_equal(out[b, h], inp.v_cache[phys, h, t % 16].astype(np.float64))
+
+
+@pytest.mark.parametrize("W", [2, 15, 16, 17, 40])
+def test_window_equals_sdpa_on_the_last_tokens(W):
+    g = np.random.default_rng(300 + W)
+    B, Hkv, G, D, bs = 3, 2, 2, 16, 4
+    lens = np.array([50, 9, 23])
+    Kc = [[g.standard_normal((int(lens[b]), D)).astype(np.float32) for _ in range(Hkv)]
+          for b in range(B)]
+    Vc = [[g.standard_normal((int(lens[b]), D)).astype(np.float32) for _ in range(Hkv)]
+          for b in range(B)]
+    nblocks = int(((lens + bs - 1) // bs).sum()) + 3
+    K, V, tables, lens32 = _scatter_contiguous(Kc, Vc, bs, nblocks, W)
+    q = g.standard_normal((B, Hkv * G, D)).astype(np.float32)
+    got = oracle.paged_decode(q, K, V, tables, lens32, scale=0.3, dtype="f32", window=W)
+    for b in range(B):
+        L = int(lens[b])
+        lo = max(0, L - W)
+        for h in range(Hkv * G):
+            kk = torch.from_numpy(Kc[b][h // G][lo:].astype(np.float64)).view(1, L - lo, D)
+            vv = torch.from_numpy(Vc[b][h // G][lo:].astype(np.float64)).view(1, L - lo, D)
+            qq = torch.from_numpy(q[b, h].astype(np.float64)).view(1, 1, D)
+            want = torch.nn.functional.scaled_dot_product_attention(
+                qq, kk, vv, scale=0.3).view(D).numpy()
+            np.testing.assert_allclose(got[b, h], want, rtol=0, atol=ATOL)
+
+
+def test_window_never_reads_released_entries():
+    inp = _tiny(seed=22, lens=(40, 33))
+    a = oracle.paged_decode_inputs(inp, window=10)
+    inp.block_tables[0, :1] = -1                      # tokens 0..15 lie before 30
+    inp.block_tables[1, :1] = -1                      # tokens 0..15 lie before 23
+    b = oracle.paged_decode_inputs(inp, window=10)
+    assert np.array_equal(a, b)
+
+
+def test_window_brute_force():
+    inp = _tiny(seed=23, lens=(5, 17, 33), H=4, Hkv=2, D=8)
+    for W in (1, 4, 16, 20):
+        got = oracle.paged_decode_inputs(inp, window=W)
+        want = brute.paged_decode(inp.q.astype(np.float64), inp.k_cache.astype(np.float64),
+                                  inp.v_cache.astype(np.float64), inp.block_tables,
+                                  inp.context_lens, inp.cfg.scale, window=W)
+        np.testing.assert_allclose(got, np.array(want).reshape(got.shape), rtol=0, atol=ATOL)

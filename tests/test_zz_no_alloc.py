@@ -29,7 +29,7 @@ def _static_ws_call(dev: DeviceInputs, out: torch.Tensor, partition_size: int) -
     return b.lib.pkv_paged_attention_decode_static_ws(
         p(out), p(dev.q), p(dev.k), p(dev.v), p(dev.bt), p(dev.cl), None, c.num_seqs,
         c.num_q_heads, c.num_kv_heads, c.head_dim, c.block_size, inp.max_blocks_per_seq,
-        inp.num_blocks, inp.max_context_len, c.scale, pkv.torch_dtype_code(dev.q.dtype),
+        inp.num_blocks, inp.max_context_len, c.scale, 0, pkv.torch_dtype_code(dev.q.dtype),
         partition_size, pkv.PKV_KERNEL_AUTO,
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
@@ -58,5 +58,5 @@ def test_static_workspace_rejects_shapes_beyond_its_size():
     assert need > b.PKV_STATIC_WORKSPACE_BYTES
     rc = b.lib.pkv_paged_attention_decode_static_ws(
         None, None, None, None, None, None, None, 4096, 64, 8, 128, 16, 8192, 1 << 20, 131072,
-        0.1, b.PKV_BF16, 512, 0, None)
+        0.1, 0, b.PKV_BF16, 512, 0, None)
     assert rc == b.PKV_EBOUNDS

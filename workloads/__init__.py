@@ -253,14 +253,22 @@ def kv_bytes_per_token(cfg: DecodeConfig) -> int:
     return 2 * cfg.num_kv_heads * cfg.head_dim * ELEM_BYTES[cfg.dtype]
 
 
-def algorithmic_bytes(cfg: DecodeConfig, lens: np.ndarray) -> int:
-    """Bytes a decode step must move at least once: K and V of every context
-    token, q in and out, the block-table entries used and the lengths."""
+def algorithmic_bytes(cfg: DecodeConfig, lens: np.ndarray, window: int = 0) -> int:
+    """Bytes a decode step must move at least once: K and V of every attended
+    token (the last `window` of each sequence when window > 0), q in and out,
+    the block-table entries used and the lengths."""
     e = ELEM_BYTES[cfg.dtype]
     lens = np.asarray(lens, dtype=np.int64)
-    kv = int(lens.sum()) * kv_bytes_per_token(cfg)
+    if window > 0:
+        lo = np.maximum(lens - window, 0)
+        att = lens - lo
+        nblk = (lens + cfg.block_size - 1) // cfg.block_size - lo // cfg.block_size
+    else:
+        att = lens
+        nblk = blocks_needed(lens, cfg.block_size)
+    kv = int(att.sum()) * kv_bytes_per_token(cfg)
     qo = 2 * lens.size * cfg.num_q_heads * cfg.head_dim * e
-    tab = int(blocks_needed(lens, cfg.block_size).sum()) * 4
+    tab = int(nblk.sum()) * 4
     return kv + qo + tab + 4 * lens.size
 
 
@@ -285,15 +293,24 @@ def draw_cow_recipe(seed: int = 5, **over) -> CowRecipe:
                      tails.astype(np.int64))
 
 
-def random_alloc_ops(seed: int, n_ops: int, max_seqs: int = 24, max_len: int = 200):
+def random_alloc_ops(seed: int, n_ops: int, max_seqs: int = 24, max_len: int = 200,
+                     swap: bool = False, slide: bool = False):
     """A seeded random script of allocator operations (add / fork / append /
-    free) for differential tests of the block manager."""
+    free, swap_out / swap_in when `swap`, sliding-window releases when
+    `slide`) for differential tests of the block manager."""
     g = rng(seed * 1000 + 9)
     ops = []
     next_id = 0
     live = []
     for _ in range(n_ops):
         r = g.random()
+        if slide and live and g.random() < 0.1:
+            ops.append(("slide", live[int(g.integers(len(live)))], int(g.integers(1, 40))))
+            continue
+        if swap and live and g.random() < 0.15:
+            ops.append(("swap_out" if g.random() < 0.5 else "swap_in",
+                        live[int(g.integers(len(live)))]))
+            continue
         if not live or (r < 0.25 and len(live) < max_seqs):
             ops.append(("add", next_id, int(g.integers(0, max_len + 1))))
             live.append(next_id)
