@@ -38,7 +38,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import CONFIGS, ELEM_BYTES, algorithmic_bytes, make_decode_inputs  # noqa: E402
+from workloads import (CONFIGS, ELEM_BYTES, algorithmic_bytes, make_decode_inputs,  # noqa: E402
+                       make_e4m3_pages)
 
 METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak) and tokens/s"
 FALLBACK_HBM_GBS = 6650.0
@@ -75,12 +76,13 @@ def measured_peaks():
     return None
 
 
-def step_bytes(cfg, lens, window: int = 0) -> int:
+def step_bytes(cfg, lens, window: int = 0, kv_dtype: str | None = None) -> int:
     """Decode algorithmic bytes + the append: read k, v of each new token,
-    write them, read the slot."""
+    write them (as E4M3 codes with kv_dtype "e4m3"), read the slot."""
     e = ELEM_BYTES[cfg.dtype]
-    append = len(lens) * (2 * 2 * cfg.num_kv_heads * cfg.head_dim * e + 8)
-    return algorithmic_bytes(cfg, lens, window) + append
+    ec = ELEM_BYTES[kv_dtype or cfg.dtype]
+    append = len(lens) * (2 * cfg.num_kv_heads * cfg.head_dim * (e + ec) + 8)
+    return algorithmic_bytes(cfg, lens, window, kv_dtype) + append
 
 
 class ClockSampler:
@@ -144,6 +146,7 @@ class ClockSampler:
 KERNEL_SOURCES = {
     "simt": ("decode_common.cuh", "decode_simt.cuh", "device_common.cuh"),
     "mma": ("decode_common.cuh", "decode_mma.cuh", "device_common.cuh"),
+    "simt_e4m3": ("decode_common.cuh", "decode_simt.cuh", "device_common.cuh"),
 }
 
 
@@ -156,8 +159,10 @@ def kernel_source_digest(variant: str) -> str:
     return h.hexdigest()[:16]
 
 
-def resolve_variant(cfg, kernel: str) -> str:
+def resolve_variant(cfg, kernel: str, kv: str = "same") -> str:
     """The decode kernel the library's automatic choice takes for cfg."""
+    if kv == "e4m3":
+        return "simt_e4m3"
     if kernel != "auto":
         return kernel
     return "mma" if cfg.dtype != "f32" and 4 <= cfg.group <= 16 else "simt"
@@ -187,12 +192,22 @@ def recorded_traffic(workload: str, variant: str, partition: int | None = None):
 # --------------------------------------------------------------------------
 # CPU oracle timing (the reference arm and the cpu_baseline field)
 
-def oracle_rate(inp, budget_s: float, seed: int = 0):
+def oracle_rate(inp, budget_s: float, seed: int = 0, pages=None):
     """Time the float64 oracle on whole sequences (all heads), in a seeded
     order, passing over the batch again until about budget_s of wall time;
-    returns (bytes/s, seconds, sample description, threads)."""
+    returns (bytes/s, seconds, sample description, threads).  pages: E4M3
+    pages (workloads.QuantisedPages) to decode instead of inp's caches."""
     import oracle
     cfg = inp.cfg
+    kvd = "e4m3" if pages is not None else None
+
+    def run_rows(rows, threads):
+        if pages is None:
+            return oracle.paged_decode_inputs(inp, rows=rows, threads=threads)
+        return oracle.paged_decode(inp.q, pages.k_cache, pages.v_cache, inp.block_tables,
+                                   inp.context_lens, scale=cfg.scale, dtype=cfg.dtype,
+                                   kv_dtype="e4m3", k_scale=pages.k_scale,
+                                   v_scale=pages.v_scale, rows=rows, threads=threads)
     threads = oracle.max_threads()
     order = np.random.default_rng(seed).permutation(cfg.num_seqs)
     nseq, ntok, nbytes, t_total = 0, 0, 0, 0.0
@@ -200,17 +215,18 @@ def oracle_rate(inp, budget_s: float, seed: int = 0):
         for b in order:
             rows = np.array([[b, h] for h in range(cfg.num_q_heads)], dtype=np.int32)
             t0 = time.perf_counter()
-            oracle.paged_decode_inputs(inp, rows=rows, threads=threads)
+            run_rows(rows, threads)
             t_total += time.perf_counter() - t0
             nseq += 1
             ntok += int(inp.context_lens[b])
-            nbytes += algorithmic_bytes(cfg, inp.context_lens[[b]])
+            nbytes += algorithmic_bytes(cfg, inp.context_lens[[b]], kv_dtype=kvd)
             if t_total >= budget_s:
                 break
         if t_total >= budget_s:
             break
     desc = (f"{nseq} sequence decodes (all {cfg.num_q_heads} heads, {ntok} context tokens; "
-            f"passes over the {cfg.num_seqs}-sequence batch of {cfg.name})")
+            f"passes over the {cfg.num_seqs}-sequence batch of {cfg.name}"
+            f"{', E4M3 pages' if pages is not None else ''})")
     return nbytes / t_total, t_total, desc, threads
 
 
@@ -289,13 +305,24 @@ def run_ours(args, cfg):
 
     # ---- inputs (seeded; each rank its own replica)
     inp = make_decode_inputs(cfg, seed=args.seed + rank)
+    e4m3 = args.kv == "e4m3"
+    if e4m3 and (cfg.dtype == "f32" or args.kernel == "mma"):
+        raise SystemExit("E4M3 pages take fp16/bf16 q and the CUDA-core kernel")
 
     def dev(a):
         if cfg.dtype == "bf16" and a.dtype == np.uint16:
             return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
         return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
-    q, kc, vc = dev(inp.q), dev(inp.k_cache), dev(inp.v_cache)
+    pages = None
+    if e4m3:
+        pages = make_e4m3_pages(inp, seed=args.seed + rank)
+        q = dev(inp.q)
+        kc = dev(pages.k_cache).view(torch.float8_e4m3fn)
+        vc = dev(pages.v_cache).view(torch.float8_e4m3fn)
+        ks, vs = dev(pages.k_scale), dev(pages.v_scale)
+    else:
+        q, kc, vc = dev(inp.q), dev(inp.k_cache), dev(inp.v_cache)
     bt, cl = dev(inp.block_tables), dev(inp.context_lens)
     B, H, D, bs = cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
     lens = inp.context_lens.astype(np.int64)
@@ -304,10 +331,18 @@ def run_ours(args, cfg):
     slots = dev(slots_np)
     # the new token of each sequence: the K/V already at its last position
     # (so every step rewrites identical bits and the workload stays fixed)
-    knew = kc.view(-1, H, bs, D)[torch.from_numpy(slots_np // bs).cuda(), :,
-                                 torch.from_numpy(slots_np % bs).cuda(), :].contiguous()
-    vnew = vc.view(-1, H, bs, D)[torch.from_numpy(slots_np // bs).cuda(), :,
-                                 torch.from_numpy(slots_np % bs).cuda(), :].contiguous()
+    # (with E4M3 pages: those values dequantised to q's type; re-quantising
+    # them reaches a fixed point after the first step)
+    sb_idx = torch.from_numpy(slots_np // bs).cuda()
+    so_idx = torch.from_numpy(slots_np % bs).cuda()
+    if e4m3:
+        knew = (kc.view(torch.uint8)[sb_idx, :, so_idx, :].view(torch.float8_e4m3fn).float() *
+                ks[None, :, None]).to(q.dtype).contiguous()
+        vnew = (vc.view(torch.uint8)[sb_idx, :, so_idx, :].view(torch.float8_e4m3fn).float() *
+                vs[None, :, None]).to(q.dtype).contiguous()
+    else:
+        knew = kc.view(-1, H, bs, D)[sb_idx, :, so_idx, :].contiguous()
+        vnew = vc.view(-1, H, bs, D)[sb_idx, :, so_idx, :].contiguous()
     out = torch.empty_like(q)
     mcl = inp.max_context_len
     # schedule the longest sequences first (host-side order from host lengths)
@@ -323,16 +358,29 @@ def run_ours(args, cfg):
     stream = torch.cuda.current_stream()
 
     def decode():
-        pkv.pkv_paged_attention_decode(out, q, kc, vc, bt, cl, cfg.scale, bs, mcl,
-                                       partition_size=P, workspace=ws, seq_order=order,
-                                       sliding_window=W, kernel=kern, stream=stream)
+        if e4m3:
+            pkv.pkv_paged_attention_decode_e4m3(out, q, kc, vc, ks, vs, bt, cl, cfg.scale, bs,
+                                                mcl, partition_size=P, workspace=ws,
+                                                seq_order=order, sliding_window=W,
+                                                stream=stream)
+        else:
+            pkv.pkv_paged_attention_decode(out, q, kc, vc, bt, cl, cfg.scale, bs, mcl,
+                                           partition_size=P, workspace=ws, seq_order=order,
+                                           sliding_window=W, kernel=kern, stream=stream)
+
+    def append():
+        if e4m3:
+            pkv.pkv_kv_cache_append_e4m3(kc, vc, knew, vnew, ks, vs, slots, stream=stream)
+        else:
+            pkv.pkv_kv_cache_append(kc, vc, knew, vnew, slots, stream=stream)
 
     def step():
-        pkv.pkv_kv_cache_append(kc, vc, knew, vnew, slots, stream=stream)
+        append()
         decode()
 
-    nbytes = step_bytes(cfg, lens, W)
-    dec_bytes = algorithmic_bytes(cfg, lens, W)
+    kvd = "e4m3" if e4m3 else None
+    nbytes = step_bytes(cfg, lens, W, kvd)
+    dec_bytes = algorithmic_bytes(cfg, lens, W, kvd)
 
     # ---- device-resident timing
     for _ in range(args.warmup):
@@ -346,7 +394,7 @@ def run_ours(args, cfg):
     with ClockSampler(local) as clocks:
         t_start.record(stream)
         for i in range(args.steps):
-            pkv.pkv_kv_cache_append(kc, vc, knew, vnew, slots, stream=stream)
+            append()
             ev_dec[i][0].record(stream)
             decode()
             ev_dec[i][1].record(stream)
@@ -395,15 +443,26 @@ def run_ours(args, cfg):
     calls = []
     for j in range(2):
         ptr = {name: ctypes.c_void_p(d_in[j].data_ptr() + offs[name]) for name, _ in fields}
-        append_args = (ctypes.c_void_p(kc.data_ptr()), ctypes.c_void_p(vc.data_ptr()),
-                       ptr["knew"], ptr["vnew"], ptr["slots"], B, H, D, bs, N_blocks, dt_code,
-                       c_stream)
-        decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"],
-                       ctypes.c_void_p(kc.data_ptr()), ctypes.c_void_p(vc.data_ptr()), ptr["bt"],
-                       ptr["cl"], ptr.get("order"), B, cfg.num_q_heads, H, D, bs,
-                       bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
-                       ctypes.c_void_p(ws.data_ptr()), ws.numel(), kern, c_stream)
+        kp, vp = ctypes.c_void_p(kc.data_ptr()), ctypes.c_void_p(vc.data_ptr())
+        if e4m3:
+            ksp, vsp = ctypes.c_void_p(ks.data_ptr()), ctypes.c_void_p(vs.data_ptr())
+            append_args = (kp, vp, ptr["knew"], ptr["vnew"], ksp, vsp, ptr["slots"], B, H, D, bs,
+                           N_blocks, dt_code, c_stream)
+            decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ksp, vsp,
+                           ptr["bt"], ptr["cl"], ptr.get("order"), B, cfg.num_q_heads, H, D,
+                           bs, bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
+                           ctypes.c_void_p(ws.data_ptr()), ws.numel(), c_stream)
+        else:
+            append_args = (kp, vp, ptr["knew"], ptr["vnew"], ptr["slots"], B, H, D, bs,
+                           N_blocks, dt_code, c_stream)
+            decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ptr["bt"],
+                           ptr["cl"], ptr.get("order"), B, cfg.num_q_heads, H, D, bs,
+                           bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
+                           ctypes.c_void_p(ws.data_ptr()), ws.numel(), kern, c_stream)
         calls.append((append_args, decode_args))
+    c_append = pkv.lib.pkv_kv_cache_append_e4m3 if e4m3 else pkv.lib.pkv_kv_cache_append
+    c_decode = (pkv.lib.pkv_paged_attention_decode_e4m3 if e4m3
+                else pkv.lib.pkv_paged_attention_decode)
 
     def e2e_step(i):
         j = i % 2
@@ -414,7 +473,7 @@ def run_ours(args, cfg):
         stream.wait_event(ev_in[j])
         stream.wait_event(ev_out[j])             # d_out[j] of step i-2 has been read back
         a_args, d_args = calls[j]
-        if pkv.lib.pkv_kv_cache_append(*a_args) or pkv.lib.pkv_paged_attention_decode(*d_args):
+        if c_append(*a_args) or c_decode(*d_args):
             raise SystemExit("C-ABI call failed in the e2e loop")
         ev_done[j].record(stream)
         with torch.cuda.stream(s_out):
@@ -456,13 +515,15 @@ def run_ours(args, cfg):
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": cfg.dtype, "data": "synthetic",
+            "dtype": "e4m3" if e4m3 else cfg.dtype, "data": "synthetic",
             "config": {"workload": cfg.name, "global_batch": B * world,
                        "seq_len": round(float(lens.mean()), 1),
                        "num_q_heads": cfg.num_q_heads, "num_kv_heads": H, "head_dim": D,
                        "block_size": bs, "partition_size": Pused, "kernel": args.kernel,
                        "schedule": "longest-first" if args.order else "batch order",
                        "sliding_window": W,
+                       "kv_pages": "e4m3 (per-head fp32 scales)" if e4m3 else cfg.dtype,
+                       "q_out": cfg.dtype,
                        "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (%.2f GB of K/V per step)" % (
                            dec_bytes / 1e9)},
@@ -476,13 +537,15 @@ def run_ours(args, cfg):
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": peak_src,
                          "decode_ms": round(dec_ms, 5), "bytes_per_launch": int(dec_bytes),
-                         "variant": resolve_variant(cfg, args.kernel),
-                         "traffic": recorded_traffic(cfg.name, resolve_variant(cfg, args.kernel),
+                         "variant": resolve_variant(cfg, args.kernel, args.kv),
+                         "traffic": recorded_traffic(cfg.name,
+                                                     resolve_variant(cfg, args.kernel, args.kv),
                                                      Pused)},
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
-            rate, secs, desc, threads = oracle_rate(inp, args.cpu_budget, seed=args.seed)
+            rate, secs, desc, threads = oracle_rate(inp, args.cpu_budget, seed=args.seed,
+                                                    pages=pages)
             line["cpu_baseline"] = {"value": round(rate / 1e9, 4), "unit": "GB/s",
                                     "cores": threads, "kind": "oracle",
                                     "sample": desc + f", {secs:.1f} s"}
@@ -721,6 +784,9 @@ def main():
     ap.add_argument("--seed", type=int, default=2)
     ap.add_argument("--window", type=int, default=0,
                     help="sliding window in tokens (0: attend to the whole context)")
+    ap.add_argument("--kv", choices=["same", "e4m3"], default="same",
+                    help="page element type: the workload's, or FP8 E4M3 codes with "
+                         "per-head scales")
     ap.add_argument("--no-order", dest="order", action="store_false",
                     help="schedule sequences in batch order instead of longest first")
     ap.add_argument("--cpu-budget", type=float, default=12.0,

@@ -74,7 +74,11 @@ typedef enum {
     PKV_EUNSUPPORTED = -7  /* valid but not built (e.g. head_dim 96) */
 } pkv_status;
 
-typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+/* Element types.  PKV_E4M3: FP8 codes (1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits; largest finite value 448, code 0x7F / 0xFF = NaN), the
+ * storage of quantised KV pages; the cache operations move them as bytes and
+ * the decode reads them through pkv_paged_attention_decode_e4m3. */
+typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2, PKV_E4M3 = 3 } pkv_dtype;
 
 /* Decode kernel choice.  AUTO takes the tensor-core kernel for 16-bit caches
  * with a query group of 4 or more heads per KV head, else the CUDA-core one. */
@@ -169,6 +173,35 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
                                pkv_stream_t stream);
 
 /*
+ * Paged decode attention over FP8 E4M3 pages ("pagedattention vllm"
+ * §Comparison with Alternatives: the paged layout combines with a quantised
+ * cache).  Page element x of KV head g stands for the value
+ * E4M3(x) * k_scale[g] (keys) or E4M3(x) * v_scale[g] (values), and the result
+ * is pkv_paged_attention_decode's over those values:
+ *   out[b,h,:] = softmax_t(scale * k_scale[g] * q[b,h,:] . E4M3(k_t))
+ *                weighted sum of v_scale[g] * E4M3(v_t),   g = h / (Hq/Hkv).
+ * The kernel folds k_scale into q and v_scale into the float32 accumulator;
+ * each code is widened exactly (every E4M3 value is a binary16 value).
+ *
+ * Arguments as pkv_paged_attention_decode, plus:
+ *   k_cache, v_cache: device E4M3 codes [num_blocks, Hkv, block_size, head_dim].
+ *   k_scale, v_scale: device float32 [num_kv_heads], finite and > 0 (not
+ *       checked on the device: the caller's quantisation scales).
+ *   dtype: PKV_F16 or PKV_BF16, the type of q and out.
+ *   head_dim in {128, 256} (a page row must be at least 128 bytes).
+ *   Always the CUDA-core kernel.  The workspace is sized as for the 16-bit
+ *   decode (pkv_decode_workspace_size).
+ * Returns PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED or PKV_ECUDA.
+ */
+PKV_API int pkv_paged_attention_decode_e4m3(
+    void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+    const float* v_scale, const int32_t* block_tables, const int32_t* context_lens,
+    const int32_t* seq_order, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+    int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+    int sliding_window, pkv_dtype dtype, int partition_size, void* workspace,
+    size_t workspace_bytes, pkv_stream_t stream);
+
+/*
  * Size of the workspace compiled into the library for
  * pkv_paged_attention_decode_static_ws: 64 MiB per GPU.
  */
@@ -227,6 +260,26 @@ PKV_API int pkv_kv_cache_append(void* k_cache, void* v_cache, const void* k, con
                         const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
                         int head_dim, int block_size, int num_blocks, pkv_dtype dtype,
                         pkv_stream_t stream);
+
+/*
+ * KV append into E4M3 pages: as pkv_kv_cache_append, but each element is
+ * quantised on the way in:
+ *   k_cache[s / bs, h, s % bs, d] = E4M3(k[t, h, d] / k_scale[h]),
+ * same for v with v_scale.  The division is a float32 division (correctly
+ * rounded), the code the nearest E4M3 value (ties to even), magnitudes
+ * beyond 448 saturate to 448 and NaN stays NaN.
+ *   k, v: device [num_tokens, Hkv, head_dim] in in_dtype (PKV_F16 or PKV_BF16),
+ *       16-byte aligned; head_dim a multiple of 16.
+ *   k_scale, v_scale: device float32 [num_kv_heads].
+ *   k_cache, v_cache: device E4M3 codes, 16-byte aligned.
+ * Slots as pkv_kv_cache_append (negative skipped, past the pool flagged
+ * PKV_DEV_BAD_SLOT).  Returns PKV_OK, PKV_EINVAL or PKV_ECUDA.
+ */
+PKV_API int pkv_kv_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, const void* v,
+                                     const float* k_scale, const float* v_scale,
+                                     const int64_t* slot_mapping, int num_tokens,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int num_blocks, pkv_dtype in_dtype, pkv_stream_t stream);
 
 /*
  * Copy-on-write block copies ("pagedattention vllm" §Copy-on-Write Sharing:

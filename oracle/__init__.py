@@ -54,6 +54,8 @@ def lib():
             L.pkvo_decode_bf16.argtypes = [ctypes.c_uint16]
             L.pkvo_decode_f32.restype = ctypes.c_double
             L.pkvo_decode_f32.argtypes = [ctypes.c_uint32]
+            L.pkvo_decode_e4m3.restype = ctypes.c_double
+            L.pkvo_decode_e4m3.argtypes = [ctypes.c_uint8]
             L.pkvo_decode_array.restype = None
             L.pkvo_decode_array.argtypes = [ctypes.c_int, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_int64]
@@ -62,8 +64,8 @@ def lib():
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                ctypes.c_int64, ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
-                ctypes.c_int64, ctypes.c_int]
+                ctypes.c_int64, ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int]
             L.pkvo_max_threads.restype = ctypes.c_int
             _lib = L
     return _lib
@@ -84,9 +86,12 @@ def decode_bits(arr: np.ndarray, dtype: str) -> np.ndarray:
 
 def paged_decode(q, k_cache, v_cache, block_tables, context_lens, *, scale: float,
                  dtype: str, num_kv_heads: int | None = None, rows=None,
-                 threads: int = 0, window: int = 0) -> np.ndarray:
+                 threads: int = 0, window: int = 0, kv_dtype: str | None = None,
+                 k_scale=None, v_scale=None) -> np.ndarray:
     """float64 paged decode attention (window > 0: over each sequence's last
-    `window` tokens only).
+    `window` tokens only).  dtype is q's storage type; kv_dtype the caches'
+    (default: the same; "e4m3" for FP8 codes, with float32 k_scale / v_scale
+    per KV head).
 
     q [B, Hq, D]; k_cache, v_cache [N, Hkv, bs, D] in the storage dtype
     (bf16 as uint16 bits); block_tables int32 [B, max_blocks];
@@ -109,10 +114,15 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, *, scale: floa
     else:
         out = np.empty((B, Hq, D), dtype=np.float64)
         rp, nr = None, 0
+    kvd = DTYPE_CODE[kv_dtype or dtype]
+    ks = None if k_scale is None else np.ascontiguousarray(k_scale, dtype=np.float32)
+    vs = None if v_scale is None else np.ascontiguousarray(v_scale, dtype=np.float32)
     rc = lib().pkvo_paged_decode(out.ctypes.data, q.ctypes.data, k_cache.ctypes.data,
                                  v_cache.ctypes.data, bt.ctypes.data, cl.ctypes.data,
                                  B, Hq, Hkv, D, bs, bt.shape[1], N, float(scale),
-                                 int(window), DTYPE_CODE[dtype], rp, nr, int(threads))
+                                 int(window), DTYPE_CODE[dtype], kvd,
+                                 None if ks is None else ks.ctypes.data,
+                                 None if vs is None else vs.ctypes.data, rp, nr, int(threads))
     if rc != 0:
         raise ValueError(f"oracle rejected the inputs (code {rc})")
     return out

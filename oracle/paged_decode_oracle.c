@@ -22,7 +22,10 @@
  *     s_t = scale * sum_d q[b,h,d] k_t[d]
  *     out[b,h,:] = sum_t exp(s_t - max s) v_t / sum_t exp(s_t - max s)
  * in float64, plain loops, no blocking and no online rescaling.  L = 0 gives a
- * zero row.  lo = 0, or with a sliding window of W tokens lo = max(0, L - W):
+ * zero row.  Quantised caches (FP8 E4M3 codes) hold code * scale, one scale
+ * per KV head for K and one for V (paging combines with quantisation:
+ * "pagedattention vllm" §Comparison with Alternatives).
+ * lo = 0, or with a sliding window of W tokens lo = max(0, L - W):
  * only the last W tokens are attended to ("pagedattention vllm" §Advanced
  * Features: sliding-window models keep only recent blocks).  The inputs are decoded bit by bit from their storage type
  * (float32, IEEE binary16, bfloat16) by this file's own decoders.
@@ -38,7 +41,7 @@
 #include <omp.h>
 #endif
 
-enum { O_F32 = 0, O_F16 = 1, O_BF16 = 2 };
+enum { O_F32 = 0, O_F16 = 1, O_BF16 = 2, O_E4M3 = 3 };
 
 /* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits */
 double pkvo_decode_f16(uint16_t h) {
@@ -88,7 +91,29 @@ double pkvo_decode_f32(uint32_t u) {
     return sign ? -v : v;
 }
 
+/* OCP FP8 E4M3 ("fn" variant): 1 sign bit, 4 exponent bits (bias 7), 3
+ * fraction bits; no infinities, S.1111.111 is NaN. */
+double pkvo_decode_e4m3(uint8_t c) {
+    int sign = (c >> 7) & 1;
+    int ex = (c >> 3) & 0xf;
+    int man = c & 0x7;
+    double v;
+    if (ex == 0) {
+        v = ldexp((double)man, -9);                  /* 2^(1-7) * man/8 */
+    } else if (ex == 15 && man == 7) {
+        v = NAN;
+    } else {
+        v = ldexp(1.0 + (double)man / 8.0, ex - 7);
+    }
+    return sign ? -v : v;
+}
+
 static double load_elem(const void* base, int64_t idx, int dtype) {
+    if (dtype == O_E4M3) {
+        uint8_t c;
+        memcpy(&c, (const char*)base + idx, 1);
+        return pkvo_decode_e4m3(c);
+    }
     if (dtype == O_F32) {
         uint32_t u;
         memcpy(&u, (const char*)base + 4 * idx, 4);
@@ -110,12 +135,16 @@ static int decode_row(double* out_row, const void* q, const void* k_cache,
                       const int32_t* context_lens, int b, int h, int num_q_heads,
                       int num_kv_heads, int head_dim, int block_size,
                       int max_blocks_per_seq, int64_t num_blocks, double scale,
-                      int window, int dtype, double* s /* scratch, >= L + head_dim */) {
+                      int window, int dtype, int kv_dtype, const float* k_scale,
+                      const float* v_scale, double* s /* scratch, >= L + head_dim */) {
     const int G = num_q_heads / num_kv_heads;
     const int g = h / G;
     const int L = context_lens[b];
     const int lo = (window > 0 && L > window) ? L - window : 0;
     const int D = head_dim;
+    /* quantised pages: value = code * scale of the KV head */
+    const double ks = k_scale ? (double)k_scale[g] : 1.0;
+    const double vs = v_scale ? (double)v_scale[g] : 1.0;
     for (int d = 0; d < D; ++d) out_row[d] = 0.0;
     if (L <= 0) return 0;
 
@@ -131,7 +160,7 @@ static int decode_row(double* out_row, const void* q, const void* k_cache,
         int64_t k_off = (((int64_t)phys * num_kv_heads + g) * block_size + t % block_size) * D;
         double acc = 0.0;
         for (int d = 0; d < D; ++d)
-            acc += qrow[d] * load_elem(k_cache, k_off + d, dtype);
+            acc += qrow[d] * (load_elem(k_cache, k_off + d, kv_dtype) * ks);
         s[t] = scale * acc;
     }
     double m = s[lo];
@@ -143,7 +172,8 @@ static int decode_row(double* out_row, const void* q, const void* k_cache,
         denom += w;
         int32_t phys = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
         int64_t v_off = (((int64_t)phys * num_kv_heads + g) * block_size + t % block_size) * D;
-        for (int d = 0; d < D; ++d) out_row[d] += w * load_elem(v_cache, v_off + d, dtype);
+        for (int d = 0; d < D; ++d)
+            out_row[d] += w * (load_elem(v_cache, v_off + d, kv_dtype) * vs);
     }
     for (int d = 0; d < D; ++d) out_row[d] /= denom;
     return 0;
@@ -159,7 +189,8 @@ int pkvo_paged_decode(double* out, const void* q, const void* k_cache,
                       const int32_t* context_lens, int num_seqs, int num_q_heads,
                       int num_kv_heads, int head_dim, int block_size,
                       int max_blocks_per_seq, int64_t num_blocks, double scale,
-                      int window, int dtype, const int32_t* rows, int64_t num_rows,
+                      int window, int dtype, int kv_dtype, const float* k_scale,
+                      const float* v_scale, const int32_t* rows, int64_t num_rows,
                       int num_threads) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         block_size <= 0 || num_q_heads % num_kv_heads != 0)
@@ -193,7 +224,7 @@ int pkvo_paged_decode(double* out, const void* q, const void* k_cache,
             if (decode_row(out + i * head_dim, q, k_cache, v_cache, block_tables,
                            context_lens, b, h, num_q_heads, num_kv_heads, head_dim,
                            block_size, max_blocks_per_seq, num_blocks, scale, window, dtype,
-                           s))
+                           kv_dtype, k_scale, v_scale, s))
                 err |= 1;
         }
         free(s);

@@ -7,6 +7,8 @@ happens in libpagedkv.so.
 
     pkv_paged_attention_decode   paged decode attention (+ log-sum-exp reduce)
     pkv_kv_cache_append          new tokens' K/V -> their slots
+    pkv_paged_attention_decode_e4m3 / pkv_kv_cache_append_e4m3
+                                 the same over FP8 E4M3 pages with per-head scales
     pkv_copy_blocks              copy-on-write block copies
     BlockAllocator               host block manager (free list, refcounts, CoW)
 """
@@ -17,7 +19,7 @@ import ctypes
 import torch
 
 from . import _binding as _b
-from ._binding import (PKV_BF16, PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD_ORDER,
+from ._binding import (PKV_BF16, PKV_E4M3, PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD_ORDER,
                        PKV_DEV_BAD_SLOT, PKV_DEV_TIMEOUT, PKV_F16, PKV_F32, PKV_KERNEL_AUTO, PKV_KERNEL_MMA,
                        PKV_KERNEL_SIMT, PagedKVError, check, lib)
 
@@ -28,10 +30,12 @@ __all__ = [
     "PagedKVError", "lib", "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_KERNEL_AUTO",
     "PKV_KERNEL_SIMT", "PKV_KERNEL_MMA", "PKV_DEV_BAD_BLOCK", "PKV_DEV_BAD_LEN",
     "PKV_DEV_BAD_SLOT", "PKV_DEV_TIMEOUT", "PKV_DEV_BAD_ORDER", "torch_dtype_code",
-    "pkv_decode_schedule_order",
+    "pkv_decode_schedule_order", "pkv_paged_attention_decode_e4m3", "pkv_kv_cache_append_e4m3",
+    "PKV_E4M3",
 ]
 
-_DTYPE = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16}
+_DTYPE = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16,
+          torch.float8_e4m3fn: PKV_E4M3}
 
 
 def torch_dtype_code(dt: torch.dtype) -> int:
@@ -119,6 +123,51 @@ def pkv_paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torc
     return out
 
 
+def pkv_paged_attention_decode_e4m3(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                                    v_cache: torch.Tensor, k_scale: torch.Tensor,
+                                    v_scale: torch.Tensor, block_tables: torch.Tensor,
+                                    context_lens: torch.Tensor, scale: float, block_size: int,
+                                    max_context_len: int, *, partition_size: int = 0,
+                                    workspace: torch.Tensor | None = None,
+                                    seq_order: torch.Tensor | None = None,
+                                    sliding_window: int = 0, stream=None) -> torch.Tensor:
+    """Paged decode over FP8 E4M3 pages (pkv_paged_attention_decode_e4m3 in
+    pagedkv.h): k_cache/v_cache torch.float8_e4m3fn [N, Hkv, block_size, D];
+    k_scale/v_scale float32 [Hkv]; q and out fp16 or bf16."""
+    for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+                 (k_scale, "k_scale"), (v_scale, "v_scale"), (block_tables, "block_tables"),
+                 (context_lens, "context_lens")):
+        _dev(t, n)
+    if seq_order is not None:
+        _dev(seq_order, "seq_order")
+        if seq_order.dtype != torch.int32 or seq_order.numel() != q.shape[0]:
+            raise PagedKVError(_b.PKV_EINVAL, "seq_order must be int32 [num_seqs]")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise PagedKVError(_b.PKV_EINVAL, "block_tables / context_lens must be int32")
+    if k_cache.dtype != torch.float8_e4m3fn or v_cache.dtype != torch.float8_e4m3fn:
+        raise PagedKVError(_b.PKV_EINVAL, "k_cache / v_cache must be float8_e4m3fn")
+    if q.dtype != out.dtype or k_scale.dtype != torch.float32 or v_scale.dtype != torch.float32:
+        raise PagedKVError(_b.PKV_EINVAL, "q/out dtypes differ or scales are not float32")
+    B, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    if (D2 != D or bs != block_size or tuple(out.shape) != (B, Hq, D) or
+            tuple(v_cache.shape) != tuple(k_cache.shape) or block_tables.shape[0] != B or
+            context_lens.shape[0] != B or k_scale.numel() != Hkv or v_scale.numel() != Hkv):
+        raise PagedKVError(_b.PKV_EINVAL, "shape mismatch")
+    ws_bytes = 0
+    if workspace is not None:
+        _dev(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    check(lib.pkv_paged_attention_decode_e4m3(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+        _ptr(block_tables), _ptr(context_lens), _ptr(seq_order), B, Hq, Hkv, D, bs,
+        block_tables.shape[1], N, int(max_context_len), float(scale), int(sliding_window),
+        torch_dtype_code(q.dtype), int(partition_size), _ptr(workspace), ws_bytes,
+        _stream(stream)),
+        "pkv_paged_attention_decode_e4m3")
+    return out
+
+
 def pkv_paged_attention_decode_static_ws(out: torch.Tensor, q: torch.Tensor,
                                          k_cache: torch.Tensor, v_cache: torch.Tensor,
                                          block_tables: torch.Tensor, context_lens: torch.Tensor,
@@ -178,6 +227,32 @@ def pkv_kv_cache_append(k_cache: torch.Tensor, v_cache: torch.Tensor, k: torch.T
                                   _ptr(slot_mapping), T, Hkv, D, bs, N,
                                   torch_dtype_code(k.dtype), _stream(stream)),
           "pkv_kv_cache_append")
+
+
+def pkv_kv_cache_append_e4m3(k_cache: torch.Tensor, v_cache: torch.Tensor, k: torch.Tensor,
+                             v: torch.Tensor, k_scale: torch.Tensor, v_scale: torch.Tensor,
+                             slot_mapping: torch.Tensor, *, stream=None) -> None:
+    """fp16/bf16 k/v [T, Hkv, D] -> E4M3 codes of k / k_scale[h] (and v) in
+    the float8_e4m3fn caches' slots."""
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache"), (k, "k"), (v, "v"),
+                 (k_scale, "k_scale"), (v_scale, "v_scale"), (slot_mapping, "slot_mapping")):
+        _dev(t, n)
+    if slot_mapping.dtype != torch.int64:
+        raise PagedKVError(_b.PKV_EINVAL, "slot_mapping must be int64")
+    if k_cache.dtype != torch.float8_e4m3fn or v_cache.dtype != torch.float8_e4m3fn or \
+            k.dtype != v.dtype or k_scale.dtype != torch.float32 or \
+            v_scale.dtype != torch.float32:
+        raise PagedKVError(_b.PKV_EINVAL, "dtype mismatch")
+    N, Hkv, bs, D = k_cache.shape
+    T = k.shape[0]
+    if (tuple(k.shape) != (T, Hkv, D) or tuple(v.shape) != (T, Hkv, D) or
+            slot_mapping.shape[0] != T or tuple(v_cache.shape) != tuple(k_cache.shape) or
+            k_scale.numel() != Hkv or v_scale.numel() != Hkv):
+        raise PagedKVError(_b.PKV_EINVAL, "shape mismatch")
+    check(lib.pkv_kv_cache_append_e4m3(_ptr(k_cache), _ptr(v_cache), _ptr(k), _ptr(v),
+                                       _ptr(k_scale), _ptr(v_scale), _ptr(slot_mapping), T,
+                                       Hkv, D, bs, N, torch_dtype_code(k.dtype), _stream(stream)),
+          "pkv_kv_cache_append_e4m3")
 
 
 def pkv_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_pairs: torch.Tensor,

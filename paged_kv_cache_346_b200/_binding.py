@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(PKG, "libpagedkv.so")
 
 PKV_OK, PKV_EINVAL, PKV_ENOMEM, PKV_ENOSEQ, PKV_EEXIST, PKV_EBOUNDS, PKV_ECUDA, \
     PKV_EUNSUPPORTED = 0, -1, -2, -3, -4, -5, -6, -7
-PKV_F32, PKV_F16, PKV_BF16 = 0, 1, 2
+PKV_F32, PKV_F16, PKV_BF16, PKV_E4M3 = 0, 1, 2, 3
 PKV_KERNEL_AUTO, PKV_KERNEL_SIMT, PKV_KERNEL_MMA = 0, 1, 2
 PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD_SLOT, PKV_DEV_TIMEOUT, PKV_DEV_BAD_ORDER = \
     1, 2, 4, 8, 16
@@ -42,9 +42,14 @@ SIGNATURES = {
     "pkv_paged_attention_decode_static_ws": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                                     _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                                                     _f32, _i32, _i32, _i32, _i32, _vp]),
+    "pkv_paged_attention_decode_e4m3": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                               _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                               _f32, _i32, _i32, _i32, _vp, _sz, _vp]),
     "pkv_decode_schedule_order": (_i32, [_vp, _i32, _vp]),
     "pkv_kv_cache_append": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                    _vp]),
+    "pkv_kv_cache_append_e4m3": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+                                        _i32, _i32, _i32, _vp]),
     "pkv_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_swap_blocks": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                _i32, _vp]),

@@ -42,6 +42,7 @@ int elem_size(pkv_dtype dt) {
         case PKV_F32: return 4;
         case PKV_F16: return 2;
         case PKV_BF16: return 2;
+        case PKV_E4M3: return 1;
     }
     return 0;
 }
@@ -79,6 +80,119 @@ bool device_view(const void* p, void** out) {
 }
 
 constexpr int kNumSMs = 148;
+
+
+// The decode behind both entry points.  e4m3: the pages hold E4M3 codes with
+// per-KV-head scales and dtype is the type of q and out.
+int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                const float* k_scale, const float* v_scale, bool e4m3,
+                const int32_t* block_tables, const int32_t* context_lens,
+                const int32_t* seq_order, int num_seqs, int num_q_heads, int num_kv_heads,
+                int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                int max_context_len, float scale, int sliding_window, pkv_dtype dtype,
+                int partition_size, void* workspace, size_t workspace_bytes, pkv_kernel kernel,
+                pkv_stream_t stream) {
+    // ---- host-side checks (nothing has been launched if these fail)
+    const int es = elem_size(dtype);
+    if (dtype == PKV_E4M3 || (e4m3 && dtype == PKV_F32)) return PKV_EINVAL;
+    if (es == 0 || num_seqs < 0 || num_seqs > 65535 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+        num_q_heads % num_kv_heads != 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
+        max_context_len < 0 || (int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size ||
+        !std::isfinite(scale) || sliding_window < 0 || partition_size < 0 ||
+        (partition_size != 0 && (partition_size % 64 != 0 || partition_size > 8192)))
+        return PKV_EINVAL;
+    if (kernel != PKV_KERNEL_AUTO && kernel != PKV_KERNEL_SIMT && kernel != PKV_KERNEL_MMA)
+        return PKV_EINVAL;
+    if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PKV_EUNSUPPORTED;
+    if (block_size != 16 && block_size != 32 && block_size != 64) return PKV_EUNSUPPORTED;
+    if (dtype == PKV_F32 && head_dim == 256) return PKV_EUNSUPPORTED;
+    if (e4m3 && head_dim == 64) return PKV_EUNSUPPORTED;
+    if (e4m3 && kernel == PKV_KERNEL_MMA) return PKV_EUNSUPPORTED;
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_EINVAL;
+    if (e4m3 && (!k_scale || !v_scale)) return PKV_EINVAL;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PKV_EINVAL;
+
+    const int G = num_q_heads / num_kv_heads;
+    // longest span a sequence attends to: with a window, at most the window
+    // plus the part of its first block ahead of it
+    const int span = sliding_window > 0
+                         ? (int)std::min<int64_t>(max_context_len,
+                                                  (int64_t)sliding_window + block_size - 1)
+                         : max_context_len;
+    const int P = partition_size ? partition_size
+                                 : pkv_decode_default_partition(num_seqs, num_kv_heads, span);
+    const int np = span > 0 ? ceil_div(span, P) : 1;
+    if (np > 1) {
+        const size_t need = pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads,
+                                                      head_dim, span, P);
+        if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PKV_EINVAL;
+    }
+
+    // the tensor-core kernel addresses the pool as one 2-D tensor of
+    // num_blocks * Hkv * block_size rows with 32-bit TMA coordinates
+    const bool mma_fits = !e4m3 && dtype != PKV_F32 && G <= 16 &&
+                          (int64_t)num_blocks * num_kv_heads * block_size < (1ll << 31);
+    bool use_mma;
+    if (kernel == PKV_KERNEL_MMA) {
+        if (!kMmaBuilt || !mma_fits) return PKV_EUNSUPPORTED;
+        use_mma = true;
+    } else if (kernel == PKV_KERNEL_SIMT) {
+        use_mma = false;
+    } else {
+        use_mma = kMmaBuilt && mma_fits && G >= 4;
+    }
+    const int hg = use_mma ? (G <= 8 ? 8 : 16)
+                           : (G % 4 == 0 && !e4m3 ? 4 : (G % 2 == 0 ? 2 : 1));
+    const int head_chunks = (G + hg - 1) / hg;
+    if ((int64_t)num_kv_heads * head_chunks > 65535) return PKV_EUNSUPPORTED;
+
+    DecodeArgs a;
+    a.out = out;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.seq_order = seq_order;
+    a.k_scale = e4m3 ? k_scale : nullptr;
+    a.v_scale = e4m3 ? v_scale : nullptr;
+    a.ws_o = static_cast<float*>(workspace);
+    a.ws_ml = np > 1 ? a.ws_o + (int64_t)num_seqs * num_q_heads * np * head_dim : nullptr;
+    a.num_seqs = num_seqs;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.group = G;
+    a.head_chunks = head_chunks;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
+    a.max_tokens = max_blocks_per_seq * block_size;
+    a.partition_size = P;
+    a.max_partitions = np;
+    a.block_size = block_size;
+    a.window = sliding_window;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    if (status_word(&a.status) != cudaSuccess) return PKV_ECUDA;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (e4m3) {
+        e = dtype == PKV_F16 ? decode_simt_e4m3_f16(a, head_dim, block_size, hg, s)
+                             : decode_simt_e4m3_bf16(a, head_dim, block_size, hg, s);
+    } else if (use_mma) {
+        e = dtype == PKV_F16 ? decode_mma_f16(a, head_dim, block_size, hg, s)
+                             : decode_mma_bf16(a, head_dim, block_size, hg, s);
+    } else {
+        switch (dtype) {
+            case PKV_F32: e = decode_simt_f32(a, head_dim, block_size, hg, s); break;
+            case PKV_F16: e = decode_simt_f16(a, head_dim, block_size, hg, s); break;
+            default: e = decode_simt_bf16(a, head_dim, block_size, hg, s); break;
+        }
+    }
+    if (e == cudaErrorInvalidValue) return PKV_EUNSUPPORTED;
+    return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
 
 }  // namespace
 }  // namespace pkv
@@ -135,103 +249,36 @@ size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads
     return (size_t)num_seqs * num_q_heads * np * (head_dim + 2) * sizeof(float);
 }
 
+
 int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* block_tables, const int32_t* context_lens,
-                               const int32_t* seq_order, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                               int block_size, int max_blocks_per_seq, int num_blocks,
-                               int max_context_len, float scale, int sliding_window,
-                               pkv_dtype dtype, int partition_size, void* workspace,
-                               size_t workspace_bytes, pkv_kernel kernel, pkv_stream_t stream) {
-    // ---- host-side checks (nothing has been launched if these fail)
-    const int es = elem_size(dtype);
-    if (es == 0 || num_seqs < 0 || num_seqs > 65535 || num_q_heads <= 0 || num_kv_heads <= 0 ||
-        num_q_heads % num_kv_heads != 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
-        max_context_len < 0 || (int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size ||
-        !std::isfinite(scale) || sliding_window < 0 || partition_size < 0 ||
-        (partition_size != 0 && (partition_size % 64 != 0 || partition_size > 8192)))
-        return PKV_EINVAL;
-    if (kernel != PKV_KERNEL_AUTO && kernel != PKV_KERNEL_SIMT && kernel != PKV_KERNEL_MMA)
-        return PKV_EINVAL;
-    if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PKV_EUNSUPPORTED;
-    if (block_size != 16 && block_size != 32 && block_size != 64) return PKV_EUNSUPPORTED;
-    if (dtype == PKV_F32 && head_dim == 256) return PKV_EUNSUPPORTED;
-    if (num_seqs == 0) return PKV_OK;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_EINVAL;
-    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-        return PKV_EINVAL;
+                               const int32_t* seq_order, int num_seqs, int num_q_heads,
+                               int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int num_blocks, int max_context_len,
+                               float scale, int sliding_window, pkv_dtype dtype,
+                               int partition_size, void* workspace, size_t workspace_bytes,
+                               pkv_kernel kernel, pkv_stream_t stream) {
+    return pkv::decode_impl(out, q, k_cache, v_cache, nullptr, nullptr, false, block_tables,
+                            context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
+                            head_dim, block_size, max_blocks_per_seq, num_blocks,
+                            max_context_len, scale, sliding_window, dtype, partition_size,
+                            workspace, workspace_bytes, kernel, stream);
+}
 
-    const int G = num_q_heads / num_kv_heads;
-    // longest span a sequence attends to: with a window, at most the window
-    // plus the part of its first block ahead of it
-    const int span = sliding_window > 0
-                         ? (int)std::min<int64_t>(max_context_len,
-                                                  (int64_t)sliding_window + block_size - 1)
-                         : max_context_len;
-    const int P = partition_size ? partition_size
-                                 : pkv_decode_default_partition(num_seqs, num_kv_heads, span);
-    const int np = span > 0 ? ceil_div(span, P) : 1;
-    if (np > 1) {
-        const size_t need = pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads,
-                                                      head_dim, span, P);
-        if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PKV_EINVAL;
-    }
-
-    // the tensor-core kernel addresses the pool as one 2-D tensor of
-    // num_blocks * Hkv * block_size rows with 32-bit TMA coordinates
-    const bool mma_fits = dtype != PKV_F32 && G <= 16 &&
-                          (int64_t)num_blocks * num_kv_heads * block_size < (1ll << 31);
-    bool use_mma;
-    if (kernel == PKV_KERNEL_MMA) {
-        if (!kMmaBuilt || !mma_fits) return PKV_EUNSUPPORTED;
-        use_mma = true;
-    } else if (kernel == PKV_KERNEL_SIMT) {
-        use_mma = false;
-    } else {
-        use_mma = kMmaBuilt && mma_fits && G >= 4;
-    }
-    const int hg = use_mma ? (G <= 8 ? 8 : 16) : (G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1));
-    const int head_chunks = (G + hg - 1) / hg;
-    if ((int64_t)num_kv_heads * head_chunks > 65535) return PKV_EUNSUPPORTED;
-
-    DecodeArgs a;
-    a.out = out;
-    a.q = q;
-    a.k_cache = k_cache;
-    a.v_cache = v_cache;
-    a.block_tables = block_tables;
-    a.context_lens = context_lens;
-    a.seq_order = seq_order;
-    a.ws_o = static_cast<float*>(workspace);
-    a.ws_ml = np > 1 ? a.ws_o + (int64_t)num_seqs * num_q_heads * np * head_dim : nullptr;
-    a.num_seqs = num_seqs;
-    a.num_q_heads = num_q_heads;
-    a.num_kv_heads = num_kv_heads;
-    a.group = G;
-    a.head_chunks = head_chunks;
-    a.max_blocks_per_seq = max_blocks_per_seq;
-    a.num_blocks = num_blocks;
-    a.max_tokens = max_blocks_per_seq * block_size;
-    a.partition_size = P;
-    a.max_partitions = np;
-    a.block_size = block_size;
-    a.window = sliding_window;
-    a.scale_log2 = scale * 1.4426950408889634f;
-    if (status_word(&a.status) != cudaSuccess) return PKV_ECUDA;
-
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e;
-    if (use_mma) {
-        e = dtype == PKV_F16 ? decode_mma_f16(a, head_dim, block_size, hg, s)
-                             : decode_mma_bf16(a, head_dim, block_size, hg, s);
-    } else {
-        switch (dtype) {
-            case PKV_F32: e = decode_simt_f32(a, head_dim, block_size, hg, s); break;
-            case PKV_F16: e = decode_simt_f16(a, head_dim, block_size, hg, s); break;
-            default: e = decode_simt_bf16(a, head_dim, block_size, hg, s); break;
-        }
-    }
-    if (e == cudaErrorInvalidValue) return PKV_EUNSUPPORTED;
-    return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
+int pkv_paged_attention_decode_e4m3(void* out, const void* q, const void* k_cache,
+                                    const void* v_cache, const float* k_scale,
+                                    const float* v_scale, const int32_t* block_tables,
+                                    const int32_t* context_lens, const int32_t* seq_order,
+                                    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int max_blocks_per_seq, int num_blocks,
+                                    int max_context_len, float scale, int sliding_window,
+                                    pkv_dtype dtype, int partition_size, void* workspace,
+                                    size_t workspace_bytes, pkv_stream_t stream) {
+    return pkv::decode_impl(out, q, k_cache, v_cache, k_scale, v_scale, true, block_tables,
+                            context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
+                            head_dim, block_size, max_blocks_per_seq, num_blocks,
+                            max_context_len, scale, sliding_window, dtype, partition_size,
+                            workspace, workspace_bytes, PKV_KERNEL_SIMT, stream);
 }
 
 int pkv_kv_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
@@ -251,6 +298,28 @@ int pkv_kv_cache_append(void* k_cache, void* v_cache, const void* k, const void*
     cudaError_t e = launch_kv_append(k_cache, v_cache, k, v, slot_mapping, num_tokens,
                                      num_kv_heads, head_dim * es, block_size, num_blocks, st,
                                      reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+int pkv_kv_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, const void* v,
+                             const float* k_scale, const float* v_scale,
+                             const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                             int head_dim, int block_size, int num_blocks, pkv_dtype in_dtype,
+                             pkv_stream_t stream) {
+    if ((in_dtype != PKV_F16 && in_dtype != PKV_BF16) || num_tokens < 0 || num_kv_heads <= 0 ||
+        head_dim <= 0 || head_dim % 16 != 0 || block_size <= 0 || num_blocks <= 0)
+        return PKV_EINVAL;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !k || !v || !slot_mapping || !k_scale || !v_scale)
+        return PKV_EINVAL;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v))
+        return PKV_EINVAL;
+    unsigned int* st;
+    if (status_word(&st) != cudaSuccess) return PKV_ECUDA;
+    cudaError_t e = launch_kv_append_e4m3(k_cache, v_cache, k, v, k_scale, v_scale, slot_mapping,
+                                          num_tokens, num_kv_heads, head_dim, block_size,
+                                          num_blocks, in_dtype == PKV_BF16, st,
+                                          reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
 

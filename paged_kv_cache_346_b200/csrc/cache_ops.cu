@@ -6,6 +6,27 @@
 
 namespace pkv {
 
+// 16 fp16 / bf16 values (two 16-byte vectors) -> 16 E4M3 codes of x / scale.
+template <typename Tin>
+__device__ __forceinline__ uint4 quantise16(const uint4* src, float scale) {
+    float f[16];
+    Elem<Tin>::to_f32(src[0], f);
+    Elem<Tin>::to_f32(src[1], f + 8);
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t x = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const __nv_fp8_storage_t c =
+                __nv_cvt_float_to_fp8(f[4 * j + b] / scale, __NV_SATFINITE, __NV_E4M3);
+            x |= (uint32_t)c << (8 * b);
+        }
+        w[j] = x;
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // One thread per 16-byte vector of the new tokens' [T, Hkv, D] rows.
 // Token t's vector r (r < H * D * e / 16) lands in its slot's row: block
 // s / bs, KV head r / head_vecs, offset s % bs ("What is PagedAttention ..."
@@ -38,6 +59,37 @@ __global__ void __launch_bounds__(256) kv_append_kernel(uint4* __restrict__ kc,
         const uint4 vx = v[i];
         kc[dst] = kx;
         vc[dst] = vx;
+    }
+}
+
+// Quantising append: one thread per 16 elements of the new tokens' [T, Hkv, D]
+// rows (two 16-byte input vectors of fp16 / bf16, one 16-byte vector of
+// codes out).  code = E4M3(x / scale[h]): a correctly rounded float32
+// division, then the hardware conversion (nearest, ties to even, saturating
+// at the largest finite code).
+template <typename Tin>
+__global__ void __launch_bounds__(256) kv_append_e4m3_kernel(
+    uint4* __restrict__ kc, uint4* __restrict__ vc, const uint4* __restrict__ k,
+    const uint4* __restrict__ v, const float* __restrict__ ks, const float* __restrict__ vs,
+    const int64_t* __restrict__ slots, int64_t total_vecs, int row_vecs, int head_vecs,
+    int num_kv_heads, int block_size, int64_t num_slots, unsigned int* status) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total_vecs; i += stride) {
+        const int64_t t = i / row_vecs;
+        const int r = (int)(i - t * row_vecs);
+        const int64_t s = slots[t];
+        if (s < 0) continue;
+        if (s >= num_slots) {
+            if (r == 0) flag(status, PKV_DEV_BAD_SLOT);
+            continue;
+        }
+        const int h = r / head_vecs;
+        const int c = r - h * head_vecs;
+        const int64_t blk = s / block_size;
+        const int off = (int)(s - blk * block_size);
+        const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_vecs + c;
+        kc[dst] = quantise16<Tin>(k + 2 * i, ks[h]);
+        vc[dst] = quantise16<Tin>(v + 2 * i, vs[h]);
     }
 }
 
@@ -133,6 +185,26 @@ cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int32_t* pair
                                unsigned int* status, cudaStream_t stream) {
     return launch_move_pages<4>(k_cache, v_cache, k_cache, v_cache, pairs, num_pairs,
                                 block_bytes, num_blocks, num_blocks, status, stream);
+}
+
+cudaError_t launch_kv_append_e4m3(void* k_cache, void* v_cache, const void* k, const void* v,
+                                  const float* k_scale, const float* v_scale,
+                                  const int64_t* slots, int num_tokens, int num_kv_heads,
+                                  int head_dim, int block_size, int num_blocks, bool bf16_in,
+                                  unsigned int* status, cudaStream_t stream) {
+    const int head_vecs = head_dim / 16;
+    const int row_vecs = head_vecs * num_kv_heads;
+    const int64_t total = (int64_t)num_tokens * row_vecs;
+    if (total == 0) return cudaSuccess;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    auto kern = bf16_in ? kv_append_e4m3_kernel<__nv_bfloat16> : kv_append_e4m3_kernel<__half>;
+    kern<<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v), k_scale, v_scale, slots,
+        total, row_vecs, head_vecs, num_kv_heads, block_size, (int64_t)num_blocks * block_size,
+        status);
+    return cudaGetLastError();
 }
 
 }  // namespace pkv

@@ -11,6 +11,13 @@ cudaError_t launch_kv_append(void* k_cache, void* v_cache, const void* k, const 
                              int row_bytes_per_head, int block_size, int num_blocks,
                              unsigned int* status, cudaStream_t stream);
 
+// E4M3 pages from fp16 (bf16_in false) or bf16 rows; head_dim a multiple of 16.
+cudaError_t launch_kv_append_e4m3(void* k_cache, void* v_cache, const void* k, const void* v,
+                                  const float* k_scale, const float* v_scale,
+                                  const int64_t* slots, int num_tokens, int num_kv_heads,
+                                  int head_dim, int block_size, int num_blocks, bool bf16_in,
+                                  unsigned int* status, cudaStream_t stream);
+
 // block_bytes = num_kv_heads * block_size * head_dim * element size.
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs,
                                int num_pairs, int64_t block_bytes, int num_blocks,

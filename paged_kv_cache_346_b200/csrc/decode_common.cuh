@@ -18,6 +18,8 @@ struct DecodeArgs {
     const int32_t* block_tables;  // [B, max_blocks_per_seq]
     const int32_t* context_lens;  // [B]
     const int32_t* seq_order;     // [B] schedule order (CTA z takes sequence seq_order[z]), or null
+    const float* k_scale;         // [Hkv] scales of E4M3 K / V pages, or null
+    const float* v_scale;
     float* ws_o;                  // [B, Hq, max_partitions, D] partition outputs
     float* ws_ml;                 // [B, Hq, max_partitions, 2] (m in log2 units, l)
     unsigned int* status;

@@ -50,11 +50,14 @@ struct SimtStages {
 // STAGES_ = 0 picks the stage count by SimtStages; WS = true adds a
 // producer warp that re-arms each stage as soon as the consumer warps have
 // released it (per-stage "empty" mbarriers) instead of a CTA-wide barrier.
-template <typename T, int D, int BS, int HG, int NW, int STAGES_ = 0, bool WS = false>
+// TC is the page element type: T itself, or E4M3 codes with T = fp16/bf16
+// for q and out.
+template <typename T, int D, int BS, int HG, int NW, int STAGES_ = 0, bool WS = false,
+          typename TC = T>
 struct SimtCfg {
-    static constexpr int ROW = D * (int)sizeof(T);
+    static constexpr int ROW = D * Elem<TC>::kBytes;
     static constexpr int CPR = ROW / 16;
-    static constexpr int EPC = Elem<T>::kPerVec;
+    static constexpr int EPC = Elem<TC>::kPerVec;
     static constexpr int TILE = 16 * NW;
     static constexpr int BPT = TILE / BS;
     static constexpr int BLK_BYTES = BS * ROW;
@@ -75,9 +78,10 @@ struct SimtCfg {
 
 // One consumer warp's share of a partition: its q slice, online-softmax state
 // and accumulator, and the per-stage work on its 16 tokens.
-template <typename T, int D, int HG, typename C>
+template <typename T, int D, int HG, typename C, typename TC = T>
 struct SimtWarp {
-    using E = Elem<T>;
+    using E = Elem<TC>;   // pages
+    using EQ = Elem<T>;   // q and out
     static constexpr int ROW = C::ROW, EPC = C::EPC, CPL = C::CPL, LPV = C::LPV;
     static constexpr int TPV = C::TPV, CPV = C::CPV;
     static constexpr int NTV = 16 / TPV;  // tokens per lane in P.V
@@ -104,21 +108,27 @@ struct SimtWarp {
         else return *reinterpret_cast<const uint4*>(Vp + (tv + j * TPV) * ROW + (lv + c * LPV) * 16);
     }
 
-    __device__ __forceinline__ void init(const T* qb, int nh, float scale_log2, int lane_) {
+    // qscale: scale * log2(e), times the K pages' scale for quantised pages
+    __device__ __forceinline__ void init(const T* qb, int nh, float qscale, int lane_) {
         lane = lane_;
         grp = lane >> 3;
         sub = lane & 7;
         lv = lane % LPV;
         tv = lane / LPV;
+        constexpr int QV = EPC / EQ::kPerVec;  // 16-byte q vectors per page chunk
 #pragma unroll
         for (int hh = 0; hh < HG; ++hh) {
 #pragma unroll
             for (int i = 0; i < CPL; ++i) {
                 if (hh < nh) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(qb + hh * D + (sub + 8 * i) * EPC);
-                    E::to_f32(v, qf[hh][i]);
 #pragma unroll
-                    for (int e = 0; e < EPC; ++e) qf[hh][i][e] *= scale_log2;
+                    for (int u = 0; u < QV; ++u) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(
+                            qb + hh * D + (sub + 8 * i) * EPC + u * EQ::kPerVec);
+                        EQ::to_f32(v, qf[hh][i] + u * EQ::kPerVec);
+                    }
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) qf[hh][i][e] *= qscale;
                 } else {
 #pragma unroll
                     for (int e = 0; e < EPC; ++e) qf[hh][i][e] = 0.f;
@@ -228,11 +238,20 @@ struct SimtWarp {
     }
 
     // Fold the token lanes together and park (m, l, acc) in the merge area.
+    // vscale: the V pages' scale for quantised pages (else 1)
     template <int NW>
-    __device__ __forceinline__ void park(int warp, float* red) {
+    __device__ __forceinline__ void park(int warp, float* red, float vscale) {
         using A = MergeArea<D, HG, NW>;
         float* red_m = red + NW * HG * A::RP;
         float* red_l = red_m + NW * HG;
+        if (vscale != 1.f) {
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+                for (int c = 0; c < CPV; ++c)
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) acc[hh][c][e] *= vscale;
+        }
 #pragma unroll
         for (int msk = LPV; msk < 32; msk <<= 1)
 #pragma unroll
@@ -264,11 +283,11 @@ struct SimtWarp {
     }
 };
 
-template <typename T, int D, int BS, int HG, int NW, int STAGES_, bool WS>
-__global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREADS,
-                                  SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::ROW <= 256 ? 3 : 1)
+template <typename T, int D, int BS, int HG, int NW, int STAGES_, bool WS, typename TC>
+__global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::THREADS,
+                                  SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::ROW <= 256 ? 3 : 1)
     decode_simt_kernel(const DecodeArgs a) {
-    using C = SimtCfg<T, D, BS, HG, NW, STAGES_, WS>;
+    using C = SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>;
     using E = Elem<T>;
     constexpr int ROW = C::ROW, TILE = C::TILE, BPT = C::BPT;
     constexpr int BLK_BYTES = C::BLK_BYTES, STAGE_BYTES = C::STAGE_BYTES;
@@ -374,9 +393,9 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREAD
     }
 
     // 3.-5. consumer warps
-    SimtWarp<T, D, HG, C> W;
+    SimtWarp<T, D, HG, C, TC> W;
     W.init(reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D, nh,
-           a.scale_log2, lane);
+           a.k_scale ? a.scale_log2 * a.k_scale[kvh] : a.scale_log2, lane);
     const uint64_t pol = WS ? 0 : policy_evict_first();
     for (int it = 0; it < ntiles; ++it) {
         const int stage = it % STAGES;
@@ -406,17 +425,18 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS>::THREAD
     if (!WS) pdl_launch_dependents();
 
     // 6. merge the warps
-    W.template park<NW>(warp, red);
+    W.template park<NW>(warp, red, a.v_scale ? a.v_scale[kvh] : 1.f);
     __syncthreads();
     merge_warps_and_store<T, D, HG, NW>(a, red, b, h0, nh, part, np, tid, WS ? THREADS : NW * 32);
 }
 
-template <typename T, int D, int BS, int HG, int NW = 4, int STAGES = 0, bool WS = false>
+template <typename T, int D, int BS, int HG, int NW = 4, int STAGES = 0, bool WS = false,
+          typename TC = T>
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
-    using C = SimtCfg<T, D, BS, HG, NW, STAGES, WS>;
+    using C = SimtCfg<T, D, BS, HG, NW, STAGES, WS, TC>;
     static SmemAttr attr;
     const int smem_simt = C::smem_bytes(a.partition_size);
-    auto kern = decode_simt_kernel<T, D, BS, HG, NW, STAGES, WS>;
+    auto kern = decode_simt_kernel<T, D, BS, HG, NW, STAGES, WS, TC>;
     cudaError_t e = attr.ensure(kern, C::smem_bytes(8192));
     if (e != cudaSuccess) return e;
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "pagedkv.h"
@@ -102,12 +103,18 @@ __device__ __forceinline__ void pdl_wait_primary() {
 
 // ---- element types --------------------------------------------------------
 
+// FP8 E4M3 codes (one byte each), the storage of quantised pages.
+struct E4M3 {
+    uint8_t bits;
+};
+
 template <typename T>
 struct Elem;
 
 template <>
 struct Elem<float> {
     static constexpr int kPerVec = 4;  // elements per 16-byte vector
+    static constexpr int kBytes = 4;
     __device__ __forceinline__ static void to_f32(const uint4& v, float* f) {
         f[0] = __uint_as_float(v.x);
         f[1] = __uint_as_float(v.y);
@@ -121,6 +128,7 @@ struct Elem<float> {
 template <>
 struct Elem<__half> {
     static constexpr int kPerVec = 8;
+    static constexpr int kBytes = 2;
     __device__ __forceinline__ static void to_f32(const uint4& v, float* f) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -138,6 +146,7 @@ struct Elem<__half> {
 template <>
 struct Elem<__nv_bfloat16> {
     static constexpr int kPerVec = 8;
+    static constexpr int kBytes = 2;
     __device__ __forceinline__ static void to_f32(const uint4& v, float* f) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -152,6 +161,27 @@ struct Elem<__nv_bfloat16> {
     }
     __device__ __forceinline__ static float load1(const __nv_bfloat16* p) {
         return __bfloat162float(*p);
+    }
+};
+
+template <>
+struct Elem<E4M3> {
+    static constexpr int kPerVec = 16;
+    static constexpr int kBytes = 1;
+    // 16 codes -> 16 floats (exact: every E4M3 value is a binary16 value)
+    __device__ __forceinline__ static void to_f32(const uint4& v, float* f) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
+                    (__nv_fp8x2_storage_t)((w[i] >> (16 * j)) & 0xffffu), __NV_E4M3);
+                const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&r));
+                f[4 * i + 2 * j] = t.x;
+                f[4 * i + 2 * j + 1] = t.y;
+            }
+        }
     }
 };
 

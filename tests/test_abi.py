@@ -104,6 +104,50 @@ def test_append_and_copy_host_checks():
     assert g(None, None, None, -1, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL
 
 
+def _decode_e4m3(**over):
+    a = dict(out=None, q=None, k=None, v=None, ks=None, vs=None, bt=None, cl=None, order=None,
+             B=4, Hq=8, Hkv=2, D=128, bs=16, mb=8, N=64, maxlen=100, scale=0.1, win=0,
+             dt=b.PKV_F16, P=0, ws=None, wsb=0, stream=None)
+    a.update(over)
+    return b.lib.pkv_paged_attention_decode_e4m3(
+        a["out"], a["q"], a["k"], a["v"], a["ks"], a["vs"], a["bt"], a["cl"], a["order"], a["B"],
+        a["Hq"], a["Hkv"], a["D"], a["bs"], a["mb"], a["N"], a["maxlen"], a["scale"], a["win"],
+        a["dt"], a["P"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(dt=b.PKV_F32), b.PKV_EINVAL),                 # q / out must be 16-bit
+    (dict(dt=b.PKV_E4M3), b.PKV_EINVAL),
+    (dict(D=64), b.PKV_EUNSUPPORTED),                   # 64-byte rows
+    (dict(Hq=6, Hkv=4), b.PKV_EINVAL),
+    (dict(), b.PKV_EINVAL),                             # null pointers
+    (dict(B=0), b.PKV_OK),
+])
+def test_decode_e4m3_host_checks(over, code):
+    assert _decode_e4m3(**over) == code
+
+
+def test_e4m3_pages_need_their_own_entry():
+    # the 16-bit decode refuses E4M3 pages (they need scales)
+    assert _decode(dt=b.PKV_E4M3) == b.PKV_EINVAL
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the scale check fails first
+    assert _decode_e4m3(out=fake, q=fake, k=fake, v=fake, bt=fake, cl=fake) == b.PKV_EINVAL
+
+
+def test_append_e4m3_host_checks():
+    f = b.lib.pkv_kv_cache_append_e4m3
+    args = [None] * 7
+    assert f(*args, 0, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_OK
+    assert f(*args, 3, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL   # null pointers
+    assert f(*args, 0, 4, 120, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL   # head_dim % 16
+    assert f(*args, 0, 4, 128, 16, 10, b.PKV_F32, None) == b.PKV_EINVAL   # input type
+    assert f(*args, 0, 4, 128, 16, 10, b.PKV_E4M3, None) == b.PKV_EINVAL
+    # E4M3 pools move as bytes through the plain cache operations
+    g = b.lib.pkv_copy_blocks
+    assert g(None, None, None, 0, 4, 128, 16, 10, b.PKV_E4M3, None) == b.PKV_OK
+    assert g(None, None, None, 0, 1, 8, 1, 10, b.PKV_E4M3, None) == b.PKV_EINVAL  # 8-byte blocks
+
+
 def test_schedule_order_longest_first():
     import numpy as np
     import paged_kv_cache_346_b200 as pkv

@@ -26,8 +26,8 @@ from dataclasses import dataclass, field, replace
 import numpy as np
 
 DTYPES = ("f32", "f16", "bf16")
-DTYPE_CODE = {"f32": 0, "f16": 1, "bf16": 2}
-ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
+DTYPE_CODE = {"f32": 0, "f16": 1, "bf16": 2, "e4m3": 3}
+ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2, "e4m3": 1}
 
 # numbers drawn per generator chunk; fixed so results do not depend on the
 # number of threads used to draw them
@@ -249,14 +249,16 @@ def make_decode_inputs(cfg: DecodeConfig, seed: int = 0, *, shuffle: bool = True
     return DecodeInputs(cfg, q, k, v, tables, lens, num_blocks)
 
 
-def kv_bytes_per_token(cfg: DecodeConfig) -> int:
-    return 2 * cfg.num_kv_heads * cfg.head_dim * ELEM_BYTES[cfg.dtype]
+def kv_bytes_per_token(cfg: DecodeConfig, kv_dtype: str | None = None) -> int:
+    return 2 * cfg.num_kv_heads * cfg.head_dim * ELEM_BYTES[kv_dtype or cfg.dtype]
 
 
-def algorithmic_bytes(cfg: DecodeConfig, lens: np.ndarray, window: int = 0) -> int:
+def algorithmic_bytes(cfg: DecodeConfig, lens: np.ndarray, window: int = 0,
+                      kv_dtype: str | None = None) -> int:
     """Bytes a decode step must move at least once: K and V of every attended
     token (the last `window` of each sequence when window > 0), q in and out,
-    the block-table entries used and the lengths."""
+    the block-table entries used and the lengths (and the per-head scales of
+    quantised pages, kv_dtype "e4m3")."""
     e = ELEM_BYTES[cfg.dtype]
     lens = np.asarray(lens, dtype=np.int64)
     if window > 0:
@@ -266,10 +268,69 @@ def algorithmic_bytes(cfg: DecodeConfig, lens: np.ndarray, window: int = 0) -> i
     else:
         att = lens
         nblk = blocks_needed(lens, cfg.block_size)
-    kv = int(att.sum()) * kv_bytes_per_token(cfg)
+    kv = int(att.sum()) * kv_bytes_per_token(cfg, kv_dtype)
     qo = 2 * lens.size * cfg.num_q_heads * cfg.head_dim * e
     tab = int(nblk.sum()) * 4
-    return kv + qo + tab + 4 * lens.size
+    scales = 8 * cfg.num_kv_heads if kv_dtype == "e4m3" else 0
+    return kv + qo + tab + 4 * lens.size + scales
+
+
+# ---------------------------------------------------------------------------
+# quantised (FP8 E4M3) pages
+
+# Codes: sign uniform, the other 7 bits uniform over [0, E4M3_TOP] (exponent
+# field <= 12, magnitudes below 64; no NaN), drawn from seeded PCG64 chunks
+# like normal_fill.  Scales: one per KV head for K and for V, uniform in
+# [1/64, 1/16], so the stored values span about +-4.
+E4M3_TOP = 0x67
+
+
+def e4m3_codes(shape, seed: int, threads: int = 8) -> np.ndarray:
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint8)
+    nchunks = (n + _CHUNK - 1) // _CHUNK
+    seeds = np.random.SeedSequence(seed).spawn(max(nchunks, 1))
+
+    def work(i):
+        lo = i * _CHUNK
+        hi = min(n, lo + _CHUNK)
+        g = np.random.Generator(np.random.PCG64(seeds[i]))
+        mag = g.integers(0, E4M3_TOP + 1, size=hi - lo, dtype=np.uint8)
+        sign = g.integers(0, 2, size=hi - lo, dtype=np.uint8) << np.uint8(7)
+        out[lo:hi] = mag | sign
+
+    if nchunks <= 1:
+        for i in range(nchunks):
+            work(i)
+    else:
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(work, range(nchunks)))
+    return out.reshape(shape)
+
+
+def e4m3_scales(num_kv_heads: int, seed: int) -> tuple[np.ndarray, np.ndarray]:
+    g = rng(seed * 1000 + 11)
+    ks = g.uniform(1 / 64, 1 / 16, size=num_kv_heads).astype(np.float32)
+    vs = g.uniform(1 / 64, 1 / 16, size=num_kv_heads).astype(np.float32)
+    return ks, vs
+
+
+@dataclass
+class QuantisedPages:
+    k_cache: np.ndarray   # uint8 E4M3 codes [N, Hkv, bs, D]
+    v_cache: np.ndarray
+    k_scale: np.ndarray   # float32 [Hkv]
+    v_scale: np.ndarray
+
+
+def make_e4m3_pages(inp: "DecodeInputs", seed: int = 0, threads: int = 8) -> QuantisedPages:
+    """E4M3 pages of the same shape as inp's caches (same tables and lengths;
+    inp.q stays the query)."""
+    shape = inp.k_cache.shape
+    k = e4m3_codes(shape, seed * 1000 + 14, threads)
+    v = e4m3_codes(shape, seed * 1000 + 15, threads)
+    ks, vs = e4m3_scales(shape[1], seed)
+    return QuantisedPages(k, v, ks, vs)
 
 
 # ---------------------------------------------------------------------------
