@@ -147,6 +147,8 @@ KERNEL_SOURCES = {
     "simt": ("decode_common.cuh", "decode_simt.cuh", "device_common.cuh"),
     "mma": ("decode_common.cuh", "decode_mma.cuh", "device_common.cuh"),
     "simt_e4m3": ("decode_common.cuh", "decode_simt.cuh", "device_common.cuh"),
+    "mma_e4m3": ("decode_common.cuh", "decode_mma.cuh", "decode_mma_e4m3.cuh",
+                 "device_common.cuh"),
 }
 
 
@@ -162,6 +164,8 @@ def kernel_source_digest(variant: str) -> str:
 def resolve_variant(cfg, kernel: str, kv: str = "same") -> str:
     """The decode kernel the library's automatic choice takes for cfg."""
     if kv == "e4m3":
+        if kernel == "mma" or (kernel == "auto" and cfg.group <= 16):
+            return "mma_e4m3"
         return "simt_e4m3"
     if kernel != "auto":
         return kernel
@@ -306,8 +310,8 @@ def run_ours(args, cfg):
     # ---- inputs (seeded; each rank its own replica)
     inp = make_decode_inputs(cfg, seed=args.seed + rank)
     e4m3 = args.kv == "e4m3"
-    if e4m3 and (cfg.dtype == "f32" or args.kernel == "mma"):
-        raise SystemExit("E4M3 pages take fp16/bf16 q and the CUDA-core kernel")
+    if e4m3 and cfg.dtype == "f32":
+        raise SystemExit("E4M3 pages take fp16/bf16 q")
 
     def dev(a):
         if cfg.dtype == "bf16" and a.dtype == np.uint16:
@@ -362,7 +366,7 @@ def run_ours(args, cfg):
             pkv.pkv_paged_attention_decode_e4m3(out, q, kc, vc, ks, vs, bt, cl, cfg.scale, bs,
                                                 mcl, partition_size=P, workspace=ws,
                                                 seq_order=order, sliding_window=W,
-                                                stream=stream)
+                                                kernel=kern, stream=stream)
         else:
             pkv.pkv_paged_attention_decode(out, q, kc, vc, bt, cl, cfg.scale, bs, mcl,
                                            partition_size=P, workspace=ws, seq_order=order,
@@ -451,7 +455,7 @@ def run_ours(args, cfg):
             decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ksp, vsp,
                            ptr["bt"], ptr["cl"], ptr.get("order"), B, cfg.num_q_heads, H, D,
                            bs, bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
-                           ctypes.c_void_p(ws.data_ptr()), ws.numel(), c_stream)
+                           ctypes.c_void_p(ws.data_ptr()), ws.numel(), kern, c_stream)
         else:
             append_args = (kp, vp, ptr["knew"], ptr["vnew"], ptr["slots"], B, H, D, bs,
                            N_blocks, dt_code, c_stream)

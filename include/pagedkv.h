@@ -81,7 +81,8 @@ typedef enum {
 typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2, PKV_E4M3 = 3 } pkv_dtype;
 
 /* Decode kernel choice.  AUTO takes the tensor-core kernel for 16-bit caches
- * with a query group of 4 or more heads per KV head, else the CUDA-core one. */
+ * with a query group of 4 to 16 heads per KV head and for E4M3 pages with a
+ * group of at most 16, else the CUDA-core one. */
 typedef enum { PKV_KERNEL_AUTO = 0, PKV_KERNEL_SIMT = 1, PKV_KERNEL_MMA = 2 } pkv_kernel;
 
 /* Device status bits (pkv_device_status) */
@@ -180,8 +181,14 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
  * is pkv_paged_attention_decode's over those values:
  *   out[b,h,:] = softmax_t(scale * k_scale[g] * q[b,h,:] . E4M3(k_t))
  *                weighted sum of v_scale[g] * E4M3(v_t),   g = h / (Hq/Hkv).
- * The kernel folds k_scale into q and v_scale into the float32 accumulator;
- * each code is widened exactly (every E4M3 value is a binary16 value).
+ * Each code is widened exactly (every E4M3 value is a binary16 value).  The
+ * tensor-core kernel (AUTO for groups of at most 16 heads) multiplies fp16
+ * operands with fp32 accumulation: q enters it scaled by a power of two that
+ * puts max |q| of the CTA's heads in [2^14, 2^15) (exact unless an element
+ * falls below the fp16 normal range there), P is rounded to fp16, and the
+ * logits are multiplied by scale * k_scale (and the power of two) in fp32.
+ * The CUDA-core kernel works in fp32 throughout, k_scale folded into q and
+ * v_scale into the accumulator.
  *
  * Arguments as pkv_paged_attention_decode, plus:
  *   k_cache, v_cache: device E4M3 codes [num_blocks, Hkv, block_size, head_dim].
@@ -189,8 +196,9 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
  *       checked on the device: the caller's quantisation scales).
  *   dtype: PKV_F16 or PKV_BF16, the type of q and out.
  *   head_dim in {128, 256} (a page row must be at least 128 bytes).
- *   Always the CUDA-core kernel.  The workspace is sized as for the 16-bit
- *   decode (pkv_decode_workspace_size).
+ *   kernel: PKV_KERNEL_AUTO, SIMT or MMA (MMA: groups of at most 16 heads).
+ *   The workspace is sized as for the 16-bit decode
+ *   (pkv_decode_workspace_size).
  * Returns PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED or PKV_ECUDA.
  */
 PKV_API int pkv_paged_attention_decode_e4m3(
@@ -199,7 +207,7 @@ PKV_API int pkv_paged_attention_decode_e4m3(
     const int32_t* seq_order, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
     int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
     int sliding_window, pkv_dtype dtype, int partition_size, void* workspace,
-    size_t workspace_bytes, pkv_stream_t stream);
+    size_t workspace_bytes, pkv_kernel kernel, pkv_stream_t stream);
 
 /*
  * Size of the workspace compiled into the library for

@@ -130,7 +130,8 @@ def pkv_paged_attention_decode_e4m3(out: torch.Tensor, q: torch.Tensor, k_cache:
                                     max_context_len: int, *, partition_size: int = 0,
                                     workspace: torch.Tensor | None = None,
                                     seq_order: torch.Tensor | None = None,
-                                    sliding_window: int = 0, stream=None) -> torch.Tensor:
+                                    sliding_window: int = 0, kernel: int = PKV_KERNEL_AUTO,
+                                    stream=None) -> torch.Tensor:
     """Paged decode over FP8 E4M3 pages (pkv_paged_attention_decode_e4m3 in
     pagedkv.h): k_cache/v_cache torch.float8_e4m3fn [N, Hkv, block_size, D];
     k_scale/v_scale float32 [Hkv]; q and out fp16 or bf16."""
@@ -162,7 +163,7 @@ def pkv_paged_attention_decode_e4m3(out: torch.Tensor, q: torch.Tensor, k_cache:
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
         _ptr(block_tables), _ptr(context_lens), _ptr(seq_order), B, Hq, Hkv, D, bs,
         block_tables.shape[1], N, int(max_context_len), float(scale), int(sliding_window),
-        torch_dtype_code(q.dtype), int(partition_size), _ptr(workspace), ws_bytes,
+        torch_dtype_code(q.dtype), int(partition_size), _ptr(workspace), ws_bytes, int(kernel),
         _stream(stream)),
         "pkv_paged_attention_decode_e4m3")
     return out

@@ -9,6 +9,7 @@
 #include "cache_ops.cuh"
 #include "decode_dispatch.cuh"
 #include "decode_mma.cuh"
+#include "decode_mma_e4m3.cuh"
 
 namespace pkv {
 
@@ -107,7 +108,6 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     if (block_size != 16 && block_size != 32 && block_size != 64) return PKV_EUNSUPPORTED;
     if (dtype == PKV_F32 && head_dim == 256) return PKV_EUNSUPPORTED;
     if (e4m3 && head_dim == 64) return PKV_EUNSUPPORTED;
-    if (e4m3 && kernel == PKV_KERNEL_MMA) return PKV_EUNSUPPORTED;
     if (num_seqs == 0) return PKV_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_EINVAL;
     if (e4m3 && (!k_scale || !v_scale)) return PKV_EINVAL;
@@ -132,7 +132,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
 
     // the tensor-core kernel addresses the pool as one 2-D tensor of
     // num_blocks * Hkv * block_size rows with 32-bit TMA coordinates
-    const bool mma_fits = !e4m3 && dtype != PKV_F32 && G <= 16 &&
+    const bool mma_fits = dtype != PKV_F32 && G <= 16 &&
                           (int64_t)num_blocks * num_kv_heads * block_size < (1ll << 31);
     bool use_mma;
     if (kernel == PKV_KERNEL_MMA) {
@@ -141,7 +141,9 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     } else if (kernel == PKV_KERNEL_SIMT) {
         use_mma = false;
     } else {
-        use_mma = kMmaBuilt && mma_fits && G >= 4;
+        // E4M3 pages: the tensor cores for every group size (the conversions
+        // would bound the CUDA-core kernel below the memory roofline)
+        use_mma = kMmaBuilt && mma_fits && (G >= 4 || e4m3);
     }
     const int hg = use_mma ? (G <= 8 ? 8 : 16)
                            : (G % 4 == 0 && !e4m3 ? 4 : (G % 2 == 0 ? 2 : 1));
@@ -177,7 +179,10 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (e4m3) {
+    if (e4m3 && use_mma) {
+        e = dtype == PKV_F16 ? decode_mma_e4m3_f16(a, head_dim, block_size, hg, s)
+                             : decode_mma_e4m3_bf16(a, head_dim, block_size, hg, s);
+    } else if (e4m3) {
         e = dtype == PKV_F16 ? decode_simt_e4m3_f16(a, head_dim, block_size, hg, s)
                              : decode_simt_e4m3_bf16(a, head_dim, block_size, hg, s);
     } else if (use_mma) {
@@ -273,12 +278,13 @@ int pkv_paged_attention_decode_e4m3(void* out, const void* q, const void* k_cach
                                     int block_size, int max_blocks_per_seq, int num_blocks,
                                     int max_context_len, float scale, int sliding_window,
                                     pkv_dtype dtype, int partition_size, void* workspace,
-                                    size_t workspace_bytes, pkv_stream_t stream) {
+                                    size_t workspace_bytes, pkv_kernel kernel,
+                                    pkv_stream_t stream) {
     return pkv::decode_impl(out, q, k_cache, v_cache, k_scale, v_scale, true, block_tables,
                             context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
                             head_dim, block_size, max_blocks_per_seq, num_blocks,
                             max_context_len, scale, sliding_window, dtype, partition_size,
-                            workspace, workspace_bytes, PKV_KERNEL_SIMT, stream);
+                            workspace, workspace_bytes, kernel, stream);
 }
 
 int pkv_kv_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,

@@ -14,8 +14,9 @@ std::once_flag g_encode_once;
 }  // namespace
 
 // The pool viewed as a 2-D tensor: `rows` = num_blocks * Hkv * BS rows of
-// head_dim 16-bit elements; boxes of 64 columns x box_rows rows, 128-byte
-// swizzle (the layout the kernel's ldmatrix addressing assumes).
+// head_dim elements (2 bytes: f16 / bf16, 1 byte: E4M3 codes as uint8); boxes
+// of 128 bytes x box_rows rows, 128-byte swizzle (the layout the kernels'
+// ldmatrix addressing assumes).
 cudaError_t make_cache_tensor_map(CUtensorMap* map, const void* base, int dtype_bytes,
                                   bool bf16, int head_dim, int64_t rows, int box_rows) {
     std::call_once(g_encode_once, [] {
@@ -29,10 +30,14 @@ cudaError_t make_cache_tensor_map(CUtensorMap* map, const void* base, int dtype_
     if (!g_encode) return cudaErrorNotSupported;
     const cuuint64_t gdim[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
     const cuuint64_t gstride[1] = {(cuuint64_t)head_dim * dtype_bytes};
-    const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    const cuuint32_t box[2] = {128u / (cuuint32_t)dtype_bytes, (cuuint32_t)box_rows};
     const cuuint32_t estride[2] = {1u, 1u};
+    const CUtensorMapDataType dt = dtype_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : bf16           ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (dtype_bytes != 1 && dtype_bytes != 2) return cudaErrorInvalidValue;
     const CUresult r = g_encode(
-        map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+        map, dt, 2,
         const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

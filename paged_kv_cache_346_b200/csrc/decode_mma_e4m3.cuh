@@ -1,0 +1,417 @@
+// Paged decode attention over FP8 E4M3 pages on the tensor cores.
+//
+// The same two contractions as the 16-bit tensor-core kernel,
+//   S[h, t] = sum_d Q[h, d] K[t, d]        O^T[d, h] = sum_t V[t, d] P[h, t],
+// with mma.sync m16n8k16 in fp16 (fp32 accumulation).  The pages stay one
+// byte per element all the way into the registers: ldmatrix moves 16-byte
+// rows of codes, and each register of four codes becomes two f16x2 operand
+// registers with the hardware E4M3 -> f16x2 conversion (exact: every E4M3
+// value is an f16 value).  Quantised pages are the paged layout combined with
+// a compressed cache ("pagedattention vllm" §Comparison with Alternatives).
+//
+// Operand layouts (the contraction order is free, so the byte layout that
+// ldmatrix delivers is kept and the other operand is arranged to match):
+//   * K as the B operand of S: ldmatrix (non-transposed) hands lane (g, t4)
+//     the codes K[t = g][4 t4 .. 4 t4 + 3] of a 16-dim step.  The low pair
+//     serves logical k = 2 t4, 2 t4 + 1, the high pair k = 2 t4 + 8, + 9, so
+//     Q's A fragment takes dims 4 t4, 4 t4 + 1 and 4 t4 + 2, 4 t4 + 3 at those
+//     positions.
+//   * V^T as the A operand of O^T: ldmatrix.trans on 2-byte units hands lane
+//     (g, t4) the codes V[2 t4][2 g], V[2 t4][2 g + 1], V[2 t4 + 1][2 g],
+//     V[2 t4 + 1][2 g + 1].  One byte permute makes the token pairs of dims
+//     2 g and 2 g + 1: A rows g and g + 8 of an m-tile are dims 2 g and 2 g + 1
+//     of its 16, and the tokens (k) keep their natural order, so P^T comes
+//     straight from the S accumulators as in the 16-bit kernel.
+//
+// q (fp16 or bf16) enters the fp16 MMA multiplied by a power of two 2^e that
+// puts its largest magnitude in [2^14, 2^15) (exact for every value that stays
+// an f16 normal); the logits are multiplied back by scale * log2(e) *
+// k_scale * 2^-e in fp32, and the output by v_scale.
+#pragma once
+
+#include "decode_mma.cuh"
+
+namespace pkv {
+
+// STAGES_ = 0: four stages when K + V fit 72 KB per CTA (head_dim 128: three
+// CTAs per SM), else three (the merge area of 16 heads needs that much).
+template <int D, int BS, int NW, int STAGES_ = 0>
+struct MmaE4m3Cfg {
+    static constexpr int TILE = 16 * NW;        // tokens per stage
+    static constexpr int NX = D / 128;          // 128-column boxes per row
+    static constexpr int BOX_BYTES = BS * 128;  // one box: BS rows x 128 bytes
+    static constexpr int BLK_BYTES = BS * D;    // one (block, head) page
+    static constexpr int BPT = TILE / BS;
+    static constexpr int STAGE_BYTES = TILE * D;  // one of K / V
+    static constexpr int FIT = 73728 / (2 * STAGE_BYTES);
+    static constexpr int STAGES = STAGES_ ? STAGES_ : (FIT >= 4 ? 4 : 3);
+    static_assert(TILE % BS == 0 && BS % 8 == 0 && D % 128 == 0, "whole blocks, 128-byte rows");
+
+    static int smem_bytes(int partition_size) {
+        return 1024 + round_up(partition_size / BS * 4, 128) + 1024 + STAGES * 2 * STAGE_BYTES;
+    }
+};
+
+// four E4M3 codes (bytes 0..3) -> f16x2 of bytes 0, 1 (lo) and of bytes 2, 3
+// (hi); the lower byte of each pair goes to the lower half
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
+
+__device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(x), "r"(sel));
+    return r;
+}
+
+template <typename T, int D, int BS, int NH, int NW, int STAGES_>
+__global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
+    decode_mma_e4m3_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
+                           const __grid_constant__ CUtensorMap tmv) {
+    using C = MmaE4m3Cfg<D, BS, NW, STAGES_>;
+    using M = Mma<__half>;
+    constexpr int TILE = C::TILE, NX = C::NX, BOX_BYTES = C::BOX_BYTES;
+    constexpr int BLK_BYTES = C::BLK_BYTES, BPT = C::BPT, STAGE_BYTES = C::STAGE_BYTES;
+    constexpr int STAGES = C::STAGES;
+    constexpr int KSTEPS = D / 16;   // k-steps of QK, m-tiles of PV (one 16-byte chunk each)
+    constexpr int KP = KSTEPS / 2;   // ldmatrix.x4 loads per warp tile (two chunks each)
+    constexpr int RB = NH / 8;
+    constexpr bool EARLY = D <= 128 && NH == 8;
+
+    extern __shared__ __align__(1024) unsigned char smem_mma8[];
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int kvh = blockIdx.y / a.head_chunks;
+    const int hc = blockIdx.y - kvh * a.head_chunks;
+    const int part = blockIdx.x;
+    const int h0 = kvh * a.group + hc * NH;
+    const int nh = min(NH, a.group - hc * NH);
+    const bool reporter = (tid == 0 && part == 0 && blockIdx.y == 0);
+    const int b = scheduled_seq(a, blockIdx.z, reporter);
+    if (b < 0) return;
+
+    const TablePrefetch pf = table_prefetch(a, b, part, a.partition_size / BS, tid);
+    const Span sp = seq_span(a, b, reporter);
+    const int L = sp.L, np = sp.np;
+    T* out = reinterpret_cast<T*>(a.out);
+    if (L == 0) {
+        if (part == 0)
+            for (int i = tid; i < nh * D; i += NW * 32)
+                out[((int64_t)b * a.num_q_heads + h0 + i / D) * D + i % D] = Elem<T>::from_f32(0.f);
+        return;
+    }
+    if (part >= np) return;
+
+    const int P = a.partition_size;
+    const int t0 = sp.base + part * P;
+    const int ntok = min(L, t0 + P) - t0;
+    const int mask_lo = part == 0 ? sp.lo - sp.base : 0;
+    const int ntiles = (ntok + TILE - 1) / TILE;
+    const int nblk = (ntok + BS - 1) / BS;
+
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem_mma8);
+    int32_t* s_tab = reinterpret_cast<int32_t*>(smem_mma8 + 1024);
+    unsigned char* s_kv;
+    {
+        const uint32_t base = smem_u32(smem_mma8 + 1024 + round_up(P / BS * 4, 128));
+        const uint32_t aligned = (base + 1023u) & ~1023u;  // 128-byte swizzle: 1 KB atoms
+        s_kv = smem_mma8 + 1024 + round_up(P / BS * 4, 128) + (aligned - base);
+    }
+
+    table_hoist(a, b, t0 / BS, nblk, pf, s_tab, tid, NW * 32);
+    if (tid == 0) {
+        s_abort = 0;
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    const uint64_t pol = policy_evict_first();
+    auto issue = [&](int tile, int stage) {
+        const int jb = tile * BPT;
+        const int je = min(nblk, jb + BPT);
+        mbar_arrive_expect_tx(&full[stage], (uint32_t)((je - jb) * BLK_BYTES * 2));
+        unsigned char* kd = s_kv + stage * 2 * STAGE_BYTES;
+        unsigned char* vd = kd + STAGE_BYTES;
+        for (int j = jb; j < je; ++j) {
+            const int y = (s_tab[j] * a.num_kv_heads + kvh) * BS;
+#pragma unroll
+            for (int x = 0; x < NX; ++x) {
+                const int off = ((j - jb) * NX + x) * BOX_BYTES;
+                tma_load_2d(kd + off, &tmk, x * 128, y, &full[stage], pol);
+                tma_load_2d(vd + off, &tmv, x * 128, y, &full[stage], pol);
+            }
+        }
+    };
+    if (tid == 0) {
+        const int pre = min(STAGES, ntiles);
+        for (int s = 0; s < pre; ++s) issue(s, s);
+    }
+
+    // Q as the A operand (rows = heads g, g + 8), dims in the order the K
+    // codes arrive: k = 2 t4 + j -> dim 4 t4 + j, k = 2 t4 + 8 + j -> 4 t4 + 2 + j.
+    uint32_t qa[KSTEPS][4];
+    float qmul;  // logits multiplier: scale * log2(e) * k_scale * 2^-e
+    {
+        const T* qb = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D;
+        float qf[KSTEPS][2][4];
+        float mx = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int hh = g + 8 * r;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) qf[ks][r][j] = 0.f;
+                if (hh < nh) {
+                    const T* src = qb + hh * D + ks * 16 + 4 * t4;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        qf[ks][r][j] = Elem<T>::load1(src + j);
+                        mx = fmaxf(mx, fabsf(qf[ks][r][j]));
+                    }
+                }
+            }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        // 2^e with mx * 2^e in [2^14, 2^15): e = 141 - biased exponent of mx
+        const int be = (__float_as_int(mx) >> 23) & 0xff;
+        int e = be == 0 ? 0 : 141 - be;
+        e = max(-126, min(126, e));
+        const float up = __int_as_float((127 + e) << 23);
+        const float down = __int_as_float((127 - e) << 23);
+        qmul = a.scale_log2 * a.k_scale[kvh] * down;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const __half2 lo = __floats2half2_rn(qf[ks][r][0] * up, qf[ks][r][1] * up);
+                const __half2 hi = __floats2half2_rn(qf[ks][r][2] * up, qf[ks][r][3] * up);
+                qa[ks][r] = *reinterpret_cast<const uint32_t*>(&lo);      // a0a1 / a2a3
+                qa[ks][2 + r] = *reinterpret_cast<const uint32_t*>(&hi);  // a4a5 / a6a7
+            }
+    }
+
+    float m[RB], l[RB];
+    float o[KSTEPS][RB][4];
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) {
+        m[rb] = -INFINITY;
+        l[rb] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[mt][rb][i] = 0.f;
+    }
+
+    // ldmatrix.x4 row addresses: matrices (tokens 0-7, chunk c), (tokens 8-15,
+    // chunk c), (tokens 0-7, chunk c + 1), (tokens 8-15, chunk c + 1)
+    const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1);
+    const int lchunk = lane >> 4;
+
+    for (int it = 0; it < ntiles; ++it) {
+        const int stage = it % STAGES;
+        const bool ok = mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status);
+        if (!ok) s_abort = 1;
+        const int wvalid = ntok - (it * TILE + warp * 16);
+        const int wlo = mask_lo - (it * TILE + warp * 16);
+        const bool work = ok && wvalid > 0 && wlo < 16 && wlo < wvalid;
+        const int tt0 = warp * 16;
+        const int jw = tt0 / BS;
+        const int rr = tt0 % BS + lrow;
+        const uint32_t kbase = smem_u32(s_kv + stage * 2 * STAGE_BYTES) +
+                               (uint32_t)(jw * NX * BOX_BYTES + rr * 128);
+        const int swz = rr & 7;
+        auto addr = [&](int kp) {  // chunk pair kp: chunks 2 kp, 2 kp + 1
+            const int chunk = 2 * kp + lchunk;
+            return kbase + (chunk >> 3) * BOX_BYTES + (((chunk & 7) ^ swz) << 4);
+        };
+        uint32_t kf[EARLY ? KP : 1][4], vf[EARLY ? KP : 1][4];
+        if (EARLY && work) {
+#pragma unroll
+            for (int kp = 0; kp < (EARLY ? KP : 1); ++kp) {
+                ldsm_x4(addr(kp), kf[kp]);
+                ldsm_x4_trans(addr(kp) + STAGE_BYTES, vf[kp]);
+            }
+        }
+        auto math = [&]() {
+            // two accumulator sets (even / odd k-steps): two short MMA
+            // dependency chains instead of one long one
+            float s[2][4], s2[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s[nt][i] = s2[nt][i] = 0.f;
+#pragma unroll
+            for (int kp = 0; kp < KP; ++kp) {
+                uint32_t kc[4];
+                if constexpr (EARLY) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) kc[i] = kf[kp < (EARLY ? KP : 1) ? kp : 0][i];
+                } else {
+                    ldsm_x4(addr(kp), kc);
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {  // k-step 2 kp + h
+                    uint32_t b0, b1, b2, b3;
+                    e4m3x4_to_f16x2(kc[2 * h], b0, b1);      // tokens 0-7
+                    e4m3x4_to_f16x2(kc[2 * h + 1], b2, b3);  // tokens 8-15
+                    M::run(h ? s2[0] : s[0], qa[2 * kp + h], b0, b1);
+                    M::run(h ? s2[1] : s[1], qa[2 * kp + h], b2, b3);
+                }
+            }
+            const bool partial = wvalid < 16 || wlo > 0;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s[nt][i] = (s[nt][i] + s2[nt][i]) * qmul;
+            if (partial) {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int tok = nt * 8 + 2 * t4 + (i & 1);
+                        if (tok < wlo || tok >= wvalid) s[nt][i] = -INFINITY;
+                    }
+            }
+            uint32_t pb[RB][2];
+            float alpha_c[RB][2];
+            bool grew = false;  // a running max moved: the accumulators need rescaling
+#pragma unroll
+            for (int rb = 0; rb < RB; ++rb) {
+                const int i0 = 2 * rb;
+                float mx = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float mnew = fmaxf(m[rb], mx);
+                const float alpha = exp2f(m[rb] - mnew);
+                grew |= alpha != 1.f;
+                float p[2][2], pr[2][2];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    p[nt][0] = exp2f(s[nt][i0] - mnew);
+                    p[nt][1] = exp2f(s[nt][i0 + 1] - mnew);
+                    pb[rb][nt] = M::pack(p[nt][0], p[nt][1], pr[nt][0], pr[nt][1]);
+                }
+                float ps = (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+                l[rb] = l[rb] * alpha + ps;
+                m[rb] = mnew;
+                alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
+                alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
+            }
+            grew = __any_sync(0xffffffffu, grew);
+#pragma unroll
+            for (int kp = 0; kp < KP; ++kp) {
+                uint32_t vc[4];
+                if constexpr (EARLY) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) vc[i] = vf[kp < (EARLY ? KP : 1) ? kp : 0][i];
+                } else {
+                    ldsm_x4_trans(addr(kp) + STAGE_BYTES, vc);
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {  // m-tile 2 kp + h
+                    const int mt = 2 * kp + h;
+                    uint32_t va[4];
+                    // (V[r0][2g], V[r0][2g+1], V[r1][2g], V[r1][2g+1]) ->
+                    // (V[r0][2g], V[r1][2g] | V[r0][2g+1], V[r1][2g+1])
+                    e4m3x4_to_f16x2(byte_perm(vc[2 * h], 0x3120u), va[0], va[1]);
+                    e4m3x4_to_f16x2(byte_perm(vc[2 * h + 1], 0x3120u), va[2], va[3]);
+                    if (partial) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int tk = (i >> 1) * 8 + 2 * t4;
+                            const uint32_t keep =
+                                (tk >= wlo && tk < wvalid ? 0x0000ffffu : 0u) |
+                                (tk + 1 >= wlo && tk + 1 < wvalid ? 0xffff0000u : 0u);
+                            va[i] &= keep;
+                        }
+                    }
+#pragma unroll
+                    for (int rb = 0; rb < RB; ++rb) {
+                        if (grew) {
+                            o[mt][rb][0] *= alpha_c[rb][0];
+                            o[mt][rb][1] *= alpha_c[rb][1];
+                            o[mt][rb][2] *= alpha_c[rb][0];
+                            o[mt][rb][3] *= alpha_c[rb][1];
+                        }
+                        M::run(o[mt][rb], va, pb[rb][0], pb[rb][1]);
+                    }
+                }
+            }
+        };
+        if (!EARLY && work) math();
+        __syncthreads();  // the stage is free again
+        if (s_abort) break;
+        if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage);
+        if (EARLY && work) math();
+    }
+    if (s_abort) return;
+    pdl_launch_dependents();
+
+    // merge the warps; A rows g, g + 8 of m-tile mt are dims 16 mt + 2 g, + 1
+    using A = MergeArea<D, NH, NW>;
+    static_assert(A::BYTES <= STAGES * 2 * STAGE_BYTES, "merge area");
+    float* red = reinterpret_cast<float*>(s_kv);
+    float* red_m = red + NW * NH * A::RP;
+    float* red_l = red_m + NW * NH;
+    const float vs = a.v_scale[kvh];
+#pragma unroll
+    for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+        for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int head = 8 * rb + 2 * t4 + (i & 1);
+                const int dim = mt * 16 + 2 * g + (i >> 1);
+                red[(warp * NH + head) * A::RP + dim] = o[mt][rb][i] * vs;
+            }
+    if (t4 == 0) {
+#pragma unroll
+        for (int rb = 0; rb < RB; ++rb) {
+            red_m[warp * NH + g + 8 * rb] = m[rb];
+            red_l[warp * NH + g + 8 * rb] = l[rb];
+        }
+    }
+    __syncthreads();
+    merge_warps_and_store<T, D, NH, NW>(a, red, b, h0, nh, part, np, tid, NW * 32);
+}
+
+template <typename T, int D, int BS, int NH, int NW = 4, int STAGES = 0>
+cudaError_t launch_decode_mma_e4m3(const DecodeArgs& a, cudaStream_t stream) {
+    using C = MmaE4m3Cfg<D, BS, NW, STAGES>;
+    static SmemAttr attr;
+    auto kern = decode_mma_e4m3_kernel<T, D, BS, NH, NW, STAGES>;
+    cudaError_t e = attr.ensure(kern, C::smem_bytes(8192));
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
+    CUtensorMap tk, tv;
+    e = make_cache_tensor_map(&tk, a.k_cache, 1, false, D, rows, BS);
+    if (e != cudaSuccess) return e;
+    e = make_cache_tensor_map(&tv, a.v_cache, 1, false, D, rows, BS);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
+    kern<<<grid, NW * 32, C::smem_bytes(a.partition_size), stream>>>(a, tk, tv);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || a.max_partitions <= 1) return e;
+    return launch_lse_reduce<T, D>(a, stream);
+}
+
+cudaError_t decode_mma_e4m3_f16(const DecodeArgs& a, int head_dim, int block_size, int hg,
+                                cudaStream_t stream);
+cudaError_t decode_mma_e4m3_bf16(const DecodeArgs& a, int head_dim, int block_size, int hg,
+                                 cudaStream_t stream);
+
+}  // namespace pkv

@@ -107,24 +107,31 @@ def test_append_and_copy_host_checks():
 def _decode_e4m3(**over):
     a = dict(out=None, q=None, k=None, v=None, ks=None, vs=None, bt=None, cl=None, order=None,
              B=4, Hq=8, Hkv=2, D=128, bs=16, mb=8, N=64, maxlen=100, scale=0.1, win=0,
-             dt=b.PKV_F16, P=0, ws=None, wsb=0, stream=None)
+             dt=b.PKV_F16, P=0, ws=None, wsb=0, kern=0, stream=None)
     a.update(over)
     return b.lib.pkv_paged_attention_decode_e4m3(
         a["out"], a["q"], a["k"], a["v"], a["ks"], a["vs"], a["bt"], a["cl"], a["order"], a["B"],
         a["Hq"], a["Hkv"], a["D"], a["bs"], a["mb"], a["N"], a["maxlen"], a["scale"], a["win"],
-        a["dt"], a["P"], a["ws"], a["wsb"], a["stream"])
+        a["dt"], a["P"], a["ws"], a["wsb"], a["kern"], a["stream"])
 
 
 @pytest.mark.parametrize("over,code", [
     (dict(dt=b.PKV_F32), b.PKV_EINVAL),                 # q / out must be 16-bit
     (dict(dt=b.PKV_E4M3), b.PKV_EINVAL),
     (dict(D=64), b.PKV_EUNSUPPORTED),                   # 64-byte rows
+    (dict(kern=9), b.PKV_EINVAL),
     (dict(Hq=6, Hkv=4), b.PKV_EINVAL),
     (dict(), b.PKV_EINVAL),                             # null pointers
     (dict(B=0), b.PKV_OK),
 ])
 def test_decode_e4m3_host_checks(over, code):
     assert _decode_e4m3(**over) == code
+
+
+def test_decode_e4m3_mma_group_limit():
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the kernel check fails first
+    assert _decode_e4m3(out=fake, q=fake, k=fake, v=fake, ks=fake, vs=fake, bt=fake, cl=fake,
+                        Hq=34, Hkv=2, maxlen=50, kern=b.PKV_KERNEL_MMA) == b.PKV_EUNSUPPORTED
 
 
 def test_e4m3_pages_need_their_own_entry():

@@ -42,7 +42,8 @@ class E4M3Inputs:
         self.cl = to_device(inp.context_lens)
         self.out = torch.empty_like(self.q)
 
-    def decode(self, partition_size=0, sliding_window=0, seq_order=None, fill_out=None):
+    def decode(self, partition_size=0, sliding_window=0, seq_order=None, fill_out=None,
+               kernel=pkv.PKV_KERNEL_AUTO):
         c = self.inp.cfg
         mcl = self.inp.max_context_len
         span = min(mcl, sliding_window + c.block_size - 1) if sliding_window > 0 else mcl
@@ -54,7 +55,8 @@ class E4M3Inputs:
         pkv.pkv_paged_attention_decode_e4m3(self.out, self.q, self.k, self.v, self.ks, self.vs,
                                             self.bt, self.cl, c.scale, c.block_size, mcl,
                                             partition_size=partition_size, workspace=ws,
-                                            sliding_window=sliding_window, seq_order=seq_order)
+                                            sliding_window=sliding_window, seq_order=seq_order,
+                                            kernel=kernel)
         torch.cuda.synchronize()
         return self.out
 
@@ -64,6 +66,9 @@ class E4M3Inputs:
                                    self.inp.block_tables, self.inp.context_lens, scale=c.scale,
                                    dtype=c.dtype, kv_dtype="e4m3", k_scale=self.pages.k_scale,
                                    v_scale=self.pages.v_scale, rows=rows, window=window)
+
+
+KERNELS = (pkv.PKV_KERNEL_SIMT, pkv.PKV_KERNEL_MMA)
 
 
 def _cfg(dtype, Hq, Hkv, D, bs, lens, pool_extra=7):
@@ -130,8 +135,9 @@ def test_decode_e4m3_ragged(dtype, G, partition):
     inp = make_decode_inputs(cfg, seed=70 + G)
     dev = E4M3Inputs(inp, seed=70 + G)
     ref = dev.oracle()
-    got = to_f64(dev.decode(partition_size=partition, fill_out=7.0))
-    assert_close(got, ref, dtype, f"e4m3 {dtype} G={G} P={partition}")
+    for kern in KERNELS:
+        got = to_f64(dev.decode(partition_size=partition, fill_out=7.0, kernel=kern))
+        assert_close(got, ref, dtype, f"e4m3 {dtype} G={G} P={partition} kernel={kern}")
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
@@ -142,9 +148,10 @@ def test_decode_e4m3_head_dims_block_sizes(dtype, D, bs):
     inp = make_decode_inputs(cfg, seed=80 + bs)
     dev = E4M3Inputs(inp, seed=80 + bs)
     ref = dev.oracle()
-    for P in (0, 64):
-        got = to_f64(dev.decode(partition_size=P, fill_out=-3.0))
-        assert_close(got, ref, dtype, f"e4m3 {dtype} D={D} bs={bs} P={P}")
+    for kern in KERNELS:
+        for P in (0, 64):
+            got = to_f64(dev.decode(partition_size=P, fill_out=-3.0, kernel=kern))
+            assert_close(got, ref, dtype, f"e4m3 {dtype} D={D} bs={bs} P={P} kernel={kern}")
 
 
 @pytest.mark.parametrize("W", [1, 17, 600])
@@ -154,19 +161,22 @@ def test_decode_e4m3_window_and_order(W):
     dev = E4M3Inputs(inp, seed=90)
     ref = dev.oracle(window=W)
     order = torch.from_numpy(pkv.pkv_decode_schedule_order(inp.context_lens)).cuda()
-    a = to_f64(dev.decode(partition_size=64, sliding_window=W))
-    assert_close(a, ref, "bf16", f"e4m3 W={W}")
-    b = to_f64(dev.decode(partition_size=64, sliding_window=W, seq_order=order, fill_out=1.0))
-    assert np.array_equal(a, b)
+    for kern in KERNELS:
+        a = to_f64(dev.decode(partition_size=64, sliding_window=W, kernel=kern))
+        assert_close(a, ref, "bf16", f"e4m3 W={W} kernel={kern}")
+        b = to_f64(dev.decode(partition_size=64, sliding_window=W, seq_order=order,
+                              fill_out=1.0, kernel=kern))
+        assert np.array_equal(a, b)
 
 
 def test_decode_e4m3_zero_length_and_unsupported():
     cfg = _cfg("f16", 2, 2, 128, 16, (0, 5))
     inp = make_decode_inputs(cfg, seed=91)
     dev = E4M3Inputs(inp, seed=91)
-    out = to_f64(dev.decode(fill_out=9.0))
-    assert np.all(out[0] == 0.0)
-    assert_close(out, dev.oracle(), "f16", "e4m3 zero length")
+    for kern in KERNELS:
+        out = to_f64(dev.decode(fill_out=9.0, kernel=kern))
+        assert np.all(out[0] == 0.0)
+        assert_close(out, dev.oracle(), "f16", f"e4m3 zero length kernel={kern}")
     # head_dim 64 rows are 64 bytes: not built
     cfg64 = _cfg("f16", 2, 2, 64, 16, (5, 5))
     dev64 = E4M3Inputs(make_decode_inputs(cfg64, seed=92), seed=92)
@@ -187,15 +197,54 @@ def test_decode_e4m3_full_size_sampled_rows():
                      axis=0)
     ref = dev.oracle(rows=rows)
     order = torch.from_numpy(pkv.pkv_decode_schedule_order(inp.context_lens)).cuda()
-    out = dev.decode(seq_order=order)
-    got = to_f64(out[torch.from_numpy(rows[:, 0]).long().cuda(),
-                     torch.from_numpy(rows[:, 1]).long().cuda()])
-    assert_close(got, ref, c.dtype, "llama2_13b_layer e4m3")
-    full = to_f64(out)
-    assert np.all(np.isfinite(full))
-    # convex combinations of the values: never beyond the largest |value|
     vmax = float(np.max(np.abs(dev.v.float().cpu().numpy()))) * float(dev.vs.max())
-    assert np.all(np.abs(full) <= vmax * 1.01 + 1e-3)
+    for kern in (pkv.PKV_KERNEL_AUTO, pkv.PKV_KERNEL_SIMT):
+        out = dev.decode(seq_order=order, kernel=kern)
+        got = to_f64(out[torch.from_numpy(rows[:, 0]).long().cuda(),
+                         torch.from_numpy(rows[:, 1]).long().cuda()])
+        assert_close(got, ref, c.dtype, f"llama2_13b_layer e4m3 kernel={kern}")
+        full = to_f64(out)
+        assert np.all(np.isfinite(full))
+        # convex combinations of the values: never beyond the largest |value|
+        assert np.all(np.abs(full) <= vmax * 1.01 + 1e-3)
+
+
+@pytest.mark.parametrize("G", [1, 8])
+def test_decode_e4m3_poisoned_slots_and_extreme_q(G):
+    """NaN codes in slots no sequence uses change no bit; q far outside the
+    fp16 range (bf16 q of 1e30 and 1e-30 magnitudes) still gives the
+    oracle's result on the tensor-core kernel (q enters it rescaled by a
+    power of two)."""
+    cfg = _cfg("bf16", 2 * G, 2, 128, 16, RAGGED)
+    inp = make_decode_inputs(cfg, seed=95)
+    dev = E4M3Inputs(inp, seed=95)
+    a = dev.decode(partition_size=64).clone()
+    live = np.zeros((inp.num_blocks, 16), dtype=bool)
+    for bb, L in enumerate(inp.context_lens):
+        for j in range((int(L) + 15) // 16):
+            live[inp.block_tables[bb, j], :min(16, int(L) - 16 * j)] = True
+    kc = dev.pages.k_cache.copy()
+    vc = dev.pages.v_cache.copy()
+    kc.transpose(0, 2, 1, 3)[~live] = 0x7F
+    vc.transpose(0, 2, 1, 3)[~live] = 0xFF
+    dev.k.copy_(_codes(kc))
+    dev.v.copy_(_codes(vc))
+    b = dev.decode(partition_size=64, fill_out=5.0).clone()
+    assert torch.equal(a, b)
+    dev.k.copy_(_codes(dev.pages.k_cache))
+    dev.v.copy_(_codes(dev.pages.v_cache))
+    for mag in (1e30, 1e-30):
+        from workloads import round_to_dtype
+        qx = round_to_dtype(inp.q.view(np.uint16).astype(np.uint32).__lshift__(16)
+                            .view(np.float32) * np.float32(mag), "bf16")
+        dev.inp = type(inp)(inp.cfg, qx, inp.k_cache, inp.v_cache, inp.block_tables,
+                            inp.context_lens, inp.num_blocks)
+        dev.q.copy_(to_device(qx, "bf16"))
+        ref = dev.oracle()
+        for kern in KERNELS:
+            got = to_f64(dev.decode(kernel=kern, fill_out=2.0))
+            assert_close(got, ref, "bf16", f"e4m3 q x {mag} kernel={kern}")
+    dev.inp = inp
 
 
 # ---------------------------------------------------------------------------
