@@ -44,7 +44,7 @@ struct MmaE4m3Cfg {
     static constexpr int BPT = TILE / BS;
     static constexpr int STAGE_BYTES = TILE * D;  // one of K / V
     static constexpr int FIT = 73728 / (2 * STAGE_BYTES);
-    static constexpr int STAGES = STAGES_ ? STAGES_ : (FIT >= 4 ? 4 : 3);
+    static constexpr int STAGES = STAGES_ ? STAGES_ : 3;
     static_assert(TILE % BS == 0 && BS % 8 == 0 && D % 128 == 0, "whole blocks, 128-byte rows");
 
     static int smem_bytes(int partition_size) {
@@ -61,6 +61,16 @@ __device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& lo, uint32
         "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
         : "=r"(lo), "=r"(hi)
         : "r"(w));
+}
+
+// d += A B, fp16 operands given as separate registers (a constant 0 for an
+// all-zero row block lets the compiler use the zero register)
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) {
@@ -160,7 +170,9 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
 
     // Q as the A operand (rows = heads g, g + 8), dims in the order the K
     // codes arrive: k = 2 t4 + j -> dim 4 t4 + j, k = 2 t4 + 8 + j -> 4 t4 + 2 + j.
-    uint32_t qa[KSTEPS][4];
+    // rows g + 8 (heads 8..15) exist only when NH == 16
+    constexpr int QR = NH == 16 ? 4 : 2;
+    uint32_t qa[KSTEPS][QR];
     float qmul;  // logits multiplier: scale * log2(e) * k_scale * 2^-e
     {
         const T* qb = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D;
@@ -197,8 +209,11 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
             for (int r = 0; r < 2; ++r) {
                 const __half2 lo = __floats2half2_rn(qf[ks][r][0] * up, qf[ks][r][1] * up);
                 const __half2 hi = __floats2half2_rn(qf[ks][r][2] * up, qf[ks][r][3] * up);
-                qa[ks][r] = *reinterpret_cast<const uint32_t*>(&lo);      // a0a1 / a2a3
-                qa[ks][2 + r] = *reinterpret_cast<const uint32_t*>(&hi);  // a4a5 / a6a7
+                if (NH == 16 || r == 0) {
+                    // NH 16: qa = a0a1, a2a3, a4a5, a6a7; NH 8: qa = a0a1, a4a5
+                    qa[ks][NH == 16 ? r : 0] = *reinterpret_cast<const uint32_t*>(&lo);
+                    qa[ks][NH == 16 ? 2 + r : 1] = *reinterpret_cast<const uint32_t*>(&hi);
+                }
             }
     }
 
@@ -266,8 +281,11 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                     uint32_t b0, b1, b2, b3;
                     e4m3x4_to_f16x2(kc[2 * h], b0, b1);      // tokens 0-7
                     e4m3x4_to_f16x2(kc[2 * h + 1], b2, b3);  // tokens 8-15
-                    M::run(h ? s2[0] : s[0], qa[2 * kp + h], b0, b1);
-                    M::run(h ? s2[1] : s[1], qa[2 * kp + h], b2, b3);
+                    const uint32_t* q4 = qa[2 * kp + h];
+                    const uint32_t a0 = q4[0], a1 = NH == 16 ? q4[1] : 0u;
+                    const uint32_t a2 = NH == 16 ? q4[2] : q4[1], a3 = NH == 16 ? q4[3] : 0u;
+                    mma_f16(h ? s2[0] : s[0], a0, a1, a2, a3, b0, b1);
+                    mma_f16(h ? s2[1] : s[1], a0, a1, a2, a3, b2, b3);
                 }
             }
             const bool partial = wvalid < 16 || wlo > 0;
@@ -284,34 +302,46 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                         if (tok < wlo || tok >= wvalid) s[nt][i] = -INFINITY;
                     }
             }
-            uint32_t pb[RB][2];
-            float alpha_c[RB][2];
-            bool grew = false;  // a running max moved: the accumulators need rescaling
+            // Softmax against a reference max m that moves only when a logit
+            // exceeds it by more than 2^8 (then p <= 256 fits fp16 and the
+            // accumulators are rescaled); l is kept per lane (this lane's
+            // tokens) and summed over the row's four lanes at the end.  The
+            // result is the same softmax: every p and l of a head shares m.
+            bool up = false;
+            float tmax[RB];
 #pragma unroll
             for (int rb = 0; rb < RB; ++rb) {
                 const int i0 = 2 * rb;
-                float mx = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                const float mnew = fmaxf(m[rb], mx);
-                const float alpha = exp2f(m[rb] - mnew);
-                grew |= alpha != 1.f;
-                float p[2][2], pr[2][2];
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    p[nt][0] = exp2f(s[nt][i0] - mnew);
-                    p[nt][1] = exp2f(s[nt][i0 + 1] - mnew);
-                    pb[rb][nt] = M::pack(p[nt][0], p[nt][1], pr[nt][0], pr[nt][1]);
-                }
-                float ps = (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-                ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-                ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-                l[rb] = l[rb] * alpha + ps;
-                m[rb] = mnew;
-                alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
-                alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
+                tmax[rb] = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
+                up |= tmax[rb] > m[rb] + 8.f;
             }
-            grew = __any_sync(0xffffffffu, grew);
+            const bool grew = __any_sync(0xffffffffu, up);
+            float alpha_c[RB][2];
+            if (grew) {
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) {
+                    float mx = tmax[rb];
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    const float mnew = fmaxf(m[rb], mx);
+                    const float alpha = exp2f(m[rb] - mnew);
+                    l[rb] *= alpha;
+                    m[rb] = mnew;
+                    alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
+                    alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
+                }
+            }
+            uint32_t pb[RB][2];
+#pragma unroll
+            for (int rb = 0; rb < RB; ++rb) {
+                const int i0 = 2 * rb;
+                float pr[2][2];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+                    pb[rb][nt] = M::pack(exp2f(s[nt][i0] - m[rb]), exp2f(s[nt][i0 + 1] - m[rb]),
+                                         pr[nt][0], pr[nt][1]);
+                l[rb] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+            }
 #pragma unroll
             for (int kp = 0; kp < KP; ++kp) {
                 uint32_t vc[4];
@@ -347,7 +377,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                             o[mt][rb][2] *= alpha_c[rb][0];
                             o[mt][rb][3] *= alpha_c[rb][1];
                         }
-                        M::run(o[mt][rb], va, pb[rb][0], pb[rb][1]);
+                        mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
                     }
                 }
             }
@@ -378,6 +408,11 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                 const int dim = mt * 16 + 2 * g + (i >> 1);
                 red[(warp * NH + head) * A::RP + dim] = o[mt][rb][i] * vs;
             }
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) {
+        l[rb] += __shfl_xor_sync(0xffffffffu, l[rb], 1);
+        l[rb] += __shfl_xor_sync(0xffffffffu, l[rb], 2);
+    }
     if (t4 == 0) {
 #pragma unroll
         for (int rb = 0; rb < RB; ++rb) {
