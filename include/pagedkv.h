@@ -426,6 +426,41 @@ PKV_API int pkv_alloc_is_swapped(const pkv_alloc* a, int64_t seq_id, int* swappe
  */
 PKV_API int pkv_alloc_slide_window(pkv_alloc* a, int64_t seq_id, int window, int* released);
 
+/*
+ * Prefix cache ("pagedattention vllm" §vLLM Integration and §Advanced
+ * Features: automatic prefix caching shares common prompt starts across
+ * requests; "PagedAttention" glossary entry: prompt caching lets later
+ * requests that begin the same way skip that work).
+ *
+ * pkv_alloc_add_seq_prefix adds sequence seq_id for a prompt of num_tokens
+ * token ids (host int32).  Full block j of the prompt (tokens [j*bs, (j+1)*bs))
+ * has the key (registration id of block j-1, or 0 for j = 0; its bs token
+ * ids).  For j = 0, 1, ... while a registered block has block j's key, the
+ * sequence takes that block (one more reference; an evictable block comes
+ * back); the first miss ends the walk, so a hit always means the whole prompt
+ * up to that block is identical.  The remaining blocks are taken in logical
+ * order (as pkv_alloc_add_seq) and each full one is registered under its key
+ * with the next registration id; the partial last block is never registered.
+ * *cached_tokens = hits * block_size: the prompt tokens whose K/V are already
+ * in the pool (the caller computes and appends only the rest).  All or nothing
+ * (PKV_ENOMEM, PKV_EEXIST).
+ *
+ * A registered block whose reference count reaches zero (any release:
+ * free_seq, a copy-on-write source, swap_out, slide_window) is kept with its
+ * contents on the evictable list, least recently released first, instead of
+ * the free stack.  Every allocation pops the free stack and, only when it is
+ * empty, evicts the head of the evictable list (unregistering it); capacity
+ * checks count both.  Registered blocks are always full prompt blocks, so no
+ * append ever writes into one.  pkv_alloc_free_list lists the free stack only.
+ */
+PKV_API int pkv_alloc_add_seq_prefix(pkv_alloc* a, int64_t seq_id, const int32_t* tokens,
+                                     int num_tokens, int* cached_tokens);
+/* Registered blocks (in use or evictable) and evictable blocks. */
+PKV_API int pkv_alloc_cache_stats(const pkv_alloc* a, int32_t* cached_blocks,
+                                  int32_t* evictable_blocks);
+/* Evictable blocks, next to be evicted first. */
+PKV_API int pkv_alloc_evictable_list(const pkv_alloc* a, int32_t* out, int capacity, int* n_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -46,6 +46,25 @@ Sliding window ("pagedattention vllm" §Advanced Features: sliding-window models
 keep only recent blocks): slide_window(seq, W) releases, in logical order,
 every block j with (j + 1) * block_size <= len - W (one reference dropped, the
 entry becomes -1); fork, free and swap skip -1 entries.
+
+Prefix cache ("pagedattention vllm" §vLLM Integration, §Advanced Features:
+prefix caching; lastdictionary "PagedAttention": prompt caching lets requests
+that begin the same way skip that part):
+  - add_seq_prefix(seq, tokens): full block j of the prompt has the key
+    (registration id of block j - 1, or 0 for j = 0; its block_size tokens).
+    Walking j = 0, 1, ... while a registered block has that key, the sequence
+    takes those blocks (one more reference; an evictable one comes back);
+    the first miss ends the walk.  The remaining blocks are taken in logical
+    order and each full one is registered under its key with the next
+    registration id (1, 2, ...); the partial last block is never registered.
+    It reports the number of prompt tokens found (hits * block_size); all or
+    nothing;
+  - a registered block whose count reaches zero is not pushed on the free
+    stack but appended to the evictable list; taking a block pops the free
+    stack, or, when that is empty, evicts the head of the evictable list
+    (least recently released), unregistering it;
+  - capacity of an allocation = free stack + evictable list (minus evictable
+    blocks the same call takes back as hits).
 """
 from __future__ import annotations
 
@@ -65,6 +84,34 @@ class BlockManagerModel:
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
         self.swapped: set[int] = set()
+        # prefix cache
+        self.key_of: dict[int, tuple] = {}      # registered block -> (parent id, tokens)
+        self.reg_of: dict[int, int] = {}        # registered block -> registration id
+        self.block_of: dict[tuple, int] = {}    # key -> registered block
+        self.next_reg = 1
+        self.evictable: list[int] = []          # least recently released first
+
+    # -- block supply -----------------------------------------------------
+    def _available(self) -> int:
+        return len(self.free) + len(self.evictable)
+
+    def _take(self) -> int:
+        if self.free:
+            blk = self.free.pop()
+        else:
+            blk = self.evictable.pop(0)
+            del self.block_of[self.key_of.pop(blk)]
+            del self.reg_of[blk]
+        self.ref[blk] = 1
+        return blk
+
+    def _release(self, blk: int) -> None:
+        self.ref[blk] -= 1
+        if self.ref[blk] == 0:
+            if blk in self.reg_of:
+                self.evictable.append(blk)
+            else:
+                self.free.append(blk)
 
     # -- operations -------------------------------------------------------
     def add_seq(self, seq_id: int, num_tokens: int) -> int:
@@ -73,16 +120,49 @@ class BlockManagerModel:
         if seq_id in self.tables:
             return EEXIST
         need = (num_tokens + self.block_size - 1) // self.block_size
-        if need > len(self.free):
+        if need > self._available():
             return ENOMEM
-        table = []
-        for _ in range(need):
-            blk = self.free.pop()
-            self.ref[blk] = 1
-            table.append(blk)
-        self.tables[seq_id] = table
+        self.tables[seq_id] = [self._take() for _ in range(need)]
         self.lens[seq_id] = num_tokens
         return OK
+
+    def add_seq_prefix(self, seq_id: int, tokens):
+        """-> (status, prompt tokens found in the cache)"""
+        tokens = [int(t) for t in tokens]
+        if seq_id in self.tables:
+            return EEXIST, 0
+        bs = self.block_size
+        nfull = len(tokens) // bs
+        need = (len(tokens) + bs - 1) // bs
+        hits, parent = [], 0
+        for j in range(nfull):
+            blk = self.block_of.get((parent, tuple(tokens[j * bs:(j + 1) * bs])))
+            if blk is None:
+                break
+            hits.append(blk)
+            parent = self.reg_of[blk]
+        back = sum(1 for b in hits if self.ref[b] == 0)
+        if need - len(hits) > self._available() - back:
+            return ENOMEM, 0
+        table = []
+        for blk in hits:
+            if self.ref[blk] == 0:
+                self.evictable.remove(blk)
+            self.ref[blk] += 1
+            table.append(blk)
+        for j in range(len(hits), need):
+            blk = self._take()
+            table.append(blk)
+            if j < nfull:
+                key = (parent, tuple(tokens[j * bs:(j + 1) * bs]))
+                self.key_of[blk] = key
+                self.block_of[key] = blk
+                self.reg_of[blk] = self.next_reg
+                self.next_reg += 1
+                parent = self.reg_of[blk]
+        self.tables[seq_id] = table
+        self.lens[seq_id] = len(tokens)
+        return OK, len(hits) * bs
 
     def fork(self, parent: int, child: int) -> int:
         if parent not in self.tables:
@@ -109,18 +189,15 @@ class BlockManagerModel:
         n = self.lens[seq_id]
         src = dst = -1
         if n % self.block_size == 0:
-            if not self.free:
+            if not self._available():
                 return ENOMEM, -1, -1, -1
-            blk = self.free.pop()
-            self.ref[blk] = 1
-            table.append(blk)
+            table.append(self._take())
         elif self.ref[table[-1]] > 1:
-            if not self.free:
+            if not self._available():
                 return ENOMEM, -1, -1, -1
-            dst = self.free.pop()
-            self.ref[dst] = 1
+            dst = self._take()
             src = table[-1]
-            self.ref[src] -= 1
+            self._release(src)   # stays > 0: another sequence still holds it
             table[-1] = dst
         slot = table[-1] * self.block_size + n % self.block_size
         self.lens[seq_id] = n + 1
@@ -134,11 +211,8 @@ class BlockManagerModel:
             self.swapped.discard(seq_id)
         else:
             for blk in self.tables.pop(seq_id):
-                if blk < 0:
-                    continue
-                self.ref[blk] -= 1
-                if self.ref[blk] == 0:
-                    self.free.append(blk)
+                if blk >= 0:
+                    self._release(blk)
         del self.lens[seq_id]
         return OK
 
@@ -157,9 +231,7 @@ class BlockManagerModel:
                 continue
             h = self.host_free.pop()
             pairs.append((blk, h))
-            self.ref[blk] -= 1
-            if self.ref[blk] == 0:
-                self.free.append(blk)
+            self._release(blk)
             table[i] = h
         self.swapped.add(seq_id)
         return OK, pairs
@@ -171,14 +243,13 @@ class BlockManagerModel:
         if seq_id not in self.swapped:
             return EINVAL, []
         table = self.tables[seq_id]
-        if sum(1 for h in table if h >= 0) > len(self.free):
+        if sum(1 for h in table if h >= 0) > self._available():
             return ENOMEM, []
         pairs = []
         for i, h in enumerate(table):
             if h < 0:
                 continue
-            d = self.free.pop()
-            self.ref[d] = 1
+            d = self._take()
             pairs.append((h, d))
             self.host_free.append(h)
             table[i] = d
@@ -201,9 +272,7 @@ class BlockManagerModel:
                 break
             if table[j] < 0:
                 continue
-            self.ref[table[j]] -= 1
-            if self.ref[table[j]] == 0:
-                self.free.append(table[j])
+            self._release(table[j])
             table[j] = -1
             released += 1
         return OK, released
@@ -235,6 +304,13 @@ class BlockManagerModel:
             reserved=0,
         )
 
+    def cache_stats(self) -> tuple[int, int]:
+        """(registered blocks, evictable blocks)"""
+        return len(self.reg_of), len(self.evictable)
+
+    def evictable_list(self) -> list[int]:
+        return list(self.evictable)
+
     def host_free_list(self) -> list[int]:
         return list(reversed(self.host_free))
 
@@ -259,4 +335,6 @@ class BlockManagerModel:
             return self.swap_in(op[1])
         if kind == "slide":
             return self.slide_window(op[1], op[2])
+        if kind == "prefix":
+            return self.add_seq_prefix(op[1], op[2])
         raise ValueError(kind)

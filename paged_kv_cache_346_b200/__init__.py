@@ -384,6 +384,30 @@ class BlockAllocator:
         st = lib.pkv_alloc_slide_window(self._h, seq_id, window, ctypes.byref(n))
         return st, (n.value if st == 0 else 0)
 
+    def add_seq_prefix(self, seq_id: int, tokens):
+        """New sequence for a prompt of token ids, reusing cached full blocks of
+        an identical prefix.  -> (status, prompt tokens found in the cache)"""
+        import numpy as np
+        tk = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = ctypes.c_int(0)
+        st = lib.pkv_alloc_add_seq_prefix(self._h, seq_id, tk.ctypes.data if tk.size else None,
+                                          tk.size, ctypes.byref(n))
+        return st, (n.value if st == 0 else 0)
+
+    def cache_stats(self) -> tuple[int, int]:
+        """(registered prefix blocks, evictable blocks)"""
+        c, e = ctypes.c_int32(0), ctypes.c_int32(0)
+        check(lib.pkv_alloc_cache_stats(self._h, ctypes.byref(c), ctypes.byref(e)),
+              "pkv_alloc_cache_stats")
+        return c.value, e.value
+
+    def evictable_list(self) -> list[int]:
+        n = ctypes.c_int(0)
+        buf = (ctypes.c_int32 * max(self.num_blocks, 1))()
+        check(lib.pkv_alloc_evictable_list(self._h, buf, self.num_blocks, ctypes.byref(n)),
+              "pkv_alloc_evictable_list")
+        return list(buf[:n.value])
+
     def is_swapped(self, seq_id: int) -> bool:
         v = ctypes.c_int(0)
         check(lib.pkv_alloc_is_swapped(self._h, seq_id, ctypes.byref(v)), "pkv_alloc_is_swapped")
@@ -405,6 +429,8 @@ class BlockAllocator:
             return self.append_slot(op[1])
         if kind == "free":
             return self.free_seq(op[1])
+        if kind == "prefix":
+            return self.add_seq_prefix(op[1], op[2])
         raise ValueError(kind)
 
     # queries

@@ -60,6 +60,9 @@ SIGNATURES = {
     "pkv_alloc_swap_in": (_i32, [_vp, _i64, _vp, _i32, _c.POINTER(_i32)]),
     "pkv_alloc_is_swapped": (_i32, [_vp, _i64, _c.POINTER(_i32)]),
     "pkv_alloc_slide_window": (_i32, [_vp, _i64, _i32, _c.POINTER(_i32)]),
+    "pkv_alloc_add_seq_prefix": (_i32, [_vp, _i64, _vp, _i32, _c.POINTER(_i32)]),
+    "pkv_alloc_cache_stats": (_i32, [_vp, _c.POINTER(_c.c_int32), _c.POINTER(_c.c_int32)]),
+    "pkv_alloc_evictable_list": (_i32, [_vp, _vp, _i32, _c.POINTER(_i32)]),
     "pkv_alloc_destroy": (None, [_vp]),
     "pkv_alloc_add_seq": (_i32, [_vp, _i64, _i32]),
     "pkv_alloc_fork": (_i32, [_vp, _i64, _i64]),

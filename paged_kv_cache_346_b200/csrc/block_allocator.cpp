@@ -9,7 +9,18 @@
 // of swapped-out sequences ("pagedattention vllm" §Memory Management:
 // swapping blocks to CPU memory).  Every operation either completes or
 // leaves all of it untouched.
+//
+// Prefix cache ("pagedattention vllm" §vLLM Integration and §Advanced
+// Features: prefix caching; "PagedAttention" glossary entry: prompt caching
+// lets later requests that start the same way skip that part).  A full
+// prompt block is registered under (registration id of the block before it,
+// its block_size token ids); a new prompt walks its full blocks and reuses
+// each registered block whose key matches, so a hit means the whole prefix up
+// to that block is identical.  A registered block whose count drops to zero
+// is kept (evictable, least recently released first) until an allocation finds
+// the free stack empty and takes it back.
 #include <cstdint>
+#include <cstring>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -35,9 +46,87 @@ struct pkv_alloc {
     int32_t used_blocks = 0;
     int32_t shared_blocks = 0;
 
+    // ---- prefix cache (allocated on first use)
+    std::vector<int64_t> reg_id;       // per block: registration id, 0 = not registered
+    std::vector<int64_t> reg_parent;   // per block: registration id of the block before it
+    std::vector<int32_t> reg_tokens;   // per block: its block_size token ids
+    std::unordered_multimap<uint64_t, int32_t> reg_map;  // key hash -> registered blocks
+    int64_t next_reg = 1;
+    int32_t cached_blocks = 0;
+    // evictable registered blocks: a doubly linked list over block ids,
+    // least recently released at the head
+    std::vector<int32_t> ev_prev, ev_next;
+    int32_t ev_head = -1, ev_tail = -1, evictable = 0;
+
+    bool cache_on() const { return !reg_id.empty(); }
+    void cache_init() {
+        if (cache_on()) return;
+        reg_id.assign(num_blocks, 0);
+        reg_parent.assign(num_blocks, 0);
+        reg_tokens.assign((size_t)num_blocks * block_size, 0);
+        ev_prev.assign(num_blocks, -1);
+        ev_next.assign(num_blocks, -1);
+    }
+    static uint64_t key_hash(int64_t parent, const int32_t* tokens, int n) {
+        uint64_t h = 1469598103934665603ull;  // FNV-1a, 64 bit
+        auto mix = [&](uint64_t v) {
+            for (int i = 0; i < 8; ++i) {
+                h ^= (v >> (8 * i)) & 0xffu;
+                h *= 1099511628211ull;
+            }
+        };
+        mix((uint64_t)parent);
+        for (int i = 0; i < n; ++i) mix((uint64_t)(uint32_t)tokens[i]);
+        return h;
+    }
+    // the registered block with this exact key, or -1
+    int32_t lookup(int64_t parent, const int32_t* tokens) const {
+        auto range = reg_map.equal_range(key_hash(parent, tokens, block_size));
+        for (auto it = range.first; it != range.second; ++it) {
+            const int32_t b = it->second;
+            if (reg_parent[b] == parent &&
+                std::memcmp(&reg_tokens[(size_t)b * block_size], tokens,
+                            sizeof(int32_t) * block_size) == 0)
+                return b;
+        }
+        return -1;
+    }
+    void ev_push(int32_t b) {
+        ev_prev[b] = ev_tail;
+        ev_next[b] = -1;
+        if (ev_tail >= 0) ev_next[ev_tail] = b; else ev_head = b;
+        ev_tail = b;
+        ++evictable;
+    }
+    void ev_remove(int32_t b) {
+        if (ev_prev[b] >= 0) ev_next[ev_prev[b]] = ev_next[b]; else ev_head = ev_next[b];
+        if (ev_next[b] >= 0) ev_prev[ev_next[b]] = ev_prev[b]; else ev_tail = ev_prev[b];
+        ev_prev[b] = ev_next[b] = -1;
+        --evictable;
+    }
+    void unregister(int32_t b) {
+        auto range = reg_map.equal_range(
+            key_hash(reg_parent[b], &reg_tokens[(size_t)b * block_size], block_size));
+        for (auto it = range.first; it != range.second; ++it)
+            if (it->second == b) {
+                reg_map.erase(it);
+                break;
+            }
+        reg_id[b] = 0;
+        --cached_blocks;
+    }
+    int64_t available() const { return (int64_t)free_stack.size() + evictable; }
+
     int32_t take() {
-        int32_t b = free_stack.back();
-        free_stack.pop_back();
+        int32_t b;
+        if (!free_stack.empty()) {
+            b = free_stack.back();
+            free_stack.pop_back();
+        } else {  // evict the least recently released cached block
+            b = ev_head;
+            ev_remove(b);
+            unregister(b);
+        }
         ref[b] = 1;
         ++used_blocks;
         ++refcount_sum;
@@ -54,7 +143,8 @@ struct pkv_alloc {
         if (ref[b] == 1) --shared_blocks;
         if (ref[b] == 0) {
             --used_blocks;
-            free_stack.push_back(b);
+            if (cache_on() && reg_id[b] != 0) ev_push(b);
+            else free_stack.push_back(b);
         }
     }
 };
@@ -94,7 +184,7 @@ int pkv_alloc_add_seq(pkv_alloc* a, int64_t seq_id, int num_tokens) {
     if (!a || num_tokens < 0) return PKV_EINVAL;
     if (a->seqs.count(seq_id)) return PKV_EEXIST;
     const int64_t need = ((int64_t)num_tokens + a->block_size - 1) / a->block_size;
-    if (need > (int64_t)a->free_stack.size()) return PKV_ENOMEM;
+    if (need > a->available()) return PKV_ENOMEM;
     pkv_alloc::Seq s;
     s.len = num_tokens;
     s.table.reserve(need);
@@ -128,10 +218,10 @@ int pkv_alloc_append_slot(pkv_alloc* a, int64_t seq_id, int64_t* slot, int32_t* 
     const int64_t off = s.len % a->block_size;
     int32_t src = -1, dst = -1;
     if (off == 0) {
-        if (a->free_stack.empty()) return PKV_ENOMEM;
+        if (a->available() == 0) return PKV_ENOMEM;
         s.table.push_back(a->take());
     } else if (a->ref[s.table.back()] > 1) {
-        if (a->free_stack.empty()) return PKV_ENOMEM;
+        if (a->available() == 0) return PKV_ENOMEM;
         dst = a->take();
         src = s.table.back();
         a->drop_ref(src);  // stays > 0: another sequence still holds it
@@ -272,7 +362,7 @@ int pkv_alloc_swap_in(pkv_alloc* a, int64_t seq_id, int32_t* pairs, int capacity
     for (int32_t h : s.table) n += h >= 0;
     *num_pairs = n;
     if (n > capacity) return PKV_EBOUNDS;
-    if (n > (int)a->free_stack.size()) return PKV_ENOMEM;
+    if (n > a->available()) return PKV_ENOMEM;
     int k = 0;
     for (int32_t& h : s.table) {
         if (h < 0) continue;
@@ -303,6 +393,85 @@ int pkv_alloc_slide_window(pkv_alloc* a, int64_t seq_id, int window, int* releas
         s.table[j] = -1;
         ++*released;
     }
+    return PKV_OK;
+}
+
+int pkv_alloc_add_seq_prefix(pkv_alloc* a, int64_t seq_id, const int32_t* tokens,
+                             int num_tokens, int* cached_tokens) {
+    if (!a || num_tokens < 0 || (num_tokens > 0 && !tokens) || !cached_tokens) return PKV_EINVAL;
+    if (a->seqs.count(seq_id)) return PKV_EEXIST;
+    try {
+        a->cache_init();
+    } catch (...) {
+        return PKV_ENOMEM;
+    }
+    const int bs = a->block_size;
+    const int64_t nfull = num_tokens / bs;
+    const int64_t need = ((int64_t)num_tokens + bs - 1) / bs;
+    // 1. the registered prefix (read only)
+    std::vector<int32_t> hits;
+    int64_t parent = 0, evictable_hits = 0;
+    for (int64_t j = 0; j < nfull; ++j) {
+        const int32_t b = a->lookup(parent, tokens + j * bs);
+        if (b < 0) break;
+        hits.push_back(b);
+        evictable_hits += a->ref[b] == 0;
+        parent = a->reg_id[b];
+    }
+    const int64_t fresh = need - (int64_t)hits.size();
+    if (fresh > a->available() - evictable_hits) return PKV_ENOMEM;
+    // 2. take the hits, then allocate (and register the full blocks among) the rest
+    pkv_alloc::Seq s;
+    s.len = num_tokens;
+    try {
+        s.table.reserve(need);
+        a->reg_map.reserve(a->reg_map.size() + nfull);
+    } catch (...) {
+        return PKV_ENOMEM;
+    }
+    for (int32_t b : hits) {
+        if (a->ref[b] == 0) {
+            a->ev_remove(b);
+            a->ref[b] = 1;
+            ++a->used_blocks;
+            ++a->refcount_sum;
+        } else {
+            a->add_ref(b);
+        }
+        s.table.push_back(b);
+    }
+    for (int64_t j = (int64_t)hits.size(); j < need; ++j) {
+        const int32_t b = a->take();
+        s.table.push_back(b);
+        if (j < nfull) {
+            const int32_t* tk = tokens + j * bs;
+            a->reg_id[b] = a->next_reg++;
+            a->reg_parent[b] = parent;
+            std::memcpy(&a->reg_tokens[(size_t)b * bs], tk, sizeof(int32_t) * bs);
+            a->reg_map.emplace(pkv_alloc::key_hash(parent, tk, bs), b);
+            ++a->cached_blocks;
+            parent = a->reg_id[b];
+        }
+    }
+    *cached_tokens = (int)(hits.size() * bs);
+    a->logical_tokens += num_tokens;
+    a->seqs.emplace(seq_id, std::move(s));
+    return PKV_OK;
+}
+
+int pkv_alloc_cache_stats(const pkv_alloc* a, int32_t* cached_blocks, int32_t* evictable_blocks) {
+    if (!a || !cached_blocks || !evictable_blocks) return PKV_EINVAL;
+    *cached_blocks = a->cached_blocks;
+    *evictable_blocks = a->evictable;
+    return PKV_OK;
+}
+
+int pkv_alloc_evictable_list(const pkv_alloc* a, int32_t* out, int capacity, int* n_out) {
+    if (!a || !n_out || capacity < 0 || (capacity > 0 && !out)) return PKV_EINVAL;
+    *n_out = a->evictable;
+    if (a->evictable > capacity) return PKV_EBOUNDS;
+    int k = 0;
+    for (int32_t b = a->ev_head; b >= 0; b = a->ev_next[b]) out[k++] = b;
     return PKV_OK;
 }
 

@@ -249,7 +249,6 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         const int rr = tt0 % BS + lrow;      // this lane's row within that block
         const uint32_t kbase = smem_u32(s_kv + stage * 2 * STAGE_BYTES) +
                                (uint32_t)(jw * NX * BOX_BYTES + rr * 128);
-        const uint32_t vbase = kbase + STAGE_BYTES;
         const int swz = rr & 7;
         auto kaddr = [&](int ks) {
             const int chunk = ks * 2 + lchunk;  // 16-byte chunk of the row

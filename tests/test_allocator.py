@@ -129,3 +129,123 @@ def test_random_scripts_with_windows_bit_exact(seed):
         if i % 20 == 0:
             same_state(nat, mod)
     same_state(nat, mod)
+
+
+# ---------------------------------------------------------------------------
+# prefix cache
+
+def same_cache_state(native: BlockAllocator, model: bm.BlockManagerModel):
+    same_state(native, model)
+    assert native.cache_stats() == model.cache_stats()
+    assert native.evictable_list() == model.evictable_list()
+
+
+@pytest.mark.parametrize("seed", range(12))
+@pytest.mark.parametrize("bs", [1, 4, 16])
+def test_random_scripts_with_prefix_cache_bit_exact(seed, bs):
+    N = {1: 240, 4: 64, 16: 24}[bs]   # tight enough that evictions happen
+    nat, mod = BlockAllocator(N, bs, num_host_blocks=24), bm.BlockManagerModel(N, bs, 24)
+    ops = random_alloc_ops(seed, 400, max_len=60, prefix=True, swap=seed % 3 == 0,
+                           slide=seed % 3 == 1)
+    assert any(op[0] == "prefix" for op in ops)
+    hits = 0
+    for i, op in enumerate(ops):
+        r_nat, r_mod = nat.apply(op), mod.apply(op)
+        assert r_nat == r_mod, (i, op)
+        if op[0] == "prefix" and r_mod[0] == 0:
+            hits += r_mod[1]
+        if i % 20 == 0:
+            same_cache_state(nat, mod)
+    same_cache_state(nat, mod)
+    assert hits > 0          # the scripts do reuse cached prefixes
+
+
+def _invariants(model: bm.BlockManagerModel):
+    st = model.stats()
+    cached, evictable = model.cache_stats()
+    assert st["free_blocks"] + evictable + st["used_blocks"] == model.num_blocks
+    assert set(model.free) .isdisjoint(model.evictable)
+    assert all(model.ref[b] == 0 for b in model.evictable)
+    assert all(b in model.reg_of for b in model.evictable)
+    assert cached == len(model.block_of)
+    # a registered block is full and holds exactly the tokens of its key
+    for blk, (parent, toks) in model.key_of.items():
+        assert len(toks) == model.block_size
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_prefix_model_invariants(seed):
+    mod = bm.BlockManagerModel(40, 4, 16)
+    for op in random_alloc_ops(seed, 400, max_len=60, prefix=True, swap=True, slide=True):
+        mod.apply(op)
+        _invariants(mod)
+
+
+def test_prefix_sharing_by_hand():
+    """Worked example: block size 4, prompts A = 0..9, B = A[:8] + others."""
+    for x in (BlockAllocator(8, 4), bm.BlockManagerModel(8, 4)):
+        A = list(range(10))
+        B = list(range(8)) + [70, 71, 72]
+        C = [0, 1, 2, 3, 99, 5, 6, 7]      # differs inside block 1
+        assert x.add_seq_prefix(0, A) == (0, 0)        # nothing cached yet
+        tA = x.block_table(0)
+        assert tA == [0, 1, 2]
+        assert x.add_seq_prefix(1, B) == (0, 8)        # blocks 0, 1 reused
+        tB = x.block_table(1)
+        assert tB[:2] == tA[:2] and tB[2] not in tA
+        assert x.refcount(tA[0]) == 2 and x.refcount(tA[2]) == 1
+        assert x.add_seq_prefix(2, C) == (0, 4)        # only block 0 matches
+        assert x.block_table(2)[0] == tA[0] and x.block_table(2)[1] not in tA + tB
+        # the partial last blocks were never registered: A's third block has 2
+        # tokens, B's 3; registered = A's 2 full blocks + C's second block
+        assert x.cache_stats() == (3, 0)
+        # free everything: registered blocks become evictable in the order
+        # their counts reach zero (B frees A's block 1, C frees block 0, then
+        # its own registered block 1)
+        c1 = x.block_table(2)[1]
+        for sid in (0, 1, 2):
+            assert x.free_seq(sid) == 0
+        assert x.cache_stats() == (3, 3)
+        assert x.evictable_list() == [tA[1], tA[0], c1]
+        # a new prompt with A's start takes the evictable blocks back
+        assert x.add_seq_prefix(3, A[:8]) == (0, 8)
+        assert x.block_table(3) == tA[:2]
+        assert x.cache_stats() == (3, 1)
+
+
+def test_prefix_eviction_order_and_capacity():
+    for x in (BlockAllocator(4, 2), bm.BlockManagerModel(4, 2)):
+        assert x.add_seq_prefix(0, [1, 2, 3, 4]) == (0, 0)   # blocks 0, 1 registered
+        assert x.free_seq(0) == 0                              # both evictable: 0 then 1
+        assert x.evictable_list() == [0, 1]
+        assert x.stats()["free_blocks"] == 2
+        # 4 blocks needed: 2 from the free stack, then evict 0, then 1
+        assert x.add_seq(1, 8) == 0
+        assert x.block_table(1) == [2, 3, 0, 1]
+        assert x.cache_stats() == (0, 0)
+        assert x.add_seq_prefix(2, [1, 2]) == (-2, 0)        # ENOMEM, nothing changed
+        assert x.free_seq(1) == 0
+        assert x.add_seq_prefix(2, [1, 2, 3, 4]) == (0, 0)   # nothing cached any more
+
+
+def test_prefix_hit_needs_whole_prefix():
+    """Equal tokens at an equal position but a different earlier block do not
+    match: a hit means the entire prefix is identical."""
+    for x in (BlockAllocator(16, 2), bm.BlockManagerModel(16, 2)):
+        assert x.add_seq_prefix(0, [5, 5, 7, 7]) == (0, 0)
+        assert x.add_seq_prefix(1, [6, 6, 7, 7]) == (0, 0)
+        assert x.block_table(1)[1] != x.block_table(0)[1]
+        assert x.add_seq_prefix(2, [6, 6, 7, 7, 8]) == (0, 4)
+        assert x.block_table(2)[:2] == x.block_table(1)
+
+
+def test_prefix_capacity_counts_evictable_hits():
+    """An evictable block that the same call takes back as a hit cannot also
+    be evicted to satisfy the call's fresh blocks."""
+    for x in (BlockAllocator(3, 2), bm.BlockManagerModel(3, 2)):
+        assert x.add_seq_prefix(0, [1, 1, 2, 2]) == (0, 0)
+        assert x.free_seq(0) == 0                 # 2 evictable + 1 free
+        # hits 2 blocks (both evictable) + needs 2 fresh: only 1 free -> ENOMEM
+        assert x.add_seq_prefix(1, [1, 1, 2, 2, 3, 3, 4]) == (-2, 0)
+        assert x.cache_stats() == (2, 2)
+        assert x.add_seq_prefix(1, [1, 1, 2, 2, 3]) == (0, 4)

@@ -355,14 +355,20 @@ def draw_cow_recipe(seed: int = 5, **over) -> CowRecipe:
 
 
 def random_alloc_ops(seed: int, n_ops: int, max_seqs: int = 24, max_len: int = 200,
-                     swap: bool = False, slide: bool = False):
+                     swap: bool = False, slide: bool = False, prefix: bool = False):
     """A seeded random script of allocator operations (add / fork / append /
     free, swap_out / swap_in when `swap`, sliding-window releases when
-    `slide`) for differential tests of the block manager."""
+    `slide`, prompts through the prefix cache when `prefix`) for differential
+    tests of the block manager.  Prefix prompts start with one of four fixed
+    token sequences (synthetic token ids) cut at a random length, and some
+    continue with random tokens, so prompts share prefixes of varied lengths."""
     g = rng(seed * 1000 + 9)
     ops = []
     next_id = 0
     live = []
+    if prefix:
+        gp = rng(seed * 1000 + 10)
+        templates = [gp.integers(0, 50, size=max_len) for _ in range(4)]
     for _ in range(n_ops):
         r = g.random()
         if slide and live and g.random() < 0.1:
@@ -373,7 +379,14 @@ def random_alloc_ops(seed: int, n_ops: int, max_seqs: int = 24, max_len: int = 2
                         live[int(g.integers(len(live)))]))
             continue
         if not live or (r < 0.25 and len(live) < max_seqs):
-            ops.append(("add", next_id, int(g.integers(0, max_len + 1))))
+            n = int(g.integers(0, max_len + 1))
+            if prefix and gp.random() < 0.7:
+                t = templates[int(gp.integers(4))][:n].copy()
+                cut = int(gp.integers(0, n + 1)) if gp.random() < 0.5 else n
+                t[cut:] = gp.integers(0, 50, size=n - cut)
+                ops.append(("prefix", next_id, tuple(int(x) for x in t)))
+            else:
+                ops.append(("add", next_id, n))
             live.append(next_id)
             next_id += 1
         elif r < 0.45 and len(live) < max_seqs:
