@@ -33,8 +33,8 @@
 
 namespace pkv {
 
-// STAGES_ = 0: four stages when K + V fit 72 KB per CTA (head_dim 128: three
-// CTAs per SM), else three (the merge area of 16 heads needs that much).
+// STAGES_ = 0: three stages (48 KB of K + V at head_dim 128; four measured
+// the same on B200, and three leave room for the merge area of 16 heads).
 template <int D, int BS, int NW, int STAGES_ = 0>
 struct MmaE4m3Cfg {
     static constexpr int TILE = 16 * NW;        // tokens per stage
@@ -43,7 +43,6 @@ struct MmaE4m3Cfg {
     static constexpr int BLK_BYTES = BS * D;    // one (block, head) page
     static constexpr int BPT = TILE / BS;
     static constexpr int STAGE_BYTES = TILE * D;  // one of K / V
-    static constexpr int FIT = 73728 / (2 * STAGE_BYTES);
     static constexpr int STAGES = STAGES_ ? STAGES_ : 3;
     static_assert(TILE % BS == 0 && BS % 8 == 0 && D % 128 == 0, "whole blocks, 128-byte rows");
 
