@@ -285,3 +285,26 @@ def test_sliding_window_released_blocks_are_never_read(dtype, G):
     b = DeviceInputs(inp).decode(sliding_window=W).clone()
     assert pkv.pkv_device_status(clear=True) == 0
     assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# a grid of several waves, every element
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("partition,W", [(64, 0), (0, 0), (64, 100), (512, 0)])
+def test_many_waves_all_rows(dtype, partition, W):
+    """160 ragged sequences x 8 KV heads x 4-head groups (a grid of several
+    waves of CTAs per SM): every output element against the oracle, and the
+    longest-first order changes no bit."""
+    g = np.random.default_rng(33)
+    lens = tuple(int(x) for x in g.integers(1, 700, size=160))
+    cfg = _cfg(dtype, 32, 8, 128, 16, lens)
+    inp = make_decode_inputs(cfg, seed=33)
+    ref = oracle.paged_decode_inputs(inp, window=W)
+    dev = DeviceInputs(inp)
+    got = to_f64(dev.decode(partition_size=partition, fill_out=5.0, sliding_window=W))
+    assert_close(got, ref, dtype, f"{dtype} P={partition} W={W}")
+    order = torch.from_numpy(pkv.pkv_decode_schedule_order(inp.context_lens)).cuda()
+    again = to_f64(dev.decode(partition_size=partition, seq_order=order, fill_out=-5.0,
+                              sliding_window=W))
+    assert np.array_equal(got, again)
