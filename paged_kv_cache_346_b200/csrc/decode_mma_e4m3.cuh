@@ -33,21 +33,26 @@
 
 namespace pkv {
 
-// STAGES_ = 0: three stages (48 KB of K + V at head_dim 128; four measured
-// the same on B200, and three leave room for the merge area of 16 heads).
+// Every warp streams its own 16-token slices through a private ring of
+// STAGES stages (STAGES_ = 0: 4 at head_dim 128, 2 at 256), one 16-row TMA box
+// per 128 columns of K and of V per slice, issued by the warp's lane 0, so no
+// barrier ties the warps together until the final merge.  Measured on B200
+// against one ring shared by the CTA (refilled after a CTA barrier by one
+// thread): +20 % on the MHA layer, +15 % on the GQA batch, +24-32 % on long
+// contexts.
 template <int D, int BS, int NW, int STAGES_ = 0>
 struct MmaE4m3Cfg {
-    static constexpr int TILE = 16 * NW;        // tokens per stage
-    static constexpr int NX = D / 128;          // 128-column boxes per row
-    static constexpr int BOX_BYTES = BS * 128;  // one box: BS rows x 128 bytes
-    static constexpr int BLK_BYTES = BS * D;    // one (block, head) page
-    static constexpr int BPT = TILE / BS;
-    static constexpr int STAGE_BYTES = TILE * D;  // one of K / V
-    static constexpr int STAGES = STAGES_ ? STAGES_ : 3;
-    static_assert(TILE % BS == 0 && BS % 8 == 0 && D % 128 == 0, "whole blocks, 128-byte rows");
+    static constexpr int TILE = 16 * NW;          // tokens per round of all warps
+    static constexpr int NX = D / 128;            // 128-column boxes per row
+    static constexpr int BOX_BYTES = 16 * 128;    // one box: 16 rows x 128 bytes
+    static constexpr int SLICE_BYTES = 16 * D;    // one warp's 16 tokens of K (or V)
+    static constexpr int STAGES = STAGES_ ? STAGES_ : (D <= 128 ? 4 : 2);
+    static constexpr int WARP_RING = STAGES * 2 * SLICE_BYTES;
+    static constexpr int RING_BYTES = NW * WARP_RING;
+    static_assert(BS % 16 == 0 && D % 128 == 0, "16-token slices of 128-byte rows");
 
     static int smem_bytes(int partition_size) {
-        return 1024 + round_up(partition_size / BS * 4, 128) + 1024 + STAGES * 2 * STAGE_BYTES;
+        return 1024 + round_up(partition_size / BS * 4, 128) + 1024 + RING_BYTES;
     }
 };
 
@@ -85,7 +90,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     using C = MmaE4m3Cfg<D, BS, NW, STAGES_>;
     using M = Mma<__half>;
     constexpr int TILE = C::TILE, NX = C::NX, BOX_BYTES = C::BOX_BYTES;
-    constexpr int BLK_BYTES = C::BLK_BYTES, BPT = C::BPT, STAGE_BYTES = C::STAGE_BYTES;
+    constexpr int SLICE_BYTES = C::SLICE_BYTES, WARP_RING = C::WARP_RING;
     constexpr int STAGES = C::STAGES;
     constexpr int KSTEPS = D / 16;   // k-steps of QK, m-tiles of PV (one 16-byte chunk each)
     constexpr int KP = KSTEPS / 2;   // ldmatrix.x4 loads per warp tile (two chunks each)
@@ -122,10 +127,11 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     const int t0 = sp.base + part * P;
     const int ntok = min(L, t0 + P) - t0;
     const int mask_lo = part == 0 ? sp.lo - sp.base : 0;
-    const int ntiles = (ntok + TILE - 1) / TILE;
     const int nblk = (ntok + BS - 1) / BS;
+    // this warp's slices: tokens [k * TILE + warp * 16, + 16), k < nslices
+    const int nslices = ntok > warp * 16 ? (ntok - warp * 16 + TILE - 1) / TILE : 0;
 
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem_mma8);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem_mma8);  // [NW][STAGES]
     int32_t* s_tab = reinterpret_cast<int32_t*>(smem_mma8 + 1024);
     unsigned char* s_kv;
     {
@@ -140,30 +146,27 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
 #pragma unroll
-        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < NW * STAGES; ++s) mbar_init(&full[s], 1);
         fence_barrier_init();
     }
     __syncthreads();
 
     const uint64_t pol = policy_evict_first();
-    auto issue = [&](int tile, int stage) {
-        const int jb = tile * BPT;
-        const int je = min(nblk, jb + BPT);
-        mbar_arrive_expect_tx(&full[stage], (uint32_t)((je - jb) * BLK_BYTES * 2));
-        unsigned char* kd = s_kv + stage * 2 * STAGE_BYTES;
-        unsigned char* vd = kd + STAGE_BYTES;
-        for (int j = jb; j < je; ++j) {
-            const int y = (s_tab[j] * a.num_kv_heads + kvh) * BS;
+    unsigned char* ring = s_kv + warp * WARP_RING;
+    uint64_t* wfull = full + warp * STAGES;
+    auto issue = [&](int k, int stage) {  // this warp's slice k (lane 0 only)
+        const int tok = k * TILE + warp * 16;
+        const int y = (s_tab[tok / BS] * a.num_kv_heads + kvh) * BS + tok % BS;
+        mbar_arrive_expect_tx(&wfull[stage], (uint32_t)(2 * SLICE_BYTES));
+        unsigned char* kd = ring + stage * 2 * SLICE_BYTES;
 #pragma unroll
-            for (int x = 0; x < NX; ++x) {
-                const int off = ((j - jb) * NX + x) * BOX_BYTES;
-                tma_load_2d(kd + off, &tmk, x * 128, y, &full[stage], pol);
-                tma_load_2d(vd + off, &tmv, x * 128, y, &full[stage], pol);
-            }
+        for (int x = 0; x < NX; ++x) {
+            tma_load_2d(kd + x * BOX_BYTES, &tmk, x * 128, y, &wfull[stage], pol);
+            tma_load_2d(kd + SLICE_BYTES + x * BOX_BYTES, &tmv, x * 128, y, &wfull[stage], pol);
         }
     };
-    if (tid == 0) {
-        const int pre = min(STAGES, ntiles);
+    if (lane == 0) {
+        const int pre = min(STAGES, nslices);
         for (int s = 0; s < pre; ++s) issue(s, s);
     }
 
@@ -232,20 +235,20 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     // chunk c), (tokens 0-7, chunk c + 1), (tokens 8-15, chunk c + 1)
     const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1);
     const int lchunk = lane >> 4;
+    const int swz = lrow & 7;
 
-    for (int it = 0; it < ntiles; ++it) {
+    for (int it = 0; it < nslices; ++it) {
         const int stage = it % STAGES;
-        const bool ok = mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status);
-        if (!ok) s_abort = 1;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&wfull[stage],
+                                                          (uint32_t)((it / STAGES) & 1), a.status));
+        if (!ok) {
+            s_abort = 1;
+            break;
+        }
         const int wvalid = ntok - (it * TILE + warp * 16);
         const int wlo = mask_lo - (it * TILE + warp * 16);
-        const bool work = ok && wvalid > 0 && wlo < 16 && wlo < wvalid;
-        const int tt0 = warp * 16;
-        const int jw = tt0 / BS;
-        const int rr = tt0 % BS + lrow;
-        const uint32_t kbase = smem_u32(s_kv + stage * 2 * STAGE_BYTES) +
-                               (uint32_t)(jw * NX * BOX_BYTES + rr * 128);
-        const int swz = rr & 7;
+        const bool work = wlo < 16 && wlo < wvalid;
+        const uint32_t kbase = smem_u32(ring + stage * 2 * SLICE_BYTES) + (uint32_t)(lrow * 128);
         auto addr = [&](int kp) {  // chunk pair kp: chunks 2 kp, 2 kp + 1
             const int chunk = 2 * kp + lchunk;
             return kbase + (chunk >> 3) * BOX_BYTES + (((chunk & 7) ^ swz) << 4);
@@ -255,7 +258,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
 #pragma unroll
             for (int kp = 0; kp < (EARLY ? KP : 1); ++kp) {
                 ldsm_x4(addr(kp), kf[kp]);
-                ldsm_x4_trans(addr(kp) + STAGE_BYTES, vf[kp]);
+                ldsm_x4_trans(addr(kp) + SLICE_BYTES, vf[kp]);
             }
         }
         auto math = [&]() {
@@ -348,7 +351,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) vc[i] = vf[kp < (EARLY ? KP : 1) ? kp : 0][i];
                 } else {
-                    ldsm_x4_trans(addr(kp) + STAGE_BYTES, vc);
+                    ldsm_x4_trans(addr(kp) + SLICE_BYTES, vc);
                 }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {  // m-tile 2 kp + h
@@ -382,17 +385,17 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
             }
         };
         if (!EARLY && work) math();
-        __syncthreads();  // the stage is free again
-        if (s_abort) break;
-        if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage);
+        __syncwarp();  // the warp's reads of the stage are done: refill it
+        if (lane == 0 && it + STAGES < nslices) issue(it + STAGES, stage);
         if (EARLY && work) math();
     }
+    __syncthreads();  // every warp is out of its ring (or gave up)
     if (s_abort) return;
     pdl_launch_dependents();
 
     // merge the warps; A rows g, g + 8 of m-tile mt are dims 16 mt + 2 g, + 1
     using A = MergeArea<D, NH, NW>;
-    static_assert(A::BYTES <= STAGES * 2 * STAGE_BYTES, "merge area");
+    static_assert(A::BYTES <= C::RING_BYTES, "merge area");
     float* red = reinterpret_cast<float*>(s_kv);
     float* red_m = red + NW * NH * A::RP;
     float* red_l = red_m + NW * NH;
@@ -432,9 +435,9 @@ cudaError_t launch_decode_mma_e4m3(const DecodeArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
     CUtensorMap tk, tv;
-    e = make_cache_tensor_map(&tk, a.k_cache, 1, false, D, rows, BS);
+    e = make_cache_tensor_map(&tk, a.k_cache, 1, false, D, rows, 16);
     if (e != cudaSuccess) return e;
-    e = make_cache_tensor_map(&tv, a.v_cache, 1, false, D, rows, BS);
+    e = make_cache_tensor_map(&tv, a.v_cache, 1, false, D, rows, 16);
     if (e != cudaSuccess) return e;
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
     kern<<<grid, NW * 32, C::smem_bytes(a.partition_size), stream>>>(a, tk, tv);
