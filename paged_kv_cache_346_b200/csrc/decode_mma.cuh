@@ -92,20 +92,24 @@ struct Mma<__nv_bfloat16> {
     }
 };
 
-// STAGES_ = 0: the most stages (2 or 3) whose ring lets three CTAs share an SM.
+// Every warp streams its own 16-token slices through a private ring of
+// STAGES stages (STAGES_ = 0: as many as fit 64 KB per CTA, at least 2), one
+// 16-row TMA box per 64 columns of K and of V per slice, issued by the warp's
+// lane 0: no barrier ties the warps together until the final merge.
 template <int D, int BS, int NW, int STAGES_ = 0>
 struct MmaCfg {
-    static constexpr int TILE = 16 * NW;         // tokens per stage
-    static constexpr int NX = D / 64;            // 64-column boxes per row
-    static constexpr int BOX_BYTES = BS * 128;   // one box: BS rows x 128 bytes
-    static constexpr int BLK_BYTES = BS * D * 2; // one (block, head) page
-    static constexpr int BPT = TILE / BS;
-    static constexpr int STAGE_BYTES = TILE * D * 2;  // one of K / V
-    static constexpr int STAGES = STAGES_ ? STAGES_ : ((2 * STAGE_BYTES) * 3 <= 73728 ? 3 : 2);
-    static_assert(TILE % BS == 0 && BS % 8 == 0, "whole blocks per stage, swizzle rows");
+    static constexpr int TILE = 16 * NW;          // tokens per round of all warps
+    static constexpr int NX = D / 64;             // 64-column boxes per row
+    static constexpr int BOX_BYTES = 16 * 128;    // one box: 16 rows x 128 bytes
+    static constexpr int SLICE_BYTES = 16 * D * 2;  // one warp's 16 tokens of K (or V)
+    static constexpr int FIT = 65536 / (NW * 2 * SLICE_BYTES);
+    static constexpr int STAGES = STAGES_ ? STAGES_ : (FIT >= 4 ? 4 : (FIT >= 2 ? FIT : 2));
+    static constexpr int WARP_RING = STAGES * 2 * SLICE_BYTES;
+    static constexpr int RING_BYTES = NW * WARP_RING;
+    static_assert(BS % 16 == 0, "16-token slices");
 
     static int smem_bytes(int partition_size) {
-        return 1024 + round_up(partition_size / BS * 4, 128) + 1024 + STAGES * 2 * STAGE_BYTES;
+        return 1024 + round_up(partition_size / BS * 4, 128) + 1024 + RING_BYTES;
     }
 };
 
@@ -118,7 +122,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     using C = MmaCfg<D, BS, NW, STAGES_>;
     using M = Mma<T>;
     constexpr int TILE = C::TILE, NX = C::NX, BOX_BYTES = C::BOX_BYTES;
-    constexpr int BLK_BYTES = C::BLK_BYTES, BPT = C::BPT, STAGE_BYTES = C::STAGE_BYTES;
+    constexpr int SLICE_BYTES = C::SLICE_BYTES, WARP_RING = C::WARP_RING;
     constexpr int STAGES = C::STAGES;
     constexpr int KSTEPS = D / 16;   // k-steps of the QK product, m-tiles of PV
     constexpr int RB = NH / 8;       // 8-head row blocks
@@ -156,10 +160,11 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     const int t0 = sp.base + part * P;
     const int ntok = min(L, t0 + P) - t0;
     const int mask_lo = part == 0 ? sp.lo - sp.base : 0;  // tokens ahead of the window
-    const int ntiles = (ntok + TILE - 1) / TILE;
     const int nblk = (ntok + BS - 1) / BS;
+    // this warp's slices: tokens [k * TILE + warp * 16, + 16), k < nslices
+    const int nslices = ntok > warp * 16 ? (ntok - warp * 16 + TILE - 1) / TILE : 0;
 
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem_mma);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem_mma);  // [NW][STAGES]
     int32_t* s_tab = reinterpret_cast<int32_t*>(smem_mma + 1024);
     unsigned char* s_kv;
     {
@@ -174,30 +179,29 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
 #pragma unroll
-        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < NW * STAGES; ++s) mbar_init(&full[s], 1);
         fence_barrier_init();
     }
     __syncthreads();
 
     const uint64_t pol = policy_evict_first();
-    auto issue = [&](int tile, int stage) {
-        const int jb = tile * BPT;
-        const int je = min(nblk, jb + BPT);
-        mbar_arrive_expect_tx(&full[stage], (uint32_t)((je - jb) * BLK_BYTES * 2));
-        unsigned char* kd = s_kv + stage * 2 * STAGE_BYTES;
-        unsigned char* vd = kd + STAGE_BYTES;
-        for (int j = jb; j < je; ++j) {
-            const int y = (s_tab[j] * a.num_kv_heads + kvh) * BS;
+    // this warp's ring and barriers, recomputed where used (no long-lived
+    // 64-bit pointers next to the fragment registers)
+    const uint32_t ring_s = smem_u32(s_kv) + (uint32_t)(warp * WARP_RING);
+    auto issue = [&](int k, int stage) {  // this warp's slice k (lane 0 only)
+        const int tok = k * TILE + warp * 16;
+        const int y = (s_tab[tok / BS] * a.num_kv_heads + kvh) * BS + tok % BS;
+        uint64_t* bar = full + warp * STAGES + stage;
+        mbar_arrive_expect_tx(bar, (uint32_t)(2 * SLICE_BYTES));
+        unsigned char* kd = s_kv + warp * WARP_RING + stage * 2 * SLICE_BYTES;
 #pragma unroll
-            for (int x = 0; x < NX; ++x) {
-                const int off = ((j - jb) * NX + x) * BOX_BYTES;
-                tma_load_2d(kd + off, &tmk, x * 64, y, &full[stage], pol);
-                tma_load_2d(vd + off, &tmv, x * 64, y, &full[stage], pol);
-            }
+        for (int x = 0; x < NX; ++x) {
+            tma_load_2d(kd + x * BOX_BYTES, &tmk, x * 64, y, bar, pol);
+            tma_load_2d(kd + SLICE_BYTES + x * BOX_BYTES, &tmv, x * 64, y, bar, pol);
         }
     };
-    if (tid == 0) {
-        const int pre = min(STAGES, ntiles);
+    if (lane == 0) {
+        const int pre = min(STAGES, nslices);
         for (int s = 0; s < pre; ++s) issue(s, s);
     }
 
@@ -237,19 +241,20 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     const int lrow = (lane >> 4) * 8 + (lane & 7);
     const int lchunk = (lane >> 3) & 1;
 
-    for (int it = 0; it < ntiles; ++it) {
+    const int swz = lrow & 7;
+
+    for (int it = 0; it < nslices; ++it) {
         const int stage = it % STAGES;
-        const bool ok = mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status);
-        if (!ok) s_abort = 1;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(full + warp * STAGES + stage,
+                                                          (uint32_t)((it / STAGES) & 1), a.status));
+        if (!ok) {
+            s_abort = 1;
+            break;
+        }
         const int wvalid = ntok - (it * TILE + warp * 16);
         const int wlo = mask_lo - (it * TILE + warp * 16);
-        const bool work = ok && wvalid > 0 && wlo < 16 && wlo < wvalid;
-        const int tt0 = warp * 16;           // first token of the warp in the stage
-        const int jw = tt0 / BS;             // its block within the stage
-        const int rr = tt0 % BS + lrow;      // this lane's row within that block
-        const uint32_t kbase = smem_u32(s_kv + stage * 2 * STAGE_BYTES) +
-                               (uint32_t)(jw * NX * BOX_BYTES + rr * 128);
-        const int swz = rr & 7;
+        const bool work = wlo < 16 && wlo < wvalid;
+        const uint32_t kbase = ring_s + (uint32_t)(stage * 2 * SLICE_BYTES + lrow * 128);
         auto kaddr = [&](int ks) {
             const int chunk = ks * 2 + lchunk;  // 16-byte chunk of the row
             return kbase + (chunk >> 3) * BOX_BYTES + (((chunk & 7) ^ swz) << 4);
@@ -261,7 +266,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
 #pragma unroll
             for (int ks = 0; ks < (EARLY ? KSTEPS : 1); ++ks) {
                 ldsm_x4(kaddr(ks), kf[ks]);
-                ldsm_x4_trans(kaddr(ks) + STAGE_BYTES, vf[ks]);
+                ldsm_x4_trans(kaddr(ks) + SLICE_BYTES, vf[ks]);
             }
         }
         auto math = [&]() {
@@ -326,7 +331,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) va[i] = vf[mt < (EARLY ? KSTEPS : 1) ? mt : 0][i];
                 } else {
-                    ldsm_x4_trans(kaddr(mt) + STAGE_BYTES, va);
+                    ldsm_x4_trans(kaddr(mt) + SLICE_BYTES, va);
                 }
                 if (partial) {
                     // zero values of masked tokens (0 * NaN would poison)
@@ -350,17 +355,17 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
             }
         };
         if (!EARLY && work) math();
-        __syncthreads();  // the stage is free again
-        if (s_abort) break;
-        if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage);
+        __syncwarp();  // the warp's reads of the stage are done: refill it
+        if (lane == 0 && it + STAGES < nslices) issue(it + STAGES, stage);
         if (EARLY && work) math();
     }
+    __syncthreads();  // every warp is out of its ring (or gave up)
     if (s_abort) return;
     pdl_launch_dependents();
 
     // merge the warps (padded rows: lanes of one store hit distinct banks)
     using A = MergeArea<D, NH, NW>;
-    static_assert(A::BYTES <= STAGES * 2 * STAGE_BYTES, "merge area");
+    static_assert(A::BYTES <= C::RING_BYTES, "merge area");
     float* red = reinterpret_cast<float*>(s_kv);
     float* red_m = red + NW * NH * A::RP;
     float* red_l = red_m + NW * NH;
@@ -399,9 +404,9 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
     const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
     CUtensorMap tk, tv;
     const bool bf = std::is_same<T, __nv_bfloat16>::value;
-    e = make_cache_tensor_map(&tk, a.k_cache, 2, bf, D, rows, BS);
+    e = make_cache_tensor_map(&tk, a.k_cache, 2, bf, D, rows, 16);
     if (e != cudaSuccess) return e;
-    e = make_cache_tensor_map(&tv, a.v_cache, 2, bf, D, rows, BS);
+    e = make_cache_tensor_map(&tv, a.v_cache, 2, bf, D, rows, 16);
     if (e != cudaSuccess) return e;
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
     kern<<<grid, NW * 32, C::smem_bytes(a.partition_size), stream>>>(a, tk, tv);

@@ -34,7 +34,7 @@
 namespace pkv {
 
 // Every warp streams its own 16-token slices through a private ring of
-// STAGES stages (STAGES_ = 0: 4 at head_dim 128, 2 at 256), one 16-row TMA box
+// STAGES stages (STAGES_ = 0: 4), one 16-row TMA box
 // per 128 columns of K and of V per slice, issued by the warp's lane 0, so no
 // barrier ties the warps together until the final merge.  Measured on B200
 // against one ring shared by the CTA (refilled after a CTA barrier by one
@@ -46,7 +46,7 @@ struct MmaE4m3Cfg {
     static constexpr int NX = D / 128;            // 128-column boxes per row
     static constexpr int BOX_BYTES = 16 * 128;    // one box: 16 rows x 128 bytes
     static constexpr int SLICE_BYTES = 16 * D;    // one warp's 16 tokens of K (or V)
-    static constexpr int STAGES = STAGES_ ? STAGES_ : (D <= 128 ? 4 : 2);
+    static constexpr int STAGES = STAGES_ ? STAGES_ : 4;
     static constexpr int WARP_RING = STAGES * 2 * SLICE_BYTES;
     static constexpr int RING_BYTES = NW * WARP_RING;
     static_assert(BS % 16 == 0 && D % 128 == 0, "16-token slices of 128-byte rows");
@@ -152,17 +152,19 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     __syncthreads();
 
     const uint64_t pol = policy_evict_first();
-    unsigned char* ring = s_kv + warp * WARP_RING;
-    uint64_t* wfull = full + warp * STAGES;
+    // this warp's ring and barriers, recomputed where used (no long-lived
+    // 64-bit pointers next to the fragment registers)
+    const uint32_t ring_s = smem_u32(s_kv) + (uint32_t)(warp * WARP_RING);
     auto issue = [&](int k, int stage) {  // this warp's slice k (lane 0 only)
         const int tok = k * TILE + warp * 16;
         const int y = (s_tab[tok / BS] * a.num_kv_heads + kvh) * BS + tok % BS;
-        mbar_arrive_expect_tx(&wfull[stage], (uint32_t)(2 * SLICE_BYTES));
-        unsigned char* kd = ring + stage * 2 * SLICE_BYTES;
+        uint64_t* bar = full + warp * STAGES + stage;
+        mbar_arrive_expect_tx(bar, (uint32_t)(2 * SLICE_BYTES));
+        unsigned char* kd = s_kv + warp * WARP_RING + stage * 2 * SLICE_BYTES;
 #pragma unroll
         for (int x = 0; x < NX; ++x) {
-            tma_load_2d(kd + x * BOX_BYTES, &tmk, x * 128, y, &wfull[stage], pol);
-            tma_load_2d(kd + SLICE_BYTES + x * BOX_BYTES, &tmv, x * 128, y, &wfull[stage], pol);
+            tma_load_2d(kd + x * BOX_BYTES, &tmk, x * 128, y, bar, pol);
+            tma_load_2d(kd + SLICE_BYTES + x * BOX_BYTES, &tmv, x * 128, y, bar, pol);
         }
     };
     if (lane == 0) {
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
 
     for (int it = 0; it < nslices; ++it) {
         const int stage = it % STAGES;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&wfull[stage],
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(full + warp * STAGES + stage,
                                                           (uint32_t)((it / STAGES) & 1), a.status));
         if (!ok) {
             s_abort = 1;
@@ -248,7 +250,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         const int wvalid = ntok - (it * TILE + warp * 16);
         const int wlo = mask_lo - (it * TILE + warp * 16);
         const bool work = wlo < 16 && wlo < wvalid;
-        const uint32_t kbase = smem_u32(ring + stage * 2 * SLICE_BYTES) + (uint32_t)(lrow * 128);
+        const uint32_t kbase = ring_s + (uint32_t)(stage * 2 * SLICE_BYTES + lrow * 128);
         auto addr = [&](int kp) {  // chunk pair kp: chunks 2 kp, 2 kp + 1
             const int chunk = 2 * kp + lchunk;
             return kbase + (chunk >> 3) * BOX_BYTES + (((chunk & 7) ^ swz) << 4);
