@@ -325,6 +325,19 @@ PKV_API int pkv_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const v
  */
 PKV_API int pkv_device_status(unsigned int* flags, int clear);
 
+/*
+ * Failure-detection self-test.  Every wait inside the decode kernels (for a
+ * page copy to land) is bounded: after ~2 s it gives up, sets
+ * PKV_DEV_TIMEOUT, lets its own copies still in flight land (again bounded)
+ * and leaves, so a broken input or a lost copy ends the kernel with a status
+ * the host reads instead of a hung GPU.  This launches one thread that makes
+ * the same bounded wait on a barrier that nothing completes, giving up after
+ * limit_cycles clock cycles (1 .. 4e9; ~0.5 ms per 1e6 at 2 GHz); afterwards
+ * pkv_device_status reports PKV_DEV_TIMEOUT and the device stays usable.
+ * Returns PKV_OK, PKV_EINVAL or PKV_ECUDA.
+ */
+PKV_API int pkv_debug_wait_timeout(long long limit_cycles, pkv_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Host block allocator ("pagedattention vllm" §Memory Management: a free list,
  * allocate on demand, free when the sequence completes; §Copy-on-Write

@@ -31,7 +31,7 @@ __all__ = [
     "PKV_KERNEL_SIMT", "PKV_KERNEL_MMA", "PKV_DEV_BAD_BLOCK", "PKV_DEV_BAD_LEN",
     "PKV_DEV_BAD_SLOT", "PKV_DEV_TIMEOUT", "PKV_DEV_BAD_ORDER", "torch_dtype_code",
     "pkv_decode_schedule_order", "pkv_paged_attention_decode_e4m3", "pkv_kv_cache_append_e4m3",
-    "PKV_E4M3",
+    "PKV_E4M3", "pkv_debug_wait_timeout",
 ]
 
 _DTYPE = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16,
@@ -292,6 +292,13 @@ def pkv_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tenso
                               _ptr(block_pairs), block_pairs.numel() // 2, Ns, Nd, Hkv, D, bs,
                               torch_dtype_code(src_k.dtype), _stream(stream)),
           "pkv_swap_blocks")
+
+
+def pkv_debug_wait_timeout(limit_cycles: int, *, stream=None) -> None:
+    """Run the bounded-wait self-test: one kernel gives up waiting after
+    limit_cycles clock cycles and flags PKV_DEV_TIMEOUT."""
+    check(lib.pkv_debug_wait_timeout(int(limit_cycles), _stream(stream)),
+          "pkv_debug_wait_timeout")
 
 
 def pkv_device_status(clear: bool = False) -> int:

@@ -54,6 +54,7 @@ SIGNATURES = {
     "pkv_swap_blocks": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                _i32, _vp]),
     "pkv_device_status": (_i32, [_c.POINTER(_c.c_uint), _i32]),
+    "pkv_debug_wait_timeout": (_i32, [_c.c_longlong, _vp]),
     "pkv_alloc_create": (_i32, [_i32, _i32, _c.POINTER(_vp)]),
     "pkv_alloc_create_swap": (_i32, [_i32, _i32, _i32, _c.POINTER(_vp)]),
     "pkv_alloc_swap_out": (_i32, [_vp, _i64, _vp, _i32, _c.POINTER(_i32)]),

@@ -6,6 +6,8 @@
 #include <cmath>
 #include <cstdint>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "cache_ops.cuh"
 #include "decode_dispatch.cuh"
 #include "decode_mma.cuh"
@@ -15,6 +17,14 @@ namespace pkv {
 
 // The device status word (one per device), read by pkv_device_status.
 __device__ unsigned int g_status_word;
+
+// An NVTX range around each call that launches device work, so a timeline
+// (ncu, Nsight Systems) shows the library's calls by name.  Header-only NVTX:
+// without a tool attached a range costs a few nanoseconds.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
 
 namespace {
 
@@ -263,6 +273,7 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
                                float scale, int sliding_window, pkv_dtype dtype,
                                int partition_size, void* workspace, size_t workspace_bytes,
                                pkv_kernel kernel, pkv_stream_t stream) {
+    NvtxRange range("pkv_paged_attention_decode");
     return pkv::decode_impl(out, q, k_cache, v_cache, nullptr, nullptr, false, block_tables,
                             context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
                             head_dim, block_size, max_blocks_per_seq, num_blocks,
@@ -280,6 +291,7 @@ int pkv_paged_attention_decode_e4m3(void* out, const void* q, const void* k_cach
                                     pkv_dtype dtype, int partition_size, void* workspace,
                                     size_t workspace_bytes, pkv_kernel kernel,
                                     pkv_stream_t stream) {
+    NvtxRange range("pkv_paged_attention_decode_e4m3");
     return pkv::decode_impl(out, q, k_cache, v_cache, k_scale, v_scale, true, block_tables,
                             context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
                             head_dim, block_size, max_blocks_per_seq, num_blocks,
@@ -291,6 +303,7 @@ int pkv_kv_cache_append(void* k_cache, void* v_cache, const void* k, const void*
                         const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
                         int head_dim, int block_size, int num_blocks, pkv_dtype dtype,
                         pkv_stream_t stream) {
+    NvtxRange range("pkv_kv_cache_append");
     const int es = elem_size(dtype);
     if (es == 0 || num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
         num_blocks <= 0 || (head_dim * es) % 16 != 0)
@@ -312,6 +325,7 @@ int pkv_kv_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, const 
                              const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
                              int head_dim, int block_size, int num_blocks, pkv_dtype in_dtype,
                              pkv_stream_t stream) {
+    NvtxRange range("pkv_kv_cache_append_e4m3");
     if ((in_dtype != PKV_F16 && in_dtype != PKV_BF16) || num_tokens < 0 || num_kv_heads <= 0 ||
         head_dim <= 0 || head_dim % 16 != 0 || block_size <= 0 || num_blocks <= 0)
         return PKV_EINVAL;
@@ -332,6 +346,7 @@ int pkv_kv_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, const 
 int pkv_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_pairs, int num_pairs,
                     int num_kv_heads, int head_dim, int block_size, int num_blocks,
                     pkv_dtype dtype, pkv_stream_t stream) {
+    NvtxRange range("pkv_copy_blocks");
     const int es = elem_size(dtype);
     if (es == 0 || num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
         num_blocks <= 0)
@@ -352,6 +367,7 @@ int pkv_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src
                     const int32_t* block_pairs, int num_pairs, int src_num_blocks,
                     int dst_num_blocks, int num_kv_heads, int head_dim, int block_size,
                     pkv_dtype dtype, pkv_stream_t stream) {
+    NvtxRange range("pkv_swap_blocks");
     const int es = elem_size(dtype);
     if (es == 0 || num_pairs < 0 || src_num_blocks <= 0 || dst_num_blocks <= 0 ||
         num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
@@ -370,6 +386,14 @@ int pkv_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src
     cudaError_t e = launch_swap_blocks(dk, dv, sk, sv, static_cast<const int32_t*>(pp), num_pairs,
                                        block_bytes, src_num_blocks, dst_num_blocks, st,
                                        reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+int pkv_debug_wait_timeout(long long limit_cycles, pkv_stream_t stream) {
+    if (limit_cycles < 1 || limit_cycles > kWaitCycles) return PKV_EINVAL;
+    unsigned int* st;
+    if (status_word(&st) != cudaSuccess) return PKV_ECUDA;
+    cudaError_t e = launch_wait_timeout(limit_cycles, st, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
 

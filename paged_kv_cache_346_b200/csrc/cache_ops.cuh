@@ -29,4 +29,8 @@ cudaError_t launch_swap_blocks(void* dst_k, void* dst_v, const void* src_k, cons
                                int src_blocks, int dst_blocks, unsigned int* status,
                                cudaStream_t stream);
 
+// One thread waits (bounded by `limit` clock cycles) on an mbarrier that
+// nothing completes, flags PKV_DEV_TIMEOUT and returns (selftest.cu).
+cudaError_t launch_wait_timeout(long long limit, unsigned int* status, cudaStream_t stream);
+
 }  // namespace pkv

@@ -245,6 +245,12 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                                                           (uint32_t)((it / STAGES) & 1), a.status));
         if (!ok) {
             s_abort = 1;
+            // let this warp's copies still in flight land (bounded) before
+            // the CTA leaves
+            if (lane == 0)
+                for (int k = it; k < min(nslices, it + STAGES); ++k)
+                    mbar_wait(full + warp * STAGES + k % STAGES, (uint32_t)((k / STAGES) & 1),
+                              a.status);
             break;
         }
         const int wvalid = ntok - (it * TILE + warp * 16);

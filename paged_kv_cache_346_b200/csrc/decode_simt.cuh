@@ -397,6 +397,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::TH
     W.init(reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D, nh,
            a.k_scale ? a.scale_log2 * a.k_scale[kvh] : a.scale_log2, lane);
     const uint64_t pol = WS ? 0 : policy_evict_first();
+    int it_stop = ntiles;  // the tile a timed-out wait stopped at
     for (int it = 0; it < ntiles; ++it) {
         const int stage = it % STAGES;
         if (!mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status)) s_abort = 1;
@@ -415,13 +416,22 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::TH
             if (lane == 0) mbar_arrive(&empty[stage]);
         } else {
             __syncthreads();
-            if (s_abort) break;
+            if (s_abort) {
+                it_stop = it;
+                break;
+            }
             if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage, pol);
         }
         if (W.EARLY && work) W.compute(wlo, wvalid, s_p[warp]);
     }
     if (WS) __syncthreads();  // producer and consumers: every stage consumed
-    if (s_abort) return;
+    if (s_abort) {
+        // let the copies still in flight land (bounded) before the CTA leaves
+        if (!WS && tid == 0)
+            for (int k = it_stop; k < min(ntiles, it_stop + STAGES); ++k)
+                mbar_wait(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), a.status);
+        return;
+    }
     if (!WS) pdl_launch_dependents();
 
     // 6. merge the warps

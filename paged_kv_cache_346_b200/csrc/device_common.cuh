@@ -59,19 +59,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for phase `parity` of the barrier to complete, giving up after
-// kWaitCycles; on giving up the status word gets PKV_DEV_TIMEOUT.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          unsigned int* status) {
+// `limit` clock cycles; on giving up the status word gets PKV_DEV_TIMEOUT.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
+                                                unsigned int* status, long long limit) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(a, parity)) {
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             flag(status, PKV_DEV_TIMEOUT);
             return false;
         }
     }
     return true;
+}
+
+// The kernels' waits: kWaitCycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned int* status) {
+    return mbar_wait_limit(bar, parity, status, kWaitCycles);
 }
 
 // L2 policy for data read exactly once (the K/V pages of a decode step).

@@ -161,3 +161,10 @@ def test_schedule_order_longest_first():
     lens = np.array([5, 100, 7, 100, 0, 64], dtype=np.int32)
     assert pkv.pkv_decode_schedule_order(lens).tolist() == [1, 3, 5, 2, 0, 4]
     assert pkv.pkv_decode_schedule_order(np.zeros(0, np.int32)).tolist() == []
+
+
+def test_wait_timeout_selftest_host_checks():
+    f = b.lib.pkv_debug_wait_timeout
+    assert f(0, None) == b.PKV_EINVAL
+    assert f(-5, None) == b.PKV_EINVAL
+    assert f(5_000_000_000, None) == b.PKV_EINVAL
