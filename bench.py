@@ -163,7 +163,7 @@ def kernel_source_digest(variant: str) -> str:
 
 def resolve_variant(cfg, kernel: str, kv: str = "same") -> str:
     """The decode kernel the library's automatic choice takes for cfg."""
-    if kv == "e4m3":
+    if kv.startswith("e4m3"):
         if kernel == "mma" or (kernel == "auto" and cfg.group <= 16):
             return "mma_e4m3"
         return "simt_e4m3"
@@ -309,7 +309,8 @@ def run_ours(args, cfg):
 
     # ---- inputs (seeded; each rank its own replica)
     inp = make_decode_inputs(cfg, seed=args.seed + rank)
-    e4m3 = args.kv == "e4m3"
+    e4m3 = args.kv in ("e4m3", "e4m3-page")
+    per_page = args.kv == "e4m3-page"
     if e4m3 and cfg.dtype == "f32":
         raise SystemExit("E4M3 pages take fp16/bf16 q")
 
@@ -320,7 +321,7 @@ def run_ours(args, cfg):
 
     pages = None
     if e4m3:
-        pages = make_e4m3_pages(inp, seed=args.seed + rank)
+        pages = make_e4m3_pages(inp, seed=args.seed + rank, per_page=per_page)
         q = dev(inp.q)
         kc = dev(pages.k_cache).view(torch.float8_e4m3fn)
         vc = dev(pages.v_cache).view(torch.float8_e4m3fn)
@@ -340,10 +341,12 @@ def run_ours(args, cfg):
     sb_idx = torch.from_numpy(slots_np // bs).cuda()
     so_idx = torch.from_numpy(slots_np % bs).cuda()
     if e4m3:
+        ksel = ks[sb_idx] if per_page else ks[None, :]   # [B or 1, Hkv]
+        vsel = vs[sb_idx] if per_page else vs[None, :]
         knew = (kc.view(torch.uint8)[sb_idx, :, so_idx, :].view(torch.float8_e4m3fn).float() *
-                ks[None, :, None]).to(q.dtype).contiguous()
+                ksel[:, :, None]).to(q.dtype).contiguous()
         vnew = (vc.view(torch.uint8)[sb_idx, :, so_idx, :].view(torch.float8_e4m3fn).float() *
-                vs[None, :, None]).to(q.dtype).contiguous()
+                vsel[:, :, None]).to(q.dtype).contiguous()
     else:
         knew = kc.view(-1, H, bs, D)[sb_idx, :, so_idx, :].contiguous()
         vnew = vc.view(-1, H, bs, D)[sb_idx, :, so_idx, :].contiguous()
@@ -450,9 +453,10 @@ def run_ours(args, cfg):
         kp, vp = ctypes.c_void_p(kc.data_ptr()), ctypes.c_void_p(vc.data_ptr())
         if e4m3:
             ksp, vsp = ctypes.c_void_p(ks.data_ptr()), ctypes.c_void_p(vs.data_ptr())
-            append_args = (kp, vp, ptr["knew"], ptr["vnew"], ksp, vsp, ptr["slots"], B, H, D, bs,
-                           N_blocks, dt_code, c_stream)
-            decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ksp, vsp,
+            spb = 1 if per_page else 0
+            append_args = (kp, vp, ptr["knew"], ptr["vnew"], ksp, vsp, spb, ptr["slots"], B, H, D,
+                           bs, N_blocks, dt_code, c_stream)
+            decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ksp, vsp, spb,
                            ptr["bt"], ptr["cl"], ptr.get("order"), B, cfg.num_q_heads, H, D,
                            bs, bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
                            ctypes.c_void_p(ws.data_ptr()), ws.numel(), kern, c_stream)
@@ -526,7 +530,8 @@ def run_ours(args, cfg):
                        "block_size": bs, "partition_size": Pused, "kernel": args.kernel,
                        "schedule": "longest-first" if args.order else "batch order",
                        "sliding_window": W,
-                       "kv_pages": "e4m3 (per-head fp32 scales)" if e4m3 else cfg.dtype,
+                       "kv_pages": ("e4m3 (per-page fp32 scales)" if per_page else
+                                    "e4m3 (per-head fp32 scales)") if e4m3 else cfg.dtype,
                        "q_out": cfg.dtype,
                        "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (%.2f GB of K/V per step)" % (
@@ -788,9 +793,9 @@ def main():
     ap.add_argument("--seed", type=int, default=2)
     ap.add_argument("--window", type=int, default=0,
                     help="sliding window in tokens (0: attend to the whole context)")
-    ap.add_argument("--kv", choices=["same", "e4m3"], default="same",
+    ap.add_argument("--kv", choices=["same", "e4m3", "e4m3-page"], default="same",
                     help="page element type: the workload's, or FP8 E4M3 codes with "
-                         "per-head scales")
+                         "per-head (e4m3) or per-page (e4m3-page) scales")
     ap.add_argument("--no-order", dest="order", action="store_false",
                     help="schedule sequences in batch order instead of longest first")
     ap.add_argument("--cpu-budget", type=float, default=12.0,

@@ -176,11 +176,13 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
 /*
  * Paged decode attention over FP8 E4M3 pages ("pagedattention vllm"
  * §Comparison with Alternatives: the paged layout combines with a quantised
- * cache).  Page element x of KV head g stands for the value
- * E4M3(x) * k_scale[g] (keys) or E4M3(x) * v_scale[g] (values), and the result
- * is pkv_paged_attention_decode's over those values:
- *   out[b,h,:] = softmax_t(scale * k_scale[g] * q[b,h,:] . E4M3(k_t))
- *                weighted sum of v_scale[g] * E4M3(v_t),   g = h / (Hq/Hkv).
+ * cache).  Page element x of KV head g in physical block n stands for the
+ * value E4M3(x) * k_scale[g] (keys) or E4M3(x) * v_scale[g] (values) -- or,
+ * with scale_per_block = 1, k_scale[n * Hkv + g] and v_scale[n * Hkv + g],
+ * one scale per page -- and the result is pkv_paged_attention_decode's over
+ * those values:
+ *   out[b,h,:] = softmax_t(scale * q[b,h,:] . (k_scale * E4M3(k_t)))
+ *                weighted sum of v_scale * E4M3(v_t),   g = h / (Hq/Hkv).
  * Each code is widened exactly (every E4M3 value is a binary16 value).  The
  * tensor-core kernel (AUTO for groups of at most 16 heads) multiplies fp16
  * operands with fp32 accumulation: q enters it scaled by a power of two that
@@ -188,11 +190,14 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
  * falls below the fp16 normal range there), P is rounded to fp16, and the
  * logits are multiplied by scale * k_scale (and the power of two) in fp32.
  * The CUDA-core kernel works in fp32 throughout, k_scale folded into q and
- * v_scale into the accumulator.
+ * v_scale into the accumulator (per page: into that page's logits and
+ * weights); the tensor-core kernel applies a page's v_scale in fp32 to that
+ * page's P.V product, so P stays an fp16 value at most 256.
  *
  * Arguments as pkv_paged_attention_decode, plus:
  *   k_cache, v_cache: device E4M3 codes [num_blocks, Hkv, block_size, head_dim].
- *   k_scale, v_scale: device float32 [num_kv_heads], finite and > 0 (not
+ *   k_scale, v_scale: device float32 [num_kv_heads] (scale_per_block 0) or
+ *       [num_blocks][num_kv_heads] (scale_per_block 1), finite and > 0 (not
  *       checked on the device: the caller's quantisation scales).
  *   dtype: PKV_F16 or PKV_BF16, the type of q and out.
  *   head_dim in {128, 256} (a page row must be at least 128 bytes).
@@ -203,7 +208,8 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
  */
 PKV_API int pkv_paged_attention_decode_e4m3(
     void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
-    const float* v_scale, const int32_t* block_tables, const int32_t* context_lens,
+    const float* v_scale, int scale_per_block, const int32_t* block_tables,
+    const int32_t* context_lens,
     const int32_t* seq_order, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
     int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
     int sliding_window, pkv_dtype dtype, int partition_size, void* workspace,
@@ -273,19 +279,23 @@ PKV_API int pkv_kv_cache_append(void* k_cache, void* v_cache, const void* k, con
  * KV append into E4M3 pages: as pkv_kv_cache_append, but each element is
  * quantised on the way in:
  *   k_cache[s / bs, h, s % bs, d] = E4M3(k[t, h, d] / k_scale[h]),
- * same for v with v_scale.  The division is a float32 division (correctly
+ * same for v with v_scale; with scale_per_block = 1 the scale is that of the
+ * page the slot lies in, k_scale[(s / bs) * Hkv + h] (set before the block's
+ * first token).  The division is a float32 division (correctly
  * rounded), the code the nearest E4M3 value (ties to even), magnitudes
  * beyond 448 saturate to 448 and NaN stays NaN.
  *   k, v: device [num_tokens, Hkv, head_dim] in in_dtype (PKV_F16 or PKV_BF16),
  *       16-byte aligned; head_dim a multiple of 16.
- *   k_scale, v_scale: device float32 [num_kv_heads].
+ *   k_scale, v_scale: device float32 [num_kv_heads] or, with
+ *       scale_per_block = 1, [num_blocks][num_kv_heads].
  *   k_cache, v_cache: device E4M3 codes, 16-byte aligned.
  * Slots as pkv_kv_cache_append (negative skipped, past the pool flagged
  * PKV_DEV_BAD_SLOT).  Returns PKV_OK, PKV_EINVAL or PKV_ECUDA.
  */
 PKV_API int pkv_kv_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, const void* v,
                                      const float* k_scale, const float* v_scale,
-                                     const int64_t* slot_mapping, int num_tokens,
+                                     int scale_per_block, const int64_t* slot_mapping,
+                                     int num_tokens,
                                      int num_kv_heads, int head_dim, int block_size,
                                      int num_blocks, pkv_dtype in_dtype, pkv_stream_t stream);
 

@@ -65,7 +65,8 @@ def lib():
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int64, ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int]
+                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64,
+                ctypes.c_int]
             L.pkvo_max_threads.restype = ctypes.c_int
             _lib = L
     return _lib
@@ -91,7 +92,7 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, *, scale: floa
     """float64 paged decode attention (window > 0: over each sequence's last
     `window` tokens only).  dtype is q's storage type; kv_dtype the caches'
     (default: the same; "e4m3" for FP8 codes, with float32 k_scale / v_scale
-    per KV head).
+    per KV head [Hkv], or per page [N, Hkv]).
 
     q [B, Hq, D]; k_cache, v_cache [N, Hkv, bs, D] in the storage dtype
     (bf16 as uint16 bits); block_tables int32 [B, max_blocks];
@@ -117,12 +118,22 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, *, scale: floa
     kvd = DTYPE_CODE[kv_dtype or dtype]
     ks = None if k_scale is None else np.ascontiguousarray(k_scale, dtype=np.float32)
     vs = None if v_scale is None else np.ascontiguousarray(v_scale, dtype=np.float32)
+    per_block = 0
+    for sc in (ks, vs):
+        if sc is not None:
+            if sc.shape == (N, Hkv):
+                per_block = 1
+            elif sc.shape != (Hkv,):
+                raise ValueError("scales must be [Hkv] or [num_blocks, Hkv]")
+    if ks is not None and vs is not None and ks.shape != vs.shape:
+        raise ValueError("k_scale and v_scale must have the same shape")
     rc = lib().pkvo_paged_decode(out.ctypes.data, q.ctypes.data, k_cache.ctypes.data,
                                  v_cache.ctypes.data, bt.ctypes.data, cl.ctypes.data,
                                  B, Hq, Hkv, D, bs, bt.shape[1], N, float(scale),
                                  int(window), DTYPE_CODE[dtype], kvd,
                                  None if ks is None else ks.ctypes.data,
-                                 None if vs is None else vs.ctypes.data, rp, nr, int(threads))
+                                 None if vs is None else vs.ctypes.data, per_block, rp, nr,
+                                 int(threads))
     if rc != 0:
         raise ValueError(f"oracle rejected the inputs (code {rc})")
     return out

@@ -89,9 +89,18 @@ def kv_cache_append_e4m3(k_cache: np.ndarray, v_cache: np.ndarray, k: np.ndarray
                          slot_mapping: np.ndarray, k_scale: np.ndarray, v_scale: np.ndarray,
                          in_dtype: str) -> None:
     """Append with quantisation: k_cache/v_cache uint8 codes [N, Hkv, bs, D];
-    k/v [T, Hkv, D] in in_dtype; scales float32 [Hkv]."""
+    k/v [T, Hkv, D] in in_dtype; scales float32 [Hkv] (per KV head) or
+    [N, Hkv] (per page: the scale of the block the slot lies in)."""
     ks = np.asarray(k_scale, dtype=np.float32)
     vs = np.asarray(v_scale, dtype=np.float32)
-    kq = e4m3_encode(to_f32(k, in_dtype) / ks[None, :, None])
-    vq = e4m3_encode(to_f32(v, in_dtype) / vs[None, :, None])
-    kv_cache_append(k_cache, v_cache, kq, vq, slot_mapping)
+    bs = k_cache.shape[2]
+    slots = np.asarray(slot_mapping, dtype=np.int64)
+    if ks.ndim == 1:
+        ksel = np.broadcast_to(ks, (len(slots), ks.size))
+        vsel = np.broadcast_to(vs, (len(slots), vs.size))
+    else:  # per page; padding slots (< 0) are never written, any row will do
+        blk = np.where(slots >= 0, slots // bs, 0)
+        ksel, vsel = ks[blk], vs[blk]
+    kq = e4m3_encode(to_f32(k, in_dtype) / ksel[:, :, None])
+    vq = e4m3_encode(to_f32(v, in_dtype) / vsel[:, :, None])
+    kv_cache_append(k_cache, v_cache, kq, vq, slots)

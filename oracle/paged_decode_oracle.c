@@ -22,9 +22,10 @@
  *     s_t = scale * sum_d q[b,h,d] k_t[d]
  *     out[b,h,:] = sum_t exp(s_t - max s) v_t / sum_t exp(s_t - max s)
  * in float64, plain loops, no blocking and no online rescaling.  L = 0 gives a
- * zero row.  Quantised caches (FP8 E4M3 codes) hold code * scale, one scale
- * per KV head for K and one for V (paging combines with quantisation:
- * "pagedattention vllm" §Comparison with Alternatives).
+ * zero row.  Quantised caches (FP8 E4M3 codes) hold code * scale, with one
+ * scale per KV head for K and one for V, or one per (physical block, KV head)
+ * page (paging combines with quantisation: "pagedattention vllm"
+ * §Comparison with Alternatives).
  * lo = 0, or with a sliding window of W tokens lo = max(0, L - W):
  * only the last W tokens are attended to ("pagedattention vllm" §Advanced
  * Features: sliding-window models keep only recent blocks).  The inputs are decoded bit by bit from their storage type
@@ -136,15 +137,13 @@ static int decode_row(double* out_row, const void* q, const void* k_cache,
                       int num_kv_heads, int head_dim, int block_size,
                       int max_blocks_per_seq, int64_t num_blocks, double scale,
                       int window, int dtype, int kv_dtype, const float* k_scale,
-                      const float* v_scale, double* s /* scratch, >= L + head_dim */) {
+                      const float* v_scale, int scale_per_block,
+                      double* s /* scratch, >= L + head_dim */) {
     const int G = num_q_heads / num_kv_heads;
     const int g = h / G;
     const int L = context_lens[b];
     const int lo = (window > 0 && L > window) ? L - window : 0;
     const int D = head_dim;
-    /* quantised pages: value = code * scale of the KV head */
-    const double ks = k_scale ? (double)k_scale[g] : 1.0;
-    const double vs = v_scale ? (double)v_scale[g] : 1.0;
     for (int d = 0; d < D; ++d) out_row[d] = 0.0;
     if (L <= 0) return 0;
 
@@ -158,6 +157,9 @@ static int decode_row(double* out_row, const void* q, const void* k_cache,
         int32_t phys = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
         if (phys < 0 || phys >= num_blocks) return -1;
         int64_t k_off = (((int64_t)phys * num_kv_heads + g) * block_size + t % block_size) * D;
+        /* quantised pages: value = code * scale of the KV head (or of the page) */
+        const int64_t si = scale_per_block ? (int64_t)phys * num_kv_heads + g : g;
+        const double ks = k_scale ? (double)k_scale[si] : 1.0;
         double acc = 0.0;
         for (int d = 0; d < D; ++d)
             acc += qrow[d] * (load_elem(k_cache, k_off + d, kv_dtype) * ks);
@@ -172,6 +174,8 @@ static int decode_row(double* out_row, const void* q, const void* k_cache,
         denom += w;
         int32_t phys = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
         int64_t v_off = (((int64_t)phys * num_kv_heads + g) * block_size + t % block_size) * D;
+        const int64_t si = scale_per_block ? (int64_t)phys * num_kv_heads + g : g;
+        const double vs = v_scale ? (double)v_scale[si] : 1.0;
         for (int d = 0; d < D; ++d)
             out_row[d] += w * (load_elem(v_cache, v_off + d, kv_dtype) * vs);
     }
@@ -190,8 +194,8 @@ int pkvo_paged_decode(double* out, const void* q, const void* k_cache,
                       int num_kv_heads, int head_dim, int block_size,
                       int max_blocks_per_seq, int64_t num_blocks, double scale,
                       int window, int dtype, int kv_dtype, const float* k_scale,
-                      const float* v_scale, const int32_t* rows, int64_t num_rows,
-                      int num_threads) {
+                      const float* v_scale, int scale_per_block, const int32_t* rows,
+                      int64_t num_rows, int num_threads) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         block_size <= 0 || num_q_heads % num_kv_heads != 0)
         return -2;
@@ -224,7 +228,7 @@ int pkvo_paged_decode(double* out, const void* q, const void* k_cache,
             if (decode_row(out + i * head_dim, q, k_cache, v_cache, block_tables,
                            context_lens, b, h, num_q_heads, num_kv_heads, head_dim,
                            block_size, max_blocks_per_seq, num_blocks, scale, window, dtype,
-                           kv_dtype, k_scale, v_scale, s))
+                           kv_dtype, k_scale, v_scale, scale_per_block, s))
                 err |= 1;
         }
         free(s);

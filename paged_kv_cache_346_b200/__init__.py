@@ -134,7 +134,8 @@ def pkv_paged_attention_decode_e4m3(out: torch.Tensor, q: torch.Tensor, k_cache:
                                     stream=None) -> torch.Tensor:
     """Paged decode over FP8 E4M3 pages (pkv_paged_attention_decode_e4m3 in
     pagedkv.h): k_cache/v_cache torch.float8_e4m3fn [N, Hkv, block_size, D];
-    k_scale/v_scale float32 [Hkv]; q and out fp16 or bf16."""
+    k_scale/v_scale float32 [Hkv], or [N, Hkv] for a scale per page; q and
+    out fp16 or bf16."""
     for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
                  (k_scale, "k_scale"), (v_scale, "v_scale"), (block_tables, "block_tables"),
                  (context_lens, "context_lens")):
@@ -153,15 +154,17 @@ def pkv_paged_attention_decode_e4m3(out: torch.Tensor, q: torch.Tensor, k_cache:
     N, Hkv, bs, D2 = k_cache.shape
     if (D2 != D or bs != block_size or tuple(out.shape) != (B, Hq, D) or
             tuple(v_cache.shape) != tuple(k_cache.shape) or block_tables.shape[0] != B or
-            context_lens.shape[0] != B or k_scale.numel() != Hkv or v_scale.numel() != Hkv):
+            context_lens.shape[0] != B or tuple(k_scale.shape) != tuple(v_scale.shape) or
+            tuple(k_scale.shape) not in ((Hkv,), (N, Hkv))):
         raise PagedKVError(_b.PKV_EINVAL, "shape mismatch")
+    per_block = 1 if k_scale.dim() == 2 else 0
     ws_bytes = 0
     if workspace is not None:
         _dev(workspace, "workspace")
         ws_bytes = workspace.numel() * workspace.element_size()
     check(lib.pkv_paged_attention_decode_e4m3(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
-        _ptr(block_tables), _ptr(context_lens), _ptr(seq_order), B, Hq, Hkv, D, bs,
+        per_block, _ptr(block_tables), _ptr(context_lens), _ptr(seq_order), B, Hq, Hkv, D, bs,
         block_tables.shape[1], N, int(max_context_len), float(scale), int(sliding_window),
         torch_dtype_code(q.dtype), int(partition_size), _ptr(workspace), ws_bytes, int(kernel),
         _stream(stream)),
@@ -234,7 +237,8 @@ def pkv_kv_cache_append_e4m3(k_cache: torch.Tensor, v_cache: torch.Tensor, k: to
                              v: torch.Tensor, k_scale: torch.Tensor, v_scale: torch.Tensor,
                              slot_mapping: torch.Tensor, *, stream=None) -> None:
     """fp16/bf16 k/v [T, Hkv, D] -> E4M3 codes of k / k_scale[h] (and v) in
-    the float8_e4m3fn caches' slots."""
+    the float8_e4m3fn caches' slots; k_scale/v_scale [Hkv], or [N, Hkv] for
+    the scale of the page each slot lies in."""
     for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache"), (k, "k"), (v, "v"),
                  (k_scale, "k_scale"), (v_scale, "v_scale"), (slot_mapping, "slot_mapping")):
         _dev(t, n)
@@ -248,10 +252,12 @@ def pkv_kv_cache_append_e4m3(k_cache: torch.Tensor, v_cache: torch.Tensor, k: to
     T = k.shape[0]
     if (tuple(k.shape) != (T, Hkv, D) or tuple(v.shape) != (T, Hkv, D) or
             slot_mapping.shape[0] != T or tuple(v_cache.shape) != tuple(k_cache.shape) or
-            k_scale.numel() != Hkv or v_scale.numel() != Hkv):
+            tuple(k_scale.shape) != tuple(v_scale.shape) or
+            tuple(k_scale.shape) not in ((Hkv,), (N, Hkv))):
         raise PagedKVError(_b.PKV_EINVAL, "shape mismatch")
     check(lib.pkv_kv_cache_append_e4m3(_ptr(k_cache), _ptr(v_cache), _ptr(k), _ptr(v),
-                                       _ptr(k_scale), _ptr(v_scale), _ptr(slot_mapping), T,
+                                       _ptr(k_scale), _ptr(v_scale),
+                                       1 if k_scale.dim() == 2 else 0, _ptr(slot_mapping), T,
                                        Hkv, D, bs, N, torch_dtype_code(k.dtype), _stream(stream)),
           "pkv_kv_cache_append_e4m3")
 

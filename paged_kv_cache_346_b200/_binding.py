@@ -42,14 +42,15 @@ SIGNATURES = {
     "pkv_paged_attention_decode_static_ws": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                                     _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                                                     _f32, _i32, _i32, _i32, _i32, _vp]),
-    "pkv_paged_attention_decode_e4m3": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
-                                               _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
-                                               _f32, _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
+    "pkv_paged_attention_decode_e4m3": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
+                                               _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                               _i32, _f32, _i32, _i32, _i32, _vp, _sz, _i32,
+                                               _vp]),
     "pkv_decode_schedule_order": (_i32, [_vp, _i32, _vp]),
     "pkv_kv_cache_append": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                    _vp]),
-    "pkv_kv_cache_append_e4m3": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
-                                        _i32, _i32, _i32, _vp]),
+    "pkv_kv_cache_append_e4m3": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32,
+                                        _i32, _i32, _i32, _i32, _vp]),
     "pkv_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_swap_blocks": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                _i32, _vp]),

@@ -96,7 +96,7 @@ constexpr int kNumSMs = 148;
 // The decode behind both entry points.  e4m3: the pages hold E4M3 codes with
 // per-KV-head scales and dtype is the type of q and out.
 int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
-                const float* k_scale, const float* v_scale, bool e4m3,
+                const float* k_scale, const float* v_scale, int scale_per_block, bool e4m3,
                 const int32_t* block_tables, const int32_t* context_lens,
                 const int32_t* seq_order, int num_seqs, int num_q_heads, int num_kv_heads,
                 int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
@@ -120,7 +120,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     if (e4m3 && head_dim == 64) return PKV_EUNSUPPORTED;
     if (num_seqs == 0) return PKV_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_EINVAL;
-    if (e4m3 && (!k_scale || !v_scale)) return PKV_EINVAL;
+    if (e4m3 && (!k_scale || !v_scale || (scale_per_block != 0 && scale_per_block != 1)))
+        return PKV_EINVAL;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
         return PKV_EINVAL;
 
@@ -170,6 +171,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     a.seq_order = seq_order;
     a.k_scale = e4m3 ? k_scale : nullptr;
     a.v_scale = e4m3 ? v_scale : nullptr;
+    a.scale_per_block = e4m3 ? scale_per_block : 0;
     a.ws_o = static_cast<float*>(workspace);
     a.ws_ml = np > 1 ? a.ws_o + (int64_t)num_seqs * num_q_heads * np * head_dim : nullptr;
     a.num_seqs = num_seqs;
@@ -274,7 +276,7 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
                                int partition_size, void* workspace, size_t workspace_bytes,
                                pkv_kernel kernel, pkv_stream_t stream) {
     NvtxRange range("pkv_paged_attention_decode");
-    return pkv::decode_impl(out, q, k_cache, v_cache, nullptr, nullptr, false, block_tables,
+    return pkv::decode_impl(out, q, k_cache, v_cache, nullptr, nullptr, 0, false, block_tables,
                             context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
                             head_dim, block_size, max_blocks_per_seq, num_blocks,
                             max_context_len, scale, sliding_window, dtype, partition_size,
@@ -283,7 +285,8 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
 
 int pkv_paged_attention_decode_e4m3(void* out, const void* q, const void* k_cache,
                                     const void* v_cache, const float* k_scale,
-                                    const float* v_scale, const int32_t* block_tables,
+                                    const float* v_scale, int scale_per_block,
+                                    const int32_t* block_tables,
                                     const int32_t* context_lens, const int32_t* seq_order,
                                     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                     int block_size, int max_blocks_per_seq, int num_blocks,
@@ -292,7 +295,8 @@ int pkv_paged_attention_decode_e4m3(void* out, const void* q, const void* k_cach
                                     size_t workspace_bytes, pkv_kernel kernel,
                                     pkv_stream_t stream) {
     NvtxRange range("pkv_paged_attention_decode_e4m3");
-    return pkv::decode_impl(out, q, k_cache, v_cache, k_scale, v_scale, true, block_tables,
+    return pkv::decode_impl(out, q, k_cache, v_cache, k_scale, v_scale, scale_per_block, true,
+                            block_tables,
                             context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
                             head_dim, block_size, max_blocks_per_seq, num_blocks,
                             max_context_len, scale, sliding_window, dtype, partition_size,
@@ -321,13 +325,14 @@ int pkv_kv_cache_append(void* k_cache, void* v_cache, const void* k, const void*
 }
 
 int pkv_kv_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, const void* v,
-                             const float* k_scale, const float* v_scale,
+                             const float* k_scale, const float* v_scale, int scale_per_block,
                              const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
                              int head_dim, int block_size, int num_blocks, pkv_dtype in_dtype,
                              pkv_stream_t stream) {
     NvtxRange range("pkv_kv_cache_append_e4m3");
     if ((in_dtype != PKV_F16 && in_dtype != PKV_BF16) || num_tokens < 0 || num_kv_heads <= 0 ||
-        head_dim <= 0 || head_dim % 16 != 0 || block_size <= 0 || num_blocks <= 0)
+        head_dim <= 0 || head_dim % 16 != 0 || block_size <= 0 || num_blocks <= 0 ||
+        (scale_per_block != 0 && scale_per_block != 1))
         return PKV_EINVAL;
     if (num_tokens == 0) return PKV_OK;
     if (!k_cache || !v_cache || !k || !v || !slot_mapping || !k_scale || !v_scale)
@@ -338,7 +343,8 @@ int pkv_kv_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, const 
     if (status_word(&st) != cudaSuccess) return PKV_ECUDA;
     cudaError_t e = launch_kv_append_e4m3(k_cache, v_cache, k, v, k_scale, v_scale, slot_mapping,
                                           num_tokens, num_kv_heads, head_dim, block_size,
-                                          num_blocks, in_dtype == PKV_BF16, st,
+                                          num_blocks, in_dtype == PKV_BF16, scale_per_block != 0,
+                                          st,
                                           reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }

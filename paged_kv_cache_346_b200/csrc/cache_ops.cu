@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(256) kv_append_e4m3_kernel(
     uint4* __restrict__ kc, uint4* __restrict__ vc, const uint4* __restrict__ k,
     const uint4* __restrict__ v, const float* __restrict__ ks, const float* __restrict__ vs,
     const int64_t* __restrict__ slots, int64_t total_vecs, int row_vecs, int head_vecs,
-    int num_kv_heads, int block_size, int64_t num_slots, unsigned int* status) {
+    int num_kv_heads, int block_size, int64_t num_slots, int per_block, unsigned int* status) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total_vecs; i += stride) {
         const int64_t t = i / row_vecs;
@@ -88,8 +88,9 @@ __global__ void __launch_bounds__(256) kv_append_e4m3_kernel(
         const int64_t blk = s / block_size;
         const int off = (int)(s - blk * block_size);
         const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_vecs + c;
-        kc[dst] = quantise16<Tin>(k + 2 * i, ks[h]);
-        vc[dst] = quantise16<Tin>(v + 2 * i, vs[h]);
+        const int64_t si = per_block ? blk * num_kv_heads + h : h;
+        kc[dst] = quantise16<Tin>(k + 2 * i, ks[si]);
+        vc[dst] = quantise16<Tin>(v + 2 * i, vs[si]);
     }
 }
 
@@ -191,7 +192,7 @@ cudaError_t launch_kv_append_e4m3(void* k_cache, void* v_cache, const void* k, c
                                   const float* k_scale, const float* v_scale,
                                   const int64_t* slots, int num_tokens, int num_kv_heads,
                                   int head_dim, int block_size, int num_blocks, bool bf16_in,
-                                  unsigned int* status, cudaStream_t stream) {
+                                  bool per_block, unsigned int* status, cudaStream_t stream) {
     const int head_vecs = head_dim / 16;
     const int row_vecs = head_vecs * num_kv_heads;
     const int64_t total = (int64_t)num_tokens * row_vecs;
@@ -203,7 +204,7 @@ cudaError_t launch_kv_append_e4m3(void* k_cache, void* v_cache, const void* k, c
         static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
         static_cast<const uint4*>(k), static_cast<const uint4*>(v), k_scale, v_scale, slots,
         total, row_vecs, head_vecs, num_kv_heads, block_size, (int64_t)num_blocks * block_size,
-        status);
+        per_block ? 1 : 0, status);
     return cudaGetLastError();
 }
 

@@ -16,7 +16,7 @@ cudaError_t launch_kv_append_e4m3(void* k_cache, void* v_cache, const void* k, c
                                   const float* k_scale, const float* v_scale,
                                   const int64_t* slots, int num_tokens, int num_kv_heads,
                                   int head_dim, int block_size, int num_blocks, bool bf16_in,
-                                  unsigned int* status, cudaStream_t stream);
+                                  bool per_block, unsigned int* status, cudaStream_t stream);
 
 // block_bytes = num_kv_heads * block_size * head_dim * element size.
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs,

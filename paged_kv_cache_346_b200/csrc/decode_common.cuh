@@ -18,8 +18,8 @@ struct DecodeArgs {
     const int32_t* block_tables;  // [B, max_blocks_per_seq]
     const int32_t* context_lens;  // [B]
     const int32_t* seq_order;     // [B] schedule order (CTA z takes sequence seq_order[z]), or null
-    const float* k_scale;         // [Hkv] scales of E4M3 K / V pages, or null
-    const float* v_scale;
+    const float* k_scale;         // scales of E4M3 K / V pages, or null: [Hkv], or
+    const float* v_scale;         // [num_blocks, Hkv] when scale_per_block
     float* ws_o;                  // [B, Hq, max_partitions, D] partition outputs
     float* ws_ml;                 // [B, Hq, max_partitions, 2] (m in log2 units, l)
     unsigned int* status;
@@ -35,6 +35,7 @@ struct DecodeArgs {
     int max_partitions;           // grid.x = ceil(longest attended span / partition_size)
     int block_size;
     int window;                   // sliding window in tokens, 0 = attend to the whole context
+    int scale_per_block;          // E4M3 scales per (block, KV head) page
     float scale_log2;             // scale * log2(e): logits are kept in base 2
 };
 

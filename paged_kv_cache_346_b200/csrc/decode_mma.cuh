@@ -23,6 +23,8 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "decode_common.cuh"
 
 namespace pkv {
@@ -302,7 +304,11 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                     const int tok = nt * 8 + 2 * t4 + (i & 1);
                     s[nt][i] = (tok >= wlo && tok < wvalid) ? s[nt][i] * a.scale_log2 : -INFINITY;
                 }
-            uint32_t pb[RB][2];
+            // P enters the MMA in T.  bf16 keeps 8 significant bits, too few
+            // for the weights: P = hi + lo, two bf16 terms (~16 bits), and
+            // two P.V products.  fp16's 11 bits are kept as one term.
+            constexpr bool SPLIT = std::is_same<T, __nv_bfloat16>::value;
+            uint32_t pb[RB][2], pl[RB][2];
             float alpha_c[RB][2];
 #pragma unroll
             for (int rb = 0; rb < RB; ++rb) {
@@ -318,6 +324,12 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                     p[nt][0] = exp2f(s[nt][i0] - mnew);
                     p[nt][1] = exp2f(s[nt][i0 + 1] - mnew);
                     pb[rb][nt] = M::pack(p[nt][0], p[nt][1], pr[nt][0], pr[nt][1]);
+                    if constexpr (SPLIT) {
+                        float r0, r1;
+                        pl[rb][nt] = M::pack(p[nt][0] - pr[nt][0], p[nt][1] - pr[nt][1], r0, r1);
+                        pr[nt][0] += r0;  // the weights P.V uses, hi + lo
+                        pr[nt][1] += r1;
+                    }
                 }
                 float ps = (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
                 ps += __shfl_xor_sync(0xffffffffu, ps, 1);
@@ -357,6 +369,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                     o[mt][rb][2] *= alpha_c[rb][0];
                     o[mt][rb][3] *= alpha_c[rb][1];
                     M::run(o[mt][rb], va, pb[rb][0], pb[rb][1]);
+                    if constexpr (SPLIT) M::run(o[mt][rb], va, pl[rb][0], pl[rb][1]);
                 }
             }
         };

@@ -26,7 +26,11 @@
 // q (fp16 or bf16) enters the fp16 MMA multiplied by a power of two 2^e that
 // puts its largest magnitude in [2^14, 2^15) (exact for every value that stays
 // an f16 normal); the logits are multiplied back by scale * log2(e) *
-// k_scale * 2^-e in fp32, and the output by v_scale.
+// k_scale * 2^-e in fp32, and the output by v_scale.  With a scale per page,
+// a warp's 16-token slice lies in one block: its logits take that page's
+// k_scale, and its P.V product (a fresh fp32 accumulator) is added to the
+// output multiplied by that page's v_scale, so P stays an fp16 value at most
+// 256 whatever the scales.
 #pragma once
 
 #include "decode_mma.cuh"
@@ -83,7 +87,9 @@ __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) {
     return r;
 }
 
-template <typename T, int D, int BS, int NH, int NW, int STAGES_>
+// PPB: a scale per page (a.scale_per_block), a compile-time choice so the
+// per-head path carries no per-slice scale code.
+template <typename T, int D, int BS, int NH, int NW, int STAGES_, bool PPB>
 __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     decode_mma_e4m3_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv) {
@@ -206,7 +212,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         e = max(-126, min(126, e));
         const float up = __int_as_float((127 + e) << 23);
         const float down = __int_as_float((127 - e) << 23);
-        qmul = a.scale_log2 * a.k_scale[kvh] * down;
+        qmul = a.scale_log2 * (PPB ? 1.f : a.k_scale[kvh]) * down;
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks)
 #pragma unroll
@@ -239,6 +245,9 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     const int lchunk = lane >> 4;
     const int swz = lrow & 7;
 
+    // the output's V scale: the KV head's (per-page scales enter slice by slice)
+    const float vs_out = PPB ? 1.f : a.v_scale[kvh];
+
     for (int it = 0; it < nslices; ++it) {
         const int stage = it % STAGES;
         const bool ok = __all_sync(0xffffffffu, mbar_wait(full + warp * STAGES + stage,
@@ -257,6 +266,14 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         const int wlo = mask_lo - (it * TILE + warp * 16);
         const bool work = wlo < 16 && wlo < wvalid;
         const uint32_t kbase = ring_s + (uint32_t)(stage * 2 * SLICE_BYTES + lrow * 128);
+        // this slice's page scales (per-page mode): logits and P.V multipliers
+        float kmul = qmul, vmul = 1.f;
+        if (PPB && work) {
+            const int64_t si =
+                (int64_t)s_tab[(it * TILE + warp * 16) / BS] * a.num_kv_heads + kvh;
+            kmul = qmul * a.k_scale[si];
+            vmul = a.v_scale[si];
+        }
         auto addr = [&](int kp) {  // chunk pair kp: chunks 2 kp, 2 kp + 1
             const int chunk = 2 * kp + lchunk;
             return kbase + (chunk >> 3) * BOX_BYTES + (((chunk & 7) ^ swz) << 4);
@@ -302,7 +319,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) s[nt][i] = (s[nt][i] + s2[nt][i]) * qmul;
+                for (int i = 0; i < 4; ++i) s[nt][i] = (s[nt][i] + s2[nt][i]) * kmul;
             if (partial) {
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
@@ -387,7 +404,14 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                             o[mt][rb][2] *= alpha_c[rb][0];
                             o[mt][rb][3] *= alpha_c[rb][1];
                         }
-                        mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
+                        if constexpr (PPB) {  // this page's P.V, then times its v_scale
+                            float d4[4] = {0.f, 0.f, 0.f, 0.f};
+                            mma_f16(d4, va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) o[mt][rb][i] = fmaf(d4[i], vmul, o[mt][rb][i]);
+                        } else {
+                            mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
+                        }
                     }
                 }
             }
@@ -407,7 +431,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     float* red = reinterpret_cast<float*>(s_kv);
     float* red_m = red + NW * NH * A::RP;
     float* red_l = red_m + NW * NH;
-    const float vs = a.v_scale[kvh];
+    const float vs = vs_out;
 #pragma unroll
     for (int mt = 0; mt < KSTEPS; ++mt)
 #pragma unroll
@@ -437,9 +461,10 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
 template <typename T, int D, int BS, int NH, int NW = 4, int STAGES = 0>
 cudaError_t launch_decode_mma_e4m3(const DecodeArgs& a, cudaStream_t stream) {
     using C = MmaE4m3Cfg<D, BS, NW, STAGES>;
-    static SmemAttr attr;
-    auto kern = decode_mma_e4m3_kernel<T, D, BS, NH, NW, STAGES>;
-    cudaError_t e = attr.ensure(kern, C::smem_bytes(8192));
+    static SmemAttr attr[2];  // one per kernel variant
+    auto kern = a.scale_per_block ? decode_mma_e4m3_kernel<T, D, BS, NH, NW, STAGES, true>
+                                  : decode_mma_e4m3_kernel<T, D, BS, NH, NW, STAGES, false>;
+    cudaError_t e = attr[a.scale_per_block ? 1 : 0].ensure(kern, C::smem_bytes(8192));
     if (e != cudaSuccess) return e;
     const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
     CUtensorMap tk, tv;

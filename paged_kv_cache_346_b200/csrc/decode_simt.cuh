@@ -29,6 +29,8 @@
 //      workspace for the log-sum-exp reduce.
 #pragma once
 
+#include <type_traits>
+
 #include "decode_common.cuh"
 
 namespace pkv {
@@ -164,8 +166,12 @@ struct SimtWarp {
 
     // The fetched 16 tokens; tokens [wlo, wvalid) of them are attended to
     // (before wlo: ahead of a sliding window; from wvalid: past the end).
-    // s_p: this warp's [HG][16] weight scratch.
-    __device__ __forceinline__ void compute(int wlo, int wvalid, float (*s_p)[16]) {
+    // s_p: this warp's [HG][16] weight scratch.  E4M3 pages with a scale per
+    // page: kts multiplies the logits and vts the weights of the V sum (the
+    // row sum l keeps the plain weights).
+    __device__ __forceinline__ void compute(int wlo, int wvalid, float (*s_p)[16],
+                                            float kts = 1.f, float vts = 1.f) {
+        constexpr bool Q8 = std::is_same<TC, E4M3>::value;
         float s[HG][4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -187,7 +193,7 @@ struct SimtWarp {
                 d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 1);
                 d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 2);
                 d[hh] += __shfl_xor_sync(0xffffffffu, d[hh], 4);
-                s[hh][r] = (tok >= wlo && tok < wvalid) ? d[hh] : -INFINITY;
+                s[hh][r] = (tok >= wlo && tok < wvalid) ? (Q8 ? d[hh] * kts : d[hh]) : -INFINITY;
             }
         }
 #pragma unroll
@@ -213,7 +219,7 @@ struct SimtWarp {
                 for (int e = 0; e < EPC; ++e) acc[hh][c][e] *= alpha;
             if (sub == 0) {
 #pragma unroll
-                for (int r = 0; r < 4; ++r) s_p[hh][r * 4 + grp] = s[hh][r];
+                for (int r = 0; r < 4; ++r) s_p[hh][r * 4 + grp] = Q8 ? s[hh][r] * vts : s[hh][r];
             }
         }
         __syncwarp();
@@ -395,7 +401,8 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::TH
     // 3.-5. consumer warps
     SimtWarp<T, D, HG, C, TC> W;
     W.init(reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D, nh,
-           a.k_scale ? a.scale_log2 * a.k_scale[kvh] : a.scale_log2, lane);
+           a.k_scale && !a.scale_per_block ? a.scale_log2 * a.k_scale[kvh] : a.scale_log2,
+           lane);
     const uint64_t pol = WS ? 0 : policy_evict_first();
     int it_stop = ntiles;  // the tile a timed-out wait stopped at
     for (int it = 0; it < ntiles; ++it) {
@@ -409,7 +416,14 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::TH
             const unsigned char* Kw = s_kv + stage * 2 * STAGE_BYTES + warp * 16 * ROW;
             W.fetch(Kw, Kw + STAGE_BYTES);
         }
-        if (!W.EARLY && !s_abort && work) W.compute(wlo, wvalid, s_p[warp]);
+        float kts = 1.f, vts = 1.f;  // page scales of this warp's tokens (per-page mode)
+        if (a.scale_per_block && work) {
+            const int64_t si =
+                (int64_t)s_tab[(it * TILE + warp * 16) / BS] * a.num_kv_heads + kvh;
+            kts = a.k_scale[si];
+            vts = a.v_scale[si];
+        }
+        if (!W.EARLY && !s_abort && work) W.compute(wlo, wvalid, s_p[warp], kts, vts);
         // the stage's data is in registers (or used): hand the stage back
         if (WS) {
             __syncwarp();
@@ -422,7 +436,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::TH
             }
             if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage, pol);
         }
-        if (W.EARLY && work) W.compute(wlo, wvalid, s_p[warp]);
+        if (W.EARLY && work) W.compute(wlo, wvalid, s_p[warp], kts, vts);
     }
     if (WS) __syncthreads();  // producer and consumers: every stage consumed
     if (s_abort) {
@@ -435,7 +449,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::TH
     if (!WS) pdl_launch_dependents();
 
     // 6. merge the warps
-    W.template park<NW>(warp, red, a.v_scale ? a.v_scale[kvh] : 1.f);
+    W.template park<NW>(warp, red, a.v_scale && !a.scale_per_block ? a.v_scale[kvh] : 1.f);
     __syncthreads();
     merge_warps_and_store<T, D, HG, NW>(a, red, b, h0, nh, part, np, tid, WS ? THREADS : NW * 32);
 }

@@ -56,6 +56,10 @@ def _decode(**over):
     (dict(win=-1), b.PKV_EINVAL),
     (dict(dt=7), b.PKV_EINVAL),
     (dict(kern=9), b.PKV_EINVAL),
+    (dict(spb=2, out=ctypes.c_void_p(1 << 20), q=ctypes.c_void_p(1 << 20),
+          k=ctypes.c_void_p(1 << 20), v=ctypes.c_void_p(1 << 20), ks=ctypes.c_void_p(1 << 20),
+          vs=ctypes.c_void_p(1 << 20), bt=ctypes.c_void_p(1 << 20),
+          cl=ctypes.c_void_p(1 << 20)), b.PKV_EINVAL),     # scale mode 0 or 1
     (dict(D=96), b.PKV_EUNSUPPORTED),
     (dict(bs=8, maxlen=50), b.PKV_EUNSUPPORTED),
     (dict(dt=b.PKV_F32, D=256), b.PKV_EUNSUPPORTED),
@@ -105,12 +109,13 @@ def test_append_and_copy_host_checks():
 
 
 def _decode_e4m3(**over):
-    a = dict(out=None, q=None, k=None, v=None, ks=None, vs=None, bt=None, cl=None, order=None,
-             B=4, Hq=8, Hkv=2, D=128, bs=16, mb=8, N=64, maxlen=100, scale=0.1, win=0,
+    a = dict(out=None, q=None, k=None, v=None, ks=None, vs=None, spb=0, bt=None, cl=None,
+             order=None, B=4, Hq=8, Hkv=2, D=128, bs=16, mb=8, N=64, maxlen=100, scale=0.1, win=0,
              dt=b.PKV_F16, P=0, ws=None, wsb=0, kern=0, stream=None)
     a.update(over)
     return b.lib.pkv_paged_attention_decode_e4m3(
-        a["out"], a["q"], a["k"], a["v"], a["ks"], a["vs"], a["bt"], a["cl"], a["order"], a["B"],
+        a["out"], a["q"], a["k"], a["v"], a["ks"], a["vs"], a["spb"], a["bt"], a["cl"], a["order"],
+        a["B"],
         a["Hq"], a["Hkv"], a["D"], a["bs"], a["mb"], a["N"], a["maxlen"], a["scale"], a["win"],
         a["dt"], a["P"], a["ws"], a["wsb"], a["kern"], a["stream"])
 
@@ -120,6 +125,10 @@ def _decode_e4m3(**over):
     (dict(dt=b.PKV_E4M3), b.PKV_EINVAL),
     (dict(D=64), b.PKV_EUNSUPPORTED),                   # 64-byte rows
     (dict(kern=9), b.PKV_EINVAL),
+    (dict(spb=2, out=ctypes.c_void_p(1 << 20), q=ctypes.c_void_p(1 << 20),
+          k=ctypes.c_void_p(1 << 20), v=ctypes.c_void_p(1 << 20), ks=ctypes.c_void_p(1 << 20),
+          vs=ctypes.c_void_p(1 << 20), bt=ctypes.c_void_p(1 << 20),
+          cl=ctypes.c_void_p(1 << 20)), b.PKV_EINVAL),     # scale mode 0 or 1
     (dict(Hq=6, Hkv=4), b.PKV_EINVAL),
     (dict(), b.PKV_EINVAL),                             # null pointers
     (dict(B=0), b.PKV_OK),
@@ -143,7 +152,7 @@ def test_e4m3_pages_need_their_own_entry():
 
 def test_append_e4m3_host_checks():
     f = b.lib.pkv_kv_cache_append_e4m3
-    args = [None] * 7
+    args = [None] * 6 + [0, None]   # pointers, scale_per_block = 0, slot_mapping
     assert f(*args, 0, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_OK
     assert f(*args, 3, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL   # null pointers
     assert f(*args, 0, 4, 120, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL   # head_dim % 16
@@ -168,3 +177,9 @@ def test_wait_timeout_selftest_host_checks():
     assert f(0, None) == b.PKV_EINVAL
     assert f(-5, None) == b.PKV_EINVAL
     assert f(5_000_000_000, None) == b.PKV_EINVAL
+
+
+def test_append_e4m3_scale_mode_checked():
+    f = b.lib.pkv_kv_cache_append_e4m3
+    assert f(*([None] * 6), 2, None, 0, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_EINVAL
+    assert f(*([None] * 6), 1, None, 0, 4, 128, 16, 10, b.PKV_F16, None) == b.PKV_OK

@@ -29,10 +29,15 @@ def _codes(a: np.ndarray) -> torch.Tensor:
 class E4M3Inputs:
     """Device copies of a decode batch whose pages are E4M3 codes."""
 
-    def __init__(self, inp, seed):
+    def __init__(self, inp, seed, per_page=False, v_scale_range=None):
         c = inp.cfg
         self.inp = inp
-        self.pages = make_e4m3_pages(inp, seed)
+        self.pages = make_e4m3_pages(inp, seed, per_page=per_page)
+        if v_scale_range is not None:  # widen the V scales (per-page tests)
+            g = np.random.default_rng(seed + 77)
+            lo, hi = v_scale_range
+            self.pages.v_scale = np.exp(g.uniform(np.log(lo), np.log(hi),
+                                                  size=self.pages.v_scale.shape)).astype(np.float32)
         self.q = to_device(inp.q, c.dtype)
         self.k = _codes(self.pages.k_cache)
         self.v = _codes(self.pages.v_cache)
@@ -282,3 +287,75 @@ def test_swap_e4m3_round_trip():
     torch.cuda.synchronize()
     assert np.array_equal(dK.view(torch.uint8).cpu().numpy()[20:30], K[:10])
     assert np.array_equal(dV.view(torch.uint8).cpu().numpy()[20:30], V[:10])
+
+
+# ---------------------------------------------------------------------------
+# a scale per page ([num_blocks, Hkv])
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_append_e4m3_per_page_bit_exact(dtype):
+    N, H, bs, D, T = 30, 4, 16, 128, 200
+    g = np.random.default_rng(55)
+    K = np.zeros((N, H, bs, D), np.uint8)
+    V = np.zeros_like(K)
+    k = normal_fill((T, H, D), dtype, 31)
+    v = normal_fill((T, H, D), dtype, 32)
+    ks = np.exp(g.uniform(np.log(1e-3), np.log(0.5), size=(N, H))).astype(np.float32)
+    vs = np.exp(g.uniform(np.log(1e-3), np.log(50.0), size=(N, H))).astype(np.float32)
+    slots = g.choice(N * bs, size=T, replace=False).astype(np.int64)
+    slots[g.random(T) < 0.1] = -1
+    dK, dV = _codes(K), _codes(V)
+    pkv.pkv_kv_cache_append_e4m3(dK, dV, to_device(k, dtype), to_device(v, dtype),
+                                 torch.from_numpy(ks).cuda(), torch.from_numpy(vs).cuda(),
+                                 torch.from_numpy(slots).cuda())
+    kv_cache_append_e4m3(K, V, k, v, slots, ks, vs, dtype)
+    torch.cuda.synchronize()
+    assert np.array_equal(dK.view(torch.uint8).cpu().numpy(), K)
+    assert np.array_equal(dV.view(torch.uint8).cpu().numpy(), V)
+
+
+@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("partition", [0, 64])
+def test_decode_e4m3_per_page_scales(G, partition):
+    """Per-page scales from the workload generator (uniform in [1/64, 1/16])."""
+    cfg = _cfg("bf16", 2 * G, 2, 128, 16, RAGGED)
+    inp = make_decode_inputs(cfg, seed=120 + G)
+    dev = E4M3Inputs(inp, seed=120 + G, per_page=True)
+    ref = dev.oracle()
+    for kern in KERNELS:
+        got = to_f64(dev.decode(partition_size=partition, kernel=kern, fill_out=6.0))
+        assert_close(got, ref, "bf16", f"per-page G={G} P={partition} kernel={kern}")
+
+
+@pytest.mark.parametrize("G", [1, 8])
+def test_decode_e4m3_per_page_scales_five_decades(G):
+    """V page scales spread over five decades (5e-3 .. 500), so outputs are
+    small weighted means of values up to ~2e5.  The CUDA-core kernel keeps
+    every weight in fp32 and meets the usual tolerance.  The tensor-core
+    kernel rounds each weight p to fp16 (relative error <= 2^-11) before the
+    P.V product, so an output carries absolute error up to
+    2^-11 * max|v| (sum of |dp| |v| over sum of p); its bound here is
+    2^-10 * max|v| + 1e-2 |ref|."""
+    cfg = _cfg("bf16", 2 * G, 2, 128, 16, RAGGED)
+    inp = make_decode_inputs(cfg, seed=140 + G)
+    dev = E4M3Inputs(inp, seed=140 + G, per_page=True, v_scale_range=(5e-3, 500.0))
+    ref = dev.oracle()
+    got = to_f64(dev.decode(kernel=pkv.PKV_KERNEL_SIMT, fill_out=6.0))
+    assert_close(got, ref, "bf16", f"per-page wide G={G} CUDA cores")
+    vd = torch.from_numpy(dev.pages.v_cache).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    vmax = float(np.max(np.abs(vd * dev.pages.v_scale[:, :, None, None])))
+    got = to_f64(dev.decode(kernel=pkv.PKV_KERNEL_MMA, fill_out=6.0))
+    err = np.abs(got - ref)
+    tol = 2.0 ** -10 * vmax + 1e-2 * np.abs(ref)
+    assert np.all(err <= tol), (float(err.max()), vmax)
+
+
+def test_decode_e4m3_per_page_window_and_bs32():
+    cfg = _cfg("f16", 8, 2, 128, 32, RAGGED)
+    inp = make_decode_inputs(cfg, seed=130)
+    dev = E4M3Inputs(inp, seed=130, per_page=True)
+    for W in (0, 40):
+        ref = dev.oracle(window=W)
+        for kern in KERNELS:
+            got = to_f64(dev.decode(partition_size=64, sliding_window=W, kernel=kern))
+            assert_close(got, ref, "f16", f"per-page bs32 W={W} kernel={kern}")

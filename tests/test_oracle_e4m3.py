@@ -160,3 +160,59 @@ def test_quantised_decode_power_of_two_scales_equal_f16_decode():
     assert torch.equal(v16.float(), vd * torch.from_numpy(vs)[None, :, None, None])
     want = oracle.paged_decode(q, k16.numpy(), v16.numpy(), bt, lens, scale=0.3, dtype="f16")
     np.testing.assert_array_equal(got, want)
+
+
+# ---------------------------------------------------------------------------
+# per-page scales ([num_blocks, Hkv])
+
+def test_per_page_scales_broadcast_equal_per_head():
+    q, kc, vc, bt, lens, ks, vs = _tiny_quantised_case(21)
+    N = kc.shape[0]
+    a = oracle.paged_decode(q, kc, vc, bt, lens, scale=0.2, dtype="f16", kv_dtype="e4m3",
+                            k_scale=ks, v_scale=vs)
+    b = oracle.paged_decode(q, kc, vc, bt, lens, scale=0.2, dtype="f16", kv_dtype="e4m3",
+                            k_scale=np.tile(ks, (N, 1)), v_scale=np.tile(vs, (N, 1)))
+    np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("window", [0, 4])
+def test_per_page_scales_vs_brute(window):
+    q, kc, vc, bt, lens, _, _ = _tiny_quantised_case(22)
+    N, Hkv = kc.shape[:2]
+    g = np.random.default_rng(5)
+    ks = g.uniform(0.001, 0.05, size=(N, Hkv)).astype(np.float32)
+    vs = g.uniform(0.01, 300.0, size=(N, Hkv)).astype(np.float32)
+    got = oracle.paged_decode(q, kc, vc, bt, lens, scale=0.3, dtype="f16", kv_dtype="e4m3",
+                              k_scale=ks, v_scale=vs, window=window)
+    kd = torch.from_numpy(kc).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    vd = torch.from_numpy(vc).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    kd = kd * ks.astype(np.float64)[:, :, None, None]
+    vd = vd * vs.astype(np.float64)[:, :, None, None]
+    want = np.array(brute.paged_decode(q.astype(np.float64), kd, vd, bt, lens, 0.3,
+                                       window=window))
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_append_per_page_scales():
+    rng = np.random.default_rng(9)
+    N, H, bs, D, T = 6, 2, 4, 16, 10
+    k = (rng.standard_normal((T, H, D))).astype(np.float16)
+    v = (rng.standard_normal((T, H, D))).astype(np.float16)
+    ks = rng.uniform(0.005, 0.02, size=(N, H)).astype(np.float32)
+    vs = rng.uniform(0.005, 0.02, size=(N, H)).astype(np.float32)
+    slots = rng.permutation(N * bs)[:T].astype(np.int64)
+    slots[1] = -1
+    kc = np.zeros((N, H, bs, D), np.uint8)
+    vc = np.zeros_like(kc)
+    kv_cache_append_e4m3(kc, vc, k, v, slots, ks, vs, "f16")
+    for t, s in enumerate(slots):
+        if s < 0:
+            continue
+        blk, off = divmod(int(s), bs)
+        for h in range(H):
+            want_k = torch.from_numpy(k[t, h].astype(np.float32) / ks[blk, h]) \
+                .to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            assert np.array_equal(kc[blk, h, off], want_k)
+            want_v = torch.from_numpy(v[t, h].astype(np.float32) / vs[blk, h]) \
+                .to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            assert np.array_equal(vc[blk, h, off], want_v)

@@ -315,6 +315,15 @@ def e4m3_scales(num_kv_heads: int, seed: int) -> tuple[np.ndarray, np.ndarray]:
     return ks, vs
 
 
+def e4m3_page_scales(num_blocks: int, num_kv_heads: int, seed: int):
+    """Per-page scales ([num_blocks, Hkv] for K and for V), uniform in
+    [1/64, 1/16] like the per-head ones."""
+    g = rng(seed * 1000 + 12)
+    ks = g.uniform(1 / 64, 1 / 16, size=(num_blocks, num_kv_heads)).astype(np.float32)
+    vs = g.uniform(1 / 64, 1 / 16, size=(num_blocks, num_kv_heads)).astype(np.float32)
+    return ks, vs
+
+
 @dataclass
 class QuantisedPages:
     k_cache: np.ndarray   # uint8 E4M3 codes [N, Hkv, bs, D]
@@ -323,13 +332,17 @@ class QuantisedPages:
     v_scale: np.ndarray
 
 
-def make_e4m3_pages(inp: "DecodeInputs", seed: int = 0, threads: int = 8) -> QuantisedPages:
+def make_e4m3_pages(inp: "DecodeInputs", seed: int = 0, threads: int = 8,
+                    per_page: bool = False) -> QuantisedPages:
     """E4M3 pages of the same shape as inp's caches (same tables and lengths;
-    inp.q stays the query)."""
+    inp.q stays the query), with per-head scales, or per-page ones."""
     shape = inp.k_cache.shape
     k = e4m3_codes(shape, seed * 1000 + 14, threads)
     v = e4m3_codes(shape, seed * 1000 + 15, threads)
-    ks, vs = e4m3_scales(shape[1], seed)
+    if per_page:
+        ks, vs = e4m3_page_scales(shape[0], shape[1], seed)
+    else:
+        ks, vs = e4m3_scales(shape[1], seed)
     return QuantisedPages(k, v, ks, vs)
 
 
