@@ -41,18 +41,35 @@ def test_largest_partition_split_k(dtype, G):
         assert_close(got, ref, dtype, f"P=8192 G={G} kernel={kern}")
 
 
-def test_many_sequences_one_grid():
-    """6000 short sequences (grid.z = 6000), 8 KV heads, groups of 4."""
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_many_sequences_one_grid(dtype):
+    """6000 short sequences (grid.z = 6000), 8 KV heads, groups of 4: outputs
+    are means of a few values, where the rounding of the softmax weights
+    shows most."""
     g = np.random.default_rng(102)
     lens = tuple(int(x) for x in g.integers(0, 40, size=6000))
-    cfg = _cfg("bf16", 32, 8, 128, 16, lens)
+    cfg = _cfg(dtype, 32, 8, 128, 16, lens)
     inp = make_decode_inputs(cfg, seed=102)
     ref = oracle.paged_decode_inputs(inp)
     dev = DeviceInputs(inp)
     order = torch.from_numpy(pkv.pkv_decode_schedule_order(inp.context_lens)).cuda()
-    for kern in _kernels("bf16", 4):
+    for kern in _kernels(dtype, 4):
         got = to_f64(dev.decode(kernel=kern, seq_order=order, fill_out=-2.0))
-        assert_close(got, ref, "bf16", f"6000 sequences kernel={kern}")
+        assert_close(got, ref, dtype, f"6000 sequences {dtype} kernel={kern}")
+
+
+@pytest.mark.parametrize("G", [1, 4])
+def test_many_short_sequences_e4m3(G):
+    """The same stress for E4M3 pages (fp16 weights in the tensor-core kernel)."""
+    g = np.random.default_rng(105)
+    lens = tuple(int(x) for x in g.integers(0, 40, size=3000))
+    cfg = _cfg("f16", 4 * G, 4, 128, 16, lens)
+    inp = make_decode_inputs(cfg, seed=105)
+    dev = E4M3Inputs(inp, seed=105)
+    ref = dev.oracle()
+    for kern in (pkv.PKV_KERNEL_SIMT, pkv.PKV_KERNEL_MMA):
+        got = to_f64(dev.decode(kernel=kern, fill_out=-2.0))
+        assert_close(got, ref, "f16", f"3000 sequences e4m3 G={G} kernel={kern}")
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
