@@ -90,8 +90,9 @@ def test_workspace_size_formula():
 
 def test_default_partition_rule():
     d = b.lib.pkv_decode_default_partition
-    assert d(64, 40, 2048) == 2048
-    assert d(8, 8, 131072) == 2048
+    assert d(64, 40, 2048) == 4096      # many units: 4096 (one partition here)
+    assert d(256, 8, 8192) == 4096
+    assert d(8, 8, 131072) == 2048      # few long sequences: 2048
     assert d(1, 1, 4096) == 64          # tiny batches split finer
     p = d(4, 4, 512)
     assert 64 <= p <= 512 and p % 64 == 0
