@@ -103,9 +103,10 @@ PKV_API int pkv_decode_has_kernel(pkv_kernel kernel);
 
 /*
  * Partition size the decode uses when `partition_size` is 0, for this shape:
- * 2048 tokens, halved while the grid would hold fewer than ~6 CTAs per SM.
- * Tuned with a longest-first seq_order; without one, 1024 can be faster when
- * lengths are very uneven.
+ * 4096 tokens when num_seqs * num_kv_heads >= 1024, else 2048, halved while
+ * the grid would hold fewer than ~6 CTAs per SM.  Tuned with a longest-first
+ * seq_order; without one, shorter partitions can be faster when lengths are
+ * very uneven.
  */
 PKV_API int pkv_decode_default_partition(int num_seqs, int num_kv_heads, int max_context_len);
 
