@@ -13,7 +13,7 @@ cudaError_t dispatch_decode_simt(const DecodeArgs& a, int head_dim, int block_si
                                  cudaStream_t stream) {
 #define PKV_SIMT_CASE(D_, BS_, HG_)                                   \
     if (head_dim == D_ && block_size == BS_ && hg == HG_)             \
-        return launch_decode_simt<T, D_, BS_, HG_, 4, 0, false, TC>(a, stream);
+        return launch_decode_simt<T, D_, BS_, HG_, 4, 0, TC>(a, stream);
 // E4M3 pages stop at 2 heads per CTA: 16 values per 16-byte chunk double the
 // q and accumulator registers, and 4 heads would spill.
 #define PKV_SIMT_HG(D_, BS_)                                 \

@@ -12,13 +12,15 @@
 // so P never leaves registers.
 //
 // Pages are staged with 2-D tiled TMA (cp.async.bulk.tensor) over the cache
-// viewed as [N * Hkv * BS rows, D columns], boxes of 64 columns x BS rows,
+// viewed as [N * Hkv * BS rows, D columns], boxes of 64 columns x 16 rows,
 // 128-byte swizzle: row r of a box keeps its 16-byte chunk c at position
 // c ^ (r % 8), so the ldmatrix reads of 8 rows at one column hit 8 different
-// bank groups.  Each warp copies its fragments of a stage into registers and
-// the stage is refilled before the math runs.  Everything else (table hoist,
-// mbarrier ring, per-warp online softmax, warp merge, split-K workspace)
-// mirrors the CUDA-core kernel.
+// bank groups.  Each warp streams its own 16-token slices through a private
+// ring of stages (its lane 0 issues the copies): it copies a slice's
+// fragments into registers, refills that stage at once and then does the
+// math, with no CTA barrier until the final merge.  Everything else (table
+// hoist, per-warp online softmax, warp merge, split-K workspace) mirrors the
+// CUDA-core kernel.
 #pragma once
 
 #include <cuda.h>

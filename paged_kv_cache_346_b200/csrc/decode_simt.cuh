@@ -9,13 +9,14 @@
 //   1. The table entries of the partition are read once, coalesced, into
 //      shared memory (4-byte entries, "pagedattention vllm" §Implementation
 //      Details).
-//   2. One thread issues 1-D bulk copies (TMA, cp.async.bulk) of whole
-//      (block, KV head) pages -- BS x D contiguous elements each for K and for
-//      V -- into a ring of STAGES shared-memory stages of TILE = 16 * NW tokens,
-//      completing on an mbarrier per stage.  Each warp first copies its part
-//      of a stage into registers; the stage is refilled (copy of stage
-//      i + STAGES) as soon as every warp has done so, before the math runs.
-//   3. Warp w takes tokens [16w, 16w + 16) of each stage.  QK: 8 lanes per
+//   2. Every warp streams its own 16-token slices (tokens [16w, 16w + 16) of
+//      each round of TILE = 16 * NW tokens) through a private ring of STAGES
+//      shared-memory stages: its lane 0 issues 1-D bulk copies (TMA,
+//      cp.async.bulk) of the slice's 16 contiguous rows of a (block, KV head)
+//      page for K and for V, completing on the stage's mbarrier.  The warp
+//      copies the slice into registers, refills that stage at once and then
+//      does the math; no barrier ties the warps together until the merge.
+//   3. Warp w takes tokens [16w, 16w + 16) of each round.  QK: 8 lanes per
 //      token, each with D/8 dims of q (float32, pre-scaled by scale*log2 e) in
 //      registers; 3 xor-shuffles finish each dot product.  Tokens past the
 //      sequence end get a logit of -inf and their values are never read, so
@@ -49,32 +50,30 @@ struct SimtStages {
         kBudget / kStageBytes >= 4 ? 4 : (kBudget / kStageBytes >= 3 ? 3 : 2);
 };
 
-// STAGES_ = 0 picks the stage count by SimtStages; WS = true adds a
-// producer warp that re-arms each stage as soon as the consumer warps have
-// released it (per-stage "empty" mbarriers) instead of a CTA-wide barrier.
+// STAGES_ = 0 picks the stage count by SimtStages (stages per warp ring; the
+// CTA's rings together hold what one CTA-wide ring of that depth would).
 // TC is the page element type: T itself, or E4M3 codes with T = fp16/bf16
 // for q and out.
-template <typename T, int D, int BS, int HG, int NW, int STAGES_ = 0, bool WS = false,
-          typename TC = T>
+template <typename T, int D, int BS, int HG, int NW, int STAGES_ = 0, typename TC = T>
 struct SimtCfg {
     static constexpr int ROW = D * Elem<TC>::kBytes;
     static constexpr int CPR = ROW / 16;
     static constexpr int EPC = Elem<TC>::kPerVec;
     static constexpr int TILE = 16 * NW;
-    static constexpr int BPT = TILE / BS;
-    static constexpr int BLK_BYTES = BS * ROW;
-    static constexpr int STAGE_BYTES = TILE * ROW;  // one of K / V
+    static constexpr int SLICE_BYTES = 16 * ROW;    // one warp's 16 tokens of K (or V)
+    static constexpr int STAGE_BYTES = TILE * ROW;  // all warps' slices of one stage
     static constexpr int STAGES = STAGES_ ? STAGES_ : SimtStages<ROW, NW>::kStages;
+    static constexpr int WARP_RING = STAGES * 2 * SLICE_BYTES;
     static constexpr int CPL = CPR / 8;
     static constexpr int LPV = CPR < 32 ? CPR : 32;
     static constexpr int TPV = 32 / LPV;
     static constexpr int CPV = CPR / LPV;
-    static constexpr int THREADS = (NW + (WS ? 1 : 0)) * 32;
-    static_assert(TILE % BS == 0, "a stage holds whole blocks");
+    static constexpr int THREADS = NW * 32;
+    static_assert(BS % 16 == 0, "16-token slices of whole rows");
     static_assert(CPR % 8 == 0, "rows of at least 128 bytes");
 
     static int smem_bytes(int partition_size) {
-        return 128 + round_up(partition_size / BS * 4, 128) + STAGES * 2 * STAGE_BYTES;
+        return 256 + round_up(partition_size / BS * 4, 128) + STAGES * 2 * STAGE_BYTES;
     }
 };
 
@@ -289,14 +288,14 @@ struct SimtWarp {
     }
 };
 
-template <typename T, int D, int BS, int HG, int NW, int STAGES_, bool WS, typename TC>
-__global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::THREADS,
-                                  SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::ROW <= 256 ? 3 : 1)
+template <typename T, int D, int BS, int HG, int NW, int STAGES_, typename TC>
+__global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::THREADS,
+                                  SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::ROW <= 256 ? 3 : 1)
     decode_simt_kernel(const DecodeArgs a) {
-    using C = SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>;
+    using C = SimtCfg<T, D, BS, HG, NW, STAGES_, TC>;
     using E = Elem<T>;
-    constexpr int ROW = C::ROW, TILE = C::TILE, BPT = C::BPT;
-    constexpr int BLK_BYTES = C::BLK_BYTES, STAGE_BYTES = C::STAGE_BYTES;
+    constexpr int ROW = C::ROW, TILE = C::TILE, SLICE_BYTES = C::SLICE_BYTES;
+    constexpr int STAGE_BYTES = C::STAGE_BYTES, WARP_RING = C::WARP_RING;
     constexpr int STAGES = C::STAGES, THREADS = C::THREADS;
 
     extern __shared__ __align__(128) unsigned char smem_simt[];
@@ -330,91 +329,71 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::TH
     const int t0 = sp.base + part * P;
     const int ntok = min(L, t0 + P) - t0;
     const int mask_lo = part == 0 ? sp.lo - sp.base : 0;  // tokens ahead of the window
-    const int ntiles = (ntok + TILE - 1) / TILE;
     const int nblk = (ntok + BS - 1) / BS;
+    // this warp's slices: tokens [k * TILE + warp * 16, + 16), k < nslices
+    const int nslices = ntok > warp * 16 ? (ntok - warp * 16 + TILE - 1) / TILE : 0;
 
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem_simt);
-    uint64_t* empty = full + STAGES;  // WS only
-    int32_t* s_tab = reinterpret_cast<int32_t*>(smem_simt + 128);
-    unsigned char* s_kv = smem_simt + 128 + round_up(P / BS * 4, 128);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem_simt);  // [NW][STAGES]
+    int32_t* s_tab = reinterpret_cast<int32_t*>(smem_simt + 256);
+    unsigned char* s_kv = smem_simt + 256 + round_up(P / BS * 4, 128);
+    static_assert(NW * STAGES * 8 <= 256, "barriers");
 
     // 1. table slice -> shared memory
     table_hoist(a, b, t0 / BS, nblk, pf, s_tab, tid, THREADS);
     if (tid == 0) {
         s_abort = 0;
-#pragma unroll
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            if (WS) mbar_init(&empty[s], NW);
-        }
+        for (int s = 0; s < NW * STAGES; ++s) mbar_init(&full[s], 1);
         fence_barrier_init();
     }
     __syncthreads();
 
+    // 2. this warp's ring: lane 0 issues the copies of slice k into a stage
     const unsigned char* kbase = reinterpret_cast<const unsigned char*>(a.k_cache);
     const unsigned char* vbase = reinterpret_cast<const unsigned char*>(a.v_cache);
-    auto issue = [&](int tile, int stage, uint64_t pol) {
-        const int jb = tile * BPT;
-        const int je = min(nblk, jb + BPT);
-        mbar_arrive_expect_tx(&full[stage], (uint32_t)((je - jb) * BLK_BYTES * 2));
-        unsigned char* kd = s_kv + stage * 2 * STAGE_BYTES;
-        unsigned char* vd = kd + STAGE_BYTES;
-        for (int j = jb; j < je; ++j) {
-            const int64_t off = ((int64_t)s_tab[j] * a.num_kv_heads + kvh) * BLK_BYTES;
-            bulk_load(kd + (j - jb) * BLK_BYTES, kbase + off, BLK_BYTES, &full[stage], pol);
-            bulk_load(vd + (j - jb) * BLK_BYTES, vbase + off, BLK_BYTES, &full[stage], pol);
-        }
+    const uint64_t pol = policy_evict_first();
+    auto issue = [&](int k, int stage) {
+        const int tok = k * TILE + warp * 16;
+        const int64_t off =
+            (((int64_t)s_tab[tok / BS] * a.num_kv_heads + kvh) * BS + tok % BS) * ROW;
+        uint64_t* bar = full + warp * STAGES + stage;
+        unsigned char* kd = s_kv + warp * WARP_RING + stage * 2 * SLICE_BYTES;
+        mbar_arrive_expect_tx(bar, (uint32_t)(2 * SLICE_BYTES));
+        bulk_load(kd, kbase + off, SLICE_BYTES, bar, pol);
+        bulk_load(kd + SLICE_BYTES, vbase + off, SLICE_BYTES, bar, pol);
     };
+    if (lane == 0) {
+        const int pre = min(STAGES, nslices);
+        for (int s = 0; s < pre; ++s) issue(s, s);
+    }
 
-    float* red = reinterpret_cast<float*>(s_kv);  // merge area, after the last stage
+    float* red = reinterpret_cast<float*>(s_kv);  // merge area, once the rings are drained
     static_assert(MergeArea<D, HG, NW>::BYTES <= STAGES * 2 * STAGE_BYTES, "merge area");
 
-    if (WS && warp == NW) {
-        // 2. producer warp: keep every stage loaded as soon as it is released
-        if (lane == 0) {
-            const uint64_t pol = policy_evict_first();
-            for (int it = 0; it < ntiles; ++it) {
-                const int stage = it % STAGES;
-                if (it >= STAGES &&
-                    !mbar_wait(&empty[stage], (uint32_t)(((it / STAGES) - 1) & 1), a.status)) {
-                    s_abort = 1;
-                    break;
-                }
-                if (s_abort) break;
-                issue(it, stage, pol);
-            }
-        }
-        __syncthreads();  // matches the consumers' barrier before the merge
-        if (s_abort) return;
-        pdl_launch_dependents();
-        __syncthreads();
-        merge_warps_and_store<T, D, HG, NW>(a, red, b, h0, nh, part, np, tid, THREADS);
-        return;
-    }
-
-    if (!WS && tid == 0) {
-        const uint64_t pol = policy_evict_first();
-        const int pre = min(STAGES, ntiles);
-        for (int s = 0; s < pre; ++s) issue(s, s, pol);
-    }
-
-    // 3.-5. consumer warps
+    // 3.-5. the warps
     SimtWarp<T, D, HG, C, TC> W;
     W.init(reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D, nh,
            a.k_scale && !a.scale_per_block ? a.scale_log2 * a.k_scale[kvh] : a.scale_log2,
            lane);
-    const uint64_t pol = WS ? 0 : policy_evict_first();
-    int it_stop = ntiles;  // the tile a timed-out wait stopped at
-    for (int it = 0; it < ntiles; ++it) {
+    for (int it = 0; it < nslices; ++it) {
         const int stage = it % STAGES;
-        if (!mbar_wait(&full[stage], (uint32_t)((it / STAGES) & 1), a.status)) s_abort = 1;
-        if (WS && s_abort) break;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(full + warp * STAGES + stage,
+                                                          (uint32_t)((it / STAGES) & 1), a.status));
+        if (!ok) {
+            s_abort = 1;
+            // let this warp's copies still in flight land (bounded) before
+            // the CTA leaves
+            if (lane == 0)
+                for (int k = it; k < min(nslices, it + STAGES); ++k)
+                    mbar_wait(full + warp * STAGES + k % STAGES, (uint32_t)((k / STAGES) & 1),
+                              a.status);
+            break;
+        }
         const int wvalid = ntok - (it * TILE + warp * 16);  // tokens this warp owns
         const int wlo = mask_lo - (it * TILE + warp * 16);
-        const bool work = wvalid > 0 && wlo < 16 && wlo < wvalid;
-        if (!s_abort && work) {
-            const unsigned char* Kw = s_kv + stage * 2 * STAGE_BYTES + warp * 16 * ROW;
-            W.fetch(Kw, Kw + STAGE_BYTES);
+        const bool work = wlo < 16 && wlo < wvalid;
+        if (work) {
+            const unsigned char* Kw = s_kv + warp * WARP_RING + stage * 2 * SLICE_BYTES;
+            W.fetch(Kw, Kw + SLICE_BYTES);
         }
         float kts = 1.f, vts = 1.f;  // page scales of this warp's tokens (per-page mode)
         if (a.scale_per_block && work) {
@@ -423,44 +402,28 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, WS, TC>::TH
             kts = a.k_scale[si];
             vts = a.v_scale[si];
         }
-        if (!W.EARLY && !s_abort && work) W.compute(wlo, wvalid, s_p[warp], kts, vts);
-        // the stage's data is in registers (or used): hand the stage back
-        if (WS) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-        } else {
-            __syncthreads();
-            if (s_abort) {
-                it_stop = it;
-                break;
-            }
-            if (tid == 0 && it + STAGES < ntiles) issue(it + STAGES, stage, pol);
-        }
+        if (!W.EARLY && work) W.compute(wlo, wvalid, s_p[warp], kts, vts);
+        // the slice is in registers (or used): refill its stage
+        __syncwarp();
+        if (lane == 0 && it + STAGES < nslices) issue(it + STAGES, stage);
         if (W.EARLY && work) W.compute(wlo, wvalid, s_p[warp], kts, vts);
     }
-    if (WS) __syncthreads();  // producer and consumers: every stage consumed
-    if (s_abort) {
-        // let the copies still in flight land (bounded) before the CTA leaves
-        if (!WS && tid == 0)
-            for (int k = it_stop; k < min(ntiles, it_stop + STAGES); ++k)
-                mbar_wait(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), a.status);
-        return;
-    }
-    if (!WS) pdl_launch_dependents();
+    __syncthreads();  // every warp is out of its ring (or gave up)
+    if (s_abort) return;
+    pdl_launch_dependents();
 
     // 6. merge the warps
     W.template park<NW>(warp, red, a.v_scale && !a.scale_per_block ? a.v_scale[kvh] : 1.f);
     __syncthreads();
-    merge_warps_and_store<T, D, HG, NW>(a, red, b, h0, nh, part, np, tid, WS ? THREADS : NW * 32);
+    merge_warps_and_store<T, D, HG, NW>(a, red, b, h0, nh, part, np, tid, NW * 32);
 }
 
-template <typename T, int D, int BS, int HG, int NW = 4, int STAGES = 0, bool WS = false,
-          typename TC = T>
+template <typename T, int D, int BS, int HG, int NW = 4, int STAGES = 0, typename TC = T>
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
-    using C = SimtCfg<T, D, BS, HG, NW, STAGES, WS, TC>;
+    using C = SimtCfg<T, D, BS, HG, NW, STAGES, TC>;
     static SmemAttr attr;
     const int smem_simt = C::smem_bytes(a.partition_size);
-    auto kern = decode_simt_kernel<T, D, BS, HG, NW, STAGES, WS, TC>;
+    auto kern = decode_simt_kernel<T, D, BS, HG, NW, STAGES, TC>;
     cudaError_t e = attr.ensure(kern, C::smem_bytes(8192));
     if (e != cudaSuccess) return e;
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
