@@ -220,16 +220,19 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float
 //   M = max_p m_p,  w_p = l_p 2^(m_p - M),  out = sum_p w_p o_p / sum_p w_p.
 // One CTA of 128 threads per row; rows that fit one partition were written by
 // the decode kernel and are skipped.  Launched as a programmatic dependent of
-// the decode kernel: it waits for the decode grid's writes before reading.
+// the decode kernel: rows of one partition leave before the wait, during the
+// decode's tail; the others wait for the decode grid's writes before reading.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
     constexpr int NW = 4;
     constexpr int PER_LANE = D / 32;  // floats of o per lane
-    pdl_wait_primary();
     const int h = blockIdx.x;
     const int b = blockIdx.y;
+    // the partition count depends only on the inputs, not on the decode
+    // grid's output: rows with one partition leave before the wait
     const int np = seq_span(a, b, false).np;
     if (np <= 1) return;
+    pdl_wait_primary();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row = (int64_t)b * a.num_q_heads + h;
     const float* ml = a.ws_ml + row * a.max_partitions * 2;

@@ -128,6 +128,12 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         return;
     }
     if (part >= np) return;
+    // A sequence that fits one partition needs no merge: release the reduce
+    // grid at once (it starts when every CTA of this grid has released it or
+    // left, and its rows of one partition leave without waiting).  CTAs of
+    // split sequences release it after their loop, so a grid of mostly split
+    // sequences keeps the reduce from taking SM slots while it streams.
+    if (np == 1) pdl_launch_dependents();
 
     const int P = a.partition_size;
     const int t0 = sp.base + part * P;
@@ -423,7 +429,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     }
     __syncthreads();  // every warp is out of its ring (or gave up)
     if (s_abort) return;
-    pdl_launch_dependents();
+    if (np > 1) pdl_launch_dependents();
 
     // merge the warps; A rows g, g + 8 of m-tile mt are dims 16 mt + 2 g, + 1
     using A = MergeArea<D, NH, NW>;
