@@ -2,7 +2,10 @@
 //
 // The same two contractions as the 16-bit tensor-core kernel,
 //   S[h, t] = sum_d Q[h, d] K[t, d]        O^T[d, h] = sum_t V[t, d] P[h, t],
-// with mma.sync m16n8k16 in fp16 (fp32 accumulation).  The pages stay one
+// with mma.sync m16n8k16 in fp16 (fp32 accumulation).  A tile of 8 heads
+// computes S as K Q^T (M = the slice's 16 tokens, N = 8 heads: one MMA per
+// 16-dim step, where an 8-head S^T tile fills half of M); a 16-head tile
+// computes S^T as Q K^T (M = heads, N = tokens).  The pages stay one
 // byte per element all the way into the registers: ldmatrix moves 16-byte
 // rows of codes, and each register of four codes becomes two f16x2 operand
 // registers with the hardware E4M3 -> f16x2 conversion (exact: every E4M3
@@ -11,17 +14,20 @@
 //
 // Operand layouts (the contraction order is free, so the byte layout that
 // ldmatrix delivers is kept and the other operand is arranged to match):
-//   * K as the B operand of S: ldmatrix (non-transposed) hands lane (g, t4)
-//     the codes K[t = g][4 t4 .. 4 t4 + 3] of a 16-dim step.  The low pair
-//     serves logical k = 2 t4, 2 t4 + 1, the high pair k = 2 t4 + 8, + 9, so
-//     Q's A fragment takes dims 4 t4, 4 t4 + 1 and 4 t4 + 2, 4 t4 + 3 at those
-//     positions.
+//   * K: ldmatrix (non-transposed) hands lane (g, t4) the codes
+//     K[t = g][4 t4 .. 4 t4 + 3] of a 16-dim step (and of t = g + 8).  The low
+//     pair serves logical k = 2 t4, 2 t4 + 1, the high pair k = 2 t4 + 8, + 9,
+//     so Q's fragment (B columns of an 8-head tile, A rows of a 16-head tile)
+//     takes dims 4 t4, 4 t4 + 1 and 4 t4 + 2, 4 t4 + 3 at those positions.
+//     An 8-head tile's S accumulator gives lane (g, t4) tokens g, g + 8 of
+//     heads 2 t4, 2 t4 + 1; after rounding to fp16, one movmatrix.trans per 8
+//     tokens turns it into P^T's B fragment (head g, tokens 2 t4, 2 t4 + 1).
+//     A 16-head tile's S^T accumulator is already that fragment.
 //   * V^T as the A operand of O^T: ldmatrix.trans on 2-byte units hands lane
 //     (g, t4) the codes V[2 t4][2 g], V[2 t4][2 g + 1], V[2 t4 + 1][2 g],
 //     V[2 t4 + 1][2 g + 1].  One byte permute makes the token pairs of dims
 //     2 g and 2 g + 1: A rows g and g + 8 of an m-tile are dims 2 g and 2 g + 1
-//     of its 16, and the tokens (k) keep their natural order, so P^T comes
-//     straight from the S accumulators as in the 16-bit kernel.
+//     of its 16, and the tokens (k) keep their natural order.
 //
 // q (fp16 or bf16) enters the fp16 MMA multiplied by a power of two 2^e that
 // puts its largest magnitude in [2^14, 2^15) (exact for every value that stays
@@ -79,6 +85,14 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1,
         "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// transpose an 8 x 8 matrix of 16-bit values held in the mma fragment layout
+// (lane (g, t4): row g, columns 2 t4 and 2 t4 + 1)
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t r;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) {
@@ -233,17 +247,22 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
             }
     }
 
-    float m[RB], l[RB];
+    // softmax state: 8-head tiles keep it for heads 2 t4, 2 t4 + 1 (the S
+    // columns of this lane), 16-head tiles for heads g + 8 rb (its S^T rows)
+    constexpr int MS = NH == 8 ? 2 : RB;
+    float m[MS], l[MS];
+#pragma unroll
+    for (int j = 0; j < MS; ++j) {
+        m[j] = -INFINITY;
+        l[j] = 0.f;
+    }
     float o[KSTEPS][RB][4];
 #pragma unroll
-    for (int rb = 0; rb < RB; ++rb) {
-        m[rb] = -INFINITY;
-        l[rb] = 0.f;
+    for (int rb = 0; rb < RB; ++rb)
 #pragma unroll
         for (int mt = 0; mt < KSTEPS; ++mt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) o[mt][rb][i] = 0.f;
-    }
 
     // ldmatrix.x4 row addresses: matrices (tokens 0-7, chunk c), (tokens 8-15,
     // chunk c), (tokens 0-7, chunk c + 1), (tokens 8-15, chunk c + 1)
@@ -293,87 +312,153 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
             }
         }
         auto math = [&]() {
-            // two accumulator sets (even / odd k-steps): two short MMA
-            // dependency chains instead of one long one
-            float s[2][4], s2[2][4];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) s[nt][i] = s2[nt][i] = 0.f;
-#pragma unroll
-            for (int kp = 0; kp < KP; ++kp) {
-                uint32_t kc[4];
+            const bool partial = wvalid < 16 || wlo > 0;
+            bool grew;               // the reference max moved: rescale o
+            float alpha_c[RB][2];    // rescale factors of o's columns 2 t4, 2 t4 + 1
+            uint32_t pb[RB][2];      // P^T as the B operand: tokens 0-7, 8-15
+            auto kcodes = [&](int kp, uint32_t (&kc)[4]) {
                 if constexpr (EARLY) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) kc[i] = kf[kp < (EARLY ? KP : 1) ? kp : 0][i];
                 } else {
                     ldsm_x4(addr(kp), kc);
                 }
+            };
+            if constexpr (NH == 8) {
+                // S[t, h] = K Q^T with the slice's 16 tokens as M and the 8
+                // heads as N: one MMA per 16-dim step (an 8-head S^T tile
+                // would fill half of M).  K codes of tokens g / g + 8 are the
+                // A rows, q the B columns; two accumulator sets (even / odd
+                // steps) make two short dependency chains.
+                float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {  // k-step 2 kp + h
-                    uint32_t b0, b1, b2, b3;
-                    e4m3x4_to_f16x2(kc[2 * h], b0, b1);      // tokens 0-7
-                    e4m3x4_to_f16x2(kc[2 * h + 1], b2, b3);  // tokens 8-15
-                    const uint32_t* q4 = qa[2 * kp + h];
-                    const uint32_t a0 = q4[0], a1 = NH == 16 ? q4[1] : 0u;
-                    const uint32_t a2 = NH == 16 ? q4[2] : q4[1], a3 = NH == 16 ? q4[3] : 0u;
-                    mma_f16(h ? s2[0] : s[0], a0, a1, a2, a3, b0, b1);
-                    mma_f16(h ? s2[1] : s[1], a0, a1, a2, a3, b2, b3);
+                for (int kp = 0; kp < KP; ++kp) {
+                    uint32_t kc[4];
+                    kcodes(kp, kc);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {  // k-step 2 kp + h
+                        uint32_t k0, k1, k2, k3;
+                        e4m3x4_to_f16x2(kc[2 * h], k0, k1);      // token g
+                        e4m3x4_to_f16x2(kc[2 * h + 1], k2, k3);  // token g + 8
+                        const uint32_t* q4 = qa[2 * kp + h];
+                        mma_f16(h ? s2 : s, k0, k2, k1, k3, q4[0], q4[1]);
+                    }
                 }
-            }
-            const bool partial = wvalid < 16 || wlo > 0;
+                // lane (g, t4): s[0], s[1] = token g, heads 2 t4, 2 t4 + 1;
+                // s[2], s[3] = token g + 8
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+                for (int i = 0; i < 4; ++i) {
+                    s[i] = (s[i] + s2[i]) * kmul;
+                    const int tok = g + 8 * (i >> 1);
+                    if (partial && (tok < wlo || tok >= wvalid)) s[i] = -INFINITY;
+                }
+                // lazy reference max per head (see below); a head's tokens
+                // are spread over the 8 lanes of one t4
+                bool up = false;
+                float tmax[2];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) s[nt][i] = (s[nt][i] + s2[nt][i]) * kmul;
-            if (partial) {
+                for (int j = 0; j < 2; ++j) {
+                    tmax[j] = fmaxf(s[j], s[2 + j]);
+                    up |= tmax[j] > m[j] + 8.f;
+                }
+                grew = __any_sync(0xffffffffu, up);
+                if (grew) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        float mx = tmax[j];
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                        const float mnew = fmaxf(m[j], mx);
+                        const float alpha = exp2f(m[j] - mnew);
+                        l[j] *= alpha;
+                        m[j] = mnew;
+                        alpha_c[0][j] = alpha;
+                    }
+                }
+                float pr[4];
+                const uint32_t p0 = M::pack(exp2f(s[0] - m[0]), exp2f(s[1] - m[1]), pr[0], pr[1]);
+                const uint32_t p1 = M::pack(exp2f(s[2] - m[0]), exp2f(s[3] - m[1]), pr[2], pr[3]);
+                l[0] += pr[0] + pr[2];
+                l[1] += pr[1] + pr[3];
+                // P (tokens x heads) -> P^T fragments: lane (g, t4) gets head
+                // g, tokens 2 t4, 2 t4 + 1 (of 0-7, then of 8-15)
+                pb[0][0] = movmatrix_trans(p0);
+                pb[0][1] = movmatrix_trans(p1);
+            } else {
+                // 16-head tiles: S^T[h, t] = Q K^T, heads as M, the slice's
+                // tokens as N (two n-tiles), two accumulator sets
+                float s[2][4], s2[2][4];
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int tok = nt * 8 + 2 * t4 + (i & 1);
-                        if (tok < wlo || tok >= wvalid) s[nt][i] = -INFINITY;
-                    }
-            }
-            // Softmax against a reference max m that moves only when a logit
-            // exceeds it by more than 2^8 (then p <= 256 fits fp16 and the
-            // accumulators are rescaled); l is kept per lane (this lane's
-            // tokens) and summed over the row's four lanes at the end.  The
-            // result is the same softmax: every p and l of a head shares m.
-            bool up = false;
-            float tmax[RB];
+                    for (int i = 0; i < 4; ++i) s[nt][i] = s2[nt][i] = 0.f;
 #pragma unroll
-            for (int rb = 0; rb < RB; ++rb) {
-                const int i0 = 2 * rb;
-                tmax[rb] = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
-                up |= tmax[rb] > m[rb] + 8.f;
-            }
-            const bool grew = __any_sync(0xffffffffu, up);
-            float alpha_c[RB][2];
-            if (grew) {
+                for (int kp = 0; kp < KP; ++kp) {
+                    uint32_t kc[4];
+                    kcodes(kp, kc);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {  // k-step 2 kp + h
+                        uint32_t b0, b1, b2, b3;
+                        e4m3x4_to_f16x2(kc[2 * h], b0, b1);      // tokens 0-7
+                        e4m3x4_to_f16x2(kc[2 * h + 1], b2, b3);  // tokens 8-15
+                        const uint32_t* q4 = qa[2 * kp + h];
+                        mma_f16(h ? s2[0] : s[0], q4[0], q4[1], q4[2], q4[3], b0, b1);
+                        mma_f16(h ? s2[1] : s[1], q4[0], q4[1], q4[2], q4[3], b2, b3);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) s[nt][i] = (s[nt][i] + s2[nt][i]) * kmul;
+                if (partial) {
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int tok = nt * 8 + 2 * t4 + (i & 1);
+                            if (tok < wlo || tok >= wvalid) s[nt][i] = -INFINITY;
+                        }
+                }
+                // Softmax against a reference max m that moves only when a
+                // logit exceeds it by more than 2^8 (then p <= 256 fits fp16
+                // and the accumulators are rescaled); l is kept per lane (this
+                // lane's tokens) and summed over the head's lanes at the end.
+                // The result is the same softmax: every p and l of a head
+                // shares m.
+                bool up = false;
+                float tmax[RB];
 #pragma unroll
                 for (int rb = 0; rb < RB; ++rb) {
-                    float mx = tmax[rb];
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                    const float mnew = fmaxf(m[rb], mx);
-                    const float alpha = exp2f(m[rb] - mnew);
-                    l[rb] *= alpha;
-                    m[rb] = mnew;
-                    alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
-                    alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
+                    const int i0 = 2 * rb;
+                    tmax[rb] = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
+                    up |= tmax[rb] > m[rb] + 8.f;
                 }
-            }
-            uint32_t pb[RB][2];
+                grew = __any_sync(0xffffffffu, up);
+                if (grew) {
 #pragma unroll
-            for (int rb = 0; rb < RB; ++rb) {
-                const int i0 = 2 * rb;
-                float pr[2][2];
+                    for (int rb = 0; rb < RB; ++rb) {
+                        float mx = tmax[rb];
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                        const float mnew = fmaxf(m[rb], mx);
+                        const float alpha = exp2f(m[rb] - mnew);
+                        l[rb] *= alpha;
+                        m[rb] = mnew;
+                        alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
+                        alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
+                    }
+                }
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-                    pb[rb][nt] = M::pack(exp2f(s[nt][i0] - m[rb]), exp2f(s[nt][i0 + 1] - m[rb]),
-                                         pr[nt][0], pr[nt][1]);
-                l[rb] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+                for (int rb = 0; rb < RB; ++rb) {
+                    const int i0 = 2 * rb;
+                    float pr[2][2];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+                        pb[rb][nt] = M::pack(exp2f(s[nt][i0] - m[rb]), exp2f(s[nt][i0 + 1] - m[rb]),
+                                             pr[nt][0], pr[nt][1]);
+                    l[rb] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+                }
             }
 #pragma unroll
             for (int kp = 0; kp < KP; ++kp) {
@@ -448,16 +533,32 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                 const int dim = mt * 16 + 2 * g + (i >> 1);
                 red[(warp * NH + head) * A::RP + dim] = o[mt][rb][i] * vs;
             }
+    if constexpr (NH == 8) {  // heads 2 t4 + j, summed over the lanes of one t4
 #pragma unroll
-    for (int rb = 0; rb < RB; ++rb) {
-        l[rb] += __shfl_xor_sync(0xffffffffu, l[rb], 1);
-        l[rb] += __shfl_xor_sync(0xffffffffu, l[rb], 2);
-    }
-    if (t4 == 0) {
+        for (int j = 0; j < 2; ++j) {
+            l[j] += __shfl_xor_sync(0xffffffffu, l[j], 4);
+            l[j] += __shfl_xor_sync(0xffffffffu, l[j], 8);
+            l[j] += __shfl_xor_sync(0xffffffffu, l[j], 16);
+        }
+        if (g == 0) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                red_m[warp * NH + 2 * t4 + j] = m[j];
+                red_l[warp * NH + 2 * t4 + j] = l[j];
+            }
+        }
+    } else {  // heads g + 8 rb, summed over the lanes of one g
 #pragma unroll
         for (int rb = 0; rb < RB; ++rb) {
-            red_m[warp * NH + g + 8 * rb] = m[rb];
-            red_l[warp * NH + g + 8 * rb] = l[rb];
+            l[rb] += __shfl_xor_sync(0xffffffffu, l[rb], 1);
+            l[rb] += __shfl_xor_sync(0xffffffffu, l[rb], 2);
+        }
+        if (t4 == 0) {
+#pragma unroll
+            for (int rb = 0; rb < RB; ++rb) {
+                red_m[warp * NH + g + 8 * rb] = m[rb];
+                red_l[warp * NH + g + 8 * rb] = l[rb];
+            }
         }
     }
     __syncthreads();
