@@ -5,11 +5,14 @@
 // systemdesign.academy: grouped-query attention lets several heads share one
 // set of keys and values), each K/V page feeds G dot products per token: for
 // G >= 4 the two products of a CTA's tile are small dense contractions,
-//   S^T[h, t] = sum_d Q[h, d] K[t, d]           (M = heads, N = tokens, K = dims)
-//   O^T[d, h] = sum_t V[t, d] P[h, t]           (M = dims, N = heads, K = tokens)
-// done with mma.sync m16n8k16 (fp16/bf16 inputs, fp32 accumulation).  The QK
-// accumulator layout of S^T is exactly the B-operand layout P^T needs for PV,
-// so P never leaves registers.
+//   S[t, h] = sum_d K[t, d] Q[h, d]   8-head tiles  (M = tokens, N = heads, K = dims)
+//   S^T[h, t] = sum_d Q[h, d] K[t, d] 16-head tiles (M = heads, N = tokens, K = dims)
+//   O^T[d, h] = sum_t V[t, d] P[h, t]               (M = dims, N = heads, K = tokens)
+// done with mma.sync m16n8k16 (fp16/bf16 inputs, fp32 accumulation).  With
+// 8 heads, S puts the warp's 16 tokens in M (an S^T tile would leave half of
+// M empty): one MMA per 16-dim step; one movmatrix.trans per 8 tokens turns
+// the rounded P into the B fragment of P^T.  A 16-head tile's S^T
+// accumulator already has that layout.  P never leaves registers.
 //
 // Pages are staged with 2-D tiled TMA (cp.async.bulk.tensor) over the cache
 // viewed as [N * Hkv * BS rows, D columns], boxes of 64 columns x 16 rows,
@@ -52,6 +55,14 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(addr));
+}
+
+// transpose an 8 x 8 matrix of 16-bit values held in the mma fragment layout
+// (lane (g, t4): row g, columns 2 t4 and 2 t4 + 1)
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t r;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+    return r;
 }
 
 template <typename T>
@@ -215,37 +226,46 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         for (int s = 0; s < pre; ++s) issue(s, s);
     }
 
-    // Q as the A operand: rows = heads (g, g + 8), columns = dims.
-    uint32_t qa[KSTEPS][4];
+    // Q: dims 2 t4, 2 t4 + 1 (lo) and 8 + 2 t4, + 1 (hi) of a 16-dim step for
+    // head g (and g + 8) -- the B column g of an 8-head tile's S, the A rows
+    // g, g + 8 of a 16-head tile's S^T.
+    constexpr int QR = NH == 8 ? 1 : 2;
+    uint32_t qa[KSTEPS][2 * QR];  // [lo g, (lo g + 8,) hi g, (hi g + 8)]
     {
         const T* qb = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D;
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks) {
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {  // r = 0: head g, r = 1: head g + 8
+            for (int r = 0; r < QR; ++r) {  // r = 0: head g, r = 1: head g + 8
                 const int hh = g + 8 * r;
                 uint32_t lo = 0, hi = 0;
                 if (hh < nh) {
                     lo = *reinterpret_cast<const uint32_t*>(qb + hh * D + ks * 16 + 2 * t4);
                     hi = *reinterpret_cast<const uint32_t*>(qb + hh * D + ks * 16 + 8 + 2 * t4);
                 }
-                qa[ks][r] = lo;       // a0 (r = 0) / a1 (r = 1)
-                qa[ks][2 + r] = hi;   // a2 / a3
+                qa[ks][r] = lo;
+                qa[ks][QR + r] = hi;
             }
         }
     }
 
-    float m[RB], l[RB];
+    // softmax state: 8-head tiles keep it for heads 2 t4, 2 t4 + 1 (the S
+    // columns of this lane; l per lane, summed at the end), 16-head tiles
+    // for heads g + 8 rb (the S^T rows; l summed every slice)
+    constexpr int MS = NH == 8 ? 2 : RB;
+    float m[MS], l[MS];
+#pragma unroll
+    for (int j = 0; j < MS; ++j) {
+        m[j] = -INFINITY;
+        l[j] = 0.f;
+    }
     float o[KSTEPS][RB][4];
 #pragma unroll
-    for (int rb = 0; rb < RB; ++rb) {
-        m[rb] = -INFINITY;
-        l[rb] = 0.f;
+    for (int rb = 0; rb < RB; ++rb)
 #pragma unroll
         for (int mt = 0; mt < KSTEPS; ++mt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) o[mt][rb][i] = 0.f;
-    }
 
     // ldmatrix row addresses: lane -> (token within the warp's 16, chunk parity)
     const int lrow = (lane >> 4) * 8 + (lane & 7);
@@ -286,67 +306,122 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
             }
         }
         auto math = [&]() {
-            // S^T = Q K^T: two n-tiles of 8 tokens
-            float s[2][4];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
-#pragma unroll
-            for (int ks = 0; ks < KSTEPS; ++ks) {
-                uint32_t kb[4];
+            auto kfrag = [&](int ks, uint32_t (&kb)[4]) {
+                // kb: token g dims 2 t4 (+1), token g dims 8 + 2 t4 (+1),
+                // token g + 8 dims 2 t4 (+1), token g + 8 dims 8 + 2 t4 (+1)
                 if constexpr (EARLY) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) kb[i] = kf[ks < (EARLY ? KSTEPS : 1) ? ks : 0][i];
                 } else {
                     ldsm_x4(kaddr(ks), kb);
                 }
-                M::run(s[0], qa[ks], kb[0], kb[1]);
-                M::run(s[1], qa[ks], kb[2], kb[3]);
-            }
-            // logits in base 2, masked past the sequence end
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int tok = nt * 8 + 2 * t4 + (i & 1);
-                    s[nt][i] = (tok >= wlo && tok < wvalid) ? s[nt][i] * a.scale_log2 : -INFINITY;
-                }
+            };
             // P enters the MMA in T.  bf16 keeps 8 significant bits, too few
             // for the weights: P = hi + lo, two bf16 terms (~16 bits), and
             // two P.V products.  fp16's 11 bits are kept as one term.
             constexpr bool SPLIT = std::is_same<T, __nv_bfloat16>::value;
             uint32_t pb[RB][2], pl[RB][2];
             float alpha_c[RB][2];
+            if constexpr (NH == 8) {
+                // S = K Q^T: A rows = tokens g, g + 8, B column = head g
+                float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int rb = 0; rb < RB; ++rb) {
-                const int i0 = 2 * rb;  // s[nt][i0], s[nt][i0 + 1]: head g + 8 rb
-                float mx = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                const float mnew = fmaxf(m[rb], mx);
-                const float alpha = exp2f(m[rb] - mnew);
-                float p[2][2], pr[2][2];
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    p[nt][0] = exp2f(s[nt][i0] - mnew);
-                    p[nt][1] = exp2f(s[nt][i0 + 1] - mnew);
-                    pb[rb][nt] = M::pack(p[nt][0], p[nt][1], pr[nt][0], pr[nt][1]);
-                    if constexpr (SPLIT) {
-                        float r0, r1;
-                        pl[rb][nt] = M::pack(p[nt][0] - pr[nt][0], p[nt][1] - pr[nt][1], r0, r1);
-                        pr[nt][0] += r0;  // the weights P.V uses, hi + lo
-                        pr[nt][1] += r1;
-                    }
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    uint32_t kb[4];
+                    kfrag(ks, kb);
+                    const uint32_t ka[4] = {kb[0], kb[2], kb[1], kb[3]};
+                    M::run(s, ka, qa[ks][0], qa[ks][1]);
                 }
-                float ps = (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-                ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-                ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-                l[rb] = l[rb] * alpha + ps;
-                m[rb] = mnew;
-                // O^T columns of this thread are heads 2 t4, 2 t4 + 1 (+ 8 rb)
-                alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
-                alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
+                // lane (g, t4): s[0], s[1] = token g, heads 2 t4, 2 t4 + 1;
+                // s[2], s[3] = token g + 8; logits in base 2, masked past the
+                // sequence end
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int tok = g + 8 * (i >> 1);
+                    s[i] = (tok >= wlo && tok < wvalid) ? s[i] * a.scale_log2 : -INFINITY;
+                }
+                float mnew[2], p[4], pr[4];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {  // head 2 t4 + j: its tokens sit on the 8 lanes of t4
+                    float mx = fmaxf(s[j], s[2 + j]);
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    mnew[j] = fmaxf(m[j], mx);
+                    alpha_c[0][j] = exp2f(m[j] - mnew[j]);
+                    m[j] = mnew[j];
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) p[i] = exp2f(s[i] - mnew[i & 1]);
+                const uint32_t h0p = M::pack(p[0], p[1], pr[0], pr[1]);
+                const uint32_t h1p = M::pack(p[2], p[3], pr[2], pr[3]);
+                // P (tokens x heads) -> P^T fragments: head g, tokens 2 t4,
+                // 2 t4 + 1 of 0-7, then of 8-15
+                pb[0][0] = movmatrix_trans(h0p);
+                pb[0][1] = movmatrix_trans(h1p);
+                if constexpr (SPLIT) {
+                    float r[4];
+                    const uint32_t l0p = M::pack(p[0] - pr[0], p[1] - pr[1], r[0], r[1]);
+                    const uint32_t l1p = M::pack(p[2] - pr[2], p[3] - pr[3], r[2], r[3]);
+                    pl[0][0] = movmatrix_trans(l0p);
+                    pl[0][1] = movmatrix_trans(l1p);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) pr[i] += r[i];  // the weights P.V uses, hi + lo
+                }
+#pragma unroll
+                for (int j = 0; j < 2; ++j) l[j] = l[j] * alpha_c[0][j] + (pr[j] + pr[2 + j]);
+            } else {
+                // S^T = Q K^T: two n-tiles of 8 tokens
+                float s[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    uint32_t kb[4];
+                    kfrag(ks, kb);
+                    M::run(s[0], qa[ks], kb[0], kb[1]);
+                    M::run(s[1], qa[ks], kb[2], kb[3]);
+                }
+                // logits in base 2, masked past the sequence end
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int tok = nt * 8 + 2 * t4 + (i & 1);
+                        s[nt][i] = (tok >= wlo && tok < wvalid) ? s[nt][i] * a.scale_log2 : -INFINITY;
+                    }
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) {
+                    const int i0 = 2 * rb;  // s[nt][i0], s[nt][i0 + 1]: head g + 8 rb
+                    float mx = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    const float mnew = fmaxf(m[rb], mx);
+                    const float alpha = exp2f(m[rb] - mnew);
+                    float p[2][2], pr[2][2];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        p[nt][0] = exp2f(s[nt][i0] - mnew);
+                        p[nt][1] = exp2f(s[nt][i0 + 1] - mnew);
+                        pb[rb][nt] = M::pack(p[nt][0], p[nt][1], pr[nt][0], pr[nt][1]);
+                        if constexpr (SPLIT) {
+                            float r0, r1;
+                            pl[rb][nt] = M::pack(p[nt][0] - pr[nt][0], p[nt][1] - pr[nt][1], r0, r1);
+                            pr[nt][0] += r0;  // the weights P.V uses, hi + lo
+                            pr[nt][1] += r1;
+                        }
+                    }
+                    float ps = (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+                    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+                    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+                    l[rb] = l[rb] * alpha + ps;
+                    m[rb] = mnew;
+                    // O^T columns of this thread are heads 2 t4, 2 t4 + 1 (+ 8 rb)
+                    alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
+                    alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
+                }
             }
             // O^T += V^T P^T
             const bool partial = wvalid < 16 || wlo > 0;
@@ -406,7 +481,21 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                 const int dim = mt * 16 + g + 8 * (i >> 1);
                 red[(warp * NH + head) * A::RP + dim] = o[mt][rb][i];
             }
-    if (t4 == 0) {
+    if constexpr (NH == 8) {  // heads 2 t4 + j, l summed over the lanes of one t4
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            l[j] += __shfl_xor_sync(0xffffffffu, l[j], 4);
+            l[j] += __shfl_xor_sync(0xffffffffu, l[j], 8);
+            l[j] += __shfl_xor_sync(0xffffffffu, l[j], 16);
+        }
+        if (g == 0) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                red_m[warp * NH + 2 * t4 + j] = m[j];
+                red_l[warp * NH + 2 * t4 + j] = l[j];
+            }
+        }
+    } else if (t4 == 0) {
 #pragma unroll
         for (int rb = 0; rb < RB; ++rb) {
             red_m[warp * NH + g + 8 * rb] = m[rb];

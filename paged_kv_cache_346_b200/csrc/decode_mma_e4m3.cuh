@@ -87,14 +87,6 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1,
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// transpose an 8 x 8 matrix of 16-bit values held in the mma fragment layout
-// (lane (g, t4): row g, columns 2 t4 and 2 t4 + 1)
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-    uint32_t r;
-    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
-    return r;
-}
-
 __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(x), "r"(sel));
