@@ -308,7 +308,7 @@ def run_ours(args, cfg):
             "mma": pkv.PKV_KERNEL_MMA}[args.kernel]
 
     # ---- inputs (seeded; each rank its own replica)
-    inp = make_decode_inputs(cfg, seed=args.seed + rank)
+    inp = make_decode_inputs(cfg, seed=args.seed + rank, shuffle=args.tables == "shuffled")
     e4m3 = args.kv in ("e4m3", "e4m3-page")
     per_page = args.kv == "e4m3-page"
     if e4m3 and cfg.dtype == "f32":
@@ -529,6 +529,7 @@ def run_ours(args, cfg):
                        "num_q_heads": cfg.num_q_heads, "num_kv_heads": H, "head_dim": D,
                        "block_size": bs, "partition_size": Pused, "kernel": args.kernel,
                        "schedule": "longest-first" if args.order else "batch order",
+                       "block_tables": args.tables,
                        "sliding_window": W,
                        "kv_pages": ("e4m3 (per-page fp32 scales)" if per_page else
                                     "e4m3 (per-head fp32 scales)") if e4m3 else cfg.dtype,
@@ -796,6 +797,9 @@ def main():
     ap.add_argument("--kv", choices=["same", "e4m3", "e4m3-page"], default="same",
                     help="page element type: the workload's, or FP8 E4M3 codes with "
                          "per-head (e4m3) or per-page (e4m3-page) scales")
+    ap.add_argument("--tables", choices=["shuffled", "identity"], default="shuffled",
+                    help="physical block ids: a seeded permutation of the pool, or the "
+                         "identity (each sequence's pages contiguous in memory)")
     ap.add_argument("--no-order", dest="order", action="store_false",
                     help="schedule sequences in batch order instead of longest first")
     ap.add_argument("--cpu-budget", type=float, default=12.0,
