@@ -17,14 +17,14 @@ static cudaError_t dispatch_mma_e4m3(const DecodeArgs& a, int head_dim, int bloc
     if (two) {
 #define PKV_MMA8_TWO(BS_, NH_)                                        \
     if (block_size == BS_ && nh == NH_)                               \
-        return launch_decode_mma_e4m3<T, 128, BS_, NH_, 2>(a, stream);
+        return launch_decode_mma_e4m3<T, 128, BS_, NH_, 2, NH_ == 8 ? 3 : 0>(a, stream);
         PKV_MMA8_TWO(16, 8) PKV_MMA8_TWO(16, 16) PKV_MMA8_TWO(32, 8) PKV_MMA8_TWO(32, 16)
         PKV_MMA8_TWO(64, 8) PKV_MMA8_TWO(64, 16)
 #undef PKV_MMA8_TWO
     }
 #define PKV_MMA8_CASE(D_, BS_, NH_)                                   \
     if (head_dim == D_ && block_size == BS_ && nh == NH_)             \
-        return launch_decode_mma_e4m3<T, D_, BS_, NH_>(a, stream);
+        return launch_decode_mma_e4m3<T, D_, BS_, NH_, 4, (D_ == 128 && NH_ == 8) ? 3 : 0>(a, stream);
 #define PKV_MMA8_NH(D_, BS_) PKV_MMA8_CASE(D_, BS_, 8) PKV_MMA8_CASE(D_, BS_, 16)
 #define PKV_MMA8_BS(D_) PKV_MMA8_NH(D_, 16) PKV_MMA8_NH(D_, 32) PKV_MMA8_NH(D_, 64)
     PKV_MMA8_BS(128)

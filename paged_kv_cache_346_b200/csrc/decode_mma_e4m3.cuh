@@ -93,10 +93,21 @@ __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) {
     return r;
 }
 
+// CTAs per SM the register allocation is held to.  8-head tiles at head_dim
+// 128 fit 128 registers without spills, so with 3-stage rings (whose shared
+// memory then also fits) four 4-warp or eight 2-warp CTAs share an SM: 16
+// warps instead of 12 to cover the issue latency of the conversions and the
+// softmax.  Otherwise three CTAs (8-head tiles) or one.
+template <int D, int NH, int NW, int STAGES_>
+struct E4m3MinBlocks {
+    static constexpr int value =
+        (D <= 128 && NH == 8) ? (D == 128 && STAGES_ == 3 ? 16 / NW : 3) : 1;
+};
+
 // PPB: a scale per page (a.scale_per_block), a compile-time choice so the
 // per-head path carries no per-slice scale code.
 template <typename T, int D, int BS, int NH, int NW, int STAGES_, bool PPB>
-__global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
+__global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::value)
     decode_mma_e4m3_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv) {
     using C = MmaE4m3Cfg<D, BS, NW, STAGES_>;
