@@ -62,7 +62,8 @@ struct MmaE4m3Cfg {
     static_assert(BS % 16 == 0 && D % 128 == 0, "16-token slices of 128-byte rows");
 
     static int smem_bytes(int partition_size) {
-        return 1024 + round_up(partition_size / BS * 4, 128) + 1024 + RING_BYTES;
+        // barriers, table slice, slack to the ring's 1 KB (swizzle atom) alignment
+        return 128 + round_up(partition_size / BS * 4, 128) + 1024 + RING_BYTES;
     }
 };
 
@@ -161,12 +162,13 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
     const int nslices = ntok > warp * 16 ? (ntok - warp * 16 + TILE - 1) / TILE : 0;
 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem_mma8);  // [NW][STAGES]
-    int32_t* s_tab = reinterpret_cast<int32_t*>(smem_mma8 + 1024);
+    static_assert(NW * STAGES * 8 <= 128, "barriers");
+    int32_t* s_tab = reinterpret_cast<int32_t*>(smem_mma8 + 128);
     unsigned char* s_kv;
     {
-        const uint32_t base = smem_u32(smem_mma8 + 1024 + round_up(P / BS * 4, 128));
+        const uint32_t base = smem_u32(smem_mma8 + 128 + round_up(P / BS * 4, 128));
         const uint32_t aligned = (base + 1023u) & ~1023u;  // 128-byte swizzle: 1 KB atoms
-        s_kv = smem_mma8 + 1024 + round_up(P / BS * 4, 128) + (aligned - base);
+        s_kv = smem_mma8 + 128 + round_up(P / BS * 4, 128) + (aligned - base);
     }
 
     table_hoist(a, b, t0 / BS, nblk, pf, s_tab, tid, NW * 32);
