@@ -3,13 +3,18 @@
 
 namespace pkv {
 
-// CTA shape: 2 warps (6 CTAs per SM) when the CTAs are many and short-lived
-// relative to their start-up -- one live head (MHA) or partitions of at most
-// 512 tokens; else 4 warps (3 CTAs per SM).  Measured on B200 (E4M3 pages,
-// head_dim 128, bs 16, per-warp rings of 4 stages): the 2-warp shape is 6 %
-// faster on the MHA layer and 10-15 % faster with 512-token partitions, equal
-// on the GQA batch and 11 % slower on long contexts with 2048-token
-// partitions.
+// CTA shape: 2 warps when the CTAs are many and short-lived relative to
+// their start-up -- one live head (MHA) or partitions of at most 512 tokens;
+// else 4 warps.  Measured on B200 (E4M3 pages, head_dim 128, bs 16, per-warp
+// rings of 4 stages, 12 warps per SM): the 2-warp shape is 6 % faster on the
+// MHA layer and 10-15 % faster with 512-token partitions, and on the GQA
+// batch with 4096-token partitions 26 % slower (its longest partitions, at
+// half the warps each, become the tail).
+//
+// 8-head tiles at head_dim 128 take 3-stage rings and 128 registers, so
+// eight 2-warp or four 4-warp CTAs share an SM (16 warps): 1-9 % faster than
+// 4-stage rings at 12 warps per SM, by workload.  16-head tiles and head_dim
+// 256 keep 4 stages.
 template <typename T>
 static cudaError_t dispatch_mma_e4m3(const DecodeArgs& a, int head_dim, int block_size, int nh,
                                      cudaStream_t stream) {
