@@ -98,7 +98,7 @@ PKV_API const char* pkv_status_string(int status);
 /* ABI version: major * 10000 + minor * 100 + patch. */
 PKV_API int pkv_version(void);
 
-/* 1 if this build of the library contains decode kernel `kernel`, else 0. */
+/* 1 if the library was compiled with decode kernel `kernel`, else 0. */
 PKV_API int pkv_decode_has_kernel(pkv_kernel kernel);
 
 /*
