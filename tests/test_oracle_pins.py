@@ -141,6 +141,25 @@ def _tiny(seed=0, lens=(1, 7, 16, 33), H=4, Hkv=4, D=64, bs=16, pool=16, dtype="
     return make_decode_inputs(cfg, seed)
 
 
+def test_identity_tables_are_contiguous_runs():
+    """--tables identity: each sequence's pages are one contiguous run of the
+    pool, in logical order, sequences one after another; the shuffled pool
+    holds the same block counts as a permutation of those ids."""
+    cfg = DecodeConfig("t", 5, 4, 4, 64, 16, "f32", ("fixed", (1, 7, 16, 33, 48)),
+                       pool=("fixed", 24))
+    ident = make_decode_inputs(cfg, 3, shuffle=False)
+    shuf = make_decode_inputs(cfg, 3)
+    nb = [(L + 15) // 16 for L in (1, 7, 16, 33, 48)]
+    start = 0
+    for b, n in enumerate(nb):
+        assert ident.block_tables[b, :n].tolist() == list(range(start, start + n))
+        assert (ident.block_tables[b, n:] == -1).all()
+        assert ((shuf.block_tables[b, :n] >= 0).all() and (shuf.block_tables[b, n:] == -1).all())
+        start += n
+    used = shuf.block_tables[shuf.block_tables >= 0]
+    assert len(set(used.tolist())) == sum(nb)
+
+
 def test_single_token_returns_v_exactly():
     inp = _tiny(lens=(1, 1, 1))
     out = oracle.paged_decode_inputs(inp)
