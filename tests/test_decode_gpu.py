@@ -67,15 +67,20 @@ def test_head_dims_and_block_sizes(dtype, D, bs):
             assert_close(got, ref, dtype, f"{dtype} D={D} bs={bs} P={P} kernel={kern}")
 
 
-@pytest.mark.parametrize("G", [3, 5, 6, 16])
-def test_uneven_groups(G):
-    cfg = _cfg("bf16", 2 * G, 2, 128, 16, (5, 77, 600))
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("G", [3, 5, 6, 7, 9, 12, 16])
+def test_uneven_groups(dtype, G):
+    """Groups that fill an 8-head tile (3-7) or a 16-head tile (9, 12) only in
+    part: the heads past the group are zero q rows of the tile and are never
+    stored; split and unsplit."""
+    cfg = _cfg(dtype, 2 * G, 2, 128, 16, (5, 77, 600))
     inp = make_decode_inputs(cfg, seed=20 + G)
     ref = oracle.paged_decode_inputs(inp)
     dev = DeviceInputs(inp)
-    for kern in _kernels_for("bf16", G):
-        got = to_f64(dev.decode(kernel=kern))
-        assert_close(got, ref, "bf16", f"G={G} kernel={kern}")
+    for kern in _kernels_for(dtype, G):
+        for P in (0, 64):
+            got = to_f64(dev.decode(partition_size=P, kernel=kern))
+            assert_close(got, ref, dtype, f"{dtype} G={G} P={P} kernel={kern}")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])

@@ -314,6 +314,24 @@ def test_append_e4m3_per_page_bit_exact(dtype):
     assert np.array_equal(dV.view(torch.uint8).cpu().numpy(), V)
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("G", [5, 7, 9, 12])
+@pytest.mark.parametrize("per_page", [False, True])
+def test_decode_e4m3_partial_head_tiles(dtype, G, per_page):
+    """Groups that fill an 8-head tile (5, 7) or a 16-head tile (9, 12) only in
+    part: the heads past the group are zero q columns (rows) of the tile and
+    are never stored; split and unsplit, per-head and per-page scales."""
+    cfg = _cfg(dtype, 2 * G, 2, 128, 16, RAGGED)
+    inp = make_decode_inputs(cfg, seed=140 + G)
+    dev = E4M3Inputs(inp, seed=140 + G, per_page=per_page)
+    ref = dev.oracle()
+    for kern in KERNELS:
+        for P in (0, 64):
+            got = to_f64(dev.decode(partition_size=P, fill_out=5.0, kernel=kern))
+            assert_close(got, ref, dtype,
+                         f"e4m3 {dtype} G={G} per_page={per_page} P={P} kernel={kern}")
+
+
 @pytest.mark.parametrize("G", [1, 4, 8])
 @pytest.mark.parametrize("partition", [0, 64])
 def test_decode_e4m3_per_page_scales(G, partition):
