@@ -130,9 +130,10 @@ PKV_API size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_
  * compute as if contiguous).  A sequence with length 0 gets a zero row.
  *
  * The context of each sequence is cut into partitions of `partition_size`
- * tokens; one CTA takes one (sequence, KV head, partition) with all the query
- * heads of that KV head's group; sequences longer than one partition are
- * merged by a log-sum-exp reduce over the workspace.  Accumulation is float32;
+ * tokens; one CTA takes one (sequence, KV head, partition) with a tile of
+ * that KV head's query heads (up to 4 on the CUDA cores, 8 or 16 on the
+ * tensor cores); sequences longer than one partition are merged by a
+ * log-sum-exp reduce over the workspace.  Accumulation is float32;
  * `out` is written in `dtype` (round to nearest even).
  *
  * Arguments:
