@@ -29,6 +29,21 @@ def test_every_declared_symbol_is_exported():
     assert names == set(b.SIGNATURES), names ^ set(b.SIGNATURES)
 
 
+def test_header_constants_match_the_binding():
+    """Every #define PKV_* number in include/*.h has the binding's value."""
+    found = {}
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        for name, val in re.findall(r"^#define\s+(PKV_\w+)\s+\(?(\d+)u?", open(h).read(),
+                                    flags=re.M):
+            found[name] = int(val)
+    assert {"PKV_DEV_BAD_BLOCK", "PKV_DEV_TIMEOUT", "PKV_DEV_DRAIN_TIMEOUT"} <= set(found)
+    for name, val in found.items():
+        if name == "PKV_STATIC_WORKSPACE_BYTES":
+            continue   # an expression, checked below
+        assert getattr(b, name) == val, name
+    assert b.PKV_STATIC_WORKSPACE_BYTES == 64 * 1024 * 1024
+
+
 def test_status_strings_and_version():
     assert b.lib.pkv_status_string(0) == b"ok"
     assert b.lib.pkv_status_string(-2) == b"no free block"
