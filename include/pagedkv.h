@@ -91,6 +91,18 @@ typedef enum { PKV_KERNEL_AUTO = 0, PKV_KERNEL_SIMT = 1, PKV_KERNEL_MMA = 2 } pk
 #define PKV_DEV_BAD_SLOT 4u     /* a slot at or past num_blocks * block_size */
 #define PKV_DEV_TIMEOUT 8u      /* a bounded wait inside a kernel gave up */
 #define PKV_DEV_BAD_ORDER 16u   /* a seq_order entry outside [0, num_seqs) */
+#define PKV_DEV_DRAIN_TIMEOUT 32u /* after a wait gave up, a copy still had not landed
+                                     when the kernel's block left (see below) */
+#define PKV_DEV_BAD_GROUP 64u   /* a shared-prefix group whose members disagree
+                                   (prefix length, table entries) */
+/*
+ * After PKV_DEV_TIMEOUT the outputs of that call are lost (the blocks whose
+ * wait gave up wrote nothing).  With PKV_DEV_DRAIN_TIMEOUT as well, a page
+ * copy may have landed in shared memory after its block left, i.e. in a
+ * later block's: treat every result computed on the device since the flag
+ * was last cleared as lost, this call's and those of kernels that ran beside
+ * it.  Neither happens with valid inputs on a healthy device.
+ */
 
 /* Name of a status code. */
 PKV_API const char* pkv_status_string(int status);
@@ -189,12 +201,16 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
  * tensor-core kernel (AUTO for groups of at most 16 heads) multiplies fp16
  * operands with fp32 accumulation: q enters it scaled by a power of two that
  * puts max |q| of the CTA's heads in [2^14, 2^15) (exact unless an element
- * falls below the fp16 normal range there), P is rounded to fp16, and the
- * logits are multiplied by scale * k_scale (and the power of two) in fp32.
+ * falls below the fp16 normal range there), each softmax weight p enters as
+ * two fp16 terms, hi = fp16(p) and lo = fp16(p - hi) (about 22 significant
+ * bits, so the weights' rounding stays far below the fp16 / bf16 output
+ * tolerance whatever the values' magnitudes), and the logits are multiplied
+ * by scale * k_scale (and the power of two) in fp32.
  * The CUDA-core kernel works in fp32 throughout, k_scale folded into q and
  * v_scale into the accumulator (per page: into that page's logits and
  * weights); the tensor-core kernel applies a page's v_scale in fp32 to that
- * page's P.V product, so P stays an fp16 value at most 256.
+ * page's P.V product, so P stays an fp16 value at most 256 whatever the
+ * scales.
  *
  * Arguments as pkv_paged_attention_decode, plus:
  *   k_cache, v_cache: device E4M3 codes [num_blocks, Hkv, block_size, head_dim].
@@ -238,9 +254,10 @@ PKV_API int pkv_paged_attention_decode_e4m3(
  *     more scratch than that (pkv_decode_workspace_size(...) >
  *     PKV_STATIC_WORKSPACE_BYTES), e.g. far longer contexts or bigger
  *     batches; use pkv_paged_attention_decode with a caller workspace then.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and keeps it; make that
- *     first call before any stream capture begins.
+ *   - The first call in a CUDA context (normally a device's primary context)
+ *     looks up the array's device address there (cudaGetSymbolAddress, with
+ *     that context current) and keeps it for that context; make that first
+ *     call before any stream capture begins.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents.  Nothing in it needs to start at zero, but calls that can
  *     overlap on the GPU (different streams, no ordering between them) race
@@ -253,6 +270,92 @@ PKV_API int pkv_paged_attention_decode_static_ws(
     int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
     int sliding_window, pkv_dtype dtype, int partition_size, pkv_kernel kernel,
     pkv_stream_t stream);
+
+/* Largest shared-prefix group (sequences) of the shared-prefix decode. */
+#define PKV_MAX_PREFIX_GROUP 64
+
+/*
+ * Shared-prefix decode: pkv_paged_attention_decode's result, computed so that
+ * a prefix of blocks held by several sequences is read from memory once for
+ * all of them.  Sequences that hold the same physical blocks for their first
+ * S tokens share those keys and values: parallel samples forked from one
+ * prompt keep the prompt's blocks until they write into them
+ * ("pagedattention vllm" §Copy-on-Write Sharing), and requests that hit the
+ * same cached prompt blocks hold those (§Advanced Features, prefix caching).
+ *   - A group is up to PKV_MAX_PREFIX_GROUP sequences whose tables agree on
+ *     their first S / block_size entries (S a positive multiple of
+ *     block_size, at most each member's length); seq_prefix_len[b] = S for
+ *     its members, 0 for sequences in no group (pkv_decode_prefix_groups
+ *     finds the groups of a batch from its tables).
+ *   - The group pass runs on the tensor cores: one CTA per (prefix partition,
+ *     KV head, chunk of up to 16 rows) of a group, whose rows are the
+ *     members' query heads of that KV head, so each prefix page is read once
+ *     and feeds every member's heads, as a query group shares its KV head.
+ *   - The regular pass takes tokens [S, L_b) of every sequence ([0, L_b)
+ *     outside groups) with the usual kernel choice; the log-sum-exp reduce
+ *     merges the prefix's partial results with the rest's.
+ * The summation order differs from pkv_paged_attention_decode's, so results
+ * agree within rounding, not bit for bit.
+ *
+ * Arguments as pkv_paged_attention_decode (dtype PKV_F16 or PKV_BF16,
+ * sliding_window 0, query groups of at most 16 heads per KV head), plus:
+ *   seq_prefix_len: device int32 [num_seqs].
+ *   group_members: device int32 [num_groups][max_group_size]: batch indices
+ *       of each group's members, -1 after the last; a sequence is in at most
+ *       one group.  May be NULL when num_groups is 0.
+ *   num_groups >= 0; 1 <= max_group_size <= PKV_MAX_PREFIX_GROUP.
+ *   max_prefix_len: host-side bound of seq_prefix_len, a multiple of
+ *       block_size, <= max_context_len.
+ *   workspace: pkv_decode_prefix_groups_workspace_size(...) bytes, 16-byte
+ *       aligned (NULL when that is 0).
+ * A member whose prefix length differs from its group's first member's, a
+ * member whose table differs from the first member's over the prefix, or a
+ * prefix that is not whole blocks of its sequence sets PKV_DEV_BAD_GROUP
+ * (results unspecified); a sequence with seq_prefix_len > 0 that is in no
+ * group is not detected (its result is unspecified).
+ * Returns PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED or PKV_ECUDA.
+ */
+PKV_API int pkv_paged_attention_decode_prefix_groups(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* seq_order,
+    const int32_t* seq_prefix_len, const int32_t* group_members, int num_groups,
+    int max_group_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+    int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len,
+    int max_prefix_len, float scale, pkv_dtype dtype, int partition_size, void* workspace,
+    size_t workspace_bytes, pkv_kernel kernel, pkv_stream_t stream);
+
+/*
+ * Workspace bytes of pkv_paged_attention_decode_prefix_groups: float32
+ * partial results of ceil(max_prefix_len / P) prefix partitions and
+ * ceil(max_context_len / P) further partitions per (sequence, query head);
+ * partition_size 0 = pkv_decode_default_partition(num_seqs, num_kv_heads,
+ * max_context_len).  0 when no row needs a merge; 0 for invalid sizes.
+ */
+PKV_API size_t pkv_decode_prefix_groups_workspace_size(int num_seqs, int num_q_heads,
+                                                       int num_kv_heads, int head_dim,
+                                                       int max_context_len, int max_prefix_len,
+                                                       int partition_size);
+
+/*
+ * Host helper: the shared-prefix groups of a batch, from its host block
+ * tables and lengths.  Sequences are bucketed by the physical block of their
+ * first full block; each bucket, in batch order, is cut into groups of at
+ * most max_group_size (2 .. PKV_MAX_PREFIX_GROUP) members, and a group's
+ * prefix is the longest run of table entries all its members share over
+ * their full blocks.  Groups whose prefix has fewer than min_prefix_blocks
+ * (>= 1) blocks, and single sequences, are left out.
+ *   seq_prefix_len: [num_seqs] out: the prefix tokens (0 outside groups).
+ *   group_members: [group_capacity][max_group_size] out, -1 padded; a
+ *       capacity of num_seqs / 2 always suffices.
+ *   *num_groups: out.
+ * Returns PKV_OK, PKV_EINVAL or PKV_EBOUNDS (capacity too small; the outputs
+ * are then incomplete).
+ */
+PKV_API int pkv_decode_prefix_groups(const int32_t* block_tables, const int32_t* context_lens,
+                                     int num_seqs, int max_blocks_per_seq, int block_size,
+                                     int max_group_size, int min_prefix_blocks,
+                                     int32_t* seq_prefix_len, int32_t* group_members,
+                                     int group_capacity, int* num_groups);
 
 /*
  * Host helper: order_out[0..n) = the sequence indices sorted by decreasing

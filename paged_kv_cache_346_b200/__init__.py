@@ -20,8 +20,9 @@ import torch
 
 from . import _binding as _b
 from ._binding import (PKV_BF16, PKV_E4M3, PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD_ORDER,
-                       PKV_DEV_BAD_SLOT, PKV_DEV_TIMEOUT, PKV_F16, PKV_F32, PKV_KERNEL_AUTO, PKV_KERNEL_MMA,
-                       PKV_KERNEL_SIMT, PagedKVError, check, lib)
+                       PKV_DEV_BAD_GROUP, PKV_DEV_BAD_SLOT, PKV_DEV_DRAIN_TIMEOUT, PKV_DEV_TIMEOUT,
+                       PKV_F16, PKV_F32,
+                       PKV_KERNEL_AUTO, PKV_KERNEL_MMA, PKV_KERNEL_SIMT, PagedKVError, check, lib)
 
 __all__ = [
     "pkv_paged_attention_decode", "pkv_decode_workspace_size", "pkv_decode_has_kernel",
@@ -29,8 +30,11 @@ __all__ = [
     "pkv_kv_cache_append", "pkv_copy_blocks", "pkv_device_status", "BlockAllocator",
     "PagedKVError", "lib", "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_KERNEL_AUTO",
     "PKV_KERNEL_SIMT", "PKV_KERNEL_MMA", "PKV_DEV_BAD_BLOCK", "PKV_DEV_BAD_LEN",
-    "PKV_DEV_BAD_SLOT", "PKV_DEV_TIMEOUT", "PKV_DEV_BAD_ORDER", "torch_dtype_code",
+    "PKV_DEV_BAD_SLOT", "PKV_DEV_TIMEOUT", "PKV_DEV_BAD_ORDER", "PKV_DEV_DRAIN_TIMEOUT",
+    "torch_dtype_code",
     "pkv_decode_schedule_order", "pkv_paged_attention_decode_e4m3", "pkv_kv_cache_append_e4m3",
+    "pkv_paged_attention_decode_prefix_groups", "pkv_decode_prefix_groups",
+    "pkv_decode_prefix_groups_workspace_size", "PKV_DEV_BAD_GROUP",
     "PKV_E4M3", "pkv_debug_wait_timeout",
 ]
 
@@ -198,6 +202,82 @@ def pkv_paged_attention_decode_static_ws(out: torch.Tensor, q: torch.Tensor,
         int(partition_size), int(kernel), _stream(stream)),
         f"pkv_paged_attention_decode_static_ws (scratch limit "
         f"{_b.PKV_STATIC_WORKSPACE_BYTES} bytes)")
+    return out
+
+
+def pkv_decode_prefix_groups(block_tables, context_lens, block_size: int,
+                             max_group_size: int = 16, min_prefix_blocks: int = 1):
+    """Host arrays: the shared-prefix groups of a batch (pkv_decode_prefix_groups
+    in pagedkv.h).  -> (seq_prefix_len int32 [B], group_members int32
+    [num_groups, max_group_size], -1 padded)"""
+    import numpy as np
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    B = lens.size
+    if bt.ndim != 2 or bt.shape[0] != B:
+        raise PagedKVError(_b.PKV_EINVAL, "block_tables must be [num_seqs, max_blocks]")
+    spl = np.zeros(B, dtype=np.int32)
+    cap = max(B // 2, 1)
+    members = np.full((cap, max_group_size), -1, dtype=np.int32)
+    ng = ctypes.c_int(0)
+    check(lib.pkv_decode_prefix_groups(bt.ctypes.data if B else None,
+                                       lens.ctypes.data if B else None, B, bt.shape[1],
+                                       block_size, max_group_size, min_prefix_blocks,
+                                       spl.ctypes.data, members.ctypes.data, cap,
+                                       ctypes.byref(ng)), "pkv_decode_prefix_groups")
+    return spl, members[:ng.value].copy()
+
+
+def pkv_decode_prefix_groups_workspace_size(num_seqs: int, num_q_heads: int, num_kv_heads: int,
+                                            head_dim: int, max_context_len: int,
+                                            max_prefix_len: int, partition_size: int = 0) -> int:
+    return int(lib.pkv_decode_prefix_groups_workspace_size(
+        num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, max_prefix_len,
+        partition_size))
+
+
+def pkv_paged_attention_decode_prefix_groups(
+        out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+        block_tables: torch.Tensor, context_lens: torch.Tensor, seq_prefix_len: torch.Tensor,
+        group_members: torch.Tensor, scale: float, block_size: int, max_context_len: int,
+        max_prefix_len: int, *, partition_size: int = 0,
+        workspace: torch.Tensor | None = None, seq_order: torch.Tensor | None = None,
+        kernel: int = PKV_KERNEL_AUTO, stream=None) -> torch.Tensor:
+    """out [B, Hq, D] <- paged decode attention with shared prefixes read once
+    per group (pkv_paged_attention_decode_prefix_groups in pagedkv.h).
+    seq_prefix_len int32 [B] and group_members int32 [num_groups, max_group_size]
+    on the device (pkv_decode_prefix_groups builds them on the host);
+    workspace: pkv_decode_prefix_groups_workspace_size(...) bytes."""
+    for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+                 (block_tables, "block_tables"), (context_lens, "context_lens"),
+                 (seq_prefix_len, "seq_prefix_len"), (group_members, "group_members")):
+        _dev(t, n)
+    if seq_order is not None:
+        _dev(seq_order, "seq_order")
+    if (block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32 or
+            seq_prefix_len.dtype != torch.int32 or group_members.dtype != torch.int32):
+        raise PagedKVError(_b.PKV_EINVAL, "tables, lengths and groups must be int32")
+    if not (q.dtype == out.dtype == k_cache.dtype == v_cache.dtype):
+        raise PagedKVError(_b.PKV_EINVAL, "q, out, k_cache, v_cache must share a dtype")
+    B, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    if (D2 != D or bs != block_size or tuple(out.shape) != (B, Hq, D) or
+            tuple(v_cache.shape) != tuple(k_cache.shape) or block_tables.shape[0] != B or
+            context_lens.shape[0] != B or seq_prefix_len.shape[0] != B or
+            group_members.dim() != 2):
+        raise PagedKVError(_b.PKV_EINVAL, "shape mismatch")
+    ng, mgs = group_members.shape
+    ws_bytes = 0
+    if workspace is not None:
+        _dev(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    check(lib.pkv_paged_attention_decode_prefix_groups(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), _ptr(seq_order), _ptr(seq_prefix_len),
+        _ptr(group_members) if ng else None, ng, max(mgs, 1), B, Hq, Hkv, D, bs,
+        block_tables.shape[1], N, int(max_context_len), int(max_prefix_len), float(scale),
+        torch_dtype_code(q.dtype), int(partition_size), _ptr(workspace), ws_bytes, int(kernel),
+        _stream(stream)), "pkv_paged_attention_decode_prefix_groups")
     return out
 
 

@@ -5,10 +5,15 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <mutex>
+
+#include <cuda.h>
 
 #include <nvtx3/nvToolsExt.h>
 
 #include "cache_ops.cuh"
+#include "context_cache.h"
+#include "decode_request.h"
 #include "decode_dispatch.cuh"
 #include "decode_mma.cuh"
 #include "decode_mma_e4m3.cuh"
@@ -27,25 +32,48 @@ struct NvtxRange {
 };
 
 namespace {
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+std::once_flag g_ctx_once;
+}  // namespace
 
-constexpr int kMaxDevices = 64;
-std::atomic<unsigned int*> g_status_ptr[kMaxDevices];
-
-// Device address of the status word on the current device, looked up once
-// per device (the host-side symbol is only a handle, never a device address).
-cudaError_t status_word(unsigned int** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    unsigned int* p = g_status_ptr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        e = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_status_word);
-        if (e != cudaSuccess) return e;
-        g_status_ptr[dev].store(p, std::memory_order_release);
-    }
-    *out = p;
+cudaError_t current_context_id(unsigned long long* id) {
+    std::call_once(g_ctx_once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f);
+    });
+    if (!g_ctx_get_current || !g_ctx_get_id) return cudaErrorNotSupported;
+    CUcontext c = nullptr;
+    if (g_ctx_get_current(&c) != CUDA_SUCCESS) return cudaErrorUnknown;
+    *id = 0;
+    if (c && g_ctx_get_id(c, id) != CUDA_SUCCESS) return cudaErrorUnknown;
     return cudaSuccess;
+}
+
+namespace {
+
+PerContext g_status_addr;
+
+// Device address of the status word in the current context, looked up once
+// per context (the host-side symbol is only a handle, never a device address).
+cudaError_t status_word(unsigned int** out) {
+    void* p = nullptr;
+    const cudaError_t e = per_context_value(g_status_addr, &p, [](void** o) {
+        return cudaGetSymbolAddress(o, g_status_word);
+    });
+    *out = static_cast<unsigned int*>(p);
+    return e;
 }
 
 int elem_size(pkv_dtype dt) {
@@ -93,122 +121,219 @@ bool device_view(const void* p, void** out) {
 constexpr int kNumSMs = 148;
 
 
-// The decode behind both entry points.  e4m3: the pages hold E4M3 codes with
-// per-KV-head scales and dtype is the type of q and out.
-int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
-                const float* k_scale, const float* v_scale, int scale_per_block, bool e4m3,
-                const int32_t* block_tables, const int32_t* context_lens,
-                const int32_t* seq_order, int num_seqs, int num_q_heads, int num_kv_heads,
-                int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
-                int max_context_len, float scale, int sliding_window, pkv_dtype dtype,
-                int partition_size, void* workspace, size_t workspace_bytes, pkv_kernel kernel,
-                pkv_stream_t stream) {
-    // ---- host-side checks (nothing has been launched if these fail)
-    const int es = elem_size(dtype);
-    if (dtype == PKV_E4M3 || (e4m3 && dtype == PKV_F32)) return PKV_EINVAL;
-    if (es == 0 || num_seqs < 0 || num_seqs > 65535 || num_q_heads <= 0 || num_kv_heads <= 0 ||
-        num_q_heads % num_kv_heads != 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
-        max_context_len < 0 || (int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size ||
-        !std::isfinite(scale) || sliding_window < 0 || partition_size < 0 ||
-        (partition_size != 0 && (partition_size % 64 != 0 || partition_size > 8192)))
+}  // namespace
+
+int plan_decode(const DecodeRequest& r, DecodePlan* plan) {
+    const int es = elem_size(r.dtype);
+    if (r.dtype == PKV_E4M3 || (r.e4m3 && r.dtype == PKV_F32)) return PKV_EINVAL;
+    if (es == 0 || r.num_seqs < 0 || r.num_seqs > 65535 || r.num_q_heads <= 0 ||
+        r.num_kv_heads <= 0 || r.num_q_heads % r.num_kv_heads != 0 ||
+        r.max_blocks_per_seq <= 0 || r.num_blocks <= 0 || r.max_context_len < 0 ||
+        (int64_t)r.max_context_len > (int64_t)r.max_blocks_per_seq * r.block_size ||
+        !std::isfinite(r.scale) || r.sliding_window < 0 || r.partition_size < 0 ||
+        (r.partition_size != 0 && (r.partition_size % 64 != 0 || r.partition_size > 8192)))
         return PKV_EINVAL;
-    if (kernel != PKV_KERNEL_AUTO && kernel != PKV_KERNEL_SIMT && kernel != PKV_KERNEL_MMA)
+    if (r.kernel != PKV_KERNEL_AUTO && r.kernel != PKV_KERNEL_SIMT && r.kernel != PKV_KERNEL_MMA)
         return PKV_EINVAL;
-    if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PKV_EUNSUPPORTED;
-    if (block_size != 16 && block_size != 32 && block_size != 64) return PKV_EUNSUPPORTED;
-    if (dtype == PKV_F32 && head_dim == 256) return PKV_EUNSUPPORTED;
-    if (e4m3 && head_dim == 64) return PKV_EUNSUPPORTED;
-    if (num_seqs == 0) return PKV_OK;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_EINVAL;
-    if (e4m3 && (!k_scale || !v_scale || (scale_per_block != 0 && scale_per_block != 1)))
+    if (r.head_dim != 64 && r.head_dim != 128 && r.head_dim != 256) return PKV_EUNSUPPORTED;
+    if (r.block_size != 16 && r.block_size != 32 && r.block_size != 64) return PKV_EUNSUPPORTED;
+    if (r.dtype == PKV_F32 && r.head_dim == 256) return PKV_EUNSUPPORTED;
+    if (r.e4m3 && r.head_dim == 64) return PKV_EUNSUPPORTED;
+    plan->empty = r.num_seqs == 0;
+    if (plan->empty) return PKV_OK;
+    if (!r.out || !r.q || !r.k_cache || !r.v_cache || !r.block_tables || !r.context_lens)
         return PKV_EINVAL;
-    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    if (r.e4m3 && (!r.k_scale || !r.v_scale || (r.scale_per_block != 0 && r.scale_per_block != 1)))
+        return PKV_EINVAL;
+    if (!aligned16(r.out) || !aligned16(r.q) || !aligned16(r.k_cache) || !aligned16(r.v_cache))
         return PKV_EINVAL;
 
-    const int G = num_q_heads / num_kv_heads;
+    const int G = r.num_q_heads / r.num_kv_heads;
     // longest span a sequence attends to: with a window, at most the window
     // plus the part of its first block ahead of it
-    const int span = sliding_window > 0
-                         ? (int)std::min<int64_t>(max_context_len,
-                                                  (int64_t)sliding_window + block_size - 1)
-                         : max_context_len;
-    const int P = partition_size ? partition_size
-                                 : pkv_decode_default_partition(num_seqs, num_kv_heads, span);
-    const int np = span > 0 ? ceil_div(span, P) : 1;
-    if (np > 1) {
-        const size_t need = pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads,
-                                                      head_dim, span, P);
-        if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PKV_EINVAL;
-    }
+    plan->span = r.sliding_window > 0
+                     ? (int)std::min<int64_t>(r.max_context_len,
+                                              (int64_t)r.sliding_window + r.block_size - 1)
+                     : r.max_context_len;
+    plan->partition_size = r.partition_size ? r.partition_size
+                                            : pkv_decode_default_partition(
+                                                  r.num_seqs, r.num_kv_heads, plan->span);
+    plan->max_partitions = plan->span > 0 ? ceil_div(plan->span, plan->partition_size) : 1;
+    plan->workspace_bytes =
+        plan->max_partitions > 1
+            ? pkv_decode_workspace_size(r.num_seqs, r.num_q_heads, r.num_kv_heads, r.head_dim,
+                                        plan->span, plan->partition_size)
+            : 0;
 
     // the tensor-core kernel addresses the pool as one 2-D tensor of
     // num_blocks * Hkv * block_size rows with 32-bit TMA coordinates
-    const bool mma_fits = dtype != PKV_F32 && G <= 16 &&
-                          (int64_t)num_blocks * num_kv_heads * block_size < (1ll << 31);
-    bool use_mma;
-    if (kernel == PKV_KERNEL_MMA) {
+    const bool mma_fits = r.dtype != PKV_F32 && G <= 16 &&
+                          (int64_t)r.num_blocks * r.num_kv_heads * r.block_size < (1ll << 31);
+    if (r.kernel == PKV_KERNEL_MMA) {
         if (!kMmaBuilt || !mma_fits) return PKV_EUNSUPPORTED;
-        use_mma = true;
-    } else if (kernel == PKV_KERNEL_SIMT) {
-        use_mma = false;
+        plan->use_mma = true;
+    } else if (r.kernel == PKV_KERNEL_SIMT) {
+        plan->use_mma = false;
     } else {
         // E4M3 pages: the tensor cores for every group size (the conversions
         // would bound the CUDA-core kernel below the memory roofline)
-        use_mma = kMmaBuilt && mma_fits && (G >= 4 || e4m3);
+        plan->use_mma = kMmaBuilt && mma_fits && (G >= 4 || r.e4m3);
     }
-    const int hg = use_mma ? (G <= 8 ? 8 : 16)
-                           : (G % 4 == 0 && !e4m3 ? 4 : (G % 2 == 0 ? 2 : 1));
-    const int head_chunks = (G + hg - 1) / hg;
-    if ((int64_t)num_kv_heads * head_chunks > 65535) return PKV_EUNSUPPORTED;
+    plan->heads_per_cta = plan->use_mma ? (G <= 8 ? 8 : 16)
+                                        : (G % 4 == 0 && !r.e4m3 ? 4 : (G % 2 == 0 ? 2 : 1));
+    plan->head_chunks = (G + plan->heads_per_cta - 1) / plan->heads_per_cta;
+    if ((int64_t)r.num_kv_heads * plan->head_chunks > 65535) return PKV_EUNSUPPORTED;
+    return PKV_OK;
+}
 
+namespace {
+
+// Kernel arguments of a planned decode whose workspace rows hold ws_slots
+// partial results.
+DecodeArgs decode_args(const DecodeRequest& r, const DecodePlan& plan, void* workspace,
+                       int ws_slots) {
     DecodeArgs a;
-    a.out = out;
-    a.q = q;
-    a.k_cache = k_cache;
-    a.v_cache = v_cache;
-    a.block_tables = block_tables;
-    a.context_lens = context_lens;
-    a.seq_order = seq_order;
-    a.k_scale = e4m3 ? k_scale : nullptr;
-    a.v_scale = e4m3 ? v_scale : nullptr;
-    a.scale_per_block = e4m3 ? scale_per_block : 0;
+    a.out = r.out;
+    a.q = r.q;
+    a.k_cache = r.k_cache;
+    a.v_cache = r.v_cache;
+    a.block_tables = r.block_tables;
+    a.context_lens = r.context_lens;
+    a.seq_order = r.seq_order;
+    a.k_scale = r.e4m3 ? r.k_scale : nullptr;
+    a.v_scale = r.e4m3 ? r.v_scale : nullptr;
+    a.scale_per_block = r.e4m3 ? r.scale_per_block : 0;
+    a.seq_start = nullptr;
+    a.group_members = nullptr;
+    a.group_stride = 0;
+    a.ws_slots = ws_slots;
     a.ws_o = static_cast<float*>(workspace);
-    a.ws_ml = np > 1 ? a.ws_o + (int64_t)num_seqs * num_q_heads * np * head_dim : nullptr;
-    a.num_seqs = num_seqs;
-    a.num_q_heads = num_q_heads;
-    a.num_kv_heads = num_kv_heads;
-    a.group = G;
-    a.head_chunks = head_chunks;
-    a.max_blocks_per_seq = max_blocks_per_seq;
-    a.num_blocks = num_blocks;
-    a.max_tokens = max_blocks_per_seq * block_size;
-    a.partition_size = P;
-    a.max_partitions = np;
-    a.block_size = block_size;
-    a.window = sliding_window;
-    a.scale_log2 = scale * 1.4426950408889634f;
-    if (status_word(&a.status) != cudaSuccess) return PKV_ECUDA;
+    a.ws_ml = ws_slots > 1
+                  ? a.ws_o + (int64_t)r.num_seqs * r.num_q_heads * ws_slots * r.head_dim
+                  : nullptr;
+    a.num_seqs = r.num_seqs;
+    a.num_q_heads = r.num_q_heads;
+    a.num_kv_heads = r.num_kv_heads;
+    a.group = r.num_q_heads / r.num_kv_heads;
+    a.head_chunks = plan.head_chunks;
+    a.max_blocks_per_seq = r.max_blocks_per_seq;
+    a.num_blocks = r.num_blocks;
+    a.max_tokens = r.max_blocks_per_seq * r.block_size;
+    a.partition_size = plan.partition_size;
+    a.max_partitions = plan.max_partitions;
+    a.block_size = r.block_size;
+    a.window = r.sliding_window;
+    a.scale_log2 = r.scale * 1.4426950408889634f;
+    a.status = nullptr;
+    return a;
+}
 
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+// The partition kernel the plan chose (and the reduce when rows merge).
+int launch_planned(const DecodeRequest& r, const DecodePlan& plan, const DecodeArgs& a,
+                   cudaStream_t s) {
+    const int D = r.head_dim, bs = r.block_size, hg = plan.heads_per_cta;
     cudaError_t e;
-    if (e4m3 && use_mma) {
-        e = dtype == PKV_F16 ? decode_mma_e4m3_f16(a, head_dim, block_size, hg, s)
-                             : decode_mma_e4m3_bf16(a, head_dim, block_size, hg, s);
-    } else if (e4m3) {
-        e = dtype == PKV_F16 ? decode_simt_e4m3_f16(a, head_dim, block_size, hg, s)
-                             : decode_simt_e4m3_bf16(a, head_dim, block_size, hg, s);
-    } else if (use_mma) {
-        e = dtype == PKV_F16 ? decode_mma_f16(a, head_dim, block_size, hg, s)
-                             : decode_mma_bf16(a, head_dim, block_size, hg, s);
+    if (r.e4m3 && plan.use_mma) {
+        e = r.dtype == PKV_F16 ? decode_mma_e4m3_f16(a, D, bs, hg, s)
+                               : decode_mma_e4m3_bf16(a, D, bs, hg, s);
+    } else if (r.e4m3) {
+        e = r.dtype == PKV_F16 ? decode_simt_e4m3_f16(a, D, bs, hg, s)
+                               : decode_simt_e4m3_bf16(a, D, bs, hg, s);
+    } else if (plan.use_mma) {
+        e = r.dtype == PKV_F16 ? decode_mma_f16(a, D, bs, hg, s) : decode_mma_bf16(a, D, bs, hg, s);
     } else {
-        switch (dtype) {
-            case PKV_F32: e = decode_simt_f32(a, head_dim, block_size, hg, s); break;
-            case PKV_F16: e = decode_simt_f16(a, head_dim, block_size, hg, s); break;
-            default: e = decode_simt_bf16(a, head_dim, block_size, hg, s); break;
+        switch (r.dtype) {
+            case PKV_F32: e = decode_simt_f32(a, D, bs, hg, s); break;
+            case PKV_F16: e = decode_simt_f16(a, D, bs, hg, s); break;
+            default: e = decode_simt_bf16(a, D, bs, hg, s); break;
         }
     }
     if (e == cudaErrorInvalidValue) return PKV_EUNSUPPORTED;
     return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+}  // namespace
+
+int run_decode(const DecodeRequest& r, const DecodePlan& plan, void* workspace,
+               size_t workspace_bytes, cudaStream_t s) {
+    if (plan.empty) return PKV_OK;
+    if (plan.workspace_bytes > 0 &&
+        (!workspace || workspace_bytes < plan.workspace_bytes || !aligned16(workspace)))
+        return PKV_EINVAL;
+    DecodeArgs a = decode_args(r, plan, workspace, plan.max_partitions);
+    if (status_word(&a.status) != cudaSuccess) return PKV_ECUDA;
+    return launch_planned(r, plan, a, s);
+}
+
+namespace {
+
+// Workspace slots per row of the shared-prefix decode: the prefix's
+// partitions, then the rest's.
+int prefix_slots(int max_prefix_len, int partition_size) {
+    return max_prefix_len > 0 ? ceil_div(max_prefix_len, partition_size) : 0;
+}
+
+int prefix_groups_impl(const DecodeRequest& r, const int32_t* seq_prefix_len,
+                       const int32_t* group_members, int num_groups, int max_group_size,
+                       int max_prefix_len, void* workspace, size_t workspace_bytes,
+                       cudaStream_t s) {
+    if (r.sliding_window != 0 || (r.dtype != PKV_F16 && r.dtype != PKV_BF16 &&
+                                  r.dtype != PKV_F32))
+        return PKV_EINVAL;
+    if (num_groups < 0 || num_groups > 65535 || max_group_size < 1 ||
+        max_group_size > PKV_MAX_PREFIX_GROUP || max_prefix_len < 0 ||
+        max_prefix_len % std::max(r.block_size, 1) != 0 || max_prefix_len > r.max_context_len)
+        return PKV_EINVAL;
+    DecodePlan plan;
+    int rc = plan_decode(r, &plan);
+    if (rc != PKV_OK || plan.empty) return rc;
+    if (r.dtype == PKV_F32) return PKV_EUNSUPPORTED;  // the group pass is fp16 / bf16
+    if (!seq_prefix_len || (num_groups > 0 && !group_members)) return PKV_EINVAL;
+    const int G = r.num_q_heads / r.num_kv_heads;
+    const int pslots = prefix_slots(max_prefix_len, plan.partition_size);
+    const int ws_slots = pslots + plan.max_partitions;
+    const size_t need = ws_slots > 1 ? (size_t)r.num_seqs * r.num_q_heads * ws_slots *
+                                           (r.head_dim + 2) * sizeof(float)
+                                     : 0;
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+        return PKV_EINVAL;
+    // the group pass: tiles of 8 or 16 (member, head) rows on the tensor cores
+    const bool groups = num_groups > 0 && pslots > 0;
+    const int rows = max_group_size * G;
+    const int nh = rows <= 8 ? 8 : 16;
+    const int chunks = ceil_div(rows, nh);
+    if (groups && (!kMmaBuilt || G > 16 ||
+                   (int64_t)r.num_blocks * r.num_kv_heads * r.block_size >= (1ll << 31) ||
+                   (int64_t)r.num_kv_heads * chunks > 65535))
+        return PKV_EUNSUPPORTED;
+
+    DecodeArgs a = decode_args(r, plan, workspace, ws_slots);
+    if (status_word(&a.status) != cudaSuccess) return PKV_ECUDA;
+    a.seq_start = seq_prefix_len;
+    if (groups) {
+        DecodeArgs ag = a;
+        ag.seq_order = nullptr;
+        ag.group_members = group_members;
+        ag.group_stride = max_group_size;
+        ag.head_chunks = chunks;
+        ag.max_partitions = pslots;
+        const cudaError_t e =
+            r.dtype == PKV_F16
+                ? decode_mma_groups_f16(ag, r.head_dim, r.block_size, nh, num_groups, s)
+                : decode_mma_groups_bf16(ag, r.head_dim, r.block_size, nh, num_groups, s);
+        if (e == cudaErrorInvalidValue) return PKV_EUNSUPPORTED;
+        if (e != cudaSuccess) return PKV_ECUDA;
+    }
+    return launch_planned(r, plan, a, s);
+}
+
+// The decode behind both caller-workspace entry points.
+int decode_impl(const DecodeRequest& r, void* workspace, size_t workspace_bytes,
+                pkv_stream_t stream) {
+    DecodePlan plan;
+    const int rc = plan_decode(r, &plan);
+    if (rc != PKV_OK) return rc;
+    return run_decode(r, plan, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -280,11 +405,11 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
                                int partition_size, void* workspace, size_t workspace_bytes,
                                pkv_kernel kernel, pkv_stream_t stream) {
     NvtxRange range("pkv_paged_attention_decode");
-    return pkv::decode_impl(out, q, k_cache, v_cache, nullptr, nullptr, 0, false, block_tables,
-                            context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
-                            head_dim, block_size, max_blocks_per_seq, num_blocks,
-                            max_context_len, scale, sliding_window, dtype, partition_size,
-                            workspace, workspace_bytes, kernel, stream);
+    const DecodeRequest r{out, q, k_cache, v_cache, nullptr, nullptr, 0, false, block_tables,
+                          context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
+                          head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
+                          scale, sliding_window, dtype, partition_size, kernel};
+    return pkv::decode_impl(r, workspace, workspace_bytes, stream);
 }
 
 int pkv_paged_attention_decode_e4m3(void* out, const void* q, const void* k_cache,
@@ -299,12 +424,45 @@ int pkv_paged_attention_decode_e4m3(void* out, const void* q, const void* k_cach
                                     size_t workspace_bytes, pkv_kernel kernel,
                                     pkv_stream_t stream) {
     NvtxRange range("pkv_paged_attention_decode_e4m3");
-    return pkv::decode_impl(out, q, k_cache, v_cache, k_scale, v_scale, scale_per_block, true,
-                            block_tables,
-                            context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
-                            head_dim, block_size, max_blocks_per_seq, num_blocks,
-                            max_context_len, scale, sliding_window, dtype, partition_size,
-                            workspace, workspace_bytes, kernel, stream);
+    const DecodeRequest r{out, q, k_cache, v_cache, k_scale, v_scale, scale_per_block, true,
+                          block_tables, context_lens, seq_order, num_seqs, num_q_heads,
+                          num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                          max_context_len, scale, sliding_window, dtype, partition_size, kernel};
+    return pkv::decode_impl(r, workspace, workspace_bytes, stream);
+}
+
+size_t pkv_decode_prefix_groups_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                               int head_dim, int max_context_len,
+                                               int max_prefix_len, int partition_size) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        max_context_len < 0 || max_prefix_len < 0 || max_prefix_len > max_context_len ||
+        partition_size < 0)
+        return 0;
+    const int p = partition_size ? partition_size
+                                 : pkv_decode_default_partition(num_seqs, num_kv_heads,
+                                                                max_context_len);
+    const int64_t slots = pkv::prefix_slots(max_prefix_len, p) +
+                          (max_context_len > 0 ? ceil_div(max_context_len, p) : 1);
+    if (slots <= 1) return 0;
+    return (size_t)num_seqs * num_q_heads * slots * (head_dim + 2) * sizeof(float);
+}
+
+int pkv_paged_attention_decode_prefix_groups(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* seq_order,
+    const int32_t* seq_prefix_len, const int32_t* group_members, int num_groups,
+    int max_group_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+    int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len,
+    int max_prefix_len, float scale, pkv_dtype dtype, int partition_size, void* workspace,
+    size_t workspace_bytes, pkv_kernel kernel, pkv_stream_t stream) {
+    NvtxRange range("pkv_paged_attention_decode_prefix_groups");
+    const DecodeRequest r{out, q, k_cache, v_cache, nullptr, nullptr, 0, false, block_tables,
+                          context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
+                          head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
+                          scale, 0, dtype, partition_size, kernel};
+    return pkv::prefix_groups_impl(r, seq_prefix_len, group_members, num_groups, max_group_size,
+                                   max_prefix_len, workspace, workspace_bytes,
+                                   reinterpret_cast<cudaStream_t>(stream));
 }
 
 int pkv_kv_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,

@@ -1,9 +1,9 @@
 // Arguments and the log-sum-exp reduce shared by both decode kernels.
 #pragma once
 
-#include <atomic>
 #include <cmath>
 
+#include "context_cache.h"
 #include "device_common.cuh"
 
 namespace pkv {
@@ -20,8 +20,13 @@ struct DecodeArgs {
     const int32_t* seq_order;     // [B] schedule order (CTA z takes sequence seq_order[z]), or null
     const float* k_scale;         // scales of E4M3 K / V pages, or null: [Hkv], or
     const float* v_scale;         // [num_blocks, Hkv] when scale_per_block
-    float* ws_o;                  // [B, Hq, max_partitions, D] partition outputs
-    float* ws_ml;                 // [B, Hq, max_partitions, 2] (m in log2 units, l)
+    // shared-prefix decode: tokens [0, seq_start[b]) of sequence b were
+    // attended by the group pass (whole blocks shared with the other members
+    // of its group); null = every sequence starts at token 0
+    const int32_t* seq_start;     // [B] or null
+    const int32_t* group_members; // [num_groups][group_stride] batch indices, -1 padded
+    float* ws_o;                  // [B, Hq, ws_slots, D] partial outputs (normalised)
+    float* ws_ml;                 // [B, Hq, ws_slots, 2] (m in log2 units, l)
     unsigned int* status;
     int num_seqs;
     int num_q_heads;
@@ -33,6 +38,8 @@ struct DecodeArgs {
     int max_tokens;               // max_blocks_per_seq * BS
     int partition_size;           // tokens per partition
     int max_partitions;           // grid.x = ceil(longest attended span / partition_size)
+    int ws_slots;                 // partial results per row in the workspace
+    int group_stride;             // group_members row length
     int block_size;
     int window;                   // sliding window in tokens, 0 = attend to the whole context
     int scale_per_block;          // E4M3 scales per (block, KV head) page
@@ -67,17 +74,35 @@ __device__ __forceinline__ int seq_len(const DecodeArgs& a, int b, bool report) 
 // max(0, L - W) ("pagedattention vllm" §Advanced Features: sliding-window
 // models keep only the recent blocks); the partitions then start at the
 // block holding lo (base), and the first lo - base tokens are masked.
+// With a shared prefix of S tokens (seq_start), the partitions cover [S, L)
+// and their partial results take workspace slots ceil(S / P) onwards, after
+// the group pass's slots of the prefix.
 struct Span {
-    int L;     // sequence length
-    int lo;    // first attended token
-    int base;  // first token of partition 0 (block aligned)
-    int np;    // partitions
+    int L;       // sequence length
+    int lo;      // first attended token
+    int base;    // first token of partition 0 (block aligned)
+    int np;      // partitions
+    int slot0;   // workspace slot of partition 0
+    bool direct; // one partial result in all: written straight to out
 };
 
 __device__ __forceinline__ Span seq_span(const DecodeArgs& a, int b, bool report) {
     Span sp;
     sp.L = seq_len(a, b, report);
     sp.lo = (a.window > 0 && sp.L > a.window) ? sp.L - a.window : 0;
+    sp.slot0 = 0;
+    if (a.seq_start) {
+        int st = a.seq_start[b];
+        // the prefix must be whole blocks of the sequence, within the slots
+        // the group pass has (ws_slots - max_partitions of them)
+        if (st < 0 || st > sp.L || st % a.block_size != 0 ||
+            (st + a.partition_size - 1) / a.partition_size > a.ws_slots - a.max_partitions) {
+            if (report) flag(a.status, PKV_DEV_BAD_GROUP);
+            st = 0;
+        }
+        sp.lo = max(sp.lo, st);
+        sp.slot0 = (st + a.partition_size - 1) / a.partition_size;
+    }
     sp.base = sp.lo - sp.lo % a.block_size;
     int n = (sp.L - sp.base + a.partition_size - 1) / a.partition_size;
     if (n > a.max_partitions) {
@@ -85,6 +110,30 @@ __device__ __forceinline__ Span seq_span(const DecodeArgs& a, int b, bool report
         n = a.max_partitions;
     }
     sp.np = n;
+    sp.direct = sp.slot0 == 0 && n <= 1;
+    return sp;
+}
+
+// The shared prefix of a group as the group pass cuts it: tokens [0, S),
+// S = seq_start of the group's first member b (whole blocks of b), in
+// partitions of partition_size whose partial results take workspace slots
+// 0, 1, ... of every member row.  A prefix that is not whole blocks of b or
+// needs more than max_partitions (the group pass's grid) is flagged and left
+// out (S = 0: the regular pass then takes the whole sequence).
+__device__ __forceinline__ Span group_span(const DecodeArgs& a, int b, bool report) {
+    Span sp;
+    const int L = seq_len(a, b, false);
+    int st = a.seq_start[b];
+    if (st < 0 || st > L || st % a.block_size != 0 ||
+        (st + a.partition_size - 1) / a.partition_size > a.max_partitions) {
+        if (report) flag(a.status, PKV_DEV_BAD_GROUP);
+        st = 0;
+    }
+    sp.L = st;
+    sp.lo = sp.base = 0;
+    sp.np = (st + a.partition_size - 1) / a.partition_size;
+    sp.slot0 = 0;
+    sp.direct = false;
     return sp;
 }
 
@@ -101,9 +150,9 @@ struct TablePrefetch {
 
 __device__ __forceinline__ TablePrefetch table_prefetch(const DecodeArgs& a, int b, int part,
                                                         int blocks_per_part, int tid) {
-    // (with a sliding window partition 0 starts at a block known only after
-    // the length is read: no early read then)
-    TablePrefetch pf{0, part == 0 && a.window == 0 && tid < blocks_per_part &&
+    // (with a sliding window or a shared prefix partition 0 starts at a
+    // block known only after the length is read: no early read then)
+    TablePrefetch pf{0, part == 0 && a.window == 0 && !a.seq_start && tid < blocks_per_part &&
                             tid < a.max_blocks_per_seq};
     if (pf.ok) pf.v = a.block_tables[(int64_t)b * a.max_blocks_per_seq + tid];
     return pf;
@@ -137,24 +186,25 @@ struct MergeArea {
 };
 
 // Merge NW parked warp states (acc rows, m, l in `red`, written and
-// synchronised by the caller) of nh heads and write the output rows (one
-// partition) or the partition's (m, l, o) to the workspace.  All threads of
-// the CTA take part.  Per head: M = max_w m_w, den = sum_w 2^(m_w - M) l_w,
-// o = sum_w (2^(m_w - M) / den) acc_w.
-template <typename T, int D, int NH, int NW>
-__device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float* red, int b,
-                                                      int h0, int nh, int part, int np, int tid,
-                                                      int nthreads) {
+// synchronised by the caller) of nh heads and write the output rows (direct:
+// the row's only partial result) or the partial (m, l, o) to workspace slot
+// `slot`.  Tile row hh is global row row_of(hh) = sequence * Hq + head.  All
+// threads of the CTA take part.  Per head: M = max_w m_w,
+// den = sum_w 2^(m_w - M) l_w, o = sum_w (2^(m_w - M) / den) acc_w.
+template <typename T, int D, int NH, int NW, typename RowOf>
+__device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float* red,
+                                                      RowOf row_of, int nh, int slot,
+                                                      bool direct, int tid, int nthreads) {
     using A = MergeArea<D, NH, NW>;
     float* red_m = red + NW * NH * A::RP;
     float* red_l = red_m + NW * NH;
     float* red_s = red_l + NW * NH;
-    const int64_t row0 = (int64_t)b * a.num_q_heads + h0;
     T* out = reinterpret_cast<T*>(a.out);
     if constexpr (NH == 1) {
         // one head: every thread folds the NW warp states for its elements
         // (measured faster than a serial scale step plus a barrier here)
         (void)red_s;
+        const int64_t row = row_of(0);
         for (int d = tid; d < D; d += nthreads) {
             float M = -INFINITY;
 #pragma unroll
@@ -166,10 +216,10 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float
                 num = fmaf(f, red[w * A::RP + d], num);
                 den = fmaf(f, red_l[w], den);
             }
-            if (np == 1) {
-                out[row0 * D + d] = Elem<T>::from_f32(num / den);
+            if (direct) {
+                out[row * D + d] = Elem<T>::from_f32(num / den);
             } else {
-                const int64_t pr = row0 * a.max_partitions + part;
+                const int64_t pr = row * a.ws_slots + slot;
                 a.ws_o[pr * D + d] = num / den;
                 if (d == 0) {
                     a.ws_ml[pr * 2] = M;
@@ -194,8 +244,8 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float
             const float inv = 1.f / den;
 #pragma unroll
             for (int w = 0; w < NW; ++w) red_s[w * NH + tid] = f[w] * inv;
-            if (np > 1) {
-                const int64_t pr = (row0 + tid) * a.max_partitions + part;
+            if (!direct && row_of(tid) >= 0) {
+                const int64_t pr = row_of(tid) * a.ws_slots + slot;
                 a.ws_ml[pr * 2] = M;
                 a.ws_ml[pr * 2 + 1] = den;
             }
@@ -203,14 +253,16 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float
         __syncthreads();
         for (int i = tid; i < nh * D; i += nthreads) {
             const int hh = i / D, d = i - hh * D;
+            const int64_t row = row_of(hh);  // < 0: a row the group pass skips
+            if (row < 0) continue;
             float o = 0.f;
 #pragma unroll
             for (int w = 0; w < NW; ++w)
                 o = fmaf(red_s[w * NH + hh], red[(w * NH + hh) * A::RP + d], o);
-            if (np == 1)
-                out[(row0 + hh) * D + d] = Elem<T>::from_f32(o);
+            if (direct)
+                out[row * D + d] = Elem<T>::from_f32(o);
             else
-                a.ws_o[((row0 + hh) * a.max_partitions + part) * D + d] = o;
+                a.ws_o[(row * a.ws_slots + slot) * D + d] = o;
         }
     }
 }
@@ -218,10 +270,11 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float
 // Merge the partitions of one (sequence, query head) row: with per-partition
 // maxima m_p (base-2 logits), sums l_p and normalised outputs o_p,
 //   M = max_p m_p,  w_p = l_p 2^(m_p - M),  out = sum_p w_p o_p / sum_p w_p.
-// One CTA of 128 threads per row; rows that fit one partition were written by
-// the decode kernel and are skipped.  Launched as a programmatic dependent of
-// the decode kernel: rows of one partition leave before the wait, during the
-// decode's tail; the others wait for the decode grid's writes before reading.
+// One CTA of 128 threads per row; rows with one partial result in all were
+// written by the decode kernel and are skipped.  Launched as a programmatic
+// dependent of the decode kernel: those rows leave before the wait, during
+// the decode's tail; the others wait for the decode grid's writes before
+// reading.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
     constexpr int NW = 4;
@@ -229,14 +282,15 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
     const int h = blockIdx.x;
     const int b = blockIdx.y;
     // the partition count depends only on the inputs, not on the decode
-    // grid's output: rows with one partition leave before the wait
-    const int np = seq_span(a, b, false).np;
-    if (np <= 1) return;
+    // grid's output: rows with one partial result leave before the wait
+    const Span sp = seq_span(a, b, false);
+    if (sp.direct) return;
+    const int np = sp.slot0 + sp.np;  // the group pass's slots, then this row's partitions
     pdl_wait_primary();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row = (int64_t)b * a.num_q_heads + h;
-    const float* ml = a.ws_ml + row * a.max_partitions * 2;
-    const float* o = a.ws_o + row * a.max_partitions * D;
+    const float* ml = a.ws_ml + row * a.ws_slots * 2;
+    const float* o = a.ws_o + row * a.ws_slots * D;
 
     __shared__ float s_max[NW];
     __shared__ float s_den[NW];
@@ -284,19 +338,17 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
     }
 }
 
-// Per-device "dynamic shared memory size set" bookkeeping for one kernel.
+// "Dynamic shared memory limit raised" bookkeeping for one kernel, per CUDA
+// context (the attribute belongs to the context's copy of the module).
 struct SmemAttr {
-    std::atomic<unsigned long long> done{0};
+    PerContext done;
     template <typename K>
     cudaError_t ensure(K kernel, int bytes) {
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e != cudaSuccess) return e;
-        const unsigned long long bit = 1ull << (dev & 63);
-        if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
-        return e;
+        void* v = nullptr;
+        return per_context_value(done, &v, [&](void** o) {
+            *o = reinterpret_cast<void*>(1);
+            return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        });
     }
 };
 

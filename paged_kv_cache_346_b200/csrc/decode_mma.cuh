@@ -130,7 +130,19 @@ struct MmaCfg {
 
 // NH = 8 or 16 query heads per CTA (the M rows of the QK product / the N
 // columns of the PV product); heads past the group are zero rows.
-template <typename T, int D, int BS, int NH, int NW, int STAGES_>
+//
+// GROUPS: the group pass of the shared-prefix decode.  Sequences that hold
+// the same physical blocks for their first S tokens (parallel samples forked
+// from one prompt, requests that hit the same cached prompt blocks: "pagedattention
+// vllm" §Copy-on-Write Sharing, §Advanced Features) form a group; one CTA
+// takes (prefix partition, KV head, chunk of tile rows) of group blockIdx.z,
+// whose tile rows are the (member, query head) pairs of that KV head,
+// member-major, so every page of the shared prefix is read once for all
+// members and feeds all their heads, as a query group shares its KV head's
+// pages.  The prefix's partial results go to workspace slots [0, ceil(S/P))
+// of each member row; the regular pass starts those sequences at token S and
+// the log-sum-exp reduce merges both.
+template <typename T, int D, int BS, int NH, int NW, int STAGES_, bool GROUPS = false>
 __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
@@ -147,6 +159,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
 
     extern __shared__ __align__(1024) unsigned char smem_mma[];
     __shared__ int s_abort;
+    __shared__ int64_t s_row[GROUPS ? NH : 1];  // group pass: tile row -> sequence * Hq + head
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
@@ -154,17 +167,45 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     const int hc = blockIdx.y - kvh * a.head_chunks;
     const int part = blockIdx.x;
     const int h0 = kvh * a.group + hc * NH;
-    const int nh = min(NH, a.group - hc * NH);
     const bool reporter = (tid == 0 && part == 0 && blockIdx.y == 0);
-    const int b = scheduled_seq(a, blockIdx.z, reporter);
-    if (b < 0) return;
-
-    const TablePrefetch pf = table_prefetch(a, b, part, a.partition_size / BS, tid);
-    const Span sp = seq_span(a, b, reporter);
+    int b, nh, nmem = 0;
+    const int32_t* members = nullptr;
+    TablePrefetch pf{0, false};
+    Span sp;
+    if constexpr (GROUPS) {
+        members = a.group_members + (int64_t)blockIdx.z * a.group_stride;
+        while (nmem < a.group_stride && members[nmem] >= 0) ++nmem;
+        b = nmem > 0 ? members[0] : -1;
+        if ((unsigned)b >= (unsigned)a.num_seqs) {
+            if (nmem > 0 && reporter) flag(a.status, PKV_DEV_BAD_GROUP);
+            return;
+        }
+        nh = min(NH, nmem * a.group - hc * NH);
+        if (nh <= 0) return;
+        sp = group_span(a, b, reporter);
+        if (tid < NH) {  // this chunk's rows; a member with another prefix is flagged, skipped
+            const int r = hc * NH + tid;
+            int64_t row = -1;
+            if (r < nmem * a.group) {
+                const int m = members[r / a.group];
+                if ((unsigned)m < (unsigned)a.num_seqs && a.seq_start[m] == sp.L)
+                    row = (int64_t)m * a.num_q_heads + kvh * a.group + r % a.group;
+                else if (r % a.group == 0)
+                    flag(a.status, PKV_DEV_BAD_GROUP);
+            }
+            s_row[tid] = row;
+        }
+    } else {
+        nh = min(NH, a.group - hc * NH);
+        b = scheduled_seq(a, blockIdx.z, reporter);
+        if (b < 0) return;
+        pf = table_prefetch(a, b, part, a.partition_size / BS, tid);
+        sp = seq_span(a, b, reporter);
+    }
     const int L = sp.L, np = sp.np;
     T* out = reinterpret_cast<T*>(a.out);
     if (L == 0) {
-        if (part == 0)
+        if (!GROUPS && part == 0)
             for (int i = tid; i < nh * D; i += NW * 32)
                 out[((int64_t)b * a.num_q_heads + h0 + i / D) * D + i % D] = Elem<T>::from_f32(0.f);
         return;
@@ -175,7 +216,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     // left, and its rows of one partition leave without waiting).  CTAs of
     // split sequences release it after their loop, so a grid of mostly split
     // sequences keeps the reduce from taking SM slots while it streams.
-    if (np == 1) pdl_launch_dependents();
+    if (sp.direct) pdl_launch_dependents();
 
     const int P = a.partition_size;
     const int t0 = sp.base + part * P;
@@ -225,6 +266,18 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         const int pre = min(STAGES, nslices);
         for (int s = 0; s < pre; ++s) issue(s, s);
     }
+    if constexpr (GROUPS) {
+        // every member must hold the first member's blocks (else flagged; the
+        // result then reads the first member's)
+        const int32_t* t_first = a.block_tables + (int64_t)b * a.max_blocks_per_seq + t0 / BS;
+        for (int i = tid; i < nblk * (nmem - 1); i += NW * 32) {
+            const int m = members[1 + i / nblk];
+            if ((unsigned)m < (unsigned)a.num_seqs &&
+                a.block_tables[(int64_t)m * a.max_blocks_per_seq + t0 / BS + i % nblk] !=
+                    t_first[i % nblk])
+                flag(a.status, PKV_DEV_BAD_GROUP);
+        }
+    }
 
     // Q: dims 2 t4, 2 t4 + 1 (lo) and 8 + 2 t4, + 1 (hi) of a 16-dim step for
     // head g (and g + 8) -- the B column g of an 8-head tile's S, the A rows
@@ -233,15 +286,23 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     uint32_t qa[KSTEPS][2 * QR];  // [lo g, (lo g + 8,) hi g, (hi g + 8)]
     {
         const T* qb = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D;
+        const T* qr[QR];
+#pragma unroll
+        for (int r = 0; r < QR; ++r) {  // r = 0: head g, r = 1: head g + 8
+            const int hh = g + 8 * r;
+            if constexpr (GROUPS)
+                qr[r] = s_row[hh] >= 0 ? reinterpret_cast<const T*>(a.q) + s_row[hh] * D : nullptr;
+            else
+                qr[r] = hh < nh ? qb + hh * D : nullptr;
+        }
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks) {
 #pragma unroll
-            for (int r = 0; r < QR; ++r) {  // r = 0: head g, r = 1: head g + 8
-                const int hh = g + 8 * r;
+            for (int r = 0; r < QR; ++r) {
                 uint32_t lo = 0, hi = 0;
-                if (hh < nh) {
-                    lo = *reinterpret_cast<const uint32_t*>(qb + hh * D + ks * 16 + 2 * t4);
-                    hi = *reinterpret_cast<const uint32_t*>(qb + hh * D + ks * 16 + 8 + 2 * t4);
+                if (qr[r]) {
+                    lo = *reinterpret_cast<const uint32_t*>(qr[r] + ks * 16 + 2 * t4);
+                    hi = *reinterpret_cast<const uint32_t*>(qr[r] + ks * 16 + 8 + 2 * t4);
                 }
                 qa[ks][r] = lo;
                 qa[ks][QR + r] = hi;
@@ -282,9 +343,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
             // let this warp's copies still in flight land (bounded) before
             // the CTA leaves
             if (lane == 0)
-                for (int k = it; k < min(nslices, it + STAGES); ++k)
-                    mbar_wait(full + warp * STAGES + k % STAGES, (uint32_t)((k / STAGES) & 1),
-                              a.status);
+                drain_ring(full + warp * STAGES, STAGES, it, min(nslices, it + STAGES), a.status);
             break;
         }
         const int wvalid = ntok - (it * TILE + warp * 16);
@@ -463,7 +522,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     }
     __syncthreads();  // every warp is out of its ring (or gave up)
     if (s_abort) return;
-    if (np > 1) pdl_launch_dependents();
+    if (!sp.direct) pdl_launch_dependents();
 
     // merge the warps (padded rows: lanes of one store hit distinct banks)
     using A = MergeArea<D, NH, NW>;
@@ -503,7 +562,13 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         }
     }
     __syncthreads();
-    merge_warps_and_store<T, D, NH, NW>(a, red, b, h0, nh, part, np, tid, NW * 32);
+    if constexpr (GROUPS)
+        merge_warps_and_store<T, D, NH, NW>(a, red, [&](int hh) { return s_row[hh]; }, nh, part,
+                                            false, tid, NW * 32);
+    else
+        merge_warps_and_store<T, D, NH, NW>(
+            a, red, [&](int hh) { return (int64_t)b * a.num_q_heads + h0 + hh; }, nh,
+            sp.slot0 + part, sp.direct, tid, NW * 32);
 }
 
 // Host side: tensor maps over the K and V pools, launch, optional reduce.
@@ -527,12 +592,38 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
     kern<<<grid, NW * 32, C::smem_bytes(a.partition_size), stream>>>(a, tk, tv);
     e = cudaGetLastError();
-    if (e != cudaSuccess || a.max_partitions <= 1) return e;
+    if (e != cudaSuccess || a.ws_slots <= 1) return e;
     return launch_lse_reduce<T, D>(a, stream);
+}
+
+// The group pass of the shared-prefix decode: grid (prefix partitions,
+// Hkv x row chunks, groups); writes workspace slots only (the reduce runs
+// after the regular pass).
+template <typename T, int D, int BS, int NH, int NW = 4, int STAGES = 0>
+cudaError_t launch_decode_mma_groups(const DecodeArgs& a, int num_groups, cudaStream_t stream) {
+    using C = MmaCfg<D, BS, NW, STAGES>;
+    static SmemAttr attr;
+    auto kern = decode_mma_kernel<T, D, BS, NH, NW, STAGES, true>;
+    cudaError_t e = attr.ensure(kern, C::smem_bytes(8192));
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
+    CUtensorMap tk, tv;
+    const bool bf = std::is_same<T, __nv_bfloat16>::value;
+    e = make_cache_tensor_map(&tk, a.k_cache, 2, bf, D, rows, 16);
+    if (e != cudaSuccess) return e;
+    e = make_cache_tensor_map(&tv, a.v_cache, 2, bf, D, rows, 16);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, num_groups);
+    kern<<<grid, NW * 32, C::smem_bytes(a.partition_size), stream>>>(a, tk, tv);
+    return cudaGetLastError();
 }
 
 cudaError_t decode_mma_f16(const DecodeArgs& a, int head_dim, int block_size, int hg,
                            cudaStream_t stream);
+cudaError_t decode_mma_groups_f16(const DecodeArgs& a, int head_dim, int block_size, int hg,
+                                  int num_groups, cudaStream_t stream);
+cudaError_t decode_mma_groups_bf16(const DecodeArgs& a, int head_dim, int block_size, int hg,
+                                   int num_groups, cudaStream_t stream);
 cudaError_t decode_mma_bf16(const DecodeArgs& a, int head_dim, int block_size, int hg,
                             cudaStream_t stream);
 

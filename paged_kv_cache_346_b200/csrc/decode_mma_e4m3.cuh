@@ -37,6 +37,13 @@
 // k_scale, and its P.V product (a fresh fp32 accumulator) is added to the
 // output multiplied by that page's v_scale, so P stays an fp16 value at most
 // 256 whatever the scales.
+//
+// Each softmax weight p (fp32) enters the P.V product as two fp16 terms,
+// hi = fp16(p) and lo = fp16(p - hi), in two MMAs on the same V fragment: one
+// fp16 term keeps 11 significant bits, and the output error it leaves,
+// ~2^-11 times the largest |v|, exceeds the fp16 / bf16 tolerance once values
+// are large (e.g. per-page V scales spread over decades); hi + lo keeps ~22.
+// The row sums l add the same hi + lo, so the weights stay normalised.
 #pragma once
 
 #include "decode_mma.cuh"
@@ -151,7 +158,7 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
     // left, and its rows of one partition leave without waiting).  CTAs of
     // split sequences release it after their loop, so a grid of mostly split
     // sequences keeps the reduce from taking SM slots while it streams.
-    if (np == 1) pdl_launch_dependents();
+    if (sp.direct) pdl_launch_dependents();
 
     const int P = a.partition_size;
     const int t0 = sp.base + part * P;
@@ -287,9 +294,7 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
             // let this warp's copies still in flight land (bounded) before
             // the CTA leaves
             if (lane == 0)
-                for (int k = it; k < min(nslices, it + STAGES); ++k)
-                    mbar_wait(full + warp * STAGES + k % STAGES, (uint32_t)((k / STAGES) & 1),
-                              a.status);
+                drain_ring(full + warp * STAGES, STAGES, it, min(nslices, it + STAGES), a.status);
             break;
         }
         const int wvalid = ntok - (it * TILE + warp * 16);
@@ -320,7 +325,8 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
             const bool partial = wvalid < 16 || wlo > 0;
             bool grew;               // the reference max moved: rescale o
             float alpha_c[RB][2];    // rescale factors of o's columns 2 t4, 2 t4 + 1
-            uint32_t pb[RB][2];      // P^T as the B operand: tokens 0-7, 8-15
+            uint32_t pb[RB][2];      // P^T as the B operand: tokens 0-7, 8-15 (fp16 hi)
+            uint32_t pl[RB][2];      // the fp16 remainders p - hi, same layout (lo)
             auto kcodes = [&](int kp, uint32_t (&kc)[4]) {
                 if constexpr (EARLY) {
 #pragma unroll
@@ -381,15 +387,22 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
                         alpha_c[0][j] = alpha;
                     }
                 }
-                float pr[4];
-                const uint32_t p0 = M::pack(exp2f(s[0] - m[0]), exp2f(s[1] - m[1]), pr[0], pr[1]);
-                const uint32_t p1 = M::pack(exp2f(s[2] - m[0]), exp2f(s[3] - m[1]), pr[2], pr[3]);
-                l[0] += pr[0] + pr[2];
-                l[1] += pr[1] + pr[3];
+                float p[4], pr[4], rr[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) p[i] = exp2f(s[i] - m[i & 1]);
+                const uint32_t p0 = M::pack(p[0], p[1], pr[0], pr[1]);
+                const uint32_t p1 = M::pack(p[2], p[3], pr[2], pr[3]);
+                const uint32_t r0 = M::pack(p[0] - pr[0], p[1] - pr[1], rr[0], rr[1]);
+                const uint32_t r1 = M::pack(p[2] - pr[2], p[3] - pr[3], rr[2], rr[3]);
+                // the weights the P.V products use are hi + lo
+                l[0] += (pr[0] + rr[0]) + (pr[2] + rr[2]);
+                l[1] += (pr[1] + rr[1]) + (pr[3] + rr[3]);
                 // P (tokens x heads) -> P^T fragments: lane (g, t4) gets head
                 // g, tokens 2 t4, 2 t4 + 1 (of 0-7, then of 8-15)
                 pb[0][0] = movmatrix_trans(p0);
                 pb[0][1] = movmatrix_trans(p1);
+                pl[0][0] = movmatrix_trans(r0);
+                pl[0][1] = movmatrix_trans(r1);
             } else {
                 // 16-head tiles: S^T[h, t] = Q K^T, heads as M, the slice's
                 // tokens as N (two n-tiles), two accumulator sets
@@ -457,12 +470,17 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
 #pragma unroll
                 for (int rb = 0; rb < RB; ++rb) {
                     const int i0 = 2 * rb;
-                    float pr[2][2];
+                    float pr[2][2], rr[2][2];
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-                        pb[rb][nt] = M::pack(exp2f(s[nt][i0] - m[rb]), exp2f(s[nt][i0 + 1] - m[rb]),
-                                             pr[nt][0], pr[nt][1]);
-                    l[rb] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const float p0 = exp2f(s[nt][i0] - m[rb]);
+                        const float p1 = exp2f(s[nt][i0 + 1] - m[rb]);
+                        pb[rb][nt] = M::pack(p0, p1, pr[nt][0], pr[nt][1]);
+                        pl[rb][nt] = M::pack(p0 - pr[nt][0], p1 - pr[nt][1], rr[nt][0], rr[nt][1]);
+                    }
+                    // the weights the P.V products use are hi + lo
+                    l[rb] += ((pr[0][0] + rr[0][0]) + (pr[0][1] + rr[0][1])) +
+                             ((pr[1][0] + rr[1][0]) + (pr[1][1] + rr[1][1]));
                 }
             }
 #pragma unroll
@@ -503,10 +521,12 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
                         if constexpr (PPB) {  // this page's P.V, then times its v_scale
                             float d4[4] = {0.f, 0.f, 0.f, 0.f};
                             mma_f16(d4, va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
+                            mma_f16(d4, va[0], va[1], va[2], va[3], pl[rb][0], pl[rb][1]);
 #pragma unroll
                             for (int i = 0; i < 4; ++i) o[mt][rb][i] = fmaf(d4[i], vmul, o[mt][rb][i]);
                         } else {
                             mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
+                            mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pl[rb][0], pl[rb][1]);
                         }
                     }
                 }
@@ -519,7 +539,7 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
     }
     __syncthreads();  // every warp is out of its ring (or gave up)
     if (s_abort) return;
-    if (np > 1) pdl_launch_dependents();
+    if (!sp.direct) pdl_launch_dependents();
 
     // merge the warps; A rows g, g + 8 of m-tile mt are dims 16 mt + 2 g, + 1
     using A = MergeArea<D, NH, NW>;
@@ -567,7 +587,9 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
         }
     }
     __syncthreads();
-    merge_warps_and_store<T, D, NH, NW>(a, red, b, h0, nh, part, np, tid, NW * 32);
+    merge_warps_and_store<T, D, NH, NW>(
+        a, red, [&](int hh) { return (int64_t)b * a.num_q_heads + h0 + hh; }, nh,
+        sp.slot0 + part, sp.direct, tid, NW * 32);
 }
 
 template <typename T, int D, int BS, int NH, int NW = 4, int STAGES = 0>
@@ -587,7 +609,7 @@ cudaError_t launch_decode_mma_e4m3(const DecodeArgs& a, cudaStream_t stream) {
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
     kern<<<grid, NW * 32, C::smem_bytes(a.partition_size), stream>>>(a, tk, tv);
     e = cudaGetLastError();
-    if (e != cudaSuccess || a.max_partitions <= 1) return e;
+    if (e != cudaSuccess || a.ws_slots <= 1) return e;
     return launch_lse_reduce<T, D>(a, stream);
 }
 

@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::THREAD
     // left, and its rows of one partition leave without waiting).  CTAs of
     // split sequences release it after their loop, so a grid of mostly split
     // sequences keeps the reduce from taking SM slots while it streams.
-    if (np == 1) pdl_launch_dependents();
+    if (sp.direct) pdl_launch_dependents();
 
     const int P = a.partition_size;
     const int t0 = sp.base + part * P;
@@ -389,9 +389,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::THREAD
             // let this warp's copies still in flight land (bounded) before
             // the CTA leaves
             if (lane == 0)
-                for (int k = it; k < min(nslices, it + STAGES); ++k)
-                    mbar_wait(full + warp * STAGES + k % STAGES, (uint32_t)((k / STAGES) & 1),
-                              a.status);
+                drain_ring(full + warp * STAGES, STAGES, it, min(nslices, it + STAGES), a.status);
             break;
         }
         const int wvalid = ntok - (it * TILE + warp * 16);  // tokens this warp owns
@@ -416,12 +414,14 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::THREAD
     }
     __syncthreads();  // every warp is out of its ring (or gave up)
     if (s_abort) return;
-    if (np > 1) pdl_launch_dependents();
+    if (!sp.direct) pdl_launch_dependents();
 
     // 6. merge the warps
     W.template park<NW>(warp, red, a.v_scale && !a.scale_per_block ? a.v_scale[kvh] : 1.f);
     __syncthreads();
-    merge_warps_and_store<T, D, HG, NW>(a, red, b, h0, nh, part, np, tid, NW * 32);
+    merge_warps_and_store<T, D, HG, NW>(
+        a, red, [&](int hh) { return (int64_t)b * a.num_q_heads + h0 + hh; }, nh,
+        sp.slot0 + part, sp.direct, tid, NW * 32);
 }
 
 template <typename T, int D, int BS, int HG, int NW = 4, int STAGES = 0, typename TC = T>
@@ -435,7 +435,7 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
     kern<<<grid, C::THREADS, smem_simt, stream>>>(a);
     e = cudaGetLastError();
-    if (e != cudaSuccess || a.max_partitions <= 1) return e;
+    if (e != cudaSuccess || a.ws_slots <= 1) return e;
     return launch_lse_reduce<T, D>(a, stream);
 }
 

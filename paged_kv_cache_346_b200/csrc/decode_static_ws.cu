@@ -11,35 +11,30 @@
 // The array is a file-scope __device__ variable, so every GPU that loads this
 // library's device code holds PKV_STATIC_WORKSPACE_BYTES of it until the
 // process exits.  On the host its name is only a handle: its device address
-// is looked up once per device with cudaGetSymbolAddress (with that device
-// current) on the first call made on that device, and that address is what
-// the kernels receive.
-#include <atomic>
+// is looked up with cudaGetSymbolAddress on the first call made in each CUDA
+// context (normally a device's primary context), with that context current,
+// and that address is what the kernels receive.
 #include <cstdint>
 
 #include <cuda_runtime.h>
 
+#include "context_cache.h"
+#include "decode_request.h"
 #include "pagedkv.h"
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_static_workspace[PKV_STATIC_WORKSPACE_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_static_workspace_addr[kMaxDevices];
+pkv::PerContext g_static_workspace_addr;
 
-// Device address of the array on the current device (set up on first use).
+// Device address of the array in the current context (looked up on first use
+// in each context, with that context current).
 int static_workspace_address(void** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ECUDA;
-    if (dev < 0 || dev >= kMaxDevices) return PKV_ECUDA;
-    void* p = g_static_workspace_addr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || !p) return PKV_ECUDA;
-        g_static_workspace_addr[dev].store(p, std::memory_order_release);
-    }
-    *out = p;
-    return PKV_OK;
+    const cudaError_t e = pkv::per_context_value(g_static_workspace_addr, out, [](void** o) {
+        return cudaGetSymbolAddress(o, g_static_workspace);
+    });
+    return e == cudaSuccess && *out ? PKV_OK : PKV_ECUDA;
 }
 
 }  // namespace
@@ -51,24 +46,24 @@ extern "C" int pkv_paged_attention_decode_static_ws(
     int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
     int sliding_window, pkv_dtype dtype, int partition_size, pkv_kernel kernel,
     pkv_stream_t stream) {
-    const int64_t span = sliding_window > 0 && (int64_t)sliding_window + block_size - 1 <
-                                                   (int64_t)max_context_len
-                             ? (int64_t)sliding_window + block_size - 1
-                             : (int64_t)max_context_len;
-    const size_t need = pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
-                                                  (int)span, partition_size);
-    if (need > (size_t)PKV_STATIC_WORKSPACE_BYTES) return PKV_EBOUNDS;
+    // the regular entry point's argument checks and partitioning, first, so a
+    // bad argument gets the same status here as there
+    const pkv::DecodeRequest r{out, q, k_cache, v_cache, nullptr, nullptr, 0, false,
+                               block_tables, context_lens, seq_order, num_seqs, num_q_heads,
+                               num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                               max_context_len, scale, sliding_window, dtype, partition_size,
+                               kernel};
+    pkv::DecodePlan plan;
+    int rc = pkv::plan_decode(r, &plan);
+    if (rc != PKV_OK || plan.empty) return rc;
+    if (plan.workspace_bytes > (size_t)PKV_STATIC_WORKSPACE_BYTES) return PKV_EBOUNDS;
     void* ws = nullptr;
-    if (need > 0) {
-        const int rc = static_workspace_address(&ws);
+    if (plan.workspace_bytes > 0) {
+        rc = static_workspace_address(&ws);
         if (rc != PKV_OK) return rc;
     }
-    // Everything else -- argument checks, kernels, results -- is the regular
-    // entry point's.  Nothing in the workspace has to start at zero: every
-    // entry the merge reads is written earlier in the same call.
-    return pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
-                                      seq_order, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                                      max_blocks_per_seq, num_blocks, max_context_len, scale,
-                                      sliding_window, dtype, partition_size, ws,
-                                      ws ? (size_t)PKV_STATIC_WORKSPACE_BYTES : 0, kernel, stream);
+    // Nothing in the workspace has to start at zero: every entry the merge
+    // reads is written earlier in the same call.
+    return pkv::run_decode(r, plan, ws, ws ? (size_t)PKV_STATIC_WORKSPACE_BYTES : 0,
+                           reinterpret_cast<cudaStream_t>(stream));
 }

@@ -80,6 +80,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     return mbar_wait_limit(bar, parity, status, kWaitCycles);
 }
 
+// After a wait gave up: wait again (bounded) for the copies of slices
+// [from, to) of a ring of `stages` barriers, so none lands in shared memory
+// after the CTA has left.  A copy that does not land even then could still
+// write into a later CTA's shared memory on that SM: that is flagged
+// PKV_DEV_DRAIN_TIMEOUT, beside the PKV_DEV_TIMEOUT of the waits themselves.
+__device__ __forceinline__ void drain_ring(uint64_t* bars, int stages, int from, int to,
+                                           unsigned int* status) {
+    for (int k = from; k < to; ++k)
+        if (!mbar_wait(bars + k % stages, (uint32_t)((k / stages) & 1), status))
+            flag(status, PKV_DEV_DRAIN_TIMEOUT);
+}
+
 // L2 policy for data read exactly once (the K/V pages of a decode step).
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
