@@ -43,6 +43,7 @@ from workloads import (CONFIGS, ELEM_BYTES, algorithmic_bytes, make_decode_input
 
 METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak) and tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+RATED_HBM_GBS = 8000.0      # B200's rated HBM3e bandwidth (the copy peak above is measured)
 
 
 # --------------------------------------------------------------------------
@@ -76,13 +77,14 @@ def measured_peaks():
     return None
 
 
-def step_bytes(cfg, lens, window: int = 0, kv_dtype: str | None = None) -> int:
+def step_bytes(cfg, lens, window: int = 0, kv_dtype: str | None = None,
+               per_page_scales: bool = False) -> int:
     """Decode algorithmic bytes + the append: read k, v of each new token,
     write them (as E4M3 codes with kv_dtype "e4m3"), read the slot."""
     e = ELEM_BYTES[cfg.dtype]
     ec = ELEM_BYTES[kv_dtype or cfg.dtype]
     append = len(lens) * (2 * cfg.num_kv_heads * cfg.head_dim * (e + ec) + 8)
-    return algorithmic_bytes(cfg, lens, window, kv_dtype) + append
+    return algorithmic_bytes(cfg, lens, window, kv_dtype, per_page_scales) + append
 
 
 class ClockSampler:
@@ -172,10 +174,13 @@ def resolve_variant(cfg, kernel: str, kv: str = "same") -> str:
     return "mma" if cfg.dtype != "f32" and 4 <= cfg.group <= 16 else "simt"
 
 
-def recorded_traffic(workload: str, variant: str, partition: int | None = None):
+def recorded_traffic(workload: str, variant: str, partition: int | None = None,
+                     kv: str = "same"):
     """DRAM bytes per decode call from a committed ncu summary, if it was
-    taken on the current kernel sources (else None)."""
-    p = os.path.join(ROOT, "profiles", f"decode_{variant}_{workload}.md")
+    taken on the current kernel sources (else None).  Summaries of runs with a
+    scale per E4M3 page carry the suffix _page."""
+    suffix = "_page" if kv == "e4m3-page" else ""
+    p = os.path.join(ROOT, "profiles", f"decode_{variant}_{workload}{suffix}.md")
     if not os.path.exists(p):
         return None
     rec = {}
@@ -196,7 +201,8 @@ def recorded_traffic(workload: str, variant: str, partition: int | None = None):
 # --------------------------------------------------------------------------
 # CPU oracle timing (the reference arm and the cpu_baseline field)
 
-def oracle_rate(inp, budget_s: float, seed: int = 0, pages=None):
+def oracle_rate(inp, budget_s: float, seed: int = 0, pages=None, window: int = 0,
+                per_page: bool = False):
     """Time the float64 oracle on whole sequences (all heads), in a seeded
     order, passing over the batch again until about budget_s of wall time;
     returns (bytes/s, seconds, sample description, threads).  pages: E4M3
@@ -207,11 +213,12 @@ def oracle_rate(inp, budget_s: float, seed: int = 0, pages=None):
 
     def run_rows(rows, threads):
         if pages is None:
-            return oracle.paged_decode_inputs(inp, rows=rows, threads=threads)
+            return oracle.paged_decode_inputs(inp, rows=rows, threads=threads, window=window)
         return oracle.paged_decode(inp.q, pages.k_cache, pages.v_cache, inp.block_tables,
                                    inp.context_lens, scale=cfg.scale, dtype=cfg.dtype,
                                    kv_dtype="e4m3", k_scale=pages.k_scale,
-                                   v_scale=pages.v_scale, rows=rows, threads=threads)
+                                   v_scale=pages.v_scale, rows=rows, threads=threads,
+                                   window=window)
     threads = oracle.max_threads()
     order = np.random.default_rng(seed).permutation(cfg.num_seqs)
     nseq, ntok, nbytes, t_total = 0, 0, 0, 0.0
@@ -223,7 +230,7 @@ def oracle_rate(inp, budget_s: float, seed: int = 0, pages=None):
             t_total += time.perf_counter() - t0
             nseq += 1
             ntok += int(inp.context_lens[b])
-            nbytes += algorithmic_bytes(cfg, inp.context_lens[[b]], kv_dtype=kvd)
+            nbytes += algorithmic_bytes(cfg, inp.context_lens[[b]], window, kvd, per_page)
             if t_total >= budget_s:
                 break
         if t_total >= budget_s:
@@ -238,29 +245,46 @@ def run_reference(args, cfg):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    inp = make_decode_inputs(cfg, seed=args.seed)
+    inp = make_decode_inputs(cfg, seed=args.seed, shuffle=args.tables == "shuffled")
     import oracle
+    e4m3 = args.kv in ("e4m3", "e4m3-page")
+    per_page = args.kv == "e4m3-page"
+    pages = make_e4m3_pages(inp, seed=args.seed, per_page=per_page) if e4m3 else None
+    kvd = "e4m3" if e4m3 else None
+    W = args.window
     threads = oracle.max_threads()
-    # calibrate on one sequence, then size each step's sample so the whole
+
+    def run_rows(rows):
+        if pages is None:
+            return oracle.paged_decode_inputs(inp, rows=rows, threads=threads, window=W)
+        return oracle.paged_decode(inp.q, pages.k_cache, pages.v_cache, inp.block_tables,
+                                   inp.context_lens, scale=cfg.scale, dtype=cfg.dtype,
+                                   kv_dtype="e4m3", k_scale=pages.k_scale,
+                                   v_scale=pages.v_scale, rows=rows, threads=threads, window=W)
+
+    # calibrate on a few sequences, then size each step's sample so the whole
     # run stays within about --ref-budget seconds
-    rate, _, _, _ = oracle_rate(inp, 0.0, seed=args.seed)
+    cal = np.arange(min(4, cfg.num_seqs))
+    t0 = time.perf_counter()
+    run_rows(np.array([[b, h] for b in cal for h in range(cfg.num_q_heads)], dtype=np.int32))
+    rate = algorithmic_bytes(cfg, inp.context_lens[cal], W, kvd, per_page) / max(
+        time.perf_counter() - t0, 1e-6)
     steps_total = args.steps + args.warmup
     budget = args.ref_budget / max(steps_total, 1)
-    seq_bytes = algorithmic_bytes(cfg, inp.context_lens) / cfg.num_seqs
+    seq_bytes = algorithmic_bytes(cfg, inp.context_lens, W, kvd, per_page) / cfg.num_seqs
     nseq = int(max(1, min(cfg.num_seqs, math.floor(rate * budget / seq_bytes))))
     g = np.random.default_rng(args.seed)
-    samples = []
     times = []
     nbytes = []
     for i in range(steps_total):
         seqs = g.choice(cfg.num_seqs, size=nseq, replace=False)
         rows = np.array([[b, h] for b in seqs for h in range(cfg.num_q_heads)], dtype=np.int32)
         t0 = time.perf_counter()
-        oracle.paged_decode_inputs(inp, rows=rows, threads=threads)
+        run_rows(rows)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
-            nbytes.append(algorithmic_bytes(cfg, inp.context_lens[seqs]))
+            nbytes.append(algorithmic_bytes(cfg, inp.context_lens[seqs], W, kvd, per_page))
     value = sum(nbytes) / sum(times) / 1e9
     sample = (f"{nseq} of {cfg.num_seqs} sequences per step (all {cfg.num_q_heads} heads), "
               f"float64 C oracle, {threads} threads")
@@ -269,8 +293,7 @@ def run_reference(args, cfg):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * sum(times) / len(times), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "global_batch": cfg.num_seqs,
-                   "seq_len": float(np.mean(inp.context_lens)), "parallelism": "none (host CPU)"},
+        "config": workload_config(cfg, inp.context_lens, args.gpus, args.tables, W, args.kv),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -284,11 +307,186 @@ def run_reference(args, cfg):
 # --------------------------------------------------------------------------
 # GPU arm
 
+def workload_config(cfg, lens, world: int, tables: str, window: int, kv: str) -> dict:
+    """The workload a line measures (the same dict on both arms)."""
+    per_page = kv == "e4m3-page"
+    kv_pages = (("e4m3 (per-page fp32 scales)" if per_page else "e4m3 (per-head fp32 scales)")
+                if kv.startswith("e4m3") else cfg.dtype)
+    kvd = "e4m3" if kv.startswith("e4m3") else None
+    dec = algorithmic_bytes(cfg, lens, window, kvd, per_page)
+    return {"workload": cfg.name, "global_batch": cfg.num_seqs * world,
+            "seq_len": round(float(np.mean(lens)), 1), "num_q_heads": cfg.num_q_heads,
+            "num_kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
+            "block_size": cfg.block_size, "block_tables": tables, "sliding_window": window,
+            "kv_pages": kv_pages, "q_out": cfg.dtype, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (%.2f GB of K/V per step)" % (dec / 1e9)}
+
+
+class Workload:
+    """One decode workload on the device: seeded inputs, the step (append of
+    each sequence's new token + decode) and its byte counts."""
+
+    def __init__(self, args, cfg, kv: str, rank: int, partition: int, window: int):
+        import torch
+
+        import paged_kv_cache_346_b200 as pkv
+        self.cfg, self.kv = cfg, kv
+        self.kern = {"auto": pkv.PKV_KERNEL_AUTO, "simt": pkv.PKV_KERNEL_SIMT,
+                     "mma": pkv.PKV_KERNEL_MMA}[args.kernel]
+        inp = make_decode_inputs(cfg, seed=args.seed + rank, shuffle=args.tables == "shuffled")
+        self.inp = inp
+        self.e4m3 = e4m3 = kv in ("e4m3", "e4m3-page")
+        self.per_page = per_page = kv == "e4m3-page"
+        if e4m3 and cfg.dtype == "f32":
+            raise SystemExit("E4M3 pages take fp16/bf16 q")
+
+        def dev(a):
+            if cfg.dtype == "bf16" and a.dtype == np.uint16:
+                return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+            return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        self.dev = dev
+
+        self.pages = None
+        if e4m3:
+            self.pages = pages = make_e4m3_pages(inp, seed=args.seed + rank, per_page=per_page)
+            self.q = dev(inp.q)
+            self.kc = dev(pages.k_cache).view(torch.float8_e4m3fn)
+            self.vc = dev(pages.v_cache).view(torch.float8_e4m3fn)
+            self.ks, self.vs = dev(pages.k_scale), dev(pages.v_scale)
+        else:
+            self.q, self.kc, self.vc = dev(inp.q), dev(inp.k_cache), dev(inp.v_cache)
+            self.ks = self.vs = None
+        self.bt, self.cl = dev(inp.block_tables), dev(inp.context_lens)
+        B, H, D, bs = cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
+        self.lens = lens = inp.context_lens.astype(np.int64)
+        last = lens - 1
+        slots_np = (inp.block_tables[np.arange(B), last // bs].astype(np.int64) * bs + last % bs)
+        self.slots = dev(slots_np)
+        # the new token of each sequence: the K/V already at its last position
+        # (so every step rewrites identical bits and the workload stays fixed)
+        # (with E4M3 pages: those values dequantised to q's type; re-quantising
+        # them reaches a fixed point after the first step)
+        sb_idx = torch.from_numpy(slots_np // bs).cuda()
+        so_idx = torch.from_numpy(slots_np % bs).cuda()
+        if e4m3:
+            ksel = self.ks[sb_idx] if per_page else self.ks[None, :]   # [B or 1, Hkv]
+            vsel = self.vs[sb_idx] if per_page else self.vs[None, :]
+            self.knew = (self.kc.view(torch.uint8)[sb_idx, :, so_idx, :].view(
+                torch.float8_e4m3fn).float() * ksel[:, :, None]).to(self.q.dtype).contiguous()
+            self.vnew = (self.vc.view(torch.uint8)[sb_idx, :, so_idx, :].view(
+                torch.float8_e4m3fn).float() * vsel[:, :, None]).to(self.q.dtype).contiguous()
+        else:
+            self.knew = self.kc.view(-1, H, bs, D)[sb_idx, :, so_idx, :].contiguous()
+            self.vnew = self.vc.view(-1, H, bs, D)[sb_idx, :, so_idx, :].contiguous()
+        self.out = torch.empty_like(self.q)
+        self.mcl = mcl = inp.max_context_len
+        # schedule the longest sequences first (host-side order from host lengths)
+        order_np = pkv.pkv_decode_schedule_order(inp.context_lens) if args.order else None
+        self.order = dev(order_np) if order_np is not None else None
+        self.P = P = partition
+        self.W = W = window
+        span = min(mcl, W + bs - 1) if W > 0 else mcl
+        ws_bytes = pkv.pkv_decode_workspace_size(B, cfg.num_q_heads, H, D, span, P)
+        self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+        self.Pused = P or pkv.pkv_decode_default_partition(B, H, span)
+        self.launches_per_step = 1 + 1 + (1 if math.ceil(span / self.Pused) > 1 else 0)
+        kvd = "e4m3" if e4m3 else None
+        self.step_bytes = step_bytes(cfg, lens, W, kvd, per_page)
+        self.dec_bytes = algorithmic_bytes(cfg, lens, W, kvd, per_page)
+        self.variant = resolve_variant(cfg, args.kernel, kv)
+        self.pkv = pkv
+
+    def decode(self, stream):
+        pkv, c = self.pkv, self.cfg
+        if self.e4m3:
+            pkv.pkv_paged_attention_decode_e4m3(
+                self.out, self.q, self.kc, self.vc, self.ks, self.vs, self.bt, self.cl, c.scale,
+                c.block_size, self.mcl, partition_size=self.P, workspace=self.ws,
+                seq_order=self.order, sliding_window=self.W, kernel=self.kern, stream=stream)
+        else:
+            pkv.pkv_paged_attention_decode(
+                self.out, self.q, self.kc, self.vc, self.bt, self.cl, c.scale, c.block_size,
+                self.mcl, partition_size=self.P, workspace=self.ws, seq_order=self.order,
+                sliding_window=self.W, kernel=self.kern, stream=stream)
+
+    def append(self, stream):
+        if self.e4m3:
+            self.pkv.pkv_kv_cache_append_e4m3(self.kc, self.vc, self.knew, self.vnew, self.ks,
+                                              self.vs, self.slots, stream=stream)
+        else:
+            self.pkv.pkv_kv_cache_append(self.kc, self.vc, self.knew, self.vnew, self.slots,
+                                         stream=stream)
+
+
+def time_blocks(w: Workload, steps: int, warmup: int, min_device_s: float, barrier, local,
+                max_blocks: int = 400):
+    """Warm up, then time blocks of exactly `steps` steps (each bracketed by a
+    barrier and a synchronize, CUDA events on the launching stream, events
+    around every decode call too) until at least min_device_s of device time
+    has been timed (and at least 3 blocks).  NVML clocks are sampled
+    throughout.  -> (block ms list, mean decode ms per block list, clocks)"""
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        w.append(stream)
+        w.decode(stream)
+    torch.cuda.synchronize()
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    blocks, dec = [], []
+    with ClockSampler(local) as clocks:
+        while True:
+            barrier()
+            torch.cuda.synchronize()
+            t_start.record(stream)
+            for i in range(steps):
+                w.append(stream)
+                ev_dec[i][0].record(stream)
+                w.decode(stream)
+                ev_dec[i][1].record(stream)
+            t_end.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            blocks.append(t_start.elapsed_time(t_end))
+            dec.append(statistics.mean(a.elapsed_time(b) for a, b in ev_dec))
+            if (len(blocks) >= 3 and sum(blocks) * 1e-3 >= min_device_s) or \
+                    len(blocks) >= max_blocks:
+                break
+    flags = w.pkv.pkv_device_status(clear=True)
+    if flags:
+        raise SystemExit(f"device status flags {flags:#x} during the benchmark")
+    return blocks, dec, clocks.summary()
+
+
+def median_block(blocks, dec):
+    """The median block (by step time) and its decode time."""
+    i = sorted(range(len(blocks)), key=lambda k: blocks[k])[len(blocks) // 2]
+    return blocks[i], dec[i]
+
+
+def hbm_peak():
+    peaks = measured_peaks()
+    if peaks and "hbm_gbs" in peaks:
+        return float(peaks["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def roofline_of(w: Workload, dec_ms: float, args) -> dict:
+    peak, src = hbm_peak()
+    achieved = w.dec_bytes / (dec_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "paged decode (partition kernel + LSE reduce)",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_source": src,
+            "frac_of_rated_8tbs": round(achieved / RATED_HBM_GBS, 4),
+            "decode_ms": round(dec_ms, 5), "bytes_per_launch": int(w.dec_bytes),
+            "variant": w.variant,
+            "traffic": recorded_traffic(w.cfg.name, w.variant, w.Pused, w.kv)}
+
+
 def run_ours(args, cfg):
     import torch
     import torch.distributed as dist
-
-    import paged_kv_cache_346_b200 as pkv
 
     rank, world, local = dist_env()
     if not torch.cuda.is_available():
@@ -303,116 +501,14 @@ def run_ours(args, cfg):
         if world > 1:
             dist.barrier()
 
-    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[cfg.dtype]
-    kern = {"auto": pkv.PKV_KERNEL_AUTO, "simt": pkv.PKV_KERNEL_SIMT,
-            "mma": pkv.PKV_KERNEL_MMA}[args.kernel]
-
-    # ---- inputs (seeded; each rank its own replica)
-    inp = make_decode_inputs(cfg, seed=args.seed + rank, shuffle=args.tables == "shuffled")
-    e4m3 = args.kv in ("e4m3", "e4m3-page")
-    per_page = args.kv == "e4m3-page"
-    if e4m3 and cfg.dtype == "f32":
-        raise SystemExit("E4M3 pages take fp16/bf16 q")
-
-    def dev(a):
-        if cfg.dtype == "bf16" and a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
-        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
-
-    pages = None
-    if e4m3:
-        pages = make_e4m3_pages(inp, seed=args.seed + rank, per_page=per_page)
-        q = dev(inp.q)
-        kc = dev(pages.k_cache).view(torch.float8_e4m3fn)
-        vc = dev(pages.v_cache).view(torch.float8_e4m3fn)
-        ks, vs = dev(pages.k_scale), dev(pages.v_scale)
-    else:
-        q, kc, vc = dev(inp.q), dev(inp.k_cache), dev(inp.v_cache)
-    bt, cl = dev(inp.block_tables), dev(inp.context_lens)
+    w = Workload(args, cfg, args.kv, rank, args.partition, args.window)
+    pkv = w.pkv
     B, H, D, bs = cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
-    lens = inp.context_lens.astype(np.int64)
-    last = lens - 1
-    slots_np = (inp.block_tables[np.arange(B), last // bs].astype(np.int64) * bs + last % bs)
-    slots = dev(slots_np)
-    # the new token of each sequence: the K/V already at its last position
-    # (so every step rewrites identical bits and the workload stays fixed)
-    # (with E4M3 pages: those values dequantised to q's type; re-quantising
-    # them reaches a fixed point after the first step)
-    sb_idx = torch.from_numpy(slots_np // bs).cuda()
-    so_idx = torch.from_numpy(slots_np % bs).cuda()
-    if e4m3:
-        ksel = ks[sb_idx] if per_page else ks[None, :]   # [B or 1, Hkv]
-        vsel = vs[sb_idx] if per_page else vs[None, :]
-        knew = (kc.view(torch.uint8)[sb_idx, :, so_idx, :].view(torch.float8_e4m3fn).float() *
-                ksel[:, :, None]).to(q.dtype).contiguous()
-        vnew = (vc.view(torch.uint8)[sb_idx, :, so_idx, :].view(torch.float8_e4m3fn).float() *
-                vsel[:, :, None]).to(q.dtype).contiguous()
-    else:
-        knew = kc.view(-1, H, bs, D)[sb_idx, :, so_idx, :].contiguous()
-        vnew = vc.view(-1, H, bs, D)[sb_idx, :, so_idx, :].contiguous()
-    out = torch.empty_like(q)
-    mcl = inp.max_context_len
-    # schedule the longest sequences first (host-side order from host lengths)
-    order_np = pkv.pkv_decode_schedule_order(inp.context_lens) if args.order else None
-    order = dev(order_np) if order_np is not None else None
-    P = args.partition
-    W = args.window
-    span = min(mcl, W + bs - 1) if W > 0 else mcl
-    ws_bytes = pkv.pkv_decode_workspace_size(B, cfg.num_q_heads, H, D, span, P)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
-    Pused = P or pkv.pkv_decode_default_partition(B, H, span)
-    launches_per_step = 1 + 1 + (1 if math.ceil(span / Pused) > 1 else 0)
     stream = torch.cuda.current_stream()
 
-    def decode():
-        if e4m3:
-            pkv.pkv_paged_attention_decode_e4m3(out, q, kc, vc, ks, vs, bt, cl, cfg.scale, bs,
-                                                mcl, partition_size=P, workspace=ws,
-                                                seq_order=order, sliding_window=W,
-                                                kernel=kern, stream=stream)
-        else:
-            pkv.pkv_paged_attention_decode(out, q, kc, vc, bt, cl, cfg.scale, bs, mcl,
-                                           partition_size=P, workspace=ws, seq_order=order,
-                                           sliding_window=W, kernel=kern, stream=stream)
-
-    def append():
-        if e4m3:
-            pkv.pkv_kv_cache_append_e4m3(kc, vc, knew, vnew, ks, vs, slots, stream=stream)
-        else:
-            pkv.pkv_kv_cache_append(kc, vc, knew, vnew, slots, stream=stream)
-
-    def step():
-        append()
-        decode()
-
-    kvd = "e4m3" if e4m3 else None
-    nbytes = step_bytes(cfg, lens, W, kvd)
-    dec_bytes = algorithmic_bytes(cfg, lens, W, kvd)
-
-    # ---- device-resident timing
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        t_start.record(stream)
-        for i in range(args.steps):
-            append()
-            ev_dec[i][0].record(stream)
-            decode()
-            ev_dec[i][1].record(stream)
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    barrier()
-    ms = t_start.elapsed_time(t_end)
-    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_dec)
-    flags = pkv.pkv_device_status(clear=True)
-    if flags:
-        raise SystemExit(f"device status flags {flags:#x} during the benchmark")
+    # ---- device-resident timing: blocks of --steps steps, the median block
+    blocks, decs, clocks = time_blocks(w, args.steps, args.warmup, args.min_time, barrier, local)
+    ms, dec_ms = median_block(blocks, decs)
 
     # ---- end to end through the public API: every step copies its inputs
     # (q, the new tokens' K/V, slots, tables, lengths, schedule order) from
@@ -422,9 +518,11 @@ def run_ours(args, cfg):
     # input and two output buffers and two copy streams let step i+1's upload
     # and step i-1's readback run under step i's kernels; events order every
     # reuse.
-    fields = [("q", q), ("knew", knew), ("vnew", vnew), ("slots", slots), ("bt", bt), ("cl", cl)]
-    if order is not None:
-        fields.append(("order", order))
+    q, kc, vc, out, ws = w.q, w.kc, w.vc, w.out, w.ws
+    fields = [("q", q), ("knew", w.knew), ("vnew", w.vnew), ("slots", w.slots), ("bt", w.bt),
+              ("cl", w.cl)]
+    if w.order is not None:
+        fields.append(("order", w.order))
     offs, total = {}, 0
     for name, t in fields:
         offs[name] = total
@@ -447,29 +545,30 @@ def run_ours(args, cfg):
     c_stream = ctypes.c_void_p(stream.cuda_stream)
     dt_code = pkv.torch_dtype_code(q.dtype)
     N_blocks = kc.shape[0]
+    P, W, mcl = w.P, w.W, w.mcl
     calls = []
     for j in range(2):
         ptr = {name: ctypes.c_void_p(d_in[j].data_ptr() + offs[name]) for name, _ in fields}
         kp, vp = ctypes.c_void_p(kc.data_ptr()), ctypes.c_void_p(vc.data_ptr())
-        if e4m3:
-            ksp, vsp = ctypes.c_void_p(ks.data_ptr()), ctypes.c_void_p(vs.data_ptr())
-            spb = 1 if per_page else 0
+        if w.e4m3:
+            ksp, vsp = ctypes.c_void_p(w.ks.data_ptr()), ctypes.c_void_p(w.vs.data_ptr())
+            spb = 1 if w.per_page else 0
             append_args = (kp, vp, ptr["knew"], ptr["vnew"], ksp, vsp, spb, ptr["slots"], B, H, D,
                            bs, N_blocks, dt_code, c_stream)
             decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ksp, vsp, spb,
                            ptr["bt"], ptr["cl"], ptr.get("order"), B, cfg.num_q_heads, H, D,
-                           bs, bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
-                           ctypes.c_void_p(ws.data_ptr()), ws.numel(), kern, c_stream)
+                           bs, w.bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
+                           ctypes.c_void_p(ws.data_ptr()), ws.numel(), w.kern, c_stream)
         else:
             append_args = (kp, vp, ptr["knew"], ptr["vnew"], ptr["slots"], B, H, D, bs,
                            N_blocks, dt_code, c_stream)
             decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ptr["bt"],
                            ptr["cl"], ptr.get("order"), B, cfg.num_q_heads, H, D, bs,
-                           bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
-                           ctypes.c_void_p(ws.data_ptr()), ws.numel(), kern, c_stream)
+                           w.bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
+                           ctypes.c_void_p(ws.data_ptr()), ws.numel(), w.kern, c_stream)
         calls.append((append_args, decode_args))
-    c_append = pkv.lib.pkv_kv_cache_append_e4m3 if e4m3 else pkv.lib.pkv_kv_cache_append
-    c_decode = (pkv.lib.pkv_paged_attention_decode_e4m3 if e4m3
+    c_append = pkv.lib.pkv_kv_cache_append_e4m3 if w.e4m3 else pkv.lib.pkv_kv_cache_append
+    c_decode = (pkv.lib.pkv_paged_attention_decode_e4m3 if w.e4m3
                 else pkv.lib.pkv_paged_attention_decode)
 
     def e2e_step(i):
@@ -489,7 +588,7 @@ def run_ours(args, cfg):
             h_out[j].copy_(d_out[j], non_blocking=True)
             ev_out[j].record(s_out)
 
-    e2e_steps = max(4, min(args.steps, 400))
+    e2e_steps = max(4, min(args.steps * 20, 1000))
     for i in range(max(args.warmup, 3)):
         e2e_step(i)
     torch.cuda.synchronize()
@@ -506,56 +605,71 @@ def run_ours(args, cfg):
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     assert torch.equal(h_out[0], out.cpu()) and torch.equal(h_out[1], out.cpu())
+    del d_in, d_out, h_in, h_out
+
+    # ---- the other workloads the targets name, measured the same way
+    also = []
+    for spec in ([] if args.also == "none" else args.also.split(",")):
+        name, _, kv = spec.partition(":")
+        kv = kv or "same"
+        if name == cfg.name and kv == args.kv:
+            continue
+        w2 = Workload(args, CONFIGS[name], kv, rank, CONFIGS[name].partition_size, 0)
+        b2, d2, c2 = time_blocks(w2, args.steps, args.warmup, args.min_time, barrier, local)
+        m2, dm2 = median_block(b2, d2)
+        m2, dm2 = max_over_ranks([m2, dm2], world)
+        also.append((w2, b2, m2, dm2, c2))
+        del w2
 
     # ---- max over ranks
     ms, dec_ms, e2e_ms = max_over_ranks([ms, dec_ms, e2e_ms], world)
 
     if rank == 0:
         per_step_ms = ms / args.steps
-        value = world * nbytes / (per_step_ms * 1e-3) / 1e9
-        peaks = measured_peaks()
-        if peaks and "hbm_gbs" in peaks:
-            peak, peak_src = float(peaks["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
-        else:
-            peak, peak_src = FALLBACK_HBM_GBS, "fallback"
-        achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+        value = world * w.step_bytes / (per_step_ms * 1e-3) / 1e9
+        peak, _ = hbm_peak()
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3" if e4m3 else cfg.dtype, "data": "synthetic",
-            "config": {"workload": cfg.name, "global_batch": B * world,
-                       "seq_len": round(float(lens.mean()), 1),
-                       "num_q_heads": cfg.num_q_heads, "num_kv_heads": H, "head_dim": D,
-                       "block_size": bs, "partition_size": Pused, "kernel": args.kernel,
-                       "schedule": "longest-first" if args.order else "batch order",
-                       "block_tables": args.tables,
-                       "sliding_window": W,
-                       "kv_pages": ("e4m3 (per-page fp32 scales)" if per_page else
-                                    "e4m3 (per-head fp32 scales)") if e4m3 else cfg.dtype,
-                       "q_out": cfg.dtype,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (%.2f GB of K/V per step)" % (
-                           dec_bytes / 1e9)},
+            "dtype": "e4m3" if w.e4m3 else cfg.dtype, "data": "synthetic",
+            "config": workload_config(cfg, w.lens, world, args.tables, w.W, args.kv),
+            "impl_config": {"partition_size": w.Pused, "kernel": args.kernel,
+                            "schedule": "longest-first" if args.order else "batch order"},
+            "timing": {"blocks": len(blocks), "steps_per_block": args.steps,
+                       "block_ms_median": round(ms, 4), "block_ms_min": round(min(blocks), 4),
+                       "block_ms_max": round(max(blocks), 4),
+                       "device_s_timed": round(sum(blocks) * 1e-3, 3),
+                       "note": "median of the timed blocks; each block is --steps steps "
+                               "bracketed by a barrier and a synchronize"},
             "tokens_per_s": round(world * B / (per_step_ms * 1e-3), 1),
             "pct_of_hbm_peak": round(100 * value / world / peak, 2),
-            "e2e": {"value": round(world * nbytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "pct_of_rated_hbm_8tbs": round(100 * value / world / RATED_HBM_GBS, 2),
+            "e2e": {"value": round(world * w.step_bytes / (e2e_ms * 1e-3) / 1e9, 2),
+                    "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                     "ms_per_step": round(e2e_ms, 4)},
-            "gpu_launches": launches_per_step * args.steps,
-            "roofline": {"bound": "hbm", "kernel": "paged decode (partition kernel + LSE reduce)",
-                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "peak_source": peak_src,
-                         "decode_ms": round(dec_ms, 5), "bytes_per_launch": int(dec_bytes),
-                         "variant": resolve_variant(cfg, args.kernel, args.kv),
-                         "traffic": recorded_traffic(cfg.name,
-                                                     resolve_variant(cfg, args.kernel, args.kv),
-                                                     Pused)},
-            "clocks": clocks.summary(),
+            "gpu_launches": w.launches_per_step * args.steps,
+            "roofline": roofline_of(w, dec_ms, args),
+            "clocks": clocks,
         }
+        if also:
+            line["also"] = []
+            for w2, b2, m2, dm2, c2 in also:
+                st = m2 / args.steps
+                v2 = world * w2.step_bytes / (st * 1e-3) / 1e9
+                line["also"].append({
+                    "config": workload_config(w2.cfg, w2.lens, world, args.tables, 0, w2.kv),
+                    "impl_config": {"partition_size": w2.Pused, "kernel": args.kernel,
+                                    "schedule": "longest-first" if args.order else "batch order"},
+                    "value": round(v2, 2), "unit": "GB/s", "ms_per_step": round(st, 5),
+                    "tokens_per_s": round(world * w2.cfg.num_seqs / (st * 1e-3), 1),
+                    "pct_of_hbm_peak": round(100 * v2 / world / peak, 2),
+                    "blocks": len(b2), "device_s_timed": round(sum(b2) * 1e-3, 3),
+                    "roofline": roofline_of(w2, dm2, args), "clocks": c2})
         if world == 1 and not args.no_cpu_baseline:
-            rate, secs, desc, threads = oracle_rate(inp, args.cpu_budget, seed=args.seed,
-                                                    pages=pages)
+            rate, secs, desc, threads = oracle_rate(w.inp, args.cpu_budget, seed=args.seed,
+                                                    pages=w.pages, window=w.W,
+                                                    per_page=w.per_page)
             line["cpu_baseline"] = {"value": round(rate / 1e9, 4), "unit": "GB/s",
                                     "cores": threads, "kind": "oracle",
                                     "sample": desc + f", {secs:.1f} s"}
@@ -573,7 +687,10 @@ def run_cow(args):
     (i) the fork step -- every sample appends its first token, the allocator
     hands out 7 block copies per prompt, and the step runs copy_blocks,
     kv_cache_append and the decode; (ii) a steady step once every sample has
-    a private tail of U[1, 512] tokens -- append + decode, no copies."""
+    a private tail of U[1, 512] tokens -- append + decode, no copies.  The
+    decode is the shared-prefix decode (each prompt's shared blocks read once
+    for its samples); the regular decode of the same step is timed beside it
+    ("regular_decode")."""
     import torch
 
     import paged_kv_cache_346_b200 as pkv
@@ -612,11 +729,28 @@ def run_cow(args):
         L = int(lens_np.max())
         ws = torch.empty(max(16, pkv.pkv_decode_workspace_size(B, H, H, D, L)),
                          dtype=torch.uint8, device="cuda")
+        # the shared prompt blocks of each prompt's samples, found from the
+        # host tables (the allocator's), for the shared-prefix decode
+        spl_np, mem_np = pkv.pkv_decode_prefix_groups(tables_np, lens_np, bs)
+        spl, mem = torch.from_numpy(spl_np).cuda(), torch.from_numpy(mem_np).cuda()
+        mpl = int(spl_np.max())
+        ws_g = torch.empty(max(16, pkv.pkv_decode_prefix_groups_workspace_size(B, H, H, D, L,
+                                                                              mpl)),
+                           dtype=torch.uint8, device="cuda")
         npairs = len(pairs_np)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(3)]
 
-        def step(timed=False):
+        def decode(grouped):
+            if grouped:
+                pkv.pkv_paged_attention_decode_prefix_groups(out, q, kc, vc, tables, lens, spl,
+                                                             mem, scale, bs, L, mpl,
+                                                             workspace=ws_g, stream=stream)
+            else:
+                pkv.pkv_paged_attention_decode(out, q, kc, vc, tables, lens, scale, bs, L,
+                                               workspace=ws, stream=stream)
+
+        def step(grouped, timed=False):
             if timed:
                 ev[0][0].record(stream)
             if npairs:
@@ -628,24 +762,28 @@ def run_cow(args):
             if timed:
                 ev[1][1].record(stream)
                 ev[2][0].record(stream)
-            pkv.pkv_paged_attention_decode(out, q, kc, vc, tables, lens, scale, bs, L,
-                                           workspace=ws, stream=stream)
+            decode(grouped)
             if timed:
                 ev[2][1].record(stream)
 
-        for _ in range(args.warmup):
-            step()
-        torch.cuda.synchronize()
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        parts = np.zeros(3)
-        t0.record(stream)
-        for _ in range(args.steps):
-            step(timed=True)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        ms = t0.elapsed_time(t1) / args.steps
-        # per-kernel times of the last step (events were re-recorded each step)
-        parts = [a.elapsed_time(b) for a, b in ev]
+        def timed_steps(grouped):
+            for _ in range(args.warmup):
+                step(grouped)
+            torch.cuda.synchronize()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(args.steps):
+                step(grouped, timed=True)
+            t1.record(stream)
+            torch.cuda.synchronize()
+            # per-kernel times of the last step (events were re-recorded each step)
+            return t0.elapsed_time(t1) / args.steps, [a.elapsed_time(b) for a, b in ev]
+
+        ms_r, parts_r = timed_steps(False)
+        out_r = out.clone()
+        ms, parts = timed_steps(True)
+        # the two decodes differ only in summation order
+        diff = float((out.float() - out_r.float()).abs().max())
         # bytes: logical = every sequence's K/V as read; unique = distinct
         # physical (block, slot) entries the decode reads
         kv_tok = 2 * H * D * e
@@ -664,9 +802,15 @@ def run_cow(args):
         return {
             "ms_per_step": round(ms, 5),
             "copy_pairs": npairs,
+            "prefix_groups": int(len(mem_np)),
+            "shared_prefix_tokens_mean": round(float(spl_np.mean()), 1),
             "kernel_ms_last_step": {"copy_blocks": round(parts[0], 5),
                                     "kv_append": round(parts[1], 5),
                                     "decode": round(parts[2], 5)},
+            "regular_decode": {"ms_per_step": round(ms_r, 5), "decode_ms": round(parts_r[2], 5),
+                               "decode_unique_GBps": round((unique + qo + tab) /
+                                                           (parts_r[2] * 1e-3) / 1e9, 1)},
+            "max_abs_diff_vs_regular": diff,
             "logical_bytes": logical + qo + tab + copy + append,
             "unique_bytes": unique + qo + tab + copy + append,
             "effective_GBps": round((logical + qo + tab + copy + append) / (ms * 1e-3) / 1e9, 1),
@@ -807,6 +951,12 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="seconds of oracle work for --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--min-time", type=float, default=0.5,
+                    help="time blocks of --steps steps until at least this many seconds of "
+                         "device time (and 3 blocks); the median block is reported")
+    ap.add_argument("--also", default="gqa_bs16,gqa_bs32,gqa_bs16:e4m3,llama2_13b_layer:e4m3",
+                    help="further workloads[:kv] measured the same way and reported under "
+                         "\"also\" (none: only the main one)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     if args.workload == "cow_sampling":

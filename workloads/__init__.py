@@ -254,11 +254,12 @@ def kv_bytes_per_token(cfg: DecodeConfig, kv_dtype: str | None = None) -> int:
 
 
 def algorithmic_bytes(cfg: DecodeConfig, lens: np.ndarray, window: int = 0,
-                      kv_dtype: str | None = None) -> int:
+                      kv_dtype: str | None = None, per_page_scales: bool = False) -> int:
     """Bytes a decode step must move at least once: K and V of every attended
     token (the last `window` of each sequence when window > 0), q in and out,
-    the block-table entries used and the lengths (and the per-head scales of
-    quantised pages, kv_dtype "e4m3")."""
+    the block-table entries used and the lengths (and the scales of quantised
+    pages, kv_dtype "e4m3": one K and one V float32 per KV head, or per
+    attended (block, KV head) page with per_page_scales)."""
     e = ELEM_BYTES[cfg.dtype]
     lens = np.asarray(lens, dtype=np.int64)
     if window > 0:
@@ -271,7 +272,9 @@ def algorithmic_bytes(cfg: DecodeConfig, lens: np.ndarray, window: int = 0,
     kv = int(att.sum()) * kv_bytes_per_token(cfg, kv_dtype)
     qo = 2 * lens.size * cfg.num_q_heads * cfg.head_dim * e
     tab = int(nblk.sum()) * 4
-    scales = 8 * cfg.num_kv_heads if kv_dtype == "e4m3" else 0
+    scales = 0
+    if kv_dtype == "e4m3":
+        scales = 8 * cfg.num_kv_heads * (int(nblk.sum()) if per_page_scales else 1)
     return kv + qo + tab + 4 * lens.size + scales
 
 
