@@ -38,8 +38,12 @@ struct DecodeArgs {
     int max_tokens;               // max_blocks_per_seq * BS
     int partition_size;           // tokens per partition
     int max_partitions;           // grid.x = ceil(longest attended span / partition_size)
+    const int32_t* plan_cta;      // planned decode: [grid + 1] item ranges of the CTAs
+    const int32_t* plan_items;    // [items][PKV_PLAN_ITEM_WORDS] pieces
+    int32_t* plan_counts;         // [units] warps counted in per unit, zero between calls
     int ws_slots;                 // partial results per row in the workspace
     int group_stride;             // group_members row length
+    int after_groups;             // launched as a programmatic dependent of the group pass
     int block_size;
     int window;                   // sliding window in tokens, 0 = attend to the whole context
     int scale_per_block;          // E4M3 scales per (block, KV head) page
@@ -187,13 +191,15 @@ struct MergeArea {
 
 // Merge NW parked warp states (acc rows, m, l in `red`, written and
 // synchronised by the caller) of nh heads and write the output rows (direct:
-// the row's only partial result) or the partial (m, l, o) to workspace slot
-// `slot`.  Tile row hh is global row row_of(hh) = sequence * Hq + head.  All
-// threads of the CTA take part.  Per head: M = max_w m_w,
-// den = sum_w 2^(m_w - M) l_w, o = sum_w (2^(m_w - M) / den) acc_w.
-template <typename T, int D, int NH, int NW, typename RowOf>
+// the row's only partial result) or the partial (m, l, o) to the workspace.
+// Tile row hh is output row row_of(hh) = sequence * Hq + head, and partial
+// row part_of(hh) of the workspace (ws_o rows of D floats, ws_ml rows of 2);
+// rows with row_of(hh) < 0 are skipped.  All threads of the CTA take part.
+// Per head: M = max_w m_w, den = sum_w 2^(m_w - M) l_w,
+// o = sum_w (2^(m_w - M) / den) acc_w.
+template <typename T, int D, int NH, int NW, typename RowOf, typename PartOf>
 __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float* red,
-                                                      RowOf row_of, int nh, int slot,
+                                                      RowOf row_of, PartOf part_of, int nh,
                                                       bool direct, int tid, int nthreads) {
     using A = MergeArea<D, NH, NW>;
     float* red_m = red + NW * NH * A::RP;
@@ -219,7 +225,7 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float
             if (direct) {
                 out[row * D + d] = Elem<T>::from_f32(num / den);
             } else {
-                const int64_t pr = row * a.ws_slots + slot;
+                const int64_t pr = part_of(0);
                 a.ws_o[pr * D + d] = num / den;
                 if (d == 0) {
                     a.ws_ml[pr * 2] = M;
@@ -245,7 +251,7 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float
 #pragma unroll
             for (int w = 0; w < NW; ++w) red_s[w * NH + tid] = f[w] * inv;
             if (!direct && row_of(tid) >= 0) {
-                const int64_t pr = row_of(tid) * a.ws_slots + slot;
+                const int64_t pr = part_of(tid);
                 a.ws_ml[pr * 2] = M;
                 a.ws_ml[pr * 2 + 1] = den;
             }
@@ -262,42 +268,30 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float
             if (direct)
                 out[row * D + d] = Elem<T>::from_f32(o);
             else
-                a.ws_o[(row * a.ws_slots + slot) * D + d] = o;
+                a.ws_o[part_of(hh) * D + d] = o;
         }
     }
 }
 
-// Merge the partitions of one (sequence, query head) row: with per-partition
-// maxima m_p (base-2 logits), sums l_p and normalised outputs o_p,
+// Merge n partial results of one (sequence, query head) row into out_row:
+// with per-partial maxima m_p (base-2 logits), sums l_p and normalised
+// outputs o_p,
 //   M = max_p m_p,  w_p = l_p 2^(m_p - M),  out = sum_p w_p o_p / sum_p w_p.
-// One CTA of 128 threads per row; rows with one partial result in all were
-// written by the decode kernel and are skipped.  Launched as a programmatic
-// dependent of the decode kernel: those rows leave before the wait, during
-// the decode's tail; the others wait for the decode grid's writes before
-// reading.
+// Partial p's (m, l) is at ml + p * ml_stride, its o at o + p * o_stride.
+// All 128 threads of the CTA take part.
 template <typename T, int D>
-__global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
+__device__ __forceinline__ void merge_partials(const float* ml, int64_t ml_stride,
+                                               const float* o, int64_t o_stride, int np,
+                                               T* out_row) {
     constexpr int NW = 4;
     constexpr int PER_LANE = D / 32;  // floats of o per lane
-    const int h = blockIdx.x;
-    const int b = blockIdx.y;
-    // the partition count depends only on the inputs, not on the decode
-    // grid's output: rows with one partial result leave before the wait
-    const Span sp = seq_span(a, b, false);
-    if (sp.direct) return;
-    const int np = sp.slot0 + sp.np;  // the group pass's slots, then this row's partitions
-    pdl_wait_primary();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t row = (int64_t)b * a.num_q_heads + h;
-    const float* ml = a.ws_ml + row * a.ws_slots * 2;
-    const float* o = a.ws_o + row * a.ws_slots * D;
-
     __shared__ float s_max[NW];
     __shared__ float s_den[NW];
     __shared__ float s_num[NW][D];
 
     float M = -INFINITY;
-    for (int p = tid; p < np; p += 128) M = fmaxf(M, ml[2 * p]);
+    for (int p = tid; p < np; p += 128) M = fmaxf(M, ml[p * ml_stride]);
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
     if (lane == 0) s_max[warp] = M;
@@ -309,9 +303,9 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
     for (int i = 0; i < PER_LANE; ++i) num[i] = 0.f;
     float den = 0.f;
     for (int p = warp; p < np; p += NW) {
-        const float w = ml[2 * p + 1] * exp2f(ml[2 * p] - M);
+        const float w = ml[p * ml_stride + 1] * exp2f(ml[p * ml_stride] - M);
         den += w;
-        const float* op = o + (int64_t)p * D + lane * PER_LANE;
+        const float* op = o + p * o_stride + lane * PER_LANE;
         if constexpr (PER_LANE % 4 == 0) {
 #pragma unroll
             for (int i = 0; i < PER_LANE; i += 4) {
@@ -331,11 +325,66 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
     if (lane == 0) s_den[warp] = den;
     __syncthreads();
     const float total = s_den[0] + s_den[1] + s_den[2] + s_den[3];
-    T* out = reinterpret_cast<T*>(a.out) + row * D;
     for (int d = tid; d < D; d += 128) {
         const float x = s_num[0][d] + s_num[1][d] + s_num[2][d] + s_num[3][d];
-        out[d] = Elem<T>::from_f32(x / total);
+        out_row[d] = Elem<T>::from_f32(x / total);
     }
+}
+
+// Merge the partitions of one (sequence, query head) row (merge_partials).
+// One CTA of 128 threads per row; rows with one partial result in all were
+// written by the decode kernel and are skipped.  Launched as a programmatic
+// dependent of the decode kernel: those rows leave before the wait, during
+// the decode's tail; the others wait for the decode grid's writes before
+// reading.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
+    const int h = blockIdx.x;
+    const int b = blockIdx.y;
+    // the partition count depends only on the inputs, not on the decode
+    // grid's output: rows with one partial result leave before the wait
+    const Span sp = seq_span(a, b, false);
+    if (sp.direct) return;
+    const int np = sp.slot0 + sp.np;  // the group pass's slots, then this row's partitions
+    pdl_wait_primary();
+    const int64_t row = (int64_t)b * a.num_q_heads + h;
+    merge_partials<T, D>(a.ws_ml + row * a.ws_slots * 2, 2, a.ws_o + row * a.ws_slots * D, D, np,
+                         reinterpret_cast<T*>(a.out) + row * D);
+}
+
+// The regular pass of the shared-prefix decode may start while the group
+// pass still runs (it is a programmatic dependent of it; neither reads the
+// other's results).  The log-sum-exp reduce, a programmatic dependent of the
+// regular pass, reads both: so no CTA of the regular pass leaves before the
+// group pass has completed and its writes are visible.  Held by every CTA of
+// the regular pass; releases at each exit.
+struct GroupPassWait {
+    const DecodeArgs& a;
+    __device__ __forceinline__ ~GroupPassWait() {
+        if (a.after_groups) pdl_wait_primary();
+    }
+};
+
+// Launch a decode kernel; with after_groups as a programmatic dependent of
+// the kernel before it in the stream (the group pass).
+template <typename K, typename... Args>
+cudaError_t launch_decode_kernel(K kernel, dim3 grid, dim3 block, int smem, cudaStream_t stream,
+                                 bool after_groups, Args... args) {
+    if (!after_groups) {
+        kernel<<<grid, block, smem, stream>>>(args...);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 // "Dynamic shared memory limit raised" bookkeeping for one kernel, per CUDA

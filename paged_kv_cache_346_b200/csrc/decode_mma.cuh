@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     extern __shared__ __align__(1024) unsigned char smem_mma[];
     __shared__ int s_abort;
     __shared__ int64_t s_row[GROUPS ? NH : 1];  // group pass: tile row -> sequence * Hq + head
+    const GroupPassWait group_pass_wait{a};
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
@@ -173,6 +174,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     TablePrefetch pf{0, false};
     Span sp;
     if constexpr (GROUPS) {
+        pdl_launch_dependents();  // the regular pass may start beside this grid
         members = a.group_members + (int64_t)blockIdx.z * a.group_stride;
         while (nmem < a.group_stride && members[nmem] >= 0) ++nmem;
         b = nmem > 0 ? members[0] : -1;
@@ -563,12 +565,16 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     }
     __syncthreads();
     if constexpr (GROUPS)
-        merge_warps_and_store<T, D, NH, NW>(a, red, [&](int hh) { return s_row[hh]; }, nh, part,
-                                            false, tid, NW * 32);
+        merge_warps_and_store<T, D, NH, NW>(
+            a, red, [&](int hh) { return s_row[hh]; },
+            [&](int hh) { return s_row[hh] * a.ws_slots + part; }, nh, false, tid, NW * 32);
     else
         merge_warps_and_store<T, D, NH, NW>(
-            a, red, [&](int hh) { return (int64_t)b * a.num_q_heads + h0 + hh; }, nh,
-            sp.slot0 + part, sp.direct, tid, NW * 32);
+            a, red, [&](int hh) { return (int64_t)b * a.num_q_heads + h0 + hh; },
+            [&](int hh) {
+                return ((int64_t)b * a.num_q_heads + h0 + hh) * a.ws_slots + sp.slot0 + part;
+            },
+            nh, sp.direct, tid, NW * 32);
 }
 
 // Host side: tensor maps over the K and V pools, launch, optional reduce.
@@ -590,8 +596,8 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
     e = make_cache_tensor_map(&tv, a.v_cache, 2, bf, D, rows, 16);
     if (e != cudaSuccess) return e;
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
-    kern<<<grid, NW * 32, C::smem_bytes(a.partition_size), stream>>>(a, tk, tv);
-    e = cudaGetLastError();
+    e = launch_decode_kernel(kern, grid, dim3(NW * 32), C::smem_bytes(a.partition_size), stream,
+                             a.after_groups != 0, a, tk, tv);
     if (e != cudaSuccess || a.ws_slots <= 1) return e;
     return launch_lse_reduce<T, D>(a, stream);
 }

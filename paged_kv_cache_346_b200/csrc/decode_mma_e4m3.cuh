@@ -112,6 +112,281 @@ struct E4m3MinBlocks {
         (D <= 128 && NH == 8) ? (D == 128 && STAGES_ == 3 ? 16 / NW : 3) : 1;
 };
 
+// q (fp16 or bf16) as the fp16 MMA operand: rows g (and g + 8 when NH is 16)
+// of the tile, qrow(hh) giving head hh's row (nullptr: a zero row), dims in
+// the order ldmatrix delivers the K codes (k = 2 t4 + j -> dim 4 t4 + j,
+// k = 2 t4 + 8 + j -> dim 4 t4 + 2 + j), scaled by the power of two 2^e that
+// puts the tile's largest |q| in [2^14, 2^15).  Returns the logits'
+// multiplier, mul * 2^-e.  All 32 lanes take part.
+template <typename T, int D, int NH, typename QRow>
+__device__ __forceinline__ float e4m3_prepare_q(QRow qrow, float mul,
+                                                uint32_t (&qa)[D / 16][NH == 16 ? 4 : 2], int g,
+                                                int t4) {
+    constexpr int KSTEPS = D / 16;
+    float qf[KSTEPS][2][4];
+    float mx = 0.f;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const T* row = qrow(g + 8 * r);
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                qf[ks][r][j] = row ? Elem<T>::load1(row + ks * 16 + 4 * t4 + j) : 0.f;
+                mx = fmaxf(mx, fabsf(qf[ks][r][j]));
+            }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    // 2^e with mx * 2^e in [2^14, 2^15): e = 141 - biased exponent of mx
+    const int be = (__float_as_int(mx) >> 23) & 0xff;
+    int e = be == 0 ? 0 : 141 - be;
+    e = max(-126, min(126, e));
+    const float up = __int_as_float((127 + e) << 23);
+    const float down = __int_as_float((127 - e) << 23);
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const __half2 lo = __floats2half2_rn(qf[ks][r][0] * up, qf[ks][r][1] * up);
+            const __half2 hi = __floats2half2_rn(qf[ks][r][2] * up, qf[ks][r][3] * up);
+            if (NH == 16 || r == 0) {
+                // NH 16: qa = a0a1, a2a3, a4a5, a6a7; NH 8: qa = a0a1, a4a5
+                qa[ks][NH == 16 ? r : 0] = *reinterpret_cast<const uint32_t*>(&lo);
+                qa[ks][NH == 16 ? 2 + r : 1] = *reinterpret_cast<const uint32_t*>(&hi);
+            }
+        }
+    return mul * down;
+}
+
+// One warp's work on one 16-token slice of K and V (codes in its ring stage,
+// or already in kf / vf with EARLY): the logits, the online softmax against
+// the lazy reference max, and O^T += V^T P^T with P as fp16 hi + lo.  The
+// state (m, l, o) is the warp's; addr(kp) is the ldmatrix address of chunk
+// pair kp of the slice's K rows (V rows: + 16 D bytes); tokens outside
+// [wlo, wvalid) of the slice are masked.
+template <int D, int NH, bool PPB, bool EARLY, typename Addr>
+__device__ __forceinline__ void e4m3_slice_math(
+    const uint32_t (&qa)[D / 16][NH == 16 ? 4 : 2], float (&m)[NH == 8 ? 2 : NH / 8],
+    float (&l)[NH == 8 ? 2 : NH / 8], float (&o)[D / 16][NH / 8][4],
+    const uint32_t (&kf)[EARLY ? D / 32 : 1][4], const uint32_t (&vf)[EARLY ? D / 32 : 1][4],
+    Addr addr, int wvalid, int wlo, float kmul, float vmul, int g, int t4) {
+    using M = Mma<__half>;
+    constexpr int KSTEPS = D / 16, KP = KSTEPS / 2, RB = NH / 8;
+    constexpr int SLICE_BYTES = 16 * D;
+    (void)vmul;
+    (void)SLICE_BYTES;
+    const bool partial = wvalid < 16 || wlo > 0;
+    bool grew;               // the reference max moved: rescale o
+    float alpha_c[RB][2];    // rescale factors of o's columns 2 t4, 2 t4 + 1
+    uint32_t pb[RB][2];      // P^T as the B operand: tokens 0-7, 8-15 (fp16 hi)
+    uint32_t pl[RB][2];      // the fp16 remainders p - hi, same layout (lo)
+    auto kcodes = [&](int kp, uint32_t (&kc)[4]) {
+        if constexpr (EARLY) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) kc[i] = kf[kp < (EARLY ? KP : 1) ? kp : 0][i];
+        } else {
+            ldsm_x4(addr(kp), kc);
+        }
+    };
+    if constexpr (NH == 8) {
+        // S[t, h] = K Q^T with the slice's 16 tokens as M and the 8
+        // heads as N: one MMA per 16-dim step (an 8-head S^T tile
+        // would fill half of M).  K codes of tokens g / g + 8 are the
+        // A rows, q the B columns; two accumulator sets (even / odd
+        // steps) make two short dependency chains.
+        float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kp = 0; kp < KP; ++kp) {
+            uint32_t kc[4];
+            kcodes(kp, kc);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // k-step 2 kp + h
+                uint32_t k0, k1, k2, k3;
+                e4m3x4_to_f16x2(kc[2 * h], k0, k1);      // token g
+                e4m3x4_to_f16x2(kc[2 * h + 1], k2, k3);  // token g + 8
+                const uint32_t* q4 = qa[2 * kp + h];
+                mma_f16(h ? s2 : s, k0, k2, k1, k3, q4[0], q4[1]);
+            }
+        }
+        // lane (g, t4): s[0], s[1] = token g, heads 2 t4, 2 t4 + 1;
+        // s[2], s[3] = token g + 8
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            s[i] = (s[i] + s2[i]) * kmul;
+            const int tok = g + 8 * (i >> 1);
+            if (partial && (tok < wlo || tok >= wvalid)) s[i] = -INFINITY;
+        }
+        // lazy reference max per head (see below); a head's tokens
+        // are spread over the 8 lanes of one t4
+        bool up = false;
+        float tmax[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            tmax[j] = fmaxf(s[j], s[2 + j]);
+            up |= tmax[j] > m[j] + 8.f;
+        }
+        grew = __any_sync(0xffffffffu, up);
+        if (grew) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                float mx = tmax[j];
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float mnew = fmaxf(m[j], mx);
+                const float alpha = exp2f(m[j] - mnew);
+                l[j] *= alpha;
+                m[j] = mnew;
+                alpha_c[0][j] = alpha;
+            }
+        }
+        float p[4], pr[4], rr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) p[i] = exp2f(s[i] - m[i & 1]);
+        const uint32_t p0 = M::pack(p[0], p[1], pr[0], pr[1]);
+        const uint32_t p1 = M::pack(p[2], p[3], pr[2], pr[3]);
+        const uint32_t r0 = M::pack(p[0] - pr[0], p[1] - pr[1], rr[0], rr[1]);
+        const uint32_t r1 = M::pack(p[2] - pr[2], p[3] - pr[3], rr[2], rr[3]);
+        // the weights the P.V products use are hi + lo
+        l[0] += (pr[0] + rr[0]) + (pr[2] + rr[2]);
+        l[1] += (pr[1] + rr[1]) + (pr[3] + rr[3]);
+        // P (tokens x heads) -> P^T fragments: lane (g, t4) gets head
+        // g, tokens 2 t4, 2 t4 + 1 (of 0-7, then of 8-15)
+        pb[0][0] = movmatrix_trans(p0);
+        pb[0][1] = movmatrix_trans(p1);
+        pl[0][0] = movmatrix_trans(r0);
+        pl[0][1] = movmatrix_trans(r1);
+    } else {
+        // 16-head tiles: S^T[h, t] = Q K^T, heads as M, the slice's
+        // tokens as N (two n-tiles), two accumulator sets
+        float s[2][4], s2[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s[nt][i] = s2[nt][i] = 0.f;
+#pragma unroll
+        for (int kp = 0; kp < KP; ++kp) {
+            uint32_t kc[4];
+            kcodes(kp, kc);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // k-step 2 kp + h
+                uint32_t b0, b1, b2, b3;
+                e4m3x4_to_f16x2(kc[2 * h], b0, b1);      // tokens 0-7
+                e4m3x4_to_f16x2(kc[2 * h + 1], b2, b3);  // tokens 8-15
+                const uint32_t* q4 = qa[2 * kp + h];
+                mma_f16(h ? s2[0] : s[0], q4[0], q4[1], q4[2], q4[3], b0, b1);
+                mma_f16(h ? s2[1] : s[1], q4[0], q4[1], q4[2], q4[3], b2, b3);
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s[nt][i] = (s[nt][i] + s2[nt][i]) * kmul;
+        if (partial) {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int tok = nt * 8 + 2 * t4 + (i & 1);
+                    if (tok < wlo || tok >= wvalid) s[nt][i] = -INFINITY;
+                }
+        }
+        // Softmax against a reference max m that moves only when a
+        // logit exceeds it by more than 2^8 (then p <= 256 fits fp16
+        // and the accumulators are rescaled); l is kept per lane (this
+        // lane's tokens) and summed over the head's lanes at the end.
+        // The result is the same softmax: every p and l of a head
+        // shares m.
+        bool up = false;
+        float tmax[RB];
+#pragma unroll
+        for (int rb = 0; rb < RB; ++rb) {
+            const int i0 = 2 * rb;
+            tmax[rb] = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
+            up |= tmax[rb] > m[rb] + 8.f;
+        }
+        grew = __any_sync(0xffffffffu, up);
+        if (grew) {
+#pragma unroll
+            for (int rb = 0; rb < RB; ++rb) {
+                float mx = tmax[rb];
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float mnew = fmaxf(m[rb], mx);
+                const float alpha = exp2f(m[rb] - mnew);
+                l[rb] *= alpha;
+                m[rb] = mnew;
+                alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
+                alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
+            }
+        }
+#pragma unroll
+        for (int rb = 0; rb < RB; ++rb) {
+            const int i0 = 2 * rb;
+            float pr[2][2], rr[2][2];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const float p0 = exp2f(s[nt][i0] - m[rb]);
+                const float p1 = exp2f(s[nt][i0 + 1] - m[rb]);
+                pb[rb][nt] = M::pack(p0, p1, pr[nt][0], pr[nt][1]);
+                pl[rb][nt] = M::pack(p0 - pr[nt][0], p1 - pr[nt][1], rr[nt][0], rr[nt][1]);
+            }
+            // the weights the P.V products use are hi + lo
+            l[rb] += ((pr[0][0] + rr[0][0]) + (pr[0][1] + rr[0][1])) +
+                     ((pr[1][0] + rr[1][0]) + (pr[1][1] + rr[1][1]));
+        }
+    }
+#pragma unroll
+    for (int kp = 0; kp < KP; ++kp) {
+        uint32_t vc[4];
+        if constexpr (EARLY) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) vc[i] = vf[kp < (EARLY ? KP : 1) ? kp : 0][i];
+        } else {
+            ldsm_x4_trans(addr(kp) + SLICE_BYTES, vc);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // m-tile 2 kp + h
+            const int mt = 2 * kp + h;
+            uint32_t va[4];
+            // (V[r0][2g], V[r0][2g+1], V[r1][2g], V[r1][2g+1]) ->
+            // (V[r0][2g], V[r1][2g] | V[r0][2g+1], V[r1][2g+1])
+            e4m3x4_to_f16x2(byte_perm(vc[2 * h], 0x3120u), va[0], va[1]);
+            e4m3x4_to_f16x2(byte_perm(vc[2 * h + 1], 0x3120u), va[2], va[3]);
+            if (partial) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int tk = (i >> 1) * 8 + 2 * t4;
+                    const uint32_t keep =
+                        (tk >= wlo && tk < wvalid ? 0x0000ffffu : 0u) |
+                        (tk + 1 >= wlo && tk + 1 < wvalid ? 0xffff0000u : 0u);
+                    va[i] &= keep;
+                }
+            }
+#pragma unroll
+            for (int rb = 0; rb < RB; ++rb) {
+                if (grew) {
+                    o[mt][rb][0] *= alpha_c[rb][0];
+                    o[mt][rb][1] *= alpha_c[rb][1];
+                    o[mt][rb][2] *= alpha_c[rb][0];
+                    o[mt][rb][3] *= alpha_c[rb][1];
+                }
+                if constexpr (PPB) {  // this page's P.V, then times its v_scale
+                    float d4[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_f16(d4, va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
+                    mma_f16(d4, va[0], va[1], va[2], va[3], pl[rb][0], pl[rb][1]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) o[mt][rb][i] = fmaf(d4[i], vmul, o[mt][rb][i]);
+                } else {
+                    mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
+                    mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pl[rb][0], pl[rb][1]);
+                }
+            }
+        }
+    }
+}
+
 // PPB: a scale per page (a.scale_per_block), a compile-time choice so the
 // per-head path carries no per-slice scale code.
 template <typename T, int D, int BS, int NH, int NW, int STAGES_, bool PPB>
@@ -211,53 +486,14 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
     }
 
     // Q as the A operand (rows = heads g, g + 8), dims in the order the K
-    // codes arrive: k = 2 t4 + j -> dim 4 t4 + j, k = 2 t4 + 8 + j -> 4 t4 + 2 + j.
-    // rows g + 8 (heads 8..15) exist only when NH == 16
+    // codes arrive (e4m3_prepare_q)
     constexpr int QR = NH == 16 ? 4 : 2;
     uint32_t qa[KSTEPS][QR];
-    float qmul;  // logits multiplier: scale * log2(e) * k_scale * 2^-e
-    {
-        const T* qb = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D;
-        float qf[KSTEPS][2][4];
-        float mx = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < KSTEPS; ++ks)
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int hh = g + 8 * r;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) qf[ks][r][j] = 0.f;
-                if (hh < nh) {
-                    const T* src = qb + hh * D + ks * 16 + 4 * t4;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        qf[ks][r][j] = Elem<T>::load1(src + j);
-                        mx = fmaxf(mx, fabsf(qf[ks][r][j]));
-                    }
-                }
-            }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        // 2^e with mx * 2^e in [2^14, 2^15): e = 141 - biased exponent of mx
-        const int be = (__float_as_int(mx) >> 23) & 0xff;
-        int e = be == 0 ? 0 : 141 - be;
-        e = max(-126, min(126, e));
-        const float up = __int_as_float((127 + e) << 23);
-        const float down = __int_as_float((127 - e) << 23);
-        qmul = a.scale_log2 * (PPB ? 1.f : a.k_scale[kvh]) * down;
-#pragma unroll
-        for (int ks = 0; ks < KSTEPS; ++ks)
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const __half2 lo = __floats2half2_rn(qf[ks][r][0] * up, qf[ks][r][1] * up);
-                const __half2 hi = __floats2half2_rn(qf[ks][r][2] * up, qf[ks][r][3] * up);
-                if (NH == 16 || r == 0) {
-                    // NH 16: qa = a0a1, a2a3, a4a5, a6a7; NH 8: qa = a0a1, a4a5
-                    qa[ks][NH == 16 ? r : 0] = *reinterpret_cast<const uint32_t*>(&lo);
-                    qa[ks][NH == 16 ? 2 + r : 1] = *reinterpret_cast<const uint32_t*>(&hi);
-                }
-            }
-    }
+    const T* qb = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0) * D;
+    // logits multiplier: scale * log2(e) * k_scale * 2^-e
+    const float qmul = e4m3_prepare_q<T, D, NH>(
+        [&](int hh) { return hh < nh ? qb + hh * D : nullptr; },
+        a.scale_log2 * (PPB ? 1.f : a.k_scale[kvh]), qa, g, t4);
 
     // softmax state: 8-head tiles keep it for heads 2 t4, 2 t4 + 1 (the S
     // columns of this lane), 16-head tiles for heads g + 8 rb (its S^T rows)
@@ -322,215 +558,8 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
             }
         }
         auto math = [&]() {
-            const bool partial = wvalid < 16 || wlo > 0;
-            bool grew;               // the reference max moved: rescale o
-            float alpha_c[RB][2];    // rescale factors of o's columns 2 t4, 2 t4 + 1
-            uint32_t pb[RB][2];      // P^T as the B operand: tokens 0-7, 8-15 (fp16 hi)
-            uint32_t pl[RB][2];      // the fp16 remainders p - hi, same layout (lo)
-            auto kcodes = [&](int kp, uint32_t (&kc)[4]) {
-                if constexpr (EARLY) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) kc[i] = kf[kp < (EARLY ? KP : 1) ? kp : 0][i];
-                } else {
-                    ldsm_x4(addr(kp), kc);
-                }
-            };
-            if constexpr (NH == 8) {
-                // S[t, h] = K Q^T with the slice's 16 tokens as M and the 8
-                // heads as N: one MMA per 16-dim step (an 8-head S^T tile
-                // would fill half of M).  K codes of tokens g / g + 8 are the
-                // A rows, q the B columns; two accumulator sets (even / odd
-                // steps) make two short dependency chains.
-                float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int kp = 0; kp < KP; ++kp) {
-                    uint32_t kc[4];
-                    kcodes(kp, kc);
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {  // k-step 2 kp + h
-                        uint32_t k0, k1, k2, k3;
-                        e4m3x4_to_f16x2(kc[2 * h], k0, k1);      // token g
-                        e4m3x4_to_f16x2(kc[2 * h + 1], k2, k3);  // token g + 8
-                        const uint32_t* q4 = qa[2 * kp + h];
-                        mma_f16(h ? s2 : s, k0, k2, k1, k3, q4[0], q4[1]);
-                    }
-                }
-                // lane (g, t4): s[0], s[1] = token g, heads 2 t4, 2 t4 + 1;
-                // s[2], s[3] = token g + 8
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    s[i] = (s[i] + s2[i]) * kmul;
-                    const int tok = g + 8 * (i >> 1);
-                    if (partial && (tok < wlo || tok >= wvalid)) s[i] = -INFINITY;
-                }
-                // lazy reference max per head (see below); a head's tokens
-                // are spread over the 8 lanes of one t4
-                bool up = false;
-                float tmax[2];
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    tmax[j] = fmaxf(s[j], s[2 + j]);
-                    up |= tmax[j] > m[j] + 8.f;
-                }
-                grew = __any_sync(0xffffffffu, up);
-                if (grew) {
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        float mx = tmax[j];
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                        const float mnew = fmaxf(m[j], mx);
-                        const float alpha = exp2f(m[j] - mnew);
-                        l[j] *= alpha;
-                        m[j] = mnew;
-                        alpha_c[0][j] = alpha;
-                    }
-                }
-                float p[4], pr[4], rr[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) p[i] = exp2f(s[i] - m[i & 1]);
-                const uint32_t p0 = M::pack(p[0], p[1], pr[0], pr[1]);
-                const uint32_t p1 = M::pack(p[2], p[3], pr[2], pr[3]);
-                const uint32_t r0 = M::pack(p[0] - pr[0], p[1] - pr[1], rr[0], rr[1]);
-                const uint32_t r1 = M::pack(p[2] - pr[2], p[3] - pr[3], rr[2], rr[3]);
-                // the weights the P.V products use are hi + lo
-                l[0] += (pr[0] + rr[0]) + (pr[2] + rr[2]);
-                l[1] += (pr[1] + rr[1]) + (pr[3] + rr[3]);
-                // P (tokens x heads) -> P^T fragments: lane (g, t4) gets head
-                // g, tokens 2 t4, 2 t4 + 1 (of 0-7, then of 8-15)
-                pb[0][0] = movmatrix_trans(p0);
-                pb[0][1] = movmatrix_trans(p1);
-                pl[0][0] = movmatrix_trans(r0);
-                pl[0][1] = movmatrix_trans(r1);
-            } else {
-                // 16-head tiles: S^T[h, t] = Q K^T, heads as M, the slice's
-                // tokens as N (two n-tiles), two accumulator sets
-                float s[2][4], s2[2][4];
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) s[nt][i] = s2[nt][i] = 0.f;
-#pragma unroll
-                for (int kp = 0; kp < KP; ++kp) {
-                    uint32_t kc[4];
-                    kcodes(kp, kc);
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {  // k-step 2 kp + h
-                        uint32_t b0, b1, b2, b3;
-                        e4m3x4_to_f16x2(kc[2 * h], b0, b1);      // tokens 0-7
-                        e4m3x4_to_f16x2(kc[2 * h + 1], b2, b3);  // tokens 8-15
-                        const uint32_t* q4 = qa[2 * kp + h];
-                        mma_f16(h ? s2[0] : s[0], q4[0], q4[1], q4[2], q4[3], b0, b1);
-                        mma_f16(h ? s2[1] : s[1], q4[0], q4[1], q4[2], q4[3], b2, b3);
-                    }
-                }
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) s[nt][i] = (s[nt][i] + s2[nt][i]) * kmul;
-                if (partial) {
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int tok = nt * 8 + 2 * t4 + (i & 1);
-                            if (tok < wlo || tok >= wvalid) s[nt][i] = -INFINITY;
-                        }
-                }
-                // Softmax against a reference max m that moves only when a
-                // logit exceeds it by more than 2^8 (then p <= 256 fits fp16
-                // and the accumulators are rescaled); l is kept per lane (this
-                // lane's tokens) and summed over the head's lanes at the end.
-                // The result is the same softmax: every p and l of a head
-                // shares m.
-                bool up = false;
-                float tmax[RB];
-#pragma unroll
-                for (int rb = 0; rb < RB; ++rb) {
-                    const int i0 = 2 * rb;
-                    tmax[rb] = fmaxf(fmaxf(s[0][i0], s[0][i0 + 1]), fmaxf(s[1][i0], s[1][i0 + 1]));
-                    up |= tmax[rb] > m[rb] + 8.f;
-                }
-                grew = __any_sync(0xffffffffu, up);
-                if (grew) {
-#pragma unroll
-                    for (int rb = 0; rb < RB; ++rb) {
-                        float mx = tmax[rb];
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                        const float mnew = fmaxf(m[rb], mx);
-                        const float alpha = exp2f(m[rb] - mnew);
-                        l[rb] *= alpha;
-                        m[rb] = mnew;
-                        alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
-                        alpha_c[rb][1] = __shfl_sync(0xffffffffu, alpha, (2 * t4 + 1) * 4);
-                    }
-                }
-#pragma unroll
-                for (int rb = 0; rb < RB; ++rb) {
-                    const int i0 = 2 * rb;
-                    float pr[2][2], rr[2][2];
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        const float p0 = exp2f(s[nt][i0] - m[rb]);
-                        const float p1 = exp2f(s[nt][i0 + 1] - m[rb]);
-                        pb[rb][nt] = M::pack(p0, p1, pr[nt][0], pr[nt][1]);
-                        pl[rb][nt] = M::pack(p0 - pr[nt][0], p1 - pr[nt][1], rr[nt][0], rr[nt][1]);
-                    }
-                    // the weights the P.V products use are hi + lo
-                    l[rb] += ((pr[0][0] + rr[0][0]) + (pr[0][1] + rr[0][1])) +
-                             ((pr[1][0] + rr[1][0]) + (pr[1][1] + rr[1][1]));
-                }
-            }
-#pragma unroll
-            for (int kp = 0; kp < KP; ++kp) {
-                uint32_t vc[4];
-                if constexpr (EARLY) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) vc[i] = vf[kp < (EARLY ? KP : 1) ? kp : 0][i];
-                } else {
-                    ldsm_x4_trans(addr(kp) + SLICE_BYTES, vc);
-                }
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {  // m-tile 2 kp + h
-                    const int mt = 2 * kp + h;
-                    uint32_t va[4];
-                    // (V[r0][2g], V[r0][2g+1], V[r1][2g], V[r1][2g+1]) ->
-                    // (V[r0][2g], V[r1][2g] | V[r0][2g+1], V[r1][2g+1])
-                    e4m3x4_to_f16x2(byte_perm(vc[2 * h], 0x3120u), va[0], va[1]);
-                    e4m3x4_to_f16x2(byte_perm(vc[2 * h + 1], 0x3120u), va[2], va[3]);
-                    if (partial) {
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int tk = (i >> 1) * 8 + 2 * t4;
-                            const uint32_t keep =
-                                (tk >= wlo && tk < wvalid ? 0x0000ffffu : 0u) |
-                                (tk + 1 >= wlo && tk + 1 < wvalid ? 0xffff0000u : 0u);
-                            va[i] &= keep;
-                        }
-                    }
-#pragma unroll
-                    for (int rb = 0; rb < RB; ++rb) {
-                        if (grew) {
-                            o[mt][rb][0] *= alpha_c[rb][0];
-                            o[mt][rb][1] *= alpha_c[rb][1];
-                            o[mt][rb][2] *= alpha_c[rb][0];
-                            o[mt][rb][3] *= alpha_c[rb][1];
-                        }
-                        if constexpr (PPB) {  // this page's P.V, then times its v_scale
-                            float d4[4] = {0.f, 0.f, 0.f, 0.f};
-                            mma_f16(d4, va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
-                            mma_f16(d4, va[0], va[1], va[2], va[3], pl[rb][0], pl[rb][1]);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) o[mt][rb][i] = fmaf(d4[i], vmul, o[mt][rb][i]);
-                        } else {
-                            mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
-                            mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pl[rb][0], pl[rb][1]);
-                        }
-                    }
-                }
-            }
+            e4m3_slice_math<D, NH, PPB, EARLY>(qa, m, l, o, kf, vf, addr, wvalid, wlo, kmul, vmul,
+                                               g, t4);
         };
         if (!EARLY && work) math();
         __syncwarp();  // the warp's reads of the stage are done: refill it
@@ -588,8 +617,11 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
     }
     __syncthreads();
     merge_warps_and_store<T, D, NH, NW>(
-        a, red, [&](int hh) { return (int64_t)b * a.num_q_heads + h0 + hh; }, nh,
-        sp.slot0 + part, sp.direct, tid, NW * 32);
+        a, red, [&](int hh) { return (int64_t)b * a.num_q_heads + h0 + hh; },
+        [&](int hh) {
+            return ((int64_t)b * a.num_q_heads + h0 + hh) * a.ws_slots + sp.slot0 + part;
+        },
+        nh, sp.direct, tid, NW * 32);
 }
 
 template <typename T, int D, int BS, int NH, int NW = 4, int STAGES = 0>
@@ -617,5 +649,11 @@ cudaError_t decode_mma_e4m3_f16(const DecodeArgs& a, int head_dim, int block_siz
                                 cudaStream_t stream);
 cudaError_t decode_mma_e4m3_bf16(const DecodeArgs& a, int head_dim, int block_size, int hg,
                                  cudaStream_t stream);
+// The planned decode over E4M3 pages on planned_ctas persistent CTAs of nw
+// warps (decode_stream_e4m3.cuh), or with occupancy != nullptr only the
+// resident CTAs per SM of that kernel.
+cudaError_t decode_stream_e4m3(const DecodeArgs& a, bool bf16, int head_dim, int block_size,
+                               int hg, int nw, int planned_ctas, int* occupancy,
+                               cudaStream_t stream);
 
 }  // namespace pkv

@@ -301,6 +301,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::THREAD
     extern __shared__ __align__(128) unsigned char smem_simt[];
     __shared__ float s_p[NW][HG][16];
     __shared__ volatile int s_abort;
+    const GroupPassWait group_pass_wait{a};
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kvh = blockIdx.y / a.head_chunks;
@@ -420,8 +421,9 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::THREAD
     W.template park<NW>(warp, red, a.v_scale && !a.scale_per_block ? a.v_scale[kvh] : 1.f);
     __syncthreads();
     merge_warps_and_store<T, D, HG, NW>(
-        a, red, [&](int hh) { return (int64_t)b * a.num_q_heads + h0 + hh; }, nh,
-        sp.slot0 + part, sp.direct, tid, NW * 32);
+        a, red, [&](int hh) { return (int64_t)b * a.num_q_heads + h0 + hh; },
+        [&](int hh) { return ((int64_t)b * a.num_q_heads + h0 + hh) * a.ws_slots + sp.slot0 + part; },
+        nh, sp.direct, tid, NW * 32);
 }
 
 template <typename T, int D, int BS, int HG, int NW = 4, int STAGES = 0, typename TC = T>
@@ -433,8 +435,8 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
     cudaError_t e = attr.ensure(kern, C::smem_bytes(8192));
     if (e != cudaSuccess) return e;
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
-    kern<<<grid, C::THREADS, smem_simt, stream>>>(a);
-    e = cudaGetLastError();
+    e = launch_decode_kernel(kern, grid, dim3(C::THREADS), smem_simt, stream, a.after_groups != 0,
+                             a);
     if (e != cudaSuccess || a.ws_slots <= 1) return e;
     return launch_lse_reduce<T, D>(a, stream);
 }

@@ -33,9 +33,9 @@ def test_header_constants_match_the_binding():
     """Every #define PKV_* number in include/*.h has the binding's value."""
     found = {}
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
-        for name, val in re.findall(r"^#define\s+(PKV_\w+)\s+\(?(\d+)u?", open(h).read(),
-                                    flags=re.M):
-            found[name] = int(val)
+        for name, val in re.findall(r"^#define\s+(PKV_\w+)\s+\(?(0x[0-9A-Fa-f]+|\d+)u?",
+                                    open(h).read(), flags=re.M):
+            found[name] = int(val, 0)
     assert {"PKV_DEV_BAD_BLOCK", "PKV_DEV_TIMEOUT", "PKV_DEV_DRAIN_TIMEOUT"} <= set(found)
     for name, val in found.items():
         if name == "PKV_STATIC_WORKSPACE_BYTES":

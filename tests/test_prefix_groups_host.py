@@ -15,7 +15,7 @@ def test_by_hand():
     # 0, 1, 2 share blocks 5, 6 (seq 2 holds 8 at position 2); 3, 4, 6 share
     # 1, 2 (seq 4 has only two full blocks); 5 has no full block
     assert spl.tolist() == [32, 32, 32, 32, 32, 0, 32]
-    assert members.tolist() == [[0, 1, 2] + [-1] * 13, [3, 4, 6] + [-1] * 13]
+    assert members.tolist() == [[0, 1, 2], [3, 4, 6]]
     # groups of at most 2: the leftover member of each bucket stays out
     spl, members = pkv.pkv_decode_prefix_groups(bt, lens, 16, max_group_size=2)
     assert members.tolist() == [[0, 1], [3, 4]]
@@ -23,7 +23,7 @@ def test_by_hand():
     # a prefix of at least 3 blocks: 0, 1, 2 share only two; seq 4 has only
     # two full blocks, so 3 and 6 share all four of theirs
     spl, members = pkv.pkv_decode_prefix_groups(bt, lens, 16, min_prefix_blocks=3)
-    assert members.tolist() == [[3, 6] + [-1] * 14]
+    assert members.tolist() == [[3, 6]]
     assert spl.tolist() == [0, 0, 0, 64, 0, 0, 64]
 
 
