@@ -326,8 +326,7 @@ class Workload:
     """One decode workload on the device: seeded inputs, the step (append of
     each sequence's new token + decode) and its byte counts."""
 
-    def __init__(self, args, cfg, kv: str, rank: int, partition: int, window: int,
-                 planned: bool = False):
+    def __init__(self, args, cfg, kv: str, rank: int, partition: int, window: int):
         import torch
 
         import paged_kv_cache_346_b200 as pkv
@@ -391,34 +390,15 @@ class Workload:
         self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
         self.Pused = P or pkv.pkv_decode_default_partition(B, H, span)
         self.launches_per_step = 1 + 1 + (1 if math.ceil(span / self.Pused) > 1 else 0)
-        # planned decode (E4M3 pages): a host plan over persistent CTAs, built
-        # once from the host lengths (they do not change from step to step)
-        self.planned = planned and e4m3
-        if planned and not e4m3:
-            raise SystemExit("the planned decode takes E4M3 pages")
-        if self.planned:
-            C = pkv.pkv_decode_planned_ctas(cfg.num_q_heads, H, D, bs, pkv.PKV_E4M3)
-            self.plan_np = pkv.pkv_decode_plan(inp.context_lens, cfg.num_q_heads, H, D, bs,
-                                               num_ctas=C, sliding_window=W, seq_order=order_np)
-            self.plan_dev = dev(self.plan_np)
-            self.plan_hdr = pkv.plan_header(self.plan_np)
-            self.ws = pkv.planned_workspace(self.plan_np, D)
-            self.Pused = self.plan_hdr["piece_tokens"]
-            self.launches_per_step = 1 + 1
         kvd = "e4m3" if e4m3 else None
         self.step_bytes = step_bytes(cfg, lens, W, kvd, per_page)
         self.dec_bytes = algorithmic_bytes(cfg, lens, W, kvd, per_page)
-        self.variant = resolve_variant(cfg, args.kernel, kv) + ("_planned" if self.planned else "")
+        self.variant = resolve_variant(cfg, args.kernel, kv)
         self.pkv = pkv
 
     def decode(self, stream):
         pkv, c = self.pkv, self.cfg
-        if self.planned:
-            pkv.pkv_paged_attention_decode_planned(
-                self.out, self.q, self.kc, self.vc, self.ks, self.vs, self.bt, self.cl,
-                self.plan_np, self.plan_dev, c.scale, c.block_size, workspace=self.ws,
-                stream=stream)
-        elif self.e4m3:
+        if self.e4m3:
             pkv.pkv_paged_attention_decode_e4m3(
                 self.out, self.q, self.kc, self.vc, self.ks, self.vs, self.bt, self.cl, c.scale,
                 c.block_size, self.mcl, partition_size=self.P, workspace=self.ws,
@@ -521,7 +501,7 @@ def run_ours(args, cfg):
         if world > 1:
             dist.barrier()
 
-    w = Workload(args, cfg, args.kv, rank, args.partition, args.window, args.planned)
+    w = Workload(args, cfg, args.kv, rank, args.partition, args.window)
     pkv = w.pkv
     B, H, D, bs = cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
     stream = torch.cuda.current_stream()
@@ -543,8 +523,6 @@ def run_ours(args, cfg):
               ("cl", w.cl)]
     if w.order is not None:
         fields.append(("order", w.order))
-    if w.planned:
-        fields.append(("plan", w.plan_dev))
     offs, total = {}, 0
     for name, t in fields:
         offs[name] = total
@@ -566,7 +544,6 @@ def run_ours(args, cfg):
         e.record(stream)
     c_stream = ctypes.c_void_p(stream.cuda_stream)
     dt_code = pkv.torch_dtype_code(q.dtype)
-    hdr_np = np.ascontiguousarray(w.plan_np[:16]) if w.planned else None
     N_blocks = kc.shape[0]
     P, W, mcl = w.P, w.W, w.mcl
     calls = []
@@ -578,16 +555,10 @@ def run_ours(args, cfg):
             spb = 1 if w.per_page else 0
             append_args = (kp, vp, ptr["knew"], ptr["vnew"], ksp, vsp, spb, ptr["slots"], B, H, D,
                            bs, N_blocks, dt_code, c_stream)
-            if w.planned:
-                decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ksp, vsp,
-                               spb, ptr["bt"], ptr["cl"], ptr["plan"], hdr_np.ctypes.data, B,
-                               cfg.num_q_heads, H, D, bs, w.bt.shape[1], N_blocks, cfg.scale,
-                               dt_code, ctypes.c_void_p(ws.data_ptr()), ws.numel(), c_stream)
-            else:
-                decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ksp, vsp,
-                               spb, ptr["bt"], ptr["cl"], ptr.get("order"), B, cfg.num_q_heads,
-                               H, D, bs, w.bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
-                               ctypes.c_void_p(ws.data_ptr()), ws.numel(), w.kern, c_stream)
+            decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ksp, vsp,
+                           spb, ptr["bt"], ptr["cl"], ptr.get("order"), B, cfg.num_q_heads,
+                           H, D, bs, w.bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
+                           ctypes.c_void_p(ws.data_ptr()), ws.numel(), w.kern, c_stream)
         else:
             append_args = (kp, vp, ptr["knew"], ptr["vnew"], ptr["slots"], B, H, D, bs,
                            N_blocks, dt_code, c_stream)
@@ -597,8 +568,7 @@ def run_ours(args, cfg):
                            ctypes.c_void_p(ws.data_ptr()), ws.numel(), w.kern, c_stream)
         calls.append((append_args, decode_args))
     c_append = pkv.lib.pkv_kv_cache_append_e4m3 if w.e4m3 else pkv.lib.pkv_kv_cache_append
-    c_decode = (pkv.lib.pkv_paged_attention_decode_planned if w.planned else
-                pkv.lib.pkv_paged_attention_decode_e4m3 if w.e4m3
+    c_decode = (pkv.lib.pkv_paged_attention_decode_e4m3 if w.e4m3
                 else pkv.lib.pkv_paged_attention_decode)
 
     def e2e_step(i):
@@ -640,12 +610,11 @@ def run_ours(args, cfg):
     # ---- the other workloads the targets name, measured the same way
     also = []
     for spec in ([] if args.also == "none" else args.also.split(",")):
-        name, kv, mode = (spec.split(":") + ["", ""])[:3]
+        name, _, kv = spec.partition(":")
         kv = kv or "same"
-        if name == cfg.name and kv == args.kv and (mode == "planned") == args.planned:
+        if name == cfg.name and kv == args.kv:
             continue
-        w2 = Workload(args, CONFIGS[name], kv, rank, CONFIGS[name].partition_size, 0,
-                      mode == "planned")
+        w2 = Workload(args, CONFIGS[name], kv, rank, CONFIGS[name].partition_size, 0)
         b2, d2, c2 = time_blocks(w2, args.steps, args.warmup, args.min_time, barrier, local)
         m2, dm2 = median_block(b2, d2)
         m2, dm2 = max_over_ranks([m2, dm2], world)
@@ -666,8 +635,7 @@ def run_ours(args, cfg):
             "dtype": "e4m3" if w.e4m3 else cfg.dtype, "data": "synthetic",
             "config": workload_config(cfg, w.lens, world, args.tables, w.W, args.kv),
             "impl_config": {"partition_size": w.Pused, "kernel": args.kernel,
-                            "schedule": ("host plan, persistent CTAs" if w.planned else
-                                         "longest-first" if args.order else "batch order")},
+                            "schedule": "longest-first" if args.order else "batch order"},
             "timing": {"blocks": len(blocks), "steps_per_block": args.steps,
                        "block_ms_median": round(ms, 4), "block_ms_min": round(min(blocks), 4),
                        "block_ms_max": round(max(blocks), 4),
@@ -692,9 +660,7 @@ def run_ours(args, cfg):
                 line["also"].append({
                     "config": workload_config(w2.cfg, w2.lens, world, args.tables, 0, w2.kv),
                     "impl_config": {"partition_size": w2.Pused, "kernel": args.kernel,
-                                    "schedule": ("host plan, persistent CTAs" if w2.planned else
-                                                 "longest-first" if args.order else
-                                                 "batch order")},
+                                    "schedule": "longest-first" if args.order else "batch order"},
                     "value": round(v2, 2), "unit": "GB/s", "ms_per_step": round(st, 5),
                     "tokens_per_s": round(world * w2.cfg.num_seqs / (st * 1e-3), 1),
                     "pct_of_hbm_peak": round(100 * v2 / world / peak, 2),
@@ -984,8 +950,6 @@ def main():
                     help="seconds of oracle work for the cpu_baseline field")
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="seconds of oracle work for --impl reference")
-    ap.add_argument("--planned", action="store_true",
-                    help="E4M3 pages: the planned decode (host plan over persistent CTAs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--min-time", type=float, default=0.5,
                     help="time blocks of --steps steps until at least this many seconds of "

@@ -95,7 +95,6 @@ typedef enum { PKV_KERNEL_AUTO = 0, PKV_KERNEL_SIMT = 1, PKV_KERNEL_MMA = 2 } pk
                                      when the kernel's block left (see below) */
 #define PKV_DEV_BAD_GROUP 64u   /* a shared-prefix group whose members disagree
                                    (prefix length, table entries) */
-#define PKV_DEV_BAD_PLAN 128u   /* a planned-decode item that does not fit its batch */
 /*
  * After PKV_DEV_TIMEOUT the outputs of that call are lost (the blocks whose
  * wait gave up wrote nothing).  With PKV_DEV_DRAIN_TIMEOUT as well, a page
@@ -357,110 +356,6 @@ PKV_API int pkv_decode_prefix_groups(const int32_t* block_tables, const int32_t*
                                      int max_group_size, int min_prefix_blocks,
                                      int32_t* seq_prefix_len, int32_t* group_members,
                                      int group_capacity, int* num_groups);
-
-/* ------------------------------------------------------------------------
- * Planned decode: the same attention as pkv_paged_attention_decode_e4m3,
- * with the work laid out on the host from host-side lengths.  The attended
- * tokens of every (sequence, KV head, tile of query heads) unit are cut into
- * pieces and spread over a fixed number of persistent CTAs, largest first,
- * each to the least loaded CTA.  Every warp of a CTA then streams its share
- * of the CTA's pieces (slices of 16 tokens) through its own ring without
- * waiting for the other warps -- the next piece's table and first pages are
- * fetched while it works on the current one -- and leaves a partial softmax
- * state per piece in the workspace; the warp that completes a unit merges
- * them and writes the output rows.  Against one CTA per (sequence, KV head,
- * partition): no set-up between pieces, no CTA per empty partition, no long
- * partition setting the kernel's length, no reduce kernel.  E4M3 pages,
- * query groups of at most 16 heads per KV head, head_dim 128 or 256.
- * ------------------------------------------------------------------------ */
-#define PKV_PLAN_MAGIC 0x324E4C50      /* "PLN2" */
-#define PKV_PLAN_HEADER_WORDS 16
-#define PKV_PLAN_ITEM_WORDS 16
-
-/* The plan's first PKV_PLAN_HEADER_WORDS int32 words. */
-typedef struct {
-    int32_t magic;           /* PKV_PLAN_MAGIC */
-    int32_t num_ctas;        /* persistent CTAs of the decode */
-    int32_t num_items;       /* pieces */
-    int32_t num_merges;      /* units cut into more than one piece (information) */
-    int32_t num_slots;       /* workspace slots: pieces x warps per CTA */
-    int32_t num_seqs;
-    int32_t num_q_heads;
-    int32_t num_kv_heads;
-    int32_t heads_per_cta;   /* query heads of one tile: 8 or 16 */
-    int32_t head_chunks;     /* tiles per KV head */
-    int32_t block_size;
-    int32_t sliding_window;
-    int32_t piece_tokens;    /* at most this many tokens per piece, a multiple of 64 */
-    int32_t words;           /* int32 words of the whole plan */
-    int32_t max_cta_tokens;  /* the most loaded CTA's work, in tokens plus a share per piece */
-    int32_t warps_per_cta;   /* 2 (one head per KV head at head_dim 128) or 4 */
-} pkv_decode_plan_header;
-
-/*
- * Build a plan (host).  context_lens: host int32 [num_seqs] (the lengths the
- * decode will see); seq_order: NULL or a host permutation (pieces of earlier
- * sequences come first among equal sizes).  num_q_heads / num_kv_heads <= 16;
- * head_dim 128 or 256; sliding_window as in pkv_paged_attention_decode;
- * num_ctas > 0 (to fill the GPU: pkv_decode_planned_ctas); piece_tokens 0 =
- * automatic (about one CTA's share, at least 256), else a multiple of 64 up
- * to 512 x warps per CTA (1024 or 2048).
- * *header gets the plan's header (also when plan is NULL: a size query);
- * with plan != NULL the plan is written there, plan_capacity int32 words
- * (PKV_EBOUNDS when header->words is more).  Returns PKV_OK, PKV_EINVAL or
- * PKV_EBOUNDS.
- *
- * Plan layout after the header: cta_begin[num_ctas + 1] (CTA c runs items
- * [cta_begin[c], cta_begin[c + 1])); items[num_items][16] = (sequence,
- * KV head * head_chunks + tile, first token, end token, tokens masked at the
- * start (before a sliding window), unit (its sequence and tile in schedule
- * order), the unit's first workspace slot, the unit's pieces, this piece's
- * index in the unit, then zeros).  Warp w writes slot first + index *
- * warps_per_cta + w.
- */
-PKV_API int pkv_decode_plan(const int32_t* context_lens, const int32_t* seq_order,
-                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                            int block_size, int sliding_window, int num_ctas, int piece_tokens,
-                            int32_t* plan, size_t plan_capacity, pkv_decode_plan_header* header);
-
-/*
- * CTAs that fill the current GPU for the planned decode of this shape
- * (SMs x resident CTAs per SM of the kernel it will run), or 0 for a shape
- * the planned decode does not take.  kv_dtype: PKV_E4M3.
- */
-PKV_API int pkv_decode_planned_ctas(int num_q_heads, int num_kv_heads, int head_dim,
-                                    int block_size, pkv_dtype kv_dtype);
-
-/*
- * Workspace bytes of the planned decode: one int32 counter per unit
- * (num_seqs x num_kv_heads x head_chunks, padded to 256 bytes), then float32
- * partial states, one per slot and query head of a tile.  The counters must
- * be zero before the first call on a workspace (allocate it zero-filled);
- * every call leaves them zero -- except one that set PKV_DEV_TIMEOUT or
- * PKV_DEV_BAD_PLAN, after which the workspace must be zero-filled again.
- */
-PKV_API size_t pkv_decode_planned_workspace_size(const pkv_decode_plan_header* header,
-                                                 int head_dim);
-
-/*
- * The planned decode.  Arguments as pkv_paged_attention_decode_e4m3, plus:
- *   plan: device copy of a plan from pkv_decode_plan; header: host copy of
- *       its header (the launch is sized from it).  The plan must describe
- *       this batch (its lengths, sliding window and schedule); a piece with
- *       a field out of range is skipped and flagged (PKV_DEV_BAD_PLAN), and
- *       its unit's rows are then left unwritten.
- *   workspace: pkv_decode_planned_workspace_size(header, head_dim) bytes,
- *       16-byte aligned, counters zero (above).  Calls sharing a workspace
- *       must not overlap on the GPU.
- * Returns PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED or PKV_ECUDA.
- */
-PKV_API int pkv_paged_attention_decode_planned(
-    void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
-    const float* v_scale, int scale_per_block, const int32_t* block_tables,
-    const int32_t* context_lens, const int32_t* plan, const pkv_decode_plan_header* header,
-    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-    int max_blocks_per_seq, int num_blocks, float scale, pkv_dtype dtype, void* workspace,
-    size_t workspace_bytes, pkv_stream_t stream);
 
 /*
  * Host helper: order_out[0..n) = the sequence indices sorted by decreasing

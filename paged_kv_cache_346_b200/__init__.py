@@ -20,7 +20,7 @@ import torch
 
 from . import _binding as _b
 from ._binding import (PKV_BF16, PKV_E4M3, PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD_ORDER,
-                       PKV_DEV_BAD_GROUP, PKV_DEV_BAD_PLAN, PKV_DEV_BAD_SLOT, PKV_DEV_DRAIN_TIMEOUT, PKV_DEV_TIMEOUT,
+                       PKV_DEV_BAD_GROUP, PKV_DEV_BAD_SLOT, PKV_DEV_DRAIN_TIMEOUT, PKV_DEV_TIMEOUT,
                        PKV_F16, PKV_F32,
                        PKV_KERNEL_AUTO, PKV_KERNEL_MMA, PKV_KERNEL_SIMT, PagedKVError, check, lib)
 
@@ -34,10 +34,7 @@ __all__ = [
     "torch_dtype_code",
     "pkv_decode_schedule_order", "pkv_paged_attention_decode_e4m3", "pkv_kv_cache_append_e4m3",
     "pkv_paged_attention_decode_prefix_groups", "pkv_decode_prefix_groups",
-    "pkv_decode_prefix_groups_workspace_size", "PKV_DEV_BAD_GROUP", "PKV_DEV_BAD_PLAN",
-    "pkv_decode_plan", "plan_header", "pkv_decode_planned_ctas",
-    "pkv_decode_planned_workspace_size", "pkv_paged_attention_decode_planned",
-    "planned_workspace",
+    "pkv_decode_prefix_groups_workspace_size", "PKV_DEV_BAD_GROUP",
     "PKV_E4M3", "pkv_debug_wait_timeout",
 ]
 
@@ -285,94 +282,6 @@ def pkv_paged_attention_decode_prefix_groups(
         block_tables.shape[1], N, int(max_context_len), int(max_prefix_len), float(scale),
         torch_dtype_code(q.dtype), int(partition_size), _ptr(workspace), ws_bytes, int(kernel),
         _stream(stream)), "pkv_paged_attention_decode_prefix_groups")
-    return out
-
-
-PLAN_HEADER_FIELDS = ("magic", "num_ctas", "num_items", "num_merges", "num_slots", "num_seqs",
-                      "num_q_heads", "num_kv_heads", "heads_per_cta", "head_chunks",
-                      "block_size", "sliding_window", "piece_tokens", "words",
-                      "max_cta_tokens", "warps_per_cta")
-
-
-def pkv_decode_plan(context_lens, num_q_heads: int, num_kv_heads: int, head_dim: int,
-                    block_size: int, *, num_ctas: int, sliding_window: int = 0, seq_order=None,
-                    piece_tokens: int = 0):
-    """Host int32 plan of the planned decode (pkv_decode_plan in pagedkv.h) from
-    host lengths.  -> numpy int32 array; its first 16 words are the header
-    (PLAN_HEADER_FIELDS)."""
-    import numpy as np
-    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
-    order = None if seq_order is None else np.ascontiguousarray(seq_order, dtype=np.int32)
-    hdr = np.zeros(_b.PKV_PLAN_HEADER_WORDS, dtype=np.int32)
-    args = [lens.ctypes.data if lens.size else None,
-            None if order is None else order.ctypes.data, lens.size, num_q_heads, num_kv_heads,
-            head_dim, block_size, sliding_window, num_ctas, piece_tokens]
-    check(lib.pkv_decode_plan(*args, None, 0, hdr.ctypes.data), "pkv_decode_plan")
-    plan = np.zeros(int(hdr[13]), dtype=np.int32)
-    check(lib.pkv_decode_plan(*args, plan.ctypes.data, plan.size, hdr.ctypes.data),
-          "pkv_decode_plan")
-    return plan
-
-
-def plan_header(plan) -> dict:
-    return {k: int(v) for k, v in zip(PLAN_HEADER_FIELDS, plan[:_b.PKV_PLAN_HEADER_WORDS])}
-
-
-def pkv_decode_planned_ctas(num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
-                            kv_dtype: int = PKV_E4M3) -> int:
-    return int(lib.pkv_decode_planned_ctas(num_q_heads, num_kv_heads, head_dim, block_size,
-                                           kv_dtype))
-
-
-def pkv_decode_planned_workspace_size(plan, head_dim: int) -> int:
-    import numpy as np
-    hdr = np.ascontiguousarray(plan[:_b.PKV_PLAN_HEADER_WORDS], dtype=np.int32)
-    return int(lib.pkv_decode_planned_workspace_size(hdr.ctypes.data, head_dim))
-
-
-def planned_workspace(plan, head_dim: int, device="cuda") -> torch.Tensor:
-    """A zero-filled workspace for the planned decode (its unit counters must
-    start at zero; every call leaves them so)."""
-    return torch.zeros(max(16, pkv_decode_planned_workspace_size(plan, head_dim)),
-                       dtype=torch.uint8, device=device)
-
-
-def pkv_paged_attention_decode_planned(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
-                                       v_cache: torch.Tensor, k_scale: torch.Tensor | None,
-                                       v_scale: torch.Tensor | None, block_tables: torch.Tensor,
-                                       context_lens: torch.Tensor, plan_host, plan_dev: torch.Tensor,
-                                       scale: float, block_size: int, *,
-                                       workspace: torch.Tensor | None = None,
-                                       stream=None) -> torch.Tensor:
-    """out [B, Hq, D] <- the planned decode (pkv_paged_attention_decode_planned
-    in pagedkv.h).  plan_host: the numpy plan (its header sizes the launch);
-    plan_dev: its device copy (int32).  E4M3 pages with k_scale / v_scale
-    ([Hkv] per head or [N, Hkv] per page).  workspace: planned_workspace(...)
-    (zero-filled once, reused call after call)."""
-    import numpy as np
-    for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
-                 (block_tables, "block_tables"), (context_lens, "context_lens"),
-                 (plan_dev, "plan")):
-        _dev(t, n)
-    B, Hq, D = q.shape
-    N, Hkv, bs, D2 = k_cache.shape
-    if D2 != D or bs != block_size or tuple(out.shape) != (B, Hq, D):
-        raise PagedKVError(_b.PKV_EINVAL, "shape mismatch")
-    per_page = 0
-    if k_scale is not None:
-        _dev(k_scale, "k_scale")
-        _dev(v_scale, "v_scale")
-        per_page = 1 if k_scale.dim() == 2 else 0
-    hdr = np.ascontiguousarray(plan_host[:_b.PKV_PLAN_HEADER_WORDS], dtype=np.int32)
-    ws_bytes = 0
-    if workspace is not None:
-        _dev(workspace, "workspace")
-        ws_bytes = workspace.numel() * workspace.element_size()
-    check(lib.pkv_paged_attention_decode_planned(
-        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), per_page,
-        _ptr(block_tables), _ptr(context_lens), _ptr(plan_dev), hdr.ctypes.data, B, Hq, Hkv, D,
-        bs, block_tables.shape[1], N, float(scale), torch_dtype_code(q.dtype), _ptr(workspace),
-        ws_bytes, _stream(stream)), "pkv_paged_attention_decode_planned")
     return out
 
 

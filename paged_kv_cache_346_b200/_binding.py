@@ -18,10 +18,9 @@ PKV_OK, PKV_EINVAL, PKV_ENOMEM, PKV_ENOSEQ, PKV_EEXIST, PKV_EBOUNDS, PKV_ECUDA, 
 PKV_F32, PKV_F16, PKV_BF16, PKV_E4M3 = 0, 1, 2, 3
 PKV_KERNEL_AUTO, PKV_KERNEL_SIMT, PKV_KERNEL_MMA = 0, 1, 2
 PKV_DEV_BAD_BLOCK, PKV_DEV_BAD_LEN, PKV_DEV_BAD_SLOT, PKV_DEV_TIMEOUT, PKV_DEV_BAD_ORDER, \
-    PKV_DEV_DRAIN_TIMEOUT, PKV_DEV_BAD_GROUP, PKV_DEV_BAD_PLAN = 1, 2, 4, 8, 16, 32, 64, 128
+    PKV_DEV_DRAIN_TIMEOUT, PKV_DEV_BAD_GROUP = 1, 2, 4, 8, 16, 32, 64
 PKV_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024
 PKV_MAX_PREFIX_GROUP = 64
-PKV_PLAN_MAGIC, PKV_PLAN_HEADER_WORDS, PKV_PLAN_ITEM_WORDS = 0x324E4C50, 16, 16
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is not built; run `python paged_kv_cache_346_b200/build.py`")
@@ -56,13 +55,6 @@ SIGNATURES = {
     "pkv_decode_prefix_groups_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
     "pkv_decode_prefix_groups": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32,
                                         _vp]),
-    "pkv_decode_plan": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp,
-                               _sz, _vp]),
-    "pkv_decode_planned_ctas": (_i32, [_i32, _i32, _i32, _i32, _i32]),
-    "pkv_decode_planned_workspace_size": (_sz, [_vp, _i32]),
-    "pkv_paged_attention_decode_planned": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
-                                                  _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
-                                                  _i32, _f32, _i32, _vp, _sz, _vp]),
     "pkv_kv_cache_append": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                    _vp]),
     "pkv_kv_cache_append_e4m3": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32,

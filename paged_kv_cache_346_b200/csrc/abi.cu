@@ -188,7 +188,7 @@ int plan_decode(const DecodeRequest& r, DecodePlan* plan) {
 
 namespace {
 
-// Kernel arguments of a planned decode whose workspace rows hold ws_slots
+// Kernel arguments of a checked decode call whose workspace rows hold ws_slots
 // partial results.
 DecodeArgs decode_args(const DecodeRequest& r, const DecodePlan& plan, void* workspace,
                        int ws_slots) {
@@ -207,8 +207,6 @@ DecodeArgs decode_args(const DecodeRequest& r, const DecodePlan& plan, void* wor
     a.group_members = nullptr;
     a.group_stride = 0;
     a.after_groups = 0;
-    a.plan_cta = a.plan_items = nullptr;
-    a.plan_counts = nullptr;
     a.ws_slots = ws_slots;
     a.ws_o = static_cast<float*>(workspace);
     a.ws_ml = ws_slots > 1
@@ -232,7 +230,7 @@ DecodeArgs decode_args(const DecodeRequest& r, const DecodePlan& plan, void* wor
 }
 
 // The partition kernel the plan chose (and the reduce when rows merge).
-int launch_planned(const DecodeRequest& r, const DecodePlan& plan, const DecodeArgs& a,
+int launch_decode_kernels(const DecodeRequest& r, const DecodePlan& plan, const DecodeArgs& a,
                    cudaStream_t s) {
     const int D = r.head_dim, bs = r.block_size, hg = plan.heads_per_cta;
     cudaError_t e;
@@ -265,7 +263,7 @@ int run_decode(const DecodeRequest& r, const DecodePlan& plan, void* workspace,
         return PKV_EINVAL;
     DecodeArgs a = decode_args(r, plan, workspace, plan.max_partitions);
     if (status_word(&a.status) != cudaSuccess) return PKV_ECUDA;
-    return launch_planned(r, plan, a, s);
+    return launch_decode_kernels(r, plan, a, s);
 }
 
 namespace {
@@ -328,7 +326,7 @@ int prefix_groups_impl(const DecodeRequest& r, const int32_t* seq_prefix_len,
         if (e != cudaSuccess) return PKV_ECUDA;
         a.after_groups = 1;  // overlap the regular pass with the group pass's last wave
     }
-    return launch_planned(r, plan, a, s);
+    return launch_decode_kernels(r, plan, a, s);
 }
 
 // The decode behind both caller-workspace entry points.
@@ -467,88 +465,6 @@ int pkv_paged_attention_decode_prefix_groups(
     return pkv::prefix_groups_impl(r, seq_prefix_len, group_members, num_groups, max_group_size,
                                    max_prefix_len, workspace, workspace_bytes,
                                    reinterpret_cast<cudaStream_t>(stream));
-}
-
-int pkv_decode_planned_ctas(int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                            pkv_dtype kv_dtype) {
-    if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
-        num_q_heads / num_kv_heads > 16 || kv_dtype != PKV_E4M3 ||
-        (head_dim != 128 && head_dim != 256) ||
-        (block_size != 16 && block_size != 32 && block_size != 64))
-        return 0;
-    DecodeArgs a = {};
-    a.group = num_q_heads / num_kv_heads;
-    const int hg = a.group <= 8 ? 8 : 16;
-    const int nw = head_dim == 128 && a.group == 1 ? 2 : 4;
-    int occ = 0, dev = 0, sms = 0;
-    if (decode_stream_e4m3(a, false, head_dim, block_size, hg, nw, 0, &occ, nullptr) !=
-            cudaSuccess ||
-        cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-        cudaGetLastError();
-        return 0;
-    }
-    return occ * sms;
-}
-
-namespace {
-int64_t plan_units(const pkv_decode_plan_header* h) {
-    return (int64_t)h->num_seqs * h->num_kv_heads * h->head_chunks;
-}
-}  // namespace
-
-size_t pkv_decode_planned_workspace_size(const pkv_decode_plan_header* h, int head_dim) {
-    if (!h || h->magic != PKV_PLAN_MAGIC || h->num_slots < 0 || h->num_seqs < 0 ||
-        h->num_kv_heads <= 0 || h->head_chunks <= 0 || h->heads_per_cta <= 0 || head_dim <= 0)
-        return 0;
-    const size_t counters = (size_t)(plan_units(h) + 63) / 64 * 256;
-    return counters + (size_t)h->num_slots * h->heads_per_cta * (head_dim + 2) * sizeof(float);
-}
-
-int pkv_paged_attention_decode_planned(
-    void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
-    const float* v_scale, int scale_per_block, const int32_t* block_tables,
-    const int32_t* context_lens, const int32_t* plan, const pkv_decode_plan_header* h,
-    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-    int max_blocks_per_seq, int num_blocks, float scale, pkv_dtype dtype, void* workspace,
-    size_t workspace_bytes, pkv_stream_t stream) {
-    NvtxRange range("pkv_paged_attention_decode_planned");
-    if (!h || h->magic != PKV_PLAN_MAGIC || h->num_seqs != num_seqs ||
-        h->num_q_heads != num_q_heads || h->num_kv_heads != num_kv_heads ||
-        h->block_size != block_size || h->num_ctas <= 0 || h->num_items < 0 ||
-        h->num_slots < 0 || h->piece_tokens <= 0 || h->piece_tokens % 64 != 0 ||
-        h->piece_tokens > 512 * h->warps_per_cta ||
-        h->warps_per_cta != (head_dim == 128 && num_q_heads == num_kv_heads ? 2 : 4))
-        return PKV_EINVAL;
-    if (!k_scale || !v_scale) return PKV_EUNSUPPORTED;  // the planned kernel reads E4M3 pages
-    // the regular decode's checks of the batch (sizes, pointers, types)
-    const DecodeRequest r{out, q, k_cache, v_cache, k_scale, v_scale, scale_per_block, true,
-                          block_tables, context_lens, nullptr, num_seqs, num_q_heads,
-                          num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
-                          max_blocks_per_seq * block_size, scale, h->sliding_window, dtype,
-                          h->piece_tokens, PKV_KERNEL_MMA};
-    DecodePlan p;
-    const int rc = plan_decode(r, &p);
-    if (rc != PKV_OK || p.empty) return rc;
-    if (p.heads_per_cta != h->heads_per_cta || p.head_chunks != h->head_chunks || !plan)
-        return PKV_EINVAL;
-    const size_t need = pkv_decode_planned_workspace_size(h, head_dim);
-    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PKV_EINVAL;
-    DecodeArgs a = decode_args(r, p, nullptr, h->num_slots);
-    if (status_word(&a.status) != cudaSuccess) return PKV_ECUDA;
-    a.plan_cta = plan + PKV_PLAN_HEADER_WORDS;
-    a.plan_items = a.plan_cta + h->num_ctas + 1;
-    a.plan_counts = static_cast<int32_t*>(workspace);
-    const size_t counters = (size_t)(plan_units(h) + 63) / 64 * 256;
-    a.ws_ml = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + counters);
-    a.ws_o = a.ws_ml + (int64_t)h->num_slots * h->heads_per_cta * 2;
-    a.partition_size = h->piece_tokens;
-    a.max_partitions = 1;
-    const cudaError_t e = decode_stream_e4m3(a, dtype == PKV_BF16, head_dim, block_size,
-                                             h->heads_per_cta, h->warps_per_cta, h->num_ctas,
-                                             nullptr, reinterpret_cast<cudaStream_t>(stream));
-    if (e == cudaErrorInvalidValue) return PKV_EUNSUPPORTED;
-    return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
 
 int pkv_kv_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,

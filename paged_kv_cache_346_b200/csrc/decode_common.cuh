@@ -38,9 +38,6 @@ struct DecodeArgs {
     int max_tokens;               // max_blocks_per_seq * BS
     int partition_size;           // tokens per partition
     int max_partitions;           // grid.x = ceil(longest attended span / partition_size)
-    const int32_t* plan_cta;      // planned decode: [grid + 1] item ranges of the CTAs
-    const int32_t* plan_items;    // [items][PKV_PLAN_ITEM_WORDS] pieces
-    int32_t* plan_counts;         // [units] warps counted in per unit, zero between calls
     int ws_slots;                 // partial results per row in the workspace
     int group_stride;             // group_members row length
     int after_groups;             // launched as a programmatic dependent of the group pass

@@ -1,5 +1,5 @@
 // Tensor-core paged decode over E4M3 pages: instantiations.
-#include "decode_stream_e4m3.cuh"
+#include "decode_mma_e4m3.cuh"
 
 namespace pkv {
 
@@ -47,57 +47,6 @@ cudaError_t decode_mma_e4m3_f16(const DecodeArgs& a, int head_dim, int block_siz
 cudaError_t decode_mma_e4m3_bf16(const DecodeArgs& a, int head_dim, int block_size, int hg,
                                  cudaStream_t stream) {
     return dispatch_mma_e4m3<__nv_bfloat16>(a, head_dim, block_size, hg, stream);
-}
-
-// The planned decode: the same CTA shapes and ring depths as the regular
-// grid's (2 warps for one live head at head_dim 128, else 4; 3-stage rings
-// for 8-head tiles at head_dim 128).
-template <typename T, int D, int BS, int NH, int NW, int STAGES>
-static cudaError_t launch_stream(const DecodeArgs& a, int ctas, int* occupancy,
-                                 cudaStream_t stream) {
-    using S = StreamCfg<D, BS, NW, STAGES>;
-    static SmemAttr attr[2];
-    auto kern = a.scale_per_block ? decode_stream_e4m3_kernel<T, D, BS, NH, NW, STAGES, true>
-                                  : decode_stream_e4m3_kernel<T, D, BS, NH, NW, STAGES, false>;
-    cudaError_t e = attr[a.scale_per_block ? 1 : 0].ensure(kern, S::SMEM);
-    if (e != cudaSuccess) return e;
-    if (occupancy)
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kern, NW * 32, S::SMEM);
-    const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
-    CUtensorMap tk, tv;
-    e = make_cache_tensor_map(&tk, a.k_cache, 1, false, D, rows, 16);
-    if (e != cudaSuccess) return e;
-    e = make_cache_tensor_map(&tv, a.v_cache, 1, false, D, rows, 16);
-    if (e != cudaSuccess) return e;
-    kern<<<ctas, NW * 32, S::SMEM, stream>>>(a, tk, tv);
-    return cudaGetLastError();
-}
-
-template <typename T>
-static cudaError_t dispatch_stream(const DecodeArgs& a, int head_dim, int block_size, int nh,
-                                   int nw, int ctas, int* occupancy, cudaStream_t stream) {
-#define PKV_ST_CASE(D_, BS_, NH_, NW_)                                                  \
-    if (head_dim == D_ && block_size == BS_ && nh == NH_ && nw == NW_)                  \
-        return launch_stream<T, D_, BS_, NH_, NW_, (D_ == 128 && NH_ == 8) ? 3 : 0>(a, ctas, \
-                                                                                occupancy, stream);
-#define PKV_ST_NH(D_, BS_, NW_) PKV_ST_CASE(D_, BS_, 8, NW_) PKV_ST_CASE(D_, BS_, 16, NW_)
-#define PKV_ST_BS(D_, NW_) PKV_ST_NH(D_, 16, NW_) PKV_ST_NH(D_, 32, NW_) PKV_ST_NH(D_, 64, NW_)
-    PKV_ST_BS(128, 2)
-    PKV_ST_BS(128, 4)
-    PKV_ST_BS(256, 4)
-#undef PKV_ST_BS
-#undef PKV_ST_NH
-#undef PKV_ST_CASE
-    return cudaErrorInvalidValue;
-}
-
-cudaError_t decode_stream_e4m3(const DecodeArgs& a, bool bf16, int head_dim, int block_size,
-                               int hg, int nw, int planned_ctas, int* occupancy,
-                               cudaStream_t stream) {
-    return bf16 ? dispatch_stream<__nv_bfloat16>(a, head_dim, block_size, hg, nw, planned_ctas,
-                                                 occupancy, stream)
-                : dispatch_stream<__half>(a, head_dim, block_size, hg, nw, planned_ctas,
-                                          occupancy, stream);
 }
 
 }  // namespace pkv

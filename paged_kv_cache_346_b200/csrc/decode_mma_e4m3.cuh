@@ -649,11 +649,4 @@ cudaError_t decode_mma_e4m3_f16(const DecodeArgs& a, int head_dim, int block_siz
                                 cudaStream_t stream);
 cudaError_t decode_mma_e4m3_bf16(const DecodeArgs& a, int head_dim, int block_size, int hg,
                                  cudaStream_t stream);
-// The planned decode over E4M3 pages on planned_ctas persistent CTAs of nw
-// warps (decode_stream_e4m3.cuh), or with occupancy != nullptr only the
-// resident CTAs per SM of that kernel.
-cudaError_t decode_stream_e4m3(const DecodeArgs& a, bool bf16, int head_dim, int block_size,
-                               int hg, int nw, int planned_ctas, int* occupancy,
-                               cudaStream_t stream);
-
 }  // namespace pkv

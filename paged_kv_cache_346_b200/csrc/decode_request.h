@@ -55,7 +55,7 @@ struct DecodePlan {
 // PKV_EINVAL or PKV_EUNSUPPORTED; nothing is launched.
 int plan_decode(const DecodeRequest& r, DecodePlan* plan);
 
-// Launches the planned decode with `workspace` (at least plan.workspace_bytes
+// Launches the decode the plan describes, with `workspace` (at least plan.workspace_bytes
 // of device memory, 16-byte aligned, when that is non-zero; checked).
 int run_decode(const DecodeRequest& r, const DecodePlan& plan, void* workspace,
                size_t workspace_bytes, cudaStream_t stream);
