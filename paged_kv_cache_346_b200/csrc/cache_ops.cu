@@ -40,6 +40,9 @@ __global__ void __launch_bounds__(256) kv_append_kernel(uint4* __restrict__ kc,
                                                          int head_vecs, int num_kv_heads,
                                                          int block_size, int64_t num_slots,
                                                          unsigned int* status) {
+    // the decode that usually follows waits for this grid to finish anyway:
+    // let it launch (and set up) while the appends run
+    pdl_launch_dependents();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total_vecs; i += stride) {
         const int64_t t = i / row_vecs;
@@ -73,6 +76,7 @@ __global__ void __launch_bounds__(256) kv_append_e4m3_kernel(
     const uint4* __restrict__ v, const float* __restrict__ ks, const float* __restrict__ vs,
     const int64_t* __restrict__ slots, int64_t total_vecs, int row_vecs, int head_vecs,
     int num_kv_heads, int block_size, int64_t num_slots, int per_block, unsigned int* status) {
+    pdl_launch_dependents();  // as kv_append_kernel
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total_vecs; i += stride) {
         const int64_t t = i / row_vecs;

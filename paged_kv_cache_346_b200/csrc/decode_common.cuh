@@ -362,15 +362,13 @@ struct GroupPassWait {
     }
 };
 
-// Launch a decode kernel; with after_groups as a programmatic dependent of
-// the kernel before it in the stream (the group pass).
+// Launch a decode kernel as a programmatic dependent of the kernel before it
+// in the stream: its CTAs may become resident while that kernel (the KV
+// append, or the group pass) runs, and wait in griddepcontrol.wait before
+// reading anything (or, after the group pass, only before they leave).
 template <typename K, typename... Args>
 cudaError_t launch_decode_kernel(K kernel, dim3 grid, dim3 block, int smem, cudaStream_t stream,
-                                 bool after_groups, Args... args) {
-    if (!after_groups) {
-        kernel<<<grid, block, smem, stream>>>(args...);
-        return cudaGetLastError();
-    }
+                                 Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;

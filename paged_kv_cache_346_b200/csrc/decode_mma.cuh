@@ -161,6 +161,9 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     __shared__ int s_abort;
     __shared__ int64_t s_row[GROUPS ? NH : 1];  // group pass: tile row -> sequence * Hq + head
     const GroupPassWait group_pass_wait{a};
+    // launched as a programmatic dependent of the kernel before it (usually
+    // the KV append): nothing is read before that kernel's writes are visible
+    if (!a.after_groups) pdl_wait_primary();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
@@ -597,7 +600,7 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
     e = launch_decode_kernel(kern, grid, dim3(NW * 32), C::smem_bytes(a.partition_size), stream,
-                             a.after_groups != 0, a, tk, tv);
+                             a, tk, tv);
     if (e != cudaSuccess || a.ws_slots <= 1) return e;
     return launch_lse_reduce<T, D>(a, stream);
 }

@@ -405,6 +405,9 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
 
     extern __shared__ __align__(1024) unsigned char smem_mma8[];
     __shared__ int s_abort;
+    // launched as a programmatic dependent of the kernel before it (usually
+    // the KV append): nothing is read before that kernel's writes are visible
+    if (!a.after_groups) pdl_wait_primary();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
@@ -639,8 +642,8 @@ cudaError_t launch_decode_mma_e4m3(const DecodeArgs& a, cudaStream_t stream) {
     e = make_cache_tensor_map(&tv, a.v_cache, 1, false, D, rows, 16);
     if (e != cudaSuccess) return e;
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
-    kern<<<grid, NW * 32, C::smem_bytes(a.partition_size), stream>>>(a, tk, tv);
-    e = cudaGetLastError();
+    e = launch_decode_kernel(kern, grid, dim3(NW * 32), C::smem_bytes(a.partition_size), stream,
+                             a, tk, tv);
     if (e != cudaSuccess || a.ws_slots <= 1) return e;
     return launch_lse_reduce<T, D>(a, stream);
 }

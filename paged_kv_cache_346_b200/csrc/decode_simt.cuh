@@ -302,6 +302,9 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::THREAD
     __shared__ float s_p[NW][HG][16];
     __shared__ volatile int s_abort;
     const GroupPassWait group_pass_wait{a};
+    // launched as a programmatic dependent of the kernel before it (usually
+    // the KV append): nothing is read before that kernel's writes are visible
+    if (!a.after_groups) pdl_wait_primary();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kvh = blockIdx.y / a.head_chunks;
@@ -435,8 +438,7 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
     cudaError_t e = attr.ensure(kern, C::smem_bytes(8192));
     if (e != cudaSuccess) return e;
     dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
-    e = launch_decode_kernel(kern, grid, dim3(C::THREADS), smem_simt, stream, a.after_groups != 0,
-                             a);
+    e = launch_decode_kernel(kern, grid, dim3(C::THREADS), smem_simt, stream, a);
     if (e != cudaSuccess || a.ws_slots <= 1) return e;
     return launch_lse_reduce<T, D>(a, stream);
 }
