@@ -299,22 +299,41 @@ __device__ __forceinline__ void merge_partials(const float* ml, int64_t ml_strid
 #pragma unroll
     for (int i = 0; i < PER_LANE; ++i) num[i] = 0.f;
     float den = 0.f;
-    for (int p = warp; p < np; p += NW) {
-        const float w = ml[p * ml_stride + 1] * exp2f(ml[p * ml_stride] - M);
-        den += w;
-        const float* op = o + p * o_stride + lane * PER_LANE;
-        if constexpr (PER_LANE % 4 == 0) {
+    // U partials per warp in flight: every load of a group is issued before
+    // the first is used, so a row of many partitions (long contexts) costs a
+    // few memory latencies, not one per partition
+    constexpr int U = 8;
+    for (int p0 = warp; p0 < np; p0 += NW * U) {
+        float pm[U], pl[U];
+        float x[U][PER_LANE];
 #pragma unroll
-            for (int i = 0; i < PER_LANE; i += 4) {
-                const float4 x = *reinterpret_cast<const float4*>(op + i);
-                num[i] = fmaf(w, x.x, num[i]);
-                num[i + 1] = fmaf(w, x.y, num[i + 1]);
-                num[i + 2] = fmaf(w, x.z, num[i + 2]);
-                num[i + 3] = fmaf(w, x.w, num[i + 3]);
+        for (int u = 0; u < U; ++u) {
+            const int p = p0 + u * NW;
+            const bool in = p < np;
+            pm[u] = in ? ml[p * ml_stride] : -INFINITY;
+            pl[u] = in ? ml[p * ml_stride + 1] : 0.f;
+            const float* op = o + (in ? p : 0) * o_stride + lane * PER_LANE;
+            if constexpr (PER_LANE % 4 == 0) {
+#pragma unroll
+                for (int i = 0; i < PER_LANE; i += 4) {
+                    const float4 v = in ? *reinterpret_cast<const float4*>(op + i)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    x[u][i] = v.x;
+                    x[u][i + 1] = v.y;
+                    x[u][i + 2] = v.z;
+                    x[u][i + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < PER_LANE; ++i) x[u][i] = in ? op[i] : 0.f;
             }
-        } else {
+        }
 #pragma unroll
-            for (int i = 0; i < PER_LANE; ++i) num[i] = fmaf(w, op[i], num[i]);
+        for (int u = 0; u < U; ++u) {
+            const float w = pl[u] * exp2f(pm[u] - M);  // 0 past np (2^-inf)
+            den += w;
+#pragma unroll
+            for (int i = 0; i < PER_LANE; ++i) num[i] = fmaf(w, x[u][i], num[i]);
         }
     }
 #pragma unroll

@@ -43,7 +43,11 @@
 // fp16 term keeps 11 significant bits, and the output error it leaves,
 // ~2^-11 times the largest |v|, exceeds the fp16 / bf16 tolerance once values
 // are large (e.g. per-page V scales spread over decades); hi + lo keeps ~22.
-// The row sums l add the same hi + lo, so the weights stay normalised.
+// The row sums l add the fp32 weights themselves: p - (hi + lo) is the
+// rounding of the remainder, at most 2^-23 p + 2^-25 (the second term only
+// where p is below fp16's normal range), so the normaliser differs from the
+// sum of the weights the products used by less than 2^-23 of it plus 2^-25
+// per token, against l >= 1 (the reference max's own token has p = 1).
 #pragma once
 
 #include "decode_mma.cuh"
@@ -99,6 +103,21 @@ __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(x), "r"(sel));
     return r;
+}
+
+// 2^x by the hardware approximation (relative error about 2^-22; -inf -> 0,
+// results below the smallest normal -> 0): the softmax weights and rescale
+// factors, which tolerate far more
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// a pair rounded to f16x2 (lo in the low half)
+__device__ __forceinline__ uint32_t f16x2_rn(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // CTAs per SM the register allocation is held to.  8-head tiles at head_dim
@@ -169,7 +188,7 @@ template <int D, int NH, bool PPB, bool EARLY, typename Addr>
 __device__ __forceinline__ void e4m3_slice_math(
     const uint32_t (&qa)[D / 16][NH == 16 ? 4 : 2], float (&m)[NH == 8 ? 2 : NH / 8],
     float (&l)[NH == 8 ? 2 : NH / 8], float (&o)[D / 16][NH / 8][4],
-    const uint32_t (&kf)[EARLY ? D / 32 : 1][4], const uint32_t (&vf)[EARLY ? D / 32 : 1][4],
+    const uint32_t (&kf)[EARLY ? D / 32 : 1][4], uint32_t (&vf)[EARLY ? D / 32 : 1][4],
     Addr addr, int wvalid, int wlo, float kmul, float vmul, int g, int t4) {
     using M = Mma<__half>;
     constexpr int KSTEPS = D / 16, KP = KSTEPS / 2, RB = NH / 8;
@@ -235,22 +254,21 @@ __device__ __forceinline__ void e4m3_slice_math(
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                 const float mnew = fmaxf(m[j], mx);
-                const float alpha = exp2f(m[j] - mnew);
+                const float alpha = ex2_approx(m[j] - mnew);
                 l[j] *= alpha;
                 m[j] = mnew;
                 alpha_c[0][j] = alpha;
             }
         }
-        float p[4], pr[4], rr[4];
+        float p[4], pr[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) p[i] = exp2f(s[i] - m[i & 1]);
+        for (int i = 0; i < 4; ++i) p[i] = ex2_approx(s[i] - m[i & 1]);
         const uint32_t p0 = M::pack(p[0], p[1], pr[0], pr[1]);
         const uint32_t p1 = M::pack(p[2], p[3], pr[2], pr[3]);
-        const uint32_t r0 = M::pack(p[0] - pr[0], p[1] - pr[1], rr[0], rr[1]);
-        const uint32_t r1 = M::pack(p[2] - pr[2], p[3] - pr[3], rr[2], rr[3]);
-        // the weights the P.V products use are hi + lo
-        l[0] += (pr[0] + rr[0]) + (pr[2] + rr[2]);
-        l[1] += (pr[1] + rr[1]) + (pr[3] + rr[3]);
+        const uint32_t r0 = f16x2_rn(p[0] - pr[0], p[1] - pr[1]);
+        const uint32_t r1 = f16x2_rn(p[2] - pr[2], p[3] - pr[3]);
+        l[0] += p[0] + p[2];
+        l[1] += p[1] + p[3];
         // P (tokens x heads) -> P^T fragments: lane (g, t4) gets head
         // g, tokens 2 t4, 2 t4 + 1 (of 0-7, then of 8-15)
         pb[0][0] = movmatrix_trans(p0);
@@ -314,7 +332,7 @@ __device__ __forceinline__ void e4m3_slice_math(
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
                 const float mnew = fmaxf(m[rb], mx);
-                const float alpha = exp2f(m[rb] - mnew);
+                const float alpha = ex2_approx(m[rb] - mnew);
                 l[rb] *= alpha;
                 m[rb] = mnew;
                 alpha_c[rb][0] = __shfl_sync(0xffffffffu, alpha, (2 * t4) * 4);
@@ -324,17 +342,48 @@ __device__ __forceinline__ void e4m3_slice_math(
 #pragma unroll
         for (int rb = 0; rb < RB; ++rb) {
             const int i0 = 2 * rb;
-            float pr[2][2], rr[2][2];
+            float ps[2];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                const float p0 = exp2f(s[nt][i0] - m[rb]);
-                const float p1 = exp2f(s[nt][i0 + 1] - m[rb]);
-                pb[rb][nt] = M::pack(p0, p1, pr[nt][0], pr[nt][1]);
-                pl[rb][nt] = M::pack(p0 - pr[nt][0], p1 - pr[nt][1], rr[nt][0], rr[nt][1]);
+                const float p0 = ex2_approx(s[nt][i0] - m[rb]);
+                const float p1 = ex2_approx(s[nt][i0 + 1] - m[rb]);
+                float h0, h1;
+                pb[rb][nt] = M::pack(p0, p1, h0, h1);
+                pl[rb][nt] = f16x2_rn(p0 - h0, p1 - h1);
+                ps[nt] = p0 + p1;
             }
-            // the weights the P.V products use are hi + lo
-            l[rb] += ((pr[0][0] + rr[0][0]) + (pr[0][1] + rr[0][1])) +
-                     ((pr[1][0] + rr[1][0]) + (pr[1][1] + rr[1][1]));
+            l[rb] += ps[0] + ps[1];
+        }
+    }
+    // The rescale and the masking sit outside the P.V loop, which then has
+    // no branch and schedules as one block.
+    if (grew) {
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+            for (int rb = 0; rb < RB; ++rb) {
+                o[mt][rb][0] *= alpha_c[rb][0];
+                o[mt][rb][1] *= alpha_c[rb][1];
+                o[mt][rb][2] *= alpha_c[rb][0];
+                o[mt][rb][3] *= alpha_c[rb][1];
+            }
+    }
+    // Codes of masked tokens become 0 (0 * NaN would poison the sum).  Code
+    // register 2 h of a pair holds tokens 2 t4 (bytes 0, 1) and 2 t4 + 1
+    // (bytes 2, 3), register 2 h + 1 the same tokens + 8.
+    uint32_t keep[2] = {~0u, ~0u};
+    if (partial) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int tk = 8 * j + 2 * t4;
+            keep[j] = (tk >= wlo && tk < wvalid ? 0x0000ffffu : 0u) |
+                      (tk + 1 >= wlo && tk + 1 < wvalid ? 0xffff0000u : 0u);
+        }
+        if constexpr (EARLY) {
+#pragma unroll
+            for (int kp = 0; kp < (EARLY ? KP : 1); ++kp)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) vf[kp][i] &= keep[i & 1];
         }
     }
 #pragma unroll
@@ -345,6 +394,8 @@ __device__ __forceinline__ void e4m3_slice_math(
             for (int i = 0; i < 4; ++i) vc[i] = vf[kp < (EARLY ? KP : 1) ? kp : 0][i];
         } else {
             ldsm_x4_trans(addr(kp) + SLICE_BYTES, vc);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) vc[i] &= keep[i & 1];
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // m-tile 2 kp + h
@@ -354,24 +405,8 @@ __device__ __forceinline__ void e4m3_slice_math(
             // (V[r0][2g], V[r1][2g] | V[r0][2g+1], V[r1][2g+1])
             e4m3x4_to_f16x2(byte_perm(vc[2 * h], 0x3120u), va[0], va[1]);
             e4m3x4_to_f16x2(byte_perm(vc[2 * h + 1], 0x3120u), va[2], va[3]);
-            if (partial) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int tk = (i >> 1) * 8 + 2 * t4;
-                    const uint32_t keep =
-                        (tk >= wlo && tk < wvalid ? 0x0000ffffu : 0u) |
-                        (tk + 1 >= wlo && tk + 1 < wvalid ? 0xffff0000u : 0u);
-                    va[i] &= keep;
-                }
-            }
 #pragma unroll
             for (int rb = 0; rb < RB; ++rb) {
-                if (grew) {
-                    o[mt][rb][0] *= alpha_c[rb][0];
-                    o[mt][rb][1] *= alpha_c[rb][1];
-                    o[mt][rb][2] *= alpha_c[rb][0];
-                    o[mt][rb][3] *= alpha_c[rb][1];
-                }
                 if constexpr (PPB) {  // this page's P.V, then times its v_scale
                     float d4[4] = {0.f, 0.f, 0.f, 0.f};
                     mma_f16(d4, va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
@@ -524,10 +559,11 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
     // the output's V scale: the KV head's (per-page scales enter slice by slice)
     const float vs_out = PPB ? 1.f : a.v_scale[kvh];
 
+    int stage = 0;       // it % STAGES
+    uint32_t phase = 0;  // (it / STAGES) & 1
     for (int it = 0; it < nslices; ++it) {
-        const int stage = it % STAGES;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(full + warp * STAGES + stage,
-                                                          (uint32_t)((it / STAGES) & 1), a.status));
+        const bool ok =
+            __all_sync(0xffffffffu, mbar_wait(full + warp * STAGES + stage, phase, a.status));
         if (!ok) {
             s_abort = 1;
             // let this warp's copies still in flight land (bounded) before
@@ -568,6 +604,10 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
         __syncwarp();  // the warp's reads of the stage are done: refill it
         if (lane == 0 && it + STAGES < nslices) issue(it + STAGES, stage);
         if (EARLY && work) math();
+        if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+        }
     }
     __syncthreads();  // every warp is out of its ring (or gave up)
     if (s_abort) return;
