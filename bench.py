@@ -944,7 +944,8 @@ def main():
                     choices=sorted(CONFIGS) + ["cow_sampling", "swap"])
     ap.add_argument("--kernel", choices=["auto", "simt", "mma"], default="auto")
     ap.add_argument("--partition", type=int, default=None,
-                    help="tokens per partition (default: the workload's, else automatic)")
+                    help="tokens per partition (default: automatic under --window, else the "
+                         "workload's, else automatic)")
     ap.add_argument("--seed", type=int, default=2)
     ap.add_argument("--window", type=int, default=0,
                     help="sliding window in tokens (0: attend to the whole context)")
@@ -975,7 +976,9 @@ def main():
         return run_swap(args)
     cfg = CONFIGS[args.workload]
     if args.partition is None:
-        args.partition = cfg.partition_size
+        # a workload's partition size is set for its whole contexts; behind a
+        # window the span is far shorter, so the library chooses
+        args.partition = 0 if args.window else cfg.partition_size
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

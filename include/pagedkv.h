@@ -114,11 +114,14 @@ PKV_API int pkv_version(void);
 PKV_API int pkv_decode_has_kernel(pkv_kernel kernel);
 
 /*
- * Partition size the decode uses when `partition_size` is 0, for this shape:
- * 4096 tokens when num_seqs * num_kv_heads >= 1024, else 2048, halved while
- * the grid would hold fewer than ~6 CTAs per SM.  Tuned with a longest-first
- * seq_order; without one, shorter partitions can be faster when lengths are
- * very uneven.
+ * Partition size the decode uses when `partition_size` is 0, for this shape
+ * (max_context_len: the longest span attended, i.e. at most the window plus
+ * block_size - 1 under a sliding window).  When even 2048-token partitions
+ * give at most 3 CTAs per SM (148 SMs), the smallest multiple of 64 that
+ * keeps the grid within that one wave.  Otherwise 4096 tokens when
+ * num_seqs * num_kv_heads >= 1024, else 2048, halved while the grid would
+ * hold fewer than ~6 CTAs per SM.  Tuned with a longest-first seq_order;
+ * without one, shorter partitions can be faster when lengths are very uneven.
  */
 PKV_API int pkv_decode_default_partition(int num_seqs, int num_kv_heads, int max_context_len);
 

@@ -377,10 +377,22 @@ int pkv_decode_default_partition(int num_seqs, int num_kv_heads, int max_context
     // (E4M3); on the long-context batch (64 units) 2048 beats 4096 by 2-7 %
     // and 1024 by 0-2 %.  Small batches get shorter partitions so the grid
     // still fills every SM (3 CTAs each) about twice.
+    //
+    // Little work in all (a grid under one wave of 3 CTAs per SM even at
+    // 2048 tokens, e.g. a few sequences behind a sliding window): one wave of
+    // CTAs as long as that allows, so each SM slot pays the start-up once.
+    // Measured on B200, long contexts behind a 4096-token window (64 units):
+    // 768 and 1024 tokens 11-12 % faster than 256 and 512, 2048 26 % slower.
     const int64_t units = (int64_t)(num_seqs > 0 ? num_seqs : 1) * (num_kv_heads > 0 ? num_kv_heads : 1);
+    const int64_t len = max_context_len > 0 ? max_context_len : 1;
+    const int64_t slots = 3 * kNumSMs;
+    if (units * ceil_div(len, 2048) <= slots) {
+        int q = 64;
+        while (q < 2048 && units * ceil_div(len, q) > slots) q += 64;
+        return q;
+    }
     int p = units >= 1024 ? 4096 : 2048;
-    while (p > 64 && units * ceil_div(max_context_len > 0 ? max_context_len : 1, p) < 6 * kNumSMs)
-        p /= 2;
+    while (p > 64 && units * ceil_div(len, p) < 6 * kNumSMs) p /= 2;
     return p;
 }
 

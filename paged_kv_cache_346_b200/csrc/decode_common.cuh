@@ -368,6 +368,13 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
                          reinterpret_cast<T*>(a.out) + row * D);
 }
 
+// A decode kernel's griddepcontrol.wait: before its first read of pages (or
+// scales) and its first global write.  The regular pass after the group
+// pass waits only as it leaves (GroupPassWait).
+__device__ __forceinline__ void pdl_wait_before_pages(const DecodeArgs& a) {
+    if (!a.after_groups) pdl_wait_primary();
+}
+
 // The regular pass of the shared-prefix decode may start while the group
 // pass still runs (it is a programmatic dependent of it; neither reads the
 // other's results).  The log-sum-exp reduce, a programmatic dependent of the

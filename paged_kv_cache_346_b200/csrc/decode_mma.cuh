@@ -161,9 +161,13 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     __shared__ int s_abort;
     __shared__ int64_t s_row[GROUPS ? NH : 1];  // group pass: tile row -> sequence * Hq + head
     const GroupPassWait group_pass_wait{a};
-    // launched as a programmatic dependent of the kernel before it (usually
-    // the KV append): nothing is read before that kernel's writes are visible
-    if (!a.after_groups) pdl_wait_primary();
+    // Launched as a programmatic dependent of the kernel before it (usually
+    // the KV append): the schedule, lengths and table (which that kernel does
+    // not write) are read before griddepcontrol.wait, so the start-up of the
+    // first wave overlaps it; the pages are read, and anything is written,
+    // only after it (pdl_wait_before_pages).  The group pass waits first:
+    // it releases its own dependent (the regular pass) as it starts.
+    if (GROUPS) pdl_wait_before_pages(a);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
@@ -210,9 +214,11 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     const int L = sp.L, np = sp.np;
     T* out = reinterpret_cast<T*>(a.out);
     if (L == 0) {
-        if (!GROUPS && part == 0)
+        if (!GROUPS && part == 0) {
+            pdl_wait_before_pages(a);
             for (int i = tid; i < nh * D; i += NW * 32)
                 out[((int64_t)b * a.num_q_heads + h0 + i / D) * D + i % D] = Elem<T>::from_f32(0.f);
+        }
         return;
     }
     if (part >= np) return;
@@ -267,6 +273,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
             tma_load_2d(kd + SLICE_BYTES + x * BOX_BYTES, &tmv, x * 64, y, bar, pol);
         }
     };
+    if (!GROUPS) pdl_wait_before_pages(a);
     if (lane == 0) {
         const int pre = min(STAGES, nslices);
         for (int s = 0; s < pre; ++s) issue(s, s);

@@ -105,15 +105,6 @@ __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) {
     return r;
 }
 
-// 2^x by the hardware approximation (relative error about 2^-22; -inf -> 0,
-// results below the smallest normal -> 0): the softmax weights and rescale
-// factors, which tolerate far more
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
 // a pair rounded to f16x2 (lo in the low half)
 __device__ __forceinline__ uint32_t f16x2_rn(float lo, float hi) {
     const __half2 h = __floats2half2_rn(lo, hi);
@@ -440,9 +431,11 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
 
     extern __shared__ __align__(1024) unsigned char smem_mma8[];
     __shared__ int s_abort;
-    // launched as a programmatic dependent of the kernel before it (usually
-    // the KV append): nothing is read before that kernel's writes are visible
-    if (!a.after_groups) pdl_wait_primary();
+    // Launched as a programmatic dependent of the kernel before it (usually
+    // the KV append): the schedule, lengths and table (which that kernel does
+    // not write) are read before griddepcontrol.wait, so the start-up of the
+    // first wave overlaps it; the pages and scales are read, and anything is
+    // written, only after it (pdl_wait_before_pages).
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
@@ -460,9 +453,11 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
     const int L = sp.L, np = sp.np;
     T* out = reinterpret_cast<T*>(a.out);
     if (L == 0) {
-        if (part == 0)
+        if (part == 0) {
+            pdl_wait_before_pages(a);
             for (int i = tid; i < nh * D; i += NW * 32)
                 out[((int64_t)b * a.num_q_heads + h0 + i / D) * D + i % D] = Elem<T>::from_f32(0.f);
+        }
         return;
     }
     if (part >= np) return;
@@ -518,6 +513,7 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
             tma_load_2d(kd + SLICE_BYTES + x * BOX_BYTES, &tmv, x * 128, y, bar, pol);
         }
     };
+    pdl_wait_before_pages(a);
     if (lane == 0) {
         const int pre = min(STAGES, nslices);
         for (int s = 0; s < pre; ++s) issue(s, s);

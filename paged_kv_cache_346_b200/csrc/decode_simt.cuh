@@ -302,9 +302,11 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::THREAD
     __shared__ float s_p[NW][HG][16];
     __shared__ volatile int s_abort;
     const GroupPassWait group_pass_wait{a};
-    // launched as a programmatic dependent of the kernel before it (usually
-    // the KV append): nothing is read before that kernel's writes are visible
-    if (!a.after_groups) pdl_wait_primary();
+    // Launched as a programmatic dependent of the kernel before it (usually
+    // the KV append): the schedule, lengths and table (which that kernel does
+    // not write) are read before griddepcontrol.wait, so the start-up of the
+    // first wave overlaps it; the pages are read, and anything is written,
+    // only after it (pdl_wait_before_pages).
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kvh = blockIdx.y / a.head_chunks;
@@ -321,6 +323,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::THREAD
     const int L = sp.L, np = sp.np;
     if (L == 0) {  // empty sequence: a zero row
         if (part == 0) {
+            pdl_wait_before_pages(a);
             T* out = reinterpret_cast<T*>(a.out);
             for (int i = tid; i < nh * D; i += THREADS)
                 out[((int64_t)b * a.num_q_heads + h0 + i / D) * D + i % D] = E::from_f32(0.f);
@@ -371,6 +374,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::THREAD
         bulk_load(kd, kbase + off, SLICE_BYTES, bar, pol);
         bulk_load(kd + SLICE_BYTES, vbase + off, SLICE_BYTES, bar, pol);
     };
+    pdl_wait_before_pages(a);
     if (lane == 0) {
         const int pre = min(STAGES, nslices);
         for (int s = 0; s < pre; ++s) issue(s, s);

@@ -92,6 +92,15 @@ __device__ __forceinline__ void drain_ring(uint64_t* bars, int stages, int from,
             flag(status, PKV_DEV_DRAIN_TIMEOUT);
 }
 
+// 2^x by the hardware approximation (relative error about 2^-22; -inf -> 0,
+// results below the smallest normal -> 0): softmax weights and rescale
+// factors, which tolerate far more
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // L2 policy for data read exactly once (the K/V pages of a decode step).
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;

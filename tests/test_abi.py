@@ -111,6 +111,11 @@ def test_default_partition_rule():
     assert d(1, 1, 4096) == 64          # tiny batches split finer
     p = d(4, 4, 512)
     assert 64 <= p <= 512 and p % 64 == 0
+    # a few sequences behind a 4096-token window (span 4096 + 15): one wave of
+    # at most 3 CTAs per SM, as long as that allows
+    p = d(8, 8, 4111)
+    assert p == 704 and 64 * -(-4111 // p) <= 3 * 148 < 64 * -(-4111 // (p - 64))
+    assert d(8, 8, 16384) == 1024       # 512 CTAs at 2048: the many-CTA rule
 
 
 def test_append_and_copy_host_checks():
