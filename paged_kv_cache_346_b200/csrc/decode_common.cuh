@@ -270,104 +270,6 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, float
     }
 }
 
-// Merge n partial results of one (sequence, query head) row into out_row:
-// with per-partial maxima m_p (base-2 logits), sums l_p and normalised
-// outputs o_p,
-//   M = max_p m_p,  w_p = l_p 2^(m_p - M),  out = sum_p w_p o_p / sum_p w_p.
-// Partial p's (m, l) is at ml + p * ml_stride, its o at o + p * o_stride.
-// All 128 threads of the CTA take part.
-template <typename T, int D>
-__device__ __forceinline__ void merge_partials(const float* ml, int64_t ml_stride,
-                                               const float* o, int64_t o_stride, int np,
-                                               T* out_row) {
-    constexpr int NW = 4;
-    constexpr int PER_LANE = D / 32;  // floats of o per lane
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    __shared__ float s_max[NW];
-    __shared__ float s_den[NW];
-    __shared__ float s_num[NW][D];
-
-    float M = -INFINITY;
-    for (int p = tid; p < np; p += 128) M = fmaxf(M, ml[p * ml_stride]);
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
-    if (lane == 0) s_max[warp] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
-
-    float num[PER_LANE];
-#pragma unroll
-    for (int i = 0; i < PER_LANE; ++i) num[i] = 0.f;
-    float den = 0.f;
-    // U partials per warp in flight: every load of a group is issued before
-    // the first is used, so a row of many partitions (long contexts) costs a
-    // few memory latencies, not one per partition
-    constexpr int U = 8;
-    for (int p0 = warp; p0 < np; p0 += NW * U) {
-        float pm[U], pl[U];
-        float x[U][PER_LANE];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int p = p0 + u * NW;
-            const bool in = p < np;
-            pm[u] = in ? ml[p * ml_stride] : -INFINITY;
-            pl[u] = in ? ml[p * ml_stride + 1] : 0.f;
-            const float* op = o + (in ? p : 0) * o_stride + lane * PER_LANE;
-            if constexpr (PER_LANE % 4 == 0) {
-#pragma unroll
-                for (int i = 0; i < PER_LANE; i += 4) {
-                    const float4 v = in ? *reinterpret_cast<const float4*>(op + i)
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-                    x[u][i] = v.x;
-                    x[u][i + 1] = v.y;
-                    x[u][i + 2] = v.z;
-                    x[u][i + 3] = v.w;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < PER_LANE; ++i) x[u][i] = in ? op[i] : 0.f;
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const float w = pl[u] * exp2f(pm[u] - M);  // 0 past np (2^-inf)
-            den += w;
-#pragma unroll
-            for (int i = 0; i < PER_LANE; ++i) num[i] = fmaf(w, x[u][i], num[i]);
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < PER_LANE; ++i) s_num[warp][lane * PER_LANE + i] = num[i];
-    if (lane == 0) s_den[warp] = den;
-    __syncthreads();
-    const float total = s_den[0] + s_den[1] + s_den[2] + s_den[3];
-    for (int d = tid; d < D; d += 128) {
-        const float x = s_num[0][d] + s_num[1][d] + s_num[2][d] + s_num[3][d];
-        out_row[d] = Elem<T>::from_f32(x / total);
-    }
-}
-
-// Merge the partitions of one (sequence, query head) row (merge_partials).
-// One CTA of 128 threads per row; rows with one partial result in all were
-// written by the decode kernel and are skipped.  Launched as a programmatic
-// dependent of the decode kernel: those rows leave before the wait, during
-// the decode's tail; the others wait for the decode grid's writes before
-// reading.
-template <typename T, int D>
-__global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
-    const int h = blockIdx.x;
-    const int b = blockIdx.y;
-    // the partition count depends only on the inputs, not on the decode
-    // grid's output: rows with one partial result leave before the wait
-    const Span sp = seq_span(a, b, false);
-    if (sp.direct) return;
-    const int np = sp.slot0 + sp.np;  // the group pass's slots, then this row's partitions
-    pdl_wait_primary();
-    const int64_t row = (int64_t)b * a.num_q_heads + h;
-    merge_partials<T, D>(a.ws_ml + row * a.ws_slots * 2, 2, a.ws_o + row * a.ws_slots * D, D, np,
-                         reinterpret_cast<T*>(a.out) + row * D);
-}
-
 // A decode kernel's griddepcontrol.wait: before its first read of pages (or
 // scales) and its first global write.  The regular pass after the group
 // pass waits only as it leaves (GroupPassWait).
@@ -421,22 +323,5 @@ struct SmemAttr {
         });
     }
 };
-
-// Launch the reduce after the decode kernel on the same stream, as a
-// programmatic dependent launch.
-template <typename T, int D>
-cudaError_t launch_lse_reduce(const DecodeArgs& a, cudaStream_t stream) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.num_q_heads, a.num_seqs, 1);
-    cfg.blockDim = dim3(128, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, lse_reduce_kernel<T, D>, a);
-}
 
 }  // namespace pkv

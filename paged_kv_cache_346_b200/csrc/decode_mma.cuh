@@ -31,6 +31,7 @@
 #include <type_traits>
 
 #include "decode_common.cuh"
+#include "lse_reduce.cuh"
 
 namespace pkv {
 

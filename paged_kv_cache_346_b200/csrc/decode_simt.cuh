@@ -33,6 +33,7 @@
 #include <type_traits>
 
 #include "decode_common.cuh"
+#include "lse_reduce.cuh"
 
 namespace pkv {
 

@@ -1,0 +1,259 @@
+// The split-K merge of a decode's partitions: the log-sum-exp reduce.
+//
+// A sequence longer than one partition leaves one partial result per
+// partition and query head: its maximum m_p (base-2 logits), its sum l_p and
+// its normalised output o_p.  Merged, they give exactly the attention over
+// the whole sequence ("pagedattention vllm" §Attention Computation: attention
+// taken block by block equals attention over the contiguous sequence):
+//   M = max_p m_p,  w_p = l_p 2^(m_p - M),  out = sum_p w_p o_p / sum_p w_p.
+#pragma once
+
+#include "decode_common.cuh"
+
+namespace pkv {
+
+// Two forms of the merge.  The reduce is launched as a programmatic
+// dependent of the decode, and a CTA of a split row sits resident waiting
+// for the decode grid: where rows have few partitions (a batch of mostly
+// short sequences) that CTA must be small, so the registers-only form runs,
+// 128 threads and no dynamic shared memory.  Rows of many partitions (long
+// contexts) stream their partial outputs through shared memory with bulk
+// copies (48 KB); their waiting CTAs appear only when the decode CTAs, all
+// split, finish their loops.
+constexpr int kReduceSmallThreads = 128;
+constexpr int kReduceThreads = 256;
+constexpr int kReduceStreamSlots = 16;  // partial results per row from which rows stream
+
+// Few partitions per row: merge np partial results of one row into out_row
+// from registers.  Partial p's (m, l) is at ml + p * ml_stride, its o at
+// o + p * o_stride.  All kReduceSmallThreads threads of the CTA take part.
+template <typename T, int D>
+__device__ __forceinline__ void merge_partials_small(const float* ml, int64_t ml_stride,
+                                                     const float* o, int64_t o_stride, int np,
+                                                     T* out_row) {
+    constexpr int NW = 4;
+    static_assert(NW * 32 == kReduceSmallThreads, "one warp per lane group");
+    constexpr int PER_LANE = D / 32;  // floats of o per lane
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ float s_max[NW];
+    __shared__ float s_den[NW];
+    __shared__ float s_num[NW][D];
+
+    float M = -INFINITY;
+    for (int p = tid; p < np; p += kReduceSmallThreads) M = fmaxf(M, ml[p * ml_stride]);
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
+    if (lane == 0) s_max[warp] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
+
+    float num[PER_LANE];
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) num[i] = 0.f;
+    float den = 0.f;
+    // U partials per warp in flight: every load of a group is issued before
+    // the first is used, so a row of many partitions (long contexts) costs a
+    // few memory latencies, not one per partition
+    constexpr int U = 8;
+    for (int p0 = warp; p0 < np; p0 += NW * U) {
+        float pm[U], pl[U];
+        float x[U][PER_LANE];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int p = p0 + u * NW;
+            const bool in = p < np;
+            pm[u] = in ? ml[p * ml_stride] : -INFINITY;
+            pl[u] = in ? ml[p * ml_stride + 1] : 0.f;
+            const float* op = o + (in ? p : 0) * o_stride + lane * PER_LANE;
+            if constexpr (PER_LANE % 4 == 0) {
+#pragma unroll
+                for (int i = 0; i < PER_LANE; i += 4) {
+                    const float4 v = in ? *reinterpret_cast<const float4*>(op + i)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    x[u][i] = v.x;
+                    x[u][i + 1] = v.y;
+                    x[u][i + 2] = v.z;
+                    x[u][i + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < PER_LANE; ++i) x[u][i] = in ? op[i] : 0.f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const float w = pl[u] * exp2f(pm[u] - M);  // 0 past np (2^-inf)
+            den += w;
+#pragma unroll
+            for (int i = 0; i < PER_LANE; ++i) num[i] = fmaf(w, x[u][i], num[i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) s_num[warp][lane * PER_LANE + i] = num[i];
+    if (lane == 0) s_den[warp] = den;
+    __syncthreads();
+    const float total = s_den[0] + s_den[1] + s_den[2] + s_den[3];
+    for (int d = tid; d < D; d += kReduceSmallThreads) {
+        const float x = s_num[0][d] + s_num[1][d] + s_num[2][d] + s_num[3][d];
+        out_row[d] = Elem<T>::from_f32(x / total);
+    }
+}
+
+
+
+// Chunks of a row's partial outputs streamed through shared memory: CH
+// partitions (16 KB) per chunk, STAGES chunks in flight.
+template <int D>
+struct ReduceCfg {
+    static constexpr int CH = 16384 / (D * 4);
+    static constexpr int STAGES = 3;
+    static constexpr int CHUNK_BYTES = CH * D * 4;
+    static constexpr int SMEM = 64 + STAGES * CHUNK_BYTES;  // barriers, then the ring
+    static_assert(kReduceThreads % D == 0 && CH % (kReduceThreads / D) == 0, "layout");
+};
+
+// Many partitions per row: merge np partial results of one (sequence, query
+// head) row into out_row.  Partial p's (m, l) is at ml + p * ml_stride, its o
+// at o + p * D (one
+// contiguous run of np * D floats for the row, 16-byte aligned); they were
+// written by an earlier grid.  The o rows stream into shared memory in
+// 16 KB bulk copies (TMA), three in flight, so a row of many partitions (a
+// long context in 512-token partitions: 256, 128 KB) is read at copy-engine
+// rate rather than one dependent load after another.  Thread t sums
+// dimension t % D over its share (t / D) of each chunk's partitions.  A wait
+// that gives up flags the status word and leaves the row unwritten.
+template <typename T, int D>
+__device__ __forceinline__ void merge_partials(const float* __restrict__ ml, int64_t ml_stride,
+                                               const float* __restrict__ o, int np, T* out_row,
+                                               unsigned int* status) {
+    using C = ReduceCfg<D>;
+    constexpr int NT = kReduceThreads;
+    constexpr int SPLIT = NT / D;           // threads per dimension
+    constexpr int PER = C::CH / SPLIT;      // partitions per thread and chunk
+    extern __shared__ __align__(128) unsigned char smem_red[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem_red);
+    float* ring = reinterpret_cast<float*>(smem_red + 64);
+    __shared__ float s_max[NT / 32];
+    __shared__ float s_part[SPLIT][D + 1];
+    __shared__ int s_abort;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nchunks = (np + C::CH - 1) / C::CH;
+
+    auto issue = [&](int c, int stage) {  // thread 0
+        const int n = min(C::CH, np - c * C::CH);
+        mbar_arrive_expect_tx(full + stage, (uint32_t)(n * D * 4));
+        bulk_load(ring + stage * (C::CHUNK_BYTES / 4), o + (int64_t)c * C::CH * D,
+                  (uint32_t)(n * D * 4), full + stage, policy_evict_first());
+    };
+    if (tid == 0) {
+        s_abort = 0;
+        for (int st = 0; st < C::STAGES; ++st) mbar_init(full + st, 1);
+        fence_barrier_init();
+        for (int c = 0; c < min(C::STAGES, nchunks); ++c) issue(c, c);
+    }
+
+    // M = max_p m_p while the first chunks are in flight
+    float M = -INFINITY;
+    for (int p = tid; p < np; p += NT) M = fmaxf(M, __ldg(ml + p * ml_stride));
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
+    if (lane == 0) s_max[warp] = M;
+    __syncthreads();  // also: the barriers are initialised
+    M = s_max[0];
+#pragma unroll
+    for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, s_max[w]);
+
+    const int d = tid % D, part = tid / D;
+    float num = 0.f, den = 0.f;
+    for (int c = 0; c < nchunks; ++c) {
+        const int stage = c % C::STAGES;
+        if (!mbar_wait(full + stage, (uint32_t)((c / C::STAGES) & 1), status)) s_abort = 1;
+        const float* ch = ring + stage * (C::CHUNK_BYTES / 4);
+        const int p0 = c * C::CH;
+#pragma unroll 4
+        for (int j = 0; j < PER; ++j) {
+            const int pc = part * PER + j;  // partition within the chunk
+            const int p = p0 + pc;
+            if (p < np) {
+                const float w = __ldg(ml + p * ml_stride + 1) * exp2f(__ldg(ml + p * ml_stride) - M);
+                den += w;
+                num = fmaf(w, ch[pc * D + d], num);
+            }
+        }
+        __syncthreads();  // every thread is done with this stage (and saw s_abort)
+        if (s_abort) {
+            // let the copies still in flight land (bounded) before the CTA
+            // leaves: this chunk's (some thread gave up on it) and the next
+            if (tid == 0) drain_ring(full, C::STAGES, c, min(nchunks, c + C::STAGES), status);
+            return;
+        }
+        if (tid == 0 && c + C::STAGES < nchunks) issue(c + C::STAGES, stage);
+    }
+    s_part[part][d] = num;
+    if (d == 0) s_part[part][D] = den;
+    __syncthreads();
+    if (tid < D) {
+        float x = 0.f, total = 0.f;
+#pragma unroll
+        for (int q = 0; q < SPLIT; ++q) {
+            x += s_part[q][tid];
+            total += s_part[q][D];
+        }
+        out_row[tid] = Elem<T>::from_f32(x / total);
+    }
+}
+
+// Merge the partitions of one (sequence, query head) row.  One CTA per row;
+// rows with one partial result in all were written by the decode kernel and
+// are skipped.  Launched as a programmatic dependent of the decode kernel:
+// those rows leave before the wait, during the decode's tail; the others
+// wait for the decode grid's writes before reading.
+template <typename T, int D, bool STREAM>
+__global__ void __launch_bounds__(STREAM ? kReduceThreads : kReduceSmallThreads)
+    lse_reduce_kernel(const DecodeArgs a) {
+    const int h = blockIdx.x;
+    const int b = blockIdx.y;
+    // the partition count depends only on the inputs, not on the decode
+    // grid's output: rows with one partial result leave before the wait
+    const Span sp = seq_span(a, b, false);
+    if (sp.direct) return;
+    const int np = sp.slot0 + sp.np;  // the group pass's slots, then this row's partitions
+    pdl_wait_primary();
+    const int64_t row = (int64_t)b * a.num_q_heads + h;
+    const float* ml = a.ws_ml + row * a.ws_slots * 2;
+    const float* o = a.ws_o + row * a.ws_slots * D;
+    T* out_row = reinterpret_cast<T*>(a.out) + row * D;
+    if constexpr (STREAM)
+        merge_partials<T, D>(ml, 2, o, np, out_row, a.status);
+    else
+        merge_partials_small<T, D>(ml, 2, o, D, np, out_row);
+}
+
+// Launch the reduce after the decode kernel on the same stream, as a
+// programmatic dependent launch: the streaming form when rows may hold at
+// least kReduceStreamSlots partial results, else the small one.
+template <typename T, int D>
+cudaError_t launch_lse_reduce(const DecodeArgs& a, cudaStream_t stream) {
+    const bool streamed = a.ws_slots >= kReduceStreamSlots;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.num_q_heads, a.num_seqs, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (!streamed) {
+        cfg.blockDim = dim3(kReduceSmallThreads, 1, 1);
+        cfg.dynamicSmemBytes = 0;
+        return cudaLaunchKernelEx(&cfg, lse_reduce_kernel<T, D, false>, a);
+    }
+    static SmemAttr smem_attr;
+    cudaError_t e = smem_attr.ensure(lse_reduce_kernel<T, D, true>, ReduceCfg<D>::SMEM);
+    if (e != cudaSuccess) return e;
+    cfg.blockDim = dim3(kReduceThreads, 1, 1);
+    cfg.dynamicSmemBytes = ReduceCfg<D>::SMEM;
+    return cudaLaunchKernelEx(&cfg, lse_reduce_kernel<T, D, true>, a);
+}
+
+}  // namespace pkv
