@@ -15,91 +15,82 @@ namespace pkv {
 // Two forms of the merge.  The reduce is launched as a programmatic
 // dependent of the decode, and a CTA of a split row sits resident waiting
 // for the decode grid: where rows have few partitions (a batch of mostly
-// short sequences) that CTA must be small, so the registers-only form runs,
-// 128 threads and no dynamic shared memory.  Rows of many partitions (long
-// contexts) stream their partial outputs through shared memory with bulk
-// copies (48 KB); their waiting CTAs appear only when the decode CTAs, all
-// split, finish their loops.
-constexpr int kReduceSmallThreads = 128;
+// short sequences) that CTA must be small, so the registers-only form runs:
+// one CTA of 8 warps per sequence and 8 query heads (a warp per row; far
+// fewer CTAs than rows to launch and retire), no dynamic shared memory.
+// Rows of many partitions (long contexts) stream their partial outputs
+// through shared memory with bulk copies (48 KB per CTA, one per row); their
+// waiting CTAs appear only when the decode CTAs, all split, finish their
+// loops.
+constexpr int kReduceRowsPerCta = 8;
 constexpr int kReduceThreads = 256;
 constexpr int kReduceStreamSlots = 16;  // partial results per row from which rows stream
 
-// Few partitions per row: merge np partial results of one row into out_row
-// from registers.  Partial p's (m, l) is at ml + p * ml_stride, its o at
-// o + p * o_stride.  All kReduceSmallThreads threads of the CTA take part.
+// Few partitions per row: one warp merges np partial results of one row into
+// out_row from registers.  Partial p's (m, l) is at ml + 2 p, its o at
+// o + p * D; every lane sees every partial (so holds the whole sum) and owns
+// D / 32 consecutive dimensions.  Four partials' loads are issued before the
+// first is used.
 template <typename T, int D>
-__device__ __forceinline__ void merge_partials_small(const float* ml, int64_t ml_stride,
-                                                     const float* o, int64_t o_stride, int np,
-                                                     T* out_row) {
-    constexpr int NW = 4;
-    static_assert(NW * 32 == kReduceSmallThreads, "one warp per lane group");
-    constexpr int PER_LANE = D / 32;  // floats of o per lane
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    __shared__ float s_max[NW];
-    __shared__ float s_den[NW];
-    __shared__ float s_num[NW][D];
-
+__device__ __forceinline__ void merge_row_warp(const float* __restrict__ ml,
+                                               const float* __restrict__ o, int np, T* out_row,
+                                               int lane) {
+    constexpr int PER_LANE = D / 32;
     float M = -INFINITY;
-    for (int p = tid; p < np; p += kReduceSmallThreads) M = fmaxf(M, ml[p * ml_stride]);
+    for (int p = lane; p < np; p += 32) M = fmaxf(M, __ldg(ml + 2 * p));
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
-    if (lane == 0) s_max[warp] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
-
+    auto load_o = [&](int p, float (&x)[PER_LANE]) {
+        const float* op = o + (int64_t)p * D + lane * PER_LANE;
+        if constexpr (PER_LANE % 4 == 0) {
+#pragma unroll
+            for (int i = 0; i < PER_LANE; i += 4) {
+                const float4 v = __ldg(reinterpret_cast<const float4*>(op + i));
+                x[i] = v.x;
+                x[i + 1] = v.y;
+                x[i + 2] = v.z;
+                x[i + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < PER_LANE; ++i) x[i] = __ldg(op + i);
+        }
+    };
     float num[PER_LANE];
 #pragma unroll
     for (int i = 0; i < PER_LANE; ++i) num[i] = 0.f;
     float den = 0.f;
-    // U partials per warp in flight: every load of a group is issued before
-    // the first is used, so a row of many partitions (long contexts) costs a
-    // few memory latencies, not one per partition
-    constexpr int U = 8;
-    for (int p0 = warp; p0 < np; p0 += NW * U) {
-        float pm[U], pl[U];
-        float x[U][PER_LANE];
+    constexpr int U = 4;
+    int p = 0;
+    for (; p + U <= np; p += U) {
+        float pm[U], pl[U], x[U][PER_LANE];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int p = p0 + u * NW;
-            const bool in = p < np;
-            pm[u] = in ? ml[p * ml_stride] : -INFINITY;
-            pl[u] = in ? ml[p * ml_stride + 1] : 0.f;
-            const float* op = o + (in ? p : 0) * o_stride + lane * PER_LANE;
-            if constexpr (PER_LANE % 4 == 0) {
-#pragma unroll
-                for (int i = 0; i < PER_LANE; i += 4) {
-                    const float4 v = in ? *reinterpret_cast<const float4*>(op + i)
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-                    x[u][i] = v.x;
-                    x[u][i + 1] = v.y;
-                    x[u][i + 2] = v.z;
-                    x[u][i + 3] = v.w;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < PER_LANE; ++i) x[u][i] = in ? op[i] : 0.f;
-            }
+            pm[u] = __ldg(ml + 2 * (p + u));
+            pl[u] = __ldg(ml + 2 * (p + u) + 1);
+            load_o(p + u, x[u]);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const float w = pl[u] * exp2f(pm[u] - M);  // 0 past np (2^-inf)
+            const float w = pl[u] * exp2f(pm[u] - M);
             den += w;
 #pragma unroll
             for (int i = 0; i < PER_LANE; ++i) num[i] = fmaf(w, x[u][i], num[i]);
         }
     }
+    for (; p < np; ++p) {
+        float x[PER_LANE];
+        load_o(p, x);
+        const float w = __ldg(ml + 2 * p + 1) * exp2f(__ldg(ml + 2 * p) - M);
+        den += w;
 #pragma unroll
-    for (int i = 0; i < PER_LANE; ++i) s_num[warp][lane * PER_LANE + i] = num[i];
-    if (lane == 0) s_den[warp] = den;
-    __syncthreads();
-    const float total = s_den[0] + s_den[1] + s_den[2] + s_den[3];
-    for (int d = tid; d < D; d += kReduceSmallThreads) {
-        const float x = s_num[0][d] + s_num[1][d] + s_num[2][d] + s_num[3][d];
-        out_row[d] = Elem<T>::from_f32(x / total);
+        for (int i = 0; i < PER_LANE; ++i) num[i] = fmaf(w, x[i], num[i]);
     }
+    const float inv = 1.f / den;
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i)
+        out_row[lane * PER_LANE + i] = Elem<T>::from_f32(num[i] * inv);
 }
-
-
 
 // Chunks of a row's partial outputs streamed through shared memory: CH
 // partitions (16 KB) per chunk, STAGES chunks in flight.
@@ -203,15 +194,15 @@ __device__ __forceinline__ void merge_partials(const float* __restrict__ ml, int
     }
 }
 
-// Merge the partitions of one (sequence, query head) row.  One CTA per row;
-// rows with one partial result in all were written by the decode kernel and
-// are skipped.  Launched as a programmatic dependent of the decode kernel:
-// those rows leave before the wait, during the decode's tail; the others
-// wait for the decode grid's writes before reading.
+// Merge the partitions of each (sequence, query head) row.  Rows with one
+// partial result in all were written by the decode kernel and are skipped.
+// Launched as a programmatic dependent of the decode kernel: the CTAs of
+// sequences with one partition leave before the wait, during the decode's
+// tail; the others wait for the decode grid's writes before reading.
+// STREAM: one CTA per row (grid Hq x B); else one CTA per sequence and 8
+// query heads (grid ceil(Hq / 8) x B), a warp per row.
 template <typename T, int D, bool STREAM>
-__global__ void __launch_bounds__(STREAM ? kReduceThreads : kReduceSmallThreads)
-    lse_reduce_kernel(const DecodeArgs a) {
-    const int h = blockIdx.x;
+__global__ void __launch_bounds__(kReduceThreads, 1) lse_reduce_kernel(const DecodeArgs a) {
     const int b = blockIdx.y;
     // the partition count depends only on the inputs, not on the decode
     // grid's output: rows with one partial result leave before the wait
@@ -219,14 +210,17 @@ __global__ void __launch_bounds__(STREAM ? kReduceThreads : kReduceSmallThreads)
     if (sp.direct) return;
     const int np = sp.slot0 + sp.np;  // the group pass's slots, then this row's partitions
     pdl_wait_primary();
-    const int64_t row = (int64_t)b * a.num_q_heads + h;
-    const float* ml = a.ws_ml + row * a.ws_slots * 2;
-    const float* o = a.ws_o + row * a.ws_slots * D;
-    T* out_row = reinterpret_cast<T*>(a.out) + row * D;
-    if constexpr (STREAM)
-        merge_partials<T, D>(ml, 2, o, np, out_row, a.status);
-    else
-        merge_partials_small<T, D>(ml, 2, o, D, np, out_row);
+    if constexpr (STREAM) {
+        const int64_t row = (int64_t)b * a.num_q_heads + blockIdx.x;
+        merge_partials<T, D>(a.ws_ml + row * a.ws_slots * 2, 2, a.ws_o + row * a.ws_slots * D,
+                             np, reinterpret_cast<T*>(a.out) + row * D, a.status);
+    } else {
+        const int h = blockIdx.x * kReduceRowsPerCta + (threadIdx.x >> 5);
+        if (h >= a.num_q_heads) return;
+        const int64_t row = (int64_t)b * a.num_q_heads + h;
+        merge_row_warp<T, D>(a.ws_ml + row * a.ws_slots * 2, a.ws_o + row * a.ws_slots * D, np,
+                             reinterpret_cast<T*>(a.out) + row * D, threadIdx.x & 31);
+    }
 }
 
 // Launch the reduce after the decode kernel on the same stream, as a
@@ -236,7 +230,7 @@ template <typename T, int D>
 cudaError_t launch_lse_reduce(const DecodeArgs& a, cudaStream_t stream) {
     const bool streamed = a.ws_slots >= kReduceStreamSlots;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.num_q_heads, a.num_seqs, 1);
+    cfg.blockDim = dim3(kReduceThreads, 1, 1);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -244,14 +238,15 @@ cudaError_t launch_lse_reduce(const DecodeArgs& a, cudaStream_t stream) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (!streamed) {
-        cfg.blockDim = dim3(kReduceSmallThreads, 1, 1);
+        cfg.gridDim = dim3((a.num_q_heads + kReduceRowsPerCta - 1) / kReduceRowsPerCta,
+                           a.num_seqs, 1);
         cfg.dynamicSmemBytes = 0;
         return cudaLaunchKernelEx(&cfg, lse_reduce_kernel<T, D, false>, a);
     }
     static SmemAttr smem_attr;
     cudaError_t e = smem_attr.ensure(lse_reduce_kernel<T, D, true>, ReduceCfg<D>::SMEM);
     if (e != cudaSuccess) return e;
-    cfg.blockDim = dim3(kReduceThreads, 1, 1);
+    cfg.gridDim = dim3(a.num_q_heads, a.num_seqs, 1);
     cfg.dynamicSmemBytes = ReduceCfg<D>::SMEM;
     return cudaLaunchKernelEx(&cfg, lse_reduce_kernel<T, D, true>, a);
 }
