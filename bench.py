@@ -154,6 +154,10 @@ KERNEL_SOURCES = {
 }
 
 
+SCHEDULE_NAMES = {"items": "work list, longest partition first",
+                  "order": "longest sequence first", "none": "batch order"}
+
+
 def kernel_source_digest(variant: str) -> str:
     import hashlib
     h = hashlib.sha256()
@@ -380,15 +384,21 @@ class Workload:
             self.vnew = self.vc.view(-1, H, bs, D)[sb_idx, :, so_idx, :].contiguous()
         self.out = torch.empty_like(self.q)
         self.mcl = mcl = inp.max_context_len
-        # schedule the longest sequences first (host-side order from host lengths)
-        order_np = pkv.pkv_decode_schedule_order(inp.context_lens) if args.order else None
-        self.order = dev(order_np) if order_np is not None else None
-        self.P = P = partition
         self.W = W = window
         span = min(mcl, W + bs - 1) if W > 0 else mcl
+        self.Pused = partition or pkv.pkv_decode_default_partition(B, H, span)
+        # the schedule, from host lengths: a work list of (sequence, partition)
+        # pairs longest first (cut with the resolved partition size), or the
+        # sequences longest first over the partition grid, or batch order
+        self.order = self.items = None
+        if args.schedule == "items":
+            self.items = dev(pkv.pkv_decode_schedule_items(inp.context_lens, bs, self.Pused, W))
+            partition = self.Pused
+        elif args.schedule == "order":
+            self.order = dev(pkv.pkv_decode_schedule_order(inp.context_lens))
+        self.P = P = partition
         ws_bytes = pkv.pkv_decode_workspace_size(B, cfg.num_q_heads, H, D, span, P)
         self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
-        self.Pused = P or pkv.pkv_decode_default_partition(B, H, span)
         self.launches_per_step = 1 + 1 + (1 if math.ceil(span / self.Pused) > 1 else 0)
         kvd = "e4m3" if e4m3 else None
         self.step_bytes = step_bytes(cfg, lens, W, kvd, per_page)
@@ -402,12 +412,13 @@ class Workload:
             pkv.pkv_paged_attention_decode_e4m3(
                 self.out, self.q, self.kc, self.vc, self.ks, self.vs, self.bt, self.cl, c.scale,
                 c.block_size, self.mcl, partition_size=self.P, workspace=self.ws,
-                seq_order=self.order, sliding_window=self.W, kernel=self.kern, stream=stream)
+                seq_order=self.order, items=self.items, sliding_window=self.W, kernel=self.kern,
+                stream=stream)
         else:
             pkv.pkv_paged_attention_decode(
                 self.out, self.q, self.kc, self.vc, self.bt, self.cl, c.scale, c.block_size,
                 self.mcl, partition_size=self.P, workspace=self.ws, seq_order=self.order,
-                sliding_window=self.W, kernel=self.kern, stream=stream)
+                items=self.items, sliding_window=self.W, kernel=self.kern, stream=stream)
 
     def append(self, stream):
         if self.e4m3:
@@ -520,7 +531,7 @@ def run_ours(args, cfg):
     ms, dec_ms = median_block(blocks, decs)
 
     # ---- end to end through the public API: every step copies its inputs
-    # (q, the new tokens' K/V, slots, tables, lengths, schedule order) from
+    # (q, the new tokens' K/V, slots, tables, lengths, schedule) from
     # pinned host memory and reads its output back.  The inputs of a step are
     # packed in one pinned buffer (one upload), and the C ABI is called with
     # argument lists prepared once, so the host keeps ahead of the GPU.  Two
@@ -532,6 +543,8 @@ def run_ours(args, cfg):
               ("cl", w.cl)]
     if w.order is not None:
         fields.append(("order", w.order))
+    if w.items is not None:
+        fields.append(("items", w.items))
     offs, total = {}, 0
     for name, t in fields:
         offs[name] = total
@@ -564,21 +577,29 @@ def run_ours(args, cfg):
             spb = 1 if w.per_page else 0
             append_args = (kp, vp, ptr["knew"], ptr["vnew"], ksp, vsp, spb, ptr["slots"], B, H, D,
                            bs, N_blocks, dt_code, c_stream)
+            sched = ((ptr["items"], w.items.shape[0]) if w.items is not None
+                     else (ptr.get("order"),))
             decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ksp, vsp,
-                           spb, ptr["bt"], ptr["cl"], ptr.get("order"), B, cfg.num_q_heads,
+                           spb, ptr["bt"], ptr["cl"], *sched, B, cfg.num_q_heads,
                            H, D, bs, w.bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
                            ctypes.c_void_p(ws.data_ptr()), ws.numel(), w.kern, c_stream)
         else:
             append_args = (kp, vp, ptr["knew"], ptr["vnew"], ptr["slots"], B, H, D, bs,
                            N_blocks, dt_code, c_stream)
+            sched = ((ptr["items"], w.items.shape[0]) if w.items is not None
+                     else (ptr.get("order"),))
             decode_args = (ctypes.c_void_p(d_out[j].data_ptr()), ptr["q"], kp, vp, ptr["bt"],
-                           ptr["cl"], ptr.get("order"), B, cfg.num_q_heads, H, D, bs,
+                           ptr["cl"], *sched, B, cfg.num_q_heads, H, D, bs,
                            w.bt.shape[1], N_blocks, mcl, cfg.scale, W, dt_code, P,
                            ctypes.c_void_p(ws.data_ptr()), ws.numel(), w.kern, c_stream)
         calls.append((append_args, decode_args))
     c_append = pkv.lib.pkv_kv_cache_append_e4m3 if w.e4m3 else pkv.lib.pkv_kv_cache_append
-    c_decode = (pkv.lib.pkv_paged_attention_decode_e4m3 if w.e4m3
-                else pkv.lib.pkv_paged_attention_decode)
+    if w.items is not None:
+        c_decode = (pkv.lib.pkv_paged_attention_decode_e4m3_items if w.e4m3
+                    else pkv.lib.pkv_paged_attention_decode_items)
+    else:
+        c_decode = (pkv.lib.pkv_paged_attention_decode_e4m3 if w.e4m3
+                    else pkv.lib.pkv_paged_attention_decode)
 
     def e2e_step(i):
         j = i % 2
@@ -644,7 +665,7 @@ def run_ours(args, cfg):
             "dtype": "e4m3" if w.e4m3 else cfg.dtype, "data": "synthetic",
             "config": workload_config(cfg, w.lens, world, args.tables, w.W, args.kv),
             "impl_config": {"partition_size": w.Pused, "kernel": args.kernel,
-                            "schedule": "longest-first" if args.order else "batch order"},
+                            "schedule": SCHEDULE_NAMES[args.schedule]},
             "timing": {"blocks": len(blocks), "steps_per_block": args.steps,
                        "block_ms_median": round(ms, 4), "block_ms_min": round(min(blocks), 4),
                        "block_ms_max": round(max(blocks), 4),
@@ -670,7 +691,7 @@ def run_ours(args, cfg):
                 line["also"].append({
                     "config": workload_config(w2.cfg, w2.lens, world, args.tables, 0, w2.kv),
                     "impl_config": {"partition_size": w2.Pused, "kernel": args.kernel,
-                                    "schedule": "longest-first" if args.order else "batch order"},
+                                    "schedule": SCHEDULE_NAMES[args.schedule]},
                     "value": round(v2, 2), "unit": "GB/s", "ms_per_step": round(st, 5),
                     "tokens_per_s": round(world * w2.cfg.num_seqs / (st * 1e-3), 1),
                     "pct_of_hbm_peak": round(100 * v2 / world / peak, 2),
@@ -955,8 +976,12 @@ def main():
     ap.add_argument("--tables", choices=["shuffled", "identity"], default="shuffled",
                     help="physical block ids: a seeded permutation of the pool, or the "
                          "identity (each sequence's pages contiguous in memory)")
-    ap.add_argument("--no-order", dest="order", action="store_false",
-                    help="schedule sequences in batch order instead of longest first")
+    ap.add_argument("--schedule", choices=["items", "order", "none"], default="items",
+                    help="items: a work list of (sequence, partition) pairs, longest "
+                         "partition first; order: sequences longest first over the partition "
+                         "grid; none: batch order")
+    ap.add_argument("--no-order", dest="schedule", action="store_const", const="none",
+                    help="the same as --schedule none")
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of oracle work for the cpu_baseline field")
     ap.add_argument("--ref-budget", type=float, default=90.0,

@@ -90,7 +90,7 @@ typedef enum { PKV_KERNEL_AUTO = 0, PKV_KERNEL_SIMT = 1, PKV_KERNEL_MMA = 2 } pk
 #define PKV_DEV_BAD_LEN 2u      /* a context length < 0 or past the caller's bounds */
 #define PKV_DEV_BAD_SLOT 4u     /* a slot at or past num_blocks * block_size */
 #define PKV_DEV_TIMEOUT 8u      /* a bounded wait inside a kernel gave up */
-#define PKV_DEV_BAD_ORDER 16u   /* a seq_order entry outside [0, num_seqs) */
+#define PKV_DEV_BAD_ORDER 16u   /* a seq_order entry outside [0, num_seqs), or a bad work item */
 #define PKV_DEV_DRAIN_TIMEOUT 32u /* after a wait gave up, a copy still had not landed
                                      when the kernel's block left (see below) */
 #define PKV_DEV_BAD_GROUP 64u   /* a shared-prefix group whose members disagree
@@ -367,6 +367,57 @@ PKV_API int pkv_decode_prefix_groups(const int32_t* block_tables, const int32_t*
  */
 PKV_API int pkv_decode_schedule_order(const int32_t* context_lens, int num_seqs,
                                       int32_t* order_out);
+
+/*
+ * Host helper: the work list of a decode -- every (sequence, partition) pair
+ * that has tokens to attend, longest partition first (ties by sequence, then
+ * partition), for pkv_paged_attention_decode_items and
+ * pkv_paged_attention_decode_e4m3_items.  Sequence b of length L (host
+ * context_lens) attends to [lo, L), lo = max(0, L - sliding_window) with a
+ * window (else 0); its partitions of partition_size tokens start at the
+ * block holding lo, so it has ceil((L - lo + lo % block_size) /
+ * partition_size) of them, and one (empty: the zero row) when L is 0.
+ * items_out receives 2 int32 per pair, (sequence, partition); *num_items
+ * their number.  partition_size must be the decode's (a multiple of 64 in
+ * [64, 8192]: resolve a default with pkv_decode_default_partition).
+ * Returns PKV_OK, PKV_EINVAL (bad sizes, a negative length) or PKV_EBOUNDS
+ * (more pairs than item_capacity; *num_items then holds the number needed).
+ */
+PKV_API int pkv_decode_schedule_items(const int32_t* context_lens, int num_seqs, int block_size,
+                                      int partition_size, int sliding_window,
+                                      int32_t* items_out, int item_capacity, int* num_items);
+
+/*
+ * pkv_paged_attention_decode over a work list instead of a schedule order:
+ * one CTA per (item, KV head) -- no CTA for a partition a sequence does not
+ * have, and partitions in the list's order (pkv_decode_schedule_items:
+ * longest first).  items: device int32 pairs (sequence, partition),
+ * num_items of them, 1 <= num_items <= 65535; partition_size: the one the
+ * list was cut with (> 0).  Every partition a sequence has must be listed
+ * once (else rows stay unwritten or partial); an item whose sequence is
+ * outside [0, num_seqs) or whose partition is negative is skipped and
+ * flagged (PKV_DEV_BAD_ORDER), one past the sequence's partitions is
+ * skipped.  Results equal pkv_paged_attention_decode's with the same
+ * partition_size, bit for bit.  The other arguments and the workspace are
+ * as there.
+ */
+PKV_API int pkv_paged_attention_decode_items(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* items,
+    int num_items, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int num_blocks, int max_context_len, float scale, int sliding_window,
+    pkv_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes,
+    pkv_kernel kernel, pkv_stream_t stream);
+
+/* pkv_paged_attention_decode_e4m3 over a work list (as above). */
+PKV_API int pkv_paged_attention_decode_e4m3_items(
+    void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+    const float* v_scale, int scale_per_block, const int32_t* block_tables,
+    const int32_t* context_lens, const int32_t* items, int num_items, int num_seqs,
+    int num_q_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+    int num_blocks, int max_context_len, float scale, int sliding_window, pkv_dtype dtype,
+    int partition_size, void* workspace, size_t workspace_bytes, pkv_kernel kernel,
+    pkv_stream_t stream);
 
 /*
  * KV append: the key and value of each new token go into the slot the block

@@ -32,7 +32,8 @@ __all__ = [
     "PKV_KERNEL_SIMT", "PKV_KERNEL_MMA", "PKV_DEV_BAD_BLOCK", "PKV_DEV_BAD_LEN",
     "PKV_DEV_BAD_SLOT", "PKV_DEV_TIMEOUT", "PKV_DEV_BAD_ORDER", "PKV_DEV_DRAIN_TIMEOUT",
     "torch_dtype_code",
-    "pkv_decode_schedule_order", "pkv_paged_attention_decode_e4m3", "pkv_kv_cache_append_e4m3",
+    "pkv_decode_schedule_order", "pkv_decode_schedule_items", "pkv_paged_attention_decode_e4m3",
+    "pkv_kv_cache_append_e4m3",
     "pkv_paged_attention_decode_prefix_groups", "pkv_decode_prefix_groups",
     "pkv_decode_prefix_groups_workspace_size", "PKV_DEV_BAD_GROUP",
     "PKV_E4M3", "pkv_debug_wait_timeout",
@@ -82,12 +83,29 @@ def pkv_decode_workspace_size(num_seqs: int, num_q_heads: int, num_kv_heads: int
                                              max_context_len, partition_size))
 
 
+def _check_order(seq_order, items, num_seqs: int, partition_size: int) -> None:
+    if seq_order is not None and items is not None:
+        raise PagedKVError(_b.PKV_EINVAL, "give seq_order or items, not both")
+    if seq_order is not None:
+        _dev(seq_order, "seq_order")
+        if seq_order.dtype != torch.int32 or seq_order.numel() != num_seqs:
+            raise PagedKVError(_b.PKV_EINVAL, "seq_order must be int32 [num_seqs]")
+    if items is not None:
+        _dev(items, "items")
+        if items.dtype != torch.int32 or items.dim() != 2 or items.shape[1] != 2 or \
+                not items.is_contiguous():
+            raise PagedKVError(_b.PKV_EINVAL, "items must be a contiguous int32 [n, 2] tensor")
+        if partition_size <= 0:
+            raise PagedKVError(_b.PKV_EINVAL, "a work list needs its partition_size")
+
+
 def pkv_paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
                                v_cache: torch.Tensor, block_tables: torch.Tensor,
                                context_lens: torch.Tensor, scale: float, block_size: int,
                                max_context_len: int, *, partition_size: int = 0,
                                workspace: torch.Tensor | None = None,
                                seq_order: torch.Tensor | None = None,
+                               items: torch.Tensor | None = None,
                                sliding_window: int = 0,
                                kernel: int = PKV_KERNEL_AUTO, stream=None) -> torch.Tensor:
     """out [B, Hq, D] <- paged decode attention (see pkv_paged_attention_decode
@@ -95,15 +113,15 @@ def pkv_paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torc
     int32 [B, max_blocks]; context_lens int32 [B]; max_context_len is a host
     bound of context_lens.  workspace: a CUDA tensor of at least
     pkv_decode_workspace_size(...) bytes when sequences span partitions.
-    seq_order: optional int32 [B] schedule order (pkv_decode_schedule_order).
+    seq_order: optional int32 [B] schedule order (pkv_decode_schedule_order);
+    or items: an int32 [n, 2] work list (pkv_decode_schedule_items, cut with
+    this partition_size, which must then be given) for
+    pkv_paged_attention_decode_items.
     sliding_window: 0, or attend only to each sequence's last W tokens."""
     for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
                  (block_tables, "block_tables"), (context_lens, "context_lens")):
         _dev(t, n)
-    if seq_order is not None:
-        _dev(seq_order, "seq_order")
-        if seq_order.dtype != torch.int32 or seq_order.numel() != q.shape[0]:
-            raise PagedKVError(_b.PKV_EINVAL, "seq_order must be int32 [num_seqs]")
+    _check_order(seq_order, items, q.shape[0], partition_size)
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise PagedKVError(_b.PKV_EINVAL, "block_tables / context_lens must be int32")
     if not (q.dtype == out.dtype == k_cache.dtype == v_cache.dtype):
@@ -118,6 +136,15 @@ def pkv_paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torc
     if workspace is not None:
         _dev(workspace, "workspace")
         ws_bytes = workspace.numel() * workspace.element_size()
+    if items is not None:
+        check(lib.pkv_paged_attention_decode_items(
+            _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+            _ptr(context_lens), _ptr(items), items.shape[0], B, Hq, Hkv, D, bs,
+            block_tables.shape[1], N, int(max_context_len), float(scale), int(sliding_window),
+            torch_dtype_code(q.dtype), int(partition_size), _ptr(workspace), ws_bytes,
+            int(kernel), _stream(stream)),
+            "pkv_paged_attention_decode_items")
+        return out
     check(lib.pkv_paged_attention_decode(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         _ptr(context_lens), _ptr(seq_order), B, Hq, Hkv, D, bs, block_tables.shape[1], N,
@@ -134,20 +161,19 @@ def pkv_paged_attention_decode_e4m3(out: torch.Tensor, q: torch.Tensor, k_cache:
                                     max_context_len: int, *, partition_size: int = 0,
                                     workspace: torch.Tensor | None = None,
                                     seq_order: torch.Tensor | None = None,
+                                    items: torch.Tensor | None = None,
                                     sliding_window: int = 0, kernel: int = PKV_KERNEL_AUTO,
                                     stream=None) -> torch.Tensor:
     """Paged decode over FP8 E4M3 pages (pkv_paged_attention_decode_e4m3 in
     pagedkv.h): k_cache/v_cache torch.float8_e4m3fn [N, Hkv, block_size, D];
     k_scale/v_scale float32 [Hkv], or [N, Hkv] for a scale per page; q and
-    out fp16 or bf16."""
+    out fp16 or bf16.  items: a work list as for pkv_paged_attention_decode
+    (pkv_paged_attention_decode_e4m3_items)."""
     for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
                  (k_scale, "k_scale"), (v_scale, "v_scale"), (block_tables, "block_tables"),
                  (context_lens, "context_lens")):
         _dev(t, n)
-    if seq_order is not None:
-        _dev(seq_order, "seq_order")
-        if seq_order.dtype != torch.int32 or seq_order.numel() != q.shape[0]:
-            raise PagedKVError(_b.PKV_EINVAL, "seq_order must be int32 [num_seqs]")
+    _check_order(seq_order, items, q.shape[0], partition_size)
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise PagedKVError(_b.PKV_EINVAL, "block_tables / context_lens must be int32")
     if k_cache.dtype != torch.float8_e4m3fn or v_cache.dtype != torch.float8_e4m3fn:
@@ -166,6 +192,15 @@ def pkv_paged_attention_decode_e4m3(out: torch.Tensor, q: torch.Tensor, k_cache:
     if workspace is not None:
         _dev(workspace, "workspace")
         ws_bytes = workspace.numel() * workspace.element_size()
+    if items is not None:
+        check(lib.pkv_paged_attention_decode_e4m3_items(
+            _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+            per_block, _ptr(block_tables), _ptr(context_lens), _ptr(items), items.shape[0], B,
+            Hq, Hkv, D, bs, block_tables.shape[1], N, int(max_context_len), float(scale),
+            int(sliding_window), torch_dtype_code(q.dtype), int(partition_size),
+            _ptr(workspace), ws_bytes, int(kernel), _stream(stream)),
+            "pkv_paged_attention_decode_e4m3_items")
+        return out
     check(lib.pkv_paged_attention_decode_e4m3(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
         per_block, _ptr(block_tables), _ptr(context_lens), _ptr(seq_order), B, Hq, Hkv, D, bs,
@@ -283,6 +318,27 @@ def pkv_paged_attention_decode_prefix_groups(
         torch_dtype_code(q.dtype), int(partition_size), _ptr(workspace), ws_bytes, int(kernel),
         _stream(stream)), "pkv_paged_attention_decode_prefix_groups")
     return out
+
+
+def pkv_decode_schedule_items(context_lens, block_size: int, partition_size: int,
+                              sliding_window: int = 0):
+    """Host int32 array [n, 2] of (sequence, partition) pairs, longest
+    partition first, for the decode's items argument (pkv_decode_schedule_items
+    in pagedkv.h)."""
+    import numpy as np
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    n = _b._c.c_int(0)
+    cap = int(np.maximum(lens, 0).sum() // max(1, int(partition_size))) + 2 * lens.size + 1
+    while True:
+        items = np.empty((cap, 2), dtype=np.int32)
+        rc = lib.pkv_decode_schedule_items(lens.ctypes.data, lens.size, int(block_size),
+                                           int(partition_size), int(sliding_window),
+                                           items.ctypes.data, cap, _b._c.byref(n))
+        if rc != _b.PKV_EBOUNDS or n.value <= cap:
+            break
+        cap = n.value
+    check(rc, "pkv_decode_schedule_items")
+    return items[:n.value].copy()
 
 
 def pkv_decode_schedule_order(context_lens):

@@ -48,6 +48,14 @@ SIGNATURES = {
                                                _i32, _f32, _i32, _i32, _i32, _vp, _sz, _i32,
                                                _vp]),
     "pkv_decode_schedule_order": (_i32, [_vp, _i32, _vp]),
+    "pkv_decode_schedule_items": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp]),
+    "pkv_paged_attention_decode_items": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
+                                                _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
+                                                _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
+    "pkv_paged_attention_decode_e4m3_items": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
+                                                     _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                                                     _i32, _i32, _i32, _i32, _f32, _i32, _i32,
+                                                     _i32, _vp, _sz, _i32, _vp]),
     "pkv_paged_attention_decode_prefix_groups": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                                         _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                                         _i32, _i32, _i32, _i32, _i32, _f32, _i32,

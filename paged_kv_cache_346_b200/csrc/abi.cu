@@ -135,6 +135,10 @@ int plan_decode(const DecodeRequest& r, DecodePlan* plan) {
         return PKV_EINVAL;
     if (r.kernel != PKV_KERNEL_AUTO && r.kernel != PKV_KERNEL_SIMT && r.kernel != PKV_KERNEL_MMA)
         return PKV_EINVAL;
+    // a work list: cut with an explicit partition size, instead of a schedule order
+    if (r.items && (r.seq_order || r.partition_size == 0 ||
+                    (r.num_seqs > 0 && (r.num_items < 1 || r.num_items > 65535))))
+        return PKV_EINVAL;
     if (r.head_dim != 64 && r.head_dim != 128 && r.head_dim != 256) return PKV_EUNSUPPORTED;
     if (r.block_size != 16 && r.block_size != 32 && r.block_size != 64) return PKV_EUNSUPPORTED;
     if (r.dtype == PKV_F32 && r.head_dim == 256) return PKV_EUNSUPPORTED;
@@ -200,6 +204,8 @@ DecodeArgs decode_args(const DecodeRequest& r, const DecodePlan& plan, void* wor
     a.block_tables = r.block_tables;
     a.context_lens = r.context_lens;
     a.seq_order = r.seq_order;
+    a.items = r.items;
+    a.num_items = r.items ? r.num_items : 0;
     a.k_scale = r.e4m3 ? r.k_scale : nullptr;
     a.v_scale = r.e4m3 ? r.v_scale : nullptr;
     a.scale_per_block = r.e4m3 ? r.scale_per_block : 0;
@@ -423,6 +429,43 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
                           context_lens, seq_order, num_seqs, num_q_heads, num_kv_heads,
                           head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
                           scale, sliding_window, dtype, partition_size, kernel};
+    return pkv::decode_impl(r, workspace, workspace_bytes, stream);
+}
+
+int pkv_paged_attention_decode_items(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* items,
+    int num_items, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int num_blocks, int max_context_len, float scale, int sliding_window,
+    pkv_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes,
+    pkv_kernel kernel, pkv_stream_t stream) {
+    NvtxRange range("pkv_paged_attention_decode_items");
+    if (!items && num_seqs > 0) return PKV_EINVAL;
+    DecodeRequest r{out, q, k_cache, v_cache, nullptr, nullptr, 0, false, block_tables,
+                    context_lens, nullptr, num_seqs, num_q_heads, num_kv_heads,
+                    head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
+                    scale, sliding_window, dtype, partition_size, kernel};
+    r.items = items;
+    r.num_items = num_items;
+    return pkv::decode_impl(r, workspace, workspace_bytes, stream);
+}
+
+int pkv_paged_attention_decode_e4m3_items(
+    void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+    const float* v_scale, int scale_per_block, const int32_t* block_tables,
+    const int32_t* context_lens, const int32_t* items, int num_items, int num_seqs,
+    int num_q_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+    int num_blocks, int max_context_len, float scale, int sliding_window, pkv_dtype dtype,
+    int partition_size, void* workspace, size_t workspace_bytes, pkv_kernel kernel,
+    pkv_stream_t stream) {
+    NvtxRange range("pkv_paged_attention_decode_e4m3_items");
+    if (!items && num_seqs > 0) return PKV_EINVAL;
+    DecodeRequest r{out, q, k_cache, v_cache, k_scale, v_scale, scale_per_block, true,
+                    block_tables, context_lens, nullptr, num_seqs, num_q_heads,
+                    num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                    max_context_len, scale, sliding_window, dtype, partition_size, kernel};
+    r.items = items;
+    r.num_items = num_items;
     return pkv::decode_impl(r, workspace, workspace_bytes, stream);
 }
 

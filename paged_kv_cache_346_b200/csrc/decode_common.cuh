@@ -18,6 +18,7 @@ struct DecodeArgs {
     const int32_t* block_tables;  // [B, max_blocks_per_seq]
     const int32_t* context_lens;  // [B]
     const int32_t* seq_order;     // [B] schedule order (CTA z takes sequence seq_order[z]), or null
+    const int32_t* items;         // [num_items][2] work list: CTA z takes (sequence, partition), or null
     const float* k_scale;         // scales of E4M3 K / V pages, or null: [Hkv], or
     const float* v_scale;         // [num_blocks, Hkv] when scale_per_block
     // shared-prefix decode: tokens [0, seq_start[b]) of sequence b were
@@ -29,6 +30,7 @@ struct DecodeArgs {
     float* ws_ml;                 // [B, Hq, ws_slots, 2] (m in log2 units, l)
     unsigned int* status;
     int num_seqs;
+    int num_items;                // work-list length (items only)
     int num_q_heads;
     int num_kv_heads;
     int group;                    // Hq / Hkv
@@ -57,6 +59,33 @@ __device__ __forceinline__ int scheduled_seq(const DecodeArgs& a, int z, bool re
         return -1;
     }
     return b;
+}
+
+// The (sequence, partition) this CTA works on: with a work list, item z of
+// it (grid x is 1); else grid z through the schedule order and partition
+// grid x.  b = -1: a bad order entry or item (flagged by the CTA of head
+// chunk 0).
+struct CtaUnit {
+    int b, part;
+};
+__device__ __forceinline__ CtaUnit cta_unit(const DecodeArgs& a, int tid) {
+    if (a.items) {
+        const int b = a.items[2 * blockIdx.z], part = a.items[2 * blockIdx.z + 1];
+        if ((unsigned)b >= (unsigned)a.num_seqs || part < 0) {
+            if (tid == 0 && blockIdx.y == 0) flag(a.status, PKV_DEV_BAD_ORDER);
+            return {-1, 0};
+        }
+        return {b, part};
+    }
+    const int part = blockIdx.x;
+    return {scheduled_seq(a, blockIdx.z, tid == 0 && part == 0 && blockIdx.y == 0), part};
+}
+
+// The decode grid: (partitions, KV heads x head chunks, sequences), or one
+// CTA per (item, KV head x head chunk) with a work list.
+__host__ __forceinline__ dim3 decode_grid(const DecodeArgs& a) {
+    return a.items ? dim3(1, a.num_kv_heads * a.head_chunks, a.num_items)
+                   : dim3(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
 }
 
 // Length of sequence b as the kernels use it: negative or too long lengths

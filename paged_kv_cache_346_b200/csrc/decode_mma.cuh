@@ -174,7 +174,9 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
     const int g = lane >> 2, t4 = lane & 3;
     const int kvh = blockIdx.y / a.head_chunks;
     const int hc = blockIdx.y - kvh * a.head_chunks;
-    const int part = blockIdx.x;
+    // (sequence, partition): the group pass takes partition grid x of group z
+    const CtaUnit unit = GROUPS ? CtaUnit{0, (int)blockIdx.x} : cta_unit(a, tid);
+    const int part = unit.part;
     const int h0 = kvh * a.group + hc * NH;
     const bool reporter = (tid == 0 && part == 0 && blockIdx.y == 0);
     int b, nh, nmem = 0;
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
         }
     } else {
         nh = min(NH, a.group - hc * NH);
-        b = scheduled_seq(a, blockIdx.z, reporter);
+        b = unit.b;
         if (b < 0) return;
         pf = table_prefetch(a, b, part, a.partition_size / BS, tid);
         sp = seq_span(a, b, reporter);
@@ -606,7 +608,7 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     e = make_cache_tensor_map(&tv, a.v_cache, 2, bf, D, rows, 16);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
+    const dim3 grid = decode_grid(a);
     e = launch_decode_kernel(kern, grid, dim3(NW * 32), C::smem_bytes(a.partition_size), stream,
                              a, tk, tv);
     if (e != cudaSuccess || a.ws_slots <= 1) return e;

@@ -441,11 +441,12 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
     const int g = lane >> 2, t4 = lane & 3;
     const int kvh = blockIdx.y / a.head_chunks;
     const int hc = blockIdx.y - kvh * a.head_chunks;
-    const int part = blockIdx.x;
+    const CtaUnit unit = cta_unit(a, tid);  // (sequence, partition)
+    const int part = unit.part;
     const int h0 = kvh * a.group + hc * NH;
     const int nh = min(NH, a.group - hc * NH);
     const bool reporter = (tid == 0 && part == 0 && blockIdx.y == 0);
-    const int b = scheduled_seq(a, blockIdx.z, reporter);
+    const int b = unit.b;
     if (b < 0) return;
 
     const TablePrefetch pf = table_prefetch(a, b, part, a.partition_size / BS, tid);
@@ -677,7 +678,7 @@ cudaError_t launch_decode_mma_e4m3(const DecodeArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     e = make_cache_tensor_map(&tv, a.v_cache, 1, false, D, rows, 16);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
+    const dim3 grid = decode_grid(a);
     e = launch_decode_kernel(kern, grid, dim3(NW * 32), C::smem_bytes(a.partition_size), stream,
                              a, tk, tv);
     if (e != cudaSuccess || a.ws_slots <= 1) return e;

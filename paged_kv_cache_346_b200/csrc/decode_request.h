@@ -38,6 +38,8 @@ struct DecodeRequest {
     pkv_dtype dtype;
     int partition_size;           // 0 = the default for the shape
     pkv_kernel kernel;
+    const int32_t* items = nullptr;  // work list (pairs sequence, partition) instead of seq_order
+    int num_items = 0;
 };
 
 struct DecodePlan {

@@ -312,11 +312,12 @@ __global__ void __launch_bounds__(SimtCfg<T, D, BS, HG, NW, STAGES_, TC>::THREAD
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kvh = blockIdx.y / a.head_chunks;
     const int hc = blockIdx.y - kvh * a.head_chunks;
-    const int part = blockIdx.x;
+    const CtaUnit unit = cta_unit(a, tid);  // (sequence, partition)
+    const int part = unit.part;
     const int h0 = kvh * a.group + hc * HG;
     const int nh = min(HG, a.group - hc * HG);
     const bool reporter = (tid == 0 && part == 0 && blockIdx.y == 0);
-    const int b = scheduled_seq(a, blockIdx.z, reporter);
+    const int b = unit.b;
     if (b < 0) return;
 
     const TablePrefetch pf = table_prefetch(a, b, part, a.partition_size / BS, tid);
@@ -442,7 +443,7 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
     auto kern = decode_simt_kernel<T, D, BS, HG, NW, STAGES, TC>;
     cudaError_t e = attr.ensure(kern, C::smem_bytes(8192));
     if (e != cudaSuccess) return e;
-    dim3 grid(a.max_partitions, a.num_kv_heads * a.head_chunks, a.num_seqs);
+    const dim3 grid = decode_grid(a);
     e = launch_decode_kernel(kern, grid, dim3(C::THREADS), smem_simt, stream, a);
     if (e != cudaSuccess || a.ws_slots <= 1) return e;
     return launch_lse_reduce<T, D>(a, stream);
