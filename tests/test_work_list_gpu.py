@@ -69,12 +69,14 @@ def test_items_equal_the_grid_decode_and_the_oracle(dtype, Hq, Hkv, D, kernel, P
 
 
 @pytest.mark.parametrize("per_page", [False, True])
-@pytest.mark.parametrize("G", [1, 8])
-def test_e4m3_items_equal_the_grid_decode_and_the_oracle(per_page, G):
+@pytest.mark.parametrize("G,P,W", [(1, 512, 0), (8, 512, 0), (8, 1024, 0), (8, 1024, 700),
+                                   (8, 64, 0)])
+def test_e4m3_items_equal_the_grid_decode_and_the_oracle(per_page, G, P, W):
+    """2- and 4-warp CTAs (partitions up to 512 tokens, and over), with and
+    without a window, both scale modes."""
     inp = make_decode_inputs(_cfg("bf16", 2 * G, 2, 128, 16, RAGGED), seed=52 + G)
     pages = make_e4m3_pages(inp, 5, per_page=per_page)
     c = inp.cfg
-    P = 512
 
     def codes(a):
         return torch.from_numpy(np.ascontiguousarray(a)).cuda().view(torch.float8_e4m3fn)
@@ -82,20 +84,62 @@ def test_e4m3_items_equal_the_grid_decode_and_the_oracle(per_page, G):
     k, v = codes(pages.k_cache), codes(pages.v_cache)
     ks, vs = torch.from_numpy(pages.k_scale).cuda(), torch.from_numpy(pages.v_scale).cuda()
     q, bt, cl = to_device(inp.q, "bf16"), to_device(inp.block_tables), to_device(inp.context_lens)
-    items = torch.from_numpy(pkv.pkv_decode_schedule_items(inp.context_lens, 16, P)).cuda()
+    items = torch.from_numpy(
+        pkv.pkv_decode_schedule_items(inp.context_lens, 16, P, sliding_window=W)).cuda()
+    mcl = inp.max_context_len
+    span = min(mcl, W + 15) if W else mcl
     outs = []
     for kw in ({"items": items}, {"seq_order": None}):
         out = torch.full_like(q, float("nan"))
+        pkv.pkv_paged_attention_decode_e4m3(out, q, k, v, ks, vs, bt, cl, c.scale, 16, mcl,
+                                            partition_size=P, workspace=_ws(c, span, P),
+                                            sliding_window=W, **kw)
+        torch.cuda.synchronize()
+        outs.append(out)
+    assert torch.equal(outs[0], outs[1])
+    ref = oracle.paged_decode(inp.q, pages.k_cache, pages.v_cache, inp.block_tables,
+                              inp.context_lens, scale=c.scale, dtype="bf16", kv_dtype="e4m3",
+                              k_scale=pages.k_scale, v_scale=pages.v_scale, window=W)
+    assert_close(to_f64(outs[0]), ref, "bf16", f"E4M3 G {G} P {P} W {W} per_page {per_page}")
+    assert pkv.pkv_device_status(clear=True) == 0
+
+
+@pytest.mark.parametrize("per_page", [False, True])
+def test_e4m3_gqa_batch_shape_items(per_page):
+    """The GQA batch's shape with E4M3 pages at a reduced batch, 4096-token
+    partitions: every row against the oracle, and equal to the grid decode
+    bit for bit."""
+    g = np.random.default_rng(56)
+    lens = np.exp(g.normal(np.log(512), 1.0, size=200)).astype(np.int32).clip(32, 8192)
+    lens[:3] = (8192, 6000, 4097)
+    lens[7] = 0
+    inp = make_decode_inputs(_cfg("bf16", 64, 8, 128, 16, tuple(int(x) for x in lens)), seed=57)
+    pages = make_e4m3_pages(inp, 6, per_page=per_page)
+    c = inp.cfg
+
+    def codes(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).cuda().view(torch.float8_e4m3fn)
+
+    k, v = codes(pages.k_cache), codes(pages.v_cache)
+    ks, vs = torch.from_numpy(pages.k_scale).cuda(), torch.from_numpy(pages.v_scale).cuda()
+    q, bt, cl = to_device(inp.q, "bf16"), to_device(inp.block_tables), to_device(inp.context_lens)
+    items = torch.from_numpy(pkv.pkv_decode_schedule_items(inp.context_lens, 16, 4096)).cuda()
+    order = torch.from_numpy(pkv.pkv_decode_schedule_order(inp.context_lens)).cuda()
+    outs = []
+    for kw in ({"items": items}, {"seq_order": order}):
+        out = torch.full_like(q, float("nan"))
         pkv.pkv_paged_attention_decode_e4m3(out, q, k, v, ks, vs, bt, cl, c.scale, 16,
-                                            inp.max_context_len, partition_size=P,
-                                            workspace=_ws(c, inp.max_context_len, P), **kw)
+                                            inp.max_context_len, partition_size=4096,
+                                            workspace=_ws(c, inp.max_context_len, 4096), **kw)
         torch.cuda.synchronize()
         outs.append(out)
     assert torch.equal(outs[0], outs[1])
     ref = oracle.paged_decode(inp.q, pages.k_cache, pages.v_cache, inp.block_tables,
                               inp.context_lens, scale=c.scale, dtype="bf16", kv_dtype="e4m3",
                               k_scale=pages.k_scale, v_scale=pages.v_scale)
-    assert_close(to_f64(outs[0]), ref, "bf16", f"E4M3 G {G} per_page {per_page}")
+    got = to_f64(outs[0])
+    assert (got[7] == 0).all()
+    assert_close(got, ref, "bf16", f"E4M3 GQA shape per_page {per_page}")
     assert pkv.pkv_device_status(clear=True) == 0
 
 
