@@ -6,21 +6,47 @@
 
 namespace pkv {
 
-// 16 fp16 / bf16 values (two 16-byte vectors) -> 16 E4M3 codes of x / scale.
+// 16 fp16 / bf16 values (two 16-byte vectors) -> 16 E4M3 codes of x / scale,
+// the code of the float32 quotient rounded to nearest (ties to even,
+// saturating at the largest finite code).
+//
+// Fast path: q = x * r with r = 1 / scale (float32), within 2^-23 (relative)
+// of the true quotient, so the float32 quotient lies within 2^-22 of q.  The
+// E4M3 rounding is monotone, so if q (1 - 2^-20) and q (1 + 2^-20) -- each
+// rounded again, still bracketing it -- convert to the same code, that is
+// the code of the quotient.  Otherwise (q within ~2^-20 of a rounding
+// boundary between two codes: rare) the element takes the division itself.
+// Scales outside [2^-100, 2^100] (where r could lose precision) always take
+// the division.
 template <typename Tin>
 __device__ __forceinline__ uint4 quantise16(const uint4* src, float scale) {
     float f[16];
     Elem<Tin>::to_f32(src[0], f);
     Elem<Tin>::to_f32(src[1], f + 8);
+    const bool fast = scale >= 0x1p-100f && scale <= 0x1p100f;
+    const float r = 1.f / scale;
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         uint32_t x = 0;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const __nv_fp8_storage_t c =
-                __nv_cvt_float_to_fp8(f[4 * j + b] / scale, __NV_SATFINITE, __NV_E4M3);
-            x |= (uint32_t)c << (8 * b);
+        for (int b = 0; b < 4; b += 2) {
+            const float q0 = f[4 * j + b] * r, q1 = f[4 * j + b + 1] * r;
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+                make_float2(q0 * (1.f - 0x1p-20f), q1 * (1.f - 0x1p-20f)), __NV_SATFINITE,
+                __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+                make_float2(q0 * (1.f + 0x1p-20f), q1 * (1.f + 0x1p-20f)), __NV_SATFINITE,
+                __NV_E4M3);
+            uint32_t pair = lo;
+            if (!fast || lo != hi) {  // near a boundary: the exact quotients
+                const uint32_t c0 =
+                    __nv_cvt_float_to_fp8(f[4 * j + b] / scale, __NV_SATFINITE, __NV_E4M3);
+                const uint32_t c1 =
+                    __nv_cvt_float_to_fp8(f[4 * j + b + 1] / scale, __NV_SATFINITE, __NV_E4M3);
+                pair = c0 | (c1 << 8);
+            }
+            x |= (pair & 0xffffu) << (8 * b);
         }
         w[j] = x;
     }

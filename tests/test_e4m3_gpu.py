@@ -119,6 +119,42 @@ def test_append_e4m3_bit_exact(dtype, H, D, bs):
     assert ((K & 0x7F) == 0x7E).any() and ((V & 0x78) == 0).any()
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_append_e4m3_bit_exact_at_rounding_boundaries(dtype):
+    """Values whose quotient lies on, or within an ulp of, the midpoint
+    between two E4M3 codes (ties go to the even code): the append's fast
+    multiply-by-reciprocal path must hand these to the division and still
+    match the float32 quotient's rounding bit for bit."""
+    from workloads import round_to_dtype
+    H, D, bs, N = 4, 128, 16, 8
+    codes = np.arange(126, dtype=np.uint8)
+    vals = oracle.decode_bits(codes, "e4m3")
+    mids = (vals[:-1] + vals[1:]) / 2.0                       # 125 midpoints
+    scales = np.array([1.0, 3.0, 0.1, 2.0 ** -7], np.float32)  # one per KV head
+    T = 4
+    k = np.zeros((T, H, D), np.float64)
+    for h in range(H):
+        x = np.concatenate([mids, -mids, mids * (1 + 2 ** -9), mids * (1 - 2 ** -9)])
+        x = np.resize(x * scales[h], T * D).reshape(T, D)
+        k[:, h, :] = x
+    k = round_to_dtype(k, dtype)
+    v = k[::-1].copy()
+    slots = np.arange(T, dtype=np.int64) * bs + 3
+    K = np.zeros((N, H, bs, D), np.uint8)
+    V = np.zeros_like(K)
+    dK, dV = _codes(K), _codes(V)
+    sc = torch.from_numpy(scales).cuda()
+    pkv.pkv_kv_cache_append_e4m3(dK, dV, to_device(k, dtype), to_device(v, dtype), sc, sc,
+                                 torch.from_numpy(slots).cuda())
+    kv_cache_append_e4m3(K, V, k, v, slots, scales, scales, dtype)
+    torch.cuda.synchronize()
+    assert np.array_equal(dK.view(torch.uint8).cpu().numpy(), K)
+    assert np.array_equal(dV.view(torch.uint8).cpu().numpy(), V)
+    # the first head's first 125 quotients are exact ties: each went to the
+    # neighbour with the even code
+    assert np.all(K[3 // bs, 0, 3, :125] % 2 == 0)
+
+
 def test_append_e4m3_bad_slot_flagged():
     N, H, bs, D = 4, 2, 16, 128
     dK = _codes(np.zeros((N, H, bs, D), np.uint8))
