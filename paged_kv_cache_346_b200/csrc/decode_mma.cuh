@@ -396,6 +396,15 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
             constexpr bool SPLIT = std::is_same<T, __nv_bfloat16>::value;
             uint32_t pb[RB][2], pl[RB][2];
             float alpha_c[RB][2];
+            // 2^x: the hardware approximation where the fragments sit in
+            // registers (8-head tiles, head_dim <= 128); the other tiles keep
+            // exp2f, which there holds the register count
+            auto ex2 = [](float x) {
+                if constexpr (EARLY)
+                    return ex2_approx(x);
+                else
+                    return exp2f(x);
+            };
             if constexpr (NH == 8) {
                 // S = K Q^T: A rows = tokens g, g + 8, B column = head g
                 float s[4] = {0.f, 0.f, 0.f, 0.f};
@@ -422,11 +431,11 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                     mnew[j] = fmaxf(m[j], mx);
-                    alpha_c[0][j] = exp2f(m[j] - mnew[j]);
+                    alpha_c[0][j] = ex2(m[j] - mnew[j]);
                     m[j] = mnew[j];
                 }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) p[i] = exp2f(s[i] - mnew[i & 1]);
+                for (int i = 0; i < 4; ++i) p[i] = ex2(s[i] - mnew[i & 1]);
                 const uint32_t h0p = M::pack(p[0], p[1], pr[0], pr[1]);
                 const uint32_t h1p = M::pack(p[2], p[3], pr[2], pr[3]);
                 // P (tokens x heads) -> P^T fragments: head g, tokens 2 t4,
@@ -439,8 +448,10 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                     const uint32_t l1p = M::pack(p[2] - pr[2], p[3] - pr[3], r[2], r[3]);
                     pl[0][0] = movmatrix_trans(l0p);
                     pl[0][1] = movmatrix_trans(l1p);
+                    // the weights P.V uses, hi + lo; with the fragments in
+                    // registers the row sums take p itself, within 2^-18 p
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) pr[i] += r[i];  // the weights P.V uses, hi + lo
+                    for (int i = 0; i < 4; ++i) pr[i] = EARLY ? p[i] : pr[i] + r[i];
                 }
 #pragma unroll
                 for (int j = 0; j < 2; ++j) l[j] = l[j] * alpha_c[0][j] + (pr[j] + pr[2 + j]);
@@ -499,6 +510,25 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
             }
             // O^T += V^T P^T
             const bool partial = wvalid < 16 || wlo > 0;
+            if constexpr (EARLY) {
+                // the fragments are in registers: zero the values of masked
+                // tokens once (registers 0, 1: tokens 2 t4, 2 t4 + 1, low and
+                // high half; 2, 3: the same + 8), so the loop has no branch
+                if (partial) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int tk = 8 * j + 2 * t4;
+                        const uint32_t keep =
+                            (tk >= wlo && tk < wvalid ? 0x0000ffffu : 0u) |
+                            (tk + 1 >= wlo && tk + 1 < wvalid ? 0xffff0000u : 0u);
+#pragma unroll
+                        for (int ks = 0; ks < (EARLY ? KSTEPS : 1); ++ks) {
+                            vf[ks][2 * j] &= keep;
+                            vf[ks][2 * j + 1] &= keep;
+                        }
+                    }
+                }
+            }
 #pragma unroll
             for (int mt = 0; mt < KSTEPS; ++mt) {
                 uint32_t va[4];
@@ -508,7 +538,7 @@ __global__ void __launch_bounds__(NW * 32, (D <= 128 && NH == 8) ? 3 : 1)
                 } else {
                     ldsm_x4_trans(kaddr(mt) + SLICE_BYTES, va);
                 }
-                if (partial) {
+                if (!EARLY && partial) {
                     // zero values of masked tokens (0 * NaN would poison)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
