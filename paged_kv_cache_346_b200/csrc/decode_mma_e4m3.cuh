@@ -558,6 +558,13 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
 
     int stage = 0;       // it % STAGES
     uint32_t phase = 0;  // (it / STAGES) & 1
+    // per-page mode: the scales of the warp's first slice
+    float ks_next = 1.f, vs_next = 1.f;
+    if (PPB && EARLY && nslices > 0) {
+        const int64_t si = (int64_t)s_tab[(warp * 16) / BS] * a.num_kv_heads + kvh;
+        ks_next = a.k_scale[si];
+        vs_next = a.v_scale[si];
+    }
     for (int it = 0; it < nslices; ++it) {
         const bool ok =
             __all_sync(0xffffffffu, mbar_wait(full + warp * STAGES + stage, phase, a.status));
@@ -573,9 +580,20 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
         const int wlo = mask_lo - (it * TILE + warp * 16);
         const bool work = wlo < 16 && wlo < wvalid;
         const uint32_t kbase = ring_s + (uint32_t)(stage * 2 * SLICE_BYTES + lrow * 128);
-        // this slice's page scales (per-page mode): logits and P.V multipliers
+        // this slice's page scales (per-page mode): logits and P.V multipliers;
+        // with 8-head tiles at head_dim <= 128 loaded one slice ahead (their
+        // latency hides behind a slice's math; elsewhere that spills)
         float kmul = qmul, vmul = 1.f;
-        if (PPB && work) {
+        if constexpr (PPB && EARLY) {
+            kmul = qmul * ks_next;
+            vmul = vs_next;
+            if (it + 1 < nslices) {
+                const int64_t si =
+                    (int64_t)s_tab[((it + 1) * TILE + warp * 16) / BS] * a.num_kv_heads + kvh;
+                ks_next = a.k_scale[si];
+                vs_next = a.v_scale[si];
+            }
+        } else if (PPB && work) {
             const int64_t si =
                 (int64_t)s_tab[(it * TILE + warp * 16) / BS] * a.num_kv_heads + kvh;
             kmul = qmul * a.k_scale[si];
