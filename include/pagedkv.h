@@ -211,9 +211,13 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
  * by scale * k_scale (and the power of two) in fp32.
  * The CUDA-core kernel works in fp32 throughout, k_scale folded into q and
  * v_scale into the accumulator (per page: into that page's logits and
- * weights); the tensor-core kernel applies a page's v_scale in fp32 to that
- * page's P.V product, so P stays an fp16 value at most 256 whatever the
- * scales.
+ * weights).  The tensor-core kernel keeps each warp's P.V sums in units of a
+ * reference V scale vref: a page whose v_scale lies in [vref, 128 vref]
+ * enters with its weights times v_scale / vref (then at most 2^15, still an
+ * fp16 hi + lo pair with p's precision), any other page first moves vref to
+ * its v_scale / 8 and rescales the fp32 sums; the output is multiplied by
+ * vref.  The sums stay in fp32 range for the per-page V scales of a KV head
+ * within a factor 2^80 of one another.
  *
  * Arguments as pkv_paged_attention_decode, plus:
  *   k_cache, v_cache: device E4M3 codes [num_blocks, Hkv, block_size, head_dim].

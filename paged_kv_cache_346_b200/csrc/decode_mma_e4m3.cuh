@@ -34,9 +34,12 @@
 // an f16 normal); the logits are multiplied back by scale * log2(e) *
 // k_scale * 2^-e in fp32, and the output by v_scale.  With a scale per page,
 // a warp's 16-token slice lies in one block: its logits take that page's
-// k_scale, and its P.V product (a fresh fp32 accumulator) is added to the
-// output multiplied by that page's v_scale, so P stays an fp16 value at most
-// 256 whatever the scales.
+// k_scale, and the warp keeps its P.V sums in units of a reference V scale
+// vref.  A page whose v_scale lies in [vref, 128 vref] enters with its
+// weights times v_scale / vref (then at most 2^15: still an fp16 hi + lo
+// pair, no less precise than p itself); any other page first moves vref to
+// its v_scale / 8 and rescales the fp32 sums, as a rise of the reference max
+// does.  The warp's output is multiplied by vref.
 //
 // Each softmax weight p (fp32) enters the P.V product as two fp16 terms,
 // hi = fp16(p) and lo = fp16(p - hi), in two MMAs on the same V fragment: one
@@ -174,17 +177,19 @@ __device__ __forceinline__ float e4m3_prepare_q(QRow qrow, float mul,
 // the lazy reference max, and O^T += V^T P^T with P as fp16 hi + lo.  The
 // state (m, l, o) is the warp's; addr(kp) is the ldmatrix address of chunk
 // pair kp of the slice's K rows (V rows: + 16 D bytes); tokens outside
-// [wlo, wvalid) of the slice are masked.
+// [wlo, wvalid) of the slice are masked.  PPB: the weights enter P.V times
+// pmul, the page's V scale over the warp's reference (in [1, 128], so p pmul
+// is at most 2^15), while l sums the weights themselves.
 template <int D, int NH, bool PPB, bool EARLY, typename Addr>
 __device__ __forceinline__ void e4m3_slice_math(
     const uint32_t (&qa)[D / 16][NH == 16 ? 4 : 2], float (&m)[NH == 8 ? 2 : NH / 8],
     float (&l)[NH == 8 ? 2 : NH / 8], float (&o)[D / 16][NH / 8][4],
     const uint32_t (&kf)[EARLY ? D / 32 : 1][4], uint32_t (&vf)[EARLY ? D / 32 : 1][4],
-    Addr addr, int wvalid, int wlo, float kmul, float vmul, int g, int t4) {
+    Addr addr, int wvalid, int wlo, float kmul, float pmul, int g, int t4) {
     using M = Mma<__half>;
     constexpr int KSTEPS = D / 16, KP = KSTEPS / 2, RB = NH / 8;
     constexpr int SLICE_BYTES = 16 * D;
-    (void)vmul;
+    (void)pmul;
     (void)SLICE_BYTES;
     const bool partial = wvalid < 16 || wlo > 0;
     bool grew;               // the reference max moved: rescale o
@@ -254,12 +259,16 @@ __device__ __forceinline__ void e4m3_slice_math(
         float p[4], pr[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) p[i] = ex2_approx(s[i] - m[i & 1]);
+        l[0] += p[0] + p[2];
+        l[1] += p[1] + p[3];
+        if constexpr (PPB) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) p[i] *= pmul;
+        }
         const uint32_t p0 = M::pack(p[0], p[1], pr[0], pr[1]);
         const uint32_t p1 = M::pack(p[2], p[3], pr[2], pr[3]);
         const uint32_t r0 = f16x2_rn(p[0] - pr[0], p[1] - pr[1]);
         const uint32_t r1 = f16x2_rn(p[2] - pr[2], p[3] - pr[3]);
-        l[0] += p[0] + p[2];
-        l[1] += p[1] + p[3];
         // P (tokens x heads) -> P^T fragments: lane (g, t4) gets head
         // g, tokens 2 t4, 2 t4 + 1 (of 0-7, then of 8-15)
         pb[0][0] = movmatrix_trans(p0);
@@ -336,12 +345,16 @@ __device__ __forceinline__ void e4m3_slice_math(
             float ps[2];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                const float p0 = ex2_approx(s[nt][i0] - m[rb]);
-                const float p1 = ex2_approx(s[nt][i0 + 1] - m[rb]);
+                float p0 = ex2_approx(s[nt][i0] - m[rb]);
+                float p1 = ex2_approx(s[nt][i0 + 1] - m[rb]);
+                ps[nt] = p0 + p1;
+                if constexpr (PPB) {
+                    p0 *= pmul;
+                    p1 *= pmul;
+                }
                 float h0, h1;
                 pb[rb][nt] = M::pack(p0, p1, h0, h1);
                 pl[rb][nt] = f16x2_rn(p0 - h0, p1 - h1);
-                ps[nt] = p0 + p1;
             }
             l[rb] += ps[0] + ps[1];
         }
@@ -398,16 +411,8 @@ __device__ __forceinline__ void e4m3_slice_math(
             e4m3x4_to_f16x2(byte_perm(vc[2 * h + 1], 0x3120u), va[2], va[3]);
 #pragma unroll
             for (int rb = 0; rb < RB; ++rb) {
-                if constexpr (PPB) {  // this page's P.V, then times its v_scale
-                    float d4[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_f16(d4, va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
-                    mma_f16(d4, va[0], va[1], va[2], va[3], pl[rb][0], pl[rb][1]);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) o[mt][rb][i] = fmaf(d4[i], vmul, o[mt][rb][i]);
-                } else {
-                    mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
-                    mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pl[rb][0], pl[rb][1]);
-                }
+                mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pb[rb][0], pb[rb][1]);
+                mma_f16(o[mt][rb], va[0], va[1], va[2], va[3], pl[rb][0], pl[rb][1]);
             }
         }
     }
@@ -553,8 +558,12 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
     const int lchunk = lane >> 4;
     const int swz = lrow & 7;
 
-    // the output's V scale: the KV head's (per-page scales enter slice by slice)
+    // the output's V scale: the KV head's, or (per-page scales) the warp's
+    // reference vref: o holds the P.V sums in units of vref, a page whose
+    // scale v lies in [vref, 128 vref] enters with its weights times v / vref,
+    // and any other page first moves vref to v / 8, rescaling o
     const float vs_out = PPB ? 1.f : a.v_scale[kvh];
+    float vref = 0.f, inv_vref = 0.f;
 
     int stage = 0;       // it % STAGES
     uint32_t phase = 0;  // (it / STAGES) & 1
@@ -599,6 +608,23 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
             kmul = qmul * a.k_scale[si];
             vmul = a.v_scale[si];
         }
+        float pmul = 1.f;  // per-page: this page's v_scale / vref
+        if (PPB && work) {
+            pmul = vmul * inv_vref;
+            if (!(pmul >= 1.f && pmul <= 128.f)) {  // warp-uniform, rare
+                const float vnew = vmul * 0.125f;
+                const float f = vref / vnew;  // 0 for the warp's first page (o = 0)
+#pragma unroll
+                for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+                    for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) o[mt][rb][i] *= f;
+                vref = vnew;
+                inv_vref = 8.f / vmul;
+                pmul = vmul * inv_vref;
+            }
+        }
         auto addr = [&](int kp) {  // chunk pair kp: chunks 2 kp, 2 kp + 1
             const int chunk = 2 * kp + lchunk;
             return kbase + (chunk >> 3) * BOX_BYTES + (((chunk & 7) ^ swz) << 4);
@@ -612,7 +638,7 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
             }
         }
         auto math = [&]() {
-            e4m3_slice_math<D, NH, PPB, EARLY>(qa, m, l, o, kf, vf, addr, wvalid, wlo, kmul, vmul,
+            e4m3_slice_math<D, NH, PPB, EARLY>(qa, m, l, o, kf, vf, addr, wvalid, wlo, kmul, pmul,
                                                g, t4);
         };
         if (!EARLY && work) math();
@@ -634,7 +660,7 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
     float* red = reinterpret_cast<float*>(s_kv);
     float* red_m = red + NW * NH * A::RP;
     float* red_l = red_m + NW * NH;
-    const float vs = vs_out;
+    const float vs = PPB ? vref : vs_out;
 #pragma unroll
     for (int mt = 0; mt < KSTEPS; ++mt)
 #pragma unroll
