@@ -410,24 +410,25 @@ def test_decode_e4m3_scales_five_decades(G, per_page):
 
 
 @pytest.mark.parametrize("spread", ["log_uniform_1e-20_40", "alternating_1e-20_40"])
-@pytest.mark.parametrize("G", [1, 8, 16])
-def test_decode_e4m3_per_page_v_scales_far_apart(spread, G):
+@pytest.mark.parametrize("G,D", [(1, 128), (8, 128), (16, 128), (8, 256)])
+def test_decode_e4m3_per_page_v_scales_far_apart(spread, G, D):
     """Per-page V scales far apart: log-uniform over 1e-20 .. 40, or pages
-    alternating between 1e-20 and 40 by physical block.  The tensor-core
+    alternating between 1e-20 and 40 by physical block, through the 8-head
+    tiles at head_dim 128 and 256 and the 16-head tiles.  The tensor-core
     kernel's per-warp reference V scale moves on most pages, up or down by up
     to ~2^71; outputs (weighted means dominated by the large-scale pages)
     must meet the bf16 tolerance on both kernels.  The largest scale keeps
     values (up to 448 * 40) where float32 sums of them still resolve the
     absolute tolerance after cancellation."""
-    cfg = _cfg("bf16", 2 * G, 2, 128, 16, RAGGED)
-    inp = make_decode_inputs(cfg, seed=150 + G)
-    dev = E4M3Inputs(inp, seed=150 + G, per_page=True)
+    cfg = _cfg("bf16", 2 * G, 2, D, 16, RAGGED)
+    inp = make_decode_inputs(cfg, seed=150 + G + D)
+    dev = E4M3Inputs(inp, seed=150 + G + D, per_page=True)
     n = dev.pages.v_scale.shape[0]
     if spread.startswith("alternating"):
         vs = np.where(np.arange(n) % 2 == 0, 1e-20, 40.0)[:, None]
         vs = np.broadcast_to(vs, dev.pages.v_scale.shape)
     else:
-        g = np.random.default_rng(160 + G)
+        g = np.random.default_rng(160 + G + D)
         vs = np.exp(g.uniform(np.log(1e-20), np.log(40.0), size=dev.pages.v_scale.shape))
     dev.pages.v_scale = np.ascontiguousarray(vs, dtype=np.float32)
     dev.vs = torch.from_numpy(dev.pages.v_scale).cuda()
