@@ -180,11 +180,15 @@ struct TablePrefetch {
 
 __device__ __forceinline__ TablePrefetch table_prefetch(const DecodeArgs& a, int b, int part,
                                                         int blocks_per_part, int tid) {
-    // (with a sliding window or a shared prefix partition 0 starts at a
-    // block known only after the length is read: no early read then)
-    TablePrefetch pf{0, part == 0 && a.window == 0 && !a.seq_start && tid < blocks_per_part &&
-                            tid < a.max_blocks_per_seq};
-    if (pf.ok) pf.v = a.block_tables[(int64_t)b * a.max_blocks_per_seq + tid];
+    // Partition part starts at block part * blocks_per_part, so its table
+    // slice is read alongside the length, not after it.  (With a sliding
+    // window or a shared prefix the partitions start at a block known only
+    // after the length is read: no early read then.)  An entry past the
+    // sequence's blocks is read but never used.
+    const int64_t i = (int64_t)part * blocks_per_part + tid;
+    TablePrefetch pf{0, a.window == 0 && !a.seq_start && tid < blocks_per_part &&
+                            i < a.max_blocks_per_seq};
+    if (pf.ok) pf.v = a.block_tables[(int64_t)b * a.max_blocks_per_seq + i];
     return pf;
 }
 
