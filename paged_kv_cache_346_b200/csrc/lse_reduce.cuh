@@ -16,8 +16,11 @@ namespace pkv {
 // dependent of the decode, and a CTA of a split row sits resident waiting
 // for the decode grid: where rows have few partitions (a batch of mostly
 // short sequences) that CTA must be small, so the registers-only form runs:
-// one CTA of 8 warps per sequence and 8 query heads (a warp per row; far
-// fewer CTAs than rows to launch and retire), no dynamic shared memory.
+// one CTA of 8 warps per 8 query heads of S consecutive sequences (a warp
+// per row, sequence after sequence; far fewer CTAs than rows to launch and
+// retire), no dynamic shared memory.  S keeps about two CTAs per SM: a batch
+// of many sequences, few of them split, launches a few hundred CTAs instead
+// of one per sequence, most of which only read lengths and leave.
 // Rows of many partitions (long contexts) stream their partial outputs
 // through shared memory with bulk copies (48 KB per CTA, one per row); their
 // waiting CTAs appear only when the decode CTAs, all split, finish their
@@ -25,6 +28,7 @@ namespace pkv {
 constexpr int kReduceRowsPerCta = 8;
 constexpr int kReduceThreads = 256;
 constexpr int kReduceStreamSlots = 16;  // partial results per row from which rows stream
+constexpr int kReduceSms = 148;         // SMs of a B200: the small form's grid size target
 
 // Few partitions per row: one warp merges np partial results of one row into
 // out_row from registers.  Partial p's (m, l) is at ml + 2 p, its o at
@@ -199,27 +203,59 @@ __device__ __forceinline__ void merge_partials(const float* __restrict__ ml, int
 // Launched as a programmatic dependent of the decode kernel: the CTAs of
 // sequences with one partition leave before the wait, during the decode's
 // tail; the others wait for the decode grid's writes before reading.
-// STREAM: one CTA per row (grid Hq x B); else one CTA per sequence and 8
-// query heads (grid ceil(Hq / 8) x B), a warp per row.
+// STREAM: one CTA per row (grid Hq x B); else one CTA per 8 query heads of
+// S = ceil(B / gridDim.y) <= 32 consecutive sequences (grid ceil(Hq / 8) x
+// ceil(B / S)), a warp per row.
 template <typename T, int D, bool STREAM>
 __global__ void __launch_bounds__(kReduceThreads, 1) lse_reduce_kernel(const DecodeArgs a) {
-    const int b = blockIdx.y;
     // the partition count depends only on the inputs, not on the decode
     // grid's output: rows with one partial result leave before the wait
-    const Span sp = seq_span(a, b, false);
-    if (sp.direct) return;
-    const int np = sp.slot0 + sp.np;  // the group pass's slots, then this row's partitions
-    pdl_wait_primary();
     if constexpr (STREAM) {
+        const int b = blockIdx.y;
+        const Span sp = seq_span(a, b, false);
+        if (sp.direct) return;
+        const int np = sp.slot0 + sp.np;  // the group pass's slots, then this row's partitions
+        pdl_wait_primary();
         const int64_t row = (int64_t)b * a.num_q_heads + blockIdx.x;
         merge_partials<T, D>(a.ws_ml + row * a.ws_slots * 2, 2, a.ws_o + row * a.ws_slots * D,
                              np, reinterpret_cast<T*>(a.out) + row * D, a.status);
-    } else {
+    } else if (gridDim.y == (unsigned)a.num_seqs) {  // one sequence per CTA
+        const int b = blockIdx.y;
+        const Span sp = seq_span(a, b, false);
+        if (sp.direct) return;
+        pdl_wait_primary();
         const int h = blockIdx.x * kReduceRowsPerCta + (threadIdx.x >> 5);
         if (h >= a.num_q_heads) return;
         const int64_t row = (int64_t)b * a.num_q_heads + h;
-        merge_row_warp<T, D>(a.ws_ml + row * a.ws_slots * 2, a.ws_o + row * a.ws_slots * D, np,
-                             reinterpret_cast<T*>(a.out) + row * D, threadIdx.x & 31);
+        merge_row_warp<T, D>(a.ws_ml + row * a.ws_slots * 2, a.ws_o + row * a.ws_slots * D,
+                             sp.slot0 + sp.np, reinterpret_cast<T*>(a.out) + row * D,
+                             threadIdx.x & 31);
+    } else {
+        __shared__ uint32_t s_split;  // bit j: sequence b0 + j has partial results to merge
+        const int S = (a.num_seqs + gridDim.y - 1) / gridDim.y;
+        const int b0 = blockIdx.y * S;
+        const int lane = threadIdx.x & 31;
+        if (threadIdx.x < 32) {
+            const int b = b0 + lane;
+            const bool split = lane < S && b < a.num_seqs && !seq_span(a, b, false).direct;
+            const uint32_t m = __ballot_sync(0xffffffffu, split);
+            if (lane == 0) s_split = m;
+        }
+        __syncthreads();
+        uint32_t split = s_split;
+        if (split == 0) return;
+        pdl_wait_primary();
+        const int h = blockIdx.x * kReduceRowsPerCta + (threadIdx.x >> 5);
+        if (h >= a.num_q_heads) return;
+        while (split) {
+            const int b = b0 + __ffs(split) - 1;
+            split &= split - 1;
+            const Span sp = seq_span(a, b, false);
+            const int np = sp.slot0 + sp.np;
+            const int64_t row = (int64_t)b * a.num_q_heads + h;
+            merge_row_warp<T, D>(a.ws_ml + row * a.ws_slots * 2, a.ws_o + row * a.ws_slots * D,
+                                 np, reinterpret_cast<T*>(a.out) + row * D, lane);
+        }
     }
 }
 
@@ -238,8 +274,13 @@ cudaError_t launch_lse_reduce(const DecodeArgs& a, cudaStream_t stream) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (!streamed) {
-        cfg.gridDim = dim3((a.num_q_heads + kReduceRowsPerCta - 1) / kReduceRowsPerCta,
-                           a.num_seqs, 1);
+        // S sequences per CTA: about two CTAs per SM, at most 32 (one ballot)
+        const int64_t hx = (a.num_q_heads + kReduceRowsPerCta - 1) / kReduceRowsPerCta;
+        const int64_t per_seq = hx * (a.num_seqs > 0 ? 1 : 0);
+        int S = (int)((per_seq * a.num_seqs + 2 * kReduceSms - 1) / (2 * kReduceSms));
+        S = S < 1 ? 1 : (S > 32 ? 32 : S);
+        const int gy = a.num_seqs > 0 ? (a.num_seqs + S - 1) / S : 1;
+        cfg.gridDim = dim3((unsigned)hx, (unsigned)gy, 1);
         cfg.dynamicSmemBytes = 0;
         return cudaLaunchKernelEx(&cfg, lse_reduce_kernel<T, D, false>, a);
     }
