@@ -217,7 +217,8 @@ PKV_API int pkv_paged_attention_decode(void* out, const void* q, const void* k_c
  * fp16 hi + lo pair with p's precision), any other page first moves vref to
  * its v_scale / 8 and rescales the fp32 sums; the output is multiplied by
  * vref.  The sums stay in fp32 range for the per-page V scales of a KV head
- * within a factor 2^80 of one another.
+ * within a factor 2^80 of one another, each at least 2^-120 (the kernel
+ * takes 8 / v_scale in fp32).
  *
  * Arguments as pkv_paged_attention_decode, plus:
  *   k_cache, v_cache: device E4M3 codes [num_blocks, Hkv, block_size, head_dim].
