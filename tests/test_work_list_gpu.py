@@ -167,3 +167,29 @@ def test_gqa_batch_shape_items():
     out = _decode(inp, "bf16", 4096, items=items)
     assert_close(to_f64(out), oracle.paged_decode_inputs(inp), "bf16", "GQA shape, items")
     assert pkv.pkv_device_status(clear=True) == 0
+
+
+@pytest.mark.parametrize("kernel", [pkv.PKV_KERNEL_MMA, pkv.PKV_KERNEL_SIMT])
+def test_reduce_several_sequences_per_cta(kernel):
+    """300 sequences, 64 query heads: the reduce's small form gives each CTA 8
+    heads of S = 9 consecutive sequences (34 CTAs in y, the last with 3),
+    with split sequences scattered among them (every 7th long, some CTAs with
+    two or none) and an empty one.  Every row against the oracle, for the
+    work list and the partition grid, which must agree bit for bit."""
+    g = np.random.default_rng(61)
+    lens = g.integers(16, 600, size=300).astype(np.int32)
+    lens[::7] = g.integers(1100, 4000, size=lens[::7].size)
+    lens[100] = 0
+    lens[101] = 1024  # exactly one 1024-token partition: direct
+    cfg = _cfg("bf16", 64, 8, 128, 16, tuple(int(x) for x in lens), pool_extra=3)
+    inp = make_decode_inputs(cfg, seed=62)
+    P = 1024
+    items = torch.from_numpy(pkv.pkv_decode_schedule_items(inp.context_lens, 16, P)).cuda()
+    order = torch.from_numpy(pkv.pkv_decode_schedule_order(inp.context_lens)).cuda()
+    listed = _decode(inp, "bf16", P, items=items, kernel=kernel)
+    grid = _decode(inp, "bf16", P, order=order, kernel=kernel)
+    assert torch.equal(listed, grid)
+    got = to_f64(listed)
+    assert (got[100] == 0).all()
+    assert_close(got, oracle.paged_decode_inputs(inp), "bf16", f"reduce S>1 kernel={kernel}")
+    assert pkv.pkv_device_status(clear=True) == 0
