@@ -567,10 +567,14 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
 
     int stage = 0;       // it % STAGES
     uint32_t phase = 0;  // (it / STAGES) & 1
-    // per-page mode: the scales of the warp's first slice
+    // per-page mode: the scales of the warp's first slice.  Scale indices
+    // are 32-bit: table entries are checked against the pool, whose
+    // num_blocks * Hkv * block_size rows this kernel's tensor maps address
+    // with 32-bit coordinates.
     float ks_next = 1.f, vs_next = 1.f;
     if (PPB && EARLY && nslices > 0) {
-        const int64_t si = (int64_t)s_tab[(warp * 16) / BS] * a.num_kv_heads + kvh;
+        const uint32_t si =
+            (uint32_t)s_tab[(warp * 16) / BS] * (uint32_t)a.num_kv_heads + (uint32_t)kvh;
         ks_next = a.k_scale[si];
         vs_next = a.v_scale[si];
     }
@@ -597,14 +601,16 @@ __global__ void __launch_bounds__(NW * 32, E4m3MinBlocks<D, NH, NW, STAGES_>::va
             kmul = qmul * ks_next;
             vmul = vs_next;
             if (it + 1 < nslices) {
-                const int64_t si =
-                    (int64_t)s_tab[((it + 1) * TILE + warp * 16) / BS] * a.num_kv_heads + kvh;
+                const uint32_t si = (uint32_t)s_tab[((it + 1) * TILE + warp * 16) / BS] *
+                                        (uint32_t)a.num_kv_heads +
+                                    (uint32_t)kvh;
                 ks_next = a.k_scale[si];
                 vs_next = a.v_scale[si];
             }
         } else if (PPB && work) {
-            const int64_t si =
-                (int64_t)s_tab[(it * TILE + warp * 16) / BS] * a.num_kv_heads + kvh;
+            const uint32_t si = (uint32_t)s_tab[(it * TILE + warp * 16) / BS] *
+                                    (uint32_t)a.num_kv_heads +
+                                (uint32_t)kvh;
             kmul = qmul * a.k_scale[si];
             vmul = a.v_scale[si];
         }
